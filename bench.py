@@ -1,0 +1,516 @@
+#!/usr/bin/env python
+"""Benchmark of the HiLS-Attention forward hot path on B200.
+
+Headline (one JSON line on rank 0):
+  decode tokens/s at a 512K-token KV cache (B=1, H=32, d=128, chunk 64, top-K 16,
+  window 512; synthetic Gaussian K/V with one needle key per head). One step = one
+  new token through the whole decode path: hils_select (Eq. 7 scores over 8191
+  chunk summaries + exact top-K) then hils_attend_decode (Eq. 10 over 16 chunks +
+  the window). Summaries are built once beforehand (hils_summarize), as a server
+  keeps them with its KV cache.
+Beside it, in the same line:
+  "prefill": algorithmic TFLOP/s of summarise + select + prefill attend on the 8K
+  prefill workload (B=1, H=32, d=128, K=16, W=512);
+  "roofline": the dominant decode kernel against the measured HBM copy bandwidth;
+  "e2e": the same decode metric through the Python binding with pinned host
+  buffers: the step's query (Q, Q_cal, positions) copied in and (O, lse) copied out
+  inside the timed region; KV cache and summaries stay resident in HBM;
+  "cpu_baseline": the float64 oracle on this host's cores, on a sample of heads.
+
+Timing: W warm-up steps, then exactly K timed steps, each preceded by a write of
+2x the L2 size (outside the step's events), timed with CUDA events on the launching
+stream; barrier + synchronize around the region; the max over ranks is reported.
+Multi-GPU (torchrun): every rank runs its own replica of the workload (weak
+scaling; the path has no exchange step) and value = all ranks' tokens / max time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hils|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hils_synth import WORKLOADS, make_decode, make_prefill  # noqa: E402
+
+METRIC = "HiLS decode tokens/s @512K ctx (%HBM roofline); prefill TFLOP/s @8K (%TC peak)"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- clocks (NVML, read-only)
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Polls the SM clock and clock-event reasons of this process's GPU every ~1 ms."""
+
+    def __init__(self, device: torch.device):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nv = pynvml
+            self.ok = True
+        except Exception as e:  # no NVML: report that clocks were not sampled
+            self.err = repr(e)
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return fn(self.h)
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append((self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM),
+                                     self._reasons()))
+            except Exception:
+                pass
+            time.sleep(0.001)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._loop, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= int(r)
+        reasons = sorted(n for b, n in _REASONS.items() if bits & b and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz)}
+
+
+# ----------------------------------------------------------------- timing helpers
+
+class Flusher:
+    """Writes a buffer of twice the L2 size, so that no step starts with warm L2."""
+
+    def __init__(self, dev):
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.buf = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1.0)
+
+
+def time_steps(fn, steps, flush, stream):
+    """Per-step device milliseconds of `fn` on `stream`, L2 flushed before each step."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for s, e in ev:
+            flush()
+            s.record(stream)
+            fn()
+            e.record(stream)
+    stream.synchronize()
+    return [s.elapsed_time(e) for s, e in ev]
+
+
+def dist_ctx():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, dev) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- decode workload
+
+def decode_bytes(w) -> dict:
+    """Algorithmic HBM bytes of one decode step (per the whole batch)."""
+    t = w.N - 1
+    c_elig = min(t // w.S, w.C)
+    es = 2
+    per_bh_sel = c_elig * (w.d * es + 4) + 2 * w.d * es + w.K * 8 + 4  # table + q~ + outputs
+    per_bh_att = w.K * w.S * w.d * es * 2 + w.W * w.d * es * 2 + 2 * w.d * es + w.K * 8 + 4
+    n = w.B * w.H
+    return {"select": n * per_bh_sel, "attend": n * per_bh_att,
+            "step": n * (c_elig * (w.d * es + 4) + w.K * w.S * w.d * es * 2 + w.W * w.d * es * 2 + 768)}
+
+
+class DecodeBench:
+    def __init__(self, w, dev):
+        import hierarchical_chunk_sparse_b200 as hils
+
+        self.hils, self.w, self.dev = hils, w, dev
+        inp = make_decode(w, device=dev)
+        self.inp = inp
+        self.p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype)
+        C = w.C
+        self.Ksum = torch.empty(w.B, w.H, C, w.d, dtype=w.dtype, device=dev)
+        self.Bsum = torch.empty(w.B, w.H, C, dtype=torch.float32, device=dev)
+        hils.hils_summarize(self.p, inp["K"], inp["LQ"], self.Ksum, self.Bsum)
+        self.qpos = (inp["cache_len"] - 1).reshape(w.B, 1).contiguous()
+        self.idx = torch.empty(w.B, w.H, 1, w.K, dtype=torch.int32, device=dev)
+        self.score = torch.empty(w.B, w.H, 1, w.K, dtype=torch.float32, device=dev)
+        self.nsel = torch.empty(w.B, w.H, 1, dtype=torch.int32, device=dev)
+        self.ws_sel = hils.alloc_workspace(self.p, hils.HILS_CALL_SELECT, 1, C, device=dev)
+        self.ws_dec = hils.alloc_workspace(self.p, hils.HILS_CALL_ATTEND_DECODE, 1, 0, device=dev)
+        self.O = torch.empty_like(inp["Q"])
+        self.lse = torch.empty(w.B, w.H, dtype=torch.float32, device=dev)
+        torch.cuda.synchronize()
+        self.launches_per_step = 2
+
+    def select(self):
+        i = self.inp
+        self.hils.hils_select(self.p, i["Qcal"], self.Ksum, self.Bsum, self.idx, self.score, self.nsel,
+                              qpos=self.qpos, workspace=self.ws_sel)
+
+    def attend(self):
+        i = self.inp
+        self.hils.hils_attend_decode(self.p, i["Q"], i["K"], i["V"], i["cache_len"], self.idx, self.score,
+                                     self.nsel, self.O, self.lse, workspace=self.ws_dec)
+
+    def step(self):
+        self.select()
+        self.attend()
+
+    def e2e_setup(self):
+        i = self.inp
+        self.h_in = {k: i[k].cpu().pin_memory() for k in ("Q", "Qcal", "cache_len")}
+        self.h_qpos = self.qpos.cpu().pin_memory()
+        self.h_O = torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory()
+        self.h_lse = torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in self.h_in.values()) + \
+            self.h_qpos.numel() * self.h_qpos.element_size()
+        d2h = self.h_O.numel() * self.h_O.element_size() + self.h_lse.numel() * self.h_lse.element_size()
+        return h2d, d2h
+
+    def e2e_step(self):
+        i = self.inp
+        for k, t in self.h_in.items():
+            i[k].copy_(t, non_blocking=True)
+        self.qpos.copy_(self.h_qpos, non_blocking=True)
+        self.step()
+        self.h_O.copy_(self.O, non_blocking=True)
+        self.h_lse.copy_(self.lse, non_blocking=True)
+
+
+# ----------------------------------------------------------------- prefill workload
+
+def prefill_flops(w) -> float:
+    """Algorithmic flops of summarise + score + chunk attention + window (per batch)."""
+    d, S, K, W, N, C = w.d, w.S, w.K, w.W, w.N, w.C
+    score = chunk = win = 0
+    for i in range(N):
+        e = min(i // S, C)
+        score += 2 * d * e
+        chunk += 4 * d * S * min(K, e)
+        win += 4 * d * min(W, i + 1)
+    summ = 4 * d * S * C
+    return float(w.B * w.H * (score + chunk + win + summ))
+
+
+class PrefillBench:
+    def __init__(self, w, dev):
+        import hierarchical_chunk_sparse_b200 as hils
+
+        self.hils, self.w = hils, w
+        self.inp = make_prefill(w, device=dev)
+        self.p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype)
+        C = w.C
+        self.Ksum = torch.empty(w.B, w.H, C, w.d, dtype=w.dtype, device=dev)
+        self.Bsum = torch.empty(w.B, w.H, C, dtype=torch.float32, device=dev)
+        self.idx = torch.empty(w.B, w.H, w.N, w.K, dtype=torch.int32, device=dev)
+        self.score = torch.empty(w.B, w.H, w.N, w.K, dtype=torch.float32, device=dev)
+        self.nsel = torch.empty(w.B, w.H, w.N, dtype=torch.int32, device=dev)
+        self.ws = hils.alloc_workspace(self.p, hils.HILS_CALL_SELECT, w.N, C, device=dev)
+        self.O = torch.empty_like(self.inp["Q"])
+        self.lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device=dev)
+        torch.cuda.synchronize()
+
+    def summarize(self):
+        i = self.inp
+        self.hils.hils_summarize(self.p, i["K"], i["LQ"], self.Ksum, self.Bsum)
+
+    def select(self):
+        i = self.inp
+        self.hils.hils_select(self.p, i["Qcal"], self.Ksum, self.Bsum, self.idx, self.score, self.nsel,
+                              workspace=self.ws)
+
+    def attend(self):
+        i = self.inp
+        self.hils.hils_attend_prefill(self.p, i["Q"], i["K"], i["V"], self.idx, self.score, self.nsel,
+                                      self.O, self.lse)
+
+    def step(self):
+        self.summarize()
+        self.select()
+        self.attend()
+
+
+# ----------------------------------------------------------------- CPU oracle baseline
+
+def oracle_decode_sample(w, dev, heads: int):
+    """Host copies of the first `heads` heads of a decode workload, with summaries."""
+    import hierarchical_chunk_sparse_b200 as hils
+
+    ws = w.replace(H=heads)
+    gen_dev = dev if dev is not None else "cpu"
+    inp = make_decode(ws, device=gen_dev)
+    if dev is not None:
+        p = hils.Params(B=ws.B, H=ws.H, d=ws.d, K=ws.K, W=ws.W, dtype=ws.dtype)
+        Ksum = torch.empty(ws.B, ws.H, ws.C, ws.d, dtype=ws.dtype, device=dev)
+        Bsum = torch.empty(ws.B, ws.H, ws.C, dtype=torch.float32, device=dev)
+        hils.hils_summarize(p, inp["K"], inp["LQ"], Ksum, Bsum)
+        torch.cuda.synchronize()
+        host = {k: v.cpu() for k, v in inp.items() if isinstance(v, torch.Tensor)}
+        host["Ksum"], host["Bsum"] = Ksum.cpu(), Bsum.cpu()
+        del inp
+        torch.cuda.empty_cache()
+    else:
+        import oracle
+
+        host = dict(inp)
+        ks, bs = oracle.summarize(host["K"], host["LQ"], ws.S, ws.scale)
+        host["Ksum"], host["Bsum"] = torch.from_numpy(ks).to(ws.dtype), torch.from_numpy(bs).float()
+    host["qpos"] = (host["cache_len"] - 1).reshape(ws.B, 1)
+    return ws, host
+
+
+def oracle_decode_step(ws, host):
+    import oracle
+
+    idx, score, nsel = oracle.select(host["Qcal"], host["Ksum"], host["Bsum"], ws.S, ws.K, ws.scale,
+                                     qpos=host["qpos"])
+    oracle.attend(host["Q"], host["K"], host["V"], idx, score, nsel, ws.S, ws.W, ws.scale, qpos=host["qpos"])
+
+
+def cpu_baseline(w, dev, heads=4, min_s=5.0, max_s=20.0):
+    import oracle
+
+    oracle.build()
+    ws, host = oracle_decode_sample(w, dev, heads)
+    oracle_decode_step(ws, host)  # warm
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle_decode_step(ws, host)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_s or (el >= max_s):
+            break
+    per_step = el / reps * (w.H / heads)  # seconds for all heads of one token
+    return {"value": w.B / per_step, "unit": "tokens/s", "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": f"{heads} of {w.H} heads of one decode step (select over {w.C - 1} chunks + attend), "
+                      f"{reps} repetitions in {el:.1f} s, time scaled by {w.H}/{heads}"}
+
+
+# ----------------------------------------------------------------- main
+
+def run_reference(args, w):
+    """The oracle as the reference arm: same metric and workload, on host cores."""
+    world, rank, local = dist_ctx()
+    if world > 1 and rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else None
+    heads = 2
+    ws, host = oracle_decode_sample(w, dev, heads)
+    for _ in range(args.warmup):
+        oracle_decode_step(ws, host)
+    t = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_decode_step(ws, host)
+        t.append((time.perf_counter() - t0) * (w.H / heads))
+    ms = 1e3 * statistics.mean(t)
+    value = w.B / (ms / 1e3)
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "kv_len": w.N, "chunk": w.S,
+                       "top_k": w.K, "window": w.W, "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.get_threads(),
+                             "kind": "oracle",
+                             "sample": f"{heads} of {w.H} heads per step, time scaled by {w.H}/{heads}"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="hils", choices=["hils", "reference"])
+    ap.add_argument("--no-prefill", action="store_true", help="skip the 8K prefill measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = WORKLOADS[4]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    world, rank, local = dist_ctx()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    import hierarchical_chunk_sparse_b200 as hils
+
+    hils.load_library()
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.Stream(dev)
+    flush = Flusher(dev)
+
+    # ---------------- headline: decode @512K
+    db = DecodeBench(w, dev)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            db.step()
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        per = time_steps(db.step, args.steps, flush, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(statistics.mean(per), world, dev)
+    value = world * w.B / (ms / 1e3)
+    # per-kernel times (same protocol)
+    t_sel = statistics.mean(time_steps(db.select, args.steps, flush, stream))
+    t_att = statistics.mean(time_steps(db.attend, args.steps, flush, stream))
+    by = decode_bytes(w)
+    hbm = peaks["hbm_gbs"]
+    sel_gbs = by["select"] / (t_sel * 1e-3) / 1e9
+    att_gbs = by["attend"] / (t_att * 1e-3) / 1e9
+    step_gbs = by["step"] / (ms * 1e-3) / 1e9
+    dominant = "select" if t_sel >= t_att else "attend"
+    dom = {"select": (sel_gbs, by["select"]), "attend": (att_gbs, by["attend"])}[dominant]
+    # end to end through the binding with host buffers
+    h2d, d2h = db.e2e_setup()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            db.e2e_step()
+    per_e2e = time_steps(db.e2e_step, args.steps, flush, stream)
+    ms_e2e = max_over_ranks(statistics.mean(per_e2e), world, dev)
+    del db
+    torch.cuda.empty_cache()
+
+    # ---------------- prefill @8K
+    prefill = None
+    if not args.no_prefill:
+        wp = WORKLOADS[2]
+        pb = PrefillBench(wp, dev)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                pb.step()
+        n = max(3, min(args.steps, 20))
+        pt = statistics.mean(time_steps(pb.step, n, flush, stream))
+        pt = max_over_ranks(pt, world, dev)
+        ks = {k: statistics.mean(time_steps(getattr(pb, k), n, flush, stream))
+              for k in ("summarize", "select", "attend")}
+        fl = prefill_flops(wp)
+        tf = fl / (pt * 1e-3) / 1e12
+        prefill = {"value": tf * world, "unit": "TFLOP/s", "ms_per_step": pt, "workload": wp.name,
+                   "algorithmic_gflop_per_step": fl / 1e9, "steps": n,
+                   "kernel_ms": ks,
+                   "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                                "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"], "traffic": None,
+                                "peak_source": f"{peak_src} bf16 dense (burst)"}}
+        del pb
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, dev)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "kv_len": w.N, "chunk": w.S,
+                       "top_k": w.K, "window": w.W, "parallelism": f"replicas{world}",
+                       "l2": "flushed before every step (2x L2 write)"},
+            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom[0], "peak": hbm,
+                         "unit": "GB/s", "frac": dom[0] / hbm, "traffic": None,
+                         "algorithmic_bytes": dom[1], "peak_source": f"{peak_src} HBM copy"},
+            "step_roofline": {"bytes": by["step"], "achieved_gbs": step_gbs, "frac_measured": step_gbs / hbm,
+                              "frac_8tbs": step_gbs / 8000.0},
+            "kernel_us": {"select": 1e3 * t_sel, "attend": 1e3 * t_att,
+                          "select_gbs": sel_gbs, "attend_gbs": att_gbs},
+            "e2e": {"value": world * w.B / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * 2,
+            "clocks": clk.summary(),
+            "prefill": prefill,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

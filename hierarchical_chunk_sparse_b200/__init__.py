@@ -1,0 +1,189 @@
+"""Python binding of libhils, the HiLS-Attention forward pass for B200 (sm_100a).
+
+Argument marshalling only: every function here turns torch CUDA tensors into the
+pointers and element strides of the C ABI (``include/hils.h``) and calls the entry
+point of the same name; all work runs in the library's CUDA kernels. There is no
+CPU fallback: if the compiled library is missing, loading fails with an error.
+
+    import hierarchical_chunk_sparse_b200 as hils
+    p = hils.Params(B=1, H=32, d=128, K=16, W=512, dtype=torch.bfloat16)
+    hils.hils_summarize(p, K, LQ, Ksum, Bsum)
+    hils.hils_select(p, Qcal, Ksum, Bsum, idx, score, nsel, workspace=ws)
+    hils.hils_attend_prefill(p, Q, K, V, idx, score, nsel, O, lse)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhils.so")
+
+HILS_F32, HILS_BF16 = 0, 1
+HILS_CALL_SELECT, HILS_CALL_ATTEND_PREFILL, HILS_CALL_ATTEND_DECODE = 0, 1, 2
+STATUS = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARG", 2: "HILS_ERR_UNSUPPORTED",
+          3: "HILS_ERR_ALIGNMENT", 4: "HILS_ERR_WORKSPACE", 5: "HILS_ERR_CUDA"}
+_DTYPES = {torch.float32: HILS_F32, torch.bfloat16: HILS_BF16}
+
+# Every function the C header declares (checked by the tests against the header).
+EXPORTS = ("hils_summarize", "hils_select", "hils_attend_prefill", "hils_attend_decode",
+           "hils_workspace_bytes", "hils_workspace_init", "hils_status_string",
+           "hils_last_cuda_error")
+
+
+class HilsError(RuntimeError):
+    def __init__(self, call: str, status: int, detail: str = ""):
+        self.status = status
+        msg = f"{call}: {STATUS.get(status, status)}"
+        super().__init__(msg + (f" ({detail})" if detail else ""))
+
+
+class _CTensor(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("sb", ctypes.c_int64), ("sh", ctypes.c_int64),
+                ("st", ctypes.c_int64)]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int), ("S", ctypes.c_int),
+                ("K", ctypes.c_int), ("W", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("scale", ctypes.c_float), ("flags", ctypes.c_uint32)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libhils.so; raises if it has not been built (no fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise ImportError(f"libhils.so not built at {path}; run "
+                              "python -m hierarchical_chunk_sparse_b200.build")
+        lib = ctypes.CDLL(path)
+        T, P, vp, i, sz = _CTensor, ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        lib.hils_summarize.argtypes = [P, T, i, T, T, vp, vp]
+        lib.hils_select.argtypes = [P, T, i, vp, T, vp, i, vp, vp, vp, vp, sz, vp]
+        lib.hils_attend_prefill.argtypes = [P, T, T, T, i, vp, vp, vp, T, vp, vp, sz, vp]
+        lib.hils_attend_decode.argtypes = [P, T, T, T, vp, vp, vp, vp, T, vp, vp, sz, vp]
+        lib.hils_workspace_bytes.argtypes = [P, i, i, i]
+        lib.hils_workspace_bytes.restype = sz
+        lib.hils_workspace_init.argtypes = [vp, sz, vp]
+        lib.hils_status_string.argtypes = [i]
+        lib.hils_status_string.restype = ctypes.c_char_p
+        lib.hils_last_cuda_error.restype = ctypes.c_char_p
+        for name in ("hils_summarize", "hils_select", "hils_attend_prefill", "hils_attend_decode",
+                     "hils_workspace_init"):
+            getattr(lib, name).restype = i
+        _lib = lib
+    return _lib
+
+
+class Params:
+    """hils_params: B, H, d, chunk size S (64), top-K, window W, dtype, scale (0 = 1/sqrt(d))."""
+
+    def __init__(self, B: int, H: int, d: int, K: int, W: int, dtype: torch.dtype = torch.bfloat16,
+                 S: int = 64, scale: float = 0.0, flags: int = 0):
+        self.B, self.H, self.d, self.K, self.W, self.S = B, H, d, K, W, S
+        self.dtype, self.scale, self.flags = dtype, scale, flags
+
+    def c(self) -> _Params:
+        dt = _DTYPES.get(self.dtype, -1) if isinstance(self.dtype, torch.dtype) else int(self.dtype)
+        return _Params(self.B, self.H, self.d, self.S, self.K, self.W, dt, self.scale, self.flags)
+
+
+def _view(t) -> _CTensor:
+    """[B, H, T, d] torch tensor (innermost stride 1) -> pointer + element strides."""
+    if t is None:
+        return _CTensor(None, 0, 0, 0)
+    if t.dim() != 4:
+        raise ValueError("expected a [B, H, T, d] tensor")
+    if t.shape[3] > 1 and t.stride(3) != 1:
+        raise ValueError("the head dimension must be contiguous")
+    return _CTensor(t.data_ptr(), t.stride(0), t.stride(1), t.stride(2))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(call: str, rc: int) -> None:
+    if rc != 0:
+        lib = load_library()
+        detail = lib.hils_last_cuda_error().decode() if rc == 5 else lib.hils_status_string(rc).decode()
+        raise HilsError(call, rc, detail)
+
+
+def hils_workspace_bytes(p: Params, call: int, Lq: int, C: int) -> int:
+    return int(load_library().hils_workspace_bytes(ctypes.byref(p.c()), call, Lq, C))
+
+
+def hils_workspace_init(workspace, ws_bytes: int | None = None, stream=None) -> None:
+    n = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check("hils_workspace_init", load_library().hils_workspace_init(_ptr(workspace), n, _stream(stream)))
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+def hils_summarize(p: Params, K, LQ, Ksum, Bsum, N: int | None = None, stream=None) -> None:
+    """Eq. 8 summaries of every complete chunk: Ksum [B,H,C,d], Bsum [B,H,C] float32."""
+    n = K.shape[2] if N is None else N
+    _check("hils_summarize", load_library().hils_summarize(
+        ctypes.byref(p.c()), _view(K), n, _view(LQ), _view(Ksum), _ptr(Bsum), _stream(stream)))
+
+
+def hils_select(p: Params, Qcal, Ksum, Bsum, idx, score, nsel, qpos=None, workspace=None,
+                Lq: int | None = None, C: int | None = None, stream=None) -> None:
+    """Eq. 7 scores and exact top-K: idx/score [B,H,Lq,K], nsel [B,H,Lq]."""
+    lq = Qcal.shape[2] if Lq is None else Lq
+    c = Ksum.shape[2] if C is None else C
+    wp, wn = _ws(workspace)
+    _check("hils_select", load_library().hils_select(
+        ctypes.byref(p.c()), _view(Qcal), lq, _ptr(qpos), _view(Ksum), _ptr(Bsum), c,
+        _ptr(idx), _ptr(score), _ptr(nsel), wp, wn, _stream(stream)))
+
+
+def hils_attend_prefill(p: Params, Q, K, V, idx, score, nsel, O, lse=None, workspace=None,
+                        N: int | None = None, stream=None) -> None:
+    """Eq. 10 for every position: O [B,H,N,d], lse [B,H,N] float32 (optional)."""
+    n = Q.shape[2] if N is None else N
+    wp, wn = _ws(workspace)
+    _check("hils_attend_prefill", load_library().hils_attend_prefill(
+        ctypes.byref(p.c()), _view(Q), _view(K), _view(V), n, _ptr(idx), _ptr(score), _ptr(nsel),
+        _view(O), _ptr(lse), wp, wn, _stream(stream)))
+
+
+def hils_attend_decode(p: Params, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse=None,
+                       workspace=None, stream=None) -> None:
+    """Eq. 10 for one new token per sequence: O [B,H,1,d], lse [B,H] float32 (optional)."""
+    wp, wn = _ws(workspace)
+    _check("hils_attend_decode", load_library().hils_attend_decode(
+        ctypes.byref(p.c()), _view(Q), _view(Kc), _view(Vc), _ptr(cache_len), _ptr(idx), _ptr(score),
+        _ptr(nsel), _view(O), _ptr(lse), wp, wn, _stream(stream)))
+
+
+def alloc_workspace(p: Params, call: int, Lq: int, C: int, device="cuda") -> torch.Tensor | None:
+    """Allocates (torch) and zeroes a workspace of the size the call needs, or None."""
+    n = hils_workspace_bytes(p, call, Lq, C)
+    if n == 0:
+        return None
+    ws = torch.empty((n + 15) // 16 * 16, dtype=torch.uint8, device=device)
+    hils_workspace_init(ws)
+    return ws

@@ -1,0 +1,340 @@
+// Hierarchical softmax over the selected chunks plus the sliding window:
+// "Hierarchical Sparse Attention Done Right" (picx.dev summary), Methodology 2, Eq. 10
+// (w_ij = exp(s_ij)/Z_{i,c(j)} * Z^_{i,c(j)}/Z^_i, with Z^_i normalising over the selected
+// chunks and the window), and the rcap.io post's pseudocode figure.
+//
+// Both kernels here split the work of one query into "units" of at most 64 tokens:
+//   - chunk unit (one kept chunk c): log-mass m_u = s^_{i,c} (the select score) and
+//     o_u = sum_{j in c} softmax_j(scale q.k_j) v_j;
+//   - window tile (64 consecutive tokens of [max(0,t-W+1), t]): log-mass
+//     m_u = log sum_j exp(scale q.k_j) over the tile and o_u its softmax-weighted v.
+// Eq. 10 is then  o = sum_u exp(m_u) o_u / sum_u exp(m_u),  lse = log sum_u exp(m_u):
+// the window tiles together give exp(LSE_W) o_W, the chunks exp(s^_c) o_c.
+//
+// Decode (one query per (b, h), memory bound): one 128-thread CTA per unit streams the
+// unit's K and V rows (16-byte cp.async into shared memory, K and V in flight
+// together), writes (m_u, o_u) to the workspace, and the last CTA of the (b, h)
+// combines them. The general prefill kernel (any dtype) gives one CTA per query and
+// walks its units in turn with a running combination; the bf16 prefill fast path is
+// a separate tensor-core kernel.
+#include <math.h>
+
+#include "hils_internal.cuh"
+
+namespace hils {
+namespace {
+
+constexpr int kThreads = 128;
+
+template <typename T, int D>
+struct UnitCfg {
+    static constexpr int kRowBytes = D * (int)sizeof(T);
+    static constexpr int kRowUnits = kRowBytes / 16;
+    static constexpr int kHalfUnits = kRowUnits / 2;
+    static constexpr int kTileBytes = kChunk * kRowBytes;
+    static constexpr int kColUnits = D / 2;
+    static constexpr int kRowGroups = kThreads / kColUnits;
+    // K tile, V tile, query row, logits, probabilities, column partial sums
+    static constexpr int kSmemBytes = 2 * kTileBytes + kRowBytes + (2 * kChunk + kRowGroups * D) * 4;
+};
+
+template <int kHalfUnits>
+__device__ __forceinline__ int rotated_unit(int k, int row, int half) {
+    if (kHalfUnits == 4) return (k + row) & 3;
+    return (k + 2 * row + half) & (kHalfUnits - 1);
+}
+
+struct UnitSmem {
+    uint8_t *kt, *vt, *q;
+    float *logit, *prob, *red;
+};
+
+template <typename T, int D>
+__device__ __forceinline__ UnitSmem unit_smem(uint8_t *base) {
+    using Cfg = UnitCfg<T, D>;
+    UnitSmem s;
+    s.kt = base;
+    s.vt = base + Cfg::kTileBytes;
+    s.q = base + 2 * Cfg::kTileBytes;
+    s.logit = reinterpret_cast<float *>(s.q + Cfg::kRowBytes);
+    s.prob = s.logit + kChunk;
+    s.red = s.prob + kChunk;
+    return s;
+}
+
+// Copies the query row and `rows` K rows (group 0), then `rows` V rows (group 1).
+template <typename T, int D>
+__device__ __forceinline__ void unit_issue(const UnitSmem &s, const T *qrow, const T *k0, int64_t kst,
+                                           const T *v0, int64_t vst, int rows) {
+    using Cfg = UnitCfg<T, D>;
+    const int tid = threadIdx.x;
+    for (int i = tid; i < rows * Cfg::kRowUnits; i += kThreads) {
+        const int r = i / Cfg::kRowUnits, un = i % Cfg::kRowUnits;
+        cp_async16(s.kt + i * 16, reinterpret_cast<const uint8_t *>(k0 + r * kst) + un * 16);
+    }
+    for (int i = tid; i < Cfg::kRowUnits; i += kThreads)
+        cp_async16(s.q + i * 16, reinterpret_cast<const uint8_t *>(qrow) + i * 16);
+    cp_async_commit();
+    for (int i = tid; i < rows * Cfg::kRowUnits; i += kThreads) {
+        const int r = i / Cfg::kRowUnits, un = i % Cfg::kRowUnits;
+        cp_async16(s.vt + i * 16, reinterpret_cast<const uint8_t *>(v0 + r * vst) + un * 16);
+    }
+    cp_async_commit();
+}
+
+// Consumes the copies of unit_issue. Returns log sum_j exp(scale q.k_j) over the
+// rows; leaves o_u = sum_j p_j v_j in s.red[0..D). All threads call it.
+template <typename T, int D>
+__device__ float unit_compute(const UnitSmem &s, int rows, float scale) {
+    using Cfg = UnitCfg<T, D>;
+    const int tid = threadIdx.x;
+    cp_async_wait<1>();
+    __syncthreads();
+    {
+        const int row = tid >> 1, half = tid & 1;
+        const uint4 *krow = reinterpret_cast<const uint4 *>(s.kt + row * Cfg::kRowBytes);
+        const uint4 *qv = reinterpret_cast<const uint4 *>(s.q);
+        float acc = 0.f;
+        if (row < rows) {
+#pragma unroll
+            for (int k = 0; k < Cfg::kHalfUnits; ++k) {
+                const int un = half * Cfg::kHalfUnits + rotated_unit<Cfg::kHalfUnits>(k, row, half);
+                acc = dot16<T>(krow[un], qv[un], acc);
+            }
+        }
+        acc += __shfl_xor_sync(kFull, acc, 1);
+        if (half == 0) s.logit[row] = row < rows ? acc * scale : -INFINITY;
+    }
+    __syncthreads();
+    if (tid < 32) {
+        const float l0 = s.logit[tid], l1 = s.logit[tid + 32];
+        const float m = warp_max(fmaxf(l0, l1));
+        const float e0 = expf(l0 - m), e1 = expf(l1 - m);
+        const float z = warp_sum(e0 + e1);
+        const float inv = 1.f / z;
+        s.prob[tid] = e0 * inv;
+        s.prob[tid + 32] = e1 * inv;
+        if (tid == 0) s.logit[0] = m + logf(z);  // row 0's logit is no longer needed
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    const float lse_tile = s.logit[0];
+    {
+        const int cu = tid % Cfg::kColUnits, rg = tid / Cfg::kColUnits;
+        float a0 = 0.f, a1 = 0.f;
+        for (int j = rg; j < rows; j += Cfg::kRowGroups) {
+            const float2 vv = load2(reinterpret_cast<const T *>(s.vt + j * Cfg::kRowBytes) + 2 * cu);
+            const float pj = s.prob[j];
+            a0 = fmaf(pj, vv.x, a0);
+            a1 = fmaf(pj, vv.y, a1);
+        }
+        s.red[rg * D + 2 * cu] = a0;
+        s.red[rg * D + 2 * cu + 1] = a1;
+        __syncthreads();
+        if (rg == 0) {
+#pragma unroll
+            for (int g = 1; g < Cfg::kRowGroups; ++g) {
+                a0 += s.red[g * D + 2 * cu];
+                a1 += s.red[g * D + 2 * cu + 1];
+            }
+            s.red[2 * cu] = a0;
+            s.red[2 * cu + 1] = a1;
+        }
+    }
+    __syncthreads();
+    return lse_tile;
+}
+
+// Unit u of a query at position t: token range and log-mass source.
+struct UnitPlan {
+    int start, rows;  // rows == 0: empty unit
+    bool is_chunk;
+    float mass;       // chunk units: the select score
+};
+
+__device__ __forceinline__ UnitPlan plan_unit(int u, int t, int K, int W, const int32_t *idx_row,
+                                              const float *score_row, int nsel) {
+    UnitPlan p{0, 0, false, -INFINITY};
+    if (t < 0) return p;
+    if (u < K) {
+        if (u >= nsel) return p;
+        const int c = idx_row[u];
+        if (c < 0) return p;
+        const int start = c * kChunk;
+        if (start > t) return p;
+        p.start = start;
+        p.rows = min(kChunk, t - start + 1);
+        p.is_chunk = true;
+        p.mass = score_row[u];
+        return p;
+    }
+    const int w0 = max(0, t - W + 1);
+    const int start = w0 + (u - K) * kChunk;
+    if (W <= 0 || start > t) return p;
+    p.start = start;
+    p.rows = min(kChunk, t - start + 1);
+    return p;
+}
+
+struct DecodeWs {
+    int *counters;
+    float *mass;
+    float *vec;
+};
+
+__host__ __device__ __forceinline__ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+__device__ __forceinline__ DecodeWs decode_ws(void *ws, int queries, int units, int D) {
+    DecodeWs w;
+    uint8_t *p = static_cast<uint8_t *>(ws);
+    w.counters = reinterpret_cast<int *>(p);
+    p += align256((size_t)queries * sizeof(int));
+    w.mass = reinterpret_cast<float *>(p);
+    p += align256((size_t)queries * units * sizeof(float));
+    w.vec = reinterpret_cast<float *>(p);
+    return w;
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void store_output(const AttendArgs &a, int b, int h, int i, int64_t qi,
+                                             const float *o, float lse) {
+    T *orow = static_cast<T *>(a.O.ptr) + b * a.O.sb + h * a.O.sh + i * a.O.st;
+    for (int x2 = threadIdx.x; x2 < D / 2; x2 += kThreads) store2(orow + 2 * x2, o[2 * x2], o[2 * x2 + 1]);
+    if (a.lse && threadIdx.x == 0) a.lse[qi] = lse;
+}
+
+// grid (units, B*H): one unit per CTA; the last CTA of each (b, h) combines.
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ int is_last;
+    const UnitSmem s = unit_smem<T, D>(smem);
+    const int u = blockIdx.x;
+    const int64_t qi = blockIdx.y;  // (b, h), one query each
+    const int b = (int)(qi / a.H), h = (int)(qi % a.H);
+    const int t = a.cache_len[b] - 1;
+    const UnitPlan p = plan_unit(u, t, a.topk, a.W, a.idx + qi * a.topk, a.score + qi * a.topk,
+                                 a.topk > 0 ? a.nsel[qi] : 0);
+    const DecodeWs ws = decode_ws(a.ws, a.B * a.H, a.units, D);
+    float *my_vec = ws.vec + ((size_t)qi * a.units + u) * D;
+    if (p.rows > 0) {
+        const T *qrow = static_cast<const T *>(a.Q.ptr) + b * a.Q.sb + h * a.Q.sh;
+        const T *k0 = static_cast<const T *>(a.K.ptr) + b * a.K.sb + h * a.K.sh + (int64_t)p.start * a.K.st;
+        const T *v0 = static_cast<const T *>(a.V.ptr) + b * a.V.sb + h * a.V.sh + (int64_t)p.start * a.V.st;
+        unit_issue<T, D>(s, qrow, k0, a.K.st, v0, a.V.st, p.rows);
+        const float lse_tile = unit_compute<T, D>(s, p.rows, a.scale);
+        for (int x = threadIdx.x; x < D; x += kThreads) my_vec[x] = s.red[x];
+        if (threadIdx.x == 0) ws.mass[qi * a.units + u] = p.is_chunk ? p.mass : lse_tile;
+    } else if (threadIdx.x == 0) {
+        ws.mass[qi * a.units + u] = -INFINITY;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = atomicAdd(&ws.counters[qi], 1) == a.units - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    // combine: o = sum_u exp(m_u - M) o_u / sum_u exp(m_u - M), lse = M + log(...)
+    float M = -INFINITY;
+    for (int v = 0; v < a.units; ++v) M = fmaxf(M, __ldcg(&ws.mass[qi * a.units + v]));
+    float *o = s.red;  // reuse shared memory for the final row
+    float zsum = 0.f;
+    for (int x = threadIdx.x; x < D; x += kThreads) o[x] = 0.f;
+    if (M != -INFINITY) {
+        for (int v = 0; v < a.units; ++v) {
+            const float m = __ldcg(&ws.mass[qi * a.units + v]);
+            if (m == -INFINITY) continue;
+            const float wv = expf(m - M);
+            zsum += wv;
+            const float *vec = ws.vec + ((size_t)qi * a.units + v) * D;
+            for (int x = threadIdx.x; x < D; x += kThreads) o[x] = fmaf(wv, __ldcg(&vec[x]), o[x]);
+        }
+        const float inv = 1.f / zsum;
+        for (int x = threadIdx.x; x < D; x += kThreads) o[x] *= inv;
+    }
+    __syncthreads();
+    store_output<T, D>(a, b, h, 0, qi, o, M == -INFINITY ? -INFINITY : M + logf(zsum));
+    if (threadIdx.x == 0) ws.counters[qi] = 0;
+}
+
+// General prefill path: one CTA per query, units in turn, running combination.
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) attend_prefill_general_kernel(AttendArgs a) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const UnitSmem s = unit_smem<T, D>(smem);
+    const int64_t qi = blockIdx.x;
+    const int i = (int)(qi % a.Lq);
+    const int h = (int)((qi / a.Lq) % a.H);
+    const int b = (int)(qi / ((int64_t)a.Lq * a.H));
+    const int t = i;
+    const int nsel = a.topk > 0 ? a.nsel[qi] : 0;
+    const T *qrow = static_cast<const T *>(a.Q.ptr) + b * a.Q.sb + h * a.Q.sh + i * a.Q.st;
+    const T *kh = static_cast<const T *>(a.K.ptr) + b * a.K.sb + h * a.K.sh;
+    const T *vh = static_cast<const T *>(a.V.ptr) + b * a.V.sb + h * a.V.sh;
+    // thread x (< D) owns output column x
+    float M = -INFINITY, zsum = 0.f, acc = 0.f;
+    for (int u = 0; u < a.units; ++u) {
+        const UnitPlan p = plan_unit(u, t, a.topk, a.W, a.idx + qi * a.topk, a.score + qi * a.topk, nsel);
+        if (p.rows == 0) continue;
+        unit_issue<T, D>(s, qrow, kh + (int64_t)p.start * a.K.st, a.K.st, vh + (int64_t)p.start * a.V.st,
+                         a.V.st, p.rows);
+        const float lse_tile = unit_compute<T, D>(s, p.rows, a.scale);
+        const float m = p.is_chunk ? p.mass : lse_tile;
+        if (m != -INFINITY) {
+            const float Mn = fmaxf(M, m);
+            const float fo = expf(M - Mn), fn = expf(m - Mn);
+            zsum = zsum * fo + fn;
+            if (threadIdx.x < D) acc = acc * fo + fn * s.red[threadIdx.x];
+            M = Mn;
+        }
+        __syncthreads();  // shared tiles are rewritten by the next unit
+    }
+    float *o = s.red;
+    if (threadIdx.x < D) o[threadIdx.x] = M == -INFINITY ? 0.f : acc / zsum;
+    __syncthreads();
+    store_output<T, D>(a, b, h, i, qi, o, M == -INFINITY ? -INFINITY : M + logf(zsum));
+}
+
+template <typename T, int D>
+hils_status launch_decode(const AttendArgs &a, cudaStream_t st) {
+    using Cfg = UnitCfg<T, D>;
+    const int nq = a.B * a.H;
+    if (nq == 0) return HILS_OK;
+    cudaError_t e = cudaFuncSetAttribute(attend_decode_kernel<T, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    attend_decode_kernel<T, D><<<dim3(a.units, nq), kThreads, Cfg::kSmemBytes, st>>>(a);
+    return record_cuda_error(cudaGetLastError());
+}
+
+template <typename T, int D>
+hils_status launch_prefill_general(const AttendArgs &a, cudaStream_t st) {
+    using Cfg = UnitCfg<T, D>;
+    const int64_t nq = (int64_t)a.B * a.H * a.Lq;
+    if (nq == 0) return HILS_OK;
+    cudaError_t e = cudaFuncSetAttribute(attend_prefill_general_kernel<T, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    attend_prefill_general_kernel<T, D><<<(unsigned)nq, kThreads, Cfg::kSmemBytes, st>>>(a);
+    return record_cuda_error(cudaGetLastError());
+}
+
+}  // namespace
+
+size_t attend_decode_ws_bytes(int queries, int units, int d) {
+    return align256((size_t)queries * sizeof(int)) + align256((size_t)queries * units * sizeof(float)) +
+           (size_t)queries * units * d * sizeof(float);
+}
+
+hils_status launch_attend_decode(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s) {
+    if (dt == HILS_BF16) return d == 64 ? launch_decode<bf16, 64>(a, s) : launch_decode<bf16, 128>(a, s);
+    return d == 64 ? launch_decode<float, 64>(a, s) : launch_decode<float, 128>(a, s);
+}
+
+hils_status launch_attend_prefill_general(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s) {
+    if (dt == HILS_BF16)
+        return d == 64 ? launch_prefill_general<bf16, 64>(a, s) : launch_prefill_general<bf16, 128>(a, s);
+    return d == 64 ? launch_prefill_general<float, 64>(a, s) : launch_prefill_general<float, 128>(a, s);
+}
+
+}  // namespace hils

@@ -1,0 +1,265 @@
+// C-ABI entry points of libhils: argument validation, workspace sizing and dispatch
+// to one kernel launcher per stage. No call allocates, frees or synchronises.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "hils_internal.cuh"
+
+namespace hils {
+
+static thread_local char g_last_error[256] = "";
+
+hils_status record_cuda_error(cudaError_t e) {
+    if (e == cudaSuccess) return HILS_OK;
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return HILS_ERR_CUDA;
+}
+
+int device_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return 1;
+    return n;
+}
+
+namespace {
+
+size_t elem_size(hils_dtype dt) { return dt == HILS_BF16 ? 2 : 4; }
+
+// Common parameter checks; fills the effective scale.
+int check_params(const hils_params *p, float *scale) {
+    if (!p) return HILS_ERR_INVALID_ARG;
+    if (p->B < 0 || p->H < 0 || p->K < 0 || p->W < 0) return HILS_ERR_INVALID_ARG;
+    if (p->dtype != HILS_F32 && p->dtype != HILS_BF16) return HILS_ERR_UNSUPPORTED;
+    if (p->d != 64 && p->d != 128) return HILS_ERR_UNSUPPORTED;
+    if (p->S != kChunk) return HILS_ERR_UNSUPPORTED;
+    if (p->K > 32) return HILS_ERR_UNSUPPORTED;
+    if (p->flags != 0) return HILS_ERR_UNSUPPORTED;
+    if (!isfinite(p->scale)) return HILS_ERR_INVALID_ARG;
+    *scale = p->scale != 0.f ? p->scale : (float)(1.0 / sqrt((double)p->d));
+    return HILS_OK;
+}
+
+bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+
+// A [B, H, T, d] view with T rows used: non-null when it holds elements, 16-byte
+// aligned base and strides.
+int check_view(const void *ptr, int64_t sb, int64_t sh, int64_t st, int64_t rows, const hils_params *p) {
+    if ((int64_t)p->B * p->H * rows == 0) return HILS_OK;
+    if (!ptr) return HILS_ERR_INVALID_ARG;
+    const int64_t es = (int64_t)elem_size(p->dtype);
+    if (!aligned16(ptr)) return HILS_ERR_ALIGNMENT;
+    if ((sb * es) % 16 || (sh * es) % 16 || (st * es) % 16) return HILS_ERR_ALIGNMENT;
+    return HILS_OK;
+}
+
+int check_array(const void *ptr, int64_t count) {
+    if (count > 0 && !ptr) return HILS_ERR_INVALID_ARG;
+    if (ptr && ((uintptr_t)ptr & 3u)) return HILS_ERR_ALIGNMENT;
+    return HILS_OK;
+}
+
+int check_workspace(const void *ws, size_t have, size_t need) {
+    if (need == 0) return HILS_OK;
+    if (!ws || have < need) return HILS_ERR_WORKSPACE;
+    if (!aligned16(ws)) return HILS_ERR_ALIGNMENT;
+    return HILS_OK;
+}
+
+// Units per query of the attend kernels: one per kept chunk plus the window tiles
+// (at least one, so that an empty query still gets o = 0 and lse = -inf).
+int decode_units(const hils_params *p) {
+    const int u = p->K + (p->W + kChunk - 1) / kChunk;
+    return u > 0 ? u : 1;
+}
+
+size_t select_ws_for(const hils_params *p, int Lq, int C) {
+    int ctas = 0, tiles = 0;
+    select_split_plan(p->B, p->H, Lq, C, p->K, true, device_sm_count(), &ctas, &tiles);
+    return select_ws_bytes(p->B * p->H * Lq, ctas, p->K);
+}
+
+#define HILS_TRY(expr)                 \
+    do {                               \
+        const int _rc = (expr);        \
+        if (_rc != HILS_OK) return _rc; \
+    } while (0)
+
+}  // namespace
+}  // namespace hils
+
+using namespace hils;
+
+extern "C" {
+
+const char *hils_status_string(int status) {
+    switch (status) {
+    case HILS_OK: return "ok";
+    case HILS_ERR_INVALID_ARG: return "invalid argument";
+    case HILS_ERR_UNSUPPORTED: return "unsupported configuration (d in {64,128}, S = 64, K <= 32, flags = 0)";
+    case HILS_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case HILS_ERR_WORKSPACE: return "workspace missing or too small";
+    case HILS_ERR_CUDA: return "CUDA launch error";
+    default: return "unknown status";
+    }
+}
+
+const char *hils_last_cuda_error(void) { return g_last_error; }
+
+size_t hils_workspace_bytes(const hils_params *p, int call, int Lq, int C) {
+    float scale;
+    if (check_params(p, &scale) != HILS_OK || Lq < 0 || C < 0) return 0;
+    switch (call) {
+    case HILS_CALL_SELECT: return select_ws_for(p, Lq, C);
+    case HILS_CALL_ATTEND_PREFILL: return 0;
+    case HILS_CALL_ATTEND_DECODE: return attend_decode_ws_bytes(p->B * p->H, decode_units(p), p->d);
+    default: return 0;
+    }
+}
+
+int hils_workspace_init(void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (ws_bytes == 0) return HILS_OK;
+    if (!workspace) return HILS_ERR_INVALID_ARG;
+    return record_cuda_error(cudaMemsetAsync(workspace, 0, ws_bytes, stream));
+}
+
+int hils_summarize(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ, hils_tensor Ksum,
+                   float *Bsum, cudaStream_t stream) {
+    float scale;
+    HILS_TRY(check_params(p, &scale));
+    if (N < 0) return HILS_ERR_INVALID_ARG;
+    const int C = N / kChunk;
+    HILS_TRY(check_view(K.ptr, K.sb, K.sh, K.st, (int64_t)C * kChunk, p));
+    HILS_TRY(check_view(LQ.ptr, LQ.sb, LQ.sh, LQ.st, C, p));
+    HILS_TRY(check_view(Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st, C, p));
+    HILS_TRY(check_array(Bsum, (int64_t)p->B * p->H * C));
+    SummarizeArgs a;
+    a.K = {K.ptr, K.sb, K.sh, K.st};
+    a.LQ = {LQ.ptr, LQ.sb, LQ.sh, LQ.st};
+    a.Ksum = {Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st};
+    a.Bsum = Bsum;
+    a.B = p->B;
+    a.H = p->H;
+    a.C = C;
+    a.scale = scale;
+    return launch_summarize(p->dtype, p->d, a, stream);
+}
+
+int hils_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *qpos, hils_ctensor Ksum,
+                const float *Bsum, int C, int32_t *idx, float *score, int32_t *nsel, void *workspace,
+                size_t ws_bytes, cudaStream_t stream) {
+    float scale;
+    HILS_TRY(check_params(p, &scale));
+    if (Lq < 0 || C < 0) return HILS_ERR_INVALID_ARG;
+    const int64_t nq = (int64_t)p->B * p->H * Lq;
+    HILS_TRY(check_view(Qcal.ptr, Qcal.sb, Qcal.sh, Qcal.st, Lq, p));
+    HILS_TRY(check_view(Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st, C, p));
+    HILS_TRY(check_array(Bsum, (int64_t)p->B * p->H * C));
+    HILS_TRY(check_array(idx, nq * p->K));
+    HILS_TRY(check_array(score, nq * p->K));
+    HILS_TRY(check_array(nsel, nq));
+    if (qpos && ((uintptr_t)qpos & 3u)) return HILS_ERR_ALIGNMENT;
+    if (nq == 0) return HILS_OK;
+    SelectArgs a;
+    a.Qcal = {Qcal.ptr, Qcal.sb, Qcal.sh, Qcal.st};
+    a.Ksum = {Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st};
+    a.Bsum = Bsum;
+    a.qpos = qpos;
+    a.idx = idx;
+    a.score = score;
+    a.nsel = nsel;
+    a.B = p->B;
+    a.H = p->H;
+    a.Lq = Lq;
+    a.C = C;
+    a.topk = p->K;
+    a.scale = scale;
+    select_split_plan(p->B, p->H, Lq, C, p->K, qpos != nullptr, device_sm_count(), &a.ctas_per_query,
+                      &a.tiles_per_warp);
+    HILS_TRY(check_workspace(workspace, ws_bytes, select_ws_bytes((int)nq, a.ctas_per_query, p->K)));
+    a.ws = workspace;
+    return launch_select(p->dtype, p->d, a, stream);
+}
+
+int hils_attend_prefill(const hils_params *p, hils_ctensor Q, hils_ctensor K, hils_ctensor V, int N,
+                        const int32_t *idx, const float *score, const int32_t *nsel, hils_tensor O, float *lse,
+                        void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    float scale;
+    HILS_TRY(check_params(p, &scale));
+    if (N < 0) return HILS_ERR_INVALID_ARG;
+    const int64_t nq = (int64_t)p->B * p->H * N;
+    HILS_TRY(check_view(Q.ptr, Q.sb, Q.sh, Q.st, N, p));
+    HILS_TRY(check_view(K.ptr, K.sb, K.sh, K.st, N, p));
+    HILS_TRY(check_view(V.ptr, V.sb, V.sh, V.st, N, p));
+    HILS_TRY(check_view(O.ptr, O.sb, O.sh, O.st, N, p));
+    HILS_TRY(check_array(idx, nq * p->K));
+    HILS_TRY(check_array(score, nq * p->K));
+    HILS_TRY(check_array(nsel, p->K > 0 ? nq : 0));
+    HILS_TRY(check_array(lse, 0));
+    (void)workspace;
+    (void)ws_bytes;
+    if (nq == 0) return HILS_OK;
+    AttendArgs a;
+    a.Q = {Q.ptr, Q.sb, Q.sh, Q.st};
+    a.K = {K.ptr, K.sb, K.sh, K.st};
+    a.V = {V.ptr, V.sb, V.sh, V.st};
+    a.O = {O.ptr, O.sb, O.sh, O.st};
+    a.lse = lse;
+    a.idx = idx;
+    a.score = score;
+    a.nsel = nsel;
+    a.qpos = nullptr;
+    a.cache_len = nullptr;
+    a.B = p->B;
+    a.H = p->H;
+    a.Lq = N;
+    a.topk = p->K;
+    a.W = p->W;
+    a.scale = scale;
+    a.units = decode_units(p);
+    a.ws = nullptr;
+    return launch_attend_prefill_general(p->dtype, p->d, a, stream);
+}
+
+int hils_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hils_ctensor Vc,
+                       const int32_t *cache_len, const int32_t *idx, const float *score, const int32_t *nsel,
+                       hils_tensor O, float *lse, void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    float scale;
+    HILS_TRY(check_params(p, &scale));
+    const int64_t nq = (int64_t)p->B * p->H;
+    HILS_TRY(check_view(Q.ptr, Q.sb, Q.sh, Q.st, 1, p));
+    HILS_TRY(check_view(Kc.ptr, Kc.sb, Kc.sh, Kc.st, 1, p));
+    HILS_TRY(check_view(Vc.ptr, Vc.sb, Vc.sh, Vc.st, 1, p));
+    HILS_TRY(check_view(O.ptr, O.sb, O.sh, O.st, 1, p));
+    HILS_TRY(check_array(cache_len, p->B));
+    HILS_TRY(check_array(idx, nq * p->K));
+    HILS_TRY(check_array(score, nq * p->K));
+    HILS_TRY(check_array(nsel, p->K > 0 ? nq : 0));
+    HILS_TRY(check_array(lse, 0));
+    if (nq == 0) return HILS_OK;
+    const int units = decode_units(p);
+    HILS_TRY(check_workspace(workspace, ws_bytes, attend_decode_ws_bytes((int)nq, units, p->d)));
+    AttendArgs a;
+    a.Q = {Q.ptr, Q.sb, Q.sh, Q.st};
+    a.K = {Kc.ptr, Kc.sb, Kc.sh, Kc.st};
+    a.V = {Vc.ptr, Vc.sb, Vc.sh, Vc.st};
+    a.O = {O.ptr, O.sb, O.sh, O.st};
+    a.lse = lse;
+    a.idx = idx;
+    a.score = score;
+    a.nsel = nsel;
+    a.qpos = nullptr;
+    a.cache_len = cache_len;
+    a.B = p->B;
+    a.H = p->H;
+    a.Lq = 1;
+    a.topk = p->K;
+    a.W = p->W;
+    a.scale = scale;
+    a.units = units;
+    a.ws = workspace;
+    return launch_attend_decode(p->dtype, p->d, a, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,172 @@
+// Internal declarations and device helpers of libhils (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hils.h"
+
+namespace hils {
+
+constexpr int kChunk = 64;          // chunk size S (tokens per chunk)
+constexpr unsigned kFull = 0xffffffffu;
+
+typedef __nv_bfloat16 bf16;
+
+// ------------------------------------------------------------------ launch args
+
+// Strided [B, H, T, d] view in elements.
+struct View {
+    const void *ptr;
+    int64_t sb, sh, st;
+};
+struct MutView {
+    void *ptr;
+    int64_t sb, sh, st;
+};
+
+struct SummarizeArgs {
+    View K, LQ;
+    MutView Ksum;
+    float *Bsum;
+    int B, H, C;
+    float scale;
+};
+
+struct SelectArgs {
+    View Qcal, Ksum;
+    const float *Bsum;
+    const int32_t *qpos;   // [B, Lq] or null (t = i)
+    int32_t *idx;
+    float *score;
+    int32_t *nsel;
+    int B, H, Lq, C, topk;
+    float scale;
+    // split search over chunk ranges (decode-like shapes)
+    int ctas_per_query;    // grid.x of the split kernel
+    int tiles_per_warp;    // 128-chunk tiles each warp scans
+    void *ws;              // per-query partial lists + arrival counters
+};
+
+struct AttendArgs {
+    View Q, K, V;
+    MutView O;
+    float *lse;            // [B, H, Lq] or null
+    const int32_t *idx;    // [B, H, Lq, Ksel]
+    const float *score;
+    const int32_t *nsel;
+    const int32_t *qpos;   // prefill: null (t = i); decode: null and cache_len set
+    const int32_t *cache_len;  // decode: [B]
+    int B, H, Lq, topk, W;
+    float scale;
+    int units;             // units per query: K chunk units + window tiles
+    void *ws;
+};
+
+// Host launchers (one translation unit each). They return HILS_OK or HILS_ERR_CUDA.
+hils_status launch_summarize(hils_dtype dt, int d, const SummarizeArgs &a, cudaStream_t s);
+hils_status launch_select(hils_dtype dt, int d, const SelectArgs &a, cudaStream_t s);
+hils_status launch_attend_decode(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s);
+hils_status launch_attend_prefill_general(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s);
+
+// Workspace layouts (bytes); shared by the host size query and the kernels.
+size_t select_ws_bytes(int queries, int ctas_per_query, int K);
+size_t attend_decode_ws_bytes(int queries, int units, int d);
+
+// Choice of the split search for hils_select; identical on the size query and the call.
+void select_split_plan(int B, int H, int Lq, int C, int K, bool has_qpos, int num_sms,
+                       int *ctas_per_query, int *tiles_per_warp);
+
+int device_sm_count();
+hils_status record_cuda_error(cudaError_t e);
+
+// ------------------------------------------------------------------ device helpers
+
+template <typename T>
+struct Vec;  // one 16-byte vector of T
+template <>
+struct Vec<float> {
+    static constexpr int kN = 4;
+};
+template <>
+struct Vec<bf16> {
+    static constexpr int kN = 8;
+};
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Widens the 16 bytes `v` into Vec<T>::kN floats.
+__device__ __forceinline__ void widen(const uint4 &v, float (&f)[8], bf16) {
+    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x);
+    f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z);
+    f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+}
+__device__ __forceinline__ void widen(const uint4 &v, float (&f)[4], float) {
+    f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+}
+
+// Sum of the element-wise products of two 16-byte vectors of T, added to acc.
+template <typename T>
+__device__ __forceinline__ float dot16(const uint4 &a, const uint4 &b, float acc) {
+    float fa[Vec<T>::kN], fb[Vec<T>::kN];
+    widen(a, fa, T());
+    widen(b, fb, T());
+#pragma unroll
+    for (int i = 0; i < Vec<T>::kN; ++i) acc = fmaf(fa[i], fb[i], acc);
+    return acc;
+}
+
+// Two adjacent elements of T widened to float.
+__device__ __forceinline__ float2 load2(const bf16 *p) {
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
+    return make_float2(bf16lo(w), bf16hi(w));
+}
+__device__ __forceinline__ float2 load2(const float *p) { return *reinterpret_cast<const float2 *>(p); }
+
+// Two floats rounded to T (nearest-even) and stored.
+__device__ __forceinline__ void store2(bf16 *p, float a, float b) {
+    *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(a, b);
+}
+__device__ __forceinline__ void store2(float *p, float a, float b) {
+    *reinterpret_cast<float2 *>(p) = make_float2(a, b);
+}
+
+__device__ __forceinline__ double to_double(bf16 x) { return (double)__bfloat162float(x); }
+__device__ __forceinline__ double to_double(float x) { return (double)x; }
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+// Monotone map of a float onto unsigned ints (larger float -> larger key); finite
+// floats and -inf map to keys > 0, so 0 can mean "no element".
+__device__ __forceinline__ unsigned ordered_key(float f) {
+    const unsigned b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_to_float(unsigned k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+}  // namespace hils

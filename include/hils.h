@@ -1,0 +1,194 @@
+/*
+ * libhils: HiLS-Attention forward pass on NVIDIA B200 (sm_100a). C ABI.
+ *
+ * The method is Hierarchical Landmark Sparse attention, from "Hierarchical Sparse
+ * Attention Done Right: Toward Infinite Context Modeling" (arXiv 2607.02980). The
+ * citations below name the page (picx.dev summary, or the rcap.io post) and the
+ * section or equation on it.
+ *
+ * Stages, one entry point each:
+ *   hils_summarize       landmark chunk summaries k'_c, b'_c         (summary, Methodology 1, Eq. 8)
+ *   hils_select          chunk scores s^_{i,c} and top-K selection   (summary, Eq. 7 and Methodology 2;
+ *                                                                     post, pseudocode figure)
+ *   hils_attend_prefill  hierarchical softmax over the selected chunks plus the sliding
+ *   hils_attend_decode   window, for every position of a sequence, or for one new token
+ *                        per sequence against a KV cache            (summary, Methodology 2, Eq. 10;
+ *                                                                     post, pseudocode figure)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Tensors. A 4-D tensor [B, H, T, d] is described by hils_ctensor/hils_tensor:
+ *   element (b, h, t, x) is at ptr + b*sb + h*sh + t*st + x, with strides counted in
+ *   elements of params->dtype. The head dimension x is contiguous (stride 1).
+ *   ptr must be 16-byte aligned, and sb, sh, st times the element size must be
+ *   multiples of 16 bytes (HILS_ERR_ALIGNMENT otherwise).
+ *   Plain arrays (Bsum, idx, score, nsel, lse, qpos, cache_len) are dense row-major
+ *   with the shape given beside them.
+ * Memory. Every pointer is device memory that the caller allocates and owns. The
+ *   library allocates nothing, frees nothing and never synchronises: each call
+ *   enqueues its kernels on `stream` and returns.
+ * Workspace. Calls that need scratch memory take (workspace, ws_bytes). Query the
+ *   size with hils_workspace_bytes(). The workspace carries arrival counters that
+ *   every call leaves at zero; zero a new workspace once before its first use (for
+ *   example with hils_workspace_init). Calls that share a workspace must not
+ *   overlap in time on the device.
+ * Errors. A call validates its arguments before launching anything and returns a
+ *   hils_status. HILS_ERR_CUDA means a launch failed; hils_last_cuda_error() then
+ *   gives the CUDA error text for the calling thread. No exception crosses the ABI.
+ * Threads. Calls keep no global state and may be made from several host threads.
+ *
+ * Stated readings of the method (the pages leave these open):
+ *   - Every dot product is multiplied by scale = 1/sqrt(d); the entropy bias b'_c
+ *     is added unscaled (Eq. 7).
+ *   - Chunk c holds tokens [c*S, (c+1)*S). It is eligible for the query at position
+ *     t when c < floor(t / S): only complete chunks strictly before the query's own.
+ *   - The sliding window is the W most recent tokens including the query's own,
+ *     [max(0, t-W+1), t]. It joins the selected chunks under one normaliser
+ *     Z^_i = sum_{c selected} exp(s^_{i,c}) + sum_{j in window} exp(scale q_i.k_j),
+ *     and a token that lies both in a selected chunk and in the window enters
+ *     through both terms.
+ *   - Queries with fewer than K eligible chunks keep all of them; the rest of their
+ *     selection row is padding (idx -1, score -inf). A query with no selected chunk
+ *     and an empty window gets o = 0 and lse = -inf.
+ */
+#ifndef HILS_H
+#define HILS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { HILS_F32 = 0, HILS_BF16 = 1 } hils_dtype;
+
+typedef enum {
+    HILS_OK = 0,
+    HILS_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent shape */
+    HILS_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, S != 64, K > 32, flags != 0 */
+    HILS_ERR_ALIGNMENT = 3,    /* pointer or stride not 16-byte aligned */
+    HILS_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
+    HILS_ERR_CUDA = 5          /* a kernel launch failed; see hils_last_cuda_error() */
+} hils_status;
+
+/* Read-only / writable strided view of a [B, H, T, d] tensor (strides in elements). */
+typedef struct {
+    const void *ptr;
+    int64_t sb, sh, st;
+} hils_ctensor;
+
+typedef struct {
+    void *ptr;
+    int64_t sb, sh, st;
+} hils_tensor;
+
+/* Problem description shared by every call.
+ *   B      batch (sequences), H heads (one KV head per query head),
+ *   d      head dimension: 64 or 128,
+ *   S      chunk size: 64,
+ *   K      chunks kept per query (top-K): 0..32,
+ *   W      sliding-window length in tokens: >= 0,
+ *   dtype  element type of every Q/K/V/LQ/Ksum/O tensor,
+ *   scale  softmax scale; 0 selects (float)(1/sqrt(d)),
+ *   flags  reserved, must be 0. */
+typedef struct {
+    int B, H, d, S, K, W;
+    hils_dtype dtype;
+    float scale;
+    uint32_t flags;
+} hils_params;
+
+/* Which call a workspace size is asked for. */
+typedef enum {
+    HILS_CALL_SELECT = 0,
+    HILS_CALL_ATTEND_PREFILL = 1,
+    HILS_CALL_ATTEND_DECODE = 2
+} hils_call;
+
+/* Landmark chunk summaries (summary page, Methodology 1, Eq. 8).
+ * For every complete chunk c < C = floor(N / S) of every (b, h):
+ *   l_j = scale * q'_c . k_j for the S keys of the chunk, p = softmax(l),
+ *   k'_c = sum_j p_j k_j,   b'_c = -sum_j p_j log p_j.
+ *   K     [B, H, N, d]  keys of the sequence (only the first C*S positions are read)
+ *   N     number of tokens
+ *   LQ    [B, H, C, d]  landmark query q'_c of each chunk
+ *   Ksum  [B, H, C, d]  out: k'_c in dtype (float32 sums rounded to nearest-even)
+ *   Bsum  [B, H, C]     out: b'_c, float32, dense
+ * Returns HILS_OK, or an error before any launch. */
+int hils_summarize(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ,
+                   hils_tensor Ksum, float *Bsum, cudaStream_t stream);
+
+/* Chunk scores and top-K (summary page, Eq. 7 and Methodology 2; post, pseudocode).
+ * For every query i at position t_i, every eligible chunk c < min(floor(t_i/S), C) gets
+ *   s^_{i,c} = scale * (q~_i . k'_c) + b'_c,
+ * and the K chunks with the largest s^ are kept; equal scores go to the lower chunk
+ * index. The ranking is exact: it equals the ranking of the float64 value
+ * (sum_x q~_x k'_x) * scale + b'_c (products and sums in x order, each rounded to
+ * float64) computed from the stored inputs.
+ *   Qcal  [B, H, Lq, d]  calibrated scoring query q~_i
+ *   Lq    queries per (b, h)
+ *   qpos  [B, Lq] int32 position t of each query, or NULL for t = i (prefill)
+ *   Ksum  [B, H, C, d]  summary keys k'_c;  Bsum [B, H, C] float32 entropy biases b'_c
+ *   C     number of summarised chunks
+ *   idx   [B, H, Lq, K] int32 out: kept chunks in ascending chunk index, -1 padding
+ *   score [B, H, Lq, K] float32 out: s^_{i,c} of each kept chunk (float32 evaluation,
+ *         within 2^-9 * scale * |q~| |k'_c| + 2^-20 |s^| of the exact value), -inf padding
+ *   nsel  [B, H, Lq] int32 out: number of kept chunks, min(K, eligible)
+ *   workspace, ws_bytes: scratch of hils_workspace_bytes(p, HILS_CALL_SELECT, Lq, C) bytes
+ *         (may be 0 bytes, then workspace may be NULL). */
+int hils_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *qpos,
+                hils_ctensor Ksum, const float *Bsum, int C,
+                int32_t *idx, float *score, int32_t *nsel,
+                void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Hierarchical softmax for every position of a sequence (summary page, Methodology 2,
+ * Eq. 10; post, pseudocode). Query i sits at t = i and attends to
+ *   - each kept chunk c with weight exp(s^_{i,c}) / Z^_i on the chunk's own softmax
+ *     output sum_{j in c} softmax_j(scale q_i.k_j) v_j, and
+ *   - each window token j in [max(0, i-W+1), i] with weight exp(scale q_i.k_j) / Z^_i.
+ *   Q, K, V  [B, H, N, d]
+ *   idx, score, nsel: as written by hils_select (score is used as the chunk's log-mass;
+ *         passing exact log Z_{i,c} instead gives exact block-sparse attention)
+ *   O    [B, H, N, d]  out, dtype (float32 result rounded to nearest-even)
+ *   lse  [B, H, N] float32 out: log Z^_i, or NULL
+ *   workspace, ws_bytes: hils_workspace_bytes(p, HILS_CALL_ATTEND_PREFILL, N, C). */
+int hils_attend_prefill(const hils_params *p, hils_ctensor Q, hils_ctensor K, hils_ctensor V,
+                        int N, const int32_t *idx, const float *score, const int32_t *nsel,
+                        hils_tensor O, float *lse, void *workspace, size_t ws_bytes,
+                        cudaStream_t stream);
+
+/* Hierarchical softmax for one new token per sequence against its KV cache (same
+ * passages). Sequence b holds cache_len[b] tokens and its query sits at
+ * t = cache_len[b] - 1 (the query's own key and value are the last cache entries).
+ *   Q      [B, H, 1, d]
+ *   Kc, Vc [B, H, Lmax, d] KV cache; positions >= cache_len[b] are never read
+ *   cache_len [B] int32 on the device
+ *   idx, score, nsel: [B, H, 1, K] / [B, H, 1] from hils_select with qpos = cache_len - 1
+ *   O      [B, H, 1, d] out;  lse [B, H] float32 out, or NULL
+ *   workspace, ws_bytes: hils_workspace_bytes(p, HILS_CALL_ATTEND_DECODE, 1, 0). */
+int hils_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hils_ctensor Vc,
+                       const int32_t *cache_len,
+                       const int32_t *idx, const float *score, const int32_t *nsel,
+                       hils_tensor O, float *lse, void *workspace, size_t ws_bytes,
+                       cudaStream_t stream);
+
+/* Bytes of workspace a call needs for these sizes (Lq = queries per (b, h); C =
+ * summarised chunks). Returns 0 for invalid parameters. */
+size_t hils_workspace_bytes(const hils_params *p, int call, int Lq, int C);
+
+/* Zeroes a workspace on `stream` (cudaMemsetAsync); needed once after allocation. */
+int hils_workspace_init(void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Static description of a status code. */
+const char *hils_status_string(int status);
+
+/* CUDA error text of the calling thread's last HILS_ERR_CUDA ("" if none). */
+const char *hils_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HILS_H */

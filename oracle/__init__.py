@@ -163,8 +163,9 @@ def attend(Q, Kc, Vc, idx, score, nsel, S: int, W: int, scale: float, qpos=None)
     """Eq. 10 output. Returns (O [B,H,Lq,d] float64, lse [B,H,Lq] float64)."""
     Q, Kc, Vc = _as_tensor(Q), _as_tensor(Kc), _as_tensor(Vc)
     B, H, Lq, d = Q.shape
-    idx = _i32(idx).reshape(B, H, Lq, -1)
-    K = idx.shape[3]
+    idx = _i32(idx)
+    K = idx.shape[-1]
+    idx = idx.reshape(B, H, Lq, K)
     score = _as_tensor(score).reshape(B, H, Lq, K).contiguous()
     nsel = _i32(nsel).reshape(B, H, Lq)
     O = np.zeros((B, H, Lq, d), np.float64)
@@ -195,8 +196,9 @@ def chunk_logmass(Q, Kc, idx, nsel, S: int, scale: float):
     """Exact log Z_{i,c} of each selected chunk (Introduction, chunk mass)."""
     Q, Kc = _as_tensor(Q), _as_tensor(Kc)
     B, H, Lq, d = Q.shape
-    idx = _i32(idx).reshape(B, H, Lq, -1)
-    K = idx.shape[3]
+    idx = _i32(idx)
+    K = idx.shape[-1]
+    idx = idx.reshape(B, H, Lq, K)
     nsel = _i32(nsel).reshape(B, H, Lq)
     out = np.zeros((B, H, Lq, K), np.float64)
     _check(_load().or_chunk_logmass(B, H, d, S, K, float(scale), _desc(Q), Lq, _desc(Kc),

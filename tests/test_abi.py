@@ -1,0 +1,140 @@
+"""C-ABI checks that need no GPU: the library builds and loads, it exports every
+function include/hils.h declares, and invalid arguments are rejected by the host
+checks before any launch (so these calls never touch a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hierarchical_chunk_sparse_b200 as hils
+from hierarchical_chunk_sparse_b200 import build as hbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hils.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    hbuild.build()
+    return hils.load_library()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hils_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declarations_are_exported(lib):
+    names = _declared()
+    assert "hils_summarize" in names and "hils_attend_decode" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in hils.h but not exported"
+    assert set(hils.EXPORTS) <= set(names)
+
+
+def test_library_exports_no_undeclared_entry_points(lib):
+    out = os.popen(f"nm -D --defined-only {hils.LIB_PATH}").read()
+    exported = set(re.findall(r"\b(hils_[a-z_]+)$", out, flags=re.M))
+    assert exported == set(_declared())
+
+
+def _p(**kw):
+    base = dict(B=1, H=2, d=128, K=16, W=512, dtype=hils.torch.bfloat16)
+    base.update(kw)
+    return hils.Params(**base)
+
+
+T = hils._CTensor
+ALIGNED = 0x10000  # never dereferenced: every call below fails its host checks first
+
+
+def _summ(lib, p, K=None, N=256, LQ=None, Ksum=None, Bsum=ALIGNED):
+    K = K or T(ALIGNED, 32768, 32768, 128)
+    LQ = LQ or T(ALIGNED, 512, 512, 128)
+    Ksum = Ksum or T(ALIGNED, 512, 512, 128)
+    return lib.hils_summarize(ctypes.byref(p.c()), K, N, LQ, Ksum, Bsum, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), 2), (dict(S=32), 2), (dict(K=33), 2), (dict(flags=1), 2),
+    (dict(B=-1), 1), (dict(W=-1), 1), (dict(K=-2), 1), (dict(scale=float("nan")), 1),
+])
+def test_invalid_params_rejected(lib, kw, code):
+    p = _p(**{k: v for k, v in kw.items() if k not in ("S", "flags")})
+    if "S" in kw:
+        p.S = kw["S"]
+    if "flags" in kw:
+        p.flags = kw["flags"]
+    assert _summ(lib, p, Bsum=None if code == 1 else ALIGNED) == code
+
+
+def test_bad_dtype_rejected(lib):
+    p = _p()
+    c = p.c()
+    c.dtype = 7
+    assert lib.hils_summarize(ctypes.byref(c), T(ALIGNED, 0, 0, 128), 64, T(ALIGNED, 0, 0, 128),
+                              T(ALIGNED, 0, 0, 128), ALIGNED, None) == 2
+
+
+def test_null_params_and_pointers(lib):
+    assert lib.hils_summarize(None, T(ALIGNED, 0, 0, 128), 64, T(ALIGNED, 0, 0, 128),
+                              T(ALIGNED, 0, 0, 128), ALIGNED, None) == 1
+    assert _summ(lib, _p(), K=T(None, 0, 0, 128)) == 1
+    assert _summ(lib, _p(), Bsum=None) == 1
+    assert _summ(lib, _p(), N=-5) == 1
+
+
+@pytest.mark.parametrize("view", [T(ALIGNED + 2, 32768, 32768, 128), T(ALIGNED, 32768, 32768, 132),
+                                  T(ALIGNED, 32769, 32768, 128)])
+def test_misalignment_rejected(lib, view):
+    assert _summ(lib, _p(), K=view) == 3
+
+
+def test_select_workspace_too_small(lib):
+    p = _p(B=1, H=2)
+    c = p.c()
+    need = lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_SELECT, 1, 20000)
+    assert need > 0
+    rc = lib.hils_select(ctypes.byref(c), T(ALIGNED, 256, 128, 128), 1, ALIGNED, T(ALIGNED, 0, 0, 128),
+                         ALIGNED, 20000, ALIGNED, ALIGNED, ALIGNED, ALIGNED, need - 16, None)
+    assert rc == 4
+    rc = lib.hils_select(ctypes.byref(c), T(ALIGNED, 256, 128, 128), 1, ALIGNED, T(ALIGNED, 0, 0, 128),
+                         ALIGNED, 20000, ALIGNED, ALIGNED, ALIGNED, None, need, None)
+    assert rc == 4
+
+
+def test_decode_workspace_too_small(lib):
+    p = _p(B=1, H=2)
+    c = p.c()
+    need = lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_ATTEND_DECODE, 1, 0)
+    units = 16 + 512 // 64
+    assert need >= 2 * units * 128 * 4
+    v = T(ALIGNED, 256, 128, 128)
+    rc = lib.hils_attend_decode(ctypes.byref(c), v, v, v, ALIGNED, ALIGNED, ALIGNED, ALIGNED, v,
+                                ALIGNED, ALIGNED, need - 1, None)
+    assert rc == 4
+
+
+def test_workspace_sizes(lib):
+    assert lib.hils_workspace_bytes(None, 0, 1, 1) == 0
+    assert lib.hils_workspace_bytes(ctypes.byref(_p(d=80).c()), 0, 1, 1) == 0
+    assert lib.hils_workspace_bytes(ctypes.byref(_p().c()), hils.HILS_CALL_ATTEND_PREFILL, 8192, 128) == 0
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.hils_status_string(code)
+    assert b"unknown" in lib.hils_status_string(99)
+    assert lib.hils_last_cuda_error() is not None
+
+
+def test_binding_refuses_a_missing_library(tmp_path):
+    with pytest.raises(ImportError):
+        hils._lib_saved = hils._lib
+        hils._lib = None
+        try:
+            hils.load_library(str(tmp_path / "missing.so"))
+        finally:
+            hils._lib = hils._lib_saved
