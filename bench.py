@@ -151,6 +151,15 @@ def time_steps(fn, steps, flush, stream):
     return [s.elapsed_time(e) for s, e in ev]
 
 
+def graphed(fn, stream):
+    """Captures fn (already warmed up) into a CUDA graph on `stream`; returns replay()."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    stream.synchronize()
+    return g.replay
+
+
 def dist_ctx():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -390,8 +399,52 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args):
+    """Small cases for Nsight Compute captures (a few GB on the device at most).
+
+    decode-select: the 512K decode geometry (H=32, 8191 eligible chunks, K=16) on a
+                   random summary table (68 MB) without a KV cache;
+    decode-attend: the decode attend with H=32, K=16, W=512 on a 128K-token cache (2.1 GB);
+    prefill:       the full 8K prefill workload (summarise, select, attend).
+    Runs `warmup + steps` plain launches of the case and exits."""
+    import hierarchical_chunk_sparse_b200 as hils
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hils.load_library()
+    case = args.profile
+    if case == "decode-select":
+        w = WORKLOADS[4]
+        g = torch.Generator(device=dev).manual_seed(1)
+        Q = torch.randn(w.B, w.H, 1, w.d, generator=g, device=dev).to(w.dtype)
+        Ksum = (torch.randn(w.B, w.H, w.C, w.d, generator=g, device=dev) * 0.3).to(w.dtype)
+        Bsum = torch.rand(w.B, w.H, w.C, generator=g, device=dev) * 0.5 + 3.7
+        p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype)
+        qpos = torch.full((w.B, 1), w.N - 1, dtype=torch.int32, device=dev)
+        idx = torch.empty(w.B, w.H, 1, w.K, dtype=torch.int32, device=dev)
+        score = torch.empty(w.B, w.H, 1, w.K, device=dev)
+        nsel = torch.empty(w.B, w.H, 1, dtype=torch.int32, device=dev)
+        ws = hils.alloc_workspace(p, hils.HILS_CALL_SELECT, 1, w.C, device=dev)
+        fn = lambda: hils.hils_select(p, Q, Ksum, Bsum, idx, score, nsel, qpos=qpos, workspace=ws)  # noqa
+    elif case == "decode-attend":
+        db = DecodeBench(WORKLOADS[4].replace(N=131072, needles=0), dev)
+        db.select()
+        fn = db.attend
+    elif case == "prefill":
+        fn = PrefillBench(WORKLOADS[2], dev).step
+    else:
+        raise SystemExit(f"unknown profile case {case}")
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": case, "launches": args.warmup + args.steps}))
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile", default=None,
+                    choices=["decode-select", "decode-attend", "prefill"],
+                    help="run a small case for an ncu capture and exit")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
@@ -400,6 +453,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.profile:
+        run_profile_case(args)
+        return
     w = WORKLOADS[4]
     if args.impl == "reference":
         run_reference(args, w)
@@ -427,17 +483,24 @@ def main():
         for _ in range(args.warmup):
             db.step()
     stream.synchronize()
+    # one decode step = hils_select + hils_attend_decode, replayed as a CUDA graph
+    step_g = graphed(db.step, stream)
+    sel_g = graphed(db.select, stream)
+    att_g = graphed(db.attend, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step_g()
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
-        per = time_steps(db.step, args.steps, flush, stream)
+        per = time_steps(step_g, args.steps, flush, stream)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(statistics.mean(per), world, dev)
     value = world * w.B / (ms / 1e3)
     # per-kernel times (same protocol)
-    t_sel = statistics.mean(time_steps(db.select, args.steps, flush, stream))
-    t_att = statistics.mean(time_steps(db.attend, args.steps, flush, stream))
+    t_sel = statistics.mean(time_steps(sel_g, args.steps, flush, stream))
+    t_att = statistics.mean(time_steps(att_g, args.steps, flush, stream))
     by = decode_bytes(w)
     hbm = peaks["hbm_gbs"]
     sel_gbs = by["select"] / (t_sel * 1e-3) / 1e9
@@ -463,10 +526,11 @@ def main():
         with torch.cuda.stream(stream):
             for _ in range(3):
                 pb.step()
+        stream.synchronize()
         n = max(3, min(args.steps, 20))
-        pt = statistics.mean(time_steps(pb.step, n, flush, stream))
+        pt = statistics.mean(time_steps(graphed(pb.step, stream), n, flush, stream))
         pt = max_over_ranks(pt, world, dev)
-        ks = {k: statistics.mean(time_steps(getattr(pb, k), n, flush, stream))
+        ks = {k: statistics.mean(time_steps(graphed(getattr(pb, k), stream), n, flush, stream))
               for k in ("summarize", "select", "attend")}
         fl = prefill_flops(wp)
         tf = fl / (pt * 1e-3) / 1e12

@@ -120,6 +120,20 @@ def _stream(stream):
     return stream.cuda_stream
 
 
+def _expect(call: str, name: str, t, shape, dtype=None) -> None:
+    """Shape (and dtype) check of one argument against the parameters; raises before the
+    C call, so that a mismatched tensor can never be read or written out of bounds."""
+    if t is None:
+        return
+    got = tuple(t.shape)
+    if got != tuple(shape):
+        raise ValueError(f"{call}: {name} has shape {got}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{call}: {name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{call}: {name} must be a CUDA tensor")
+
+
 def _check(call: str, rc: int) -> None:
     if rc != 0:
         lib = load_library()
@@ -145,6 +159,14 @@ def _ws(workspace):
 def hils_summarize(p: Params, K, LQ, Ksum, Bsum, N: int | None = None, stream=None) -> None:
     """Eq. 8 summaries of every complete chunk: Ksum [B,H,C,d], Bsum [B,H,C] float32."""
     n = K.shape[2] if N is None else N
+    B, H, d, C = p.B, p.H, p.d, n // p.S
+    if K.shape[0] != B or K.shape[1] != H or K.shape[3] != d or K.shape[2] < C * p.S:
+        raise ValueError(f"hils_summarize: K has shape {tuple(K.shape)} for B={B} H={H} d={d} N={n}")
+    if K.dtype != p.dtype:
+        raise ValueError("hils_summarize: K dtype differs from params")
+    _expect("hils_summarize", "LQ", LQ, (B, H, C, d), p.dtype)
+    _expect("hils_summarize", "Ksum", Ksum, (B, H, C, d), p.dtype)
+    _expect("hils_summarize", "Bsum", Bsum, (B, H, C), torch.float32)
     _check("hils_summarize", load_library().hils_summarize(
         ctypes.byref(p.c()), _view(K), n, _view(LQ), _view(Ksum), _ptr(Bsum), _stream(stream)))
 
@@ -154,6 +176,15 @@ def hils_select(p: Params, Qcal, Ksum, Bsum, idx, score, nsel, qpos=None, worksp
     """Eq. 7 scores and exact top-K: idx/score [B,H,Lq,K], nsel [B,H,Lq]."""
     lq = Qcal.shape[2] if Lq is None else Lq
     c = Ksum.shape[2] if C is None else C
+    B, H, d, K = p.B, p.H, p.d, p.K
+    _expect("hils_select", "Qcal", Qcal, (B, H, lq, d), p.dtype)
+    _expect("hils_select", "Ksum", Ksum, (B, H, c, d), p.dtype)
+    _expect("hils_select", "Bsum", Bsum, (B, H, c), torch.float32)
+    _expect("hils_select", "idx", idx, (B, H, lq, K), torch.int32)
+    _expect("hils_select", "score", score, (B, H, lq, K), torch.float32)
+    _expect("hils_select", "nsel", nsel, (B, H, lq), torch.int32)
+    if qpos is not None:
+        _expect("hils_select", "qpos", qpos, (B, lq), torch.int32)
     wp, wn = _ws(workspace)
     _check("hils_select", load_library().hils_select(
         ctypes.byref(p.c()), _view(Qcal), lq, _ptr(qpos), _view(Ksum), _ptr(Bsum), c,
@@ -164,6 +195,14 @@ def hils_attend_prefill(p: Params, Q, K, V, idx, score, nsel, O, lse=None, works
                         N: int | None = None, stream=None) -> None:
     """Eq. 10 for every position: O [B,H,N,d], lse [B,H,N] float32 (optional)."""
     n = Q.shape[2] if N is None else N
+    B, H, d, k = p.B, p.H, p.d, p.K
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("O", O)):
+        _expect("hils_attend_prefill", name, t, (B, H, n, d), p.dtype)
+    if k > 0:
+        _expect("hils_attend_prefill", "idx", idx, (B, H, n, k), torch.int32)
+        _expect("hils_attend_prefill", "score", score, (B, H, n, k), torch.float32)
+        _expect("hils_attend_prefill", "nsel", nsel, (B, H, n), torch.int32)
+    _expect("hils_attend_prefill", "lse", lse, (B, H, n), torch.float32)
     wp, wn = _ws(workspace)
     _check("hils_attend_prefill", load_library().hils_attend_prefill(
         ctypes.byref(p.c()), _view(Q), _view(K), _view(V), n, _ptr(idx), _ptr(score), _ptr(nsel),
@@ -172,7 +211,22 @@ def hils_attend_prefill(p: Params, Q, K, V, idx, score, nsel, O, lse=None, works
 
 def hils_attend_decode(p: Params, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse=None,
                        workspace=None, stream=None) -> None:
-    """Eq. 10 for one new token per sequence: O [B,H,1,d], lse [B,H] float32 (optional)."""
+    """Eq. 10 for one new token per sequence: O [B,H,1,d], lse [B,H] float32 (optional).
+
+    The cache tensors may be longer than any cache_len; the kernels read positions
+    below cache_len[b] only, which must not exceed the cache tensors' length."""
+    B, H, d, k = p.B, p.H, p.d, p.K
+    _expect("hils_attend_decode", "Q", Q, (B, H, 1, d), p.dtype)
+    _expect("hils_attend_decode", "O", O, (B, H, 1, d), p.dtype)
+    for name, t in (("Kc", Kc), ("Vc", Vc)):
+        if t.shape[0] != B or t.shape[1] != H or t.shape[3] != d or t.dtype != p.dtype or not t.is_cuda:
+            raise ValueError(f"hils_attend_decode: {name} has shape {tuple(t.shape)} / {t.dtype}")
+    _expect("hils_attend_decode", "cache_len", cache_len, (B,), torch.int32)
+    if k > 0:
+        _expect("hils_attend_decode", "idx", idx, (B, H, 1, k), torch.int32)
+        _expect("hils_attend_decode", "score", score, (B, H, 1, k), torch.float32)
+        _expect("hils_attend_decode", "nsel", nsel, (B, H, 1), torch.int32)
+    _expect("hils_attend_decode", "lse", lse, (B, H), torch.float32)
     wp, wn = _ws(workspace)
     _check("hils_attend_decode", load_library().hils_attend_decode(
         ctypes.byref(p.c()), _view(Q), _view(Kc), _view(Vc), _ptr(cache_len), _ptr(idx), _ptr(score),

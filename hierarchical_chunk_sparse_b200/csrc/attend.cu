@@ -203,6 +203,59 @@ __device__ __forceinline__ void store_output(const AttendArgs &a, int b, int h, 
     if (a.lse && threadIdx.x == 0) a.lse[qi] = lse;
 }
 
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float *scratch) {
+    v = is_max ? warp_max(v) : warp_sum(v);
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (lane == 0) scratch[w] = v;
+    __syncthreads();
+    float r = scratch[0];
+    for (int i = 1; i < kThreads / 32; ++i) r = is_max ? fmaxf(r, scratch[i]) : r + scratch[i];
+    return r;
+}
+
+// o = sum_u e^{m_u - M} o_u / sum_u e^{m_u - M} and lse = M + log(sum) over `units`
+// partials (masses m_u, vectors o_u, in global memory written by other CTAs). Writes o
+// to out[0..D) and lse to out[D]. Loads are issued in parallel: masses strided over
+// the threads, weights staged in shared memory in blocks, vectors unrolled.
+template <int D>
+__device__ void combine_units(const float *mass, const float *vec, int units, float *out, float *wts) {
+    constexpr int kBlock = 1024;
+    __shared__ float scratch[kThreads / 32];
+    float mloc = -INFINITY;
+    for (int v = threadIdx.x; v < units; v += kThreads) mloc = fmaxf(mloc, __ldcg(mass + v));
+    const float M = block_reduce(mloc, true, scratch);
+    float zloc = 0.f, acc = 0.f;
+    const int x = threadIdx.x;  // output column (D <= kThreads)
+    for (int v0 = 0; v0 < units; v0 += kBlock) {
+        const int nb = min(kBlock, units - v0);
+        __syncthreads();
+        for (int v = threadIdx.x; v < nb; v += kThreads) {
+            const float m = __ldcg(mass + v0 + v);
+            const float wv = M == -INFINITY ? 0.f : expf(m - M);
+            wts[v] = wv;
+            zloc += wv;
+        }
+        __syncthreads();
+        if (x < D) {
+            const float *col = vec + (size_t)v0 * D + x;
+            int v = 0;
+            for (; v + 8 <= nb; v += 8) {
+                float t[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) t[k] = __ldcg(col + (size_t)(v + k) * D);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) acc = fmaf(wts[v + k], t[k], acc);
+            }
+            for (; v < nb; ++v) acc = fmaf(wts[v], __ldcg(col + (size_t)v * D), acc);
+        }
+    }
+    const float Z = block_reduce(zloc, false, scratch);
+    if (x < D) out[x] = M == -INFINITY ? 0.f : acc / Z;
+    if (threadIdx.x == 0) out[D] = M == -INFINITY ? -INFINITY : M + logf(Z);
+    __syncthreads();
+}
+
 // grid (units, B*H): one unit per CTA; the last CTA of each (b, h) combines.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
@@ -225,8 +278,11 @@ __global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
         const float lse_tile = unit_compute<T, D>(s, p.rows, a.scale);
         for (int x = threadIdx.x; x < D; x += kThreads) my_vec[x] = s.red[x];
         if (threadIdx.x == 0) ws.mass[qi * a.units + u] = p.is_chunk ? p.mass : lse_tile;
-    } else if (threadIdx.x == 0) {
-        ws.mass[qi * a.units + u] = -INFINITY;
+    } else {
+        // an empty unit contributes weight 0; its vector is zeroed so that no stale value
+        // can enter the combination
+        for (int x = threadIdx.x; x < D; x += kThreads) my_vec[x] = 0.f;
+        if (threadIdx.x == 0) ws.mass[qi * a.units + u] = -INFINITY;
     }
     __threadfence();
     __syncthreads();
@@ -234,26 +290,9 @@ __global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    // combine: o = sum_u exp(m_u - M) o_u / sum_u exp(m_u - M), lse = M + log(...)
-    float M = -INFINITY;
-    for (int v = 0; v < a.units; ++v) M = fmaxf(M, __ldcg(&ws.mass[qi * a.units + v]));
-    float *o = s.red;  // reuse shared memory for the final row
-    float zsum = 0.f;
-    for (int x = threadIdx.x; x < D; x += kThreads) o[x] = 0.f;
-    if (M != -INFINITY) {
-        for (int v = 0; v < a.units; ++v) {
-            const float m = __ldcg(&ws.mass[qi * a.units + v]);
-            if (m == -INFINITY) continue;
-            const float wv = expf(m - M);
-            zsum += wv;
-            const float *vec = ws.vec + ((size_t)qi * a.units + v) * D;
-            for (int x = threadIdx.x; x < D; x += kThreads) o[x] = fmaf(wv, __ldcg(&vec[x]), o[x]);
-        }
-        const float inv = 1.f / zsum;
-        for (int x = threadIdx.x; x < D; x += kThreads) o[x] *= inv;
-    }
-    __syncthreads();
-    store_output<T, D>(a, b, h, 0, qi, o, M == -INFINITY ? -INFINITY : M + logf(zsum));
+    combine_units<D>(ws.mass + (size_t)qi * a.units, ws.vec + (size_t)qi * a.units * D, a.units, s.red,
+                     reinterpret_cast<float *>(smem) /* K tile space, no longer needed */);
+    store_output<T, D>(a, b, h, 0, qi, s.red, s.red[D]);
     if (threadIdx.x == 0) ws.counters[qi] = 0;
 }
 
@@ -300,9 +339,10 @@ hils_status launch_decode(const AttendArgs &a, cudaStream_t st) {
     using Cfg = UnitCfg<T, D>;
     const int nq = a.B * a.H;
     if (nq == 0) return HILS_OK;
-    cudaError_t e = cudaFuncSetAttribute(attend_decode_kernel<T, D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
-    if (e != cudaSuccess) return record_cuda_error(e);
+    static KernelSetup setup;
+    const hils_status stt = kernel_setup(setup, (const void *)attend_decode_kernel<T, D>, kThreads,
+                                         Cfg::kSmemBytes, nullptr);
+    if (stt != HILS_OK) return stt;
     attend_decode_kernel<T, D><<<dim3(a.units, nq), kThreads, Cfg::kSmemBytes, st>>>(a);
     return record_cuda_error(cudaGetLastError());
 }
@@ -312,9 +352,10 @@ hils_status launch_prefill_general(const AttendArgs &a, cudaStream_t st) {
     using Cfg = UnitCfg<T, D>;
     const int64_t nq = (int64_t)a.B * a.H * a.Lq;
     if (nq == 0) return HILS_OK;
-    cudaError_t e = cudaFuncSetAttribute(attend_prefill_general_kernel<T, D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
-    if (e != cudaSuccess) return record_cuda_error(e);
+    static KernelSetup setup;
+    const hils_status stt = kernel_setup(setup, (const void *)attend_prefill_general_kernel<T, D>, kThreads,
+                                         Cfg::kSmemBytes, nullptr);
+    if (stt != HILS_OK) return stt;
     attend_prefill_general_kernel<T, D><<<(unsigned)nq, kThreads, Cfg::kSmemBytes, st>>>(a);
     return record_cuda_error(cudaGetLastError());
 }

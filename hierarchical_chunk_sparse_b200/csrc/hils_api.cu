@@ -23,6 +23,31 @@ int device_sm_count() {
     return n;
 }
 
+hils_status kernel_setup(KernelSetup &cache, const void *func, int threads, int smem_bytes, int *per_sm) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (__atomic_load_n(&cache.done, __ATOMIC_ACQUIRE) & bit)) {
+        if (per_sm) *per_sm = cache.per_sm[dev];
+        return HILS_OK;
+    }
+    if (smem_bytes > 48 * 1024) {
+        e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+        if (e != cudaSuccess) return record_cuda_error(e);
+    }
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, func, threads, smem_bytes);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    if (n < 1) n = 1;
+    if (bit) {
+        cache.per_sm[dev] = n;
+        __atomic_fetch_or(&cache.done, bit, __ATOMIC_RELEASE);
+    }
+    if (per_sm) *per_sm = n;
+    return HILS_OK;
+}
+
 namespace {
 
 size_t elem_size(hils_dtype dt) { return dt == HILS_BF16 ? 2 : 4; }

@@ -81,6 +81,14 @@ void select_split_plan(int B, int H, int Lq, int C, int K, bool has_qpos, int nu
 int device_sm_count();
 hils_status record_cuda_error(cudaError_t e);
 
+// Per-kernel launch set-up done once per device: the dynamic shared memory opt-in and
+// the resident CTAs per SM. `cache` is a function-local static of the caller.
+struct KernelSetup {
+    unsigned long long done = 0;  // bit per device ordinal < 64
+    int per_sm[64] = {};
+};
+hils_status kernel_setup(KernelSetup &cache, const void *func, int threads, int smem_bytes, int *per_sm);
+
 // ------------------------------------------------------------------ device helpers
 
 template <typename T>

@@ -335,25 +335,130 @@ __global__ void __launch_bounds__(kThreads) select_warp_kernel(SelectArgs a) {
     warp_write(lists[w], a.topk, qi, a.idx, a.score, a.nsel);
 }
 
+// ---- split search (few queries, long contexts)
+//
+// A CTA screens its chunk range in passes of 1024 chunks. The screen is a coalesced
+// stream over the summary rows: kTPR threads share a row (16 B each), every thread
+// keeps its slice of q~ in registers and has kUnroll row loads in flight; the row's
+// partial dot / |dot| are combined with xor-shuffles. Screen values and radii land in
+// shared memory, and then each warp folds its 128 of them into its running exact
+// top-K list exactly as the per-query path does.
+
+template <typename T, int D>
+struct ScanCfg {
+    static constexpr int kEPV = Vec<T>::kN;       // elements per 16-byte load
+    static constexpr int kTPR = D / kEPV;         // threads per summary row: 8, 16 or 32
+    static constexpr int kRPS = kThreads / kTPR;  // rows per step
+    static constexpr int kPass = kWarps * kTile;  // 1024 chunks per pass
+    static constexpr int kSteps = kPass / kRPS;
+    static constexpr int kUnroll = 16;
+    static_assert(kSteps % kUnroll == 0, "pass size");
+};
+
+template <typename T, int D>
+__device__ void cta_screen_pass(const QueryCtx &q, const float (&qv)[Vec<T>::kN], int base, int c1,
+                                float *s_scr, float *e_scr, float *b_scr) {
+    using Cfg = ScanCfg<T, D>;
+    constexpr int kN = Vec<T>::kN;
+    const int tid = threadIdx.x, col = tid % Cfg::kTPR, r0 = tid / Cfg::kTPR;
+    for (int i = tid; i < Cfg::kPass; i += kThreads) {
+        const int c = base + i;
+        b_scr[i] = c < c1 ? q.bhead[c] : 0.f;
+    }
+    __syncthreads();
+    const T *kh = static_cast<const T *>(q.khead);
+    for (int s0 = 0; s0 < Cfg::kSteps; s0 += Cfg::kUnroll) {
+        uint4 v[Cfg::kUnroll];
+#pragma unroll
+        for (int u = 0; u < Cfg::kUnroll; ++u) {
+            const int c = base + (s0 + u) * Cfg::kRPS + r0;
+            v[u] = c < c1 ? __ldg(reinterpret_cast<const uint4 *>(kh + (int64_t)c * q.kst) + col)
+                          : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < Cfg::kUnroll; ++u) {
+            float kf[kN];
+            widen(v[u], kf, T());
+            float dot = 0.f, ad = 0.f;
+#pragma unroll
+            for (int i = 0; i < kN; ++i) {
+                dot = fmaf(qv[i], kf[i], dot);
+                ad = fmaf(fabsf(qv[i]), fabsf(kf[i]), ad);
+            }
+#pragma unroll
+            for (int o = Cfg::kTPR / 2; o > 0; o >>= 1) {
+                dot += __shfl_xor_sync(kFull, dot, o);
+                ad += __shfl_xor_sync(kFull, ad, o);
+            }
+            const int row = (s0 + u) * Cfg::kRPS + r0;
+            if (col == 0) {
+                const float sv = fmaf(dot, q.scale, b_scr[row]);
+                s_scr[row] = sv;
+                e_scr[row] = fmaf(q.scale * ad, (float)(D + 2) * 0x1p-23f, fabsf(sv) * 0x1p-22f);
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// Folds the warp's 128 screened chunks of the pass into its running list.
+template <typename T, int D>
+__device__ int warp_fold(const QueryCtx &q, const float *s_scr, const float *e_scr, int base, int c1, int K,
+                         EntryList &list, int n) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    Slots<5> p;
+    p.idx[0] = lane < n ? list.idx[lane] : -1;
+    p.s[0] = lane < n ? list.s[lane] : 0.f;
+    p.e[0] = lane < n ? list.e[lane] : 0.f;
+    p.x[0] = lane < n ? list.x[lane] : 0.0;
+#pragma unroll
+    for (int r = 1; r < 5; ++r) {
+        const int row = w * kTile + lane + 32 * (r - 1);
+        const int c = base + row;
+        const bool ok = c < c1;
+        p.idx[r] = ok ? c : -1;
+        p.s[r] = ok ? s_scr[row] : 0.f;
+        p.e[r] = ok ? e_scr[row] : 0.f;
+        p.x[r] = __longlong_as_double(0x7ff8000000000000ll);
+    }
+    const unsigned keep = warp_topk<T, D, 5>(p, K, q);
+    __syncwarp();
+    n = warp_append<5>(p, keep, list, 0);
+    __syncwarp();
+    return n;
+}
+
 // Few queries, many chunks: grid (ctas_per_query, queries).
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads) select_split_kernel(SelectArgs a) {
-    __shared__ __align__(16) float qs[D];
+__global__ void __launch_bounds__(kThreads, 2) select_split_kernel(SelectArgs a) {
+    using Cfg = ScanCfg<T, D>;
+    __shared__ float s_scr[Cfg::kPass], e_scr[Cfg::kPass], b_scr[Cfg::kPass];
     __shared__ EntryList lists[kWarps];
     __shared__ EntryList merged;
     __shared__ int is_last;
-    const int w = threadIdx.x >> 5;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t qi = blockIdx.y;
     int t;
     const QueryCtx q = make_ctx<T, D>(a, qi, t);
     const int ne = eligible(t, a.C);
-    if (w == 0) load_query_f32<T, D>(q, qs);
-    __syncthreads();
-
-    const int warp_span = a.tiles_per_warp * kTile;
-    const int c0 = (blockIdx.x * kWarps + w) * warp_span;
-    const int c1 = min(c0 + warp_span, ne);
-    warp_scan<T, D>(q, qs, c0, c1, a.topk, lists[w]);
+    float qv[Vec<T>::kN];
+    {
+        float tmp[Vec<T>::kN];
+        const int col = threadIdx.x % Cfg::kTPR;
+        widen(__ldg(reinterpret_cast<const uint4 *>(q.qrow) + col), tmp, T());
+#pragma unroll
+        for (int i = 0; i < Vec<T>::kN; ++i) qv[i] = tmp[i];
+    }
+    int n = 0;
+    for (int pass = 0; pass < a.tiles_per_warp; ++pass) {
+        const int base = (blockIdx.x * a.tiles_per_warp + pass) * Cfg::kPass;
+        if (base >= ne) break;
+        const int c1 = min(base + Cfg::kPass, ne);
+        cta_screen_pass<T, D>(q, qv, base, c1, s_scr, e_scr, b_scr);
+        n = warp_fold<T, D>(q, s_scr, e_scr, base, c1, a.topk, lists[w], n);
+        __syncthreads();
+    }
+    if (lane == 0) lists[w].n = n;
     __syncthreads();
     if (w == 0) warp_merge<T, D, 8>(q, lists, kWarps, false, a.topk, merged);
     __syncthreads();
@@ -368,7 +473,6 @@ __global__ void __launch_bounds__(kThreads) select_split_kernel(SelectArgs a) {
         static_cast<uint8_t *>(a.ws) + (((size_t)gridDim.y * sizeof(int) + 255) & ~(size_t)255));
     EntryList &mine = ws_lists[qi * gridDim.x + blockIdx.x];
     if (w == 0) {
-        const int lane = threadIdx.x;
         if (lane < merged.n) {
             mine.idx[lane] = merged.idx[lane];
             mine.s[lane] = merged.s[lane];
@@ -416,7 +520,7 @@ void select_split_plan(int B, int H, int Lq, int C, int K, bool has_qpos, int nu
         return;
     }
     const int k = K > 0 ? K : 1;
-    int tpw = 1;
+    int tpw = 1;  // 1024-chunk passes per CTA
     for (;;) {
         const int span = kWarps * kTile * tpw;
         const int ctas = (C + span - 1) / span;

@@ -147,14 +147,11 @@ hils_status launch(const SummarizeArgs &a, cudaStream_t s) {
     using Cfg = SumCfg<T, D>;
     const int64_t total = (int64_t)a.B * a.H * a.C;
     if (total == 0) return HILS_OK;
-    cudaError_t e = cudaFuncSetAttribute(summarize_kernel<T, D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
-    if (e != cudaSuccess) return record_cuda_error(e);
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, summarize_kernel<T, D>, Cfg::kThreads,
-                                                      Cfg::kSmemBytes);
-    if (e != cudaSuccess) return record_cuda_error(e);
-    if (per_sm < 1) per_sm = 1;
+    static KernelSetup setup;
+    int per_sm = 1;
+    const hils_status st = kernel_setup(setup, (const void *)summarize_kernel<T, D>, Cfg::kThreads,
+                                        Cfg::kSmemBytes, &per_sm);
+    if (st != HILS_OK) return st;
     const int64_t grid = total < (int64_t)per_sm * device_sm_count() ? total
                                                                       : (int64_t)per_sm * device_sm_count();
     summarize_kernel<T, D><<<(unsigned)grid, Cfg::kThreads, Cfg::kSmemBytes, s>>>(a);

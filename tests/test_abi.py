@@ -138,3 +138,22 @@ def test_binding_refuses_a_missing_library(tmp_path):
             hils.load_library(str(tmp_path / "missing.so"))
         finally:
             hils._lib = hils._lib_saved
+
+
+def test_binding_rejects_mismatched_shapes():
+    """The binding checks every tensor against the parameters before the C call, so a
+    mismatched buffer can never be read or written out of bounds."""
+    import torch
+
+    p = hils.Params(B=1, H=32, d=128, K=16, W=512, dtype=torch.bfloat16)
+    Q = torch.zeros(2, 3, 1, 128, dtype=torch.bfloat16)
+    Ksum = torch.zeros(2, 3, 10, 128, dtype=torch.bfloat16)
+    Bsum = torch.zeros(2, 3, 10)
+    idx = torch.zeros(2, 3, 1, 16, dtype=torch.int32)
+    with pytest.raises(ValueError, match="shape"):
+        hils.hils_select(p, Q, Ksum, Bsum, idx, idx.float(), idx[..., 0])
+    p2 = hils.Params(B=2, H=3, d=128, K=16, W=512, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="dtype"):
+        hils.hils_select(p2, Q.float(), Ksum, Bsum, idx, idx.float(), idx[..., 0])
+    with pytest.raises(ValueError, match="CUDA"):
+        hils.hils_select(p2, Q, Ksum, Bsum, idx, idx.float(), idx[..., 0])

@@ -132,7 +132,8 @@ def test_select_prefill_bit_exact(oracle, cuda_device, case):
     scores_close(score, s_ref, n_ref, case)
 
 
-def _decode_like(w, C, B=2, H=3, seed=3):
+def _decode_like(w, C, seed=3):
+    B, H = w.B, w.H
     g = torch.Generator().manual_seed(seed)
     Q = torch.randn(B, H, 1, w.d, generator=g).to(w.dtype)
     Ksum = (torch.randn(B, H, C, w.d, generator=g) * 0.3).to(w.dtype)
@@ -144,7 +145,7 @@ def _decode_like(w, C, B=2, H=3, seed=3):
                                       (3000, 16, [1000, 64 * 3000 + 5])])
 def test_select_split_paths_bit_exact(oracle, cuda_device, C, K, tpos):
     """Few queries, long contexts: the multi-CTA split search and its final merge."""
-    w = WORKLOADS[4].replace(K=K)
+    w = WORKLOADS[4].replace(B=2, H=3, K=K)
     Q, Ksum, Bsum = _decode_like(w, C)
     B = Q.shape[0]
     qpos = torch.tensor([[64 * C + 3]] * B if tpos is None else [[t] for t in tpos], dtype=torch.int32)
@@ -158,14 +159,15 @@ def test_select_split_paths_bit_exact(oracle, cuda_device, C, K, tpos):
 def test_select_planted_exact_ties(oracle, cuda_device):
     """Twenty duplicated summaries give bit-identical scores above all others; only 16
     fit, and the lower chunk indices win. A second planted group ties lower down."""
-    w = WORKLOADS[4].replace(K=16)
+    w = WORKLOADS[4].replace(B=2, H=3, K=16)
     C = 2500
     Q, Ksum, Bsum = _decode_like(w, C, seed=11)
     g = torch.Generator().manual_seed(12)
     dups = sorted(torch.randperm(C, generator=g)[:20].tolist())
+    k0, b0 = Ksum[:, :, dups[0]].clone(), Bsum[:, :, dups[0]].clone() + 50.0
     for c in dups:
-        Ksum[:, :, c] = Ksum[:, :, dups[0]]
-        Bsum[:, :, c] = Bsum[:, :, dups[0]] + 50.0
+        Ksum[:, :, c] = k0
+        Bsum[:, :, c] = b0
     qpos = torch.full((Q.shape[0], 1), 64 * C, dtype=torch.int32)
     idx, score, nsel = gpu_select(w, Q.to(cuda_device), Ksum.to(cuda_device), Bsum.to(cuda_device),
                                   qpos=qpos.to(cuda_device))
@@ -177,9 +179,10 @@ def test_select_planted_exact_ties(oracle, cuda_device):
     rows = sorted(torch.randperm(C, generator=g)[:22].tolist())
     for c in rows[:10]:
         Bsum[:, :, c] += 80.0
+    k0, b0 = Ksum[:, :, rows[10]].clone(), Bsum[:, :, rows[10]].clone() + 40.0
     for c in rows[10:]:
-        Ksum[:, :, c] = Ksum[:, :, rows[10]]
-        Bsum[:, :, c] = Bsum[:, :, rows[10]] + 40.0
+        Ksum[:, :, c] = k0
+        Bsum[:, :, c] = b0
     idx, score, nsel = gpu_select(w, Q.to(cuda_device), Ksum.to(cuda_device), Bsum.to(cuda_device),
                                   qpos=qpos.to(cuda_device))
     want = torch.tensor(sorted(rows[:10] + rows[10:16]), dtype=torch.int32)
@@ -191,7 +194,7 @@ def test_select_planted_exact_ties(oracle, cuda_device):
 @pytest.mark.parametrize("C", [100, 5000])
 def test_select_all_scores_equal(oracle, cuda_device, C):
     """Degenerate ranking (every chunk ties): the K lowest indices are kept."""
-    w = WORKLOADS[4].replace(K=16)
+    w = WORKLOADS[4].replace(B=2, H=2, K=16)
     Q = torch.ones(2, 2, 1, w.d).to(w.dtype)
     Ksum = torch.ones(2, 2, C, w.d).to(w.dtype)
     Bsum = torch.full((2, 2, C), 0.5)
