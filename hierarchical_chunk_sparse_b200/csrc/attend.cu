@@ -261,6 +261,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int is_last;
+    pdl_wait();  // launched as a dependent of the select kernels: their outputs are complete
     const UnitSmem s = unit_smem<T, D>(smem);
     const int u = blockIdx.x;
     const int64_t qi = blockIdx.y;  // (b, h), one query each
@@ -343,8 +344,8 @@ hils_status launch_decode(const AttendArgs &a, cudaStream_t st) {
     const hils_status stt = kernel_setup(setup, (const void *)attend_decode_kernel<T, D>, kThreads,
                                          Cfg::kSmemBytes, nullptr);
     if (stt != HILS_OK) return stt;
-    attend_decode_kernel<T, D><<<dim3(a.units, nq), kThreads, Cfg::kSmemBytes, st>>>(a);
-    return record_cuda_error(cudaGetLastError());
+    return launch_dependent((const void *)attend_decode_kernel<T, D>, dim3(a.units, nq), dim3(kThreads),
+                            Cfg::kSmemBytes, st, a);
 }
 
 template <typename T, int D>

@@ -102,7 +102,7 @@ int decode_units(const hils_params *p) {
 size_t select_ws_for(const hils_params *p, int Lq, int C) {
     int ctas = 0, tiles = 0;
     select_split_plan(p->B, p->H, Lq, C, p->K, true, device_sm_count(), &ctas, &tiles);
-    return select_ws_bytes(p->B * p->H * Lq, ctas, p->K);
+    return select_ws_bytes(p->B * p->H * Lq, C, ctas);
 }
 
 #define HILS_TRY(expr)                 \
@@ -202,7 +202,7 @@ int hils_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *
     a.scale = scale;
     select_split_plan(p->B, p->H, Lq, C, p->K, qpos != nullptr, device_sm_count(), &a.ctas_per_query,
                       &a.tiles_per_warp);
-    HILS_TRY(check_workspace(workspace, ws_bytes, select_ws_bytes((int)nq, a.ctas_per_query, p->K)));
+    HILS_TRY(check_workspace(workspace, ws_bytes, select_ws_bytes((int)nq, C, a.ctas_per_query)));
     a.ws = workspace;
     return launch_select(p->dtype, p->d, a, stream);
 }

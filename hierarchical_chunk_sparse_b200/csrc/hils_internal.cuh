@@ -71,7 +71,7 @@ hils_status launch_attend_decode(hils_dtype dt, int d, const AttendArgs &a, cuda
 hils_status launch_attend_prefill_general(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s);
 
 // Workspace layouts (bytes); shared by the host size query and the kernels.
-size_t select_ws_bytes(int queries, int ctas_per_query, int K);
+size_t select_ws_bytes(int queries, int C, int ctas_per_query);
 size_t attend_decode_ws_bytes(int queries, int units, int d);
 
 // Choice of the split search for hils_select; identical on the size query and the call.
@@ -89,7 +89,32 @@ struct KernelSetup {
 };
 hils_status kernel_setup(KernelSetup &cache, const void *func, int threads, int smem_bytes, int *per_sm);
 
+// Launches `func(args)` with programmatic stream serialization: the kernel may be
+// scheduled while the previous kernel on the stream drains, and must call pdl_wait()
+// before touching anything that kernel (or earlier work) writes.
+template <typename Args>
+hils_status launch_dependent(const void *func, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             const Args &args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void *argv[] = {const_cast<Args *>(&args)};
+    return record_cuda_error(cudaLaunchKernelExC(&cfg, func, argv));
+}
+
 // ------------------------------------------------------------------ device helpers
+
+// Programmatic dependent launch: wait for the preceding grid's completion (and its
+// memory), and allow the next dependent-launched grid to be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
 template <typename T>
 struct Vec;  // one 16-byte vector of T

@@ -47,6 +47,7 @@ struct EntryList {
     float s[kMaxK];
     float e[kMaxK];
     int n;
+    float bound;       // lower bound on the K-th largest lo of the range the list covers
 };
 static_assert(sizeof(EntryList) <= kListBytes, "list size");
 
@@ -99,14 +100,18 @@ __device__ __forceinline__ void screen(const QueryCtx &q, const float *qs, int c
 
 // Exact top-K of the warp's pool (R slots per lane, idx < 0 = empty). Returns the
 // lane's mask of kept slots. Uniform control flow across the warp.
+// `bound` receives a lower bound on the pool's K-th largest lo (s_K - e_max, rounded
+// down), or -inf when the pool holds at most K entries. Any chunk whose hi lies below
+// the bound of some subset of its competitors is certainly out.
 template <typename T, int D, int R>
-__device__ unsigned warp_topk(Slots<R> &p, int K, const QueryCtx &q) {
+__device__ unsigned warp_topk(Slots<R> &p, int K, const QueryCtx &q, float &bound) {
     const int lane = threadIdx.x & 31;
     unsigned valid = 0;
 #pragma unroll
     for (int r = 0; r < R; ++r)
         if (p.idx[r] >= 0) valid |= 1u << r;
     const int n = __reduce_add_sync(kFull, __popc(valid));
+    bound = -INFINITY;
     if (n <= K) return valid;
 
     float em = 0.f;
@@ -140,6 +145,7 @@ __device__ unsigned warp_topk(Slots<R> &p, int K, const QueryCtx &q) {
     }
     const float lo_cut = __fsub_rd(sK, em);
     const float hi_cut = __fadd_ru(sK1, em);
+    bound = lo_cut;
 
     unsigned in = 0, band = 0;
 #pragma unroll
@@ -234,7 +240,8 @@ __device__ void warp_scan(const QueryCtx &q, const float *qs, int c0, int c1, in
             p.x[r] = __longlong_as_double(0x7ff8000000000000ll);  // NaN: not computed
             if (c < c1) screen<T, D>(q, qs, c, p.s[r], p.e[r]);
         }
-        const unsigned keep = warp_topk<T, D, 5>(p, K, q);
+        float bnd;
+        const unsigned keep = warp_topk<T, D, 5>(p, K, q, bnd);
         __syncwarp();
         n = warp_append<5>(p, keep, list, 0);
         __syncwarp();
@@ -267,7 +274,8 @@ __device__ void warp_merge(const QueryCtx &q, const EntryList *lists, int nlists
             }
         }
     }
-    const unsigned keep = warp_topk<T, D, R>(p, K, q);
+    float bnd;
+    const unsigned keep = warp_topk<T, D, R>(p, K, q, bnd);
     __syncwarp();
     const int n = warp_append<R>(p, keep, out, 0);
     if (lane == 0) out.n = n;
@@ -335,38 +343,73 @@ __global__ void __launch_bounds__(kThreads) select_warp_kernel(SelectArgs a) {
     warp_write(lists[w], a.topk, qi, a.idx, a.score, a.nsel);
 }
 
-// ---- split search (few queries, long contexts)
+// ---- decode-shaped search (few queries, long contexts): screen, then pick
 //
-// A CTA screens its chunk range in passes of 1024 chunks. The screen is a coalesced
-// stream over the summary rows: kTPR threads share a row (16 B each), every thread
-// keeps its slice of q~ in registers and has kUnroll row loads in flight; the row's
-// partial dot / |dot| are combined with xor-shuffles. Screen values and radii land in
-// shared memory, and then each warp folds its 128 of them into its running exact
-// top-K list exactly as the per-query path does.
+// S1 select_screen_kernel: grid (chunk blocks of 256, queries), 128 threads. A
+// coalesced stream over the summary rows: kTPR threads share a row (16 bytes each),
+// every thread keeps its slice of q~ in registers, 8 row loads in flight per thread,
+// partial dot and |k|^2 combined with xor-shuffles. It writes the screen value s_c
+// and its radius e_c of every eligible chunk to the workspace. The radius uses the
+// Cauchy-Schwarz form of the fused-multiply-add bound, doubled:
+//   e_c = scale |q~| |k'_c| (d+2) 2^-23 + |s_c| 2^-22.
+// S2 select_pick_kernel: one 1024-thread CTA per query holds the query's screen
+// values in registers (16 per thread), finds a threshold T with K+1 <= #{s >= T} <= 64
+// (a normal-quantile guess, then bisection over the ordered float keys: at most 32
+// rounds, usually none), keeps the chunks with hi >= T - e_max (every chunk that can
+// still be among the top K: the K-th largest lo is at least T - e_max), and one warp
+// runs the exact interval top-K on those. Heavy ties (more than 64 candidates) fall
+// back to folding the candidates in batches of 32, which is always exact.
+// S2 is launched with programmatic dependent launch, so its launch overlaps S1's tail.
+
+constexpr int kSplitThreads = 128;
+constexpr int kSpan = 256;         // chunks per screen CTA
+constexpr int kPickThreads = 1024;
+constexpr int kPickItems = 16;     // screen values per pick thread: C <= 16384
+constexpr int kPoolCap = 64;
 
 template <typename T, int D>
 struct ScanCfg {
-    static constexpr int kEPV = Vec<T>::kN;       // elements per 16-byte load
-    static constexpr int kTPR = D / kEPV;         // threads per summary row: 8, 16 or 32
-    static constexpr int kRPS = kThreads / kTPR;  // rows per step
-    static constexpr int kPass = kWarps * kTile;  // 1024 chunks per pass
-    static constexpr int kSteps = kPass / kRPS;
-    static constexpr int kUnroll = 16;
-    static_assert(kSteps % kUnroll == 0, "pass size");
+    static constexpr int kEPV = Vec<T>::kN;             // elements per 16-byte load
+    static constexpr int kTPR = D / kEPV;               // threads per summary row: 8, 16 or 32
+    static constexpr int kRPS = kSplitThreads / kTPR;   // rows per step
+    static constexpr int kSteps = kSpan / kRPS;
+    static constexpr int kUnroll = kSteps < 8 ? kSteps : 8;
+    static_assert(kSteps % kUnroll == 0, "span");
 };
 
+__device__ __forceinline__ float2 *screen_buffer(const SelectArgs &a, int64_t qi) {
+    return static_cast<float2 *>(a.ws) + qi * a.C;
+}
+
 template <typename T, int D>
-__device__ void cta_screen_pass(const QueryCtx &q, const float (&qv)[Vec<T>::kN], int base, int c1,
-                                float *s_scr, float *e_scr, float *b_scr) {
+__global__ void __launch_bounds__(kSplitThreads) select_screen_kernel(SelectArgs a) {
     using Cfg = ScanCfg<T, D>;
     constexpr int kN = Vec<T>::kN;
+    pdl_trigger();
+    __shared__ float b_scr[kSpan];
+    const int64_t qi = blockIdx.y;
+    int t;
+    const QueryCtx q = make_ctx<T, D>(a, qi, t);
+    const int ne = eligible(t, a.C);
+    const int base = blockIdx.x * kSpan;
+    if (base >= ne) return;
+    const int c1 = min(base + kSpan, ne);
     const int tid = threadIdx.x, col = tid % Cfg::kTPR, r0 = tid / Cfg::kTPR;
-    for (int i = tid; i < Cfg::kPass; i += kThreads) {
+    float qv[kN];
+    widen(__ldg(reinterpret_cast<const uint4 *>(q.qrow) + col), qv, T());
+    float qn2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < kN; ++i) qn2 = fmaf(qv[i], qv[i], qn2);
+#pragma unroll
+    for (int o = Cfg::kTPR / 2; o > 0; o >>= 1) qn2 += __shfl_xor_sync(kFull, qn2, o);
+    for (int i = tid; i < kSpan; i += kSplitThreads) {
         const int c = base + i;
         b_scr[i] = c < c1 ? q.bhead[c] : 0.f;
     }
     __syncthreads();
+    float2 *out = screen_buffer(a, qi);
     const T *kh = static_cast<const T *>(q.khead);
+    const float ecoef = q.scale * sqrtf(qn2) * ((float)(D + 2) * 0x1p-23f);
     for (int s0 = 0; s0 < Cfg::kSteps; s0 += Cfg::kUnroll) {
         uint4 v[Cfg::kUnroll];
 #pragma unroll
@@ -379,118 +422,220 @@ __device__ void cta_screen_pass(const QueryCtx &q, const float (&qv)[Vec<T>::kN]
         for (int u = 0; u < Cfg::kUnroll; ++u) {
             float kf[kN];
             widen(v[u], kf, T());
-            float dot = 0.f, ad = 0.f;
+            float dot = 0.f, ksq = 0.f;
 #pragma unroll
             for (int i = 0; i < kN; ++i) {
                 dot = fmaf(qv[i], kf[i], dot);
-                ad = fmaf(fabsf(qv[i]), fabsf(kf[i]), ad);
+                ksq = fmaf(kf[i], kf[i], ksq);
             }
 #pragma unroll
             for (int o = Cfg::kTPR / 2; o > 0; o >>= 1) {
                 dot += __shfl_xor_sync(kFull, dot, o);
-                ad += __shfl_xor_sync(kFull, ad, o);
+                ksq += __shfl_xor_sync(kFull, ksq, o);
             }
             const int row = (s0 + u) * Cfg::kRPS + r0;
-            if (col == 0) {
+            const int c = base + row;
+            if (col == 0 && c < c1) {
                 const float sv = fmaf(dot, q.scale, b_scr[row]);
-                s_scr[row] = sv;
-                e_scr[row] = fmaf(q.scale * ad, (float)(D + 2) * 0x1p-23f, fabsf(sv) * 0x1p-22f);
+                out[c] = make_float2(sv, fmaf(ecoef, sqrtf(ksq), fabsf(sv) * 0x1p-22f));
             }
         }
     }
-    __syncthreads();
 }
 
-// Folds the warp's 128 screened chunks of the pass into its running list.
-template <typename T, int D>
-__device__ int warp_fold(const QueryCtx &q, const float *s_scr, const float *e_scr, int base, int c1, int K,
-                         EntryList &list, int n) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    Slots<5> p;
-    p.idx[0] = lane < n ? list.idx[lane] : -1;
-    p.s[0] = lane < n ? list.s[lane] : 0.f;
-    p.e[0] = lane < n ? list.e[lane] : 0.f;
-    p.x[0] = lane < n ? list.x[lane] : 0.0;
+// Staging area for the candidate pool.
+struct Pool64 {
+    double x[kPoolCap];
+    int idx[kPoolCap];
+    float s[kPoolCap];
+    float e[kPoolCap];
+};
+
+// Block-wide sum / max / min over the pick CTA (all threads call; result everywhere).
+template <int kOp>  // 0 sum, 1 max, 2 min
+__device__ __forceinline__ float block_reduce_f(float v, float *scratch) {
 #pragma unroll
-    for (int r = 1; r < 5; ++r) {
-        const int row = w * kTile + lane + 32 * (r - 1);
-        const int c = base + row;
-        const bool ok = c < c1;
-        p.idx[r] = ok ? c : -1;
-        p.s[r] = ok ? s_scr[row] : 0.f;
-        p.e[r] = ok ? e_scr[row] : 0.f;
-        p.x[r] = __longlong_as_double(0x7ff8000000000000ll);
+    for (int o = 16; o > 0; o >>= 1) {
+        const float x = __shfl_xor_sync(kFull, v, o);
+        v = kOp == 0 ? v + x : (kOp == 1 ? fmaxf(v, x) : fminf(v, x));
     }
-    const unsigned keep = warp_topk<T, D, 5>(p, K, q);
-    __syncwarp();
-    n = warp_append<5>(p, keep, list, 0);
-    __syncwarp();
-    return n;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (lane == 0) scratch[w] = v;
+    __syncthreads();
+    v = scratch[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float x = __shfl_xor_sync(kFull, v, o);
+        v = kOp == 0 ? v + x : (kOp == 1 ? fmaxf(v, x) : fminf(v, x));
+    }
+    return v;
 }
 
-// Few queries, many chunks: grid (ctas_per_query, queries).
-template <typename T, int D>
-__global__ void __launch_bounds__(kThreads, 2) select_split_kernel(SelectArgs a) {
-    using Cfg = ScanCfg<T, D>;
-    __shared__ float s_scr[Cfg::kPass], e_scr[Cfg::kPass], b_scr[Cfg::kPass];
-    __shared__ EntryList lists[kWarps];
-    __shared__ EntryList merged;
-    __shared__ int is_last;
+__device__ __forceinline__ int block_sum_i(int v, int *scratch) {
+    v = __reduce_add_sync(kFull, v);
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t qi = blockIdx.y;
+    __syncthreads();
+    if (lane == 0) scratch[w] = v;
+    __syncthreads();
+    return __reduce_add_sync(kFull, scratch[lane]);
+}
+
+// Upper normal quantile z with P(Z > z) = p (0 < p < 0.5): the rational approximation
+// of Abramowitz & Stegun 26.2.23 (|error| < 4.5e-4). Only a starting guess here.
+__device__ __forceinline__ float normal_upper_quantile(float p) {
+    const float t = sqrtf(-2.f * logf(p));
+    return t - (2.515517f + t * (0.802853f + t * 0.010328f)) /
+                   (1.f + t * (1.432788f + t * (0.189269f + t * 0.001308f)));
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kPickThreads) select_pick_kernel(SelectArgs a) {
+    __shared__ float fscr[32];
+    __shared__ int iscr[32];
+    __shared__ Pool64 pool;
+    __shared__ EntryList out;
+    pdl_wait();     // the screen grid has completed and its writes are visible
+    pdl_trigger();  // let the next dependent-launched kernel be scheduled
+    const int64_t qi = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     int t;
     const QueryCtx q = make_ctx<T, D>(a, qi, t);
     const int ne = eligible(t, a.C);
-    float qv[Vec<T>::kN];
-    {
-        float tmp[Vec<T>::kN];
-        const int col = threadIdx.x % Cfg::kTPR;
-        widen(__ldg(reinterpret_cast<const uint4 *>(q.qrow) + col), tmp, T());
-#pragma unroll
-        for (int i = 0; i < Vec<T>::kN; ++i) qv[i] = tmp[i];
-    }
-    int n = 0;
-    for (int pass = 0; pass < a.tiles_per_warp; ++pass) {
-        const int base = (blockIdx.x * a.tiles_per_warp + pass) * Cfg::kPass;
-        if (base >= ne) break;
-        const int c1 = min(base + Cfg::kPass, ne);
-        cta_screen_pass<T, D>(q, qv, base, c1, s_scr, e_scr, b_scr);
-        n = warp_fold<T, D>(q, s_scr, e_scr, base, c1, a.topk, lists[w], n);
-        __syncthreads();
-    }
-    if (lane == 0) lists[w].n = n;
-    __syncthreads();
-    if (w == 0) warp_merge<T, D, 8>(q, lists, kWarps, false, a.topk, merged);
-    __syncthreads();
-
-    if (gridDim.x == 1) {
-        if (w == 0) warp_write(merged, a.topk, qi, a.idx, a.score, a.nsel);
+    const int K = a.topk;
+    const float2 *scr = screen_buffer(a, qi);
+    if (ne <= K) {  // every eligible chunk is kept, in index order
+        for (int r = tid; r < K; r += kPickThreads) {
+            a.idx[qi * K + r] = r < ne ? r : -1;
+            a.score[qi * K + r] = r < ne ? __ldcg(&scr[r]).x : -INFINITY;
+        }
+        if (tid == 0) a.nsel[qi] = ne;
         return;
     }
-    // publish this CTA's list; the last CTA of the query merges all of them
-    int *counters = static_cast<int *>(a.ws);
-    EntryList *ws_lists = reinterpret_cast<EntryList *>(
-        static_cast<uint8_t *>(a.ws) + (((size_t)gridDim.y * sizeof(int) + 255) & ~(size_t)255));
-    EntryList &mine = ws_lists[qi * gridDim.x + blockIdx.x];
-    if (w == 0) {
-        if (lane < merged.n) {
-            mine.idx[lane] = merged.idx[lane];
-            mine.s[lane] = merged.s[lane];
-            mine.e[lane] = merged.e[lane];
-            mine.x[lane] = merged.x[lane];
+    float sv[kPickItems], ev[kPickItems];
+    float emax = 0.f, smax = -INFINITY, smin = INFINITY, sum = 0.f, sum2 = 0.f;
+#pragma unroll
+    for (int j = 0; j < kPickItems; ++j) {
+        const int c = tid + j * kPickThreads;
+        const float2 v = c < ne ? __ldcg(&scr[c]) : make_float2(-INFINITY, 0.f);
+        sv[j] = v.x;
+        ev[j] = v.y;
+        if (c < ne) {
+            emax = fmaxf(emax, v.y);
+            smax = fmaxf(smax, v.x);
+            smin = fminf(smin, v.x);
+            sum += v.x;
+            sum2 = fmaf(v.x, v.x, sum2);
         }
-        if (lane == 0) mine.n = merged.n;
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) is_last = atomicAdd(&counters[qi], 1) == (int)gridDim.x - 1;
+    }
+    emax = block_reduce_f<1>(emax, fscr);
+    smax = block_reduce_f<1>(smax, fscr);
+    smin = block_reduce_f<2>(smin, fscr);
+    sum = block_reduce_f<0>(sum, fscr);
+    sum2 = block_reduce_f<0>(sum2, fscr);
+
+    // threshold over ordered keys: invariant count(>= lo_key) >= K+1, count(>= hi_key) <= K
+    unsigned lo_key = ordered_key(smin), hi_key = ordered_key(smax) + 1u;
+    unsigned tk;
+    {
+        const float mu = sum / ne;
+        const float sd = sqrtf(fmaxf(sum2 / ne - mu * mu, 0.f));
+        const float p = fminf((float)(K + 8) / (float)ne, 0.49f);
+        const float guess = mu + normal_upper_quantile(p) * sd;
+        tk = min(max(ordered_key(guess), lo_key), hi_key - 1u);
+    }
+    for (int it = 0; it < 40; ++it) {
+        int cnt = 0;
+#pragma unroll
+        for (int j = 0; j < kPickItems; ++j) cnt += ordered_key(sv[j]) >= tk && sv[j] != -INFINITY;
+        cnt = block_sum_i(cnt, iscr);
+        if (cnt > kPoolCap) lo_key = tk;
+        else if (cnt < K + 1) hi_key = tk;
+        else break;
+        if (hi_key - lo_key <= 1u) {
+            tk = lo_key;
+            break;
+        }
+        tk = lo_key + (hi_key - lo_key) / 2u;
+    }
+    // candidates: hi >= T - e_max
+    const float cut = __fsub_rd(key_to_float(tk), emax);
+    int mine = 0;
+#pragma unroll
+    for (int j = 0; j < kPickItems; ++j) mine += sv[j] != -INFINITY && __fadd_ru(sv[j], ev[j]) >= cut;
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
     }
     __syncthreads();
-    if (!is_last) return;
-    __threadfence();
+    if (lane == 31) iscr[w] = incl;
+    __syncthreads();
+    int wbase = 0;
+    for (int k = 0; k < w; ++k) wbase += iscr[k];
+    int total = 0;
+    for (int k = 0; k < kPickThreads / 32; ++k) total += iscr[k];
+    if (total <= kPoolCap) {
+        int pos = wbase + incl - mine;
+#pragma unroll
+        for (int j = 0; j < kPickItems; ++j) {
+            if (sv[j] != -INFINITY && __fadd_ru(sv[j], ev[j]) >= cut) {
+                pool.idx[pos] = tid + j * kPickThreads;
+                pool.s[pos] = sv[j];
+                pool.e[pos] = ev[j];
+                pool.x[pos] = __longlong_as_double(0x7ff8000000000000ll);
+                ++pos;
+            }
+        }
+        __syncthreads();
+        if (w == 0) {
+            Slots<2> p;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int j = lane + 32 * r;
+                const bool ok = j < total;
+                p.idx[r] = ok ? pool.idx[j] : -1;
+                p.s[r] = ok ? pool.s[j] : 0.f;
+                p.e[r] = ok ? pool.e[j] : 0.f;
+                p.x[r] = ok ? pool.x[j] : 0.0;
+            }
+            float bnd;
+            const unsigned keep = warp_topk<T, D, 2>(p, K, q, bnd);
+            __syncwarp();
+            const int n = warp_append<2>(p, keep, out, 0);
+            if (lane == 0) out.n = n;
+            __syncwarp();
+            warp_write(out, K, qi, a.idx, a.score, a.nsel);
+        }
+        return;
+    }
+    // heavy ties: fold the candidates in index order, 32 at a time (slot 0 = running list)
     if (w == 0) {
-        warp_merge<T, D, 16>(q, &ws_lists[qi * gridDim.x], gridDim.x, true, a.topk, merged);
-        warp_write(merged, a.topk, qi, a.idx, a.score, a.nsel);
-        if (threadIdx.x == 0) counters[qi] = 0;
+        int n = 0;
+        for (int c0 = 0; c0 < ne; c0 += 32) {
+            const int c = c0 + lane;
+            const float2 v = c < ne ? __ldcg(&scr[c]) : make_float2(-INFINITY, 0.f);
+            const bool cand = c < ne && __fadd_ru(v.x, v.y) >= cut;
+            if (!__any_sync(kFull, cand)) continue;
+            Slots<2> p;
+            p.idx[0] = lane < n ? out.idx[lane] : -1;
+            p.s[0] = lane < n ? out.s[lane] : 0.f;
+            p.e[0] = lane < n ? out.e[lane] : 0.f;
+            p.x[0] = lane < n ? out.x[lane] : 0.0;
+            p.idx[1] = cand ? c : -1;
+            p.s[1] = v.x;
+            p.e[1] = v.y;
+            p.x[1] = __longlong_as_double(0x7ff8000000000000ll);
+            float bnd;
+            const unsigned keep = warp_topk<T, D, 2>(p, K, q, bnd);
+            __syncwarp();
+            n = warp_append<2>(p, keep, out, 0);
+            __syncwarp();
+        }
+        if (lane == 0) out.n = n;
+        __syncwarp();
+        warp_write(out, K, qi, a.idx, a.score, a.nsel);
     }
 }
 
@@ -502,7 +647,11 @@ hils_status launch(const SelectArgs &a, cudaStream_t s) {
         const int64_t grid = (nq + kWarps - 1) / kWarps;
         select_warp_kernel<T, D><<<(unsigned)grid, kThreads, 0, s>>>(a);
     } else {
-        select_split_kernel<T, D><<<dim3(a.ctas_per_query, (unsigned)nq), kThreads, 0, s>>>(a);
+        select_screen_kernel<T, D><<<dim3(a.ctas_per_query, (unsigned)nq), kSplitThreads, 0, s>>>(a);
+        const hils_status st = record_cuda_error(cudaGetLastError());
+        if (st != HILS_OK) return st;
+        return launch_dependent((const void *)select_pick_kernel<T, D>, dim3((unsigned)nq), dim3(kPickThreads),
+                                0, s, a);
     }
     return record_cuda_error(cudaGetLastError());
 }
@@ -512,32 +661,21 @@ hils_status launch(const SelectArgs &a, cudaStream_t s) {
 void select_split_plan(int B, int H, int Lq, int C, int K, bool has_qpos, int num_sms,
                        int *ctas_per_query, int *tiles_per_warp) {
     (void)has_qpos;
+    (void)K;
     const int64_t nq = (int64_t)B * H * Lq;
-    *tiles_per_warp = 1;
-    if (nq >= (int64_t)kWarps * num_sms || C <= kTile) {
-        *ctas_per_query = 0;  // one warp per query
-        *tiles_per_warp = (C + kTile - 1) / kTile;
+    *tiles_per_warp = (C + kTile - 1) / kTile;
+    // many queries, short tables, or tables beyond the pick kernel's register capacity:
+    // one warp per query; otherwise screen + pick
+    if (nq >= (int64_t)kWarps * num_sms || C <= kTile || C > kPickThreads * kPickItems || nq > 65535) {
+        *ctas_per_query = 0;
         return;
     }
-    const int k = K > 0 ? K : 1;
-    int tpw = 1;  // 1024-chunk passes per CTA
-    for (;;) {
-        const int span = kWarps * kTile * tpw;
-        const int ctas = (C + span - 1) / span;
-        if (ctas * k <= 16 * 32) {
-            *ctas_per_query = ctas;
-            *tiles_per_warp = tpw;
-            return;
-        }
-        ++tpw;
-    }
+    *ctas_per_query = (C + kSpan - 1) / kSpan;
 }
 
-size_t select_ws_bytes(int queries, int ctas_per_query, int K) {
-    (void)K;
-    if (ctas_per_query <= 1) return 0;
-    const size_t counters = ((size_t)queries * sizeof(int) + 255) & ~(size_t)255;
-    return counters + (size_t)queries * ctas_per_query * sizeof(EntryList);
+size_t select_ws_bytes(int queries, int C, int ctas_per_query) {
+    if (ctas_per_query <= 0) return 0;
+    return (size_t)queries * C * sizeof(float2);  // screen values and radii
 }
 
 hils_status launch_select(hils_dtype dt, int d, const SelectArgs &a, cudaStream_t s) {

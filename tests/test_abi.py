@@ -95,13 +95,13 @@ def test_misalignment_rejected(lib, view):
 def test_select_workspace_too_small(lib):
     p = _p(B=1, H=2)
     c = p.c()
-    need = lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_SELECT, 1, 20000)
-    assert need > 0
+    need = lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_SELECT, 1, 8000)
+    assert need == 2 * 8000 * 8  # a screen value and radius per (query, chunk)
     rc = lib.hils_select(ctypes.byref(c), T(ALIGNED, 256, 128, 128), 1, ALIGNED, T(ALIGNED, 0, 0, 128),
-                         ALIGNED, 20000, ALIGNED, ALIGNED, ALIGNED, ALIGNED, need - 16, None)
+                         ALIGNED, 8000, ALIGNED, ALIGNED, ALIGNED, ALIGNED, need - 16, None)
     assert rc == 4
     rc = lib.hils_select(ctypes.byref(c), T(ALIGNED, 256, 128, 128), 1, ALIGNED, T(ALIGNED, 0, 0, 128),
-                         ALIGNED, 20000, ALIGNED, ALIGNED, ALIGNED, None, need, None)
+                         ALIGNED, 8000, ALIGNED, ALIGNED, ALIGNED, None, need, None)
     assert rc == 4
 
 
