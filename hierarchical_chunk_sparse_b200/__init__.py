@@ -29,8 +29,8 @@ _DTYPES = {torch.float32: HILS_F32, torch.bfloat16: HILS_BF16}
 
 # Every function the C header declares (checked by the tests against the header).
 EXPORTS = ("hils_summarize", "hils_select", "hils_attend_prefill", "hils_attend_decode",
-           "hils_workspace_bytes", "hils_workspace_init", "hils_status_string",
-           "hils_last_cuda_error")
+           "hils_attend_decode_noalloc", "hils_workspace_bytes", "hils_workspace_init",
+           "hils_status_string", "hils_last_cuda_error")
 
 
 class HilsError(RuntimeError):
@@ -67,6 +67,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hils_select.argtypes = [P, T, i, vp, T, vp, i, vp, vp, vp, vp, sz, vp]
         lib.hils_attend_prefill.argtypes = [P, T, T, T, i, vp, vp, vp, T, vp, vp, sz, vp]
         lib.hils_attend_decode.argtypes = [P, T, T, T, vp, vp, vp, vp, T, vp, vp, sz, vp]
+        lib.hils_attend_decode_noalloc.argtypes = [P, T, T, T, vp, vp, vp, vp, T, vp, vp]
         lib.hils_workspace_bytes.argtypes = [P, i, i, i]
         lib.hils_workspace_bytes.restype = sz
         lib.hils_workspace_init.argtypes = [vp, sz, vp]
@@ -74,7 +75,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hils_status_string.restype = ctypes.c_char_p
         lib.hils_last_cuda_error.restype = ctypes.c_char_p
         for name in ("hils_summarize", "hils_select", "hils_attend_prefill", "hils_attend_decode",
-                     "hils_workspace_init"):
+                     "hils_attend_decode_noalloc", "hils_workspace_init"):
             getattr(lib, name).restype = i
         _lib = lib
     return _lib
@@ -231,6 +232,29 @@ def hils_attend_decode(p: Params, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse
     _check("hils_attend_decode", load_library().hils_attend_decode(
         ctypes.byref(p.c()), _view(Q), _view(Kc), _view(Vc), _ptr(cache_len), _ptr(idx), _ptr(score),
         _ptr(nsel), _view(O), _ptr(lse), wp, wn, _stream(stream)))
+
+
+def hils_attend_decode_noalloc(p: Params, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse=None,
+                               stream=None) -> None:
+    """hils_attend_decode with the library's built-in scratch instead of a workspace.
+
+    For callers that cannot allocate device memory; the scratch is one fixed 4 MiB
+    array per GPU, shared by every call (calls that overlap on the GPU race on it)."""
+    B, H, d, k = p.B, p.H, p.d, p.K
+    _expect("hils_attend_decode_noalloc", "Q", Q, (B, H, 1, d), p.dtype)
+    _expect("hils_attend_decode_noalloc", "O", O, (B, H, 1, d), p.dtype)
+    for name, t in (("Kc", Kc), ("Vc", Vc)):
+        if t.shape[0] != B or t.shape[1] != H or t.shape[3] != d or t.dtype != p.dtype or not t.is_cuda:
+            raise ValueError(f"hils_attend_decode_noalloc: {name} has shape {tuple(t.shape)} / {t.dtype}")
+    _expect("hils_attend_decode_noalloc", "cache_len", cache_len, (B,), torch.int32)
+    if k > 0:
+        _expect("hils_attend_decode_noalloc", "idx", idx, (B, H, 1, k), torch.int32)
+        _expect("hils_attend_decode_noalloc", "score", score, (B, H, 1, k), torch.float32)
+        _expect("hils_attend_decode_noalloc", "nsel", nsel, (B, H, 1), torch.int32)
+    _expect("hils_attend_decode_noalloc", "lse", lse, (B, H), torch.float32)
+    _check("hils_attend_decode_noalloc", load_library().hils_attend_decode_noalloc(
+        ctypes.byref(p.c()), _view(Q), _view(Kc), _view(Vc), _ptr(cache_len), _ptr(idx), _ptr(score),
+        _ptr(nsel), _view(O), _ptr(lse), _stream(stream)))
 
 
 def alloc_workspace(p: Params, call: int, Lq: int, C: int, device="cuda") -> torch.Tensor | None:

@@ -175,6 +175,28 @@ int hils_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hi
                        hils_tensor O, float *lse, void *workspace, size_t ws_bytes,
                        cudaStream_t stream);
 
+/* hils_attend_decode without a workspace argument: the library keeps the scratch
+ * memory itself, in one fixed 4 MiB array of device global memory that every GPU
+ * loading this library holds until the process exits. The paper has no counterpart;
+ * this entry point exists for callers that cannot allocate device memory: a plug-in
+ * that is handed only raw pointers and a stream by a host application owning every
+ * allocation, or code running where device allocation is forbidden or would break a
+ * fixed memory budget.
+ *   Arguments, layouts and results are those of hils_attend_decode.
+ *   Capacity: (B*H) * (K + ceil(W/64)) * (d+1) floats plus 256-byte-rounded counters
+ *   must fit in 4 MiB (hils_workspace_bytes(p, HILS_CALL_ATTEND_DECODE, 1, 0) <=
+ *   4194304); larger problems return HILS_ERR_WORKSPACE before anything is launched.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before any
+ *   stream capture. Each call then zeroes the array's counters on `stream`
+ *   (cudaMemsetAsync) and launches; nothing is allocated or freed.
+ *   All calls share the one array and it keeps the last call's contents: calls whose
+ *   work overlaps on the GPU (other streams, other host threads) race on it. */
+int hils_attend_decode_noalloc(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hils_ctensor Vc,
+                               const int32_t *cache_len,
+                               const int32_t *idx, const float *score, const int32_t *nsel,
+                               hils_tensor O, float *lse, cudaStream_t stream);
+
 /* Bytes of workspace a call needs for these sizes (Lq = queries per (b, h); C =
  * summarised chunks). Returns 0 for invalid parameters. */
 size_t hils_workspace_bytes(const hils_params *p, int call, int Lq, int C);
