@@ -176,6 +176,28 @@ __device__ __forceinline__ UnitPlan plan_unit(int u, int t, int K, int W, const 
     return p;
 }
 
+// plan_unit on already loaded inputs (the kept chunk index and score of unit u).
+__device__ __forceinline__ UnitPlan plan_unit_loaded(int u, int t, int K, int W, int c, float score, int nsel) {
+    UnitPlan p{0, 0, false, -INFINITY};
+    if (t < 0) return p;
+    if (u < K) {
+        if (u >= nsel || c < 0) return p;
+        const int start = c * kChunk;
+        if (start > t) return p;
+        p.start = start;
+        p.rows = min(kChunk, t - start + 1);
+        p.is_chunk = true;
+        p.mass = score;
+        return p;
+    }
+    const int w0 = max(0, t - W + 1);
+    const int start = w0 + (u - K) * kChunk;
+    if (W <= 0 || start > t) return p;
+    p.start = start;
+    p.rows = min(kChunk, t - start + 1);
+    return p;
+}
+
 struct DecodeWs {
     int *counters;
     float *mass;
@@ -215,44 +237,42 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float *scrat
 }
 
 // o = sum_u e^{m_u - M} o_u / sum_u e^{m_u - M} and lse = M + log(sum) over `units`
-// partials (masses m_u, vectors o_u, in global memory written by other CTAs). Writes o
-// to out[0..D) and lse to out[D]. Loads are issued in parallel: masses strided over
-// the threads, weights staged in shared memory in blocks, vectors unrolled.
+// partials (masses m_u, vectors o_u, written to global memory by other CTAs). Thread x
+// owns column x; every 32 units it issues all their mass and column loads at once and
+// folds them into a running (max, sum, weighted column) triple, so one round trip per
+// 32 units. Writes o to out[0..D) and lse to out[D].
 template <int D>
-__device__ void combine_units(const float *mass, const float *vec, int units, float *out, float *wts) {
-    constexpr int kBlock = 1024;
-    __shared__ float scratch[kThreads / 32];
-    float mloc = -INFINITY;
-    for (int v = threadIdx.x; v < units; v += kThreads) mloc = fmaxf(mloc, __ldcg(mass + v));
-    const float M = block_reduce(mloc, true, scratch);
-    float zloc = 0.f, acc = 0.f;
-    const int x = threadIdx.x;  // output column (D <= kThreads)
-    for (int v0 = 0; v0 < units; v0 += kBlock) {
-        const int nb = min(kBlock, units - v0);
-        __syncthreads();
-        for (int v = threadIdx.x; v < nb; v += kThreads) {
-            const float m = __ldcg(mass + v0 + v);
-            const float wv = M == -INFINITY ? 0.f : expf(m - M);
-            wts[v] = wv;
-            zloc += wv;
-        }
-        __syncthreads();
-        if (x < D) {
-            const float *col = vec + (size_t)v0 * D + x;
-            int v = 0;
-            for (; v + 8 <= nb; v += 8) {
-                float t[8];
+__device__ void combine_units(const float *mass, const float *vec, int units, float *out) {
+    constexpr int kB = 32;
+    const int x = threadIdx.x;
+    float M = -INFINITY, z = 0.f, acc = 0.f;
+    if (x < D) {
+        for (int v0 = 0; v0 < units; v0 += kB) {
+            float m[kB], c[kB];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) t[k] = __ldcg(col + (size_t)(v + k) * D);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) acc = fmaf(wts[v + k], t[k], acc);
+            for (int k = 0; k < kB; ++k) {
+                const bool ok = v0 + k < units;
+                m[k] = ok ? __ldcg(mass + v0 + k) : -INFINITY;
+                c[k] = ok ? __ldcg(vec + (size_t)(v0 + k) * D + x) : 0.f;
             }
-            for (; v < nb; ++v) acc = fmaf(wts[v], __ldcg(col + (size_t)v * D), acc);
+            float mb = M;
+#pragma unroll
+            for (int k = 0; k < kB; ++k) mb = fmaxf(mb, m[k]);
+            if (mb == -INFINITY) continue;
+            const float f = expf(M - mb);  // 0 when M is -inf
+            z *= f;
+            acc *= f;
+#pragma unroll
+            for (int k = 0; k < kB; ++k) {
+                const float wv = expf(m[k] - mb);
+                z += wv;
+                acc = fmaf(wv, c[k], acc);
+            }
+            M = mb;
         }
+        out[x] = M == -INFINITY ? 0.f : acc / z;
+        if (x == 0) out[D] = M == -INFINITY ? -INFINITY : M + logf(z);
     }
-    const float Z = block_reduce(zloc, false, scratch);
-    if (x < D) out[x] = M == -INFINITY ? 0.f : acc / Z;
-    if (threadIdx.x == 0) out[D] = M == -INFINITY ? -INFINITY : M + logf(Z);
     __syncthreads();
 }
 
@@ -266,9 +286,13 @@ __global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
     const int u = blockIdx.x;
     const int64_t qi = blockIdx.y;  // (b, h), one query each
     const int b = (int)(qi / a.H), h = (int)(qi % a.H);
-    const int t = a.cache_len[b] - 1;
-    const UnitPlan p = plan_unit(u, t, a.topk, a.W, a.idx + qi * a.topk, a.score + qi * a.topk,
-                                 a.topk > 0 ? a.nsel[qi] : 0);
+    // the unit's small inputs, loaded together before anything depends on them
+    const bool chunk_unit = u < a.topk;
+    const int clen = a.cache_len[b];
+    const int ns = chunk_unit ? a.nsel[qi] : 0;
+    const int cidx = chunk_unit ? a.idx[qi * a.topk + u] : -1;
+    const float csc = chunk_unit ? a.score[qi * a.topk + u] : 0.f;
+    const UnitPlan p = plan_unit_loaded(u, clen - 1, a.topk, a.W, cidx, csc, ns);
     const DecodeWs ws = decode_ws(a.ws, a.B * a.H, a.units, D);
     float *my_vec = ws.vec + ((size_t)qi * a.units + u) * D;
     if (p.rows > 0) {
@@ -291,8 +315,7 @@ __global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    combine_units<D>(ws.mass + (size_t)qi * a.units, ws.vec + (size_t)qi * a.units * D, a.units, s.red,
-                     reinterpret_cast<float *>(smem) /* K tile space, no longer needed */);
+    combine_units<D>(ws.mass + (size_t)qi * a.units, ws.vec + (size_t)qi * a.units * D, a.units, s.red);
     store_output<T, D>(a, b, h, 0, qi, s.red, s.red[D]);
     if (threadIdx.x == 0) ws.counters[qi] = 0;
 }

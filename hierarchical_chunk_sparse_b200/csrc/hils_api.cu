@@ -155,6 +155,7 @@ int hils_summarize(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ,
     HILS_TRY(check_params(p, &scale));
     if (N < 0) return HILS_ERR_INVALID_ARG;
     const int C = N / kChunk;
+    if ((int64_t)p->B * p->H * C > 0xffffffffll) return HILS_ERR_INVALID_ARG;  // chunk count fits 32 bits
     HILS_TRY(check_view(K.ptr, K.sb, K.sh, K.st, (int64_t)C * kChunk, p));
     HILS_TRY(check_view(LQ.ptr, LQ.sb, LQ.sh, LQ.st, C, p));
     HILS_TRY(check_view(Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st, C, p));
@@ -178,6 +179,7 @@ int hils_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *
     HILS_TRY(check_params(p, &scale));
     if (Lq < 0 || C < 0) return HILS_ERR_INVALID_ARG;
     const int64_t nq = (int64_t)p->B * p->H * Lq;
+    if (nq > 0x7fffffffll) return HILS_ERR_INVALID_ARG;  // query count fits in int
     HILS_TRY(check_view(Qcal.ptr, Qcal.sb, Qcal.sh, Qcal.st, Lq, p));
     HILS_TRY(check_view(Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st, C, p));
     HILS_TRY(check_array(Bsum, (int64_t)p->B * p->H * C));

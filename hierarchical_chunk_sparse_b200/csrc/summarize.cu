@@ -49,14 +49,15 @@ __global__ void __launch_bounds__(128) summarize_kernel(SummarizeArgs a) {
     float *red = prob + kChunk;
 
     const int tid = threadIdx.x;
-    const int64_t total = (int64_t)a.B * a.H * a.C;
-    const int64_t stride = gridDim.x;
+    const unsigned total = (unsigned)a.B * a.H * a.C;  // chunk count is checked to fit
+    const unsigned stride = gridDim.x;
 
-    auto issue = [&](int64_t u, int stage) {
+    auto issue = [&](unsigned u, int stage) {
         if (u < total) {
-            const int c = (int)(u % a.C);
-            const int h = (int)((u / a.C) % a.H);
-            const int b = (int)(u / ((int64_t)a.C * a.H));
+            const int c = (int)(u % (unsigned)a.C);
+            const int bh = (int)(u / (unsigned)a.C);
+            const int h = bh % a.H;
+            const int b = bh / a.H;
             const T *k0 = static_cast<const T *>(a.K.ptr) + b * a.K.sb + h * a.K.sh +
                           (int64_t)c * kChunk * a.K.st;
             const T *lq = static_cast<const T *>(a.LQ.ptr) + b * a.LQ.sb + h * a.LQ.sh + c * a.LQ.st;
@@ -74,7 +75,7 @@ __global__ void __launch_bounds__(128) summarize_kernel(SummarizeArgs a) {
     for (int s = 0; s < Cfg::kStages - 1; ++s) issue(blockIdx.x + s * stride, s);
 
     int stage = 0;
-    for (int64_t u = blockIdx.x; u < total; u += stride) {
+    for (unsigned u = blockIdx.x; u < total; u += stride) {
         issue(u + (Cfg::kStages - 1) * stride, (stage + Cfg::kStages - 1) % Cfg::kStages);
         cp_async_wait<Cfg::kStages - 1>();
         __syncthreads();
@@ -129,9 +130,10 @@ __global__ void __launch_bounds__(128) summarize_kernel(SummarizeArgs a) {
                     a0 += red[g * D + 2 * cu];
                     a1 += red[g * D + 2 * cu + 1];
                 }
-                const int c = (int)(u % a.C);
-                const int h = (int)((u / a.C) % a.H);
-                const int b = (int)(u / ((int64_t)a.C * a.H));
+                const int c = (int)(u % (unsigned)a.C);
+                const int bh = (int)(u / (unsigned)a.C);
+                const int h = bh % a.H;
+                const int b = bh / a.H;
                 T *out = static_cast<T *>(a.Ksum.ptr) + b * a.Ksum.sb + h * a.Ksum.sh + c * a.Ksum.st;
                 store2(out + 2 * cu, a0, a1);
             }

@@ -96,7 +96,8 @@ def test_select_workspace_too_small(lib):
     p = _p(B=1, H=2)
     c = p.c()
     need = lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_SELECT, 1, 8000)
-    assert need == 2 * 8000 * 8  # a screen value and radius per (query, chunk)
+    # a screen value and radius per (query, chunk), and one (max, max) pair per 64 chunks
+    assert need == 2 * (8000 + 125) * 8
     rc = lib.hils_select(ctypes.byref(c), T(ALIGNED, 256, 128, 128), 1, ALIGNED, T(ALIGNED, 0, 0, 128),
                          ALIGNED, 8000, ALIGNED, ALIGNED, ALIGNED, ALIGNED, need - 16, None)
     assert rc == 4

@@ -394,3 +394,38 @@ def test_decode_workload_full_size(oracle, cuda_device, cfg):
         assert abs(float(lse[b, h]) - lse_ref[0, 0, 0]) <= 1e-4
     del inp
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_screen_radius_covers_the_float64_score(oracle, cuda_device, d):
+    """The decode-shaped select writes every eligible chunk's float32 screen value s_c and
+    radius e_c to its workspace (the first B*H*Lq*C float pairs). The kept set is only
+    exact if |s_c - x_c| <= e_c, with x_c the oracle's float64 score: check it for every
+    chunk, and check that the observed error stays far (1/16) inside the tensor-core
+    part of the bound, scale |q| |k'| d 2^-16, so the bound is not merely lucky."""
+    w = WORKLOADS[4].replace(B=2, H=4, d=d, K=16)
+    C = 5000
+    g = torch.Generator().manual_seed(31)
+    Q = torch.randn(w.B, w.H, 1, d, generator=g).to(w.dtype)
+    Ksum = (torch.randn(w.B, w.H, C, d, generator=g) * torch.rand(w.B, w.H, C, 1, generator=g) * 2).to(w.dtype)
+    Bsum = (torch.rand(w.B, w.H, C, generator=g) * 4.0).float()
+    qpos = torch.full((w.B, 1), 64 * C + 10, dtype=torch.int32)
+    p = P(w)
+    ws = hils.alloc_workspace(p, hils.HILS_CALL_SELECT, 1, C, device=cuda_device)
+    assert ws is not None
+    idx = torch.empty(w.B, w.H, 1, w.K, dtype=torch.int32, device=cuda_device)
+    score = torch.empty(w.B, w.H, 1, w.K, device=cuda_device)
+    nsel = torch.empty(w.B, w.H, 1, dtype=torch.int32, device=cuda_device)
+    hils.hils_select(p, Q.to(cuda_device), Ksum.to(cuda_device), Bsum.to(cuda_device), idx, score, nsel,
+                     qpos=qpos.to(cuda_device), workspace=ws)
+    torch.cuda.synchronize()
+    scr = host(ws).view(torch.float32)[: w.B * w.H * C * 2].reshape(w.B, w.H, C, 2).double().numpy()
+    x = oracle.score_all(Q, Ksum, Bsum, 64, w.scale, qpos=qpos)[:, :, 0, :]
+    err = np.abs(scr[..., 0] - x)
+    assert (err <= scr[..., 1]).all(), f"radius violated: {float((err - scr[..., 1]).max()):.3e}"
+    qn = np.linalg.norm(Q.double().numpy(), axis=-1)            # [B,H,1]
+    kn = np.linalg.norm(Ksum.double().numpy(), axis=-1)         # [B,H,C]
+    tc = w.scale * qn * kn * d * 2.0 ** -16 + np.abs(x) * 2.0 ** -22
+    assert (err / tc).max() <= 1 / 16, f"observed error {float((err / tc).max()):.3f} of the bound"
+    i_ref, s_ref, n_ref = oracle.select(Q, Ksum, Bsum, 64, w.K, w.scale, qpos=qpos)
+    assert_same_selection(idx, nsel, i_ref, n_ref)
