@@ -285,6 +285,7 @@ class PrefillBench:
         self.score = torch.empty(w.B, w.H, w.N, w.K, dtype=torch.float32, device=dev)
         self.nsel = torch.empty(w.B, w.H, w.N, dtype=torch.int32, device=dev)
         self.ws = hils.alloc_workspace(self.p, hils.HILS_CALL_SELECT, w.N, C, device=dev)
+        self.ws_att = hils.alloc_workspace(self.p, hils.HILS_CALL_ATTEND_PREFILL, w.N, C, device=dev)
         self.O = torch.empty_like(self.inp["Q"])
         self.lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device=dev)
         torch.cuda.synchronize()
@@ -301,7 +302,7 @@ class PrefillBench:
     def attend(self):
         i = self.inp
         self.hils.hils_attend_prefill(self.p, i["Q"], i["K"], i["V"], self.idx, self.score, self.nsel,
-                                      self.O, self.lse)
+                                      self.O, self.lse, workspace=self.ws_att)
 
     def step(self):
         self.summarize()

@@ -137,7 +137,7 @@ size_t hils_workspace_bytes(const hils_params *p, int call, int Lq, int C) {
     if (check_params(p, &scale) != HILS_OK || Lq < 0 || C < 0) return 0;
     switch (call) {
     case HILS_CALL_SELECT: return select_ws_for(p, Lq, C);
-    case HILS_CALL_ATTEND_PREFILL: return 0;
+    case HILS_CALL_ATTEND_PREFILL: return kPrefillWsBytes;
     case HILS_CALL_ATTEND_DECODE: return attend_decode_ws_bytes(p->B * p->H, decode_units(p), p->d);
     default: return 0;
     }
@@ -224,8 +224,7 @@ int hils_attend_prefill(const hils_params *p, hils_ctensor Q, hils_ctensor K, hi
     HILS_TRY(check_array(score, nq * p->K));
     HILS_TRY(check_array(nsel, p->K > 0 ? nq : 0));
     HILS_TRY(check_array(lse, 0));
-    (void)workspace;
-    (void)ws_bytes;
+    HILS_TRY(check_workspace(workspace, ws_bytes, kPrefillWsBytes));
     if (nq == 0) return HILS_OK;
     AttendArgs a;
     a.Q = {Q.ptr, Q.sb, Q.sh, Q.st};
@@ -245,7 +244,9 @@ int hils_attend_prefill(const hils_params *p, hils_ctensor Q, hils_ctensor K, hi
     a.W = p->W;
     a.scale = scale;
     a.units = decode_units(p);
-    a.ws = nullptr;
+    a.ws = workspace;
+    if (attend_prefill_tc_supported(p->dtype, p->d, N))
+        return launch_attend_prefill_tc(a, N, static_cast<uint32_t *>(workspace), stream);
     return launch_attend_prefill_general(p->dtype, p->d, a, stream);
 }
 

@@ -69,6 +69,11 @@ hils_status launch_summarize(hils_dtype dt, int d, const SummarizeArgs &a, cudaS
 hils_status launch_select(hils_dtype dt, int d, const SelectArgs &a, cudaStream_t s);
 hils_status launch_attend_decode(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s);
 hils_status launch_attend_prefill_general(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s);
+// Tensor-core prefill (bf16, d = 128): used when supported; `status` receives a nonzero
+// word if one of its bounded waits expired.
+bool attend_prefill_tc_supported(hils_dtype dt, int d, int N);
+hils_status launch_attend_prefill_tc(const AttendArgs &a, int N, uint32_t *status, cudaStream_t s);
+constexpr size_t kPrefillWsBytes = 256;  // status word (+ padding)
 
 // Workspace layouts (bytes); shared by the host size query and the kernels.
 size_t select_ws_bytes(int queries, int C, int ctas_per_query);

@@ -150,11 +150,16 @@ int hils_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *
  *     output sum_{j in c} softmax_j(scale q_i.k_j) v_j, and
  *   - each window token j in [max(0, i-W+1), i] with weight exp(scale q_i.k_j) / Z^_i.
  *   Q, K, V  [B, H, N, d]
- *   idx, score, nsel: as written by hils_select (score is used as the chunk's log-mass;
- *         passing exact log Z_{i,c} instead gives exact block-sparse attention)
+ *   idx, score, nsel: as written by hils_select: each row's first nsel entries are
+ *         distinct chunks in ascending chunk index (score is used as the chunk's
+ *         log-mass; passing exact log Z_{i,c} instead gives exact block-sparse attention)
  *   O    [B, H, N, d]  out, dtype (float32 result rounded to nearest-even)
  *   lse  [B, H, N] float32 out: log Z^_i, or NULL
- *   workspace, ws_bytes: hils_workspace_bytes(p, HILS_CALL_ATTEND_PREFILL, N, C). */
+ *   workspace, ws_bytes: hils_workspace_bytes(p, HILS_CALL_ATTEND_PREFILL, N, C) bytes,
+ *         zeroed before first use. Its first 32-bit word is a status word: the bf16,
+ *         d = 128 path (tensor cores, bounded waits) sets it nonzero if a wait on its own
+ *         asynchronous copies or matrix operations ever expires, and then writes no output
+ *         for the affected tile. */
 int hils_attend_prefill(const hils_params *p, hils_ctensor Q, hils_ctensor K, hils_ctensor V,
                         int N, const int32_t *idx, const float *score, const int32_t *nsel,
                         hils_tensor O, float *lse, void *workspace, size_t ws_bytes,

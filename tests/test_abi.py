@@ -121,7 +121,7 @@ def test_decode_workspace_too_small(lib):
 def test_workspace_sizes(lib):
     assert lib.hils_workspace_bytes(None, 0, 1, 1) == 0
     assert lib.hils_workspace_bytes(ctypes.byref(_p(d=80).c()), 0, 1, 1) == 0
-    assert lib.hils_workspace_bytes(ctypes.byref(_p().c()), hils.HILS_CALL_ATTEND_PREFILL, 8192, 128) == 0
+    assert lib.hils_workspace_bytes(ctypes.byref(_p().c()), hils.HILS_CALL_ATTEND_PREFILL, 8192, 128) == 256
 
 
 def test_status_strings(lib):

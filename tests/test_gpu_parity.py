@@ -51,7 +51,9 @@ def gpu_prefill(w, Q, K, V, idx, score, nsel, Kk=None, W=None):
     p = P(w, K=w.K if Kk is None else Kk, W=w.W if W is None else W)
     O = torch.full_like(Q, 99.0)
     lse = torch.full(Q.shape[:3], 99.0, dtype=torch.float32, device=Q.device)
-    hils.hils_attend_prefill(p, Q, K, V, idx, score, nsel, O, lse)
+    ws = hils.alloc_workspace(p, hils.HILS_CALL_ATTEND_PREFILL, Q.shape[2], 0, device=Q.device)
+    hils.hils_attend_prefill(p, Q, K, V, idx, score, nsel, O, lse, workspace=ws)
+    assert int(host(ws[:4]).view(torch.int32)[0]) == 0, "a bounded wait expired"
     return O, lse
 
 
