@@ -177,6 +177,12 @@ def max_over_ranks(x: float, world: int, dev) -> float:
     return float(t.item())
 
 
+def job_throughput(units_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job rate: every rank processes its own replica's units in each step, and
+    the step takes as long as the slowest rank (ms_per_step is already that maximum)."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -498,7 +504,7 @@ def main():
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(statistics.mean(per), world, dev)
-    value = world * w.B / (ms / 1e3)
+    value = job_throughput(w.B, world, ms)
     # per-kernel times (same protocol)
     t_sel = statistics.mean(time_steps(sel_g, args.steps, flush, stream))
     t_att = statistics.mean(time_steps(att_g, args.steps, flush, stream))
@@ -563,7 +569,7 @@ def main():
                               "frac_8tbs": step_gbs / 8000.0},
             "kernel_us": {"select": 1e3 * t_sel, "attend": 1e3 * t_att,
                           "select_gbs": sel_gbs, "attend_gbs": att_gbs},
-            "e2e": {"value": world * w.B / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": job_throughput(w.B, world, ms_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps * 2,
             "clocks": clk.summary(),
