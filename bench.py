@@ -305,6 +305,12 @@ class PrefillBench:
         self.hils.hils_select(self.p, i["Qcal"], self.Ksum, self.Bsum, self.idx, self.score, self.nsel,
                               workspace=self.ws)
 
+    def check_status(self):
+        """The status words of select and attend: nonzero if a bounded wait expired."""
+        for name, ws in (("select", self.ws), ("attend", self.ws_att)):
+            if ws is not None and int(ws[:4].view(torch.int32)[0].item()) != 0:
+                raise RuntimeError(f"prefill {name}: a bounded wait expired (status word set)")
+
     def attend(self):
         i = self.inp
         self.hils.hils_attend_prefill(self.p, i["Q"], i["K"], i["V"], self.idx, self.score, self.nsel,
@@ -539,6 +545,8 @@ def main():
         pt = max_over_ranks(pt, world, dev)
         ks = {k: statistics.mean(time_steps(graphed(getattr(pb, k), stream), n, flush, stream))
               for k in ("summarize", "select", "attend")}
+        torch.cuda.synchronize()
+        pb.check_status()
         fl = prefill_flops(wp)
         tf = fl / (pt * 1e-3) / 1e12
         prefill = {"value": tf * world, "unit": "TFLOP/s", "ms_per_step": pt, "workload": wp.name,

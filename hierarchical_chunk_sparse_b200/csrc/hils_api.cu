@@ -100,9 +100,9 @@ int decode_units(const hils_params *p) {
 }
 
 size_t select_ws_for(const hils_params *p, int Lq, int C) {
-    int ctas = 0, tiles = 0;
-    select_split_plan(p->B, p->H, Lq, C, p->K, true, device_sm_count(), &ctas, &tiles);
-    return select_ws_bytes(p->B * p->H * Lq, C, ctas);
+    SelectArgs a;
+    select_plan(p->dtype, p->d, p->B, p->H, Lq, C, p->K, true, device_sm_count(), &a);
+    return select_ws_bytes(p->B * p->H * Lq, C, a.path);
 }
 
 #define HILS_TRY(expr)                 \
@@ -202,9 +202,8 @@ int hils_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *
     a.C = C;
     a.topk = p->K;
     a.scale = scale;
-    select_split_plan(p->B, p->H, Lq, C, p->K, qpos != nullptr, device_sm_count(), &a.ctas_per_query,
-                      &a.tiles_per_warp);
-    HILS_TRY(check_workspace(workspace, ws_bytes, select_ws_bytes((int)nq, C, a.ctas_per_query)));
+    select_plan(p->dtype, p->d, p->B, p->H, Lq, C, p->K, qpos != nullptr, device_sm_count(), &a);
+    HILS_TRY(check_workspace(workspace, ws_bytes, select_ws_bytes((int)nq, C, a.path)));
     a.ws = workspace;
     return launch_select(p->dtype, p->d, a, stream);
 }

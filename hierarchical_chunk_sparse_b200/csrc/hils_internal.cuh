@@ -43,11 +43,17 @@ struct SelectArgs {
     int32_t *nsel;
     int B, H, Lq, C, topk;
     float scale;
+    int path;              // SelectPath chosen by select_plan
     // split search over chunk ranges (decode-like shapes)
-    int ctas_per_query;    // grid.x of the split kernel
+    int ctas_per_query;    // summary blocks per query of the screen kernel
     int tiles_per_warp;    // 128-chunk tiles each warp scans
-    void *ws;              // per-query partial lists + arrival counters
+    void *ws;              // status word, then the screen values of the split search
 };
+
+// Which select kernels run: one warp per query; screen + pick (few queries, long
+// tables); tensor-core scoring with one thread per query (many bf16 queries, d = 128).
+enum SelectPath { kSelectWarp = 0, kSelectSplit = 1, kSelectTc = 2 };
+constexpr size_t kSelectStatusBytes = 256;  // status word at the front of the select workspace
 
 struct AttendArgs {
     View Q, K, V;
@@ -76,12 +82,17 @@ hils_status launch_attend_prefill_tc(const AttendArgs &a, int N, uint32_t *statu
 constexpr size_t kPrefillWsBytes = 256;  // status word (+ padding)
 
 // Workspace layouts (bytes); shared by the host size query and the kernels.
-size_t select_ws_bytes(int queries, int C, int ctas_per_query);
+size_t select_ws_bytes(int queries, int C, int path);
 size_t attend_decode_ws_bytes(int queries, int units, int d);
 
-// Choice of the split search for hils_select; identical on the size query and the call.
-void select_split_plan(int B, int H, int Lq, int C, int K, bool has_qpos, int num_sms,
-                       int *ctas_per_query, int *tiles_per_warp);
+// Choice of the select kernels (path, ctas_per_query, tiles_per_warp of `a`); the
+// workspace size depends only on the sizes, never on has_qpos, so the size query and
+// the call agree.
+void select_plan(hils_dtype dt, int d, int B, int H, int Lq, int C, int K, bool has_qpos, int num_sms,
+                 SelectArgs *a);
+// Tensor-core select (bf16, d = 128, at most 512 eligible chunks per query).
+bool select_tc_supported(hils_dtype dt, int d, int B, int H, int Lq, int C, int K, bool has_qpos);
+hils_status launch_select_tc(const SelectArgs &a, cudaStream_t s);
 
 int device_sm_count();
 hils_status record_cuda_error(cudaError_t e);

@@ -1,0 +1,343 @@
+// Exact top-K building blocks shared by the select kernels: "Hierarchical Sparse
+// Attention Done Right" (picx.dev summary), Eq. 7 and Methodology 2, and the rcap.io
+// post's pseudocode figure (keep the top K chunks per query).
+//
+// Exactness rests on interval screening. Each chunk carries a float32 screen value s
+// with a rigorous radius e; certainly-in and certainly-out chunks are settled by the
+// intervals alone, and only the chunks in between get the float64 score
+//   x_c = (sum_x q~_x k'_x) * scale + b'_c   (every product and sum rounded to float64,
+//                                             in x order).
+// The warp routines below keep a running exact top-K list over 128-chunk tiles, one
+// lane per chunk.
+#pragma once
+#include <float.h>
+#include <limits.h>
+#include <math.h>
+
+#include "hils_internal.cuh"
+
+namespace hils {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTile = 128;      // chunks scored per warp step
+constexpr int kMaxK = 32;
+constexpr int kListBytes = 768; // one list of <= 32 entries in the workspace
+
+// One list of kept entries (in shared memory or the workspace).
+struct EntryList {
+    double x[kMaxK];   // exact score, NaN if not computed
+    int idx[kMaxK];
+    float s[kMaxK];
+    float e[kMaxK];
+    int n;
+    float bound;       // lower bound on the K-th largest lo of the range the list covers
+};
+static_assert(sizeof(EntryList) <= kListBytes, "list size");
+
+template <int R>
+struct Slots {
+    int idx[R];
+    float s[R];
+    float e[R];
+    double x[R];
+};
+
+struct QueryCtx {
+    const void *qrow;       // q~_i in global memory (for exact scores)
+    const void *khead;      // k'_0 of this (b, h)
+    int64_t kst;
+    const float *bhead;     // b'_0 of this (b, h)
+    float scale;
+};
+
+template <typename T, int D>
+__device__ double exact_score(const QueryCtx &q, int c) {
+    // rows are read with 16-byte loads, half a row at a time, before the fixed-order
+    // float64 chain runs over them
+    constexpr int kN = Vec<T>::kN, kHalf = D / kN / 2;
+    const uint4 *qr = static_cast<const uint4 *>(q.qrow);
+    const uint4 *kr = reinterpret_cast<const uint4 *>(static_cast<const T *>(q.khead) + (int64_t)c * q.kst);
+    double acc = 0.0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint4 qv[kHalf], kv[kHalf];
+#pragma unroll
+        for (int u = 0; u < kHalf; ++u) {
+            qv[u] = __ldg(qr + h * kHalf + u);
+            kv[u] = __ldg(kr + h * kHalf + u);
+        }
+#pragma unroll
+        for (int u = 0; u < kHalf; ++u) {
+            float qf[kN], kf[kN];
+            widen(qv[u], qf, T());
+            widen(kv[u], kf, T());
+#pragma unroll
+            for (int i = 0; i < kN; ++i) acc = __dadd_rn(acc, __dmul_rn((double)qf[i], (double)kf[i]));
+        }
+    }
+    return __dadd_rn(__dmul_rn(acc, (double)q.scale), (double)q.bhead[c]);
+}
+
+// Float32 screen value and its error radius for chunk c; qs = query in shared memory.
+template <typename T, int D>
+__device__ __forceinline__ void screen(const QueryCtx &q, const float *qs, int c, float &s, float &e) {
+    const uint4 *kr = reinterpret_cast<const uint4 *>(static_cast<const T *>(q.khead) + (int64_t)c * q.kst);
+    constexpr int kN = Vec<T>::kN;
+    float dot = 0.f, ad = 0.f;
+#pragma unroll
+    for (int u = 0; u < D / kN; ++u) {
+        float kf[kN];
+        widen(__ldg(kr + u), kf, T());
+#pragma unroll
+        for (int i = 0; i < kN; ++i) {
+            const float qv = qs[u * kN + i];
+            dot = fmaf(qv, kf[i], dot);
+            ad = fmaf(fabsf(qv), fabsf(kf[i]), ad);
+        }
+    }
+    s = fmaf(dot, q.scale, q.bhead[c]);
+    e = fmaf(q.scale * ad, (float)(D + 2) * 0x1p-23f, fabsf(s) * 0x1p-22f);
+}
+
+// Exact top-K of the warp's pool (R slots per lane, idx < 0 = empty). Returns the
+// lane's mask of kept slots. Uniform control flow across the warp.
+// `bound` receives a lower bound on the pool's K-th largest lo (s_K - e_max, rounded
+// down), or -inf when the pool holds at most K entries. Any chunk whose hi lies below
+// the bound of some subset of its competitors is certainly out.
+template <typename T, int D, int R>
+__device__ unsigned warp_topk(Slots<R> &p, int K, const QueryCtx &q, float &bound) {
+    const int lane = threadIdx.x & 31;
+    unsigned valid = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+        if (p.idx[r] >= 0) valid |= 1u << r;
+    const int n = __reduce_add_sync(kFull, __popc(valid));
+    bound = -INFINITY;
+    if (n <= K) return valid;
+
+    float em = 0.f;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+        if (valid >> r & 1) em = fmaxf(em, p.e[r]);
+    em = warp_max(em);
+
+    // K-th and (K+1)-th largest screen values (duplicates counted separately)
+    unsigned taken = 0;
+    float sK = 0.f, sK1 = 0.f;
+    for (int it = 0; it <= K; ++it) {
+        unsigned best = 0u;
+        int bslot = -1;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            if ((valid & ~taken) >> r & 1) {
+                const unsigned k = ordered_key(p.s[r]);
+                if (k > best) {
+                    best = k;
+                    bslot = r;
+                }
+            }
+        }
+        const unsigned wmax = __reduce_max_sync(kFull, best);
+        const unsigned owners = __ballot_sync(kFull, bslot >= 0 && best == wmax);
+        if (lane == __ffs(owners) - 1) taken |= 1u << bslot;
+        const float v = key_to_float(wmax);
+        if (it == K - 1) sK = v;
+        sK1 = v;
+    }
+    const float lo_cut = __fsub_rd(sK, em);
+    const float hi_cut = __fadd_ru(sK1, em);
+    bound = lo_cut;
+
+    unsigned in = 0, band = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        if (valid >> r & 1) {
+            const float lo = __fsub_rd(p.s[r], p.e[r]);
+            const float hi = __fadd_ru(p.s[r], p.e[r]);
+            if (lo > hi_cut) in |= 1u << r;
+            else if (hi >= lo_cut) band |= 1u << r;
+        }
+    }
+    const int need = K - __reduce_add_sync(kFull, __popc(in));
+    if (need > 0) {
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            if ((band >> r & 1) && isnan(p.x[r])) p.x[r] = exact_score<T, D>(q, p.idx[r]);
+        unsigned chosen = 0;
+        for (int it = 0; it < need; ++it) {
+            double bx = -INFINITY;
+            int bi = INT_MAX;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                if ((band & ~chosen) >> r & 1) {
+                    if (p.x[r] > bx || (p.x[r] == bx && p.idx[r] < bi)) {
+                        bx = p.x[r];
+                        bi = p.idx[r];
+                    }
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const double ox = __shfl_xor_sync(kFull, bx, o);
+                const int oi = __shfl_xor_sync(kFull, bi, o);
+                if (ox > bx || (ox == bx && oi < bi)) {
+                    bx = ox;
+                    bi = oi;
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                if (((band & ~chosen) >> r & 1) && p.idx[r] == bi) chosen |= 1u << r;
+        }
+        in |= chosen;
+    }
+    return in;
+}
+
+// Appends the lane's kept slots to `list` after its first `base` entries; returns the
+// new length.
+template <int R>
+__device__ int warp_append(const Slots<R> &p, unsigned keep, EntryList &list, int base) {
+    const int lane = threadIdx.x & 31;
+    const int cnt = __popc(keep);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int pos = base + incl - cnt;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        if (keep >> r & 1) {
+            list.idx[pos] = p.idx[r];
+            list.s[pos] = p.s[r];
+            list.e[pos] = p.e[r];
+            list.x[pos] = p.x[r];
+            ++pos;
+        }
+    }
+    return base + __shfl_sync(kFull, incl, 31);
+}
+
+// Scores chunks [c0, c1) in tiles of 128 and leaves their exact top-K in `list`.
+template <typename T, int D>
+__device__ void warp_scan(const QueryCtx &q, const float *qs, int c0, int c1, int K, EntryList &list) {
+    const int lane = threadIdx.x & 31;
+    int n = 0;
+    for (int base = c0; base < c1; base += kTile) {
+        Slots<5> p;
+        // slot 0 carries the running list, one entry per lane
+        p.idx[0] = lane < n ? list.idx[lane] : -1;
+        p.s[0] = lane < n ? list.s[lane] : 0.f;
+        p.e[0] = lane < n ? list.e[lane] : 0.f;
+        p.x[0] = lane < n ? list.x[lane] : 0.0;
+#pragma unroll
+        for (int r = 1; r < 5; ++r) {
+            const int c = base + lane + 32 * (r - 1);
+            p.idx[r] = c < c1 ? c : -1;
+            p.s[r] = 0.f;
+            p.e[r] = 0.f;
+            p.x[r] = __longlong_as_double(0x7ff8000000000000ll);  // NaN: not computed
+            if (c < c1) screen<T, D>(q, qs, c, p.s[r], p.e[r]);
+        }
+        float bnd;
+        const unsigned keep = warp_topk<T, D, 5>(p, K, q, bnd);
+        __syncwarp();
+        n = warp_append<5>(p, keep, list, 0);
+        __syncwarp();
+    }
+    if (lane == 0) list.n = n;
+    __syncwarp();
+}
+
+// Reduces `nlists` lists (<= R*32 entries in total) to their exact top-K in `out`.
+template <typename T, int D, int R>
+__device__ void warp_merge(const QueryCtx &q, const EntryList *lists, int nlists, bool from_global, int K,
+                           EntryList &out) {
+    const int lane = threadIdx.x & 31;
+    Slots<R> p;
+#pragma unroll
+    for (int r = 0; r < R; ++r) p.idx[r] = -1;
+    // entry (l, j) -> pool position l*K + j -> slot (pos / 32) of lane (pos % 32)
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int pos = r * 32 + lane;
+        const int l = pos / (K > 0 ? K : 1), j = pos - l * (K > 0 ? K : 1);
+        if (K > 0 && l < nlists) {
+            const EntryList &L = lists[l];
+            const int ln = from_global ? __ldcg(&L.n) : L.n;
+            if (j < ln) {
+                p.idx[r] = from_global ? __ldcg(&L.idx[j]) : L.idx[j];
+                p.s[r] = from_global ? __ldcg(&L.s[j]) : L.s[j];
+                p.e[r] = from_global ? __ldcg(&L.e[j]) : L.e[j];
+                p.x[r] = from_global ? __ldcg(&L.x[j]) : L.x[j];
+            }
+        }
+    }
+    float bnd;
+    const unsigned keep = warp_topk<T, D, R>(p, K, q, bnd);
+    __syncwarp();
+    const int n = warp_append<R>(p, keep, out, 0);
+    if (lane == 0) out.n = n;
+    __syncwarp();
+}
+
+// Writes a kept list in ascending chunk index, padded to K.
+__device__ void warp_write(const EntryList &list, int K, int64_t qi, int32_t *idx, float *score, int32_t *nsel) {
+    const int lane = threadIdx.x & 31;
+    const int n = list.n;
+    if (lane < n) {
+        const int me = list.idx[lane];
+        int rank = 0;
+        for (int j = 0; j < n; ++j) rank += list.idx[j] < me;
+        idx[qi * K + rank] = me;
+        score[qi * K + rank] = list.s[lane];
+    } else if (lane < K) {
+        idx[qi * K + lane] = -1;
+        score[qi * K + lane] = -INFINITY;
+    }
+    if (lane == 0) nsel[qi] = n;
+}
+
+template <typename T, int D>
+__device__ __forceinline__ QueryCtx make_ctx(const SelectArgs &a, int64_t qi, int &t) {
+    const int q32 = (int)qi;  // query counts are checked to fit in int
+    const int i = q32 % a.Lq;
+    const int bh = q32 / a.Lq;
+    const int h = bh % a.H;
+    const int b = bh / a.H;
+    t = a.qpos ? a.qpos[(int64_t)b * a.Lq + i] : i;
+    QueryCtx q;
+    q.qrow = static_cast<const T *>(a.Qcal.ptr) + b * a.Qcal.sb + h * a.Qcal.sh + i * a.Qcal.st;
+    q.khead = static_cast<const T *>(a.Ksum.ptr) + b * a.Ksum.sb + h * a.Ksum.sh;
+    q.kst = a.Ksum.st;
+    q.bhead = a.Bsum + ((int64_t)b * a.H + h) * a.C;
+    q.scale = a.scale;
+    return q;
+}
+
+__device__ __forceinline__ int eligible(int t, int C) {
+    const int e = t >= 0 ? t / kChunk : 0;
+    return e < C ? e : C;
+}
+
+template <typename T, int D>
+__device__ void load_query_f32(const QueryCtx &q, float *qs) {
+    const T *qr = static_cast<const T *>(q.qrow);
+    for (int x = threadIdx.x & 31; x < D; x += 32) qs[x] = (float)qr[x];
+}
+
+// Upper-tail standard normal quantile z with P(Z > z) = p, 0 < p <= 0.5
+// (Abramowitz and Stegun 26.2.23 rational approximation, |error| < 4.5e-4); used only
+// to place a first threshold guess, never to decide membership.
+__device__ __forceinline__ float normal_upper_quantile(float p) {
+    const float t = sqrtf(-2.f * logf(p));
+    return t - (2.515517f + t * (0.802853f + t * 0.010328f)) /
+                   (1.f + t * (1.432788f + t * (0.189269f + t * 0.001308f)));
+}
+
+}  // namespace
+}  // namespace hils

@@ -96,8 +96,9 @@ def test_select_workspace_too_small(lib):
     p = _p(B=1, H=2)
     c = p.c()
     need = lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_SELECT, 1, 8000)
-    # a screen value and radius per (query, chunk), and one (max, max) pair per 64 chunks
-    assert need == 2 * (8000 + 125) * 8
+    # a 256-byte status header, then a screen value and radius per (query, chunk) and
+    # one (max, max) pair per 64 chunks
+    assert need == 256 + 2 * (8000 + 125) * 8
     rc = lib.hils_select(ctypes.byref(c), T(ALIGNED, 256, 128, 128), 1, ALIGNED, T(ALIGNED, 0, 0, 128),
                          ALIGNED, 8000, ALIGNED, ALIGNED, ALIGNED, ALIGNED, need - 16, None)
     assert rc == 4
@@ -122,6 +123,8 @@ def test_workspace_sizes(lib):
     assert lib.hils_workspace_bytes(None, 0, 1, 1) == 0
     assert lib.hils_workspace_bytes(ctypes.byref(_p(d=80).c()), 0, 1, 1) == 0
     assert lib.hils_workspace_bytes(ctypes.byref(_p().c()), hils.HILS_CALL_ATTEND_PREFILL, 8192, 128) == 256
+    # many queries: the status word alone
+    assert lib.hils_workspace_bytes(ctypes.byref(_p().c()), hils.HILS_CALL_SELECT, 8192, 128) == 256
 
 
 def test_status_strings(lib):

@@ -44,6 +44,7 @@ def gpu_select(w, Qcal, Ksum, Bsum, qpos=None, K=None):
     nsel = torch.full((B, H, Lq), 7777, dtype=torch.int32, device=Qcal.device)
     ws = hils.alloc_workspace(p, hils.HILS_CALL_SELECT, Lq, Ksum.shape[2], device=Qcal.device)
     hils.hils_select(p, Qcal, Ksum, Bsum, idx, score, nsel, qpos=qpos, workspace=ws)
+    assert int(host(ws[:4]).view(torch.int32)[0]) == 0, "a bounded wait expired"
     return idx, score, nsel
 
 
@@ -219,6 +220,82 @@ def test_select_k_extremes(oracle, cuda_device, K):
     assert_same_selection(idx, nsel, i_ref, n_ref)
     if K:
         scores_close(score, s_ref, n_ref)
+
+
+# many bf16 queries with d = 128 take the tensor-core select (scores in TMEM, one thread
+# per query); these cases reach its column blocks, explicit positions, strided views and
+# the exact fallback for rows with heavy ties
+
+def _prefill_select_case(oracle, dev, w, qpos=None, Qcal=None, Ksum=None, Bsum=None, K=None):
+    inp = make_prefill(w)
+    d = to_dev(inp, dev)
+    if Ksum is None:
+        Ksum, Bsum = gpu_summarize(w, d["K"], d["LQ"])
+    Q = d["Qcal"] if Qcal is None else Qcal
+    idx, score, nsel = gpu_select(w, Q, Ksum, Bsum, qpos=None if qpos is None else qpos.to(dev), K=K)
+    i_ref, s_ref, n_ref = oracle.select(host(Q), host(Ksum), host(Bsum), 64, w.K if K is None else K, w.scale,
+                                        qpos=qpos)
+    assert_same_selection(idx, nsel, i_ref, n_ref)
+    scores_close(score, s_ref, n_ref)
+    return idx, nsel
+
+
+@pytest.mark.parametrize("N", [64 * 300 + 17, 64 * 512 + 1, 64 * 513 + 5])
+def test_select_tc_long_prefill(oracle, cuda_device, N):
+    """300 chunks (column blocks of 256 + 64), the 512-column maximum, and 513 chunks
+    (beyond TMEM: the warp kernel)."""
+    w = WORKLOADS[2].replace(H=2 if N < 64 * 400 else 1, N=N)
+    _prefill_select_case(oracle, cuda_device, w)
+
+
+def test_select_tc_explicit_positions(oracle, cuda_device):
+    """A later slice of a sequence: queries at t = 4096 + i against 96 chunks, plus a few
+    rows moved before the first chunk and past the last."""
+    w = WORKLOADS[2].replace(B=2, H=3, N=2048)
+    inp = make_prefill(w)
+    C = 96
+    g = torch.Generator().manual_seed(21)
+    Ksum = (torch.randn(w.B, w.H, C, w.d, generator=g) * 0.3).to(w.dtype)
+    Bsum = torch.rand(w.B, w.H, C, generator=g) * 0.2 + 4.0
+    qpos = (torch.arange(w.N, dtype=torch.int32) + 4096).repeat(w.B, 1)
+    qpos[0, :5] = torch.tensor([0, 63, 64, 65, -3], dtype=torch.int32)
+    qpos[1, -3:] = 64 * 200
+    dev = cuda_device
+    _prefill_select_case(oracle, dev, w, qpos=qpos, Qcal=inp["Qcal"].to(dev), Ksum=Ksum.to(dev),
+                         Bsum=Bsum.to(dev))
+
+
+def test_select_tc_strided_views(oracle, cuda_device):
+    """Q~ and k' inside wider buffers with permuted batch and head strides."""
+    w = WORKLOADS[2].replace(B=2, H=3, N=1000)
+    C = w.N // 64
+    g = torch.Generator().manual_seed(22)
+    qbig = (torch.randn(w.H, w.B, w.N, 2 * w.d, generator=g) / 11.3).to(w.dtype).to(cuda_device)
+    kbig = (torch.randn(w.H, w.B, C, w.d + 64, generator=g) * 0.3).to(w.dtype).to(cuda_device)
+    Qcal = qbig.permute(1, 0, 2, 3)[..., w.d:]
+    Ksum = kbig.permute(1, 0, 2, 3)[..., 64:]
+    Bsum = (torch.rand(w.B, w.H, C, generator=g) * 0.3 + 4.0).to(cuda_device)
+    _prefill_select_case(oracle, cuda_device, w, Qcal=Qcal, Ksum=Ksum, Bsum=Bsum)
+
+
+@pytest.mark.parametrize("K", [1, 8, 28])
+def test_select_tc_ties_fall_back_exactly(oracle, cuda_device, K):
+    """Head 0: every summary equal (all rows tie). Head 1: twelve equal summaries on top
+    (more band entries than the per-row capacity). Head 2: ordinary scores."""
+    w = WORKLOADS[2].replace(H=3, N=64 * 60 + 9)
+    C = w.N // 64
+    g = torch.Generator().manual_seed(23)
+    Ksum = (torch.randn(1, 3, C, w.d, generator=g) * 0.3).to(w.dtype)
+    Bsum = torch.rand(1, 3, C, generator=g) * 0.2 + 4.0
+    Ksum[0, 0] = Ksum[0, 0, 0].clone()
+    Bsum[0, 0] = 4.1
+    rows = torch.randperm(C, generator=g)[:12]
+    Ksum[0, 1, rows] = Ksum[0, 1, rows[0]].clone()
+    Bsum[0, 1, rows] = 9.0
+    idx, nsel = _prefill_select_case(oracle, cuda_device, w, Qcal=make_prefill(w)["Qcal"].to(cuda_device),
+                                     Ksum=Ksum.to(cuda_device), Bsum=Bsum.to(cuda_device), K=K)
+    last = host(idx)[0, 0, -1]
+    assert (last[:K] == torch.arange(K, dtype=torch.int32)).all()  # ties: lowest indices
 
 
 def test_select_without_chunks(cuda_device):
@@ -401,7 +478,8 @@ def test_decode_workload_full_size(oracle, cuda_device, cfg):
 @pytest.mark.parametrize("d", [128, 64])
 def test_screen_radius_covers_the_float64_score(oracle, cuda_device, d):
     """The decode-shaped select writes every eligible chunk's float32 screen value s_c and
-    radius e_c to its workspace (the first B*H*Lq*C float pairs). The kept set is only
+    radius e_c to its workspace (B*H*Lq*C float pairs after the 256-byte status header,
+    which must stay zero). The kept set is only
     exact if |s_c - x_c| <= e_c, with x_c the oracle's float64 score: check it for every
     chunk, and check that the observed error stays far (1/16) inside the tensor-core
     part of the bound, scale |q| |k'| d 2^-16, so the bound is not merely lucky."""
@@ -421,7 +499,9 @@ def test_screen_radius_covers_the_float64_score(oracle, cuda_device, d):
     hils.hils_select(p, Q.to(cuda_device), Ksum.to(cuda_device), Bsum.to(cuda_device), idx, score, nsel,
                      qpos=qpos.to(cuda_device), workspace=ws)
     torch.cuda.synchronize()
-    scr = host(ws).view(torch.float32)[: w.B * w.H * C * 2].reshape(w.B, w.H, C, 2).double().numpy()
+    wsh = host(ws)
+    assert (wsh[:256] == 0).all()
+    scr = wsh[256:].view(torch.float32)[: w.B * w.H * C * 2].reshape(w.B, w.H, C, 2).double().numpy()
     x = oracle.score_all(Q, Ksum, Bsum, 64, w.scale, qpos=qpos)[:, :, 0, :]
     err = np.abs(scr[..., 0] - x)
     assert (err <= scr[..., 1]).all(), f"radius violated: {float((err - scr[..., 1]).max()):.3e}"
