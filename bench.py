@@ -4,10 +4,10 @@
 Headline (one JSON line on rank 0):
   decode tokens/s at a 512K-token KV cache (B=1, H=32, d=128, chunk 64, top-K 16,
   window 512; synthetic Gaussian K/V with one needle key per head). One step = one
-  new token through the whole decode path: hils_select (Eq. 7 scores over 8191
-  chunk summaries + exact top-K) then hils_attend_decode (Eq. 10 over 16 chunks +
-  the window). Summaries are built once beforehand (hils_summarize), as a server
-  keeps them with its KV cache.
+  new token through the whole decode path in one call, hils_decode: the select (Eq. 7
+  scores over 8191 chunk summaries + exact top-K) then the attend (Eq. 10 over 16
+  chunks + the window). Summaries are built once beforehand (hils_summarize), as a
+  server keeps them with its KV cache.
 Beside it, in the same line:
   "prefill": algorithmic TFLOP/s of summarise + select + prefill attend on the 8K
   prefill workload (B=1, H=32, d=128, K=16, W=512);
@@ -222,10 +222,12 @@ class DecodeBench:
         self.nsel = torch.empty(w.B, w.H, 1, dtype=torch.int32, device=dev)
         self.ws_sel = hils.alloc_workspace(self.p, hils.HILS_CALL_SELECT, 1, C, device=dev)
         self.ws_dec = hils.alloc_workspace(self.p, hils.HILS_CALL_ATTEND_DECODE, 1, 0, device=dev)
+        self.ws_step = hils.alloc_workspace(self.p, hils.HILS_CALL_DECODE, 1, C, device=dev)
         self.O = torch.empty_like(inp["Q"])
         self.lse = torch.empty(w.B, w.H, dtype=torch.float32, device=dev)
         torch.cuda.synchronize()
-        self.launches_per_step = 2
+        # one step = hils_decode: the screen and pick kernels of the select, then the attend
+        self.launches_per_step = 3
 
     def select(self):
         i = self.inp
@@ -238,17 +240,16 @@ class DecodeBench:
                                      self.nsel, self.O, self.lse, workspace=self.ws_dec)
 
     def step(self):
-        self.select()
-        self.attend()
+        i = self.inp
+        self.hils.hils_decode(self.p, i["Qcal"], self.Ksum, self.Bsum, i["Q"], i["K"], i["V"], i["cache_len"],
+                              self.idx, self.score, self.nsel, self.O, self.lse, workspace=self.ws_step)
 
     def e2e_setup(self):
         i = self.inp
         self.h_in = {k: i[k].cpu().pin_memory() for k in ("Q", "Qcal", "cache_len")}
-        self.h_qpos = self.qpos.cpu().pin_memory()
         self.h_O = torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory()
         self.h_lse = torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in self.h_in.values()) + \
-            self.h_qpos.numel() * self.h_qpos.element_size()
+        h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
         d2h = self.h_O.numel() * self.h_O.element_size() + self.h_lse.numel() * self.h_lse.element_size()
         return h2d, d2h
 
@@ -256,7 +257,6 @@ class DecodeBench:
         i = self.inp
         for k, t in self.h_in.items():
             i[k].copy_(t, non_blocking=True)
-        self.qpos.copy_(self.h_qpos, non_blocking=True)
         self.step()
         self.h_O.copy_(self.O, non_blocking=True)
         self.h_lse.copy_(self.lse, non_blocking=True)
@@ -496,7 +496,7 @@ def main():
         for _ in range(args.warmup):
             db.step()
     stream.synchronize()
-    # one decode step = hils_select + hils_attend_decode, replayed as a CUDA graph
+    # one decode step = hils_decode (select, then attend, as one chain), replayed as a CUDA graph
     step_g = graphed(db.step, stream)
     sel_g = graphed(db.select, stream)
     att_g = graphed(db.attend, stream)
@@ -528,6 +528,7 @@ def main():
             db.e2e_step()
     per_e2e = time_steps(db.e2e_step, args.steps, flush, stream)
     ms_e2e = max_over_ranks(statistics.mean(per_e2e), world, dev)
+    launches = args.steps * db.launches_per_step
     del db
     torch.cuda.empty_cache()
 
@@ -579,7 +580,7 @@ def main():
                           "select_gbs": sel_gbs, "attend_gbs": att_gbs},
             "e2e": {"value": job_throughput(w.B, world, ms_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps * 2,
+            "gpu_launches": launches,
             "clocks": clk.summary(),
             "prefill": prefill,
             "cpu_baseline": cpu,

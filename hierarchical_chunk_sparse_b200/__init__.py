@@ -22,13 +22,13 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libhils.so")
 
 HILS_F32, HILS_BF16 = 0, 1
-HILS_CALL_SELECT, HILS_CALL_ATTEND_PREFILL, HILS_CALL_ATTEND_DECODE = 0, 1, 2
+HILS_CALL_SELECT, HILS_CALL_ATTEND_PREFILL, HILS_CALL_ATTEND_DECODE, HILS_CALL_DECODE = 0, 1, 2, 3
 STATUS = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARG", 2: "HILS_ERR_UNSUPPORTED",
           3: "HILS_ERR_ALIGNMENT", 4: "HILS_ERR_WORKSPACE", 5: "HILS_ERR_CUDA"}
 _DTYPES = {torch.float32: HILS_F32, torch.bfloat16: HILS_BF16}
 
 # Every function the C header declares (checked by the tests against the header).
-EXPORTS = ("hils_summarize", "hils_select", "hils_attend_prefill", "hils_attend_decode",
+EXPORTS = ("hils_summarize", "hils_select", "hils_attend_prefill", "hils_attend_decode", "hils_decode",
            "hils_attend_decode_noalloc", "hils_workspace_bytes", "hils_workspace_init",
            "hils_status_string", "hils_last_cuda_error")
 
@@ -68,13 +68,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hils_attend_prefill.argtypes = [P, T, T, T, i, vp, vp, vp, T, vp, vp, sz, vp]
         lib.hils_attend_decode.argtypes = [P, T, T, T, vp, vp, vp, vp, T, vp, vp, sz, vp]
         lib.hils_attend_decode_noalloc.argtypes = [P, T, T, T, vp, vp, vp, vp, T, vp, vp]
+        lib.hils_decode.argtypes = [P, T, T, vp, i, T, T, T, vp, vp, vp, vp, T, vp, vp, sz, vp]
         lib.hils_workspace_bytes.argtypes = [P, i, i, i]
         lib.hils_workspace_bytes.restype = sz
         lib.hils_workspace_init.argtypes = [vp, sz, vp]
         lib.hils_status_string.argtypes = [i]
         lib.hils_status_string.restype = ctypes.c_char_p
         lib.hils_last_cuda_error.restype = ctypes.c_char_p
-        for name in ("hils_summarize", "hils_select", "hils_attend_prefill", "hils_attend_decode",
+        for name in ("hils_summarize", "hils_select", "hils_attend_prefill", "hils_attend_decode", "hils_decode",
                      "hils_attend_decode_noalloc", "hils_workspace_init"):
             getattr(lib, name).restype = i
         _lib = lib
@@ -232,6 +233,31 @@ def hils_attend_decode(p: Params, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse
     _check("hils_attend_decode", load_library().hils_attend_decode(
         ctypes.byref(p.c()), _view(Q), _view(Kc), _view(Vc), _ptr(cache_len), _ptr(idx), _ptr(score),
         _ptr(nsel), _view(O), _ptr(lse), wp, wn, _stream(stream)))
+
+
+def hils_decode(p: Params, Qcal, Ksum, Bsum, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse=None,
+                workspace=None, stream=None) -> None:
+    """One decode step: hils_select with qpos = cache_len - 1, then hils_attend_decode,
+    as one chain. Outputs as the two calls: idx/score [B,H,1,K], nsel [B,H,1], O, lse."""
+    B, H, d, k = p.B, p.H, p.d, p.K
+    c = Ksum.shape[2]
+    _expect("hils_decode", "Qcal", Qcal, (B, H, 1, d), p.dtype)
+    _expect("hils_decode", "Ksum", Ksum, (B, H, c, d), p.dtype)
+    _expect("hils_decode", "Bsum", Bsum, (B, H, c), torch.float32)
+    _expect("hils_decode", "Q", Q, (B, H, 1, d), p.dtype)
+    _expect("hils_decode", "O", O, (B, H, 1, d), p.dtype)
+    for name, t in (("Kc", Kc), ("Vc", Vc)):
+        if t.shape[0] != B or t.shape[1] != H or t.shape[3] != d or t.dtype != p.dtype or not t.is_cuda:
+            raise ValueError(f"hils_decode: {name} has shape {tuple(t.shape)} / {t.dtype}")
+    _expect("hils_decode", "cache_len", cache_len, (B,), torch.int32)
+    _expect("hils_decode", "idx", idx, (B, H, 1, k), torch.int32)
+    _expect("hils_decode", "score", score, (B, H, 1, k), torch.float32)
+    _expect("hils_decode", "nsel", nsel, (B, H, 1), torch.int32)
+    _expect("hils_decode", "lse", lse, (B, H), torch.float32)
+    wp, wn = _ws(workspace)
+    _check("hils_decode", load_library().hils_decode(
+        ctypes.byref(p.c()), _view(Qcal), _view(Ksum), _ptr(Bsum), c, _view(Q), _view(Kc), _view(Vc),
+        _ptr(cache_len), _ptr(idx), _ptr(score), _ptr(nsel), _view(O), _ptr(lse), wp, wn, _stream(stream)))
 
 
 def hils_attend_decode_noalloc(p: Params, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse=None,

@@ -57,8 +57,8 @@ extern "C" int hils_attend_decode_noalloc(const hils_params *p, hils_ctensor Q, 
     if (need > 0) {
         const hils_status st = scratch_address(&scratch);
         if (st != HILS_OK) return st;
-        // the arrival counters at the front of the scratch must start at zero
-        const size_t counters = ((size_t)p->B * p->H * sizeof(int) + 255) & ~(size_t)255;
+        // the arrival counters and flags at the front of the scratch must start at zero
+        const size_t counters = attend_decode_counter_bytes(p->B * p->H);
         const hils_status mz = record_cuda_error(cudaMemsetAsync(scratch, 0, counters, stream));
         if (mz != HILS_OK) return mz;
     }

@@ -32,7 +32,7 @@ hils_status kernel_setup(KernelSetup &cache, const void *func, int threads, int 
         if (per_sm) *per_sm = cache.per_sm[dev];
         return HILS_OK;
     }
-    if (smem_bytes > 48 * 1024) {
+    if (smem_bytes > 0) {  // also needed when static + dynamic shared memory passes 48 KB
         e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
         if (e != cudaSuccess) return record_cuda_error(e);
     }
@@ -100,7 +100,7 @@ int decode_units(const hils_params *p) {
 }
 
 size_t select_ws_for(const hils_params *p, int Lq, int C) {
-    SelectArgs a;
+    SelectArgs a{};
     select_plan(p->dtype, p->d, p->B, p->H, Lq, C, p->K, true, device_sm_count(), &a);
     return select_ws_bytes(p->B * p->H * Lq, C, a.path);
 }
@@ -110,6 +110,79 @@ size_t select_ws_for(const hils_params *p, int Lq, int C) {
         const int _rc = (expr);        \
         if (_rc != HILS_OK) return _rc; \
     } while (0)
+
+
+int prepare_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *qpos, int qpos_bias,
+                   hils_ctensor Ksum, const float *Bsum, int C, int32_t *idx, float *score, int32_t *nsel,
+                   SelectArgs *a, int64_t *nq_out) {
+    float scale;
+    HILS_TRY(check_params(p, &scale));
+    if (Lq < 0 || C < 0) return HILS_ERR_INVALID_ARG;
+    const int64_t nq = (int64_t)p->B * p->H * Lq;
+    if (nq > 0x7fffffffll) return HILS_ERR_INVALID_ARG;  // query count fits in int
+    HILS_TRY(check_view(Qcal.ptr, Qcal.sb, Qcal.sh, Qcal.st, Lq, p));
+    HILS_TRY(check_view(Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st, C, p));
+    HILS_TRY(check_array(Bsum, (int64_t)p->B * p->H * C));
+    HILS_TRY(check_array(idx, nq * p->K));
+    HILS_TRY(check_array(score, nq * p->K));
+    HILS_TRY(check_array(nsel, nq));
+    if (qpos && ((uintptr_t)qpos & 3u)) return HILS_ERR_ALIGNMENT;
+    *nq_out = nq;
+    a->Qcal = {Qcal.ptr, Qcal.sb, Qcal.sh, Qcal.st};
+    a->Ksum = {Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st};
+    a->Bsum = Bsum;
+    a->qpos = qpos;
+    a->qpos_bias = qpos ? qpos_bias : 0;
+    a->idx = idx;
+    a->score = score;
+    a->nsel = nsel;
+    a->B = p->B;
+    a->H = p->H;
+    a->Lq = Lq;
+    a->C = C;
+    a->topk = p->K;
+    a->scale = scale;
+    if (nq > 0) select_plan(p->dtype, p->d, p->B, p->H, Lq, C, p->K, qpos != nullptr, device_sm_count(), a);
+    return HILS_OK;
+}
+
+int prepare_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hils_ctensor Vc,
+                          const int32_t *cache_len, const int32_t *idx, const float *score, const int32_t *nsel,
+                          hils_tensor O, float *lse, AttendArgs *a) {
+    float scale;
+    HILS_TRY(check_params(p, &scale));
+    const int64_t nq = (int64_t)p->B * p->H;
+    HILS_TRY(check_view(Q.ptr, Q.sb, Q.sh, Q.st, 1, p));
+    HILS_TRY(check_view(Kc.ptr, Kc.sb, Kc.sh, Kc.st, 1, p));
+    HILS_TRY(check_view(Vc.ptr, Vc.sb, Vc.sh, Vc.st, 1, p));
+    HILS_TRY(check_view(O.ptr, O.sb, O.sh, O.st, 1, p));
+    HILS_TRY(check_array(cache_len, p->B));
+    HILS_TRY(check_array(idx, nq * p->K));
+    HILS_TRY(check_array(score, nq * p->K));
+    HILS_TRY(check_array(nsel, p->K > 0 ? nq : 0));
+    HILS_TRY(check_array(lse, 0));
+    a->Q = {Q.ptr, Q.sb, Q.sh, Q.st};
+    a->K = {Kc.ptr, Kc.sb, Kc.sh, Kc.st};
+    a->V = {Vc.ptr, Vc.sb, Vc.sh, Vc.st};
+    a->O = {O.ptr, O.sb, O.sh, O.st};
+    a->lse = lse;
+    a->idx = idx;
+    a->score = score;
+    a->nsel = nsel;
+    a->qpos = nullptr;
+    a->cache_len = cache_len;
+    a->B = p->B;
+    a->H = p->H;
+    a->Lq = 1;
+    a->topk = p->K;
+    a->W = p->W;
+    a->scale = scale;
+    a->units = decode_units(p);
+    return HILS_OK;
+}
+
+// The select part of a hils_decode workspace, rounded so the attend part starts aligned.
+size_t decode_select_part(size_t select_bytes) { return (select_bytes + 255) & ~(size_t)255; }
 
 }  // namespace
 }  // namespace hils
@@ -139,6 +212,8 @@ size_t hils_workspace_bytes(const hils_params *p, int call, int Lq, int C) {
     case HILS_CALL_SELECT: return select_ws_for(p, Lq, C);
     case HILS_CALL_ATTEND_PREFILL: return kPrefillWsBytes;
     case HILS_CALL_ATTEND_DECODE: return attend_decode_ws_bytes(p->B * p->H, decode_units(p), p->d);
+    case HILS_CALL_DECODE:
+        return decode_select_part(select_ws_for(p, 1, C)) + attend_decode_ws_bytes(p->B * p->H, decode_units(p), p->d);
     default: return 0;
     }
 }
@@ -175,34 +250,10 @@ int hils_summarize(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ,
 int hils_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *qpos, hils_ctensor Ksum,
                 const float *Bsum, int C, int32_t *idx, float *score, int32_t *nsel, void *workspace,
                 size_t ws_bytes, cudaStream_t stream) {
-    float scale;
-    HILS_TRY(check_params(p, &scale));
-    if (Lq < 0 || C < 0) return HILS_ERR_INVALID_ARG;
-    const int64_t nq = (int64_t)p->B * p->H * Lq;
-    if (nq > 0x7fffffffll) return HILS_ERR_INVALID_ARG;  // query count fits in int
-    HILS_TRY(check_view(Qcal.ptr, Qcal.sb, Qcal.sh, Qcal.st, Lq, p));
-    HILS_TRY(check_view(Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st, C, p));
-    HILS_TRY(check_array(Bsum, (int64_t)p->B * p->H * C));
-    HILS_TRY(check_array(idx, nq * p->K));
-    HILS_TRY(check_array(score, nq * p->K));
-    HILS_TRY(check_array(nsel, nq));
-    if (qpos && ((uintptr_t)qpos & 3u)) return HILS_ERR_ALIGNMENT;
+    SelectArgs a{};
+    int64_t nq = 0;
+    HILS_TRY(prepare_select(p, Qcal, Lq, qpos, 0, Ksum, Bsum, C, idx, score, nsel, &a, &nq));
     if (nq == 0) return HILS_OK;
-    SelectArgs a;
-    a.Qcal = {Qcal.ptr, Qcal.sb, Qcal.sh, Qcal.st};
-    a.Ksum = {Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st};
-    a.Bsum = Bsum;
-    a.qpos = qpos;
-    a.idx = idx;
-    a.score = score;
-    a.nsel = nsel;
-    a.B = p->B;
-    a.H = p->H;
-    a.Lq = Lq;
-    a.C = C;
-    a.topk = p->K;
-    a.scale = scale;
-    select_plan(p->dtype, p->d, p->B, p->H, Lq, C, p->K, qpos != nullptr, device_sm_count(), &a);
     HILS_TRY(check_workspace(workspace, ws_bytes, select_ws_bytes((int)nq, C, a.path)));
     a.ws = workspace;
     return launch_select(p->dtype, p->d, a, stream);
@@ -225,7 +276,7 @@ int hils_attend_prefill(const hils_params *p, hils_ctensor Q, hils_ctensor K, hi
     HILS_TRY(check_array(lse, 0));
     HILS_TRY(check_workspace(workspace, ws_bytes, kPrefillWsBytes));
     if (nq == 0) return HILS_OK;
-    AttendArgs a;
+    AttendArgs a{};
     a.Q = {Q.ptr, Q.sb, Q.sh, Q.st};
     a.K = {K.ptr, K.sb, K.sh, K.st};
     a.V = {V.ptr, V.sb, V.sh, V.st};
@@ -252,41 +303,42 @@ int hils_attend_prefill(const hils_params *p, hils_ctensor Q, hils_ctensor K, hi
 int hils_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hils_ctensor Vc,
                        const int32_t *cache_len, const int32_t *idx, const float *score, const int32_t *nsel,
                        hils_tensor O, float *lse, void *workspace, size_t ws_bytes, cudaStream_t stream) {
-    float scale;
-    HILS_TRY(check_params(p, &scale));
+    AttendArgs a{};
+    HILS_TRY(prepare_attend_decode(p, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse, &a));
     const int64_t nq = (int64_t)p->B * p->H;
-    HILS_TRY(check_view(Q.ptr, Q.sb, Q.sh, Q.st, 1, p));
-    HILS_TRY(check_view(Kc.ptr, Kc.sb, Kc.sh, Kc.st, 1, p));
-    HILS_TRY(check_view(Vc.ptr, Vc.sb, Vc.sh, Vc.st, 1, p));
-    HILS_TRY(check_view(O.ptr, O.sb, O.sh, O.st, 1, p));
-    HILS_TRY(check_array(cache_len, p->B));
-    HILS_TRY(check_array(idx, nq * p->K));
-    HILS_TRY(check_array(score, nq * p->K));
-    HILS_TRY(check_array(nsel, p->K > 0 ? nq : 0));
-    HILS_TRY(check_array(lse, 0));
     if (nq == 0) return HILS_OK;
-    const int units = decode_units(p);
-    HILS_TRY(check_workspace(workspace, ws_bytes, attend_decode_ws_bytes((int)nq, units, p->d)));
-    AttendArgs a;
-    a.Q = {Q.ptr, Q.sb, Q.sh, Q.st};
-    a.K = {Kc.ptr, Kc.sb, Kc.sh, Kc.st};
-    a.V = {Vc.ptr, Vc.sb, Vc.sh, Vc.st};
-    a.O = {O.ptr, O.sb, O.sh, O.st};
-    a.lse = lse;
-    a.idx = idx;
-    a.score = score;
-    a.nsel = nsel;
-    a.qpos = nullptr;
-    a.cache_len = cache_len;
-    a.B = p->B;
-    a.H = p->H;
-    a.Lq = 1;
-    a.topk = p->K;
-    a.W = p->W;
-    a.scale = scale;
-    a.units = units;
+    HILS_TRY(check_workspace(workspace, ws_bytes, attend_decode_ws_bytes((int)nq, a.units, p->d)));
     a.ws = workspace;
     return launch_attend_decode(p->dtype, p->d, a, stream);
+}
+
+int hils_decode(const hils_params *p, hils_ctensor Qcal, hils_ctensor Ksum, const float *Bsum, int C,
+                hils_ctensor Q, hils_ctensor Kc, hils_ctensor Vc, const int32_t *cache_len, int32_t *idx,
+                float *score, int32_t *nsel, hils_tensor O, float *lse, void *workspace, size_t ws_bytes,
+                cudaStream_t stream) {
+    SelectArgs sa{};
+    int64_t nq = 0;
+    HILS_TRY(prepare_select(p, Qcal, 1, cache_len, -1, Ksum, Bsum, C, idx, score, nsel, &sa, &nq));
+    AttendArgs aa{};
+    HILS_TRY(prepare_attend_decode(p, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse, &aa));
+    if (nq == 0) return HILS_OK;
+    const size_t sel_bytes = decode_select_part(select_ws_bytes((int)nq, C, sa.path));
+    HILS_TRY(check_workspace(workspace, ws_bytes, sel_bytes + attend_decode_ws_bytes((int)nq, aa.units, p->d)));
+    sa.ws = workspace;
+    aa.ws = static_cast<uint8_t *>(workspace) + sel_bytes;
+    // the select's first kernel is an ordinary launch, so every earlier write on the
+    // stream is complete before it starts; the attend follows the select's last kernel,
+    // so its window tiles need not wait for the select
+    aa.window_early = 1;
+    if (decode_cluster_supported(p->B, p->H, C, p->K))  // one cluster per query: the whole step
+        return launch_decode_cluster(p->dtype, p->d, sa, aa, stream);
+    if (sa.path == kSelectSplit) {
+        // the attend's chunk units repeat the pick of their query themselves
+        HILS_TRY(launch_select_screen(p->dtype, p->d, sa, stream));
+        return launch_attend_decode_pick(p->dtype, p->d, aa, sa, stream);
+    }
+    HILS_TRY(launch_select(p->dtype, p->d, sa, stream));
+    return launch_attend_decode(p->dtype, p->d, aa, stream);
 }
 
 }  // extern "C"

@@ -1,0 +1,234 @@
+// One pipeline stage of the chunk screen (Eq. 7 of "Hierarchical Sparse Attention Done
+// Right" (picx.dev summary), with the rigorous radius of the exact selection): the
+// stage layout, the cooperative copies that fill it, and the screen of its rows on
+// tensor cores (bf16) or CUDA cores (float32). Shared by the decode select and the
+// clustered decode step.
+#pragma once
+#include "select_pick.cuh"
+
+namespace hils {
+namespace {
+
+__device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float r;
+    asm("sqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// Two adjacent elements of a 16-byte vector as a float pair.
+__device__ __forceinline__ float2 pair_of(const uint4 &v, int p, bf16) {
+    const uint32_t w = p == 0 ? v.x : p == 1 ? v.y : p == 2 ? v.z : v.w;
+    return make_float2(bf16lo(w), bf16hi(w));
+}
+__device__ __forceinline__ float2 pair_of(const uint4 &v, int p, float) {
+    return p == 0 ? make_float2(__uint_as_float(v.x), __uint_as_float(v.y))
+                  : make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+
+// v[i] holds this lane's partial for row i of its 2N-lane group. Each exchange step
+// (lane offset o = N, N/2, ..., 2) sends half of the rows a lane holds to its partner
+// and keeps the other half; a last butterfly step adds the pair (l, l^1). Afterwards
+// v[0] holds the group total of row (lane_in_group >> 1).
+template <int N>
+__device__ __forceinline__ void transpose_reduce(float (&v)[N], int lane_in_group) {
+#pragma unroll
+    for (int o = N; o >= 2; o /= 2) {
+        const bool upper = (lane_in_group & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o / 2; ++i) {
+            const float keep = upper ? v[i + o / 2] : v[i];
+            const float send = upper ? v[i] : v[i + o / 2];
+            v[i] = keep + __shfl_xor_sync(kFull, send, o);
+        }
+    }
+    v[0] += __shfl_xor_sync(kFull, v[0], 1);
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// Tensor-core screen of one stage (bf16): warp w takes rows 16w..16w+15. Per k-step one
+// ldmatrix.x4 of the 16x16 row tile A and three m16n8k16 MMAs: A times q (q in column 0
+// of B), and A times its own rows 0-7 and 8-15 (Gram blocks whose diagonals are |k'|^2;
+// the B fragments of those are A's own registers). Radius: the tensor-core float32
+// accumulation order and rounding are not specified, so the bound allows d * 2^-16 of
+// scale |q| |k'| (about 2^7 times the round-to-nearest bound), plus 2^-22 |s| for the
+// final fused multiply-add; |k'|^2 itself carries a 2^-8 margin.
+template <int D>
+__device__ void screen_stage_mma(const uint8_t *st, int q_off, int bias_off, float scale, int c0, int ne,
+                                 float2 *scr_row, float2 *slots) {
+    constexpr int kRowBytes = D * 2;
+    constexpr int kKSteps = D / 16;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    const int rbase = warp * 16;
+    const uint32_t *qw = reinterpret_cast<const uint32_t *>(st + q_off);
+    float qn2 = 0.f;
+    for (int pidx = lane; pidx < D / 2; pidx += 32) {
+        const uint32_t w = qw[pidx];
+        qn2 = fmaf(bf16lo(w), bf16lo(w), fmaf(bf16hi(w), bf16hi(w), qn2));
+    }
+    qn2 = warp_sum(qn2);
+    const int lrow = rbase + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const uint32_t row_addr = (uint32_t)__cvta_generic_to_shared(st + lrow * kRowBytes);
+    float dacc[4] = {0.f, 0.f, 0.f, 0.f}, g1[4] = {0.f, 0.f, 0.f, 0.f}, g2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < kKSteps; ++ks) {
+        uint32_t a[4];
+        const int unit = ks * 2 + (lane >> 4);
+        ldmatrix_x4(a, row_addr + (uint32_t)((unit ^ (lrow & 7)) * 16));
+        const uint32_t b0 = g == 0 ? qw[ks * 8 + tq] : 0u;
+        const uint32_t b1 = g == 0 ? qw[ks * 8 + 4 + tq] : 0u;
+        mma_bf16_16816(dacc, a, b0, b1);
+        mma_bf16_16816(g1, a, a[0], a[2]);
+        mma_bf16_16816(g2, a, a[1], a[3]);
+    }
+    // diagonal of the Gram blocks: row g in lane (g, g>>1), element (g & 1)
+    const float d1 = (g & 1) ? g1[1] : g1[0];
+    const float d2 = (g & 1) ? g2[3] : g2[2];
+    const int src = g * 4 + (g >> 1);
+    const float k1 = __shfl_sync(kFull, d1, src);
+    const float k2 = __shfl_sync(kFull, d2, src);
+    const float *bias = reinterpret_cast<const float *>(st + bias_off);
+    const float ecoef = scale * sqrt_approx(qn2) * ((float)D * 0x1p-16f) * (1.f + 0x1p-8f);
+    float ms = -INFINITY, me = 0.f;
+    if (tq == 0) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int row = rbase + g + 8 * h;
+            const int c = c0 + row;
+            const float dot = h ? dacc[2] : dacc[0];
+            const float sv = fmaf(dot, scale, bias[row]);
+            const float ev = fmaf(ecoef, sqrt_approx(h ? k2 : k1), fabsf(sv) * 0x1p-22f);
+            if (c < ne) {
+                scr_row[c] = make_float2(sv, ev);
+                ms = fmaxf(ms, sv);
+                me = fmaxf(me, ev);
+            }
+        }
+    }
+    ms = warp_max(ms);
+    me = warp_max(me);
+    if (lane == 0) slots[warp] = make_float2(ms, me);
+}
+
+// Float32 screen of one stage on CUDA cores (all threads): kTPR threads share a row
+// (one 16-byte unit each), each accumulates its unit's partial dot and |k|^2 for kRPT
+// rows with packed float32 FMAs, and a transpose reduction across the kTPR lanes
+// leaves each lane the totals of one row.
+template <typename T, int D, typename Cfg>
+__device__ void screen_stage_f32(const uint8_t *st, float scale, int c0, int ne, float2 *scr_row, float2 *gscr) {
+    constexpr int kN = Vec<T>::kN;
+    const int tid = threadIdx.x, col = tid % Cfg::kTPR, rg = tid / Cfg::kTPR;
+    // query slice of this thread's unit as float pairs, and |q|^2
+    const uint4 qv = *reinterpret_cast<const uint4 *>(st + Cfg::kQOff + col * 16);
+    float2 q2[kN / 2];
+    float qn2 = 0.f;
+#pragma unroll
+    for (int p = 0; p < kN / 2; ++p) {
+        q2[p] = pair_of(qv, p, T());
+        qn2 = fmaf(q2[p].x, q2[p].x, fmaf(q2[p].y, q2[p].y, qn2));
+    }
+#pragma unroll
+    for (int o = Cfg::kTPR / 2; o > 0; o >>= 1) qn2 += __shfl_xor_sync(kFull, qn2, o);
+    float dotv[Cfg::kRPT], ksqv[Cfg::kRPT];
+#pragma unroll
+    for (int r = 0; r < Cfg::kRPT; ++r) {
+        const uint4 kv = *reinterpret_cast<const uint4 *>(st + (rg * Cfg::kRPT + r) * Cfg::kRowBytes + col * 16);
+        float2 d2 = make_float2(0.f, 0.f), k2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int p = 0; p < kN / 2; ++p) {
+            const float2 kf = pair_of(kv, p, T());
+            d2 = __ffma2_rn(q2[p], kf, d2);
+            k2 = __ffma2_rn(kf, kf, k2);
+        }
+        dotv[r] = d2.x + d2.y;
+        ksqv[r] = k2.x + k2.y;
+    }
+    transpose_reduce<Cfg::kRPT>(dotv, col);
+    transpose_reduce<Cfg::kRPT>(ksqv, col);
+    const int row = rg * Cfg::kRPT + (col >> 1);
+    const int c = c0 + row;
+    const bool valid = c < ne;
+    const float ecoef = scale * sqrtf(qn2) * ((float)(D + 2) * 0x1p-23f);
+    const float sv = fmaf(dotv[0], scale, reinterpret_cast<const float *>(st + Cfg::kBiasOff)[row]);
+    const float ev = fmaf(ecoef, sqrt_approx(ksqv[0]), fabsf(sv) * 0x1p-22f);
+    if (valid && (col & 1) == 0) scr_row[c] = make_float2(sv, ev);
+    float gs = valid ? sv : -INFINITY, ge = valid ? ev : 0.f;
+#pragma unroll
+    for (int o = Cfg::kTPR / 2; o > 0; o >>= 1) {
+        gs = fmaxf(gs, __shfl_xor_sync(kFull, gs, o));
+        ge = fmaxf(ge, __shfl_xor_sync(kFull, ge, o));
+    }
+    if (col == 0) gscr[rg] = make_float2(gs, ge);
+}
+
+// Layout of one pipeline stage of ROWS summary rows screened by NT threads: the rows
+// (16-byte units of bf16 rows permuted by (unit ^ (row & 7))), their biases, the query
+// row and the query's position.
+template <typename T, int D, int NT, int ROWS>
+struct StageCfg {
+    static constexpr int kThreads = NT;
+    static constexpr int kRows = ROWS;
+    static constexpr int kRowBytes = D * (int)sizeof(T);
+    static constexpr int kTPR = kRowBytes / 16;     // threads per row: 8, 16 or 32
+    static constexpr int kRowGroups = NT / kTPR;    // rows per step
+    static constexpr int kRPT = ROWS / kRowGroups;  // rows per thread
+    static constexpr int kBiasOff = ROWS * kRowBytes;
+    static constexpr int kQOff = kBiasOff + ROWS * 4;
+    static constexpr int kPosOff = kQOff + kRowBytes;
+    static constexpr int kStageBytes = kPosOff + 16;
+    static constexpr int kGroupsPerBlock = ROWS / kGroupRows;
+    static constexpr int kCopies = ROWS * kTPR / NT;  // 16-byte copies per thread
+    static_assert(2 * kRPT == kTPR, "half-square transpose reduction");
+    // bf16 tables are screened on tensor cores (16 rows per warp, swizzled shared rows);
+    // float32 tables on CUDA cores (kRPT rows per thread group).
+    static constexpr bool kMma = sizeof(T) == 2;
+    static_assert(!kMma || ROWS == 16 * (NT / 32), "tensor-core screen: 16 rows per warp");
+    static constexpr int kSlotRows = kMma ? 16 : kRPT;
+    static constexpr int kSlots = ROWS / kSlotRows;
+    static constexpr int kSlotsPerGroup = kGroupRows / kSlotRows;
+};
+
+// Every thread issues its share of the cp.async copies of one stage: `rows` summary
+// rows from `kh` (row stride kst elements) starting at chunk c0, their biases, the query
+// row, and the position (from `pos` if not null, else the value `pos_value`).
+template <typename T, typename Cfg>
+__device__ __forceinline__ void stage_issue(uint8_t *st, const T *kh, int64_t kst, int c0, int rows, const float *brow,
+                                            const T *qrow, const int32_t *pos, int pos_value) {
+    const int tid = threadIdx.x, col = tid % Cfg::kTPR;
+    const int r0 = tid / Cfg::kTPR;
+    const uint8_t *src = reinterpret_cast<const uint8_t *>(kh + (int64_t)(c0 + r0) * kst) + col * 16;
+    const int dcol = Cfg::kMma ? (col ^ (r0 & 7)) : col;
+    uint8_t *dst = st + r0 * Cfg::kRowBytes + dcol * 16;
+    constexpr int kStep = Cfg::kThreads / Cfg::kTPR;
+    const int64_t src_step = (int64_t)kStep * kst * (int64_t)sizeof(T);
+#pragma unroll
+    for (int k = 0; k < Cfg::kCopies; ++k)
+        if (r0 + k * kStep < rows) cp_async16(dst + k * kStep * Cfg::kRowBytes, src + k * src_step);
+    for (int r = tid; r < rows; r += Cfg::kThreads) cp_async4(st + Cfg::kBiasOff + r * 4, brow + r);
+    for (int u = tid; u < Cfg::kTPR; u += Cfg::kThreads)
+        cp_async16(st + Cfg::kQOff + u * 16, reinterpret_cast<const uint8_t *>(qrow) + u * 16);
+    if (tid == 0) {
+        if (pos) cp_async4(st + Cfg::kPosOff, pos);
+        else *reinterpret_cast<int *>(st + Cfg::kPosOff) = pos_value;
+    }
+}
+
+}  // namespace
+}  // namespace hils

@@ -19,8 +19,8 @@
 namespace hils {
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
+constexpr int kWarpKernelWarps = 8;  // warps (queries) per CTA of the warp-per-query select
+constexpr int kWarpKernelThreads = kWarpKernelWarps * 32;
 constexpr int kTile = 128;      // chunks scored per warp step
 constexpr int kMaxK = 32;
 constexpr int kListBytes = 768; // one list of <= 32 entries in the workspace
@@ -309,7 +309,7 @@ __device__ __forceinline__ QueryCtx make_ctx(const SelectArgs &a, int64_t qi, in
     const int bh = q32 / a.Lq;
     const int h = bh % a.H;
     const int b = bh / a.H;
-    t = a.qpos ? a.qpos[(int64_t)b * a.Lq + i] : i;
+    t = a.qpos ? a.qpos[(int64_t)b * a.Lq + i] + a.qpos_bias : i;
     QueryCtx q;
     q.qrow = static_cast<const T *>(a.Qcal.ptr) + b * a.Qcal.sb + h * a.Qcal.sh + i * a.Qcal.st;
     q.khead = static_cast<const T *>(a.Ksum.ptr) + b * a.Ksum.sb + h * a.Ksum.sh;

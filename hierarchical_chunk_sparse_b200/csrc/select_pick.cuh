@@ -1,0 +1,256 @@
+// Exact top-K pick of one decode query from the screen values of the decode select
+// ("Hierarchical Sparse Attention Done Right" (picx.dev summary), Eq. 7 and
+// Methodology 2; rcap.io post, pseudocode figure). Shared by the select's pick kernel
+// and the decode attend, whose chunk units repeat the (deterministic) pick of their
+// query instead of waiting for a separate kernel.
+//
+// Workspace of the decode select: a 256-byte status header, then the screen value and
+// radius (s_c, e_c) of every eligible chunk per query, then the largest s and e of every
+// 64-chunk group per query.
+#pragma once
+#include "select_common.cuh"
+
+namespace hils {
+namespace {
+
+constexpr int kGroupRows = 64;  // rows per group maximum
+constexpr int kMaxDecC = 16384; // table rows per query on this path
+constexpr int kMaxGroups = kMaxDecC / kGroupRows;  // 256
+constexpr int kPoolCap = 64;
+
+// Staging area for the candidate pool.
+struct Pool64 {
+    double x[kPoolCap];
+    int idx[kPoolCap];
+    float s[kPoolCap];
+    float e[kPoolCap];
+};
+
+
+
+// (K+1)-th largest of the first values of v[0..n) (duplicates counted) by parallel
+// ranks: value i has rank #{j: v_j > v_i} + #{j < i: v_j = v_i}, unique, and the one
+// with rank K is the answer (n > K; all NT threads call; the result in *out).
+template <int NT>
+__device__ void block_kth_plus_one(const float2 *v, int n, int K, float *out) {
+    for (int i = threadIdx.x; i < n; i += NT) {
+        const unsigned ki = ordered_key(v[i].x);
+        int rank = 0;
+        for (int j = 0; j < n; ++j) {
+            const unsigned kj = ordered_key(v[j].x);
+            rank += (kj > ki || (kj == ki && j < i)) ? 1 : 0;
+        }
+        if (rank == K) *out = v[i].x;
+    }
+}
+
+// The float32 screen value and tight radius of every pool entry on CUDA cores, four
+// threads per entry (a quarter of the row each, then two shuffle steps). Any order of
+// the float32 sums stays within the radius scale sum|q k| (d+2) 2^-23 + |s| 2^-22.
+template <typename T, int D, int NT>
+__device__ void rescreen_pool(const QueryCtx &q, const float *qs, Pool64 &pool, int total) {
+    constexpr int kN = Vec<T>::kN, kQuarter = D / 4;
+    const int tid = threadIdx.x, sub = tid & 3;
+    for (int base = 0; base < total; base += NT / 4) {  // the same trip count in every lane
+        const int j = base + (tid >> 2);
+        const bool ok = j < total;
+        float dot = 0.f, ad = 0.f;
+        int c = 0;
+        if (ok) {
+            c = pool.idx[j];
+            const uint4 *kr = reinterpret_cast<const uint4 *>(static_cast<const T *>(q.khead) + (int64_t)c * q.kst +
+                                                              sub * kQuarter);
+#pragma unroll
+            for (int u = 0; u < kQuarter / kN; ++u) {
+                float kf[kN];
+                widen(__ldg(kr + u), kf, T());
+#pragma unroll
+                for (int i = 0; i < kN; ++i) {
+                    const float qv = qs[sub * kQuarter + u * kN + i];
+                    dot = fmaf(qv, kf[i], dot);
+                    ad = fmaf(fabsf(qv), fabsf(kf[i]), ad);
+                }
+            }
+        }
+        dot += __shfl_xor_sync(kFull, dot, 1);
+        ad += __shfl_xor_sync(kFull, ad, 1);
+        dot += __shfl_xor_sync(kFull, dot, 2);
+        ad += __shfl_xor_sync(kFull, ad, 2);
+        if (ok && sub == 0) {
+            const float s = fmaf(dot, q.scale, q.bhead[c]);
+            pool.s[j] = s;
+            pool.e[j] = fmaf(q.scale * ad, (float)(D + 2) * 0x1p-23f, fabsf(s) * 0x1p-22f);
+        }
+    }
+}
+
+struct PickSmem {
+    float qs[128];
+    float2 gm[kMaxGroups];
+    uint16_t cand_g[kMaxGroups];
+    Pool64 pool;
+    EntryList out;
+    float wmax[8];  // one per warp of the picking CTA
+    float cut, tk;
+    int ncg, pool_n;
+};
+
+struct ScreenWs {
+    float2 *scr;   // [queries][C]
+    float2 *gmax;  // [queries][ceil(C/64)]
+};
+
+__host__ __device__ __forceinline__ int groups_of(int C) { return (C + kGroupRows - 1) / kGroupRows; }
+
+__host__ __device__ __forceinline__ size_t dec_ws_bytes(int64_t queries, int C) {
+    const size_t scr = (size_t)queries * (C + groups_of(C)) * sizeof(float2);
+    return kSelectStatusBytes + scr;
+}
+
+__device__ __forceinline__ ScreenWs screen_ws(const SelectArgs &a) {
+    const int64_t nq = (int64_t)a.B * a.H * a.Lq;
+    ScreenWs w;
+    w.scr = reinterpret_cast<float2 *>(static_cast<uint8_t *>(a.ws) + kSelectStatusBytes);
+    w.gmax = w.scr + nq * a.C;
+    return w;
+}
+
+// Exact top-K of one query from the screen values in the workspace (all NT threads of
+// a CTA, NT <= 256; every step below is one parallel round trip to L2).
+template <typename T, int D, int NT>
+__device__ void pick_query(const SelectArgs &a, const ScreenWs &ws, int64_t qi, PickSmem &ps) {
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    int t;
+    const QueryCtx q = make_ctx<T, D>(a, qi, t);
+    for (int x = tid; x < D; x += NT) ps.qs[x] = (float)static_cast<const T *>(q.qrow)[x];
+    const int ne = eligible(t, a.C);
+    const int K = a.topk;
+    const float2 *scr = ws.scr + qi * a.C;
+    if (ne <= K) {  // every eligible chunk is kept, in index order
+        for (int r = tid; r < K; r += NT) {
+            a.idx[qi * K + r] = r < ne ? r : -1;
+            a.score[qi * K + r] = r < ne ? __ldcg(&scr[r]).x : -INFINITY;
+        }
+        if (tid == 0) a.nsel[qi] = ne;
+        return;
+    }
+    const int G = groups_of(ne);
+    __syncthreads();  // ps.qs complete
+    if (G < K + 1) {  // short table: the exact running-list scan over every chunk
+        if (w == 0) {
+            warp_scan<T, D>(q, ps.qs, 0, ne, K, ps.out);
+            warp_write(ps.out, K, qi, a.idx, a.score, a.nsel);
+        }
+        return;
+    }
+    // T = (K+1)-th largest maximum of the 64-chunk groups (attained by K+1 distinct
+    // chunks); e_max = largest radius; every chunk with hi < T - e_max is certainly out
+    const float2 *gmx = ws.gmax + qi * groups_of(a.C);
+    float em = 0.f;
+    for (int g = tid; g < G; g += NT) {
+        const float2 v = __ldcg(&gmx[g]);
+        ps.gm[g] = v;
+        em = fmaxf(em, v.y);
+    }
+    em = warp_max(em);
+    if (tid == 0) {
+        ps.ncg = 0;
+        ps.pool_n = 0;
+    }
+    if (lane == 0) ps.wmax[w] = em;
+    __syncthreads();
+    block_kth_plus_one<NT>(ps.gm, G, K, &ps.tk);
+    __syncthreads();
+    if (tid == 0) {
+        float e2 = 0.f;
+        for (int k = 0; k < NT / 32; ++k) e2 = fmaxf(e2, ps.wmax[k]);
+        ps.cut = __fsub_rd(ps.tk, e2);
+    }
+    __syncthreads();
+    const float cut = ps.cut;
+    // candidate groups: their max s + max e can reach the cut
+    for (int g = tid; g < G; g += NT)
+        if (__fadd_ru(ps.gm[g].x, ps.gm[g].y) >= cut) ps.cand_g[atomicAdd(&ps.ncg, 1)] = (uint16_t)g;
+    __syncthreads();
+    const int ncg = ps.ncg;
+    // their chunks with hi >= cut join the pool: warp w scans candidate groups w, w+8, ...
+    for (int k0 = w; k0 < ncg; k0 += 2 * (NT / 32)) {
+        float2 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int k = k0 + (j >> 1) * (NT / 32);
+            const int c = k < ncg ? ps.cand_g[k] * kGroupRows + (j & 1) * 32 + lane : ne;
+            v[j] = c < ne ? __ldcg(&scr[c]) : make_float2(-INFINITY, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (v[j].x != -INFINITY && __fadd_ru(v[j].x, v[j].y) >= cut) {
+                const int k = k0 + (j >> 1) * (NT / 32);
+                const int pos = atomicAdd(&ps.pool_n, 1);
+                if (pos < kPoolCap) {
+                    ps.pool.idx[pos] = ps.cand_g[k] * kGroupRows + (j & 1) * 32 + lane;
+                    ps.pool.s[pos] = v[j].x;
+                    ps.pool.e[pos] = v[j].y;
+                    ps.pool.x[pos] = __longlong_as_double(0x7ff8000000000000ll);
+                }
+            }
+        }
+    }
+    __syncthreads();  // every candidate is in the pool before any thread reads it
+    const int total = ps.pool_n;
+    if (total <= kPoolCap) {
+        // the candidates are screened again on CUDA cores (round-to-nearest fused
+        // multiply-adds: the tight radius), so that few need the float64 score
+        rescreen_pool<T, D, NT>(q, ps.qs, ps.pool, total);
+        __syncthreads();
+        if (w == 0) {
+            Slots<2> sl;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int j = lane + 32 * r;
+                const bool ok = j < total;
+                sl.idx[r] = ok ? ps.pool.idx[j] : -1;
+                sl.s[r] = ok ? ps.pool.s[j] : 0.f;
+                sl.e[r] = ok ? ps.pool.e[j] : 0.f;
+                sl.x[r] = ok ? ps.pool.x[j] : 0.0;
+            }
+            float bnd;
+            const unsigned keep = warp_topk<T, D, 2>(sl, K, q, bnd);
+            __syncwarp();
+            const int n = warp_append<2>(sl, keep, ps.out, 0);
+            if (lane == 0) ps.out.n = n;
+            __syncwarp();
+            warp_write(ps.out, K, qi, a.idx, a.score, a.nsel);
+        }
+        return;
+    }
+    if (w != 0) return;
+    // heavy ties: fold the candidates in index order, 32 at a time (slot 0 = running list)
+    int n = 0;
+    for (int c0 = 0; c0 < ne; c0 += 32) {
+        const int c = c0 + lane;
+        const float2 v = c < ne ? __ldcg(&scr[c]) : make_float2(-INFINITY, 0.f);
+        const bool cand = c < ne && __fadd_ru(v.x, v.y) >= cut;
+        if (!__any_sync(kFull, cand)) continue;
+        Slots<2> sl;
+        sl.idx[0] = lane < n ? ps.out.idx[lane] : -1;
+        sl.s[0] = lane < n ? ps.out.s[lane] : 0.f;
+        sl.e[0] = lane < n ? ps.out.e[lane] : 0.f;
+        sl.x[0] = lane < n ? ps.out.x[lane] : 0.0;
+        sl.idx[1] = cand ? c : -1;
+        sl.s[1] = v.x;
+        sl.e[1] = v.y;
+        sl.x[1] = __longlong_as_double(0x7ff8000000000000ll);
+        float bnd;
+        const unsigned keep = warp_topk<T, D, 2>(sl, K, q, bnd);
+        __syncwarp();
+        n = warp_append<2>(sl, keep, ps.out, 0);
+        __syncwarp();
+    }
+    if (lane == 0) ps.out.n = n;
+    __syncwarp();
+    warp_write(ps.out, K, qi, a.idx, a.score, a.nsel);
+}
+
+}  // namespace
+}  // namespace hils

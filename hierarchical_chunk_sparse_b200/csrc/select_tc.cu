@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
     const int i = i0 + tid;
     const bool row_ok = i < a.Lq;
     int t = -1;
-    if (row_ok) t = a.qpos ? a.qpos[(int64_t)b * a.Lq + i] : i;
+    if (row_ok) t = a.qpos ? a.qpos[(int64_t)b * a.Lq + i] + a.qpos_bias : i;
     const int ne = row_ok ? eligible(t, a.C) : 0;
     if (tid == 0) {
         misc->nc = 0;

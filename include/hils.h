@@ -105,7 +105,8 @@ typedef struct {
 typedef enum {
     HILS_CALL_SELECT = 0,
     HILS_CALL_ATTEND_PREFILL = 1,
-    HILS_CALL_ATTEND_DECODE = 2
+    HILS_CALL_ATTEND_DECODE = 2,
+    HILS_CALL_DECODE = 3
 } hils_call;
 
 /* Landmark chunk summaries (summary page, Methodology 1, Eq. 8).
@@ -182,6 +183,26 @@ int hils_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hi
                        const int32_t *idx, const float *score, const int32_t *nsel,
                        hils_tensor O, float *lse, void *workspace, size_t ws_bytes,
                        cudaStream_t stream);
+
+/* One decode step: hils_select with qpos = cache_len - 1 (Lq = 1), then
+ * hils_attend_decode on its outputs, enqueued as one chain on `stream` (the same
+ * passages as the two calls). Results are those of the two calls made in turn: the
+ * same kept chunks and scores (idx, score, nsel), and O and lse within rounding of
+ * hils_attend_decode's.
+ * With B*H >= 16 and C <= 8192 each query runs in one cluster of 8 CTAs that screens,
+ * selects and attends without leaving the cluster (distributed shared memory).
+ * Inside the chain the attend's window tiles need not wait for the select: its first
+ * kernel starts only after all earlier work on the stream, so the window overlaps the
+ * chunk selection.
+ *   Qcal [B, H, 1, d]; Ksum [B, H, C, d]; Bsum [B, H, C]; C summarised chunks
+ *   Q, Kc, Vc, cache_len, O, lse: as for hils_attend_decode
+ *   idx, score [B, H, 1, K], nsel [B, H, 1]: out
+ *   workspace, ws_bytes: hils_workspace_bytes(p, HILS_CALL_DECODE, 1, C) bytes, zeroed
+ *         before first use (the select part first, then the attend part). */
+int hils_decode(const hils_params *p, hils_ctensor Qcal, hils_ctensor Ksum, const float *Bsum, int C,
+                hils_ctensor Q, hils_ctensor Kc, hils_ctensor Vc, const int32_t *cache_len,
+                int32_t *idx, float *score, int32_t *nsel, hils_tensor O, float *lse,
+                void *workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* hils_attend_decode without a workspace argument: the library keeps the scratch
  * memory itself, in one fixed 4 MiB array of device global memory that every GPU

@@ -119,6 +119,26 @@ def test_decode_workspace_too_small(lib):
     assert rc == 4
 
 
+def test_decode_chain_workspace_and_validation(lib):
+    p = _p(B=1, H=2)
+    c = p.c()
+    sel = lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_SELECT, 1, 8000)
+    att = lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_ATTEND_DECODE, 1, 0)
+    need = lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_DECODE, 1, 8000)
+    assert need == (sel + 255) // 256 * 256 + att  # select part, aligned, then the attend part
+    v = T(ALIGNED, 256, 128, 128)
+    args = [ctypes.byref(c), v, T(ALIGNED, 0, 0, 128), ALIGNED, 8000, v, v, v, ALIGNED, ALIGNED, ALIGNED, ALIGNED,
+            v, None]
+    assert lib.hils_decode(*args, ALIGNED, need - 1, None) == 4
+    assert lib.hils_decode(*args, None, need, None) == 4
+    bad = list(args)
+    bad[8] = None  # cache_len
+    assert lib.hils_decode(*bad, ALIGNED, need, None) == 1
+    bad = list(args)
+    bad[4] = -1  # C
+    assert lib.hils_decode(*bad, ALIGNED, need, None) == 1
+
+
 def test_workspace_sizes(lib):
     assert lib.hils_workspace_bytes(None, 0, 1, 1) == 0
     assert lib.hils_workspace_bytes(ctypes.byref(_p(d=80).c()), 0, 1, 1) == 0

@@ -439,6 +439,90 @@ def test_end_to_end_against_chained_oracle(oracle, cuda_device, case):
 
 # ------------------------------------------------------------------ full sizes
 
+def _decode_chain(w, d, Ksum, Bsum, ws=None):
+    p = P(w)
+    B, H = w.B, w.H
+    idx = torch.full((B, H, 1, w.K), 7777, dtype=torch.int32, device=Ksum.device)
+    score = torch.full((B, H, 1, w.K), 7777.0, device=Ksum.device)
+    nsel = torch.full((B, H, 1), 7777, dtype=torch.int32, device=Ksum.device)
+    O = torch.full_like(d["Q"], 99.0)
+    lse = torch.full((B, H), 99.0, device=Ksum.device)
+    if ws is None:
+        ws = hils.alloc_workspace(p, hils.HILS_CALL_DECODE, 1, Ksum.shape[2], device=Ksum.device)
+    hils.hils_decode(p, d["Qcal"], Ksum, Bsum, d["Q"], d["K"], d["V"], d["cache_len"], idx, score, nsel, O, lse,
+                     workspace=ws)
+    assert int(host(ws[:4]).view(torch.int32)[0]) == 0, "a bounded wait expired"
+    return idx, score, nsel, O, lse, ws
+
+
+@pytest.mark.parametrize("case", ["small16", "small6", "full"])
+def test_decode_chain_equals_separate_calls(oracle, cuda_device, case):
+    """hils_decode (one cluster of CTAs per query for B*H >= 16, else the select and
+    attend as one chain) keeps exactly the chunks and scores of hils_select and gives
+    the outputs of hils_attend_decode within the output tolerance; the small case is
+    also checked against the oracle, and every case runs twice on one workspace."""
+    full = case == "full"
+    if full:
+        w = WORKLOADS[4]
+        d = make_decode(w, device=cuda_device)
+    else:
+        w, inp = _decode_small(cuda_device, lens=(12001, 9000), H=8 if case == "small16" else 3)
+        d = to_dev(inp, cuda_device)
+    Ksum, Bsum = gpu_summarize(w, d["K"], d["LQ"])
+    qpos = (d["cache_len"] - 1).reshape(w.B, 1).contiguous()
+    i1, s1, n1 = gpu_select(w, d["Qcal"], Ksum, Bsum, qpos=qpos)
+    O1, l1 = gpu_decode(w, d["Q"], d["K"], d["V"], d["cache_len"], i1, s1, n1)
+    ws = None
+    for rep in range(2):
+        i2, s2, n2, O2, l2, ws = _decode_chain(w, d, Ksum, Bsum, ws)
+        assert torch.equal(i1, i2) and torch.equal(n1, n2) and torch.equal(s1, s2), f"selection rep {rep}"
+        assert_close(O2, host(O1).double().numpy(), w.dtype, f"O rep {rep}")
+        assert np.abs(host(l2).double().numpy() - host(l1).double().numpy()).max() <= 1e-4, f"lse rep {rep}"
+    if not full:
+        i_ref, _, n_ref = oracle.select(inp["Qcal"], host(Ksum), host(Bsum), 64, w.K, w.scale, qpos=host(qpos))
+        assert_same_selection(i2, n2, i_ref, n_ref)
+        O_ref, lse_ref = oracle.attend(inp["Q"], inp["K"], inp["V"], host(i2), host(s2), host(n2), 64, w.W,
+                                       w.scale, qpos=host(qpos))
+        assert_close(O2, O_ref, w.dtype, "O")
+        assert_close(l2, lse_ref[:, :, 0], torch.float32, "lse")
+    del d
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("lens,K,W,d,dtype", [
+    ((1, 65, 700, 12001), 16, 512, 128, torch.bfloat16),   # no chunk, all kept, short table, long
+    ((3000, 70000, 9000, 64 * 1000), 32, 1024, 128, torch.bfloat16),
+    ((5000, 12345, 64, 8000), 8, 0, 128, torch.bfloat16),  # no window
+    ((4000, 9001, 20000, 130), 16, 300, 64, torch.bfloat16),
+    ((3000, 9001, 700, 6000), 16, 512, 128, torch.float32),
+])
+def test_decode_cluster_edges(oracle, cuda_device, lens, K, W, d, dtype):
+    """hils_decode with B*H = 16 queries (one cluster each) against the oracle and the
+    separate calls: empty tables, tables of at most K chunks, fewer than K+1 groups, no
+    window, K = 32, d = 64 and float32."""
+    w = WORKLOADS[4].replace(B=len(lens), H=4, N=max(lens), K=K, W=W, d=d, dtype=dtype, needles=0)
+    inp = make_decode(w)
+    inp["cache_len"] = torch.tensor(lens, dtype=torch.int32)
+    dv = to_dev(inp, cuda_device)
+    Ksum, Bsum = gpu_summarize(w, dv["K"], dv["LQ"])
+    qpos = (dv["cache_len"] - 1).reshape(w.B, 1).contiguous()
+    i1, s1, n1 = gpu_select(w, dv["Qcal"], Ksum, Bsum, qpos=qpos)
+    O1, l1 = gpu_decode(w, dv["Q"], dv["K"], dv["V"], dv["cache_len"], i1, s1, n1)
+    i2, s2, n2, O2, l2, _ = _decode_chain(w, dv, Ksum, Bsum)
+    assert torch.equal(i1, i2) and torch.equal(n1, n2) and torch.equal(s1, s2)
+    i_ref, s_ref, n_ref = oracle.select(inp["Qcal"], host(Ksum), host(Bsum), 64, K, w.scale, qpos=host(qpos))
+    assert_same_selection(i2, n2, i_ref, n_ref)
+    scores_close(s2, s_ref, n_ref, "hils_decode scores")
+    O_ref, lse_ref = oracle.attend(inp["Q"], inp["K"], inp["V"], host(i2), host(s2), host(n2), 64, W, w.scale,
+                                   qpos=host(qpos))
+    assert_close(O2, O_ref, dtype, "O")
+    fin = np.isfinite(lse_ref[:, :, 0])
+    l2h = host(l2).double().numpy()
+    assert (np.isfinite(l2h) == fin).all()
+    assert np.abs(l2h[fin] - lse_ref[:, :, 0][fin]).max() <= 1e-4
+    assert_close(O2, host(O1).double().numpy(), dtype, "O vs separate calls")
+
+
 @pytest.mark.parametrize("cfg", [3, 4, 5])
 def test_decode_workload_full_size(oracle, cuda_device, cfg):
     """Decode workloads at full size, generated on the GPU: summaries sampled, the
