@@ -19,13 +19,12 @@
 // a separate tensor-core kernel.
 #include <math.h>
 
-#include "select_pick.cuh"
+#include "hils_internal.cuh"
 
 namespace hils {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kFlagWaitIters = 256;  // a chunk unit's wait for its query's pick (128 ns sleeps)
 
 template <typename T, int D>
 struct UnitCfg {
@@ -201,7 +200,6 @@ __device__ __forceinline__ UnitPlan plan_unit_loaded(int u, int t, int K, int W,
 
 struct DecodeWs {
     int *counters;  // [queries] units arrived
-    int *flags;     // [queries] the query's kept list is published (hils_decode chain)
     float *mass;
     float *vec;
 };
@@ -212,7 +210,6 @@ __device__ __forceinline__ DecodeWs decode_ws(void *ws, int queries, int units, 
     DecodeWs w;
     uint8_t *p = static_cast<uint8_t *>(ws);
     w.counters = reinterpret_cast<int *>(p);
-    w.flags = w.counters + queries;
     p += attend_decode_counter_bytes(queries);
     w.mass = reinterpret_cast<float *>(p);
     p += align256((size_t)queries * units * sizeof(float));
@@ -327,80 +324,6 @@ __global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
     if (threadIdx.x == 0) ws.counters[qi] = 0;
 }
 
-// hils_decode's attend, dependent-launched after the decode select's screen kernel.
-// Grid (B*H, units): blockIdx.x is the query, blockIdx.y runs over the window tiles
-// first, then the chunk slots, so that window tiles, then each query's picker, are
-// dispatched ahead of the units that wait. Window tiles start at once (the screen
-// started after all earlier work on the stream). The picker (chunk slot 0) picks its
-// query's exact top-K from the screen values, writes idx / score / nsel and publishes
-// a flag; the other chunk units wait for the flag (bounded) and, should it not come,
-// compute the same deterministic pick themselves.
-template <typename T, int D>
-__global__ void __launch_bounds__(kThreads) attend_decode_pick_kernel(AttendArgs a, SelectArgs sa) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    __shared__ int is_last, flag_seen;
-    __shared__ PickSmem ps;
-    const UnitSmem s = unit_smem<T, D>(smem);
-    const int nwin = a.units - a.topk;
-    const int y = blockIdx.y;
-    const int u = y < nwin ? a.topk + y : y - nwin;  // unit index as in attend_decode_kernel
-    const int64_t qi = blockIdx.x;                   // (b, h), one query each
-    const int b = (int)(qi / a.H), h = (int)(qi % a.H);
-    const bool chunk_unit = u < a.topk;
-    const DecodeWs ws = decode_ws(a.ws, a.B * a.H, a.units, D);
-    int ns = 0, cidx = -1;
-    float csc = 0.f;
-    if (chunk_unit) {
-        pdl_wait();  // the screen grid has completed: its screen values are visible
-        if (u == 0) {
-            pick_query<T, D, kThreads>(sa, screen_ws(sa), qi, ps);
-            __syncthreads();  // the kept list is written before the flag
-            if (threadIdx.x == 0) st_release_gpu(ws.flags + qi, 1);
-        } else {
-            if (threadIdx.x == 0) {
-                int f = 0;
-                for (int it = 0; it < kFlagWaitIters && !(f = ld_acquire_gpu(ws.flags + qi)); ++it) __nanosleep(128);
-                flag_seen = f;
-            }
-            __syncthreads();
-            if (!flag_seen) {  // the picker has not been scheduled yet: pick here
-                pick_query<T, D, kThreads>(sa, screen_ws(sa), qi, ps);
-                __syncthreads();
-            }
-        }
-        ns = __ldcg(a.nsel + qi);
-        cidx = __ldcg(a.idx + qi * a.topk + u);
-        csc = __ldcg(a.score + qi * a.topk + u);
-    }
-    const int clen = a.cache_len[b];
-    const UnitPlan p = plan_unit_loaded(u, clen - 1, a.topk, a.W, cidx, csc, ns);
-    float *my_vec = ws.vec + ((size_t)qi * a.units + u) * D;
-    if (p.rows > 0) {
-        const T *qrow = static_cast<const T *>(a.Q.ptr) + b * a.Q.sb + h * a.Q.sh;
-        const T *k0 = static_cast<const T *>(a.K.ptr) + b * a.K.sb + h * a.K.sh + (int64_t)p.start * a.K.st;
-        const T *v0 = static_cast<const T *>(a.V.ptr) + b * a.V.sb + h * a.V.sh + (int64_t)p.start * a.V.st;
-        unit_issue<T, D>(s, qrow, k0, a.K.st, v0, a.V.st, p.rows);
-        const float lse_tile = unit_compute<T, D>(s, p.rows, a.scale);
-        for (int x = threadIdx.x; x < D; x += kThreads) my_vec[x] = s.red[x];
-        if (threadIdx.x == 0) ws.mass[qi * a.units + u] = p.is_chunk ? p.mass : lse_tile;
-    } else {
-        for (int x = threadIdx.x; x < D; x += kThreads) my_vec[x] = 0.f;
-        if (threadIdx.x == 0) ws.mass[qi * a.units + u] = -INFINITY;
-    }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) is_last = atomicAdd(&ws.counters[qi], 1) == a.units - 1;
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    combine_units<D>(ws.mass + (size_t)qi * a.units, ws.vec + (size_t)qi * a.units * D, a.units, s.red);
-    store_output<T, D>(a, b, h, 0, qi, s.red, s.red[D]);
-    if (threadIdx.x == 0) {  // every unit of the query has passed its flag wait
-        ws.counters[qi] = 0;
-        ws.flags[qi] = 0;
-    }
-}
-
 // General prefill path: one CTA per query, units in turn, running combination.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) attend_prefill_general_kernel(AttendArgs a) {
@@ -453,29 +376,6 @@ hils_status launch_decode(const AttendArgs &a, cudaStream_t st) {
 }
 
 template <typename T, int D>
-hils_status launch_decode_pick(const AttendArgs &a, const SelectArgs &sa, cudaStream_t st) {
-    using Cfg = UnitCfg<T, D>;
-    const int nq = a.B * a.H;
-    if (nq == 0) return HILS_OK;
-    static KernelSetup setup;
-    const hils_status stt = kernel_setup(setup, (const void *)attend_decode_pick_kernel<T, D>, kThreads,
-                                         Cfg::kSmemBytes, nullptr);
-    if (stt != HILS_OK) return stt;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(nq, a.units);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    void *argv[] = {const_cast<AttendArgs *>(&a), const_cast<SelectArgs *>(&sa)};
-    return record_cuda_error(cudaLaunchKernelExC(&cfg, (const void *)attend_decode_pick_kernel<T, D>, argv));
-}
-
-template <typename T, int D>
 hils_status launch_prefill_general(const AttendArgs &a, cudaStream_t st) {
     using Cfg = UnitCfg<T, D>;
     const int64_t nq = (int64_t)a.B * a.H * a.Lq;
@@ -498,12 +398,6 @@ size_t attend_decode_ws_bytes(int queries, int units, int d) {
 hils_status launch_attend_decode(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s) {
     if (dt == HILS_BF16) return d == 64 ? launch_decode<bf16, 64>(a, s) : launch_decode<bf16, 128>(a, s);
     return d == 64 ? launch_decode<float, 64>(a, s) : launch_decode<float, 128>(a, s);
-}
-
-hils_status launch_attend_decode_pick(hils_dtype dt, int d, const AttendArgs &a, const SelectArgs &sa,
-                                      cudaStream_t s) {
-    if (dt == HILS_BF16) return d == 64 ? launch_decode_pick<bf16, 64>(a, sa, s) : launch_decode_pick<bf16, 128>(a, sa, s);
-    return d == 64 ? launch_decode_pick<float, 64>(a, sa, s) : launch_decode_pick<float, 128>(a, sa, s);
 }
 
 hils_status launch_attend_prefill_general(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s) {

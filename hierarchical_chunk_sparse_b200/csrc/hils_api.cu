@@ -330,13 +330,6 @@ int hils_decode(const hils_params *p, hils_ctensor Qcal, hils_ctensor Ksum, cons
     // stream is complete before it starts; the attend follows the select's last kernel,
     // so its window tiles need not wait for the select
     aa.window_early = 1;
-    if (decode_cluster_supported(p->B, p->H, C, p->K))  // one cluster per query: the whole step
-        return launch_decode_cluster(p->dtype, p->d, sa, aa, stream);
-    if (sa.path == kSelectSplit) {
-        // the attend's chunk units repeat the pick of their query themselves
-        HILS_TRY(launch_select_screen(p->dtype, p->d, sa, stream));
-        return launch_attend_decode_pick(p->dtype, p->d, aa, sa, stream);
-    }
     HILS_TRY(launch_select(p->dtype, p->d, sa, stream));
     return launch_attend_decode(p->dtype, p->d, aa, stream);
 }

@@ -76,14 +76,6 @@ struct AttendArgs {
 hils_status launch_summarize(hils_dtype dt, int d, const SummarizeArgs &a, cudaStream_t s);
 hils_status launch_select(hils_dtype dt, int d, const SelectArgs &a, cudaStream_t s);
 hils_status launch_attend_decode(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s);
-// Decode chain of hils_decode on the split select path: the select's screen kernel only,
-// then the attend whose chunk units repeat the pick of their query (dependent launch).
-hils_status launch_select_screen(hils_dtype dt, int d, const SelectArgs &a, cudaStream_t s);
-// One decode step per query in one 8-CTA cluster (select + attend, hils_decode).
-bool decode_cluster_supported(int B, int H, int C, int K);
-hils_status launch_decode_cluster(hils_dtype dt, int d, const SelectArgs &sa, const AttendArgs &aa, cudaStream_t s);
-hils_status launch_attend_decode_pick(hils_dtype dt, int d, const AttendArgs &a, const SelectArgs &sa,
-                                      cudaStream_t s);
 hils_status launch_attend_prefill_general(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s);
 // Tensor-core prefill (bf16, d = 128): used when supported; `status` receives a nonzero
 // word if one of its bounded waits expired.
@@ -94,9 +86,11 @@ constexpr size_t kPrefillWsBytes = 256;  // status word (+ padding)
 // Workspace layouts (bytes); shared by the host size query and the kernels.
 size_t select_ws_bytes(int queries, int C, int path);
 size_t attend_decode_ws_bytes(int queries, int units, int d);
-// Leading part of the decode attend workspace that must start at zero (arrival counters
-// and pick flags, two ints per query, rounded to 256 bytes); every call leaves it zero.
-__host__ __device__ inline size_t attend_decode_counter_bytes(int queries) { return ((size_t)queries * 2 * sizeof(int) + 255) & ~(size_t)255; }
+// Leading part of the decode attend workspace that must start at zero (one arrival
+// counter per query, rounded to 256 bytes); every call leaves it zero.
+__host__ __device__ inline size_t attend_decode_counter_bytes(int queries) {
+    return ((size_t)queries * sizeof(int) + 255) & ~(size_t)255;
+}
 
 // Choice of the select kernels (path, ctas_per_query, tiles_per_warp of `a`); the
 // workspace size depends only on the sizes, never on has_qpos, so the size query and
@@ -208,25 +202,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
-
-// Release store / acquire load of a flag at GPU scope.
-__device__ __forceinline__ void st_release_gpu(int *p, int v) {
-    asm volatile("st.release.gpu.global.s32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Atomic add with acquire-release semantics at GPU scope: publishes the writes that
-// happen before it (in this thread, or in the CTA through a preceding barrier) and
-// makes the writes published by earlier adders visible to this thread.
-__device__ __forceinline__ int atomic_add_acq_rel_gpu(int *p, int v) {
-    int old;
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
 }
 
 __device__ __forceinline__ float warp_max(float v) {

@@ -1,8 +1,7 @@
 // One pipeline stage of the chunk screen (Eq. 7 of "Hierarchical Sparse Attention Done
 // Right" (picx.dev summary), with the rigorous radius of the exact selection): the
 // stage layout, the cooperative copies that fill it, and the screen of its rows on
-// tensor cores (bf16) or CUDA cores (float32). Shared by the decode select and the
-// clustered decode step.
+// tensor cores (bf16) or CUDA cores (float32), for the decode select's screen kernel.
 #pragma once
 #include "select_pick.cuh"
 

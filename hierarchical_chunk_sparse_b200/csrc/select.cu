@@ -215,11 +215,6 @@ size_t select_ws_bytes(int queries, int C, int path) {
     return dec_ws_bytes(queries, C);
 }
 
-hils_status launch_select_screen(hils_dtype dt, int d, const SelectArgs &a, cudaStream_t s) {
-    if (dt == HILS_BF16) return d == 64 ? launch_screen<bf16, 64>(a, s) : launch_screen<bf16, 128>(a, s);
-    return d == 64 ? launch_screen<float, 64>(a, s) : launch_screen<float, 128>(a, s);
-}
-
 hils_status launch_select(hils_dtype dt, int d, const SelectArgs &a, cudaStream_t s) {
     if (dt == HILS_BF16) return d == 64 ? launch<bf16, 64>(a, s) : launch<bf16, 128>(a, s);
     return d == 64 ? launch<float, 64>(a, s) : launch<float, 128>(a, s);

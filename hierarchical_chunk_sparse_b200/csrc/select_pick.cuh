@@ -1,8 +1,6 @@
 // Exact top-K pick of one decode query from the screen values of the decode select
 // ("Hierarchical Sparse Attention Done Right" (picx.dev summary), Eq. 7 and
-// Methodology 2; rcap.io post, pseudocode figure). Shared by the select's pick kernel
-// and the decode attend, whose chunk units repeat the (deterministic) pick of their
-// query instead of waiting for a separate kernel.
+// Methodology 2; rcap.io post, pseudocode figure), for the decode select's pick kernel.
 //
 // Workspace of the decode select: a 256-byte status header, then the screen value and
 // radius (s_c, e_c) of every eligible chunk per query, then the largest s and e of every

@@ -189,8 +189,6 @@ int hils_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hi
  * passages as the two calls). Results are those of the two calls made in turn: the
  * same kept chunks and scores (idx, score, nsel), and O and lse within rounding of
  * hils_attend_decode's.
- * With B*H >= 16 and C <= 8192 each query runs in one cluster of 8 CTAs that screens,
- * selects and attends without leaving the cluster (distributed shared memory).
  * Inside the chain the attend's window tiles need not wait for the select: its first
  * kernel starts only after all earlier work on the stream, so the window overlaps the
  * chunk selection.

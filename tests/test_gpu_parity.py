@@ -457,10 +457,10 @@ def _decode_chain(w, d, Ksum, Bsum, ws=None):
 
 @pytest.mark.parametrize("case", ["small16", "small6", "full"])
 def test_decode_chain_equals_separate_calls(oracle, cuda_device, case):
-    """hils_decode (one cluster of CTAs per query for B*H >= 16, else the select and
-    attend as one chain) keeps exactly the chunks and scores of hils_select and gives
-    the outputs of hils_attend_decode within the output tolerance; the small case is
-    also checked against the oracle, and every case runs twice on one workspace."""
+    """hils_decode (the select and the attend as one chain, the attend's window tiles
+    not waiting for the select) keeps exactly the chunks and scores of hils_select and
+    gives the outputs of hils_attend_decode within the output tolerance; the small case
+    is also checked against the oracle, and every case runs twice on one workspace."""
     full = case == "full"
     if full:
         w = WORKLOADS[4]
@@ -496,10 +496,10 @@ def test_decode_chain_equals_separate_calls(oracle, cuda_device, case):
     ((4000, 9001, 20000, 130), 16, 300, 64, torch.bfloat16),
     ((3000, 9001, 700, 6000), 16, 512, 128, torch.float32),
 ])
-def test_decode_cluster_edges(oracle, cuda_device, lens, K, W, d, dtype):
-    """hils_decode with B*H = 16 queries (one cluster each) against the oracle and the
-    separate calls: empty tables, tables of at most K chunks, fewer than K+1 groups, no
-    window, K = 32, d = 64 and float32."""
+def test_decode_chain_edges(oracle, cuda_device, lens, K, W, d, dtype):
+    """hils_decode with B*H = 16 queries against the oracle and the separate calls:
+    empty tables, tables of at most K chunks, fewer than K+1 groups, no window, K = 32,
+    d = 64 and float32."""
     w = WORKLOADS[4].replace(B=len(lens), H=4, N=max(lens), K=K, W=W, d=d, dtype=dtype, needles=0)
     inp = make_decode(w)
     inp["cache_len"] = torch.tensor(lens, dtype=torch.int32)
