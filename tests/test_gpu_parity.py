@@ -365,6 +365,43 @@ def test_attend_prefill_exact_mass_is_block_sparse_attention(oracle, cuda_device
     assert_close(O[0, :, 64:], ref[:, 64:], w.dtype, "O")
 
 
+@pytest.mark.parametrize("B,H,N,K,W", [(2, 8, 4096 + 100, 16, 512), (1, 6, 64 * 50 + 200, 3, 100),
+                                         (2, 3, 64 * 130 + 63, 32, 300)])
+def test_attend_prefill_persistent_items(oracle, cuda_device, B, H, N, K, W):
+    """More 256-query work items than SMs (each persistent CTA runs several, with
+    ragged last items and both query tiles partly past N), B > 1, K = 3 (few shared
+    chunks: many tiles with one empty half) and K = 32."""
+    w = WORKLOADS[2].replace(B=B, H=H, N=N, K=K, W=W)
+    inp = make_prefill(w)
+    d = to_dev(inp, cuda_device)
+    Ksum, Bsum = gpu_summarize(w, d["K"], d["LQ"])
+    idx, score, nsel = gpu_select(w, d["Qcal"], Ksum, Bsum)
+    O, lse = gpu_prefill(w, d["Q"], d["K"], d["V"], idx, score, nsel)
+    O_ref, lse_ref = oracle.attend(inp["Q"], inp["K"], inp["V"], host(idx), host(score), host(nsel),
+                                   64, w.W, w.scale)
+    assert_close(O, O_ref, w.dtype, "O")
+    assert_close(lse, lse_ref, torch.float32, "lse")
+
+
+def test_attend_prefill_full_size(oracle, cuda_device):
+    """The 8K prefill workload (B=1, H=32, N=8192, K=16, W=512) in the launch
+    configuration the benchmark times: every output of three sampled heads against the
+    oracle."""
+    w = WORKLOADS[2]
+    inp = make_prefill(w)
+    d = to_dev(inp, cuda_device)
+    Ksum, Bsum = gpu_summarize(w, d["K"], d["LQ"])
+    idx, score, nsel = gpu_select(w, d["Qcal"], Ksum, Bsum)
+    O, lse = gpu_prefill(w, d["Q"], d["K"], d["V"], idx, score, nsel)
+    g = torch.Generator().manual_seed(82)
+    for h in torch.randperm(w.H, generator=g)[:3].tolist():
+        sl = slice(h, h + 1)
+        O_ref, lse_ref = oracle.attend(inp["Q"][:, sl], inp["K"][:, sl], inp["V"][:, sl], host(idx[:, sl]),
+                                       host(score[:, sl]), host(nsel[:, sl]), 64, w.W, w.scale)
+        assert_close(O[:, sl], O_ref, w.dtype, f"O head {h}")
+        assert_close(lse[:, sl], lse_ref, torch.float32, f"lse head {h}")
+
+
 def _decode_small(cuda_device, lens=(5000, 3001), K=16, W=512, H=3):
     w = WORKLOADS[4].replace(B=len(lens), H=H, N=max(lens), K=K, W=W, needles=0)
     inp = make_decode(w)
