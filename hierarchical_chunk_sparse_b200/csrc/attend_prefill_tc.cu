@@ -5,24 +5,29 @@
 //
 // A persistent CTA (one per SM) takes work items of 256 consecutive queries of one
 // (b, h): two 128-row query tiles A and B that share every key/value tile. Each item
-// walks 128-key tiles made of two 64-key halves:
-//   1. window tiles covering [max(0, t0-W+1), t0+255] (online softmax; a row's
+// walks 64-key tiles:
+//   1. the window tiles covering [max(0, t0-W+1), t0+255] (online softmax; a row's
 //      reference max is raised, and O rescaled, only when the row's tile max passes it
 //      by more than 8 in log2 units);
-//   2. the union of the chunks kept by the item's 256 queries, ascending, two chunks per
+//   2. the union of the chunks kept by the item's 256 queries, ascending, one chunk per
 //      tile; a row that kept chunk c weights that chunk's own softmax by exp(s^_c), a
 //      row that did not contributes zero.
 // Warp roles (352 threads), all hand-offs through mbarriers:
 //   warps 0-3  softmax of tile A (thread = row = TMEM lane), warps 4-7 softmax of B;
-//   warp 8     TMA loads (Q of both tiles, K and V of each 128-key tile, 2-slot ring);
-//   warp 9     tcgen05.mma issue: S_X = Q_X K^T (M=128, N=128, K=128) into TMEM, then
-//              O_X += P_X V (A operand P_X read from TMEM over the columns of S_X);
+//   warp 8     TMA loads (Q of both tiles; K and V of each key tile, 4-slot rings);
+//   warp 9     tcgen05.mma issue: S_X = Q_X K^T (M=128, N=64, K=128) into TMEM, then
+//              O_X += P_X V (M=128, N=128, K=64, the A operand P_X read from TMEM);
 //   warp 10    builds the next item's union bitmap while the others work.
-// The MMA warp alternates the two tiles (S_A(i), PV_B(i-1), S_B(i), PV_A(i), ...), so
-// the softmax of one tile runs while the tensor pipe works on the other. The tensor
-// pipe executes one thread's tcgen05.mma in issue order, which is what lets S_X(i+1)
-// reuse the TMEM columns of P_X(i) once PV_X(i) has been issued. TMEM: S_A [0,128),
-// S_B [128,256), O_A [256,384), O_B [384,512).
+// S is double-buffered per query tile and P_X(i) is written over S_X(i) (its first 32
+// columns): S_X(i+1) is computed while the softmax of tile i runs. A later MMA is not
+// ordered after the TMEM operand reads of an earlier one, so the MMA warp issues S_X(i+2)
+// into buffer i % 2 only once the completion of PV_X(i), which read P_X(i) there, has
+// been signalled on that buffer's barrier; PV_X(i) is issued a whole tile earlier, so the
+// wait rarely blocks. A parity wait is exact only while the phase before the awaited one
+// has completed; the PV barrier of a buffer is first awaited by the MMA warp (before it
+// reuses the buffer), which also makes the softmax's waits for O on it exact.
+// TMEM: S_A0 [0,64), S_A1 [64,128), S_B0 [128,192), S_B1 [192,256), O_A [256,384),
+// O_B [384,512).
 // Every mbarrier wait is bounded: on expiry the CTA records an error in the status word,
 // every role stops issuing work, the CTA drains the copies and MMAs it started, frees
 // its TMEM and exits; outputs of unfinished items are not written.
@@ -35,41 +40,43 @@ using namespace tc;
 
 constexpr int kM = 128;          // query rows per tile
 constexpr int kRows = 2 * kM;    // query rows per work item
-constexpr int kHalf = 64;        // keys per half tile (= chunk size)
+constexpr int kTile = 64;        // keys per tile (= chunk size)
 constexpr int kHead = 128;       // head dimension
-constexpr int kSoftmaxThreads = 256;
+constexpr int kSoftmaxWarps = 8;
 constexpr int kLoadWarp = 8, kMmaWarp = 9, kMapWarp = 10;
 constexpr int kThreads = 352;
-constexpr int kStages = 2;       // K/V ring depth
+constexpr int kStages = 4;       // K/V ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxBitmapWords = 256;  // union bitmap: up to 8192 chunks
 constexpr long long kWaitLimit = 1ll << 26;
 
 // shared memory map (offsets from the 1024-aligned base)
 constexpr int kQOff = 0;                                  // 2 tiles x 2 blocks x [128 rows x 128 B]
-constexpr int kKOff = 65536;                              // kStages x 2 blocks x [128 keys x 128 B]
-constexpr int kVOff = kKOff + kStages * 32768;            // same
-constexpr int kBarOff = kVOff + kStages * 32768;          // mbarriers
-constexpr int kMiscOff = kBarOff + 256;                   // tmem base, abort flag, union counts
+constexpr int kKOff = 65536;                              // kStages x 2 blocks x [64 keys x 128 B]
+constexpr int kVOff = kKOff + kStages * 16384;            // same
+constexpr int kBarOff = kVOff + kStages * 16384;          // mbarriers
+constexpr int kMiscOff = kBarOff + 512;                   // tmem base, abort flag, union counts
 constexpr int kBitmapOff = kMiscOff + 64;                 // 2 union bitmaps (double-buffered by item)
-constexpr int kSmemBytes = kBitmapOff + 2 * kMaxBitmapWords * 4 + 1024;  // + alignment slack
+constexpr int kNselOff = kBitmapOff + 2 * kMaxBitmapWords * 4;  // 2 x [256] kept counts (builder)
+constexpr int kSmemBytes = kNselOff + 2 * kRows * 4 + 1024;     // + alignment slack
 
 enum {
     kBarQfull = 0,
     kBarQfree = 1,
-    kBarKfull = 2,   // + slot
-    kBarKfree = 4,   // + slot
-    kBarVfull = 6,   // + slot
-    kBarVfree = 8,   // + slot
-    kBarSfull = 10,  // + tile (A, B)
-    kBarPfull = 12,  // + tile
-    kBarOdone = 14,  // + tile
-    kBarMapReady = 16,  // + item parity
-    kBarMapFree = 18,   // + item parity
-    kBarDrain = 20,
-    kNumBars = 21
+    kBarKfull = 2,       // + slot
+    kBarKfree = 6,       // + slot
+    kBarVfull = 10,      // + slot
+    kBarVfree = 14,      // + slot
+    kBarSfull = 18,      // + 2 * tile + buffer: S_X written
+    kBarPfull = 22,      // + 2 * tile + buffer: P_X written over it
+    kBarPVdone = 26,     // + 2 * tile + buffer: the PV that read the buffer (and every MMA
+                         //   issued before it) completed
+    kBarMapReady = 30,   // + item parity
+    kBarMapFree = 32,    // + item parity
+    kBarDrain = 34,
+    kNumBars = 35
 };
-constexpr uint32_t kMapFreeCount = kSoftmaxThreads + 2;  // softmax rows + load warp + MMA warp
+constexpr uint32_t kMapFreeCount = kSoftmaxWarps * 32 + 2;  // softmax rows + load warp + MMA warp
 
 struct TcArgs {
     AttendArgs a;
@@ -97,13 +104,54 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return r;
 }
 
+// 1/z for a normal positive z on the FMA pipe: an integer-subtraction seed (relative
+// error at most 5.1e-2, constant fitted numerically over one binade) and two Newton
+// steps r <- r (2 - z r), which square the error: below 7e-6 plus rounding.
+__device__ __forceinline__ float recip_newton(float z) {
+    float r = __int_as_float(0x7ef311c2 - __float_as_int(z));
+    r = fmaf(r, fmaf(-z, r, 1.f), r);
+    r = fmaf(r, fmaf(-z, r, 1.f), r);
+    return r;
+}
+
+// 2^x on the FMA pipe (no MUFU), for finite x: x = j + f with j = round(x) (the
+// 1.5 * 2^23 shifter) and f in [-1/2, 1/2]; 2^f by a degree-5 polynomial fitted here for
+// relative error (iteratively reweighted least squares on Chebyshev nodes; at most
+// 2.4e-7 in float32 Horner form); 2^j added to the exponent field. x is clamped to
+// [-125, 127] so the result stays a normal float (2^-125 stands for anything smaller).
+__device__ __forceinline__ float exp2_fma(float x) {
+    x = fminf(fmaxf(x, -125.f), 127.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    float p = 1.327647129e-03f;
+    p = fmaf(p, f, 9.675540961e-03f);
+    p = fmaf(p, f, 5.550713092e-02f);
+    p = fmaf(p, f, 2.402212024e-01f);
+    p = fmaf(p, f, 6.931469440e-01f);
+    p = fmaf(p, f, 1.000000119e+00f);
+    return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4b400000) << 23));
+}
+
+// Loads that the compiler keeps where they are written: a kept-list entry is fetched
+// four selections before it is needed, not at its first use.
+__device__ __forceinline__ int ldg_early(const int32_t *p) {
+    int v;
+    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ float ldg_early(const float *p) {
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
 // The work item of round r for CTA c: rounds alternate direction so that every CTA gets
 // a similar share of the expensive (late-query) items, which come first.
 __device__ __forceinline__ int item_of(int r, int c, int G) { return r * G + ((r & 1) ? (G - 1 - c) : c); }
 
 struct Item {
     int b, h, t0;
-    int ws0, nhw, nwt;  // window: first key, halves, tiles
+    int ws0, nw;  // window: first key, tiles
 };
 
 __device__ __forceinline__ Item decode_item(const TcArgs &args, int j) {
@@ -116,14 +164,13 @@ __device__ __forceinline__ Item decode_item(const TcArgs &args, int j) {
     it.h = bh % a.H;
     it.t0 = qb * kRows;
     it.ws0 = 0;
-    it.nhw = 0;
+    it.nw = 0;
     if (a.W > 0) {
         const int lo = max(0, it.t0 - a.W + 1);
         const int hi = min(args.N - 1, it.t0 + kRows - 1);
-        it.ws0 = (lo / kHalf) * kHalf;
-        it.nhw = (hi - it.ws0) / kHalf + 1;
+        it.ws0 = (lo / kTile) * kTile;
+        it.nw = (hi - it.ws0) / kTile + 1;
     }
-    it.nwt = (it.nhw + 1) >> 1;
     return it;
 }
 
@@ -147,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) {
             uint32_t cnt = 1;
-            if (i == kBarPfull || i == kBarPfull + 1) cnt = kM;
+            if (i >= kBarPfull && i < kBarPfull + 4) cnt = 4;  // one elected lane per softmax warp
             if (i == kBarMapReady || i == kBarMapReady + 1) cnt = 32;
             if (i == kBarMapFree || i == kBarMapFree + 1) cnt = kMapFreeCount;
             mbar_init(bar(i), cnt);
@@ -167,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
 
     // bounded wait; false once the CTA has aborted (the first expiry sets the flag)
     auto wait = [&](uint32_t barrier, uint32_t parity) -> bool {
-        if (*abort_flag) return false;
+        if (mbar_try_wait(barrier, parity)) return true;
         for (long long it = 0; it < kWaitLimit; ++it) {
             if (mbar_try_wait(barrier, parity)) return true;
             if ((it & 255) == 255 && *abort_flag) return false;
@@ -180,6 +227,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     auto wait_warp = [&](uint32_t barrier, uint32_t parity) -> bool {
         const bool ok = wait(barrier, parity);
         return __all_sync(kFull, ok);
+    };
+    auto arrive = [&](uint32_t barrier) {
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(barrier) : "memory");
     };
 
     const float kLog2e = 1.4426950408889634f;
@@ -194,18 +244,31 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             const int par = n & 1;
             if (n >= 2 && !wait_warp(bar(kBarMapFree + par), ((n - 2) >> 1) & 1)) break;
             uint32_t *bm = bitmaps + par * kMaxBitmapWords;
+            int *nsm = reinterpret_cast<int *>(smem + kNselOff) + par * kRows;
             for (int i = lane; i < nwords; i += 32) bm[i] = 0u;
+            // the item's rows are consecutive: their kept lists form one contiguous block,
+            // read with many loads in flight
+            const int nrows = min(kRows, args.N - it.t0);
+            const int64_t q0 = ((int64_t)it.b * a.H + it.h) * a.Lq + it.t0;
+#pragma unroll
+            for (int rr = lane; rr < kRows; rr += 32)
+                nsm[rr] = (a.topk > 0 && rr < nrows) ? min(max(__ldg(&a.nsel[q0 + rr]), 0), a.topk) : 0;
             __syncwarp();
-            if (a.topk > 0) {
-                for (int rr = lane; rr < kRows; rr += 32) {
-                    const int t = it.t0 + rr;
-                    if (t >= args.N) break;
-                    const int64_t qrow = ((int64_t)it.b * a.H + it.h) * a.Lq + t;
-                    const int ns = min(max(__ldg(&a.nsel[qrow]), 0), a.topk);
-                    const int32_t *ip = a.idx + qrow * a.topk;
-                    for (int k = 0; k < ns; ++k) {
-                        const int c = __ldg(&ip[k]);
-                        if (c >= 0 && c < args.C) atomicOr(&bm[c >> 5], 1u << (c & 31));
+            const int tot = a.topk > 0 ? nrows * a.topk : 0;
+            const int32_t *ib = a.idx + q0 * a.topk;
+            for (int e0 = 0; e0 < tot; e0 += 32 * 16) {
+                int cv[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int e = e0 + u * 32 + lane;
+                    cv[u] = e < tot ? __ldg(&ib[e]) : -1;
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int e = e0 + u * 32 + lane;
+                    if (cv[u] >= 0 && cv[u] < args.C) {
+                        const int row = e / a.topk;
+                        if (e - row * a.topk < nsm[row]) atomicOr(&bm[cv[u] >> 5], 1u << (cv[u] & 31));
                     }
                 }
             }
@@ -216,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(kFull, cnt, o);
             if (lane == 0) union_count[par] = (uint32_t)cnt;
             __syncwarp();
-            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar(kBarMapReady + par)) : "memory");
+            arrive(bar(kBarMapReady + par));
         }
     } else if (warp == kLoadWarp) {
         // ---------------------------------------------------------------- TMA loads
@@ -228,8 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             const Item it = decode_item(args, j);
             const int par = n & 1;
             if (!wait_warp(bar(kBarMapReady + par), (n >> 1) & 1)) break;
-            const int nu = (int)union_count[par];
-            const int nt = it.nwt + ((nu + 1) >> 1);
+            const int nt = it.nw + (int)union_count[par];
             const uint32_t *bm = bitmaps + par * kMaxBitmapWords;
             bool ok = true;
             if (nt > 0) {
@@ -248,46 +310,35 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
                 ++qn;
                 int cur = -1;  // union walk
                 for (int i = 0; i < nt && ok; ++i, ++g) {
-                    int k0, k1;
-                    if (i < it.nwt) {
-                        k0 = it.ws0 + kHalf * (2 * i);
-                        k1 = it.ws0 + kHalf * min(2 * i + 1, it.nhw - 1);
+                    int k0;
+                    if (i < it.nw) {
+                        k0 = it.ws0 + kTile * i;
                     } else {
-                        const int c0 = next_bit(bm, nwords, cur + 1);
-                        const int c1 = next_bit(bm, nwords, c0 + 1);
-                        cur = c1 >= 0 ? c1 : c0;
-                        k0 = c0 * kHalf;
-                        k1 = (c1 >= 0 ? c1 : c0) * kHalf;
+                        cur = next_bit(bm, nwords, cur + 1);
+                        k0 = cur * kTile;
                     }
                     const int s = g % kStages, u = g / kStages;
                     if (u > 0 && !(ok = wait_warp(bar(kBarKfree + s), (u - 1) & 1))) break;
                     if (lane == 0) {
                         ++issuedK;
-                        mbar_expect_tx(bar(kBarKfull + s), 4 * kHalf * 128);
-                        const uint32_t dst = sbase + kKOff + s * 32768;
-#pragma unroll
-                        for (int kb = 0; kb < 2; ++kb) {
-                            tma_load_4d(dst + kb * 16384, &tmK, bar(kBarKfull + s), kb * 64, k0, it.h, it.b);
-                            tma_load_4d(dst + kb * 16384 + 8192, &tmK, bar(kBarKfull + s), kb * 64, k1, it.h, it.b);
-                        }
+                        mbar_expect_tx(bar(kBarKfull + s), 2 * kTile * 128);
+                        const uint32_t dst = sbase + kKOff + s * 16384;
+                        tma_load_4d(dst, &tmK, bar(kBarKfull + s), 0, k0, it.h, it.b);
+                        tma_load_4d(dst + 8192, &tmK, bar(kBarKfull + s), 64, k0, it.h, it.b);
                     }
                     if (u > 0 && !(ok = wait_warp(bar(kBarVfree + s), (u - 1) & 1))) break;
                     if (lane == 0) {
                         ++issuedV;
-                        mbar_expect_tx(bar(kBarVfull + s), 4 * kHalf * 128);
-                        const uint32_t dst = sbase + kVOff + s * 32768;
-#pragma unroll
-                        for (int kb = 0; kb < 2; ++kb) {
-                            tma_load_4d(dst + kb * 16384, &tmV, bar(kBarVfull + s), kb * 64, k0, it.h, it.b);
-                            tma_load_4d(dst + kb * 16384 + 8192, &tmV, bar(kBarVfull + s), kb * 64, k1, it.h, it.b);
-                        }
+                        mbar_expect_tx(bar(kBarVfull + s), 2 * kTile * 128);
+                        const uint32_t dst = sbase + kVOff + s * 16384;
+                        tma_load_4d(dst, &tmV, bar(kBarVfull + s), 0, k0, it.h, it.b);
+                        tma_load_4d(dst + 8192, &tmV, bar(kBarVfull + s), 64, k0, it.h, it.b);
                     }
                 }
             }
             if (!ok) break;
             __syncwarp();
-            if (lane == 0)
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar(kBarMapFree + par)) : "memory");
+            if (lane == 0) arrive(bar(kBarMapFree + par));
         }
         // after an abort: the copies this warp started land before the CTA releases its memory
         if (lane == 0 && *abort_flag) {
@@ -304,26 +355,32 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------------- MMA issue
-        const uint32_t idS = idesc_bf16(kM, 2 * kHalf, false);
+        const uint32_t idS = idesc_bf16(kM, kTile, false);
         const uint32_t idPV = idesc_bf16(kM, kHead, true);
-        auto issue_s = [&](int x, int s) {  // S_x = Q_x K_s^T
-            const uint32_t d = tmem + x * 128;
+        auto issue_s = [&](int x, int gt) {  // S_x(gt) = Q_x K^T into buffer gt % 2
+            const int s = gt % kStages;
+            const uint32_t d = tmem + x * 128 + (gt & 1) * 64;
 #pragma unroll
             for (int ks = 0; ks < kHead / 16; ++ks) {
                 const uint32_t qa = sbase + kQOff + x * 32768 + (ks >> 2) * 16384 + (ks & 3) * 32;
-                const uint32_t ka = sbase + kKOff + s * 32768 + (ks >> 2) * 16384 + (ks & 3) * 32;
+                const uint32_t ka = sbase + kKOff + s * 16384 + (ks >> 2) * 8192 + (ks & 3) * 32;
                 mma_ss(d, smem_desc(qa, 16, 1024), smem_desc(ka, 16, 1024), idS, ks > 0);
             }
-            mma_commit(bar(kBarSfull + x));
+            mma_commit(bar(kBarSfull + 2 * x + (gt & 1)));
         };
-        auto issue_pv = [&](int x, int s, bool acc) {  // O_x (+)= P_x V_s
+        auto issue_pv = [&](int x, int gt, bool acc) {  // O_x (+)= P_x(gt) V
+            const int s = gt % kStages;
 #pragma unroll
-            for (int ks = 0; ks < 2 * kHalf / 16; ++ks) {
-                const uint32_t va = sbase + kVOff + s * 32768 + ks * 2048;
-                mma_ts(tmem + 256 + x * 128, tmem + x * 128 + ks * 8, smem_desc(va, 16384, 1024), idPV,
-                       (acc || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < kTile / 16; ++ks) {
+                const uint32_t va = sbase + kVOff + s * 16384 + ks * 2048;
+                mma_ts(tmem + 256 + x * 128, tmem + x * 128 + (gt & 1) * 64 + ks * 8, smem_desc(va, 8192, 1024),
+                       idPV, (acc || ks > 0) ? 1u : 0u);
             }
-            mma_commit(bar(kBarOdone + x));
+            mma_commit(bar(kBarPVdone + 2 * x + (gt & 1)));
+        };
+        // S_x(gt) goes into the buffer that PV_x(gt - 2) read: that PV has completed
+        auto s_free = [&](int x, int gt) {
+            return gt < 2 || wait_warp(bar(kBarPVdone + 2 * x + (gt & 1)), ((gt >> 1) - 1) & 1);
         };
         int g = 0, qn = 0;
         bool ok = true;
@@ -333,47 +390,46 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             const Item it = decode_item(args, j);
             const int par = n & 1;
             if (!(ok = wait_warp(bar(kBarMapReady + par), (n >> 1) & 1))) break;
-            const int nu = (int)union_count[par];
-            const int nt = it.nwt + ((nu + 1) >> 1);
+            const int nt = it.nw + (int)union_count[par];
             __syncwarp();
-            if (lane == 0)
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar(kBarMapFree + par)) : "memory");
+            if (lane == 0) arrive(bar(kBarMapFree + par));
             if (nt == 0) continue;
             if (!(ok = wait_warp(bar(kBarQfull), qn & 1))) break;
             ++qn;
             tc_fence_after();
-            for (int i = 0; i < nt; ++i, ++g) {
-                const int s = g % kStages, u = g / kStages;
-                if (!(ok = wait_warp(bar(kBarKfull + s), u & 1))) break;
+            // S of the item's first tile, then per tile: S of the next, PV of this one
+            auto s_pair = [&](int gt, bool last) -> bool {
+                if (!wait_warp(bar(kBarKfull + gt % kStages), (gt / kStages) & 1)) return false;
+                if (!s_free(0, gt)) return false;
                 tc_fence_after();
-                if (lane == 0) issue_s(0, s);
-                if (i > 0) {  // PV_B of the previous tile
-                    if (!(ok = wait_warp(bar(kBarPfull + 1), (g - 1) & 1))) break;
-                    tc_fence_after();
-                    if (lane == 0) {
-                        issue_pv(1, (g - 1) % kStages, i > 1);
-                        mma_commit(bar(kBarVfree + (g - 1) % kStages));
-                    }
-                }
+                if (lane == 0) issue_s(0, gt);
+                if (!s_free(1, gt)) return false;
+                tc_fence_after();
                 if (lane == 0) {
-                    issue_s(1, s);
-                    mma_commit(bar(kBarKfree + s));
-                    if (i == nt - 1) mma_commit(bar(kBarQfree));
+                    issue_s(1, gt);
+                    mma_commit(bar(kBarKfree + gt % kStages));
+                    if (last) mma_commit(bar(kBarQfree));
                 }
-                if (!(ok = wait_warp(bar(kBarPfull + 0), g & 1))) break;
-                if (!(ok = wait_warp(bar(kBarVfull + s), u & 1))) break;
-                tc_fence_after();
-                if (lane == 0) issue_pv(0, s, i > 0);
                 __syncwarp();
+                return true;
+            };
+            // S of the item's first two tiles, then per tile: PV of this one, S of the one two ahead
+            if (!(ok = s_pair(g, nt == 1))) break;
+            if (nt > 1 && !(ok = s_pair(g + 1, nt == 2))) break;
+            for (int i = 0; i < nt; ++i, ++g) {
+                if (!(ok = wait_warp(bar(kBarPfull + (g & 1)), (g >> 1) & 1))) break;
+                if (!(ok = wait_warp(bar(kBarVfull + g % kStages), (g / kStages) & 1))) break;
+                tc_fence_after();
+                if (lane == 0) issue_pv(0, g, i > 0);
+                if (!(ok = wait_warp(bar(kBarPfull + 2 + (g & 1)), (g >> 1) & 1))) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    issue_pv(1, g, i > 0);
+                    mma_commit(bar(kBarVfree + g % kStages));
+                }
+                __syncwarp();
+                if (i + 2 < nt && !(ok = s_pair(g + 2, i + 3 == nt))) break;
             }
-            if (!ok) break;
-            if (!(ok = wait_warp(bar(kBarPfull + 1), (g - 1) & 1))) break;
-            tc_fence_after();
-            if (lane == 0) {
-                issue_pv(1, (g - 1) % kStages, nt > 1);
-                mma_commit(bar(kBarVfree + (g - 1) % kStages));
-            }
-            __syncwarp();
         }
         // every MMA this warp issued completes before TMEM and shared memory are released
         if (lane == 0) {
@@ -388,9 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         const int quad = warp & 3;          // TMEM lane quadrant
         const int rloc = quad * 32 + lane;  // row within the tile = TMEM lane
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-        const uint32_t s_col = tmem + lane_base + x * 128;
         const uint32_t o_col = tmem + lane_base + 256 + x * 128;
-        int g = 0;  // tiles processed by this query tile, over all items
+        int g = 0;  // key tiles processed, over all items
         for (int r = 0, n = 0;; ++r, ++n) {
             const int j = item_of(r, cta, G);
             if (j >= args.items) break;
@@ -403,9 +458,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             const int32_t *ip = a.idx + qrow * a.topk;
             const float *sp = a.score + qrow * a.topk;
             float ref = -INFINITY;  // log2-domain reference: the largest kept chunk score
+#pragma unroll 8
             for (int k = 0; k < nsel; ++k) {
                 const int c = __ldg(&ip[k]);
-                if (c >= 0 && c < args.C) ref = fmaxf(ref, __ldg(&sp[k]) * kLog2e);
+                const float sc = __ldg(&sp[k]);
+                ref = fmaxf(ref, (c >= 0 && c < args.C) ? sc * kLog2e : -INFINITY);
             }
             // the row's kept list, four entries ahead (ascending chunk indices)
             int qc[4];
@@ -418,98 +475,75 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
                 ++kn;
             }
             if (!wait_warp(bar(kBarMapReady + par), (n >> 1) & 1)) break;
-            const int nu = (int)union_count[par];
-            const int nt = it.nwt + ((nu + 1) >> 1);
+            const int nt = it.nw + (int)union_count[par];
             const uint32_t *bm = bitmaps + par * kMaxBitmapWords;
             float m_used = ref;
             float l = 0.f;
             int cur = -1;
             bool ok = true;
             for (int i = 0; i < nt; ++i, ++g) {
-                if (!(ok = wait_warp(bar(kBarSfull + x), g & 1))) break;
+                const int bsel = g & 1;
+                if (!(ok = wait_warp(bar(kBarSfull + 2 * x + bsel), (g >> 1) & 1))) break;
                 tc_fence_after();
-                uint32_t sr[64];
-                uint32_t pk[32];
-                if (i < it.nwt) {
-                    // ---- window tile: halves at ks0, ks1 (the second may be empty)
-                    const int ks0 = it.ws0 + kHalf * (2 * i);
-                    const bool h1 = 2 * i + 1 < it.nhw;
-                    const int ks1 = ks0 + kHalf;
-                    // valid key offsets j in [jlo, jhi] of each half for this row
-                    auto range = [&](int ks, bool valid, int &jlo, int &jhi) {
-                        jlo = max(0, t - a.W + 1 - ks);
-                        jhi = min(kHalf - 1, t - ks);
-                        if (!valid || !row_ok) {
-                            jlo = kHalf;
-                            jhi = -1;
-                        }
-                    };
-                    int lo0, hi0, lo1, hi1;
-                    range(ks0, true, lo0, hi0);
-                    range(ks1, h1, lo1, hi1);
-                    const bool full0 = __all_sync(kFull, lo0 == 0 && hi0 == kHalf - 1);
-                    const bool full1 = __all_sync(kFull, lo1 == 0 && hi1 == kHalf - 1);
-                    const bool none1 = __all_sync(kFull, lo1 > hi1);
-                    auto half_max = [&](bool full, int jlo, int jhi) {
-                        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-                        if (full) {
-#pragma unroll
-                            for (int q = 0; q < 64; q += 8) {
-                                m0 = max3(m0, __uint_as_float(sr[q]), __uint_as_float(sr[q + 1]));
-                                m1 = max3(m1, __uint_as_float(sr[q + 2]), __uint_as_float(sr[q + 3]));
-                                m2 = max3(m2, __uint_as_float(sr[q + 4]), __uint_as_float(sr[q + 5]));
-                                m3 = max3(m3, __uint_as_float(sr[q + 6]), __uint_as_float(sr[q + 7]));
-                            }
-                        } else {
+                const uint32_t s_col = tmem + lane_base + x * 128 + bsel * 64;
+                uint32_t sr[64];  // S of this row, then (packed in place into sr[0..31]) its P
+                bool any = true;
+                if (i < it.nw) {
+                    // ---- window tile: keys [ks, ks + 64); valid offsets [jlo, jhi] of this row
+                    const int ks = it.ws0 + kTile * i;
+                    int jlo = max(0, t - a.W + 1 - ks);
+                    int jhi = min(kTile - 1, t - ks);
+                    if (!row_ok) {
+                        jlo = kTile;
+                        jhi = -1;
+                    }
+                    const bool full = __all_sync(kFull, jlo == 0 && jhi == kTile - 1);
+                    any = __any_sync(kFull, jlo <= jhi);
+                    if (any) {
+                        tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                        tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                        tmem_wait_ld();
+                    }
+                    if (any) {
+                        if (!full) {
 #pragma unroll
                             for (int q = 0; q < 64; ++q) {
                                 const bool v = q >= jlo && q <= jhi;
                                 sr[q] = v ? sr[q] : __float_as_uint(-INFINITY);
                             }
+                        }
+                        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-                            for (int q = 0; q < 64; q += 8) {
-                                m0 = max3(m0, __uint_as_float(sr[q]), __uint_as_float(sr[q + 1]));
-                                m1 = max3(m1, __uint_as_float(sr[q + 2]), __uint_as_float(sr[q + 3]));
-                                m2 = max3(m2, __uint_as_float(sr[q + 4]), __uint_as_float(sr[q + 5]));
-                                m3 = max3(m3, __uint_as_float(sr[q + 6]), __uint_as_float(sr[q + 7]));
+                        for (int q = 0; q < 64; q += 8) {
+                            m0 = max3(m0, __uint_as_float(sr[q]), __uint_as_float(sr[q + 1]));
+                            m1 = max3(m1, __uint_as_float(sr[q + 2]), __uint_as_float(sr[q + 3]));
+                            m2 = max3(m2, __uint_as_float(sr[q + 4]), __uint_as_float(sr[q + 5]));
+                            m3 = max3(m3, __uint_as_float(sr[q + 6]), __uint_as_float(sr[q + 7]));
+                        }
+                        const float mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * scale2;
+                        // raise the row's reference when its tile max passes it by more than 8
+                        const bool raise = mt != -INFINITY && (m_used == -INFINITY || mt > m_used + 8.f);
+                        const float f = raise ? ex2(m_used - mt) : 1.f;  // 0 when m_used is -inf
+                        if (__any_sync(kFull, raise && l > 0.f)) {
+                            // O holds earlier tiles of this item: PV_x of the previous tile completes first
+                            if (!(ok = wait_warp(bar(kBarPVdone + 2 * x + ((g - 1) & 1)), ((g - 1) >> 1) & 1))) break;
+                            tc_fence_after();
+                            // in 8-column pieces: S stays in registers meanwhile
+#pragma unroll 1
+                            for (int part = 0; part < 16; ++part) {
+                                uint32_t o[8];
+                                tmem_ld8(o_col + part * 8, o);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * f);
+                                tmem_st8(o_col + part * 8, o);
                             }
                         }
-                        return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-                    };
-                    float mt = -INFINITY;
-                    if (!none1) {
-                        tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                        tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                        tmem_wait_ld();
-                        mt = half_max(full1, lo1, hi1);
-                    }
-                    tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                    tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                    tmem_wait_ld();
-                    mt = fmaxf(mt, half_max(full0, lo0, hi0)) * scale2;
-                    // raise the row's reference when its tile max passes it by more than 8
-                    const bool raise = mt != -INFINITY && (m_used == -INFINITY || mt > m_used + 8.f);
-                    const float f = raise ? ex2(m_used - mt) : 1.f;  // 0 when m_used is -inf
-                    if (__any_sync(kFull, raise && l > 0.f)) {
-                        // O holds earlier tiles of this item: PV_x of the previous tile completes first
-                        if (!(ok = wait_warp(bar(kBarOdone + x), (g - 1) & 1))) break;
-                        tc_fence_after();
-#pragma unroll
-                        for (int part = 0; part < 4; ++part) {
-                            uint32_t o[32];
-                            tmem_ld32(o_col + part * 32, o);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * f);
-                            tmem_st32(o_col + part * 32, o);
+                        if (raise) {
+                            l *= f;
+                            m_used = mt;
                         }
-                    }
-                    if (raise) {
-                        l *= f;
-                        m_used = mt;
-                    }
-                    const float nb = m_used == -INFINITY ? 0.f : -m_used;
-                    auto half_exp = [&]() {  // sr (masked) -> pk, returns the sum
+                        const float nb = m_used == -INFINITY ? 0.f : -m_used;
                         float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
 #pragma unroll
                         for (int q = 0; q < 64; q += 4) {
@@ -521,102 +555,86 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
                             z1 += e1;
                             z2 += e2;
                             z3 += e3;
-                            pk[q >> 1] = pack_bf16(e0, e1);
-                            pk[(q >> 1) + 1] = pack_bf16(e2, e3);
+                            sr[q >> 1] = pack_bf16(e0, e1);  // sr[q/2 + 1] <= sr[q + 1]: already read
+                            sr[(q >> 1) + 1] = pack_bf16(e2, e3);
                         }
-                        return (z0 + z1) + (z2 + z3);
-                    };
-                    // half 0 (still in registers, masked) -> P columns [0, 32)
-                    l += half_exp();
-                    tmem_st32(s_col, pk);
-                    // half 1 -> P columns [32, 64)
-                    if (none1) {
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) pk[q] = 0u;
-                    } else {
-                        tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                        tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                        tmem_wait_ld();
-                        if (!full1) {
-#pragma unroll
-                            for (int q = 0; q < 64; ++q) {
-                                const bool v = q >= lo1 && q <= hi1;
-                                sr[q] = v ? sr[q] : __float_as_uint(-INFINITY);
-                            }
-                        }
-                        l += half_exp();
+                        l += (z0 + z1) + (z2 + z3);
                     }
-                    tmem_st32(s_col + 32, pk);
                 } else {
-                    // ---- chunk tile: two union chunks (the second may be empty)
-                    const int c0 = next_bit(bm, nwords, cur + 1);
-                    const int c1 = next_bit(bm, nwords, c0 + 1);
-                    cur = c1 >= 0 ? c1 : c0;
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int c = hh == 0 ? c0 : c1;
-                        const bool sel = row_ok && c >= 0 && qc[0] == c;
-                        float wgt = 0.f;
-                        if (sel) {
-                            wgt = ex2(qs[0] - m_used);
-                            l += wgt;
-                            qc[0] = qc[1];
-                            qs[0] = qs[1];
-                            qc[1] = qc[2];
-                            qs[1] = qs[2];
-                            qc[2] = qc[3];
-                            qs[2] = qs[3];
-                            qc[3] = kn < nsel ? __ldg(&ip[kn]) : INT_MAX;
-                            qs[3] = kn < nsel ? __ldg(&sp[kn]) * kLog2e : 0.f;
-                            ++kn;
+                    // ---- chunk tile: the next chunk of the union
+                    cur = next_bit(bm, nwords, cur + 1);
+                    const int c = cur;
+                    const bool sel = row_ok && c >= 0 && qc[0] == c;
+                    float wgt = 0.f;
+                    if (sel) {
+                        wgt = exp2_fma(qs[0] - m_used);  // no MUFU: it would queue behind the exp bursts
+                        l += wgt;
+                        qc[0] = qc[1];
+                        qs[0] = qs[1];
+                        qc[1] = qc[2];
+                        qs[1] = qs[2];
+                        qc[2] = qc[3];
+                        qs[2] = qs[3];
+                        qc[3] = INT_MAX;
+                        qs[3] = 0.f;
+                        if (kn < nsel) {
+                            qc[3] = ldg_early(ip + kn);
+                            qs[3] = ldg_early(sp + kn) * kLog2e;
                         }
-                        if (__any_sync(kFull, sel)) {
-                            tmem_ld32(s_col + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                            tmem_ld32(s_col + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                            tmem_wait_ld();
-                            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+                        ++kn;
+                    }
+                    any = __any_sync(kFull, sel);
+                    if (any) {
+                        tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                        tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                        tmem_wait_ld();
+                    }
+                    if (any) {
+                        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-                            for (int q = 0; q < 64; q += 8) {
-                                m0 = max3(m0, __uint_as_float(sr[q]), __uint_as_float(sr[q + 1]));
-                                m1 = max3(m1, __uint_as_float(sr[q + 2]), __uint_as_float(sr[q + 3]));
-                                m2 = max3(m2, __uint_as_float(sr[q + 4]), __uint_as_float(sr[q + 5]));
-                                m3 = max3(m3, __uint_as_float(sr[q + 6]), __uint_as_float(sr[q + 7]));
-                            }
-                            const float nb = -fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * scale2;
-                            float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
-#pragma unroll
-                            for (int q = 0; q < 64; q += 4) {
-                                const float e0 = ex2(fmaf(__uint_as_float(sr[q]), scale2, nb));
-                                const float e1 = ex2(fmaf(__uint_as_float(sr[q + 1]), scale2, nb));
-                                const float e2 = ex2(fmaf(__uint_as_float(sr[q + 2]), scale2, nb));
-                                const float e3 = ex2(fmaf(__uint_as_float(sr[q + 3]), scale2, nb));
-                                z0 += e0;
-                                z1 += e1;
-                                z2 += e2;
-                                z3 += e3;
-                                sr[q] = __float_as_uint(e0);
-                                sr[q + 1] = __float_as_uint(e1);
-                                sr[q + 2] = __float_as_uint(e2);
-                                sr[q + 3] = __float_as_uint(e3);
-                            }
-                            const float z = (z0 + z1) + (z2 + z3);
-                            const float fw = sel ? __fdividef(wgt, z) : 0.f;  // z >= 1: the max term is 1
-#pragma unroll
-                            for (int q = 0; q < 32; ++q)
-                                pk[q] = pack_bf16(__uint_as_float(sr[2 * q]) * fw, __uint_as_float(sr[2 * q + 1]) * fw);
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < 32; ++q) pk[q] = 0u;
+                        for (int q = 0; q < 64; q += 8) {
+                            m0 = max3(m0, __uint_as_float(sr[q]), __uint_as_float(sr[q + 1]));
+                            m1 = max3(m1, __uint_as_float(sr[q + 2]), __uint_as_float(sr[q + 3]));
+                            m2 = max3(m2, __uint_as_float(sr[q + 4]), __uint_as_float(sr[q + 5]));
+                            m3 = max3(m3, __uint_as_float(sr[q + 6]), __uint_as_float(sr[q + 7]));
                         }
-                        tmem_st32(s_col + hh * 32, pk);
+                        const float nb = -fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * scale2;
+                        float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+#pragma unroll
+                        for (int q = 0; q < 64; q += 4) {
+                            const float e0 = ex2(fmaf(__uint_as_float(sr[q]), scale2, nb));
+                            const float e1 = ex2(fmaf(__uint_as_float(sr[q + 1]), scale2, nb));
+                            const float e2 = ex2(fmaf(__uint_as_float(sr[q + 2]), scale2, nb));
+                            const float e3 = ex2(fmaf(__uint_as_float(sr[q + 3]), scale2, nb));
+                            z0 += e0;
+                            z1 += e1;
+                            z2 += e2;
+                            z3 += e3;
+                            sr[q] = __float_as_uint(e0);
+                            sr[q + 1] = __float_as_uint(e1);
+                            sr[q + 2] = __float_as_uint(e2);
+                            sr[q + 3] = __float_as_uint(e3);
+                        }
+                        // z >= 1 (the max term is 1): its reciprocal on the FMA pipe
+                        const float fw = sel ? wgt * recip_newton((z0 + z1) + (z2 + z3)) : 0.f;
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            sr[q] = pack_bf16(__uint_as_float(sr[2 * q]) * fw, __uint_as_float(sr[2 * q + 1]) * fw);
                     }
                 }
+                if (!ok) break;
+                if (!any) {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) sr[q] = 0u;
+                }
+                tmem_st32(s_col, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
                 tmem_wait_st();
                 tc_fence_before();
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar(kBarPfull + x)) : "memory");
+                __syncwarp();
+                if (lane == 0) arrive(bar(kBarPfull + 2 * x + bsel));
             }
             // ---- epilogue: O / l and lse
-            if (ok && nt > 0) ok = wait_warp(bar(kBarOdone + x), (g - 1) & 1);
+            if (ok && nt > 0) ok = wait_warp(bar(kBarPVdone + 2 * x + ((g - 1) & 1)), ((g - 1) >> 1) & 1);
             if (!ok) break;
             tc_fence_after();
             bf16 *orow = static_cast<bf16 *>(a.O.ptr) + it.b * a.O.sb + it.h * a.O.sh + (int64_t)t * a.O.st;
@@ -646,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             }
             if (row_ok && a.lse) a.lse[qrow] = l > 0.f ? (m_used + log2f(l)) / kLog2e : -INFINITY;
             tc_fence_before();
-            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar(kBarMapFree + par)) : "memory");
+            arrive(bar(kBarMapFree + par));
         }
     }
 
@@ -667,8 +685,8 @@ bool attend_prefill_tc_supported(hils_dtype dt, int d, int N) {
 
 hils_status launch_attend_prefill_tc(const AttendArgs &a, int N, uint32_t *status, cudaStream_t s) {
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, a.Q, a.B, a.H, N, kM) || !make_map(&mk, a.K, a.B, a.H, N, kHalf) ||
-        !make_map(&mv, a.V, a.B, a.H, N, kHalf))
+    if (!make_map(&mq, a.Q, a.B, a.H, N, kM) || !make_map(&mk, a.K, a.B, a.H, N, kTile) ||
+        !make_map(&mv, a.V, a.B, a.H, N, kTile))
         return HILS_ERR_CUDA;
     static KernelSetup setup;
     int per_sm = 0;
