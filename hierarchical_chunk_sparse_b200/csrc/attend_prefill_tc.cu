@@ -12,11 +12,12 @@
 //   2. the union of the chunks kept by the item's 256 queries, ascending, one chunk per
 //      tile; a row that kept chunk c weights that chunk's own softmax by exp(s^_c), a
 //      row that did not contributes zero.
-// Warp roles (352 threads), all hand-offs through mbarriers:
+// Warp roles (384 threads), all hand-offs through mbarriers:
 //   warps 0-3  softmax of tile A (thread = row = TMEM lane), warps 4-7 softmax of B;
 //   warp 8     TMA loads (Q of both tiles; K and V of each key tile, 4-slot rings);
-//   warp 9     tcgen05.mma issue: S_X = Q_X K^T (M=128, N=64, K=128) into TMEM, then
-//              O_X += P_X V (M=128, N=128, K=64, the A operand P_X read from TMEM);
+//   warps 9/11 tcgen05.mma issue for tile A / tile B: S_X = Q_X K^T (M=128, N=64, K=128)
+//              into TMEM, then O_X += P_X V (M=128, N=128, K=64, the A operand P_X read
+//              from TMEM); one issuer per tile, so that neither waits on the other's rows;
 //   warp 10    builds the next item's union bitmap while the others work.
 // S is double-buffered per query tile and P_X(i) is written over S_X(i) (its first 32
 // columns): S_X(i+1) is computed while the softmax of tile i runs. A later MMA is not
@@ -43,8 +44,8 @@ constexpr int kRows = 2 * kM;    // query rows per work item
 constexpr int kTile = 64;        // keys per tile (= chunk size)
 constexpr int kHead = 128;       // head dimension
 constexpr int kSoftmaxWarps = 8;
-constexpr int kLoadWarp = 8, kMmaWarp = 9, kMapWarp = 10;
-constexpr int kThreads = 352;
+constexpr int kLoadWarp = 8, kMmaWarp = 9, kMapWarp = 10, kMmaWarpB = 11;
+constexpr int kThreads = 384;
 constexpr int kStages = 4;       // K/V ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxBitmapWords = 256;  // union bitmap: up to 8192 chunks
@@ -73,10 +74,10 @@ enum {
                          //   issued before it) completed
     kBarMapReady = 30,   // + item parity
     kBarMapFree = 32,    // + item parity
-    kBarDrain = 34,
-    kNumBars = 35
+    kBarDrain = 34,      // + issuer (A, B)
+    kNumBars = 36
 };
-constexpr uint32_t kMapFreeCount = kSoftmaxWarps * 32 + 2;  // softmax rows + load warp + MMA warp
+constexpr uint32_t kMapFreeCount = kSoftmaxWarps * 32 + 3;  // softmax rows + load warp + 2 MMA warps
 
 struct TcArgs {
     AttendArgs a;
@@ -195,6 +196,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         for (int i = 0; i < kNumBars; ++i) {
             uint32_t cnt = 1;
             if (i >= kBarPfull && i < kBarPfull + 4) cnt = 4;  // one elected lane per softmax warp
+            if (i == kBarQfree || (i >= kBarKfree && i < kBarKfree + kStages) ||
+                (i >= kBarVfree && i < kBarVfree + kStages))
+                cnt = 2;  // both MMA issuers release shared operands
             if (i == kBarMapReady || i == kBarMapReady + 1) cnt = 32;
             if (i == kBarMapFree || i == kBarMapFree + 1) cnt = kMapFreeCount;
             mbar_init(bar(i), cnt);
@@ -353,8 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
                 drain(bar(kBarVfull + s), issuedV > s ? (issuedV - s + kStages - 1) / kStages : 0);
             }
         }
-    } else if (warp == kMmaWarp) {
-        // ---------------------------------------------------------------- MMA issue
+    } else if (warp == kMmaWarp || warp == kMmaWarpB) {
+        // ---------------------------------------------------------------- MMA issue (tile xm)
+        const int xm = warp == kMmaWarp ? 0 : 1;
         const uint32_t idS = idesc_bf16(kM, kTile, false);
         const uint32_t idPV = idesc_bf16(kM, kHead, true);
         auto issue_s = [&](int x, int gt) {  // S_x(gt) = Q_x K^T into buffer gt % 2
@@ -397,16 +402,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             if (!(ok = wait_warp(bar(kBarQfull), qn & 1))) break;
             ++qn;
             tc_fence_after();
-            // S of the item's first tile, then per tile: S of the next, PV of this one
-            auto s_pair = [&](int gt, bool last) -> bool {
+            auto s_one = [&](int gt, bool last) -> bool {  // S_xm(gt)
                 if (!wait_warp(bar(kBarKfull + gt % kStages), (gt / kStages) & 1)) return false;
-                if (!s_free(0, gt)) return false;
-                tc_fence_after();
-                if (lane == 0) issue_s(0, gt);
-                if (!s_free(1, gt)) return false;
+                if (!s_free(xm, gt)) return false;
                 tc_fence_after();
                 if (lane == 0) {
-                    issue_s(1, gt);
+                    issue_s(xm, gt);
                     mma_commit(bar(kBarKfree + gt % kStages));
                     if (last) mma_commit(bar(kBarQfree));
                 }
@@ -414,28 +415,25 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
                 return true;
             };
             // S of the item's first two tiles, then per tile: PV of this one, S of the one two ahead
-            if (!(ok = s_pair(g, nt == 1))) break;
-            if (nt > 1 && !(ok = s_pair(g + 1, nt == 2))) break;
+            if (!(ok = s_one(g, nt == 1))) break;
+            if (nt > 1 && !(ok = s_one(g + 1, nt == 2))) break;
             for (int i = 0; i < nt; ++i, ++g) {
-                if (!(ok = wait_warp(bar(kBarPfull + (g & 1)), (g >> 1) & 1))) break;
+                if (!(ok = wait_warp(bar(kBarPfull + 2 * xm + (g & 1)), (g >> 1) & 1))) break;
                 if (!(ok = wait_warp(bar(kBarVfull + g % kStages), (g / kStages) & 1))) break;
                 tc_fence_after();
-                if (lane == 0) issue_pv(0, g, i > 0);
-                if (!(ok = wait_warp(bar(kBarPfull + 2 + (g & 1)), (g >> 1) & 1))) break;
-                tc_fence_after();
                 if (lane == 0) {
-                    issue_pv(1, g, i > 0);
+                    issue_pv(xm, g, i > 0);
                     mma_commit(bar(kBarVfree + g % kStages));
                 }
                 __syncwarp();
-                if (i + 2 < nt && !(ok = s_pair(g + 2, i + 3 == nt))) break;
+                if (i + 2 < nt && !(ok = s_one(g + 2, i + 3 == nt))) break;
             }
         }
         // every MMA this warp issued completes before TMEM and shared memory are released
         if (lane == 0) {
-            mma_commit(bar(kBarDrain));
+            mma_commit(bar(kBarDrain + xm));
             for (long long it = 0; it < kWaitLimit; ++it)
-                if (mbar_try_wait(bar(kBarDrain), 0)) break;
+                if (mbar_try_wait(bar(kBarDrain + xm), 0)) break;
         }
         __syncwarp();
     } else {
