@@ -264,8 +264,9 @@ class DecodeBench:
 
 # ----------------------------------------------------------------- prefill workload
 
-def prefill_flops(w) -> float:
-    """Algorithmic flops of summarise + score + chunk attention + window (per batch)."""
+def prefill_flops(w, part: str = "step") -> float:
+    """Algorithmic flops of one prefill (per batch): the whole step (summarise + score +
+    chunk attention + window) or only the attend's share (chunk attention + window)."""
     d, S, K, W, N, C = w.d, w.S, w.K, w.W, w.N, w.C
     score = chunk = win = 0
     for i in range(N):
@@ -274,7 +275,15 @@ def prefill_flops(w) -> float:
         chunk += 4 * d * S * min(K, e)
         win += 4 * d * min(W, i + 1)
     summ = 4 * d * S * C
-    return float(w.B * w.H * (score + chunk + win + summ))
+    total = chunk + win if part == "attend" else score + chunk + win + summ
+    return float(w.B * w.H * total)
+
+
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) that Nsight Compute
+# measured for the current kernels, each with its command in profiles/: select_decode512k.md
+# (screen + pick of one select call), attend_decode_128k.md, attend_prefill_tc_prefill8k.md.
+# A kernel that changes after its capture reports null here until it is captured again.
+MEASURED_TRAFFIC = {"select": 69_300_992, "attend_decode": 25_235_968, "attend_prefill": 666_330_112}
 
 
 class PrefillBench:
@@ -542,7 +551,8 @@ def main():
                 pb.step()
         stream.synchronize()
         n = max(3, min(args.steps, 20))
-        pt = statistics.mean(time_steps(graphed(pb.step, stream), n, flush, stream))
+        with ClockSampler(dev) as pclk:
+            pt = statistics.mean(time_steps(graphed(pb.step, stream), n, flush, stream))
         pt = max_over_ranks(pt, world, dev)
         ks = {k: statistics.mean(time_steps(graphed(getattr(pb, k), stream), n, flush, stream))
               for k in ("summarize", "select", "attend")}
@@ -550,11 +560,17 @@ def main():
         pb.check_status()
         fl = prefill_flops(wp)
         tf = fl / (pt * 1e-3) / 1e12
+        fl_att = prefill_flops(wp, "attend")
+        tf_att = fl_att / (ks["attend"] * 1e-3) / 1e12
         prefill = {"value": tf * world, "unit": "TFLOP/s", "ms_per_step": pt, "workload": wp.name,
                    "algorithmic_gflop_per_step": fl / 1e9, "steps": n,
-                   "kernel_ms": ks,
-                   "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
-                                "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"], "traffic": None,
+                   "kernel_ms": ks, "clocks": pclk.summary(),
+                   "step_frac_of_peak": tf / peaks["bf16_tflops"],
+                   "roofline": {"bound": "tensor", "kernel": "attend", "achieved": tf_att,
+                                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                "frac": tf_att / peaks["bf16_tflops"],
+                                "traffic": MEASURED_TRAFFIC["attend_prefill"],
+                                "algorithmic_gflop": fl_att / 1e9,
                                 "peak_source": f"{peak_src} bf16 dense (burst)"}}
         del pb
         torch.cuda.empty_cache()
@@ -572,7 +588,8 @@ def main():
                        "top_k": w.K, "window": w.W, "parallelism": f"replicas{world}",
                        "l2": "flushed before every step (2x L2 write)"},
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom[0], "peak": hbm,
-                         "unit": "GB/s", "frac": dom[0] / hbm, "traffic": None,
+                         "unit": "GB/s", "frac": dom[0] / hbm,
+                         "traffic": MEASURED_TRAFFIC[dominant if dominant == "select" else "attend_decode"],
                          "algorithmic_bytes": dom[1], "peak_source": f"{peak_src} HBM copy"},
             "step_roofline": {"bytes": by["step"], "achieved_gbs": step_gbs, "frac_measured": step_gbs / hbm,
                               "frac_8tbs": step_gbs / 8000.0},
