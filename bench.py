@@ -128,14 +128,21 @@ class ClockSampler:
 # ----------------------------------------------------------------- timing helpers
 
 class Flusher:
-    """Writes a buffer of twice the L2 size, so that no step starts with warm L2."""
+    """Writes a buffer of twice the L2 size, then reads another of twice the L2 size, so
+    that no step starts with warm L2, nor with the flush's dirty lines still to be written
+    back (which would charge the step with 126 MB of write-backs it did not cause)."""
+
+    DESCRIPTION = "flushed before every step: 2x L2 written, then 2x L2 read"
 
     def __init__(self, dev):
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         self.buf = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+        self.rbuf = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
 
     def __call__(self):
         self.buf.fill_(1.0)
+        torch.sum(self.rbuf, dim=0, out=self.sink)
 
 
 def time_steps(fn, steps, flush, stream):
@@ -586,7 +593,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "kv_len": w.N, "chunk": w.S,
                        "top_k": w.K, "window": w.W, "parallelism": f"replicas{world}",
-                       "l2": "flushed before every step (2x L2 write)"},
+                       "l2": Flusher.DESCRIPTION},
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom[0], "peak": hbm,
                          "unit": "GB/s", "frac": dom[0] / hbm,
                          "traffic": MEASURED_TRAFFIC[dominant if dominant == "select" else "attend_decode"],
