@@ -469,6 +469,54 @@ def run_profile_case(args):
     print(json.dumps({"profile_case": case, "launches": args.warmup + args.steps}))
 
 
+def mean_item_union(idx: torch.Tensor, nsel: torch.Tensor, C: int) -> float:
+    """Mean number of distinct chunks kept by the queries of one 256-query work item."""
+    B, H, N, K = idx.shape
+    nb = N // 256
+    if nb == 0:
+        return 0.0
+    i = idx[:, :, : nb * 256].reshape(B, H, nb, 256 * K).long()
+    keep = (torch.arange(K, device=idx.device).view(1, 1, 1, K) < nsel[:, :, : nb * 256, None]).reshape(B, H, nb, 256 * K)
+    bits = torch.zeros(B, H, nb, C + 1, dtype=torch.int32, device=idx.device)
+    bits.scatter_(3, torch.where(keep & (i >= 0), i, torch.full_like(i, C)), 1)
+    return float(bits[..., :C].sum(-1).float().mean())
+
+
+def measure_prefill(wp, dev, stream, flush, args, world, peaks, peak_src, traffic):
+    """One prefill workload: step and per-kernel times (L2 flushed), TFLOP/s, roofline of
+    the attend kernel, mean chunk union per 256-query item."""
+    pb = PrefillBench(wp, dev)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            pb.step()
+    stream.synchronize()
+    n = max(3, min(args.steps, 20))
+    with ClockSampler(dev) as pclk:
+        pt = statistics.mean(time_steps(graphed(pb.step, stream), n, flush, stream))
+    pt = max_over_ranks(pt, world, dev)
+    ks = {k: statistics.mean(time_steps(graphed(getattr(pb, k), stream), n, flush, stream))
+          for k in ("summarize", "select", "attend")}
+    torch.cuda.synchronize()
+    pb.check_status()
+    fl = prefill_flops(wp)
+    tf = fl / (pt * 1e-3) / 1e12
+    fl_att = prefill_flops(wp, "attend")
+    tf_att = fl_att / (ks["attend"] * 1e-3) / 1e12
+    out = {"value": tf * world, "unit": "TFLOP/s", "ms_per_step": pt, "workload": wp.name,
+           "algorithmic_gflop_per_step": fl / 1e9, "steps": n,
+           "kernel_ms": ks, "clocks": pclk.summary(),
+           "step_frac_of_peak": tf / peaks["bf16_tflops"],
+           "mean_item_union_chunks": mean_item_union(pb.idx, pb.nsel, wp.C),
+           "roofline": {"bound": "tensor", "kernel": "attend", "achieved": tf_att,
+                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": tf_att / peaks["bf16_tflops"], "traffic": traffic,
+                        "algorithmic_gflop": fl_att / 1e9,
+                        "peak_source": f"{peak_src} bf16 dense (burst)"}}
+    del pb
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None,
@@ -548,39 +596,13 @@ def main():
     del db
     torch.cuda.empty_cache()
 
-    # ---------------- prefill @8K
+    # ---------------- prefill @8K (iid queries; and the query-locality variant)
     prefill = None
+    prefill_local = None
     if not args.no_prefill:
-        wp = WORKLOADS[2]
-        pb = PrefillBench(wp, dev)
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                pb.step()
-        stream.synchronize()
-        n = max(3, min(args.steps, 20))
-        with ClockSampler(dev) as pclk:
-            pt = statistics.mean(time_steps(graphed(pb.step, stream), n, flush, stream))
-        pt = max_over_ranks(pt, world, dev)
-        ks = {k: statistics.mean(time_steps(graphed(getattr(pb, k), stream), n, flush, stream))
-              for k in ("summarize", "select", "attend")}
-        torch.cuda.synchronize()
-        pb.check_status()
-        fl = prefill_flops(wp)
-        tf = fl / (pt * 1e-3) / 1e12
-        fl_att = prefill_flops(wp, "attend")
-        tf_att = fl_att / (ks["attend"] * 1e-3) / 1e12
-        prefill = {"value": tf * world, "unit": "TFLOP/s", "ms_per_step": pt, "workload": wp.name,
-                   "algorithmic_gflop_per_step": fl / 1e9, "steps": n,
-                   "kernel_ms": ks, "clocks": pclk.summary(),
-                   "step_frac_of_peak": tf / peaks["bf16_tflops"],
-                   "roofline": {"bound": "tensor", "kernel": "attend", "achieved": tf_att,
-                                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                "frac": tf_att / peaks["bf16_tflops"],
-                                "traffic": MEASURED_TRAFFIC["attend_prefill"],
-                                "algorithmic_gflop": fl_att / 1e9,
-                                "peak_source": f"{peak_src} bf16 dense (burst)"}}
-        del pb
-        torch.cuda.empty_cache()
+        prefill = measure_prefill(WORKLOADS[2], dev, stream, flush, args, world, peaks, peak_src,
+                                  MEASURED_TRAFFIC["attend_prefill"])
+        prefill_local = measure_prefill(WORKLOADS[6], dev, stream, flush, args, world, peaks, peak_src, None)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -607,6 +629,7 @@ def main():
             "gpu_launches": launches,
             "clocks": clk.summary(),
             "prefill": prefill,
+            "prefill_local": prefill_local,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

@@ -15,6 +15,11 @@ Workloads (one attention layer; chunk size S = 64 everywhere):
                          key per head whose logit against the query is 8.
   5 decode bf16 1M:      B1 H32 d128, KV cache 1048576, K32 W1024; as 4 with four
                          needles per head in distinct chunks.
+  6 prefill bf16 8K with query locality: as 2, except that Q_cal changes slowly along
+                         the sequence: Q_cal[t] = (u[t // 256] + 0.25 e[t]) / sqrt(d), with
+                         u one N(0,1) vector per 256-token block and e iid N(0,1), so that
+                         adjacent queries keep overlapping chunk sets (the regime in which
+                         the query-packing kernel shares chunks between queries).
 bf16 tensors are drawn in float32 and rounded to nearest-even.
 
 Seeds: base 20260709; the tensor with id k of workload n uses base + 100 n + k,
@@ -49,6 +54,8 @@ class Workload:
     qkv_scaled: bool = False  # Q, Q_cal, K, V divided by sqrt(d)
     needles: int = 0  # planted needle keys per (b, h)
     needle_logit: float = 8.0
+    qcal_block: int = 0  # > 0: Q_cal = block base vector + qcal_noise * iid noise
+    qcal_noise: float = 0.0
 
     @property
     def C(self) -> int:
@@ -73,6 +80,8 @@ WORKLOADS = {
                 torch.bfloat16, needles=1),
     5: Workload(5, "decode_bf16_1m", "decode", 1, 32, 128, 64, 32, 1024, 1048576,
                 torch.bfloat16, needles=4),
+    6: Workload(6, "prefill_bf16_8k_local", "prefill", 1, 32, 128, 64, 16, 512, 8192,
+                torch.bfloat16, qkv_scaled=True, qcal_block=256, qcal_noise=0.25),
 }
 
 
@@ -94,7 +103,13 @@ def make_prefill(w: Workload, device="cpu") -> dict:
     for name, shape, scaled in (("Q", (B, H, N, d), True), ("Qcal", (B, H, N, d), True),
                                 ("LQ", (B, H, C, d), False), ("K", (B, H, N, d), True),
                                 ("V", (B, H, N, d), True)):
-        x = _randn(shape, _gen(w, name, device), device)
+        g = _gen(w, name, device)
+        if name == "Qcal" and w.qcal_block > 0:
+            nb = (N + w.qcal_block - 1) // w.qcal_block
+            base = _randn((B, H, nb, d), g, device)
+            x = base.repeat_interleave(w.qcal_block, dim=2)[:, :, :N] + w.qcal_noise * _randn(shape, g, device)
+        else:
+            x = _randn(shape, g, device)
         if scaled and s != 1.0:
             x = x * s
         out[name] = x.to(w.dtype)

@@ -402,6 +402,29 @@ def test_attend_prefill_full_size(oracle, cuda_device):
         assert_close(lse[:, sl], lse_ref, torch.float32, f"lse head {h}")
 
 
+def test_prefill_query_locality_workload(oracle, cuda_device):
+    """The 8K prefill with slowly changing Q_cal (adjacent queries keep overlapping chunk
+    sets), four heads: selection bit-exact, outputs within tolerance, and each
+    256-query item's union of kept chunks far below the eligible count, which is the
+    regime of the query-packing kernel."""
+    w = WORKLOADS[6].replace(H=4)
+    inp = make_prefill(w)
+    d = to_dev(inp, cuda_device)
+    Ksum, Bsum = gpu_summarize(w, d["K"], d["LQ"])
+    idx, score, nsel = gpu_select(w, d["Qcal"], Ksum, Bsum)
+    i_ref, s_ref, n_ref = oracle.select(inp["Qcal"], host(Ksum), host(Bsum), 64, w.K, w.scale)
+    assert_same_selection(idx, nsel, i_ref, n_ref, "local")
+    scores_close(score, s_ref, n_ref, "local")
+    O, lse = gpu_prefill(w, d["Q"], d["K"], d["V"], idx, score, nsel)
+    O_ref, lse_ref = oracle.attend(inp["Q"], inp["K"], inp["V"], host(idx), host(score), host(nsel),
+                                   64, w.W, w.scale)
+    assert_close(O, O_ref, w.dtype, "O")
+    assert_close(lse, lse_ref, torch.float32, "lse")
+    ih = host(idx).reshape(w.B, w.H, w.N // 256, 256 * w.K).numpy()
+    unions = [len(set(r.tolist()) - {-1}) for r in ih.reshape(-1, 256 * w.K)[w.H:]]  # items past the first
+    assert np.mean(unions) < 40, np.mean(unions)
+
+
 def _decode_small(cuda_device, lens=(5000, 3001), K=16, W=512, H=3):
     w = WORKLOADS[4].replace(B=len(lens), H=H, N=max(lens), K=K, W=W, needles=0)
     inp = make_decode(w)
