@@ -62,10 +62,10 @@ def _load():
         i, d_, p = ctypes.c_int, ctypes.c_double, ctypes.c_void_p
         lib.or_set_threads.argtypes = [i]
         lib.or_get_threads.restype = i
-        lib.or_summarize.argtypes = [i, i, i, i, d_, T, i, T, p, p]
+        lib.or_summarize.argtypes = [i, i, i, i, i, d_, T, i, T, p, p]
         lib.or_score_all.argtypes = [i, i, i, i, d_, T, i, p, T, T, i, p]
-        lib.or_select.argtypes = [i, i, i, i, i, d_, T, i, p, T, T, i, p, p, p]
-        lib.or_attend.argtypes = [i, i, i, i, i, i, d_, T, i, p, T, T, p, T, p, p, p]
+        lib.or_select.argtypes = [i, i, i, i, i, i, d_, T, i, p, T, T, i, p, p, p]
+        lib.or_attend.argtypes = [i, i, i, i, i, i, i, d_, T, i, p, T, T, p, T, p, p, p]
         lib.or_brute_weights.argtypes = [i, i, i, i, i, d_, T, i, i, i, i, T, p, T,
                                          ctypes.c_longlong, i, p]
         lib.or_chunk_logmass.argtypes = [i, i, i, i, i, d_, T, i, T, p, p, p]
@@ -116,13 +116,22 @@ def get_threads() -> int:
     return int(_load().or_get_threads())
 
 
+def _group(h_query: int, h_kv: int) -> int:
+    if h_kv <= 0 or h_query % h_kv != 0:
+        raise ValueError(f"{h_query} query heads do not form groups over {h_kv} key-value heads")
+    return h_query // h_kv
+
+
 def summarize(K: torch.Tensor, LQ: torch.Tensor, S: int, scale: float):
-    """Eq. 8 summaries. Returns (Ksum [B,H,C,d], Bsum [B,H,C]) in float64."""
-    B, H, N, d = K.shape
+    """Eq. 8 summaries of every query head (LQ [B,H,C,d]) over the keys of its key-value
+    head (K [B,H/G,N,d]). Returns (Ksum [B,H,C,d], Bsum [B,H,C]) in float64."""
+    B, Hk, N, d = K.shape
+    H = LQ.shape[1]
+    G = _group(H, Hk)
     C = N // S
     ksum = np.zeros((B, H, C, d), np.float64)
     bsum = np.zeros((B, H, C), np.float64)
-    _check(_load().or_summarize(B, H, d, S, float(scale), _desc(K), N, _desc(LQ),
+    _check(_load().or_summarize(B, H, G, d, S, float(scale), _desc(K), N, _desc(LQ),
                                 _ptr(ksum), _ptr(bsum)), "summarize")
     return ksum, bsum
 
@@ -144,34 +153,39 @@ def score_all(Qcal, Ksum, Bsum, S: int, scale: float, qpos=None):
     return out
 
 
-def select(Qcal, Ksum, Bsum, S: int, K: int, scale: float, qpos=None):
-    """Top-K selection. Returns (idx int32, score float64, nsel int32)."""
+def select(Qcal, Ksum, Bsum, S: int, K: int, scale: float, qpos=None, group: int = 1):
+    """Top-K selection, shared by each group of `group` consecutive query heads.
+    Returns (idx int32 [B,H/G,Lq,K], score float64 [B,H,Lq,K], nsel int32 [B,H/G,Lq])."""
     Qcal, Ksum, Bsum = _as_tensor(Qcal), _as_tensor(Ksum), _as_tensor(Bsum)
     B, H, Lq, d = Qcal.shape
+    G = _group(H, H // group if group > 0 and H % group == 0 else 0)
     C = Ksum.shape[2]
-    idx = np.zeros((B, H, Lq, K), np.int32)
+    idx = np.zeros((B, H // G, Lq, K), np.int32)
     score = np.zeros((B, H, Lq, K), np.float64)
-    nsel = np.zeros((B, H, Lq), np.int32)
+    nsel = np.zeros((B, H // G, Lq), np.int32)
     qp = None if qpos is None else _i32(qpos)
-    _check(_load().or_select(B, H, d, S, K, float(scale), _desc(Qcal), Lq,
+    _check(_load().or_select(B, H, G, d, S, K, float(scale), _desc(Qcal), Lq,
                              None if qp is None else _ptr(qp), _desc(Ksum), _desc(Bsum), C,
                              _ptr(idx), _ptr(score), _ptr(nsel)), "select")
     return idx, score, nsel
 
 
 def attend(Q, Kc, Vc, idx, score, nsel, S: int, W: int, scale: float, qpos=None):
-    """Eq. 10 output. Returns (O [B,H,Lq,d] float64, lse [B,H,Lq] float64)."""
+    """Eq. 10 output for query heads Q [B,H,Lq,d] over key-value heads Kc, Vc [B,H/G,L,d]
+    with the groups' kept chunks idx [B,H/G,Lq,K], nsel [B,H/G,Lq] and each head's scores
+    [B,H,Lq,K]. Returns (O [B,H,Lq,d] float64, lse [B,H,Lq] float64)."""
     Q, Kc, Vc = _as_tensor(Q), _as_tensor(Kc), _as_tensor(Vc)
     B, H, Lq, d = Q.shape
+    G = _group(H, Kc.shape[1])
     idx = _i32(idx)
     K = idx.shape[-1]
-    idx = idx.reshape(B, H, Lq, K)
+    idx = idx.reshape(B, H // G, Lq, K)
     score = _as_tensor(score).reshape(B, H, Lq, K).contiguous()
-    nsel = _i32(nsel).reshape(B, H, Lq)
+    nsel = _i32(nsel).reshape(B, H // G, Lq)
     O = np.zeros((B, H, Lq, d), np.float64)
     lse = np.zeros((B, H, Lq), np.float64)
     qp = None if qpos is None else _i32(qpos)
-    _check(_load().or_attend(B, H, d, S, K, W, float(scale), _desc(Q), Lq,
+    _check(_load().or_attend(B, H, G, d, S, K, W, float(scale), _desc(Q), Lq,
                              None if qp is None else _ptr(qp), _desc(Kc), _desc(Vc),
                              _ptr(idx), _desc(score), _ptr(nsel), _ptr(O), _ptr(lse)), "attend")
     return O, lse

@@ -29,6 +29,12 @@
  *   - top-K ties go to the lower chunk index; the kept list is reported in
  *     ascending chunk index.
  *   - a query with no selected chunk and an empty window gets o = 0, lse = -inf.
+ *   - grouped-query attention ([summary] Methodology 3, GQA adaptation): H query heads
+ *     share H / G key-value heads, query head h reading key-value head h / G. Each query
+ *     head has its own landmark queries, summaries and chunk scores; a group's G heads
+ *     keep the same chunks, the top K of max over the group of s^_{h,i,c} (ties to the
+ *     lower index); each head weights the kept chunks with its own s^_{h,i,c} in Eq. 10.
+ *     G = 1 is plain multi-head attention.
  *
  * Arithmetic: every stored element is widened exactly to double. All sums run in
  * index order; the file must be compiled without floating-point contraction
@@ -104,10 +110,10 @@ static int eligible_chunks(int t, int S, int C) {
 
 /* --------------------------------------------------------------- Eq. 8 summaries */
 
-int or_summarize(int B, int H, int d, int S, double scale,
+int or_summarize(int B, int H, int G, int d, int S, double scale,
                  or_tensor K, int N, or_tensor LQ,
                  double *Ksum, double *Bsum) {
-    if (B < 0 || H < 0 || d <= 0 || S <= 0 || N < 0) return -1;
+    if (B < 0 || H < 0 || G <= 0 || H % G != 0 || d <= 0 || S <= 0 || N < 0) return -1;
     if (!valid_dtype(&K) || !valid_dtype(&LQ) || !Ksum || !Bsum) return -1;
     const int C = N / S;
     const long long units = (long long)B * H * C;
@@ -125,10 +131,11 @@ int or_summarize(int B, int H, int d, int S, double scale,
             const int b = (int)(u / ((long long)C * H));
             load_vec(&LQ, b, h, c, d, lq);
 
-            /* landmark logits l_j = (q'_c . k_j) / sqrt(d) over the chunk's S keys */
+            /* landmark logits l_j = (q'_c . k_j) / sqrt(d) over the chunk's S keys (of the
+               query head's key-value head h / G) */
             double m = -INFINITY;
             for (int j = 0; j < S; ++j) {
-                load_vec(&K, b, h, (long long)c * S + j, d, kj);
+                load_vec(&K, b, h / G, (long long)c * S + j, d, kj);
                 logit[j] = dot(lq, kj, d) * scale;
                 if (logit[j] > m) m = logit[j];
             }
@@ -142,7 +149,7 @@ int or_summarize(int B, int H, int d, int S, double scale,
             double entropy = 0.0;
             for (int j = 0; j < S; ++j) {
                 const double p = exp(logit[j] - m) / z;
-                load_vec(&K, b, h, (long long)c * S + j, d, kj);
+                load_vec(&K, b, h / G, (long long)c * S + j, d, kj);
                 for (int x = 0; x < d; ++x) ks[x] += p * kj[x];
                 if (p > 0.0) entropy -= p * log(p);
             }
@@ -212,39 +219,51 @@ static int by_index(const void *pa, const void *pb) {
     return (a->c > b->c) - (a->c < b->c);
 }
 
-int or_select(int B, int H, int d, int S, int K, double scale,
+int or_select(int B, int H, int G, int d, int S, int K, double scale,
               or_tensor Qcal, int Lq, const int *qpos,
               or_tensor Ksum, or_tensor Bsum, int C,
               int *idx, double *score, int *nsel) {
-    if (B < 0 || H < 0 || d <= 0 || S <= 0 || K < 0 || Lq < 0 || C < 0) return -1;
+    if (B < 0 || H < 0 || G <= 0 || H % G != 0 || d <= 0 || S <= 0 || K < 0 || Lq < 0 || C < 0) return -1;
     if (!valid_dtype(&Qcal) || !idx || !score || !nsel) return -1;
     if (C > 0 && (!valid_dtype(&Ksum) || !valid_dtype(&Bsum))) return -1;
-    const long long units = (long long)B * H * Lq;
+    const int Hk = H / G;
+    const long long units = (long long)B * Hk * Lq;  /* one per (b, group, query) */
 #pragma omp parallel num_threads(or_get_threads())
     {
-        double *q = malloc(sizeof(double) * d);
+        double *q = malloc(sizeof(double) * d * G);
         double *kb = malloc(sizeof(double) * d);
         scored *all = malloc(sizeof(scored) * (C > 0 ? C : 1));
 #pragma omp for schedule(dynamic, 4)
         for (long long u = 0; u < units; ++u) {
             const int i = (int)(u % Lq);
-            const int h = (int)((u / Lq) % H);
-            const int b = (int)(u / ((long long)Lq * H));
+            const int g = (int)((u / Lq) % Hk);
+            const int b = (int)(u / ((long long)Lq * Hk));
             const int t = qpos ? qpos[(long long)b * Lq + i] : i;
             const int ne = eligible_chunks(t, S, C);
-            load_vec(&Qcal, b, h, i, d, q);
+            for (int hh = 0; hh < G; ++hh) load_vec(&Qcal, b, g * G + hh, i, d, q + (long long)hh * d);
+            /* the group's selection score of chunk c: the largest of its heads' s^ */
             for (int c = 0; c < ne; ++c) {
-                all[c].s = chunk_score(q, &Ksum, &Bsum, b, h, c, d, scale, kb);
+                double m = -INFINITY;
+                for (int hh = 0; hh < G; ++hh) {
+                    const double sc = chunk_score(q + (long long)hh * d, &Ksum, &Bsum, b, g * G + hh, c, d, scale, kb);
+                    if (sc > m) m = sc;
+                }
+                all[c].s = m;
                 all[c].c = c;
             }
             qsort(all, ne, sizeof(scored), by_rank);
             const int n = ne < K ? ne : K;
             qsort(all, n, sizeof(scored), by_index);
-            for (int r = 0; r < K; ++r) {
-                idx[u * K + r] = r < n ? all[r].c : -1;
-                score[u * K + r] = r < n ? all[r].s : -INFINITY;
-            }
+            for (int r = 0; r < K; ++r) idx[u * K + r] = r < n ? all[r].c : -1;
             nsel[u] = n;
+            /* each head's own s^ of the kept chunks */
+            for (int hh = 0; hh < G; ++hh) {
+                const long long uh = ((long long)b * H + g * G + hh) * Lq + i;
+                for (int r = 0; r < K; ++r)
+                    score[uh * K + r] = r < n ? chunk_score(q + (long long)hh * d, &Ksum, &Bsum, b, g * G + hh,
+                                                            all[r].c, d, scale, kb)
+                                              : -INFINITY;
+            }
         }
         free(q);
         free(kb);
@@ -275,12 +294,12 @@ static void chunk_attention(const double *q, const or_tensor *Kc, const or_tenso
     }
 }
 
-int or_attend(int B, int H, int d, int S, int K, int W, double scale,
+int or_attend(int B, int H, int G, int d, int S, int K, int W, double scale,
               or_tensor Q, int Lq, const int *qpos,
               or_tensor Kc, or_tensor Vc,
               const int *idx, or_tensor score, const int *nsel,
               double *O, double *lse) {
-    if (B < 0 || H < 0 || d <= 0 || S <= 0 || K < 0 || W < 0 || Lq < 0) return -1;
+    if (B < 0 || H < 0 || G <= 0 || H % G != 0 || d <= 0 || S <= 0 || K < 0 || W < 0 || Lq < 0) return -1;
     if (!valid_dtype(&Q) || !valid_dtype(&Kc) || !valid_dtype(&Vc) || !O) return -1;
     if (K > 0 && (!idx || !nsel || !valid_dtype(&score))) return -1;
     const long long units = (long long)B * H * Lq;
@@ -298,23 +317,25 @@ int or_attend(int B, int H, int d, int S, int K, int W, double scale,
             const int h = (int)((u / Lq) % H);
             const int b = (int)(u / ((long long)Lq * H));
             const int t = qpos ? qpos[(long long)b * Lq + i] : i;
+            const int hk = h / G;                              /* key-value head */
+            const long long ug = ((long long)b * (H / G) + hk) * Lq + i;  /* the group's kept list */
             load_vec(&Q, b, h, i, d, q);
 
             /* selected chunks: log surrogate mass s^_{i,c} and chunk-local output */
             int nc = 0;
-            const int ns = K > 0 ? nsel[u] : 0;
+            const int ns = K > 0 ? nsel[ug] : 0;
             for (int r = 0; r < ns && r < K; ++r) {
-                const int c = idx[u * K + r];
+                const int c = idx[ug * K + r];
                 if (c < 0) continue;
                 mass[nc] = widen(&score, at(&score, b, h, i) + r);
-                chunk_attention(q, &Kc, &Vc, b, h, c, S, d, scale, logit, kv, vecs + (long long)nc * d);
+                chunk_attention(q, &Kc, &Vc, b, hk, c, S, d, scale, logit, kv, vecs + (long long)nc * d);
                 ++nc;
             }
             /* window tokens [max(0, t-W+1), t]: exact token logits */
             const int w0 = t - W + 1 > 0 ? t - W + 1 : 0;
             const int nw = W > 0 ? t - w0 + 1 : 0;
             for (int j = 0; j < nw; ++j) {
-                load_vec(&Kc, b, h, w0 + j, d, kv);
+                load_vec(&Kc, b, hk, w0 + j, d, kv);
                 wlogit[j] = dot(q, kv, d) * scale;
             }
 
@@ -337,7 +358,7 @@ int or_attend(int B, int H, int d, int S, int K, int W, double scale,
             for (int j = 0; j < nw; ++j) {
                 const double e = exp(wlogit[j] - M);
                 zhat += e;
-                load_vec(&Vc, b, h, w0 + j, d, kv);
+                load_vec(&Vc, b, hk, w0 + j, d, kv);
                 for (int x = 0; x < d; ++x) o[x] += e * kv[x];
             }
             for (int x = 0; x < d; ++x) o[x] /= zhat;

@@ -44,9 +44,10 @@ void or_set_threads(int n);
 int or_get_threads(void);
 
 /* Eq. 8: landmark softmax over each complete chunk, attention-weighted key k'_c and
- * entropy bias b'_c. K: [B,H,N,d]; LQ: [B,H,C,d] with C = N / S (floor).
- * Ksum: [B,H,C,d] double; Bsum: [B,H,C] double. */
-int or_summarize(int B, int H, int d, int S, double scale,
+ * entropy bias b'_c. G query heads share a key-value head (G = 1: one each).
+ * K: [B,H/G,N,d]; LQ: [B,H,C,d] with C = N / S (floor); query head h reads key-value
+ * head h / G. Ksum: [B,H,C,d] double; Bsum: [B,H,C] double. */
+int or_summarize(int B, int H, int G, int d, int S, double scale,
                  or_tensor K, int N, or_tensor LQ,
                  double *Ksum, double *Bsum);
 
@@ -58,21 +59,23 @@ int or_score_all(int B, int H, int d, int S, double scale,
                  or_tensor Qcal, int Lq, const int *qpos,
                  or_tensor Ksum, or_tensor Bsum, int C, double *out);
 
-/* Top-K over the eligible chunks, ranked by (score descending, chunk index
- * ascending). The kept chunks are listed in ascending chunk index.
- * idx: [B,H,Lq,K] int (-1 padding), score: [B,H,Lq,K] double (-inf padding),
- * nsel: [B,H,Lq] = min(K, number of eligible chunks). */
-int or_select(int B, int H, int d, int S, int K, double scale,
+/* Top-K over the eligible chunks of each group of G query heads, ranked by (the
+ * group's largest score descending, chunk index ascending). The kept chunks are
+ * listed in ascending chunk index. idx: [B,H/G,Lq,K] int (-1 padding), nsel:
+ * [B,H/G,Lq] = min(K, number of eligible chunks); score: [B,H,Lq,K] double, each
+ * head's own score of the kept chunks (-inf padding). */
+int or_select(int B, int H, int G, int d, int S, int K, double scale,
               or_tensor Qcal, int Lq, const int *qpos,
               or_tensor Ksum, or_tensor Bsum, int C,
               int *idx, double *score, int *nsel);
 
 /* Eq. 10: hierarchical softmax over the selected chunks (surrogate mass exp(score))
  * plus the sliding window [max(0, t-W+1), t] (exact token mass), with one joint
- * normaliser. Q: [B,H,Lq,d]; Kc, Vc: [B,H,L,d] (only positions <= t are read);
- * idx: [B,H,Lq,K] int; score: [B,H,Lq,K] as an or_tensor with st = K (f32 or f64);
- * nsel: [B,H,Lq]. O: [B,H,Lq,d] double; lse: [B,H,Lq] double (may be NULL). */
-int or_attend(int B, int H, int d, int S, int K, int W, double scale,
+ * normaliser. Q: [B,H,Lq,d]; Kc, Vc: [B,H/G,L,d] (only positions <= t are read;
+ * query head h reads key-value head h / G); idx: [B,H/G,Lq,K] int and nsel: [B,H/G,Lq]
+ * (the group's kept chunks); score: [B,H,Lq,K] as an or_tensor with st = K (f32 or
+ * f64). O: [B,H,Lq,d] double; lse: [B,H,Lq] double (may be NULL). */
+int or_attend(int B, int H, int G, int d, int S, int K, int W, double scale,
               or_tensor Q, int Lq, const int *qpos,
               or_tensor Kc, or_tensor Vc,
               const int *idx, or_tensor score, const int *nsel,
