@@ -48,7 +48,7 @@ class _CTensor(ctypes.Structure):
 class _Params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int), ("S", ctypes.c_int),
                 ("K", ctypes.c_int), ("W", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("scale", ctypes.c_float), ("flags", ctypes.c_uint32)]
+                ("scale", ctypes.c_float), ("flags", ctypes.c_uint32), ("H_kv", ctypes.c_int)]
 
 
 _lib = None
@@ -83,16 +83,23 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 
 class Params:
-    """hils_params: B, H, d, chunk size S (64), top-K, window W, dtype, scale (0 = 1/sqrt(d))."""
+    """hils_params: B, H query heads, d, chunk size S (64), top-K, window W, dtype, scale
+    (0 = 1/sqrt(d)), H_kv key-value heads (0 or H: multi-head; a divisor of H: groups of
+    H / H_kv query heads share a key-value head and one chunk selection)."""
 
     def __init__(self, B: int, H: int, d: int, K: int, W: int, dtype: torch.dtype = torch.bfloat16,
-                 S: int = 64, scale: float = 0.0, flags: int = 0):
+                 S: int = 64, scale: float = 0.0, flags: int = 0, H_kv: int = 0):
         self.B, self.H, self.d, self.K, self.W, self.S = B, H, d, K, W, S
-        self.dtype, self.scale, self.flags = dtype, scale, flags
+        self.dtype, self.scale, self.flags, self.H_kv = dtype, scale, flags, H_kv
+
+    @property
+    def Hk(self) -> int:
+        """Key-value heads (= the number of selection groups)."""
+        return self.H_kv if self.H_kv > 0 else self.H
 
     def c(self) -> _Params:
         dt = _DTYPES.get(self.dtype, -1) if isinstance(self.dtype, torch.dtype) else int(self.dtype)
-        return _Params(self.B, self.H, self.d, self.S, self.K, self.W, dt, self.scale, self.flags)
+        return _Params(self.B, self.H, self.d, self.S, self.K, self.W, dt, self.scale, self.flags, self.H_kv)
 
 
 def _view(t) -> _CTensor:
@@ -159,10 +166,11 @@ def _ws(workspace):
 
 
 def hils_summarize(p: Params, K, LQ, Ksum, Bsum, N: int | None = None, stream=None) -> None:
-    """Eq. 8 summaries of every complete chunk: Ksum [B,H,C,d], Bsum [B,H,C] float32."""
+    """Eq. 8 summaries of every complete chunk of every query head: K [B,Hk,N,d],
+    Ksum [B,H,C,d], Bsum [B,H,C] float32."""
     n = K.shape[2] if N is None else N
     B, H, d, C = p.B, p.H, p.d, n // p.S
-    if K.shape[0] != B or K.shape[1] != H or K.shape[3] != d or K.shape[2] < C * p.S:
+    if K.shape[0] != B or K.shape[1] != p.Hk or K.shape[3] != d or K.shape[2] < C * p.S:
         raise ValueError(f"hils_summarize: K has shape {tuple(K.shape)} for B={B} H={H} d={d} N={n}")
     if K.dtype != p.dtype:
         raise ValueError("hils_summarize: K dtype differs from params")
@@ -175,16 +183,17 @@ def hils_summarize(p: Params, K, LQ, Ksum, Bsum, N: int | None = None, stream=No
 
 def hils_select(p: Params, Qcal, Ksum, Bsum, idx, score, nsel, qpos=None, workspace=None,
                 Lq: int | None = None, C: int | None = None, stream=None) -> None:
-    """Eq. 7 scores and exact top-K: idx/score [B,H,Lq,K], nsel [B,H,Lq]."""
+    """Eq. 7 scores and exact top-K: idx [B,Hk,Lq,K] and nsel [B,Hk,Lq] per selection
+    group, score [B,H,Lq,K] per query head."""
     lq = Qcal.shape[2] if Lq is None else Lq
     c = Ksum.shape[2] if C is None else C
-    B, H, d, K = p.B, p.H, p.d, p.K
+    B, H, d, K, Hk = p.B, p.H, p.d, p.K, p.Hk
     _expect("hils_select", "Qcal", Qcal, (B, H, lq, d), p.dtype)
     _expect("hils_select", "Ksum", Ksum, (B, H, c, d), p.dtype)
     _expect("hils_select", "Bsum", Bsum, (B, H, c), torch.float32)
-    _expect("hils_select", "idx", idx, (B, H, lq, K), torch.int32)
+    _expect("hils_select", "idx", idx, (B, Hk, lq, K), torch.int32)
     _expect("hils_select", "score", score, (B, H, lq, K), torch.float32)
-    _expect("hils_select", "nsel", nsel, (B, H, lq), torch.int32)
+    _expect("hils_select", "nsel", nsel, (B, Hk, lq), torch.int32)
     if qpos is not None:
         _expect("hils_select", "qpos", qpos, (B, lq), torch.int32)
     wp, wn = _ws(workspace)
@@ -195,15 +204,16 @@ def hils_select(p: Params, Qcal, Ksum, Bsum, idx, score, nsel, qpos=None, worksp
 
 def hils_attend_prefill(p: Params, Q, K, V, idx, score, nsel, O, lse=None, workspace=None,
                         N: int | None = None, stream=None) -> None:
-    """Eq. 10 for every position: O [B,H,N,d], lse [B,H,N] float32 (optional)."""
+    """Eq. 10 for every position: Q, O [B,H,N,d], K, V [B,Hk,N,d], lse [B,H,N] float32
+    (optional)."""
     n = Q.shape[2] if N is None else N
-    B, H, d, k = p.B, p.H, p.d, p.K
-    for name, t in (("Q", Q), ("K", K), ("V", V), ("O", O)):
-        _expect("hils_attend_prefill", name, t, (B, H, n, d), p.dtype)
+    B, H, d, k, Hk = p.B, p.H, p.d, p.K, p.Hk
+    for name, t, h in (("Q", Q, H), ("K", K, Hk), ("V", V, Hk), ("O", O, H)):
+        _expect("hils_attend_prefill", name, t, (B, h, n, d), p.dtype)
     if k > 0:
-        _expect("hils_attend_prefill", "idx", idx, (B, H, n, k), torch.int32)
+        _expect("hils_attend_prefill", "idx", idx, (B, Hk, n, k), torch.int32)
         _expect("hils_attend_prefill", "score", score, (B, H, n, k), torch.float32)
-        _expect("hils_attend_prefill", "nsel", nsel, (B, H, n), torch.int32)
+        _expect("hils_attend_prefill", "nsel", nsel, (B, Hk, n), torch.int32)
     _expect("hils_attend_prefill", "lse", lse, (B, H, n), torch.float32)
     wp, wn = _ws(workspace)
     _check("hils_attend_prefill", load_library().hils_attend_prefill(
@@ -221,13 +231,13 @@ def hils_attend_decode(p: Params, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse
     _expect("hils_attend_decode", "Q", Q, (B, H, 1, d), p.dtype)
     _expect("hils_attend_decode", "O", O, (B, H, 1, d), p.dtype)
     for name, t in (("Kc", Kc), ("Vc", Vc)):
-        if t.shape[0] != B or t.shape[1] != H or t.shape[3] != d or t.dtype != p.dtype or not t.is_cuda:
+        if t.shape[0] != B or t.shape[1] != p.Hk or t.shape[3] != d or t.dtype != p.dtype or not t.is_cuda:
             raise ValueError(f"hils_attend_decode: {name} has shape {tuple(t.shape)} / {t.dtype}")
     _expect("hils_attend_decode", "cache_len", cache_len, (B,), torch.int32)
     if k > 0:
-        _expect("hils_attend_decode", "idx", idx, (B, H, 1, k), torch.int32)
+        _expect("hils_attend_decode", "idx", idx, (B, p.Hk, 1, k), torch.int32)
         _expect("hils_attend_decode", "score", score, (B, H, 1, k), torch.float32)
-        _expect("hils_attend_decode", "nsel", nsel, (B, H, 1), torch.int32)
+        _expect("hils_attend_decode", "nsel", nsel, (B, p.Hk, 1), torch.int32)
     _expect("hils_attend_decode", "lse", lse, (B, H), torch.float32)
     wp, wn = _ws(workspace)
     _check("hils_attend_decode", load_library().hils_attend_decode(
@@ -238,7 +248,7 @@ def hils_attend_decode(p: Params, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse
 def hils_decode(p: Params, Qcal, Ksum, Bsum, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse=None,
                 workspace=None, stream=None) -> None:
     """One decode step: hils_select with qpos = cache_len - 1, then hils_attend_decode,
-    as one chain. Outputs as the two calls: idx/score [B,H,1,K], nsel [B,H,1], O, lse."""
+    as one chain. Outputs as the two calls: idx [B,Hk,1,K], score [B,H,1,K], nsel [B,Hk,1], O, lse."""
     B, H, d, k = p.B, p.H, p.d, p.K
     c = Ksum.shape[2]
     _expect("hils_decode", "Qcal", Qcal, (B, H, 1, d), p.dtype)
@@ -247,12 +257,12 @@ def hils_decode(p: Params, Qcal, Ksum, Bsum, Q, Kc, Vc, cache_len, idx, score, n
     _expect("hils_decode", "Q", Q, (B, H, 1, d), p.dtype)
     _expect("hils_decode", "O", O, (B, H, 1, d), p.dtype)
     for name, t in (("Kc", Kc), ("Vc", Vc)):
-        if t.shape[0] != B or t.shape[1] != H or t.shape[3] != d or t.dtype != p.dtype or not t.is_cuda:
+        if t.shape[0] != B or t.shape[1] != p.Hk or t.shape[3] != d or t.dtype != p.dtype or not t.is_cuda:
             raise ValueError(f"hils_decode: {name} has shape {tuple(t.shape)} / {t.dtype}")
     _expect("hils_decode", "cache_len", cache_len, (B,), torch.int32)
-    _expect("hils_decode", "idx", idx, (B, H, 1, k), torch.int32)
+    _expect("hils_decode", "idx", idx, (B, p.Hk, 1, k), torch.int32)
     _expect("hils_decode", "score", score, (B, H, 1, k), torch.float32)
-    _expect("hils_decode", "nsel", nsel, (B, H, 1), torch.int32)
+    _expect("hils_decode", "nsel", nsel, (B, p.Hk, 1), torch.int32)
     _expect("hils_decode", "lse", lse, (B, H), torch.float32)
     wp, wn = _ws(workspace)
     _check("hils_decode", load_library().hils_decode(
@@ -270,13 +280,13 @@ def hils_attend_decode_noalloc(p: Params, Q, Kc, Vc, cache_len, idx, score, nsel
     _expect("hils_attend_decode_noalloc", "Q", Q, (B, H, 1, d), p.dtype)
     _expect("hils_attend_decode_noalloc", "O", O, (B, H, 1, d), p.dtype)
     for name, t in (("Kc", Kc), ("Vc", Vc)):
-        if t.shape[0] != B or t.shape[1] != H or t.shape[3] != d or t.dtype != p.dtype or not t.is_cuda:
+        if t.shape[0] != B or t.shape[1] != p.Hk or t.shape[3] != d or t.dtype != p.dtype or not t.is_cuda:
             raise ValueError(f"hils_attend_decode_noalloc: {name} has shape {tuple(t.shape)} / {t.dtype}")
     _expect("hils_attend_decode_noalloc", "cache_len", cache_len, (B,), torch.int32)
     if k > 0:
-        _expect("hils_attend_decode_noalloc", "idx", idx, (B, H, 1, k), torch.int32)
+        _expect("hils_attend_decode_noalloc", "idx", idx, (B, p.Hk, 1, k), torch.int32)
         _expect("hils_attend_decode_noalloc", "score", score, (B, H, 1, k), torch.float32)
-        _expect("hils_attend_decode_noalloc", "nsel", nsel, (B, H, 1), torch.int32)
+        _expect("hils_attend_decode_noalloc", "nsel", nsel, (B, p.Hk, 1), torch.int32)
     _expect("hils_attend_decode_noalloc", "lse", lse, (B, H), torch.float32)
     _check("hils_attend_decode_noalloc", load_library().hils_attend_decode_noalloc(
         ctypes.byref(p.c()), _view(Q), _view(Kc), _view(Vc), _ptr(cache_len), _ptr(idx), _ptr(score),

@@ -285,6 +285,8 @@ __global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
     const int u = blockIdx.x;
     const int64_t qi = blockIdx.y;  // (b, h), one query each
     const int b = (int)(qi / a.H), h = (int)(qi % a.H);
+    const int hk = h / a.G;                                   // key-value head of h
+    const int64_t qg = (int64_t)b * (a.H / a.G) + hk;         // the group's kept list
     const bool chunk_unit = u < a.topk;
     // dependent launch: chunk units wait for the preceding grid (the select's outputs
     // idx, score, nsel). Window tiles read only Q, K and V; they skip the wait only when
@@ -293,16 +295,16 @@ __global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
     if (chunk_unit || !a.window_early) pdl_wait();
     // the unit's small inputs, loaded together before anything depends on them
     const int clen = a.cache_len[b];
-    const int ns = chunk_unit ? a.nsel[qi] : 0;
-    const int cidx = chunk_unit ? a.idx[qi * a.topk + u] : -1;
+    const int ns = chunk_unit ? a.nsel[qg] : 0;
+    const int cidx = chunk_unit ? a.idx[qg * a.topk + u] : -1;
     const float csc = chunk_unit ? a.score[qi * a.topk + u] : 0.f;
     const UnitPlan p = plan_unit_loaded(u, clen - 1, a.topk, a.W, cidx, csc, ns);
     const DecodeWs ws = decode_ws(a.ws, a.B * a.H, a.units, D);
     float *my_vec = ws.vec + ((size_t)qi * a.units + u) * D;
     if (p.rows > 0) {
         const T *qrow = static_cast<const T *>(a.Q.ptr) + b * a.Q.sb + h * a.Q.sh;
-        const T *k0 = static_cast<const T *>(a.K.ptr) + b * a.K.sb + h * a.K.sh + (int64_t)p.start * a.K.st;
-        const T *v0 = static_cast<const T *>(a.V.ptr) + b * a.V.sb + h * a.V.sh + (int64_t)p.start * a.V.st;
+        const T *k0 = static_cast<const T *>(a.K.ptr) + b * a.K.sb + hk * a.K.sh + (int64_t)p.start * a.K.st;
+        const T *v0 = static_cast<const T *>(a.V.ptr) + b * a.V.sb + hk * a.V.sh + (int64_t)p.start * a.V.st;
         unit_issue<T, D>(s, qrow, k0, a.K.st, v0, a.V.st, p.rows);
         const float lse_tile = unit_compute<T, D>(s, p.rows, a.scale);
         for (int x = threadIdx.x; x < D; x += kThreads) my_vec[x] = s.red[x];
@@ -334,14 +336,16 @@ __global__ void __launch_bounds__(kThreads) attend_prefill_general_kernel(Attend
     const int h = (int)((qi / a.Lq) % a.H);
     const int b = (int)(qi / ((int64_t)a.Lq * a.H));
     const int t = i;
-    const int nsel = a.topk > 0 ? a.nsel[qi] : 0;
+    const int hk = h / a.G;                                                 // key-value head of h
+    const int64_t qg = ((int64_t)b * (a.H / a.G) + hk) * a.Lq + i;         // the group's kept list
+    const int nsel = a.topk > 0 ? a.nsel[qg] : 0;
     const T *qrow = static_cast<const T *>(a.Q.ptr) + b * a.Q.sb + h * a.Q.sh + i * a.Q.st;
-    const T *kh = static_cast<const T *>(a.K.ptr) + b * a.K.sb + h * a.K.sh;
-    const T *vh = static_cast<const T *>(a.V.ptr) + b * a.V.sb + h * a.V.sh;
+    const T *kh = static_cast<const T *>(a.K.ptr) + b * a.K.sb + hk * a.K.sh;
+    const T *vh = static_cast<const T *>(a.V.ptr) + b * a.V.sb + hk * a.V.sh;
     // thread x (< D) owns output column x
     float M = -INFINITY, zsum = 0.f, acc = 0.f;
     for (int u = 0; u < a.units; ++u) {
-        const UnitPlan p = plan_unit(u, t, a.topk, a.W, a.idx + qi * a.topk, a.score + qi * a.topk, nsel);
+        const UnitPlan p = plan_unit(u, t, a.topk, a.W, a.idx + qg * a.topk, a.score + qi * a.topk, nsel);
         if (p.rows == 0) continue;
         unit_issue<T, D>(s, qrow, kh + (int64_t)p.start * a.K.st, a.K.st, vh + (int64_t)p.start * a.V.st,
                          a.V.st, p.rows);

@@ -151,7 +151,7 @@ __device__ __forceinline__ float ldg_early(const float *p) {
 __device__ __forceinline__ int item_of(int r, int c, int G) { return r * G + ((r & 1) ? (G - 1 - c) : c); }
 
 struct Item {
-    int b, h, t0;
+    int b, h, hk, t0;  // batch, query head, its key-value head, first query
     int ws0, nw;  // window: first key, tiles
 };
 
@@ -163,6 +163,7 @@ __device__ __forceinline__ Item decode_item(const TcArgs &args, int j) {
     const int bh = j % BH;
     it.b = bh / a.H;
     it.h = bh % a.H;
+    it.hk = it.h / a.G;
     it.t0 = qb * kRows;
     it.ws0 = 0;
     it.nw = 0;
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             // the item's rows are consecutive: their kept lists form one contiguous block,
             // read with many loads in flight
             const int nrows = min(kRows, args.N - it.t0);
-            const int64_t q0 = ((int64_t)it.b * a.H + it.h) * a.Lq + it.t0;
+            const int64_t q0 = ((int64_t)it.b * (a.H / a.G) + it.hk) * a.Lq + it.t0;  // the group's kept lists
 #pragma unroll
             for (int rr = lane; rr < kRows; rr += 32)
                 nsm[rr] = (a.topk > 0 && rr < nrows) ? min(max(__ldg(&a.nsel[q0 + rr]), 0), a.topk) : 0;
@@ -327,16 +328,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
                         ++issuedK;
                         mbar_expect_tx(bar(kBarKfull + s), 2 * kTile * 128);
                         const uint32_t dst = sbase + kKOff + s * 16384;
-                        tma_load_4d(dst, &tmK, bar(kBarKfull + s), 0, k0, it.h, it.b);
-                        tma_load_4d(dst + 8192, &tmK, bar(kBarKfull + s), 64, k0, it.h, it.b);
+                        tma_load_4d(dst, &tmK, bar(kBarKfull + s), 0, k0, it.hk, it.b);
+                        tma_load_4d(dst + 8192, &tmK, bar(kBarKfull + s), 64, k0, it.hk, it.b);
                     }
                     if (u > 0 && !(ok = wait_warp(bar(kBarVfree + s), (u - 1) & 1))) break;
                     if (lane == 0) {
                         ++issuedV;
                         mbar_expect_tx(bar(kBarVfull + s), 2 * kTile * 128);
                         const uint32_t dst = sbase + kVOff + s * 16384;
-                        tma_load_4d(dst, &tmV, bar(kBarVfull + s), 0, k0, it.h, it.b);
-                        tma_load_4d(dst + 8192, &tmV, bar(kBarVfull + s), 64, k0, it.h, it.b);
+                        tma_load_4d(dst, &tmV, bar(kBarVfull + s), 0, k0, it.hk, it.b);
+                        tma_load_4d(dst + 8192, &tmV, bar(kBarVfull + s), 64, k0, it.hk, it.b);
                     }
                 }
             }
@@ -452,8 +453,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             const int t = it.t0 + x * kM + rloc;
             const bool row_ok = t < args.N;
             const int64_t qrow = ((int64_t)it.b * a.H + it.h) * a.Lq + t;
-            const int nsel = (row_ok && a.topk > 0) ? min(max(__ldg(&a.nsel[qrow]), 0), a.topk) : 0;
-            const int32_t *ip = a.idx + qrow * a.topk;
+            const int64_t qgrp = ((int64_t)it.b * (a.H / a.G) + it.hk) * a.Lq + t;  // the group's kept list
+            const int nsel = (row_ok && a.topk > 0) ? min(max(__ldg(&a.nsel[qgrp]), 0), a.topk) : 0;
+            const int32_t *ip = a.idx + qgrp * a.topk;
             const float *sp = a.score + qrow * a.topk;
             float ref = -INFINITY;  // log2-domain reference: the largest kept chunk score
 #pragma unroll 8
@@ -683,8 +685,9 @@ bool attend_prefill_tc_supported(hils_dtype dt, int d, int N) {
 
 hils_status launch_attend_prefill_tc(const AttendArgs &a, int N, uint32_t *status, cudaStream_t s) {
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, a.Q, a.B, a.H, N, kM) || !make_map(&mk, a.K, a.B, a.H, N, kTile) ||
-        !make_map(&mv, a.V, a.B, a.H, N, kTile))
+    const int Hk = a.H / a.G;
+    if (!make_map(&mq, a.Q, a.B, a.H, N, kM) || !make_map(&mk, a.K, a.B, Hk, N, kTile) ||
+        !make_map(&mv, a.V, a.B, Hk, N, kTile))
         return HILS_ERR_CUDA;
     static KernelSetup setup;
     int per_sm = 0;

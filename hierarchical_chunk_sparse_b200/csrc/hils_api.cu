@@ -62,9 +62,14 @@ int check_params(const hils_params *p, float *scale) {
     if (p->K > 32) return HILS_ERR_UNSUPPORTED;
     if (p->flags != 0) return HILS_ERR_UNSUPPORTED;
     if (!isfinite(p->scale)) return HILS_ERR_INVALID_ARG;
+    if (p->H_kv < 0 || (p->H_kv > 0 && p->H % p->H_kv != 0)) return HILS_ERR_INVALID_ARG;
+    if (p->H_kv > 0 && p->H / p->H_kv > kMaxGroupHeads) return HILS_ERR_UNSUPPORTED;
     *scale = p->scale != 0.f ? p->scale : (float)(1.0 / sqrt((double)p->d));
     return HILS_OK;
 }
+
+// Query heads per key-value head (parameters already checked).
+int groups(const hils_params *p) { return p->H_kv > 0 ? p->H / p->H_kv : 1; }
 
 bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
 
@@ -101,6 +106,7 @@ int decode_units(const hils_params *p) {
 
 size_t select_ws_for(const hils_params *p, int Lq, int C) {
     SelectArgs a{};
+    a.G = groups(p);
     select_plan(p->dtype, p->d, p->B, p->H, Lq, C, p->K, true, device_sm_count(), &a);
     return select_ws_bytes(p->B * p->H * Lq, C, a.path);
 }
@@ -123,9 +129,9 @@ int prepare_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_
     HILS_TRY(check_view(Qcal.ptr, Qcal.sb, Qcal.sh, Qcal.st, Lq, p));
     HILS_TRY(check_view(Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st, C, p));
     HILS_TRY(check_array(Bsum, (int64_t)p->B * p->H * C));
-    HILS_TRY(check_array(idx, nq * p->K));
+    HILS_TRY(check_array(idx, nq / groups(p) * p->K));
     HILS_TRY(check_array(score, nq * p->K));
-    HILS_TRY(check_array(nsel, nq));
+    HILS_TRY(check_array(nsel, nq / groups(p)));
     if (qpos && ((uintptr_t)qpos & 3u)) return HILS_ERR_ALIGNMENT;
     *nq_out = nq;
     a->Qcal = {Qcal.ptr, Qcal.sb, Qcal.sh, Qcal.st};
@@ -142,6 +148,7 @@ int prepare_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_
     a->C = C;
     a->topk = p->K;
     a->scale = scale;
+    a->G = groups(p);
     if (nq > 0) select_plan(p->dtype, p->d, p->B, p->H, Lq, C, p->K, qpos != nullptr, device_sm_count(), a);
     return HILS_OK;
 }
@@ -157,9 +164,9 @@ int prepare_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc,
     HILS_TRY(check_view(Vc.ptr, Vc.sb, Vc.sh, Vc.st, 1, p));
     HILS_TRY(check_view(O.ptr, O.sb, O.sh, O.st, 1, p));
     HILS_TRY(check_array(cache_len, p->B));
-    HILS_TRY(check_array(idx, nq * p->K));
+    HILS_TRY(check_array(idx, nq / groups(p) * p->K));
     HILS_TRY(check_array(score, nq * p->K));
-    HILS_TRY(check_array(nsel, p->K > 0 ? nq : 0));
+    HILS_TRY(check_array(nsel, p->K > 0 ? nq / groups(p) : 0));
     HILS_TRY(check_array(lse, 0));
     a->Q = {Q.ptr, Q.sb, Q.sh, Q.st};
     a->K = {Kc.ptr, Kc.sb, Kc.sh, Kc.st};
@@ -178,6 +185,7 @@ int prepare_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc,
     a->W = p->W;
     a->scale = scale;
     a->units = decode_units(p);
+    a->G = groups(p);
     return HILS_OK;
 }
 
@@ -195,7 +203,7 @@ const char *hils_status_string(int status) {
     switch (status) {
     case HILS_OK: return "ok";
     case HILS_ERR_INVALID_ARG: return "invalid argument";
-    case HILS_ERR_UNSUPPORTED: return "unsupported configuration (d in {64,128}, S = 64, K <= 32, flags = 0)";
+    case HILS_ERR_UNSUPPORTED: return "unsupported configuration (d in {64,128}, S = 64, K <= 32, flags = 0, H / H_kv <= 8)";
     case HILS_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
     case HILS_ERR_WORKSPACE: return "workspace missing or too small";
     case HILS_ERR_CUDA: return "CUDA launch error";
@@ -244,6 +252,7 @@ int hils_summarize(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ,
     a.H = p->H;
     a.C = C;
     a.scale = scale;
+    a.G = groups(p);
     return launch_summarize(p->dtype, p->d, a, stream);
 }
 
@@ -270,9 +279,9 @@ int hils_attend_prefill(const hils_params *p, hils_ctensor Q, hils_ctensor K, hi
     HILS_TRY(check_view(K.ptr, K.sb, K.sh, K.st, N, p));
     HILS_TRY(check_view(V.ptr, V.sb, V.sh, V.st, N, p));
     HILS_TRY(check_view(O.ptr, O.sb, O.sh, O.st, N, p));
-    HILS_TRY(check_array(idx, nq * p->K));
+    HILS_TRY(check_array(idx, nq / groups(p) * p->K));
     HILS_TRY(check_array(score, nq * p->K));
-    HILS_TRY(check_array(nsel, p->K > 0 ? nq : 0));
+    HILS_TRY(check_array(nsel, p->K > 0 ? nq / groups(p) : 0));
     HILS_TRY(check_array(lse, 0));
     HILS_TRY(check_workspace(workspace, ws_bytes, kPrefillWsBytes));
     if (nq == 0) return HILS_OK;
@@ -295,6 +304,7 @@ int hils_attend_prefill(const hils_params *p, hils_ctensor Q, hils_ctensor K, hi
     a.scale = scale;
     a.units = decode_units(p);
     a.ws = workspace;
+    a.G = groups(p);
     if (attend_prefill_tc_supported(p->dtype, p->d, N))
         return launch_attend_prefill_tc(a, N, static_cast<uint32_t *>(workspace), stream);
     return launch_attend_prefill_general(p->dtype, p->d, a, stream);

@@ -32,6 +32,7 @@ struct SummarizeArgs {
     float *Bsum;
     int B, H, C;
     float scale;
+    int G = 1;             // query heads per key-value head: K has H / G heads
 };
 
 struct SelectArgs {
@@ -45,6 +46,7 @@ struct SelectArgs {
     int B, H, Lq, C, topk;
     float scale;
     int path;              // SelectPath chosen by select_plan
+    int G = 1;             // query heads per group: idx and nsel have H / G heads
     // split search over chunk ranges (decode-like shapes)
     int ctas_per_query;    // summary blocks per query of the screen kernel
     int tiles_per_warp;    // 128-chunk tiles each warp scans
@@ -53,16 +55,18 @@ struct SelectArgs {
 
 // Which select kernels run: one warp per query; screen + pick (few queries, long
 // tables); tensor-core scoring with one thread per query (many bf16 queries, d = 128).
-enum SelectPath { kSelectWarp = 0, kSelectSplit = 1, kSelectTc = 2 };
+// Groups of G > 1 heads: one warp per (b, group, query) over all of the group's heads.
+constexpr int kMaxGroupHeads = 8;  // query heads per key-value head supported (H / H_kv)
+enum SelectPath { kSelectWarp = 0, kSelectSplit = 1, kSelectTc = 2, kSelectGroup = 3 };
 constexpr size_t kSelectStatusBytes = 256;  // status word at the front of the select workspace
 
 struct AttendArgs {
     View Q, K, V;
     MutView O;
     float *lse;            // [B, H, Lq] or null
-    const int32_t *idx;    // [B, H, Lq, Ksel]
-    const float *score;
-    const int32_t *nsel;
+    const int32_t *idx;    // [B, H / G, Lq, Ksel]
+    const float *score;    // [B, H, Lq, Ksel]
+    const int32_t *nsel;   // [B, H / G, Lq]
     const int32_t *qpos;   // prefill: null (t = i); decode: null and cache_len set
     const int32_t *cache_len;  // decode: [B]
     int B, H, Lq, topk, W;
@@ -70,6 +74,7 @@ struct AttendArgs {
     int units;             // units per query: K chunk units + window tiles
     int window_early;      // decode: window tiles may start before the preceding grid ends
     void *ws;
+    int G = 1;             // query heads per key-value head: K, V, idx and nsel have H / G heads
 };
 
 // Host launchers (one translation unit each). They return HILS_OK or HILS_ERR_CUDA.

@@ -30,6 +30,25 @@
 namespace hils {
 namespace {
 
+// Groups of G > 1 heads: one warp per (b, group, query) scores every chunk for all of the
+// group's heads (their query rows in shared memory as float32) and keeps the exact top K
+// of the heads' maximum.
+template <typename T, int D>
+__global__ void __launch_bounds__(kWarpKernelThreads) select_group_kernel(SelectArgs a) {
+    __shared__ __align__(16) float qs_all[kWarpKernelWarps][kMaxGroup * D];
+    __shared__ EntryList lists[kWarpKernelWarps];
+    const int w = threadIdx.x >> 5;
+    const int64_t qg = (int64_t)blockIdx.x * kWarpKernelWarps + w;
+    if (qg >= (int64_t)a.B * (a.H / a.G) * a.Lq) return;
+    int t, b, g, i;
+    const GroupCtx q = make_group_ctx<T, D>(a, qg, t, b, g, i);
+    const int ne = eligible(t, a.C);
+    for (int hh = 0; hh < q.G; ++hh) load_query_f32<T, D>(head_ctx(q, hh, (int)sizeof(T)), qs_all[w] + hh * D);
+    __syncwarp();
+    warp_scan<T, D>(q, qs_all[w], 0, ne, a.topk, lists[w]);
+    group_write<T, D>(q, qs_all[w], lists[w], a, qg, b, g, i);
+}
+
 // Many queries: one warp per query, direct output.
 template <typename T, int D>
 __global__ void __launch_bounds__(kWarpKernelThreads) select_warp_kernel(SelectArgs a) {
@@ -177,7 +196,11 @@ hils_status launch(const SelectArgs &a, cudaStream_t s) {
     const int64_t nq = (int64_t)a.B * a.H * a.Lq;
     if (nq == 0) return HILS_OK;
     if (a.path == kSelectTc) return launch_select_tc(a, s);
-    if (a.path == kSelectWarp) {
+    if (a.path == kSelectGroup) {
+        const int64_t ng = (int64_t)a.B * (a.H / a.G) * a.Lq;
+        select_group_kernel<T, D><<<(unsigned)((ng + kWarpKernelWarps - 1) / kWarpKernelWarps), kWarpKernelThreads, 0,
+                                    s>>>(a);
+    } else if (a.path == kSelectWarp) {
         const int64_t grid = (nq + kWarpKernelWarps - 1) / kWarpKernelWarps;
         select_warp_kernel<T, D><<<(unsigned)grid, kWarpKernelThreads, 0, s>>>(a);
     } else {
@@ -196,6 +219,10 @@ void select_plan(hils_dtype dt, int d, int B, int H, int Lq, int C, int K, bool 
     const int64_t nq = (int64_t)B * H * Lq;
     a->tiles_per_warp = (C + kTile - 1) / kTile;
     a->ctas_per_query = 0;
+    if (a->G > 1) {  // grouped heads: one warp per (b, group, query)
+        a->path = kSelectGroup;
+        return;
+    }
     // many queries: tensor-core scoring when the shape allows, else one warp per
     // query; short tables or tables beyond the pick kernel's register capacity also
     // take the warp kernel; otherwise screen + pick

@@ -106,8 +106,8 @@ __device__ __forceinline__ void screen(const QueryCtx &q, const float *qs, int c
 // `bound` receives a lower bound on the pool's K-th largest lo (s_K - e_max, rounded
 // down), or -inf when the pool holds at most K entries. Any chunk whose hi lies below
 // the bound of some subset of its competitors is certainly out.
-template <typename T, int D, int R>
-__device__ unsigned warp_topk(Slots<R> &p, int K, const QueryCtx &q, float &bound) {
+template <typename T, int D, int R, typename Ctx>
+__device__ unsigned warp_topk(Slots<R> &p, int K, const Ctx &q, float &bound) {
     const int lane = threadIdx.x & 31;
     unsigned valid = 0;
 #pragma unroll
@@ -223,8 +223,8 @@ __device__ int warp_append(const Slots<R> &p, unsigned keep, EntryList &list, in
 }
 
 // Scores chunks [c0, c1) in tiles of 128 and leaves their exact top-K in `list`.
-template <typename T, int D>
-__device__ void warp_scan(const QueryCtx &q, const float *qs, int c0, int c1, int K, EntryList &list) {
+template <typename T, int D, typename Ctx>
+__device__ void warp_scan(const Ctx &q, const float *qs, int c0, int c1, int K, EntryList &list) {
     const int lane = threadIdx.x & 31;
     int n = 0;
     for (int base = c0; base < c1; base += kTile) {
@@ -254,8 +254,8 @@ __device__ void warp_scan(const QueryCtx &q, const float *qs, int c0, int c1, in
 }
 
 // Reduces `nlists` lists (<= R*32 entries in total) to their exact top-K in `out`.
-template <typename T, int D, int R>
-__device__ void warp_merge(const QueryCtx &q, const EntryList *lists, int nlists, bool from_global, int K,
+template <typename T, int D, int R, typename Ctx>
+__device__ void warp_merge(const Ctx &q, const EntryList *lists, int nlists, bool from_global, int K,
                            EntryList &out) {
     const int lane = threadIdx.x & 31;
     Slots<R> p;
@@ -328,6 +328,95 @@ template <typename T, int D>
 __device__ void load_query_f32(const QueryCtx &q, float *qs) {
     const T *qr = static_cast<const T *>(q.qrow);
     for (int x = threadIdx.x & 31; x < D; x += 32) qs[x] = (float)qr[x];
+}
+
+// ---- grouped-query selection ("Hierarchical Sparse Attention Done Right", summary page,
+// Methodology 3, GQA adaptation): the G heads of a group keep the chunks with the largest
+// maximum over the group of s^_{h,i,c}. A group chunk's interval is [max lo_h, max hi_h]
+// over its heads' intervals, which contains the maximum of the heads' float64 scores; its
+// float64 value is that maximum.
+constexpr int kMaxGroup = kMaxGroupHeads;
+
+struct GroupCtx {
+    QueryCtx head;          // the group's first query head
+    int64_t qsh, ksh, bsh;  // head strides of Q~, of k' (elements) and of b' (floats)
+    int G;
+};
+
+__device__ __forceinline__ QueryCtx head_ctx(const GroupCtx &g, int hh, int es) {
+    QueryCtx q = g.head;
+    q.qrow = static_cast<const uint8_t *>(g.head.qrow) + (int64_t)hh * g.qsh * es;
+    q.khead = static_cast<const uint8_t *>(g.head.khead) + (int64_t)hh * g.ksh * es;
+    q.bhead = g.head.bhead + (int64_t)hh * g.bsh;
+    return q;
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void screen(const GroupCtx &g, const float *qs, int c, float &s, float &e) {
+    float lo = -INFINITY, hi = -INFINITY;
+    for (int hh = 0; hh < g.G; ++hh) {
+        float sh, eh;
+        screen<T, D>(head_ctx(g, hh, (int)sizeof(T)), qs + hh * D, c, sh, eh);
+        lo = fmaxf(lo, __fsub_rd(sh, eh));
+        hi = fmaxf(hi, __fadd_ru(sh, eh));
+    }
+    // [s - e, s + e] contains [lo, hi]: the midpoint's rounding is within 2^-24 |s|
+    s = 0.5f * lo + 0.5f * hi;
+    e = __fadd_ru(__fmul_ru(__fsub_ru(hi, lo), 0.5f), fabsf(s) * 0x1p-23f);
+}
+
+template <typename T, int D>
+__device__ double exact_score(const GroupCtx &g, int c) {
+    double m = -INFINITY;
+    for (int hh = 0; hh < g.G; ++hh) m = fmax(m, exact_score<T, D>(head_ctx(g, hh, (int)sizeof(T)), c));
+    return m;
+}
+
+// qg = (b, group, i): the group's first head, its strides, and the query's position
+template <typename T, int D>
+__device__ __forceinline__ GroupCtx make_group_ctx(const SelectArgs &a, int64_t qg, int &t, int &b, int &g, int &i) {
+    const int Hk = a.H / a.G;
+    const int q32 = (int)qg;
+    i = q32 % a.Lq;
+    const int bg = q32 / a.Lq;
+    g = bg % Hk;
+    b = bg / Hk;
+    t = a.qpos ? a.qpos[(int64_t)b * a.Lq + i] + a.qpos_bias : i;
+    const int h0 = g * a.G;
+    GroupCtx q;
+    q.head.qrow = static_cast<const T *>(a.Qcal.ptr) + b * a.Qcal.sb + h0 * a.Qcal.sh + i * a.Qcal.st;
+    q.head.khead = static_cast<const T *>(a.Ksum.ptr) + b * a.Ksum.sb + h0 * a.Ksum.sh;
+    q.head.kst = a.Ksum.st;
+    q.head.bhead = a.Bsum + ((int64_t)b * a.H + h0) * a.C;
+    q.head.scale = a.scale;
+    q.qsh = a.Qcal.sh;
+    q.ksh = a.Ksum.sh;
+    q.bsh = a.C;
+    q.G = a.G;
+    return q;
+}
+
+// Writes a group's kept list (ascending chunk index, padded to K) for the group, and each
+// head's own float32 screen value of the kept chunks.
+template <typename T, int D>
+__device__ void group_write(const GroupCtx &q, const float *qs, const EntryList &list, const SelectArgs &a,
+                            int64_t qg, int b, int g, int i) {
+    const int lane = threadIdx.x & 31;
+    const int K = a.topk, n = list.n;
+    int rank = lane, me = -1;
+    if (lane < n) {
+        me = list.idx[lane];
+        rank = 0;
+        for (int j = 0; j < n; ++j) rank += list.idx[j] < me;
+    }
+    if (lane < K) a.idx[qg * K + rank] = lane < n ? me : -1;
+    for (int hh = 0; hh < q.G; ++hh) {
+        const int64_t qh = ((int64_t)b * a.H + g * a.G + hh) * a.Lq + i;
+        float sh = -INFINITY, eh;
+        if (lane < n) screen<T, D>(head_ctx(q, hh, (int)sizeof(T)), qs + hh * D, me, sh, eh);
+        if (lane < K) a.score[qh * K + rank] = sh;
+    }
+    if (lane == 0) a.nsel[qg] = n;
 }
 
 // Upper-tail standard normal quantile z with P(Z > z) = p, 0 < p <= 0.5

@@ -58,8 +58,8 @@ __global__ void __launch_bounds__(128) summarize_kernel(SummarizeArgs a) {
             const int bh = (int)(u / (unsigned)a.C);
             const int h = bh % a.H;
             const int b = bh / a.H;
-            const T *k0 = static_cast<const T *>(a.K.ptr) + b * a.K.sb + h * a.K.sh +
-                          (int64_t)c * kChunk * a.K.st;
+            const T *k0 = static_cast<const T *>(a.K.ptr) + b * a.K.sb + (h / a.G) * a.K.sh +
+                          (int64_t)c * kChunk * a.K.st;  // the query head's key-value head
             const T *lq = static_cast<const T *>(a.LQ.ptr) + b * a.LQ.sb + h * a.LQ.sh + c * a.LQ.st;
             uint8_t *dst = smem + stage * Cfg::kStageBytes;
             for (int i = tid; i < Cfg::kStageUnits; i += Cfg::kThreads) {

@@ -1,7 +1,7 @@
 """Seeded synthetic inputs for the HiLS-Attention forward pass.
 
 This module only draws random tensors with the shapes, value distributions and
-planted structure of the five workloads below. It holds none of the method's
+planted structure of the workloads below. It holds none of the method's
 arithmetic, and it is the one module that both the CUDA path's callers (tests,
 bench, smoke check) and the oracle's callers share.
 
@@ -20,6 +20,12 @@ Workloads (one attention layer; chunk size S = 64 everywhere):
                          u one N(0,1) vector per 256-token block and e iid N(0,1), so that
                          adjacent queries keep overlapping chunk sets (the regime in which
                          the query-packing kernel shares chunks between queries).
+  7 prefill bf16 8K, grouped-query: as 2 with 8 key-value heads for the 32 query heads
+                         (groups of 4): K and V are [B, 8, N, d].
+  8 decode bf16 512K, grouped-query: as 4 with 8 key-value heads (groups of 4); the
+                         needle of each key-value head is planted against the query of
+                         the group's first head.
+Every workload with Hk = 0 has as many key-value heads as query heads.
 bf16 tensors are drawn in float32 and rounded to nearest-even.
 
 Seeds: base 20260709; the tensor with id k of workload n uses base + 100 n + k,
@@ -56,6 +62,15 @@ class Workload:
     needle_logit: float = 8.0
     qcal_block: int = 0  # > 0: Q_cal = block base vector + qcal_noise * iid noise
     qcal_noise: float = 0.0
+    Hk: int = 0  # key-value heads (0: one per query head)
+
+    @property
+    def Hkv(self) -> int:
+        return self.Hk if self.Hk > 0 else self.H
+
+    @property
+    def G(self) -> int:
+        return self.H // self.Hkv
 
     @property
     def C(self) -> int:
@@ -82,6 +97,10 @@ WORKLOADS = {
                 torch.bfloat16, needles=4),
     6: Workload(6, "prefill_bf16_8k_local", "prefill", 1, 32, 128, 64, 16, 512, 8192,
                 torch.bfloat16, qkv_scaled=True, qcal_block=256, qcal_noise=0.25),
+    7: Workload(7, "prefill_bf16_8k_gqa", "prefill", 1, 32, 128, 64, 16, 512, 8192, torch.bfloat16,
+                qkv_scaled=True, Hk=8),
+    8: Workload(8, "decode_bf16_512k_gqa", "decode", 1, 32, 128, 64, 16, 512, 524288,
+                torch.bfloat16, needles=1, Hk=8),
 }
 
 
@@ -96,13 +115,13 @@ def _randn(shape, g, device) -> torch.Tensor:
 
 
 def make_prefill(w: Workload, device="cpu") -> dict:
-    """Q, Q_cal, K, V [B,H,N,d] and LQ [B,H,C,d] for a prefill workload."""
-    B, H, N, d, C = w.B, w.H, w.N, w.d, w.C
+    """Q, Q_cal [B,H,N,d], K, V [B,Hk,N,d] and LQ [B,H,C,d] for a prefill workload."""
+    B, H, N, d, C, Hk = w.B, w.H, w.N, w.d, w.C, w.Hkv
     s = 1.0 / math.sqrt(d) if w.qkv_scaled else 1.0
     out = {}
     for name, shape, scaled in (("Q", (B, H, N, d), True), ("Qcal", (B, H, N, d), True),
-                                ("LQ", (B, H, C, d), False), ("K", (B, H, N, d), True),
-                                ("V", (B, H, N, d), True)):
+                                ("LQ", (B, H, C, d), False), ("K", (B, Hk, N, d), True),
+                                ("V", (B, Hk, N, d), True)):
         g = _gen(w, name, device)
         if name == "Qcal" and w.qcal_block > 0:
             nb = (N + w.qcal_block - 1) // w.qcal_block
@@ -117,18 +136,18 @@ def make_prefill(w: Workload, device="cpu") -> dict:
 
 
 def needle_positions(w: Workload, device="cpu") -> torch.Tensor:
-    """[B, H, needles] token positions of the planted needle keys (decode workloads).
+    """[B, Hk, needles] token positions of the planted needle keys (decode workloads).
 
     Positions lie in [0, t - W] with t = N - 1, so no needle is in the window; the
     needles of one (b, h) sit in distinct chunks."""
     if w.needles == 0:
-        return torch.zeros(w.B, w.H, 0, dtype=torch.int64)
+        return torch.zeros(w.B, w.Hkv, 0, dtype=torch.int64)
     g = _gen(w, "needles", "cpu")
     t = w.N - 1
     last_chunk = (t - w.W + 1) // w.S  # chunks [0, last_chunk) lie wholly before the window
-    pos = torch.empty(w.B, w.H, w.needles, dtype=torch.int64)
+    pos = torch.empty(w.B, w.Hkv, w.needles, dtype=torch.int64)
     for b in range(w.B):
-        for h in range(w.H):
+        for h in range(w.Hkv):
             chunks = torch.randperm(last_chunk, generator=g)[: w.needles]
             offs = torch.randint(0, w.S, (w.needles,), generator=g)
             pos[b, h] = chunks * w.S + offs
@@ -136,23 +155,25 @@ def needle_positions(w: Workload, device="cpu") -> torch.Tensor:
 
 
 def make_decode(w: Workload, device="cpu") -> dict:
-    """Decode inputs: Q, Q_cal [B,H,1,d], LQ [B,H,C,d], Kc, Vc [B,H,N,d] KV cache,
+    """Decode inputs: Q, Q_cal [B,H,1,d], LQ [B,H,C,d], Kc, Vc [B,Hk,N,d] KV cache,
     cache_len [B] int32 (= N; the query sits at t = N - 1) and needle positions.
 
     K and V are drawn one (b, h) slice at a time so that the float32 staging
     buffer stays at one head's size."""
-    B, H, N, d, C = w.B, w.H, w.N, w.d, w.C
+    B, H, N, d, C, Hk = w.B, w.H, w.N, w.d, w.C, w.Hkv
     q32 = _randn((B, H, 1, d), _gen(w, "Q", device), device)
     lq = torch.empty((B, H, C, d), dtype=w.dtype, device=device)
-    kc = torch.empty((B, H, N, d), dtype=w.dtype, device=device)
-    vc = torch.empty((B, H, N, d), dtype=w.dtype, device=device)
+    kc = torch.empty((B, Hk, N, d), dtype=w.dtype, device=device)
+    vc = torch.empty((B, Hk, N, d), dtype=w.dtype, device=device)
     pos = needle_positions(w)
     g_lq, g_k, g_v = _gen(w, "LQ", device), _gen(w, "K", device), _gen(w, "V", device)
     for b in range(B):
         for h in range(H):
             lq[b, h] = _randn((C, d), g_lq, device).to(w.dtype)
+    for b in range(B):
+        for h in range(Hk):
             k = _randn((N, d), g_k, device)
-            q = q32[b, h, 0]
+            q = q32[b, h * w.G, 0]
             for p in pos[b, h].tolist():
                 # k_p <- k_p + (L/scale - q.k_p) q / |q|^2, so that scale * q.k_p = L
                 k[p] += (w.needle_logit / w.scale - torch.dot(q, k[p])) * q / torch.dot(q, q)

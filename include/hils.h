@@ -50,6 +50,15 @@
  *   - Queries with fewer than K eligible chunks keep all of them; the rest of their
  *     selection row is padding (idx -1, score -inf). A query with no selected chunk
  *     and an empty window gets o = 0 and lse = -inf.
+ *   - Grouped-query attention (summary page, Methodology 3, GQA adaptation): with
+ *     Hk = params->H_kv key-value heads, the H query heads form groups of G = H / Hk
+ *     consecutive heads, query head h reading key-value head h / G. Landmark queries,
+ *     summaries and chunk scores stay per query head; the heads of a group keep the
+ *     same chunks, the K chunks with the largest maximum over the group of s^_{h,i,c}
+ *     (equal maxima to the lower chunk index), and each head weights them with its own
+ *     s^_{h,i,c} in Eq. 10. K, V, the KV cache, idx and nsel then have Hk heads; Q,
+ *     Q_cal, LQ, Ksum, Bsum, score, O and lse keep H. H_kv = 0 or H is multi-head
+ *     attention (G = 1).
  */
 #ifndef HILS_H
 #define HILS_H
@@ -68,7 +77,7 @@ typedef enum { HILS_F32 = 0, HILS_BF16 = 1 } hils_dtype;
 typedef enum {
     HILS_OK = 0,
     HILS_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent shape */
-    HILS_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, S != 64, K > 32, flags != 0 */
+    HILS_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, S != 64, K > 32, flags != 0, H / H_kv > 8 */
     HILS_ERR_ALIGNMENT = 3,    /* pointer or stride not 16-byte aligned */
     HILS_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
     HILS_ERR_CUDA = 5          /* a kernel launch failed; see hils_last_cuda_error() */
@@ -86,19 +95,23 @@ typedef struct {
 } hils_tensor;
 
 /* Problem description shared by every call.
- *   B      batch (sequences), H heads (one KV head per query head),
+ *   B      batch (sequences), H query heads,
  *   d      head dimension: 64 or 128,
  *   S      chunk size: 64,
  *   K      chunks kept per query (top-K): 0..32,
  *   W      sliding-window length in tokens: >= 0,
  *   dtype  element type of every Q/K/V/LQ/Ksum/O tensor,
  *   scale  softmax scale; 0 selects (float)(1/sqrt(d)),
- *   flags  reserved, must be 0. */
+ *   flags  reserved, must be 0,
+ *   H_kv   key-value heads: 0 (= H) or a divisor of H with H / H_kv <= 8; groups of
+ *          G = H / H_kv query heads share a key-value head and their chunk selection
+ *          (see above). */
 typedef struct {
     int B, H, d, S, K, W;
     hils_dtype dtype;
     float scale;
     uint32_t flags;
+    int H_kv;
 } hils_params;
 
 /* Which call a workspace size is asked for. */
@@ -110,10 +123,11 @@ typedef enum {
 } hils_call;
 
 /* Landmark chunk summaries (summary page, Methodology 1, Eq. 8).
- * For every complete chunk c < C = floor(N / S) of every (b, h):
+ * For every complete chunk c < C = floor(N / S) of every (b, h), h a query head:
  *   l_j = scale * q'_c . k_j for the S keys of the chunk, p = softmax(l),
  *   k'_c = sum_j p_j k_j,   b'_c = -sum_j p_j log p_j.
- *   K     [B, H, N, d]  keys of the sequence (only the first C*S positions are read)
+ *   K     [B, Hk, N, d] keys of the sequence (only the first C*S positions are read;
+ *         query head h reads key-value head h / G)
  *   N     number of tokens
  *   LQ    [B, H, C, d]  landmark query q'_c of each chunk
  *   Ksum  [B, H, C, d]  out: k'_c in dtype (float32 sums rounded to nearest-even)
@@ -134,10 +148,13 @@ int hils_summarize(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ,
  *   qpos  [B, Lq] int32 position t of each query, or NULL for t = i (prefill)
  *   Ksum  [B, H, C, d]  summary keys k'_c;  Bsum [B, H, C] float32 entropy biases b'_c
  *   C     number of summarised chunks
- *   idx   [B, H, Lq, K] int32 out: kept chunks in ascending chunk index, -1 padding
- *   score [B, H, Lq, K] float32 out: s^_{i,c} of each kept chunk (float32 evaluation,
- *         within 2^-9 * scale * |q~| |k'_c| + 2^-20 |s^| of the exact value), -inf padding
- *   nsel  [B, H, Lq] int32 out: number of kept chunks, min(K, eligible)
+ *   idx   [B, Hk, Lq, K] int32 out: kept chunks in ascending chunk index, -1 padding
+ *         (with G > 1: the group's chunks, ranked by the maximum over its heads of the
+ *         exact value below)
+ *   score [B, H, Lq, K] float32 out: s^_{i,c} of each kept chunk for each query head
+ *         (float32 evaluation, within 2^-9 * scale * |q~| |k'_c| + 2^-20 |s^| of the
+ *         exact value), -inf padding
+ *   nsel  [B, Hk, Lq] int32 out: number of kept chunks, min(K, eligible)
  *   workspace, ws_bytes: scratch of hils_workspace_bytes(p, HILS_CALL_SELECT, Lq, C) bytes
  *         (at least 256), zeroed before first use. Its first 32-bit word is a status
  *         word: the tensor-core path (bf16, d = 128, many queries; bounded waits) sets it
@@ -153,8 +170,9 @@ int hils_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *
  *   - each kept chunk c with weight exp(s^_{i,c}) / Z^_i on the chunk's own softmax
  *     output sum_{j in c} softmax_j(scale q_i.k_j) v_j, and
  *   - each window token j in [max(0, i-W+1), i] with weight exp(scale q_i.k_j) / Z^_i.
- *   Q, K, V  [B, H, N, d]
- *   idx, score, nsel: as written by hils_select: each row's first nsel entries are
+ *   Q [B, H, N, d];  K, V [B, Hk, N, d] (query head h reads key-value head h / G)
+ *   idx, score, nsel: as written by hils_select ([B, Hk, N, K], [B, H, N, K],
+ *         [B, Hk, N]): each row's first nsel entries are
  *         distinct chunks in ascending chunk index (score is used as the chunk's
  *         log-mass; passing exact log Z_{i,c} instead gives exact block-sparse attention)
  *   O    [B, H, N, d]  out, dtype (float32 result rounded to nearest-even)
@@ -173,9 +191,10 @@ int hils_attend_prefill(const hils_params *p, hils_ctensor Q, hils_ctensor K, hi
  * passages). Sequence b holds cache_len[b] tokens and its query sits at
  * t = cache_len[b] - 1 (the query's own key and value are the last cache entries).
  *   Q      [B, H, 1, d]
- *   Kc, Vc [B, H, Lmax, d] KV cache; positions >= cache_len[b] are never read
+ *   Kc, Vc [B, Hk, Lmax, d] KV cache; positions >= cache_len[b] are never read
  *   cache_len [B] int32 on the device
- *   idx, score, nsel: [B, H, 1, K] / [B, H, 1] from hils_select with qpos = cache_len - 1
+ *   idx, nsel [B, Hk, 1, K] / [B, Hk, 1] and score [B, H, 1, K] from hils_select with
+ *          qpos = cache_len - 1
  *   O      [B, H, 1, d] out;  lse [B, H] float32 out, or NULL
  *   workspace, ws_bytes: hils_workspace_bytes(p, HILS_CALL_ATTEND_DECODE, 1, 0). */
 int hils_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hils_ctensor Vc,
@@ -194,7 +213,7 @@ int hils_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hi
  * chunk selection.
  *   Qcal [B, H, 1, d]; Ksum [B, H, C, d]; Bsum [B, H, C]; C summarised chunks
  *   Q, Kc, Vc, cache_len, O, lse: as for hils_attend_decode
- *   idx, score [B, H, 1, K], nsel [B, H, 1]: out
+ *   idx [B, Hk, 1, K], score [B, H, 1, K], nsel [B, Hk, 1]: out
  *   workspace, ws_bytes: hils_workspace_bytes(p, HILS_CALL_DECODE, 1, C) bytes, zeroed
  *         before first use (the select part first, then the attend part). */
 int hils_decode(const hils_params *p, hils_ctensor Qcal, hils_ctensor Ksum, const float *Bsum, int C,

@@ -23,7 +23,8 @@ pytestmark = pytest.mark.gpu
 
 
 def P(w, **kw):
-    return hils.Params(B=w.B, H=w.H, d=w.d, K=kw.pop("K", w.K), W=kw.pop("W", w.W), dtype=w.dtype, **kw)
+    return hils.Params(B=w.B, H=w.H, d=w.d, K=kw.pop("K", w.K), W=kw.pop("W", w.W), dtype=w.dtype, H_kv=w.Hk,
+                       **kw)
 
 
 def gpu_summarize(w, K, LQ, N=None):
@@ -38,10 +39,10 @@ def gpu_summarize(w, K, LQ, N=None):
 def gpu_select(w, Qcal, Ksum, Bsum, qpos=None, K=None):
     k = w.K if K is None else K
     p = P(w, K=k)
-    B, H, Lq = Qcal.shape[0], Qcal.shape[1], Qcal.shape[2]
-    idx = torch.full((B, H, Lq, k), 7777, dtype=torch.int32, device=Qcal.device)
+    B, H, Lq, Hk = Qcal.shape[0], Qcal.shape[1], Qcal.shape[2], w.Hkv
+    idx = torch.full((B, Hk, Lq, k), 7777, dtype=torch.int32, device=Qcal.device)
     score = torch.full((B, H, Lq, k), 7777.0, dtype=torch.float32, device=Qcal.device)
-    nsel = torch.full((B, H, Lq), 7777, dtype=torch.int32, device=Qcal.device)
+    nsel = torch.full((B, Hk, Lq), 7777, dtype=torch.int32, device=Qcal.device)
     ws = hils.alloc_workspace(p, hils.HILS_CALL_SELECT, Lq, Ksum.shape[2], device=Qcal.device)
     hils.hils_select(p, Qcal, Ksum, Bsum, idx, score, nsel, qpos=qpos, workspace=ws)
     assert int(host(ws[:4]).view(torch.int32)[0]) == 0, "a bounded wait expired"
@@ -501,10 +502,10 @@ def test_end_to_end_against_chained_oracle(oracle, cuda_device, case):
 
 def _decode_chain(w, d, Ksum, Bsum, ws=None):
     p = P(w)
-    B, H = w.B, w.H
-    idx = torch.full((B, H, 1, w.K), 7777, dtype=torch.int32, device=Ksum.device)
+    B, H, Hk = w.B, w.H, w.Hkv
+    idx = torch.full((B, Hk, 1, w.K), 7777, dtype=torch.int32, device=Ksum.device)
     score = torch.full((B, H, 1, w.K), 7777.0, device=Ksum.device)
-    nsel = torch.full((B, H, 1), 7777, dtype=torch.int32, device=Ksum.device)
+    nsel = torch.full((B, Hk, 1), 7777, dtype=torch.int32, device=Ksum.device)
     O = torch.full_like(d["Q"], 99.0)
     lse = torch.full((B, H), 99.0, device=Ksum.device)
     if ws is None:
