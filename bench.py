@@ -200,15 +200,17 @@ def barrier(world):
 # ----------------------------------------------------------------- decode workload
 
 def decode_bytes(w) -> dict:
-    """Algorithmic HBM bytes of one decode step (per the whole batch)."""
+    """Algorithmic HBM bytes of one decode step (per the whole batch). The summary table
+    is per query head; the kept chunks and the window of K and V are read once per
+    key-value head (a group of query heads shares them)."""
     t = w.N - 1
     c_elig = min(t // w.S, w.C)
     es = 2
-    per_bh_sel = c_elig * (w.d * es + 4) + 2 * w.d * es + w.K * 8 + 4  # table + q~ + outputs
-    per_bh_att = w.K * w.S * w.d * es * 2 + w.W * w.d * es * 2 + 2 * w.d * es + w.K * 8 + 4
-    n = w.B * w.H
-    return {"select": n * per_bh_sel, "attend": n * per_bh_att,
-            "step": n * (c_elig * (w.d * es + 4) + w.K * w.S * w.d * es * 2 + w.W * w.d * es * 2 + 768)}
+    n, nk = w.B * w.H, w.B * w.Hkv
+    table = n * c_elig * (w.d * es + 4)
+    kv = nk * (w.K * w.S + w.W) * w.d * es * 2
+    small = n * (2 * w.d * es + w.K * 8 + 4)  # q~, q, o, kept lists, lse
+    return {"select": table + small, "attend": kv + small, "step": table + kv + small}
 
 
 class DecodeBench:
@@ -218,15 +220,15 @@ class DecodeBench:
         self.hils, self.w, self.dev = hils, w, dev
         inp = make_decode(w, device=dev)
         self.inp = inp
-        self.p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype)
+        self.p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype, H_kv=w.Hk)
         C = w.C
         self.Ksum = torch.empty(w.B, w.H, C, w.d, dtype=w.dtype, device=dev)
         self.Bsum = torch.empty(w.B, w.H, C, dtype=torch.float32, device=dev)
         hils.hils_summarize(self.p, inp["K"], inp["LQ"], self.Ksum, self.Bsum)
         self.qpos = (inp["cache_len"] - 1).reshape(w.B, 1).contiguous()
-        self.idx = torch.empty(w.B, w.H, 1, w.K, dtype=torch.int32, device=dev)
+        self.idx = torch.empty(w.B, w.Hkv, 1, w.K, dtype=torch.int32, device=dev)
         self.score = torch.empty(w.B, w.H, 1, w.K, dtype=torch.float32, device=dev)
-        self.nsel = torch.empty(w.B, w.H, 1, dtype=torch.int32, device=dev)
+        self.nsel = torch.empty(w.B, w.Hkv, 1, dtype=torch.int32, device=dev)
         self.ws_sel = hils.alloc_workspace(self.p, hils.HILS_CALL_SELECT, 1, C, device=dev)
         self.ws_dec = hils.alloc_workspace(self.p, hils.HILS_CALL_ATTEND_DECODE, 1, 0, device=dev)
         self.ws_step = hils.alloc_workspace(self.p, hils.HILS_CALL_DECODE, 1, C, device=dev)
@@ -299,13 +301,13 @@ class PrefillBench:
 
         self.hils, self.w = hils, w
         self.inp = make_prefill(w, device=dev)
-        self.p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype)
+        self.p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype, H_kv=w.Hk)
         C = w.C
         self.Ksum = torch.empty(w.B, w.H, C, w.d, dtype=w.dtype, device=dev)
         self.Bsum = torch.empty(w.B, w.H, C, dtype=torch.float32, device=dev)
-        self.idx = torch.empty(w.B, w.H, w.N, w.K, dtype=torch.int32, device=dev)
+        self.idx = torch.empty(w.B, w.Hkv, w.N, w.K, dtype=torch.int32, device=dev)
         self.score = torch.empty(w.B, w.H, w.N, w.K, dtype=torch.float32, device=dev)
-        self.nsel = torch.empty(w.B, w.H, w.N, dtype=torch.int32, device=dev)
+        self.nsel = torch.empty(w.B, w.Hkv, w.N, dtype=torch.int32, device=dev)
         self.ws = hils.alloc_workspace(self.p, hils.HILS_CALL_SELECT, w.N, C, device=dev)
         self.ws_att = hils.alloc_workspace(self.p, hils.HILS_CALL_ATTEND_PREFILL, w.N, C, device=dev)
         self.O = torch.empty_like(self.inp["Q"])
@@ -517,6 +519,36 @@ def measure_prefill(wp, dev, stream, flush, args, world, peaks, peak_src, traffi
     return out
 
 
+def measure_decode(w, dev, stream, flush, args, world, peaks):
+    """A secondary decode workload: hils_decode step time and its select and attend
+    kernels (L2 flushed), tokens/s and algorithmic GB/s."""
+    db = DecodeBench(w, dev)
+    n = max(3, min(args.steps, 50))
+    step_g, sel_g, att_g = graphed(db.step, stream), graphed(db.select, stream), graphed(db.attend, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step_g()
+    stream.synchronize()
+    with ClockSampler(dev) as clk:
+        ms = statistics.mean(time_steps(step_g, n, flush, stream))
+    ms = max_over_ranks(ms, world, dev)
+    t_sel = statistics.mean(time_steps(sel_g, n, flush, stream))
+    t_att = statistics.mean(time_steps(att_g, n, flush, stream))
+    torch.cuda.synchronize()
+    by = decode_bytes(w)
+    hbm = peaks["hbm_gbs"]
+    out = {"value": job_throughput(w.B, world, ms), "unit": "tokens/s", "ms_per_step": ms, "workload": w.name,
+           "H": w.H, "H_kv": w.Hkv, "steps": n, "clocks": clk.summary(),
+           "kernel_us": {"select": 1e3 * t_sel, "attend": 1e3 * t_att},
+           "algorithmic_bytes": by,
+           "select_frac_of_hbm": by["select"] / (t_sel * 1e-3) / 1e9 / hbm,
+           "attend_gbs": by["attend"] / (t_att * 1e-3) / 1e9,
+           "step_frac_of_hbm": by["step"] / (ms * 1e-3) / 1e9 / hbm}
+    del db, step_g, sel_g, att_g
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None,
@@ -599,10 +631,14 @@ def main():
     # ---------------- prefill @8K (iid queries; and the query-locality variant)
     prefill = None
     prefill_local = None
+    prefill_gqa = None
     if not args.no_prefill:
         prefill = measure_prefill(WORKLOADS[2], dev, stream, flush, args, world, peaks, peak_src,
                                   MEASURED_TRAFFIC["attend_prefill"])
         prefill_local = measure_prefill(WORKLOADS[6], dev, stream, flush, args, world, peaks, peak_src, None)
+        prefill_gqa = measure_prefill(WORKLOADS[7], dev, stream, flush, args, world, peaks, peak_src, None)
+    # ---------------- grouped-query decode @512K (32 query heads, 8 key-value heads)
+    decode_gqa = measure_decode(WORKLOADS[8], dev, stream, flush, args, world, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -630,6 +666,8 @@ def main():
             "clocks": clk.summary(),
             "prefill": prefill,
             "prefill_local": prefill_local,
+            "prefill_gqa": prefill_gqa,
+            "decode_gqa": decode_gqa,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

@@ -103,7 +103,7 @@ __host__ __device__ inline size_t attend_decode_counter_bytes(int queries) {
 void select_plan(hils_dtype dt, int d, int B, int H, int Lq, int C, int K, bool has_qpos, int num_sms,
                  SelectArgs *a);
 // Tensor-core select (bf16, d = 128, at most 512 eligible chunks per query).
-bool select_tc_supported(hils_dtype dt, int d, int B, int H, int Lq, int C, int K, bool has_qpos);
+bool select_tc_supported(hils_dtype dt, int d, int B, int H, int Lq, int C, int K, bool has_qpos, int G);
 hils_status launch_select_tc(const SelectArgs &a, cudaStream_t s);
 
 int device_sm_count();

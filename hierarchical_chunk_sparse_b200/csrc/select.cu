@@ -102,13 +102,14 @@ struct ScrCfg : StageCfg<T, D, kScrThreads, kScrRows> {
     static constexpr int kSmemBytes = kGscrOff + kScrRows * 8;
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
-// One CTA per query, dependent-launched after the screen grid.
-template <typename T, int D>
+// One CTA per query (per (b, group, query) for grouped heads), dependent-launched after
+// the screen grid.
+template <typename T, int D, bool kGroup>
 __global__ void __launch_bounds__(kPickThreads) select_pick_kernel(SelectArgs a) {
     __shared__ PickSmem ps;
     pdl_wait();     // the screen grid has completed and its writes are visible
     pdl_trigger();  // let the next dependent-launched kernel be scheduled
-    pick_query<T, D, kPickThreads>(a, screen_ws(a), blockIdx.x, ps);
+    pick_unit<T, D, kPickThreads, kGroup>(a, screen_ws(a), blockIdx.x, ps);
 }
 
 template <typename T, int D>
@@ -206,8 +207,11 @@ hils_status launch(const SelectArgs &a, cudaStream_t s) {
     } else {
         const hils_status st = launch_screen<T, D>(a, s);
         if (st != HILS_OK) return st;
-        return launch_dependent((const void *)select_pick_kernel<T, D>, dim3((unsigned)nq), dim3(kPickThreads), 0,
-                                s, a);
+        if (a.G > 1)
+            return launch_dependent((const void *)select_pick_kernel<T, D, true>, dim3((unsigned)(nq / a.G)),
+                                    dim3(kPickThreads), 0, s, a);
+        return launch_dependent((const void *)select_pick_kernel<T, D, false>, dim3((unsigned)nq),
+                                dim3(kPickThreads), 0, s, a);
     }
     return record_cuda_error(cudaGetLastError());
 }
@@ -219,17 +223,16 @@ void select_plan(hils_dtype dt, int d, int B, int H, int Lq, int C, int K, bool 
     const int64_t nq = (int64_t)B * H * Lq;
     a->tiles_per_warp = (C + kTile - 1) / kTile;
     a->ctas_per_query = 0;
-    if (a->G > 1) {  // grouped heads: one warp per (b, group, query)
-        a->path = kSelectGroup;
-        return;
-    }
     // many queries: tensor-core scoring when the shape allows, else one warp per
-    // query; short tables or tables beyond the pick kernel's register capacity also
-    // take the warp kernel; otherwise screen + pick
+    // query (per (b, group, query) for grouped heads); short tables or tables beyond
+    // the pick kernel's register capacity also take the warp kernel; otherwise
+    // screen + pick
     if (nq >= (int64_t)kWarpKernelWarps * num_sms || C <= kTile || C > kMaxDecC || nq > 65535 || K < 1) {
-        a->path = select_tc_supported(dt, d, B, H, Lq, C, K, has_qpos) && nq >= (int64_t)kWarpKernelWarps * num_sms
+        a->path = select_tc_supported(dt, d, B, H, Lq, C, K, has_qpos, a->G) &&
+                          nq >= (int64_t)kWarpKernelWarps * num_sms
                       ? kSelectTc
-                      : kSelectWarp;
+                  : a->G > 1 ? kSelectGroup
+                             : kSelectWarp;
         return;
     }
     a->path = kSelectSplit;

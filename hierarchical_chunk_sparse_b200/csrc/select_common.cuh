@@ -14,6 +14,8 @@
 #include <limits.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "hils_internal.cuh"
 
 namespace hils {
@@ -351,18 +353,28 @@ __device__ __forceinline__ QueryCtx head_ctx(const GroupCtx &g, int hh, int es) 
     return q;
 }
 
+// A centre and radius whose interval [s - e, s + e] contains [lo, hi] (finite): the
+// midpoint's rounding is within 2^-24 |s|.
+__device__ __forceinline__ void interval_mid(float lo, float hi, float &s, float &e) {
+    s = 0.5f * lo + 0.5f * hi;
+    e = __fadd_ru(__fmul_ru(__fsub_ru(hi, lo), 0.5f), fabsf(s) * 0x1p-23f);
+}
+
+// Folds one head's interval s +- e into the group's running [lo, hi].
+__device__ __forceinline__ void fold_interval(float s, float e, float &lo, float &hi) {
+    lo = fmaxf(lo, __fsub_rd(s, e));
+    hi = fmaxf(hi, __fadd_ru(s, e));
+}
+
 template <typename T, int D>
 __device__ __forceinline__ void screen(const GroupCtx &g, const float *qs, int c, float &s, float &e) {
     float lo = -INFINITY, hi = -INFINITY;
     for (int hh = 0; hh < g.G; ++hh) {
         float sh, eh;
         screen<T, D>(head_ctx(g, hh, (int)sizeof(T)), qs + hh * D, c, sh, eh);
-        lo = fmaxf(lo, __fsub_rd(sh, eh));
-        hi = fmaxf(hi, __fadd_ru(sh, eh));
+        fold_interval(sh, eh, lo, hi);
     }
-    // [s - e, s + e] contains [lo, hi]: the midpoint's rounding is within 2^-24 |s|
-    s = 0.5f * lo + 0.5f * hi;
-    e = __fadd_ru(__fmul_ru(__fsub_ru(hi, lo), 0.5f), fabsf(s) * 0x1p-23f);
+    interval_mid(lo, hi, s, e);
 }
 
 template <typename T, int D>

@@ -42,48 +42,75 @@ __device__ void block_kth_plus_one(const float2 *v, int n, int K, float *out) {
     }
 }
 
-// The float32 screen value and tight radius of every pool entry on CUDA cores, four
-// threads per entry (a quarter of the row each, then two shuffle steps). Any order of
-// the float32 sums stays within the radius scale sum|q k| (d+2) 2^-23 + |s| 2^-22.
+// The float32 screen value and tight radius of chunk c for one query head, four
+// threads per chunk (a quarter of the row each, then two shuffle steps; every lane of
+// the warp takes part, lanes with ok = false contribute zero). Any order of the float32
+// sums stays within the radius scale sum|q k| (d+2) 2^-23 + |s| 2^-22.
+template <typename T, int D>
+__device__ __forceinline__ void rescreen_one(const QueryCtx &q, const float *qs, int c, bool ok, float &s,
+                                             float &e) {
+    constexpr int kN = Vec<T>::kN, kQuarter = D / 4;
+    const int sub = threadIdx.x & 3;
+    float dot = 0.f, ad = 0.f;
+    if (ok) {
+        const uint4 *kr = reinterpret_cast<const uint4 *>(static_cast<const T *>(q.khead) + (int64_t)c * q.kst +
+                                                          sub * kQuarter);
+#pragma unroll
+        for (int u = 0; u < kQuarter / kN; ++u) {
+            float kf[kN];
+            widen(__ldg(kr + u), kf, T());
+#pragma unroll
+            for (int i = 0; i < kN; ++i) {
+                const float qv = qs[sub * kQuarter + u * kN + i];
+                dot = fmaf(qv, kf[i], dot);
+                ad = fmaf(fabsf(qv), fabsf(kf[i]), ad);
+            }
+        }
+    }
+    dot += __shfl_xor_sync(kFull, dot, 1);
+    ad += __shfl_xor_sync(kFull, ad, 1);
+    dot += __shfl_xor_sync(kFull, dot, 2);
+    ad += __shfl_xor_sync(kFull, ad, 2);
+    s = ok ? fmaf(dot, q.scale, q.bhead[c]) : 0.f;
+    e = fmaf(q.scale * ad, (float)(D + 2) * 0x1p-23f, fabsf(s) * 0x1p-22f);
+}
+
+// Every pool entry screened again on CUDA cores with the tight radius.
 template <typename T, int D, int NT>
 __device__ void rescreen_pool(const QueryCtx &q, const float *qs, Pool64 &pool, int total) {
-    constexpr int kN = Vec<T>::kN, kQuarter = D / 4;
-    const int tid = threadIdx.x, sub = tid & 3;
+    const int tid = threadIdx.x;
     for (int base = 0; base < total; base += NT / 4) {  // the same trip count in every lane
         const int j = base + (tid >> 2);
         const bool ok = j < total;
-        float dot = 0.f, ad = 0.f;
-        int c = 0;
-        if (ok) {
-            c = pool.idx[j];
-            const uint4 *kr = reinterpret_cast<const uint4 *>(static_cast<const T *>(q.khead) + (int64_t)c * q.kst +
-                                                              sub * kQuarter);
-#pragma unroll
-            for (int u = 0; u < kQuarter / kN; ++u) {
-                float kf[kN];
-                widen(__ldg(kr + u), kf, T());
-#pragma unroll
-                for (int i = 0; i < kN; ++i) {
-                    const float qv = qs[sub * kQuarter + u * kN + i];
-                    dot = fmaf(qv, kf[i], dot);
-                    ad = fmaf(fabsf(qv), fabsf(kf[i]), ad);
-                }
-            }
-        }
-        dot += __shfl_xor_sync(kFull, dot, 1);
-        ad += __shfl_xor_sync(kFull, ad, 1);
-        dot += __shfl_xor_sync(kFull, dot, 2);
-        ad += __shfl_xor_sync(kFull, ad, 2);
-        if (ok && sub == 0) {
-            const float s = fmaf(dot, q.scale, q.bhead[c]);
+        float s, e;
+        rescreen_one<T, D>(q, qs, ok ? pool.idx[j] : 0, ok, s, e);
+        if (ok && (tid & 3) == 0) {
             pool.s[j] = s;
-            pool.e[j] = fmaf(q.scale * ad, (float)(D + 2) * 0x1p-23f, fabsf(s) * 0x1p-22f);
+            pool.e[j] = e;
         }
     }
 }
 
+// Grouped heads: each head's tight interval, folded into the group maximum's interval.
+template <typename T, int D, int NT>
+__device__ void rescreen_pool(const GroupCtx &g, const float *qs, Pool64 &pool, int total) {
+    const int tid = threadIdx.x;
+    for (int base = 0; base < total; base += NT / 4) {
+        const int j = base + (tid >> 2);
+        const bool ok = j < total;
+        const int c = ok ? pool.idx[j] : 0;
+        float lo = -INFINITY, hi = -INFINITY;
+        for (int hh = 0; hh < g.G; ++hh) {
+            float s, e;
+            rescreen_one<T, D>(head_ctx(g, hh, (int)sizeof(T)), qs + hh * D, c, ok, s, e);
+            fold_interval(s, e, lo, hi);
+        }
+        if (ok && (tid & 3) == 0) interval_mid(lo, hi, pool.s[j], pool.e[j]);
+    }
+}
+
 struct PickSmem {
-    float qs[128];
+    float qs[kMaxGroup * 128];  // the query rows (float32) of the unit's heads
     float2 gm[kMaxGroups];
     uint16_t cand_g[kMaxGroups];
     Pool64 pool;
@@ -105,6 +132,48 @@ __host__ __device__ __forceinline__ size_t dec_ws_bytes(int64_t queries, int C) 
     return kSelectStatusBytes + scr;
 }
 
+// The screen rows one pick unit reads: one query's, or the G rows of a group's heads
+// (consecutive query heads, Lq queries apart in the workspace).
+struct ScrRows {
+    const float2 *scr, *gmx;
+    int64_t scr_hs, gmx_hs;  // head strides
+    int G;
+};
+
+// Screen value and radius of chunk c < ne for the unit: a group's is the interval of
+// the maximum over its heads.
+template <bool kGroup>
+__device__ __forceinline__ float2 scr_at(const ScrRows &r, int c) {
+    if constexpr (!kGroup) {
+        return __ldcg(&r.scr[c]);
+    } else {
+        float lo = -INFINITY, hi = -INFINITY;
+        for (int hh = 0; hh < r.G; ++hh) {
+            const float2 v = __ldcg(&r.scr[hh * r.scr_hs + c]);
+            fold_interval(v.x, v.y, lo, hi);
+        }
+        float2 o;
+        interval_mid(lo, hi, o.x, o.y);
+        return o;
+    }
+}
+
+// Largest screen value and largest radius of 64-chunk group g: for a group of heads,
+// the largest over its heads of each (the value is still attained by one chunk of the
+// group, whose group score is at least that value minus the largest radius).
+template <bool kGroup>
+__device__ __forceinline__ float2 gmax_at(const ScrRows &r, int g) {
+    float2 m = __ldcg(&r.gmx[g]);
+    if constexpr (kGroup) {
+        for (int hh = 1; hh < r.G; ++hh) {
+            const float2 v = __ldcg(&r.gmx[hh * r.gmx_hs + g]);
+            m.x = fmaxf(m.x, v.x);
+            m.y = fmaxf(m.y, v.y);
+        }
+    }
+    return m;
+}
+
 __device__ __forceinline__ ScreenWs screen_ws(const SelectArgs &a) {
     const int64_t nq = (int64_t)a.B * a.H * a.Lq;
     ScreenWs w;
@@ -113,23 +182,56 @@ __device__ __forceinline__ ScreenWs screen_ws(const SelectArgs &a) {
     return w;
 }
 
-// Exact top-K of one query from the screen values in the workspace (all NT threads of
-// a CTA, NT <= 256; every step below is one parallel round trip to L2).
-template <typename T, int D, int NT>
-__device__ void pick_query(const SelectArgs &a, const ScreenWs &ws, int64_t qi, PickSmem &ps) {
+// Exact top-K of one unit from the screen values in the workspace (all NT threads of
+// a CTA, NT <= 256; every step below is one parallel round trip to L2). A unit is one
+// query (kGroup = false) or, for grouped heads, one (b, group, query) whose chunks are
+// ranked by the maximum over the group's heads of their scores.
+template <typename T, int D, int NT, bool kGroup>
+__device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, PickSmem &ps) {
+    using Ctx = std::conditional_t<kGroup, GroupCtx, QueryCtx>;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    int t;
-    const QueryCtx q = make_ctx<T, D>(a, qi, t);
-    for (int x = tid; x < D; x += NT) ps.qs[x] = (float)static_cast<const T *>(q.qrow)[x];
+    int t, b = 0, grp = 0, i = 0;
+    Ctx q;
+    ScrRows rows;
+    rows.G = 1;
+    rows.scr_hs = (int64_t)a.Lq * a.C;
+    rows.gmx_hs = (int64_t)a.Lq * groups_of(a.C);
+    int64_t q0 = u;  // the unit's first query head's query index
+    if constexpr (kGroup) {
+        q = make_group_ctx<T, D>(a, u, t, b, grp, i);
+        q0 = ((int64_t)b * a.H + (int64_t)grp * a.G) * a.Lq + i;
+        rows.G = a.G;
+        for (int hh = 0; hh < a.G; ++hh)
+            for (int x = tid; x < D; x += NT)
+                ps.qs[hh * D + x] = (float)static_cast<const T *>(q.head.qrow)[hh * q.qsh + x];
+    } else {
+        q = make_ctx<T, D>(a, u, t);
+        for (int x = tid; x < D; x += NT) ps.qs[x] = (float)static_cast<const T *>(q.qrow)[x];
+    }
+    rows.scr = ws.scr + q0 * a.C;
+    rows.gmx = ws.gmax + q0 * groups_of(a.C);
+    auto write = [&](const EntryList &list) {
+        if constexpr (kGroup) group_write<T, D>(q, ps.qs, list, a, u, b, grp, i);
+        else warp_write(list, a.topk, u, a.idx, a.score, a.nsel);
+    };
     const int ne = eligible(t, a.C);
     const int K = a.topk;
-    const float2 *scr = ws.scr + qi * a.C;
     if (ne <= K) {  // every eligible chunk is kept, in index order
-        for (int r = tid; r < K; r += NT) {
-            a.idx[qi * K + r] = r < ne ? r : -1;
-            a.score[qi * K + r] = r < ne ? __ldcg(&scr[r]).x : -INFINITY;
+        if constexpr (kGroup) {
+            __syncthreads();  // ps.qs complete
+            if (w == 0) {
+                if (lane < ne) ps.out.idx[lane] = lane;
+                if (lane == 0) ps.out.n = ne;
+                __syncwarp();
+                write(ps.out);
+            }
+        } else {
+            for (int r = tid; r < K; r += NT) {
+                a.idx[u * K + r] = r < ne ? r : -1;
+                a.score[u * K + r] = r < ne ? __ldcg(&rows.scr[r]).x : -INFINITY;
+            }
+            if (tid == 0) a.nsel[u] = ne;
         }
-        if (tid == 0) a.nsel[qi] = ne;
         return;
     }
     const int G = groups_of(ne);
@@ -137,16 +239,15 @@ __device__ void pick_query(const SelectArgs &a, const ScreenWs &ws, int64_t qi, 
     if (G < K + 1) {  // short table: the exact running-list scan over every chunk
         if (w == 0) {
             warp_scan<T, D>(q, ps.qs, 0, ne, K, ps.out);
-            warp_write(ps.out, K, qi, a.idx, a.score, a.nsel);
+            write(ps.out);
         }
         return;
     }
     // T = (K+1)-th largest maximum of the 64-chunk groups (attained by K+1 distinct
     // chunks); e_max = largest radius; every chunk with hi < T - e_max is certainly out
-    const float2 *gmx = ws.gmax + qi * groups_of(a.C);
     float em = 0.f;
     for (int g = tid; g < G; g += NT) {
-        const float2 v = __ldcg(&gmx[g]);
+        const float2 v = gmax_at<kGroup>(rows, g);
         ps.gm[g] = v;
         em = fmaxf(em, v.y);
     }
@@ -178,7 +279,7 @@ __device__ void pick_query(const SelectArgs &a, const ScreenWs &ws, int64_t qi, 
         for (int j = 0; j < 4; ++j) {
             const int k = k0 + (j >> 1) * (NT / 32);
             const int c = k < ncg ? ps.cand_g[k] * kGroupRows + (j & 1) * 32 + lane : ne;
-            v[j] = c < ne ? __ldcg(&scr[c]) : make_float2(-INFINITY, 0.f);
+            v[j] = c < ne ? scr_at<kGroup>(rows, c) : make_float2(-INFINITY, 0.f);
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -218,7 +319,7 @@ __device__ void pick_query(const SelectArgs &a, const ScreenWs &ws, int64_t qi, 
             const int n = warp_append<2>(sl, keep, ps.out, 0);
             if (lane == 0) ps.out.n = n;
             __syncwarp();
-            warp_write(ps.out, K, qi, a.idx, a.score, a.nsel);
+            write(ps.out);
         }
         return;
     }
@@ -227,7 +328,7 @@ __device__ void pick_query(const SelectArgs &a, const ScreenWs &ws, int64_t qi, 
     int n = 0;
     for (int c0 = 0; c0 < ne; c0 += 32) {
         const int c = c0 + lane;
-        const float2 v = c < ne ? __ldcg(&scr[c]) : make_float2(-INFINITY, 0.f);
+        const float2 v = c < ne ? scr_at<kGroup>(rows, c) : make_float2(-INFINITY, 0.f);
         const bool cand = c < ne && __fadd_ru(v.x, v.y) >= cut;
         if (!__any_sync(kFull, cand)) continue;
         Slots<2> sl;
@@ -247,7 +348,7 @@ __device__ void pick_query(const SelectArgs &a, const ScreenWs &ws, int64_t qi, 
     }
     if (lane == 0) ps.out.n = n;
     __syncwarp();
-    warp_write(ps.out, K, qi, a.idx, a.score, a.nsel);
+    write(ps.out);
 }
 
 }  // namespace

@@ -30,9 +30,18 @@
 //      ascending chunk index with the float32 screen values.
 // Rows whose candidates or band entries exceed the list capacity (heavy ties) are
 // finished by the warp routine of the other select kernels, which is exact for any
-// input. Both mbarrier waits are bounded; on expiry the CTA sets the status word,
+// input. Every mbarrier wait is bounded; on expiry the CTA sets the status word,
 // waits (bounded) for the copies and MMAs it started, frees its TMEM and writes no
 // output.
+//
+// Grouped heads (summary page, Methodology 3, GQA adaptation): a CTA takes 128 queries
+// of one (b, group) and puts S_h = Q~_h K'_h^T of each of the group's G heads into its
+// own TMEM columns (the heads' operands pass through two shared-memory buffers). A
+// chunk's group value is the maximum over the heads of s_h,c; each pass folds the
+// heads' intervals s_h,c +- e_h,c into [max lo, max hi] and works on its centre and
+// radius, so the steps above apply unchanged with e_max the row's largest radius. The
+// band's float64 score is the largest of the heads' float64 scores, and each head's
+// output score of a kept chunk is its own screen value, read back from its columns.
 #include "select_common.cuh"
 #include "tc_common.cuh"
 
@@ -44,13 +53,14 @@ using namespace tc;
 constexpr int kQM = 128;           // queries per CTA (TMEM lanes)
 constexpr int kHD = 128;           // head dimension
 constexpr int kTcThreads = 128;
-constexpr int kMaxCols = 512;      // eligible chunks per CTA held in TMEM
+constexpr int kMaxCols = 512;      // TMEM columns: eligible chunks per CTA times the heads
 constexpr int kCap = 32;           // candidate slots per query (one spare slot absorbs overflow)
 constexpr int kBandCap = 8;        // float64 rescoring slots per query
 constexpr int kCollectPasses = 6;
 constexpr long long kSelWaitLimit = 1ll << 26;
+constexpr int kQBytes = 2 * kQM * 128;  // one head's query tile: 2 column blocks x 128 rows x 128 B
 
-// Reused region (after the MMA has read the operands): per-thread candidate lists,
+// Reused region (after the MMAs have read the operands): per-thread candidate lists,
 // band scores, the CTA's work list and the fallback's scratch.
 constexpr int kListS = 0;                                  // float  [kCap + 1][128]
 constexpr int kListC = kListS + (kCap + 1) * kQM * 4;      // uint16 [kCap + 1][128]
@@ -60,12 +70,17 @@ constexpr int kWork = kBandJ + kBandCap * kQM;             // uint16 [128 * kBan
 constexpr int kFbQ = kWork + kQM * kBandCap * 2;           // float  [4][128]
 constexpr int kFbList = kFbQ + 4 * kHD * 4;                // EntryList [4]
 constexpr int kReuseBytes = kFbList + 4 * kListBytes;
+// grouped heads also keep each candidate's radius, and the fallback needs the query
+// rows of all the group's heads
+constexpr int kListE = kReuseBytes;                        // float  [kCap + 1][128]
+constexpr int kFbQG = kListE + (kCap + 1) * kQM * 4;       // float  [4][kMaxGroup][128]
+constexpr int kReuseBytesG = kFbQG + 4 * kMaxGroup * kHD * 4;
 static_assert(kBandX % 8 == 0 && kFbList % 8 == 0, "alignment");
-static_assert(kReuseBytes <= 32768 + 2 * 64 * 128, "reused region fits the smallest operand area");
+static_assert(kReuseBytes <= kQBytes + 2 * 64 * 128, "reused region fits the smallest operand area");
+static_assert(kReuseBytesG <= 2 * (kQBytes + 2 * 64 * 128), "grouped reused region fits two operand buffers");
 
 struct Misc {
-    unsigned long long bar[2];  // operands loaded, MMA done
-    uint32_t qmag[kQM];         // per query row: smallest nonzero | largest bf16 magnitude << 16
+    unsigned long long bar[5];  // operands loaded (2 buffers), MMAs read a buffer (2), all MMAs done
     uint32_t tmem;
     uint32_t abort;
     int nc;
@@ -75,24 +90,31 @@ struct Misc {
     uint8_t ovf[kQM];
 };
 
+// Shared memory: nbuf operand buffers (a head's query tile, then its first ncpad summary
+// rows, both as 2 column blocks with the 128-byte swizzle), then per head the biases,
+// norms and magnitude ranges of its summary rows and of the query rows.
 struct Layout {
-    int kp, bias, kn, kmag, misc, total;
+    int buf, nbuf, bias, kn, kmag, qmag, qn, misc, total;
 };
-__host__ __device__ inline Layout layout(int ncpad) {
+__host__ __device__ inline Layout layout(int ncpad, int G) {
     Layout L;
-    L.kp = 32768;                          // Q: 2 column blocks x 128 rows x 128 B
-    L.bias = L.kp + 2 * ncpad * 128;       // summary rows: 2 column blocks x ncpad x 128 B
-    L.kn = L.bias + ncpad * 4;
-    L.kmag = L.kn + ncpad * 4;             // per summary row: magnitude range as in Misc::qmag
-    L.misc = L.kmag + ncpad * 4;
+    L.buf = kQBytes + 2 * ncpad * 128;
+    L.nbuf = G < 2 ? G : 2;
+    L.bias = L.nbuf * L.buf;               // float [G][ncpad]
+    L.kn = L.bias + G * ncpad * 4;         // float [G][ncpad]
+    L.kmag = L.kn + G * ncpad * 4;         // uint32 [G][ncpad]: smallest nonzero | largest magnitude << 16
+    L.qmag = L.kmag + G * ncpad * 4;       // uint32 [G][128], as kmag for the query rows
+    L.qn = L.qmag + G * kQM * 4;           // float [G][128]
+    L.misc = L.qn + G * kQM * 4;
     L.total = L.misc + (int)sizeof(Misc);
     return L;
 }
 
 struct TcSelArgs {
     SelectArgs a;
-    int ncpad;      // summary rows staged per CTA at most (multiple of 64)
-    uint32_t cols;  // TMEM columns allocated (power of two >= ncpad)
+    int ncpad;      // summary rows staged per CTA and head at most (multiple of 64)
+    uint32_t hcols; // TMEM columns per head (power of two >= ncpad)
+    uint32_t cols;  // TMEM columns allocated (power of two >= G * hcols)
     uint32_t *status;
 };
 
@@ -164,6 +186,7 @@ __device__ double exact_score_f32prod(const bf16 *qrow, const bf16 *krow, float 
     return __dadd_rn(__dmul_rn(acc, (double)scale), (double)bias);
 }
 
+template <bool kGroup>
 __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                 const __grid_constant__ CUtensorMap tmK,
                                                                 TcSelArgs args) {
@@ -173,17 +196,23 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const SelectArgs &a = args.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = kGroup ? a.G : 1;
     const int i0 = blockIdx.x * kQM;
-    const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+    const int units = a.H / G;                                   // heads, or groups, per batch
+    const int b = blockIdx.y / units, h0 = (blockIdx.y % units) * G;  // the CTA's first query head
     const int K = a.topk;
     const int ncpad = args.ncpad;
-    const Layout L = layout(ncpad);
+    const Layout L = layout(ncpad, G);
     const uint32_t sbase = smem_u32(smem);
     float *bias_s = reinterpret_cast<float *>(smem + L.bias);
     float *kn_s = reinterpret_cast<float *>(smem + L.kn);
     uint32_t *kmag_s = reinterpret_cast<uint32_t *>(smem + L.kmag);
+    uint32_t *qmag_s = reinterpret_cast<uint32_t *>(smem + L.qmag);
+    float *qn_s = reinterpret_cast<float *>(smem + L.qn);
     Misc *misc = reinterpret_cast<Misc *>(smem + L.misc);
-    const uint32_t bar_load = smem_u32(&misc->bar[0]), bar_mma = smem_u32(&misc->bar[1]);
+    const uint32_t bar_load[2] = {smem_u32(&misc->bar[0]), smem_u32(&misc->bar[1])};
+    const uint32_t bar_read[2] = {smem_u32(&misc->bar[2]), smem_u32(&misc->bar[3])};
+    const uint32_t bar_done = smem_u32(&misc->bar[4]);
 
     // ---- positions; the CTA's eligible range
     const int i = i0 + tid;
@@ -197,8 +226,7 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
         misc->nwork = 0;
         misc->novf = 0;
         misc->abort = 0u;
-        mbar_init(bar_load, 1);
-        mbar_init(bar_mma, 1);
+        for (int k = 0; k < 5; ++k) mbar_init(smem_u32(&misc->bar[k]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncthreads();
@@ -209,16 +237,30 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
     const int nrows = (nc + 63) & ~63;
 
     volatile uint32_t *abort_flag = &misc->abort;
-    auto wait = [&](uint32_t barrier) {
+    auto wait = [&](uint32_t barrier, uint32_t parity) {
         if (*abort_flag) return false;
         for (long long it = 0; it < kSelWaitLimit; ++it)
-            if (mbar_try_wait(barrier, 0)) return true;
+            if (mbar_try_wait(barrier, parity)) return true;
         *abort_flag = 1u;
         atomicOr(args.status, 1u);
         return false;
     };
 
-    bool issued_load = false, issued_mma = false;  // thread 0's record
+    // thread 0's record of what it started: loads per buffer, MMAs, the final commit
+    int loads[2] = {0, 0};
+    bool issued_mma = false, committed = false;
+    auto issue_load = [&](int hh) {  // head hh's operands into buffer hh & 1 (thread 0)
+        const int bf = hh & 1;
+        const uint32_t dst = sbase + bf * L.buf;
+        ++loads[bf];
+        mbar_expect_tx(bar_load[bf], kQBytes + 2 * nrows * 128);
+        tma_load_4d(dst, &tmQ, bar_load[bf], 0, i0, h0 + hh, b);
+        tma_load_4d(dst + 16384, &tmQ, bar_load[bf], 64, i0, h0 + hh, b);
+        for (int r0 = 0; r0 < nrows; r0 += 64) {
+            tma_load_4d(dst + kQBytes + r0 * 128, &tmK, bar_load[bf], 0, r0, h0 + hh, b);
+            tma_load_4d(dst + kQBytes + ncpad * 128 + r0 * 128, &tmK, bar_load[bf], 64, r0, h0 + hh, b);
+        }
+    };
     if (nc > 0) {
         if (warp == 0) {
             asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
@@ -226,67 +268,85 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
                          "r"(args.cols));
             asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
         }
-        if (tid == 0) {
-            issued_load = true;
-            mbar_expect_tx(bar_load, 2 * kQM * 128 + 2 * nrows * 128);
-            tma_load_4d(sbase, &tmQ, bar_load, 0, i0, h, b);
-            tma_load_4d(sbase + 16384, &tmQ, bar_load, 64, i0, h, b);
-            for (int r0 = 0; r0 < nrows; r0 += 64) {
-                tma_load_4d(sbase + L.kp + r0 * 128, &tmK, bar_load, 0, r0, h, b);
-                tma_load_4d(sbase + L.kp + ncpad * 128 + r0 * 128, &tmK, bar_load, 64, r0, h, b);
-            }
+        if (tid == 0)
+            for (int hh = 0; hh < L.nbuf; ++hh) issue_load(hh);
+        for (int hh = 0; hh < G; ++hh) {
+            const float *bhead = a.Bsum + ((int64_t)b * a.H + h0 + hh) * a.C;
+            for (int c = tid; c < nc; c += kTcThreads) bias_s[hh * ncpad + c] = __ldg(bhead + c);
         }
-        const float *bhead = a.Bsum + (int64_t)bh * a.C;
-        for (int c = tid; c < nc; c += kTcThreads) bias_s[c] = __ldg(bhead + c);
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
     }
     const uint32_t tmem = nc > 0 ? misc->tmem : 0u;
 
-    // ---- operands in shared memory: norms, then S = Q~ K'^T into TMEM
-    float qn = 0.f;
-    if (nc > 0 && wait(bar_load)) {
-        float knm = 0.f;
-        for (int c = tid; c < nc; c += kTcThreads) {
-            uint32_t km;
-            const float kn = sqrtf(row_stats(smem + L.kp, ncpad * 128, c, km));
-            kn_s[c] = kn;
-            kmag_s[c] = km;
-            knm = fmaxf(knm, kn);
-        }
-        knm = warp_max(knm);
-        if (lane == 0) atomicMax(&misc->knmax, __float_as_uint(knm));  // non-negative floats order as integers
-        uint32_t qm;
-        qn = sqrtf(row_stats(smem, 16384, tid, qm));
-        misc->qmag[tid] = qm;
-        if (tid == 0) {
-            tc_fence_after();
-            const int nblk = (nrows + 255) / 256;
-            for (int nb = 0; nb < nblk; ++nb) {
-                const int n = min(256, nrows - nb * 256);
-                const uint32_t idesc = idesc_bf16(kQM, n, false);
+    // ---- per head: operands in shared memory, their norms, then S_h = Q~_h K'_h^T into
+    // TMEM columns [hh * hcols, hh * hcols + nrows)
+    if (nc > 0) {
+        for (int hh = 0; hh < G; ++hh) {
+            const int bf = hh & 1;
+            const uint32_t ph = (uint32_t)(hh >> 1) & 1u;
+            const uint8_t *buf = smem + bf * L.buf;
+            if (wait(bar_load[bf], ph)) {
+                float knm = 0.f;
+                for (int c = tid; c < nc; c += kTcThreads) {
+                    uint32_t km;
+                    const float kn = sqrtf(row_stats(buf + kQBytes, ncpad * 128, c, km));
+                    kn_s[hh * ncpad + c] = kn;
+                    kmag_s[hh * ncpad + c] = km;
+                    knm = fmaxf(knm, kn);
+                }
+                if (!kGroup) {
+                    knm = warp_max(knm);
+                    if (lane == 0) atomicMax(&misc->knmax, __float_as_uint(knm));  // non-negative floats order as integers
+                }
+                uint32_t qm;
+                qn_s[hh * kQM + tid] = sqrtf(row_stats(buf, 16384, tid, qm));
+                qmag_s[hh * kQM + tid] = qm;
+                if (tid == 0 && !*abort_flag) {
+                    tc_fence_after();
+                    const uint32_t ob = sbase + bf * L.buf;
+                    const int nblk = (nrows + 255) / 256;
+                    for (int nb = 0; nb < nblk; ++nb) {
+                        const int n = min(256, nrows - nb * 256);
+                        const uint32_t idesc = idesc_bf16(kQM, n, false);
 #pragma unroll
-                for (int ks = 0; ks < kHD / 16; ++ks) {
-                    const uint32_t qa = sbase + (ks >> 2) * 16384 + (ks & 3) * 32;
-                    const uint32_t ka = sbase + L.kp + (ks >> 2) * (ncpad * 128) + nb * 256 * 128 + (ks & 3) * 32;
-                    mma_ss(tmem + nb * 256, smem_desc(qa, 16, 1024), smem_desc(ka, 16, 1024), idesc, ks > 0);
+                        for (int ks = 0; ks < kHD / 16; ++ks) {
+                            const uint32_t qa = ob + (ks >> 2) * 16384 + (ks & 3) * 32;
+                            const uint32_t ka = ob + kQBytes + (ks >> 2) * (ncpad * 128) + nb * 256 * 128 + (ks & 3) * 32;
+                            mma_ss(tmem + hh * args.hcols + nb * 256, smem_desc(qa, 16, 1024), smem_desc(ka, 16, 1024),
+                                   idesc, ks > 0);
+                        }
+                    }
+                    issued_mma = true;
+                    if (hh + 2 < G) mma_commit(bar_read[bf]);
+                    if (hh == G - 1) {
+                        mma_commit(bar_done);
+                        committed = true;
+                    }
                 }
             }
-            issued_mma = true;
-            mma_commit(bar_mma);
+            if (hh + 2 < G) {  // reload buffer bf with head hh + 2 once its MMAs have read it
+                __syncthreads();  // every thread's norms of head hh are done
+                if (tid == 0 && issued_mma && !*abort_flag && wait(bar_read[bf], ph)) issue_load(hh + 2);
+            }
         }
     }
     __syncthreads();
-    if (nc > 0) wait(bar_mma);
+    if (nc > 0) wait(bar_done, 0);
     tc_fence_after();
     __syncthreads();
     if (*abort_flag) {  // uniform: read after the barrier
         if (tid == 0) {  // let every started copy and MMA complete before leaving
-            for (int w = 0; w < 2; ++w) {
-                if (!(w == 0 ? issued_load : issued_mma)) continue;
+            for (int bf = 0; bf < 2; ++bf) {
+                if (loads[bf] == 0) continue;  // each load was issued after the previous one of its buffer completed
                 for (long long it = 0; it < kSelWaitLimit; ++it)
-                    if (mbar_try_wait(w == 0 ? bar_load : bar_mma, 0)) break;
+                    if (mbar_try_wait(bar_load[bf], (uint32_t)(loads[bf] - 1) & 1u)) break;
+            }
+            if (issued_mma) {
+                if (!committed) mma_commit(bar_done);
+                for (long long it = 0; it < kSelWaitLimit; ++it)
+                    if (mbar_try_wait(bar_done, 0)) break;
             }
         }
         tc_fence_before();
@@ -301,38 +361,72 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
     // ---- per-row selection (thread = query row = TMEM lane)
     float *ls = reinterpret_cast<float *>(smem + kListS);
     uint16_t *lc = reinterpret_cast<uint16_t *>(smem + kListC);
+    float *le = reinterpret_cast<float *>(smem + kListE);
     double *bx = reinterpret_cast<double *>(smem + kBandX);
     uint8_t *bj_s = smem + kBandJ;
     uint16_t *work = reinterpret_cast<uint16_t *>(smem + kWork);
     const float sc = a.scale;
-    const float eq = sc * qn * ((float)kHD * 0x1p-16f) * (1.f + 0x1p-8f);
+    const float eq = sc * qn_s[tid] * ((float)kHD * 0x1p-16f) * (1.f + 0x1p-8f);
     const float knmax = __uint_as_float(misc->knmax);
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     const int nbat = (ne_w + 31) >> 5;  // warp-uniform: tcgen05.ld is warp-collective
-    auto for_each = [&](auto &&f) {     // f(c, s) over this row's eligible chunks, ascending
+    // f(c, s, e) over this row's eligible chunks, ascending; e is the radius for grouped
+    // heads (unused for one head, whose radius follows from |k'_c|)
+    auto for_each = [&](auto &&f) {
         for (int bi = 0; bi < nbat; ++bi) {
-            uint32_t r[32];
-            tmem_ld32(trow + bi * 32, r);
-            tmem_wait_ld();
+            if constexpr (!kGroup) {
+                uint32_t r[32];
+                tmem_ld32(trow + bi * 32, r);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int c = bi * 32 + j;
-                if (c < ne) f(c, fmaf(__uint_as_float(r[j]), sc, bias_s[c]));
+                for (int j = 0; j < 32; ++j) {
+                    const int c = bi * 32 + j;
+                    if (c < ne) f(c, fmaf(__uint_as_float(r[j]), sc, bias_s[c]), 0.f);
+                }
+            } else {
+                float lo[32], hi[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) lo[j] = hi[j] = -INFINITY;
+                for (int hh = 0; hh < G; ++hh) {
+                    uint32_t r[32];
+                    tmem_ld32(trow + hh * args.hcols + bi * 32, r);
+                    tmem_wait_ld();
+                    const float eqh = sc * qn_s[hh * kQM + tid] * ((float)kHD * 0x1p-16f) * (1.f + 0x1p-8f);
+                    const float *bh = bias_s + hh * ncpad + bi * 32;
+                    const float *kh = kn_s + hh * ncpad + bi * 32;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if (bi * 32 + j < ne) {
+                            const float sh = fmaf(__uint_as_float(r[j]), sc, bh[j]);
+                            fold_interval(sh, fmaf(eqh, kh[j], fabsf(sh) * 0x1p-22f), lo[j], hi[j]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int c = bi * 32 + j;
+                    if (c < ne) {
+                        float s, e;
+                        interval_mid(lo[j], hi[j], s, e);
+                        f(c, s, e);
+                    }
+                }
             }
         }
     };
 
     // pass A: range and moments of the row (shifted by b'_0, which lies near every s)
     const float sref = nc > 0 ? bias_s[0] : 0.f;
-    float mn = INFINITY, mx = -INFINITY, sum = 0.f, sq = 0.f;
-    for_each([&](int, float s) {
+    float mn = INFINITY, mx = -INFINITY, sum = 0.f, sq = 0.f, emx = 0.f;
+    for_each([&](int, float s, float e) {
         mn = fminf(mn, s);
         mx = fmaxf(mx, s);
         const float dv = s - sref;
         sum += dv;
         sq = fmaf(dv, dv, sq);
+        if (kGroup) emx = fmaxf(emx, e);
     });
-    const float emax = fmaf(eq, knmax, fmaxf(fabsf(mn), fabsf(mx)) * 0x1p-22f);
+    const float emax = kGroup ? emx : fmaf(eq, knmax, fmaxf(fabsf(mn), fabsf(mx)) * 0x1p-22f);
 
     // candidate list: collect s >= tcut; certify or move the guess g and collect again
     float g = -INFINITY;  // -inf: take every eligible chunk (rows with ne <= K + 4)
@@ -351,12 +445,13 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
     for (int pass = 0; pass < kCollectPasses && __any_sync(kFull, pending); ++pass) {
         const float tcut = g == -INFINITY ? -INFINITY : __fsub_rd(__fsub_rd(g, emax), emax);
         int mm = 0;
-        for_each([&](int c, float s) {
+        for_each([&](int c, float s, float e) {
             const bool take = pending && s >= tcut;
             const int slot = min(mm, kCap);  // entries past the capacity land in the spare slot
             if (take) {
                 ls[slot * kQM + tid] = s;
                 lc[slot * kQM + tid] = (uint16_t)c;
+                if (kGroup) le[slot * kQM + tid] = e;
             }
             mm += take ? 1 : 0;
         });
@@ -395,13 +490,15 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
             g = 0.5f * (lo_g + g);
         }
     }
-    // TMEM is no longer needed
-    tc_fence_before();
-    __syncthreads();
-    if (nc > 0 && warp == 0) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(args.cols));
-    }
+    auto free_tmem = [&]() {
+        tc_fence_before();
+        __syncthreads();
+        if (nc > 0 && warp == 0) {
+            tc_fence_after();
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(args.cols));
+        }
+    };
+    if (!kGroup) free_tmem();  // one head: TMEM is no longer needed
 
     // classification on the certified list
     bool overflow = pending;
@@ -415,7 +512,7 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
             const float hi_cut = __fadd_ru(sK1, emax);
             for (int j = 0; j < m; ++j) {
                 const float s = ls[j * kQM + tid];
-                const float e = fmaf(eq, kn_s[lc[j * kQM + tid]], fabsf(s) * 0x1p-22f);
+                const float e = kGroup ? le[j * kQM + tid] : fmaf(eq, kn_s[lc[j * kQM + tid]], fabsf(s) * 0x1p-22f);
                 if (__fsub_rd(s, e) > hi_cut) keep |= 1u << j;
                 else if (__fadd_ru(s, e) >= lo_cut) bandm |= 1u << j;
             }
@@ -443,24 +540,39 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
     if (overflow) misc->ovf[atomicAdd(&misc->novf, 1)] = (uint8_t)tid;
     __syncthreads();
 
-    // float64 scores of the band entries, spread over the CTA
+    // float64 scores of the band entries, spread over the CTA (grouped heads: the
+    // largest of the heads' scores)
     const int nwork = misc->nwork;
-    const int64_t qbase = (int64_t)bh * a.Lq + i0;
+    const int64_t qbase = (int64_t)blockIdx.y * a.Lq + i0;  // the CTA's first unit (query, or group query)
     for (int w = tid; w < nwork; w += kTcThreads) {
         const int row = work[w] >> 3, k = work[w] & 7;
         const int c = lc[bj_s[k * kQM + row] * kQM + row];
+        double x = -INFINITY;
         int tq;
-        const QueryCtx q = make_ctx<bf16, kHD>(a, qbase + row, tq);
-        bx[k * kQM + row] =
-            products_exact_f32(misc->qmag[row], kmag_s[c])
-                ? exact_score_f32prod(static_cast<const bf16 *>(q.qrow),
-                                      static_cast<const bf16 *>(q.khead) + (int64_t)c * q.kst, sc, q.bhead[c])
-                : exact_score<bf16, kHD>(q, c);
+        QueryCtx q;
+        GroupCtx gq;
+        if (kGroup) {
+            int bb, gg, ii;
+            gq = make_group_ctx<bf16, kHD>(a, qbase + row, tq, bb, gg, ii);
+        } else {
+            q = make_ctx<bf16, kHD>(a, qbase + row, tq);
+        }
+        for (int hh = 0; hh < G; ++hh) {
+            if (kGroup) q = head_ctx(gq, hh, (int)sizeof(bf16));
+            const double xh =
+                products_exact_f32(qmag_s[hh * kQM + row], kmag_s[hh * ncpad + c])
+                    ? exact_score_f32prod(static_cast<const bf16 *>(q.qrow),
+                                          static_cast<const bf16 *>(q.khead) + (int64_t)c * q.kst, sc, q.bhead[c])
+                    : exact_score<bf16, kHD>(q, c);
+            x = fmax(x, xh);
+        }
+        bx[k * kQM + row] = x;
     }
     __syncthreads();
 
     // the band's best `need` by (float64 score desc, chunk asc), then the output row
-    if (!overflow && row_ok) {
+    const bool write_row = !overflow && row_ok;
+    if (write_row) {
         if (need > 0) {
             uint32_t taken = 0;
             for (int r = 0; r < need; ++r) {
@@ -487,60 +599,114 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
         for (int j = 0; j < m; ++j) {
             if (keep >> j & 1u) {
                 orow[o] = lc[j * kQM + tid];
-                srow[o] = ls[j * kQM + tid];
+                if (!kGroup) srow[o] = ls[j * kQM + tid];
                 ++o;
             }
         }
         a.nsel[qi] = o;
         for (; o < K; ++o) {
             orow[o] = -1;
-            srow[o] = -INFINITY;
+            if (!kGroup) srow[o] = -INFINITY;
         }
+    }
+    if constexpr (kGroup) {
+        // each head's own screen value of the kept chunks, read back from its columns
+        // (every lane takes part in the warp-collective loads)
+        const int mk = write_row ? m : 0;
+        int jj = 0, obase = 0;
+        for (int bi = 0; bi < nbat; ++bi) {
+            uint32_t msk = 0u;  // kept chunks of this 32-chunk batch (the list ascends)
+            for (; jj < mk && lc[jj * kQM + tid] < (bi + 1) * 32; ++jj)
+                if (keep >> jj & 1u) msk |= 1u << (lc[jj * kQM + tid] - bi * 32);
+            for (int hh = 0; hh < G; ++hh) {
+                uint32_t r[32];
+                tmem_ld32(trow + hh * args.hcols + bi * 32, r);
+                tmem_wait_ld();
+                if (msk == 0u) continue;
+                float *srow = a.score + (((int64_t)b * a.H + h0 + hh) * a.Lq + i) * K;
+                const float *bh = bias_s + hh * ncpad + bi * 32;
+                int o = obase;
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (msk >> j & 1u) srow[o++] = fmaf(__uint_as_float(r[j]), sc, bh[j]);
+            }
+            obase += __popc(msk);
+        }
+        if (write_row)
+            for (int hh = 0; hh < G; ++hh) {
+                float *srow = a.score + (((int64_t)b * a.H + h0 + hh) * a.Lq + i) * K;
+                for (int o = obase; o < K; ++o) srow[o] = -INFINITY;
+            }
+        free_tmem();
     }
 
     // rows beyond the list capacity: the exact warp routine, one row per warp
     const int novf = misc->novf;
     if (novf > 0) {
-        float *qs = reinterpret_cast<float *>(smem + kFbQ) + warp * kHD;
         EntryList &list = *reinterpret_cast<EntryList *>(smem + kFbList + warp * kListBytes);
         for (int r = warp; r < novf; r += kTcThreads / 32) {
             const int row = misc->ovf[r];
             int tq;
-            const QueryCtx q = make_ctx<bf16, kHD>(a, qbase + row, tq);
-            load_query_f32<bf16, kHD>(q, qs);
-            __syncwarp();
-            warp_scan<bf16, kHD>(q, qs, 0, eligible(tq, a.C), K, list);
-            warp_write(list, K, qbase + row, a.idx, a.score, a.nsel);
+            if constexpr (kGroup) {
+                float *qs = reinterpret_cast<float *>(smem + kFbQG) + warp * kMaxGroup * kHD;
+                int bb, gg, ii;
+                const GroupCtx q = make_group_ctx<bf16, kHD>(a, qbase + row, tq, bb, gg, ii);
+                for (int hh = 0; hh < G; ++hh) load_query_f32<bf16, kHD>(head_ctx(q, hh, (int)sizeof(bf16)), qs + hh * kHD);
+                __syncwarp();
+                warp_scan<bf16, kHD>(q, qs, 0, eligible(tq, a.C), K, list);
+                group_write<bf16, kHD>(q, qs, list, a, qbase + row, bb, gg, ii);
+            } else {
+                float *qs = reinterpret_cast<float *>(smem + kFbQ) + warp * kHD;
+                const QueryCtx q = make_ctx<bf16, kHD>(a, qbase + row, tq);
+                load_query_f32<bf16, kHD>(q, qs);
+                __syncwarp();
+                warp_scan<bf16, kHD>(q, qs, 0, eligible(tq, a.C), K, list);
+                warp_write(list, K, qbase + row, a.idx, a.score, a.nsel);
+            }
             __syncwarp();
         }
     }
 }
 
-constexpr int kMaxSmem = 1024 + 32768 + 2 * kMaxCols * 128 + kMaxCols * 12 + (int)sizeof(Misc);
+constexpr int kMaxSmem = 227 * 1024;  // the opt-in limit; each launch asks for what it uses
 
 }  // namespace
 
-bool select_tc_supported(hils_dtype dt, int d, int B, int H, int Lq, int C, int K, bool has_qpos) {
+// TMEM columns per head for a CTA whose queries see at most nc chunks.
+static uint32_t head_cols(int nc) {
+    const int ncpad = (nc + 63) & ~63;
+    uint32_t hc = 64;
+    while ((int)hc < ncpad) hc <<= 1;
+    return hc;
+}
+
+bool select_tc_supported(hils_dtype dt, int d, int B, int H, int Lq, int C, int K, bool has_qpos, int G) {
     if (dt != HILS_BF16 || d != kHD || K < 1 || K > kCap - 4) return false;
-    if (C < 1 || Lq < 1 || (int64_t)B * H > 65535) return false;
-    // every query's eligible count fits the TMEM columns; with explicit positions that
-    // is only known for C itself
+    if (C < 1 || Lq < 1 || G < 1 || G > kMaxGroup || (int64_t)B * (H / G) > 65535) return false;
+    // every query's eligible count, times the heads, fits the TMEM columns; with
+    // explicit positions that is only known for C itself
     const int nc = has_qpos ? C : min(C, (Lq - 1) / kChunk);
-    return nc >= 1 && nc <= kMaxCols && C < 65536;
+    if (nc < 1 || C >= 65536) return false;
+    const int ncpad = (nc + 63) & ~63;
+    if ((int64_t)G * head_cols(nc) > kMaxCols) return false;
+    return layout(ncpad, G).total + 1024 <= 227 * 1024;
 }
 
 hils_status launch_select_tc(const SelectArgs &a, cudaStream_t s) {
+    const int G = a.G;
     const int nc = a.qpos ? a.C : min(a.C, (a.Lq - 1) / kChunk);
     const int ncpad = (nc + 63) & ~63;
-    uint32_t cols = 64;
-    while ((int)cols < ncpad) cols <<= 1;
+    const uint32_t hcols = head_cols(nc);
+    uint32_t cols = 32;
+    while (cols < (uint32_t)G * hcols) cols <<= 1;
     CUtensorMap mq, mk;
     if (!make_map(&mq, a.Qcal, a.B, a.H, a.Lq, kQM) || !make_map(&mk, a.Ksum, a.B, a.H, a.C, 64))
         return HILS_ERR_CUDA;
-    static KernelSetup setup;
-    hils_status st = kernel_setup(setup, (const void *)select_tc_kernel, kTcThreads, kMaxSmem, nullptr);
+    const void *fn = G > 1 ? (const void *)select_tc_kernel<true> : (const void *)select_tc_kernel<false>;
+    static KernelSetup setup1, setupg;
+    hils_status st = kernel_setup(G > 1 ? setupg : setup1, fn, kTcThreads, kMaxSmem, nullptr);
     if (st != HILS_OK) return st;
-    int smem = 1024 + layout(ncpad).total;
+    int smem = 1024 + layout(ncpad, G).total;
     // at most 512 / cols CTAs per SM may be resident, so that a TMEM allocation never
     // waits on another CTA: 228 KB of shared memory per SM shared by at most that many
     const int max_ctas = 512 / (int)cols;
@@ -548,10 +714,12 @@ hils_status launch_select_tc(const SelectArgs &a, cudaStream_t s) {
     TcSelArgs ta;
     ta.a = a;
     ta.ncpad = ncpad;
+    ta.hcols = hcols;
     ta.cols = cols;
     ta.status = static_cast<uint32_t *>(a.ws);
-    dim3 grid((a.Lq + kQM - 1) / kQM, a.B * a.H);
-    select_tc_kernel<<<grid, kTcThreads, smem, s>>>(mq, mk, ta);
+    dim3 grid((a.Lq + kQM - 1) / kQM, a.B * (a.H / G));
+    if (G > 1) select_tc_kernel<true><<<grid, kTcThreads, smem, s>>>(mq, mk, ta);
+    else select_tc_kernel<false><<<grid, kTcThreads, smem, s>>>(mq, mk, ta);
     return record_cuda_error(cudaGetLastError());
 }
 

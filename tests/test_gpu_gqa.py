@@ -20,6 +20,12 @@ PREFILL_GQA = {
     "bf16_d64_g2": WORKLOADS[7].replace(H=6, Hk=3, d=64, N=700, K=5, W=100),
     "fp32_d128_g2": WORKLOADS[1].replace(H=4, Hk=2, d=128, N=640 + 9, K=3, W=70),
     "fp32_d64_g3": WORKLOADS[1].replace(H=3, Hk=1, N=512 + 33, K=4, W=64),
+    # tensor-core select: three heads per group (one operand buffer reloaded), and two
+    # heads with 256 TMEM columns each
+    "bf16_d128_g3_tc": WORKLOADS[7].replace(H=6, Hk=2, N=1536 + 37),
+    "bf16_d128_g2_tc_long": WORKLOADS[7].replace(H=4, Hk=2, N=64 * 200 + 5, K=8, W=256),
+    # three heads whose tables exceed the TMEM columns: the warp-per-query group kernel
+    "bf16_d128_g3_warp_long": WORKLOADS[7].replace(H=3, Hk=1, N=64 * 180 + 7, K=8, W=256),
 }
 
 
