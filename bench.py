@@ -436,7 +436,9 @@ def run_profile_case(args):
     decode-select: the 512K decode geometry (H=32, 8191 eligible chunks, K=16) on a
                    random summary table (68 MB) without a KV cache;
     decode-attend: the decode attend with H=32, K=16, W=512 on a 128K-token cache (2.1 GB);
-    prefill:       the full 8K prefill workload (summarise, select, attend).
+    prefill:       the full 8K prefill workload (summarise, select, attend);
+    prefill-select: the select of the 8K prefill, multi-head then grouped-query (32 query
+                   heads, 8 key-value heads), `warmup + steps` launches each.
     Runs `warmup + steps` plain launches of the case and exits."""
     import hierarchical_chunk_sparse_b200 as hils
 
@@ -463,6 +465,17 @@ def run_profile_case(args):
         fn = db.attend
     elif case == "prefill":
         fn = PrefillBench(WORKLOADS[2], dev).step
+    elif case == "prefill-select":
+        benches = [PrefillBench(WORKLOADS[n], dev) for n in (2, 7)]
+        for pb in benches:
+            pb.summarize()
+        torch.cuda.synchronize()
+        for pb in benches:
+            for _ in range(args.warmup + args.steps):
+                pb.select()
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": case, "launches": 2 * (args.warmup + args.steps)}))
+        return
     else:
         raise SystemExit(f"unknown profile case {case}")
     for _ in range(args.warmup + args.steps):
@@ -552,7 +565,7 @@ def measure_decode(w, dev, stream, flush, args, world, peaks):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None,
-                    choices=["decode-select", "decode-attend", "prefill"],
+                    choices=["decode-select", "decode-attend", "prefill", "prefill-select"],
                     help="run a small case for an ncu capture and exit")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)

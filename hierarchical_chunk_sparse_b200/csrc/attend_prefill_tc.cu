@@ -3,13 +3,17 @@
 // query-packing kernel of its Efficiency section (adjacent queries share the union of
 // their kept chunks, so the per-chunk products are dense tensor-core tiles).
 //
-// A persistent CTA (one per SM) takes work items of 256 consecutive queries of one
-// (b, h): two 128-row query tiles A and B that share every key/value tile. Each item
-// walks 64-key tiles:
-//   1. the window tiles covering [max(0, t0-W+1), t0+255] (online softmax; a row's
+// A persistent CTA (one per SM) takes work items of two 128-row query tiles A and B
+// that share every key/value tile. A tile packs P query heads that share a key-value
+// head and, with grouped-query attention, their kept chunks (the summary page's
+// M x G >= 16 packing: P = the largest power of two <= 8 dividing the group size G),
+// each with 128 / P consecutive queries; an item covers 2 x 128 / P consecutive
+// queries t0.. of those heads (P = 1: 256 queries of one head). Each item walks 64-key
+// tiles:
+//   1. the window tiles covering [max(0, t0-W+1), last query] (online softmax; a row's
 //      reference max is raised, and O rescaled, only when the row's tile max passes it
 //      by more than 8 in log2 units);
-//   2. the union of the chunks kept by the item's 256 queries, ascending, one chunk per
+//   2. the union of the chunks kept by the item's queries, ascending, one chunk per
 //      tile; a row that kept chunk c weights that chunk's own softmax by exp(s^_c), a
 //      row that did not contributes zero.
 // Warp roles (384 threads), all hand-offs through mbarriers:
@@ -82,8 +86,8 @@ constexpr uint32_t kMapFreeCount = kSoftmaxWarps * 32 + 3;  // softmax rows + lo
 struct TcArgs {
     AttendArgs a;
     int N, C;
-    int nqb;        // query items per (b, h)
-    int items;      // B * H * nqb
+    int nqb;        // query items per (b, packed heads)
+    int items;      // B * (H / P) * nqb
     uint32_t *status;  // nonzero after a wait expired
 };
 
@@ -151,31 +155,35 @@ __device__ __forceinline__ float ldg_early(const float *p) {
 __device__ __forceinline__ int item_of(int r, int c, int G) { return r * G + ((r & 1) ? (G - 1 - c) : c); }
 
 struct Item {
-    int b, h, hk, t0;  // batch, query head, its key-value head, first query
+    int b, h, hk, t0;  // batch, first packed query head, their key-value head, first query
     int ws0, nw;  // window: first key, tiles
 };
 
+template <int P>
 __device__ __forceinline__ Item decode_item(const TcArgs &args, int j) {
+    constexpr int kQt = kM / P;
     const AttendArgs &a = args.a;
-    const int BH = a.B * a.H;
+    const int hp = a.H / P;
+    const int units = a.B * hp;
     Item it;
-    const int qb = args.nqb - 1 - j / BH;  // latest query blocks first
-    const int bh = j % BH;
-    it.b = bh / a.H;
-    it.h = bh % a.H;
+    const int qb = args.nqb - 1 - j / units;  // latest query blocks first
+    const int u = j % units;
+    it.b = u / hp;
+    it.h = (u % hp) * P;
     it.hk = it.h / a.G;
-    it.t0 = qb * kRows;
+    it.t0 = qb * 2 * kQt;
     it.ws0 = 0;
     it.nw = 0;
     if (a.W > 0) {
         const int lo = max(0, it.t0 - a.W + 1);
-        const int hi = min(args.N - 1, it.t0 + kRows - 1);
+        const int hi = min(args.N - 1, it.t0 + 2 * kQt - 1);
         it.ws0 = (lo / kTile) * kTile;
         it.nw = (hi - it.ws0) / kTile + 1;
     }
     return it;
 }
 
+template <int P>
 __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                          const __grid_constant__ CUtensorMap tmK,
                                                                          const __grid_constant__ CUtensorMap tmV,
@@ -192,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     const int nwords = (args.C + 31) >> 5;
     auto bar = [&](int i) { return sbase + kBarOff + 8u * i; };
     const int G = gridDim.x, cta = blockIdx.x;
+    constexpr int kQt = kM / P;  // queries per packed head and tile
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) {
@@ -245,15 +254,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         for (int r = 0, n = 0;; ++r, ++n) {
             const int j = item_of(r, cta, G);
             if (j >= args.items) break;
-            const Item it = decode_item(args, j);
+            const Item it = decode_item<P>(args, j);
             const int par = n & 1;
             if (n >= 2 && !wait_warp(bar(kBarMapFree + par), ((n - 2) >> 1) & 1)) break;
             uint32_t *bm = bitmaps + par * kMaxBitmapWords;
             int *nsm = reinterpret_cast<int *>(smem + kNselOff) + par * kRows;
             for (int i = lane; i < nwords; i += 32) bm[i] = 0u;
-            // the item's rows are consecutive: their kept lists form one contiguous block,
+            // the item's queries are consecutive: their kept lists form one contiguous block,
             // read with many loads in flight
-            const int nrows = min(kRows, args.N - it.t0);
+            const int nrows = min(2 * kQt, args.N - it.t0);
             const int64_t q0 = ((int64_t)it.b * (a.H / a.G) + it.hk) * a.Lq + it.t0;  // the group's kept lists
 #pragma unroll
             for (int rr = lane; rr < kRows; rr += 32)
@@ -293,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         for (int r = 0, n = 0;; ++r, ++n) {
             const int j = item_of(r, cta, G);
             if (j >= args.items) break;
-            const Item it = decode_item(args, j);
+            const Item it = decode_item<P>(args, j);
             const int par = n & 1;
             if (!wait_warp(bar(kBarMapReady + par), (n >> 1) & 1)) break;
             const int nt = it.nw + (int)union_count[par];
@@ -305,12 +314,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
                 if (lane == 0) {
                     ++issuedQ;
                     mbar_expect_tx(bar(kBarQfull), 4 * kM * 128);
+                    // rows [hh * qt, (hh + 1) * qt) of tile x: head h + hh, queries t0 + x * qt ..
 #pragma unroll
                     for (int x = 0; x < 2; ++x)
 #pragma unroll
-                        for (int kb = 0; kb < 2; ++kb)
-                            tma_load_4d(sbase + kQOff + x * 32768 + kb * 16384, &tmQ, bar(kBarQfull), kb * 64,
-                                        it.t0 + x * kM, it.h, it.b);
+                        for (int hh = 0; hh < P; ++hh)
+#pragma unroll
+                            for (int kb = 0; kb < 2; ++kb)
+                                tma_load_4d(sbase + kQOff + x * 32768 + kb * 16384 + hh * kQt * 128, &tmQ,
+                                            bar(kBarQfull), kb * 64, it.t0 + x * kQt, it.h + hh, it.b);
                 }
                 ++qn;
                 int cur = -1;  // union walk
@@ -393,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         for (int r = 0, n = 0; ok; ++r, ++n) {
             const int j = item_of(r, cta, G);
             if (j >= args.items) break;
-            const Item it = decode_item(args, j);
+            const Item it = decode_item<P>(args, j);
             const int par = n & 1;
             if (!(ok = wait_warp(bar(kBarMapReady + par), (n >> 1) & 1))) break;
             const int nt = it.nw + (int)union_count[par];
@@ -442,17 +454,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         const int x = warp >> 2;            // query tile A (0) or B (1)
         const int quad = warp & 3;          // TMEM lane quadrant
         const int rloc = quad * 32 + lane;  // row within the tile = TMEM lane
+        const int hrow = rloc / kQt;        // its packed head
+        const int trow = rloc % kQt;        // and query within the tile
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const uint32_t o_col = tmem + lane_base + 256 + x * 128;
         int g = 0;  // key tiles processed, over all items
         for (int r = 0, n = 0;; ++r, ++n) {
             const int j = item_of(r, cta, G);
             if (j >= args.items) break;
-            const Item it = decode_item(args, j);
+            const Item it = decode_item<P>(args, j);
             const int par = n & 1;
-            const int t = it.t0 + x * kM + rloc;
+            const int t = it.t0 + x * kQt + trow;
             const bool row_ok = t < args.N;
-            const int64_t qrow = ((int64_t)it.b * a.H + it.h) * a.Lq + t;
+            const int64_t qrow = ((int64_t)it.b * a.H + it.h + hrow) * a.Lq + t;
             const int64_t qgrp = ((int64_t)it.b * (a.H / a.G) + it.hk) * a.Lq + t;  // the group's kept list
             const int nsel = (row_ok && a.topk > 0) ? min(max(__ldg(&a.nsel[qgrp]), 0), a.topk) : 0;
             const int32_t *ip = a.idx + qgrp * a.topk;
@@ -637,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             if (ok && nt > 0) ok = wait_warp(bar(kBarPVdone + 2 * x + ((g - 1) & 1)), ((g - 1) >> 1) & 1);
             if (!ok) break;
             tc_fence_after();
-            bf16 *orow = static_cast<bf16 *>(a.O.ptr) + it.b * a.O.sb + it.h * a.O.sh + (int64_t)t * a.O.st;
+            bf16 *orow = static_cast<bf16 *>(a.O.ptr) + it.b * a.O.sb + (it.h + hrow) * a.O.sh + (int64_t)t * a.O.st;
             const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
             for (int part = 0; part < 4; ++part) {
@@ -686,23 +700,34 @@ bool attend_prefill_tc_supported(hils_dtype dt, int d, int N) {
 hils_status launch_attend_prefill_tc(const AttendArgs &a, int N, uint32_t *status, cudaStream_t s) {
     CUtensorMap mq, mk, mv;
     const int Hk = a.H / a.G;
-    if (!make_map(&mq, a.Q, a.B, a.H, N, kM) || !make_map(&mk, a.K, a.B, Hk, N, kTile) ||
+    int P = 1;  // heads packed per tile: the largest power of two <= 8 dividing G
+    while (P < 8 && a.G % (2 * P) == 0) P *= 2;
+    const int qt = kM / P;
+    if (!make_map(&mq, a.Q, a.B, a.H, N, qt) || !make_map(&mk, a.K, a.B, Hk, N, kTile) ||
         !make_map(&mv, a.V, a.B, Hk, N, kTile))
         return HILS_ERR_CUDA;
-    static KernelSetup setup;
+    static KernelSetup setups[4];
+    const void *fns[4] = {(const void *)attend_prefill_tc_kernel<1>, (const void *)attend_prefill_tc_kernel<2>,
+                          (const void *)attend_prefill_tc_kernel<4>, (const void *)attend_prefill_tc_kernel<8>};
+    const int pi = P == 1 ? 0 : P == 2 ? 1 : P == 4 ? 2 : 3;
     int per_sm = 0;
-    const hils_status st = kernel_setup(setup, (const void *)attend_prefill_tc_kernel, kThreads, kSmemBytes, &per_sm);
+    const hils_status st = kernel_setup(setups[pi], fns[pi], kThreads, kSmemBytes, &per_sm);
     if (st != HILS_OK) return st;
     if (per_sm < 1) return HILS_ERR_CUDA;
     TcArgs ta;
     ta.a = a;
     ta.N = N;
     ta.C = N / kChunk;
-    ta.nqb = (N + kRows - 1) / kRows;
-    ta.items = a.B * a.H * ta.nqb;
+    ta.nqb = (N + 2 * qt - 1) / (2 * qt);
+    ta.items = a.B * (a.H / P) * ta.nqb;
     ta.status = status;
     const int grid = min(ta.items, per_sm * device_sm_count());
-    attend_prefill_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, ta);
+    switch (P) {
+    case 1: attend_prefill_tc_kernel<1><<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, ta); break;
+    case 2: attend_prefill_tc_kernel<2><<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, ta); break;
+    case 4: attend_prefill_tc_kernel<4><<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, ta); break;
+    default: attend_prefill_tc_kernel<8><<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, ta); break;
+    }
     return record_cuda_error(cudaGetLastError());
 }
 
