@@ -435,6 +435,7 @@ def run_profile_case(args):
 
     decode-select: the 512K decode geometry (H=32, 8191 eligible chunks, K=16) on a
                    random summary table (68 MB) without a KV cache;
+    decode-select-gqa: the same with 8 key-value heads (groups of 4 query heads);
     decode-attend: the decode attend with H=32, K=16, W=512 on a 128K-token cache (2.1 GB);
     prefill:       the full 8K prefill workload (summarise, select, attend);
     prefill-select: the select of the 8K prefill, multi-head then grouped-query (32 query
@@ -446,17 +447,17 @@ def run_profile_case(args):
     torch.cuda.set_device(dev)
     hils.load_library()
     case = args.profile
-    if case == "decode-select":
-        w = WORKLOADS[4]
+    if case in ("decode-select", "decode-select-gqa"):
+        w = WORKLOADS[4] if case == "decode-select" else WORKLOADS[8]
         g = torch.Generator(device=dev).manual_seed(1)
         Q = torch.randn(w.B, w.H, 1, w.d, generator=g, device=dev).to(w.dtype)
         Ksum = (torch.randn(w.B, w.H, w.C, w.d, generator=g, device=dev) * 0.3).to(w.dtype)
         Bsum = torch.rand(w.B, w.H, w.C, generator=g, device=dev) * 0.5 + 3.7
-        p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype)
+        p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype, H_kv=w.Hk)
         qpos = torch.full((w.B, 1), w.N - 1, dtype=torch.int32, device=dev)
-        idx = torch.empty(w.B, w.H, 1, w.K, dtype=torch.int32, device=dev)
+        idx = torch.empty(w.B, w.Hkv, 1, w.K, dtype=torch.int32, device=dev)
         score = torch.empty(w.B, w.H, 1, w.K, device=dev)
-        nsel = torch.empty(w.B, w.H, 1, dtype=torch.int32, device=dev)
+        nsel = torch.empty(w.B, w.Hkv, 1, dtype=torch.int32, device=dev)
         ws = hils.alloc_workspace(p, hils.HILS_CALL_SELECT, 1, w.C, device=dev)
         fn = lambda: hils.hils_select(p, Q, Ksum, Bsum, idx, score, nsel, qpos=qpos, workspace=ws)  # noqa
     elif case == "decode-attend":
@@ -565,7 +566,7 @@ def measure_decode(w, dev, stream, flush, args, world, peaks):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None,
-                    choices=["decode-select", "decode-attend", "prefill", "prefill-select"],
+                    choices=["decode-select", "decode-select-gqa", "decode-attend", "prefill", "prefill-select"],
                     help="run a small case for an ncu capture and exit")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)

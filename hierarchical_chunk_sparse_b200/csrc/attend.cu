@@ -326,6 +326,199 @@ __global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
     if (threadIdx.x == 0) ws.counters[qi] = 0;
 }
 
+// ---- grouped-query decode (summary page, Methodology 3, GQA adaptation): the GG query
+// heads of a group read the same key-value head and keep the same chunks, so one CTA per
+// (unit, b, group) copies the unit's K and V rows once and computes the unit for every
+// head of the group (each head with its own query, softmax and chunk score); the
+// group's last CTA combines every head's units.
+
+template <typename T, int D, int GG>
+struct GroupUnitCfg {
+    using U = UnitCfg<T, D>;
+    // K tile, V tile, the heads' query rows, logits and probabilities per head, column
+    // partial sums per head
+    static constexpr int kSmemBytes = 2 * U::kTileBytes + GG * U::kRowBytes +
+                                      (2 * GG * kChunk + GG * U::kRowGroups * D) * 4;
+};
+
+// Eq. 10's combination for the GG heads of a group at once: kThreads / GG threads per
+// head, D / (kThreads / GG) consecutive columns per thread, every load of a batch of
+// units in flight together. mass and vec hold the heads' partials one after another
+// (units per head). Writes head hh's o to out[hh * (D + 1) ..] and its lse after it.
+template <int D, int GG>
+__device__ void combine_group(const float *mass, const float *vec, int units, float *out) {
+    constexpr int kTph = kThreads / GG, kCpt = D / kTph;
+    constexpr int kB = kCpt >= 8 ? 8 : kCpt == 4 ? 16 : 32;
+    static_assert(kCpt >= 1 && kTph * kCpt == D, "columns per thread");
+    const int hh = threadIdx.x / kTph, x0 = (threadIdx.x % kTph) * kCpt;
+    const float *mh = mass + (size_t)hh * units;
+    const float *vh = vec + (size_t)hh * units * D + x0;
+    float M = -INFINITY, z = 0.f, acc[kCpt];
+#pragma unroll
+    for (int q = 0; q < kCpt; ++q) acc[q] = 0.f;
+    for (int v0 = 0; v0 < units; v0 += kB) {
+        float m[kB], c[kB][kCpt];
+#pragma unroll
+        for (int k = 0; k < kB; ++k) {
+            const bool ok = v0 + k < units;
+            m[k] = ok ? __ldcg(mh + v0 + k) : -INFINITY;
+#pragma unroll
+            for (int q = 0; q < kCpt; ++q) c[k][q] = ok ? __ldcg(vh + (size_t)(v0 + k) * D + q) : 0.f;
+        }
+        float mb = M;
+#pragma unroll
+        for (int k = 0; k < kB; ++k) mb = fmaxf(mb, m[k]);
+        if (mb == -INFINITY) continue;
+        const float f = expf(M - mb);  // 0 when M is -inf
+        z *= f;
+#pragma unroll
+        for (int q = 0; q < kCpt; ++q) acc[q] *= f;
+#pragma unroll
+        for (int k = 0; k < kB; ++k) {
+            const float wv = expf(m[k] - mb);
+            z += wv;
+#pragma unroll
+            for (int q = 0; q < kCpt; ++q) acc[q] = fmaf(wv, c[k][q], acc[q]);
+        }
+        M = mb;
+    }
+    float *oh = out + hh * (D + 1);
+#pragma unroll
+    for (int q = 0; q < kCpt; ++q) oh[x0 + q] = M == -INFINITY ? 0.f : acc[q] / z;
+    if (x0 == 0) oh[D] = M == -INFINITY ? -INFINITY : M + logf(z);
+    __syncthreads();
+}
+
+// grid (units, B * H / GG): one unit of one (b, group) per CTA.
+template <typename T, int D, int GG>
+__global__ void __launch_bounds__(kThreads) attend_decode_group_kernel(AttendArgs a) {
+    using Cfg = UnitCfg<T, D>;
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ int is_last;
+    __shared__ float lse_h[GG];
+    uint8_t *kt = smem, *vt = smem + Cfg::kTileBytes, *qsm = smem + 2 * Cfg::kTileBytes;
+    float *logit = reinterpret_cast<float *>(qsm + GG * Cfg::kRowBytes);  // [GG][64]
+    float *prob = logit + GG * kChunk;                                   // [GG][64]
+    float *red = prob + GG * kChunk;                                     // [GG][kRowGroups][D]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int u = blockIdx.x;
+    const int Hk = a.H / GG;
+    const int64_t qg = blockIdx.y;  // (b, group): the group's kept list
+    const int b = (int)(qg / Hk), hk = (int)(qg % Hk), h0 = hk * GG;
+    const int64_t qi0 = (int64_t)b * a.H + h0;  // the group's first query head
+    const bool chunk_unit = u < a.topk;
+    if (chunk_unit || !a.window_early) pdl_wait();  // as in the per-head kernel
+    const int clen = a.cache_len[b];
+    const int ns = chunk_unit ? a.nsel[qg] : 0;
+    const int cidx = chunk_unit ? a.idx[qg * a.topk + u] : -1;
+    const UnitPlan p = plan_unit_loaded(u, clen - 1, a.topk, a.W, cidx, 0.f, ns);
+    const DecodeWs ws = decode_ws(a.ws, a.B * a.H, a.units, D);
+    if (p.rows > 0) {
+        const int rows = p.rows;
+        const T *k0 = static_cast<const T *>(a.K.ptr) + b * a.K.sb + hk * a.K.sh + (int64_t)p.start * a.K.st;
+        const T *v0 = static_cast<const T *>(a.V.ptr) + b * a.V.sb + hk * a.V.sh + (int64_t)p.start * a.V.st;
+        const T *q0 = static_cast<const T *>(a.Q.ptr) + b * a.Q.sb + h0 * a.Q.sh;
+        for (int i = tid; i < rows * Cfg::kRowUnits; i += kThreads) {
+            const int r = i / Cfg::kRowUnits, un = i % Cfg::kRowUnits;
+            cp_async16(kt + i * 16, reinterpret_cast<const uint8_t *>(k0 + r * a.K.st) + un * 16);
+        }
+        for (int i = tid; i < GG * Cfg::kRowUnits; i += kThreads) {
+            const int hh = i / Cfg::kRowUnits, un = i % Cfg::kRowUnits;
+            cp_async16(qsm + i * 16, reinterpret_cast<const uint8_t *>(q0 + hh * a.Q.sh) + un * 16);
+        }
+        cp_async_commit();
+        for (int i = tid; i < rows * Cfg::kRowUnits; i += kThreads) {
+            const int r = i / Cfg::kRowUnits, un = i % Cfg::kRowUnits;
+            cp_async16(vt + i * 16, reinterpret_cast<const uint8_t *>(v0 + r * a.V.st) + un * 16);
+        }
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        {  // logits: a thread pair per key row, every head's dot product from one read of the row
+            const int row = tid >> 1, half = tid & 1;
+            const uint4 *krow = reinterpret_cast<const uint4 *>(kt + row * Cfg::kRowBytes);
+            const uint4 *qv = reinterpret_cast<const uint4 *>(qsm);
+            float acc[GG];
+#pragma unroll
+            for (int hh = 0; hh < GG; ++hh) acc[hh] = 0.f;
+            if (row < rows) {
+#pragma unroll
+                for (int k = 0; k < Cfg::kHalfUnits; ++k) {
+                    const int un = half * Cfg::kHalfUnits + rotated_unit<Cfg::kHalfUnits>(k, row, half);
+                    const uint4 kv = krow[un];
+#pragma unroll
+                    for (int hh = 0; hh < GG; ++hh) acc[hh] = dot16<T>(kv, qv[hh * Cfg::kRowUnits + un], acc[hh]);
+                }
+            }
+#pragma unroll
+            for (int hh = 0; hh < GG; ++hh) {
+                const float v = acc[hh] + __shfl_xor_sync(kFull, acc[hh], 1);
+                if (half == 0) logit[hh * kChunk + row] = row < rows ? v * a.scale : -INFINITY;
+            }
+        }
+        __syncthreads();
+        for (int hh = warp; hh < GG; hh += kThreads / 32) {  // softmax: a warp per head
+            const float l0 = logit[hh * kChunk + lane], l1 = logit[hh * kChunk + lane + 32];
+            const float m = warp_max(fmaxf(l0, l1));
+            const float e0 = expf(l0 - m), e1 = expf(l1 - m);
+            const float z = warp_sum(e0 + e1);
+            const float inv = 1.f / z;
+            prob[hh * kChunk + lane] = e0 * inv;
+            prob[hh * kChunk + lane + 32] = e1 * inv;
+            if (lane == 0) lse_h[hh] = m + logf(z);
+        }
+        cp_async_wait<0>();
+        __syncthreads();
+        {  // o_u = P V for every head from one read of each V element
+            const int cu = tid % Cfg::kColUnits, rg = tid / Cfg::kColUnits;
+            float a0[GG], a1[GG];
+#pragma unroll
+            for (int hh = 0; hh < GG; ++hh) a0[hh] = a1[hh] = 0.f;
+            for (int j = rg; j < rows; j += Cfg::kRowGroups) {
+                const float2 vv = load2(reinterpret_cast<const T *>(vt + j * Cfg::kRowBytes) + 2 * cu);
+#pragma unroll
+                for (int hh = 0; hh < GG; ++hh) {
+                    const float pj = prob[hh * kChunk + j];
+                    a0[hh] = fmaf(pj, vv.x, a0[hh]);
+                    a1[hh] = fmaf(pj, vv.y, a1[hh]);
+                }
+            }
+#pragma unroll
+            for (int hh = 0; hh < GG; ++hh) {
+                red[(hh * Cfg::kRowGroups + rg) * D + 2 * cu] = a0[hh];
+                red[(hh * Cfg::kRowGroups + rg) * D + 2 * cu + 1] = a1[hh];
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < GG * D; e += kThreads) {
+            const int hh = e / D, x = e - hh * D;
+            float v = red[hh * Cfg::kRowGroups * D + x];
+#pragma unroll
+            for (int g = 1; g < Cfg::kRowGroups; ++g) v += red[(hh * Cfg::kRowGroups + g) * D + x];
+            ws.vec[((size_t)(qi0 + hh) * a.units + u) * D + x] = v;
+        }
+        if (tid < GG)
+            ws.mass[(qi0 + tid) * a.units + u] = p.is_chunk ? a.score[(qi0 + tid) * a.topk + u] : lse_h[tid];
+    } else {
+        // an empty unit contributes weight 0 to every head
+        for (int e = tid; e < GG * D; e += kThreads) {
+            const int hh = e / D, x = e - hh * D;
+            ws.vec[((size_t)(qi0 + hh) * a.units + u) * D + x] = 0.f;
+        }
+        if (tid < GG) ws.mass[(qi0 + tid) * a.units + u] = -INFINITY;
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = atomicAdd(&ws.counters[qg], 1) == a.units - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    combine_group<D, GG>(ws.mass + (size_t)qi0 * a.units, ws.vec + (size_t)qi0 * a.units * D, a.units, red);
+    for (int hh = 0; hh < GG; ++hh)
+        store_output<T, D>(a, b, h0 + hh, 0, qi0 + hh, red + hh * (D + 1), red[hh * (D + 1) + D]);
+    if (tid == 0) ws.counters[qg] = 0;
+}
+
 // General prefill path: one CTA per query, units in turn, running combination.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) attend_prefill_general_kernel(AttendArgs a) {
@@ -366,11 +559,27 @@ __global__ void __launch_bounds__(kThreads) attend_prefill_general_kernel(Attend
     store_output<T, D>(a, b, h, i, qi, o, M == -INFINITY ? -INFINITY : M + logf(zsum));
 }
 
+template <typename T, int D, int GG>
+hils_status launch_decode_group(const AttendArgs &a, cudaStream_t st) {
+    using Cfg = GroupUnitCfg<T, D, GG>;
+    static KernelSetup setup;
+    const hils_status stt = kernel_setup(setup, (const void *)attend_decode_group_kernel<T, D, GG>, kThreads,
+                                         Cfg::kSmemBytes, nullptr);
+    if (stt != HILS_OK) return stt;
+    return launch_dependent((const void *)attend_decode_group_kernel<T, D, GG>, dim3(a.units, a.B * (a.H / GG)),
+                            dim3(kThreads), Cfg::kSmemBytes, st, a);
+}
+
 template <typename T, int D>
 hils_status launch_decode(const AttendArgs &a, cudaStream_t st) {
     using Cfg = UnitCfg<T, D>;
     const int nq = a.B * a.H;
     if (nq == 0) return HILS_OK;
+    // groups of 2, 4 or 8 heads share each unit's copies; other group sizes take a CTA
+    // per head
+    if (a.G == 2) return launch_decode_group<T, D, 2>(a, st);
+    if (a.G == 4) return launch_decode_group<T, D, 4>(a, st);
+    if (a.G == 8) return launch_decode_group<T, D, 8>(a, st);
     static KernelSetup setup;
     const hils_status stt = kernel_setup(setup, (const void *)attend_decode_kernel<T, D>, kThreads,
                                          Cfg::kSmemBytes, nullptr);

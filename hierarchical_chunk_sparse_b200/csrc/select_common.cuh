@@ -294,7 +294,8 @@ __device__ void warp_write(const EntryList &list, int K, int64_t qi, int32_t *id
     if (lane < n) {
         const int me = list.idx[lane];
         int rank = 0;
-        for (int j = 0; j < n; ++j) rank += list.idx[j] < me;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) rank += (j < n && list.idx[j] < me) ? 1 : 0;
         idx[qi * K + rank] = me;
         score[qi * K + rank] = list.s[lane];
     } else if (lane < K) {
@@ -377,10 +378,47 @@ __device__ __forceinline__ void screen(const GroupCtx &g, const float *qs, int c
     interval_mid(lo, hi, s, e);
 }
 
+// The largest of the heads' float64 scores; two heads' fixed-order chains run side by
+// side (each in its own x order, as for one head), rows read a quarter at a time.
 template <typename T, int D>
 __device__ double exact_score(const GroupCtx &g, int c) {
+    constexpr int kN = Vec<T>::kN, kQ = D / kN / 4;
     double m = -INFINITY;
-    for (int hh = 0; hh < g.G; ++hh) m = fmax(m, exact_score<T, D>(head_ctx(g, hh, (int)sizeof(T)), c));
+    for (int h0 = 0; h0 < g.G; h0 += 2) {
+        const bool two = h0 + 1 < g.G;
+        const QueryCtx q0 = head_ctx(g, h0, (int)sizeof(T));
+        const QueryCtx q1 = head_ctx(g, two ? h0 + 1 : h0, (int)sizeof(T));
+        const uint4 *qr[2] = {static_cast<const uint4 *>(q0.qrow), static_cast<const uint4 *>(q1.qrow)};
+        const uint4 *kr[2] = {reinterpret_cast<const uint4 *>(static_cast<const T *>(q0.khead) + (int64_t)c * q0.kst),
+                              reinterpret_cast<const uint4 *>(static_cast<const T *>(q1.khead) + (int64_t)c * q1.kst)};
+        double acc[2] = {0.0, 0.0};
+#pragma unroll
+        for (int part = 0; part < 4; ++part) {
+            uint4 qv[2][kQ], kv[2][kQ];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int u = 0; u < kQ; ++u) {
+                    qv[j][u] = __ldg(qr[j] + part * kQ + u);
+                    kv[j][u] = __ldg(kr[j] + part * kQ + u);
+                }
+#pragma unroll
+            for (int u = 0; u < kQ; ++u) {
+                float qf[2][kN], kf[2][kN];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    widen(qv[j][u], qf[j], T());
+                    widen(kv[j][u], kf[j], T());
+                }
+#pragma unroll
+                for (int i = 0; i < kN; ++i)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) acc[j] = __dadd_rn(acc[j], __dmul_rn((double)qf[j][i], (double)kf[j][i]));
+            }
+        }
+        m = fmax(m, __dadd_rn(__dmul_rn(acc[0], (double)q0.scale), (double)q0.bhead[c]));
+        if (two) m = fmax(m, __dadd_rn(__dmul_rn(acc[1], (double)q1.scale), (double)q1.bhead[c]));
+    }
     return m;
 }
 
@@ -419,7 +457,8 @@ __device__ void group_write(const GroupCtx &q, const float *qs, const EntryList 
     if (lane < n) {
         me = list.idx[lane];
         rank = 0;
-        for (int j = 0; j < n; ++j) rank += list.idx[j] < me;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) rank += (j < n && list.idx[j] < me) ? 1 : 0;
     }
     if (lane < K) a.idx[qg * K + rank] = lane < n ? me : -1;
     for (int hh = 0; hh < q.G; ++hh) {

@@ -26,19 +26,26 @@ struct Pool64 {
 
 
 
-// (K+1)-th largest of the first values of v[0..n) (duplicates counted) by parallel
-// ranks: value i has rank #{j: v_j > v_i} + #{j < i: v_j = v_i}, unique, and the one
-// with rank K is the answer (n > K; all NT threads call; the result in *out).
+// (K+1)-th largest of n <= kMaxGroups values (duplicates counted) from their
+// order-preserving integer keys key[0..n), padded with zeros to a multiple of 4: value i
+// has the unique rank #{j: k_j > k_i} + #{j < i: k_j = k_i}, and the one of rank K is
+// the answer (n > K; all NT threads call; the result in *out). The keys are read four
+// at a time by every thread at once (a broadcast), with no dependence between steps.
 template <int NT>
-__device__ void block_kth_plus_one(const float2 *v, int n, int K, float *out) {
+__device__ void block_kth_plus_one(const unsigned *key, int n, int K, float *out) {
+    const uint4 *k4 = reinterpret_cast<const uint4 *>(key);
+    const int n4 = (n + 3) >> 2;
     for (int i = threadIdx.x; i < n; i += NT) {
-        const unsigned ki = ordered_key(v[i].x);
-        int rank = 0;
-        for (int j = 0; j < n; ++j) {
-            const unsigned kj = ordered_key(v[j].x);
-            rank += (kj > ki || (kj == ki && j < i)) ? 1 : 0;
+        const unsigned ki = key[i];
+        int gt = 0, eq = 0;
+#pragma unroll 8
+        for (int j4 = 0; j4 < n4; ++j4) {
+            const uint4 k = k4[j4];
+            const int j = 4 * j4;
+            gt += (k.x > ki) + (k.y > ki) + (k.z > ki) + (k.w > ki);
+            eq += (k.x == ki && j < i) + (k.y == ki && j + 1 < i) + (k.z == ki && j + 2 < i) + (k.w == ki && j + 3 < i);
         }
-        if (rank == K) *out = v[i].x;
+        if (gt + eq == K) *out = key_to_float(ki);
     }
 }
 
@@ -51,6 +58,7 @@ __device__ __forceinline__ void rescreen_one(const QueryCtx &q, const float *qs,
                                              float &e) {
     constexpr int kN = Vec<T>::kN, kQuarter = D / 4;
     const int sub = threadIdx.x & 3;
+    const float bias = ok ? __ldg(q.bhead + c) : 0.f;
     float dot = 0.f, ad = 0.f;
     if (ok) {
         const uint4 *kr = reinterpret_cast<const uint4 *>(static_cast<const T *>(q.khead) + (int64_t)c * q.kst +
@@ -71,7 +79,7 @@ __device__ __forceinline__ void rescreen_one(const QueryCtx &q, const float *qs,
     ad += __shfl_xor_sync(kFull, ad, 1);
     dot += __shfl_xor_sync(kFull, dot, 2);
     ad += __shfl_xor_sync(kFull, ad, 2);
-    s = ok ? fmaf(dot, q.scale, q.bhead[c]) : 0.f;
+    s = ok ? fmaf(dot, q.scale, bias) : 0.f;
     e = fmaf(q.scale * ad, (float)(D + 2) * 0x1p-23f, fabsf(s) * 0x1p-22f);
 }
 
@@ -91,27 +99,91 @@ __device__ void rescreen_pool(const QueryCtx &q, const float *qs, Pool64 &pool, 
     }
 }
 
-// Grouped heads: each head's tight interval, folded into the group maximum's interval.
+// Grouped heads: each head's tight interval, folded into the group maximum's interval;
+// each head's own value is kept in sh[head][entry] for the output. The rows of up to
+// kHB heads are loaded together before their sums run.
 template <typename T, int D, int NT>
-__device__ void rescreen_pool(const GroupCtx &g, const float *qs, Pool64 &pool, int total) {
-    const int tid = threadIdx.x;
+__device__ void rescreen_pool(const GroupCtx &g, const float *qs, Pool64 &pool, int total, float *sh) {
+    constexpr int kN = Vec<T>::kN, kQuarter = D / 4, kU = kQuarter / kN;
+    constexpr int kHB = sizeof(T) == 2 ? 4 : 2;
+    const int tid = threadIdx.x, sub = tid & 3;
     for (int base = 0; base < total; base += NT / 4) {
         const int j = base + (tid >> 2);
         const bool ok = j < total;
         const int c = ok ? pool.idx[j] : 0;
         float lo = -INFINITY, hi = -INFINITY;
-        for (int hh = 0; hh < g.G; ++hh) {
-            float s, e;
-            rescreen_one<T, D>(head_ctx(g, hh, (int)sizeof(T)), qs + hh * D, c, ok, s, e);
-            fold_interval(s, e, lo, hi);
+        for (int h0 = 0; h0 < g.G; h0 += kHB) {
+            uint4 kv[kHB][kU];
+            float bias[kHB];
+#pragma unroll
+            for (int hb = 0; hb < kHB; ++hb) {
+                const bool live = ok && h0 + hb < g.G;
+                const QueryCtx q = head_ctx(g, h0 + hb < g.G ? h0 + hb : h0, (int)sizeof(T));
+                const uint4 *kr = reinterpret_cast<const uint4 *>(static_cast<const T *>(q.khead) +
+                                                                  (int64_t)c * q.kst + sub * kQuarter);
+#pragma unroll
+                for (int u = 0; u < kU; ++u) kv[hb][u] = live ? __ldg(kr + u) : make_uint4(0, 0, 0, 0);
+                bias[hb] = live ? __ldg(q.bhead + c) : 0.f;
+            }
+#pragma unroll
+            for (int hb = 0; hb < kHB; ++hb) {
+                if (h0 + hb >= g.G) break;  // uniform
+                const QueryCtx q = head_ctx(g, h0 + hb, (int)sizeof(T));
+                const float *qh = qs + (h0 + hb) * D + sub * kQuarter;
+                float dot = 0.f, ad = 0.f;
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    float kf[kN];
+                    widen(kv[hb][u], kf, T());
+#pragma unroll
+                    for (int i = 0; i < kN; ++i) {
+                        dot = fmaf(qh[u * kN + i], kf[i], dot);
+                        ad = fmaf(fabsf(qh[u * kN + i]), fabsf(kf[i]), ad);
+                    }
+                }
+                dot += __shfl_xor_sync(kFull, dot, 1);
+                ad += __shfl_xor_sync(kFull, ad, 1);
+                dot += __shfl_xor_sync(kFull, dot, 2);
+                ad += __shfl_xor_sync(kFull, ad, 2);
+                const float s = ok ? fmaf(dot, q.scale, bias[hb]) : 0.f;
+                const float e = fmaf(q.scale * ad, (float)(D + 2) * 0x1p-23f, fabsf(s) * 0x1p-22f);
+                fold_interval(s, e, lo, hi);
+                if (ok && sub == 0) sh[(h0 + hb) * kPoolCap + j] = s;
+            }
         }
-        if (ok && (tid & 3) == 0) interval_mid(lo, hi, pool.s[j], pool.e[j]);
+        if (ok && sub == 0) interval_mid(lo, hi, pool.s[j], pool.e[j]);
     }
+}
+
+// A group's kept list from the pool: chunk indices ascending for the group, and each
+// head's own tight screen value (sh, from rescreen_pool) of the kept chunks.
+template <typename T, int D>
+__device__ void group_write_pool(const GroupCtx &q, const EntryList &list, const Pool64 &pool, const float *sh,
+                                 int total, const SelectArgs &a, int64_t qg, int b, int g, int i) {
+    const int lane = threadIdx.x & 31;
+    const int K = a.topk, n = list.n;
+    int rank = lane, me = -1, slot = 0;
+    if (lane < n) {
+        me = list.idx[lane];
+        rank = 0;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) rank += (j < n && list.idx[j] < me) ? 1 : 0;
+#pragma unroll
+        for (int j = 0; j < kPoolCap; ++j) slot = (j < total && pool.idx[j] == me) ? j : slot;
+    }
+    if (lane < K) a.idx[qg * K + rank] = lane < n ? me : -1;
+    for (int hh = 0; hh < q.G; ++hh) {
+        const int64_t qh = ((int64_t)b * a.H + g * a.G + hh) * a.Lq + i;
+        if (lane < K) a.score[qh * K + rank] = lane < n ? sh[hh * kPoolCap + slot] : -INFINITY;
+    }
+    if (lane == 0) a.nsel[qg] = n;
 }
 
 struct PickSmem {
     float qs[kMaxGroup * 128];  // the query rows (float32) of the unit's heads
+    float pool_sh[kMaxGroup * kPoolCap];  // grouped heads: each head's value of each pool entry
     float2 gm[kMaxGroups];
+    __align__(16) unsigned gkey[kMaxGroups];  // order-preserving keys of gm[].x
     uint16_t cand_g[kMaxGroups];
     Pool64 pool;
     EntryList out;
@@ -235,8 +307,8 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
         return;
     }
     const int G = groups_of(ne);
-    __syncthreads();  // ps.qs complete
     if (G < K + 1) {  // short table: the exact running-list scan over every chunk
+        __syncthreads();  // ps.qs complete
         if (w == 0) {
             warp_scan<T, D>(q, ps.qs, 0, ne, K, ps.out);
             write(ps.out);
@@ -246,9 +318,10 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
     // T = (K+1)-th largest maximum of the 64-chunk groups (attained by K+1 distinct
     // chunks); e_max = largest radius; every chunk with hi < T - e_max is certainly out
     float em = 0.f;
-    for (int g = tid; g < G; g += NT) {
-        const float2 v = gmax_at<kGroup>(rows, g);
+    for (int g = tid; g < ((G + 3) & ~3); g += NT) {
+        const float2 v = g < G ? gmax_at<kGroup>(rows, g) : make_float2(-INFINITY, 0.f);
         ps.gm[g] = v;
+        ps.gkey[g] = g < G ? ordered_key(v.x) : 0u;  // 0: below every value's key
         em = fmaxf(em, v.y);
     }
     em = warp_max(em);
@@ -257,8 +330,8 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
         ps.pool_n = 0;
     }
     if (lane == 0) ps.wmax[w] = em;
-    __syncthreads();
-    block_kth_plus_one<NT>(ps.gm, G, K, &ps.tk);
+    __syncthreads();  // ps.qs, ps.gm and ps.gkey complete
+    block_kth_plus_one<NT>(ps.gkey, G, K, &ps.tk);
     __syncthreads();
     if (tid == 0) {
         float e2 = 0.f;
@@ -272,22 +345,25 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
         if (__fadd_ru(ps.gm[g].x, ps.gm[g].y) >= cut) ps.cand_g[atomicAdd(&ps.ncg, 1)] = (uint16_t)g;
     __syncthreads();
     const int ncg = ps.ncg;
-    // their chunks with hi >= cut join the pool: warp w scans candidate groups w, w+8, ...
-    for (int k0 = w; k0 < ncg; k0 += 2 * (NT / 32)) {
-        float2 v[4];
+    // their chunks with hi >= cut join the pool: slot e of the candidates' chunks is
+    // chunk e % 64 of candidate group e / 64; a thread loads its (up to) eight slots at
+    // once
+    constexpr int kPer = 8;
+    for (int e0 = 0; e0 < ncg * kGroupRows; e0 += NT * kPer) {
+        float2 v[kPer];
+        int cc[kPer];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int k = k0 + (j >> 1) * (NT / 32);
-            const int c = k < ncg ? ps.cand_g[k] * kGroupRows + (j & 1) * 32 + lane : ne;
-            v[j] = c < ne ? scr_at<kGroup>(rows, c) : make_float2(-INFINITY, 0.f);
+        for (int j = 0; j < kPer; ++j) {
+            const int e = e0 + j * NT + tid;
+            cc[j] = e < ncg * kGroupRows ? ps.cand_g[e / kGroupRows] * kGroupRows + e % kGroupRows : ne;
+            v[j] = cc[j] < ne ? scr_at<kGroup>(rows, cc[j]) : make_float2(-INFINITY, 0.f);
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kPer; ++j) {
             if (v[j].x != -INFINITY && __fadd_ru(v[j].x, v[j].y) >= cut) {
-                const int k = k0 + (j >> 1) * (NT / 32);
                 const int pos = atomicAdd(&ps.pool_n, 1);
                 if (pos < kPoolCap) {
-                    ps.pool.idx[pos] = ps.cand_g[k] * kGroupRows + (j & 1) * 32 + lane;
+                    ps.pool.idx[pos] = cc[j];
                     ps.pool.s[pos] = v[j].x;
                     ps.pool.e[pos] = v[j].y;
                     ps.pool.x[pos] = __longlong_as_double(0x7ff8000000000000ll);
@@ -300,7 +376,8 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
     if (total <= kPoolCap) {
         // the candidates are screened again on CUDA cores (round-to-nearest fused
         // multiply-adds: the tight radius), so that few need the float64 score
-        rescreen_pool<T, D, NT>(q, ps.qs, ps.pool, total);
+        if constexpr (kGroup) rescreen_pool<T, D, NT>(q, ps.qs, ps.pool, total, ps.pool_sh);
+        else rescreen_pool<T, D, NT>(q, ps.qs, ps.pool, total);
         __syncthreads();
         if (w == 0) {
             Slots<2> sl;
@@ -319,7 +396,8 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
             const int n = warp_append<2>(sl, keep, ps.out, 0);
             if (lane == 0) ps.out.n = n;
             __syncwarp();
-            write(ps.out);
+            if constexpr (kGroup) group_write_pool<T, D>(q, ps.out, ps.pool, ps.pool_sh, total, a, u, b, grp, i);
+            else write(ps.out);
         }
         return;
     }

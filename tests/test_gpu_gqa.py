@@ -104,13 +104,20 @@ def test_gqa_prefill_full_size(oracle, cuda_device):
         assert_close(lse[:, sq], lse_ref, torch.float32, f"lse group {hk}")
 
 
-@pytest.mark.parametrize("lens,H,Hk,K,W", [((12001, 9000), 8, 2, 16, 512), ((1, 65, 700, 5000), 4, 1, 32, 1024),
-                                           ((3000, 2000), 6, 3, 8, 0), ((2000, 1500), 8, 4, 0, 100)])
-def test_gqa_decode(oracle, cuda_device, lens, H, Hk, K, W):
+@pytest.mark.parametrize("lens,H,Hk,K,W,d,dtype", [
+    ((12001, 9000), 8, 2, 16, 512, 128, torch.bfloat16),
+    ((1, 65, 700, 5000), 4, 1, 32, 1024, 128, torch.bfloat16),
+    ((3000, 2000), 6, 3, 8, 0, 128, torch.bfloat16),    # groups of 3: a CTA per head
+    ((2000, 1500), 8, 4, 0, 100, 128, torch.bfloat16),
+    ((3000, 7001), 8, 1, 16, 300, 64, torch.bfloat16),  # groups of 8, d = 64
+    ((4000, 2500), 4, 2, 8, 200, 128, torch.float32),
+])
+def test_gqa_decode(oracle, cuda_device, lens, H, Hk, K, W, d, dtype):
     """Decode with ragged cache lengths (first token, one chunk, fewer chunks than K),
-    no window, window only: the separate select and attend, then hils_decode as one
-    chain on the same inputs, all against the oracle."""
-    w = WORKLOADS[8].replace(B=len(lens), H=H, Hk=Hk, N=max(lens), K=K, W=W, needles=0)
+    no window, window only, groups of 2, 3, 4 and 8, d = 64 and float32: the separate
+    select and attend, then hils_decode as one chain on the same inputs, all against
+    the oracle."""
+    w = WORKLOADS[8].replace(B=len(lens), H=H, Hk=Hk, N=max(lens), K=K, W=W, d=d, dtype=dtype, needles=0)
     inp = make_decode(w)
     inp["cache_len"] = torch.tensor(lens, dtype=torch.int32)
     d = to_dev(inp, cuda_device)
