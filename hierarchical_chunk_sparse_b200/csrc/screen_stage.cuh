@@ -69,9 +69,10 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
 // accumulation order and rounding are not specified, so the bound allows d * 2^-16 of
 // scale |q| |k'| (about 2^7 times the round-to-nearest bound), plus 2^-22 |s| for the
 // final fused multiply-add; |k'|^2 itself carries a 2^-8 margin.
+// (s_c, e_c) of chunk c goes to out[c - base].
 template <int D>
 __device__ void screen_stage_mma(const uint8_t *st, int q_off, int bias_off, float scale, int c0, int ne,
-                                 float2 *scr_row, float2 *slots) {
+                                 float2 *out, int base, float2 *slots) {
     constexpr int kRowBytes = D * 2;
     constexpr int kKSteps = D / 16;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
@@ -115,7 +116,7 @@ __device__ void screen_stage_mma(const uint8_t *st, int q_off, int bias_off, flo
             const float sv = fmaf(dot, scale, bias[row]);
             const float ev = fmaf(ecoef, sqrt_approx(h ? k2 : k1), fabsf(sv) * 0x1p-22f);
             if (c < ne) {
-                scr_row[c] = make_float2(sv, ev);
+                out[c - base] = make_float2(sv, ev);
                 ms = fmaxf(ms, sv);
                 me = fmaxf(me, ev);
             }
@@ -131,7 +132,8 @@ __device__ void screen_stage_mma(const uint8_t *st, int q_off, int bias_off, flo
 // rows with packed float32 FMAs, and a transpose reduction across the kTPR lanes
 // leaves each lane the totals of one row.
 template <typename T, int D, typename Cfg>
-__device__ void screen_stage_f32(const uint8_t *st, float scale, int c0, int ne, float2 *scr_row, float2 *gscr) {
+__device__ void screen_stage_f32(const uint8_t *st, float scale, int c0, int ne, float2 *out, int base,
+                                 float2 *gscr) {
     constexpr int kN = Vec<T>::kN;
     const int tid = threadIdx.x, col = tid % Cfg::kTPR, rg = tid / Cfg::kTPR;
     // query slice of this thread's unit as float pairs, and |q|^2
@@ -167,7 +169,7 @@ __device__ void screen_stage_f32(const uint8_t *st, float scale, int c0, int ne,
     const float ecoef = scale * sqrtf(qn2) * ((float)(D + 2) * 0x1p-23f);
     const float sv = fmaf(dotv[0], scale, reinterpret_cast<const float *>(st + Cfg::kBiasOff)[row]);
     const float ev = fmaf(ecoef, sqrt_approx(ksqv[0]), fabsf(sv) * 0x1p-22f);
-    if (valid && (col & 1) == 0) scr_row[c] = make_float2(sv, ev);
+    if (valid && (col & 1) == 0) out[c - base] = make_float2(sv, ev);
     float gs = valid ? sv : -INFINITY, ge = valid ? ev : 0.f;
 #pragma unroll
     for (int o = Cfg::kTPR / 2; o > 0; o >>= 1) {

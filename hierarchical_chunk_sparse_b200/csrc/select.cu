@@ -76,7 +76,11 @@ __global__ void __launch_bounds__(kWarpKernelThreads) select_warp_kernel(SelectA
 // screened on the tensor cores (mma.sync, 16 rows per warp; |k'|^2 from the Gram
 // diagonal), float32 rows on CUDA cores (kTPR threads per row, packed FMAs, a
 // transpose reduction). Written to the workspace: the screen value s_c and radius e_c
-// of every eligible chunk and the largest s and e of every 64-chunk group.
+// of every eligible chunk and the largest s and e of every 64-chunk group. For grouped
+// heads an item is a (b, group, query) and its block of the G heads' tables, screened
+// head after head by the same CTA; each head's interval s_c +- e_c is folded into the
+// group's [max lo, max hi] in shared memory, and the group's centre and radius are
+// written once, so the pick reads one row per group as for one head.
 //   CUDA cores:    e_c = scale |q~| |k'_c| (d+2) 2^-23 + |s_c| 2^-22 (Cauchy-Schwarz form
 //                  of the fused-multiply-add bound, doubled);
 //   tensor cores:  e_c = scale |q~| |k'_c| d 2^-16 (1 + 2^-8) + |s_c| 2^-22.
@@ -99,7 +103,8 @@ struct ScrCfg : StageCfg<T, D, kScrThreads, kScrRows> {
     using Base = StageCfg<T, D, kScrThreads, kScrRows>;
     static constexpr int kStages = Base::kStageBytes > 40000 ? 2 : kDecStages;
     static constexpr int kGscrOff = kStages * Base::kStageBytes;
-    static constexpr int kSmemBytes = kGscrOff + kScrRows * 8;
+    static constexpr int kFoldOff = kGscrOff + kScrRows * 8;  // grouped heads: one head's (s, e), the group's (lo, hi)
+    static constexpr int kSmemBytes = kFoldOff + 2 * kScrRows * 8;
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 // One CTA per query (per (b, group, query) for grouped heads), dependent-launched after
@@ -112,7 +117,7 @@ __global__ void __launch_bounds__(kPickThreads) select_pick_kernel(SelectArgs a)
     pick_unit<T, D, kPickThreads, kGroup>(a, screen_ws(a), blockIdx.x, ps);
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kFold>
 __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(SelectArgs a) {
     using Cfg = ScrCfg<T, D>;
     extern __shared__ __align__(16) uint8_t smem[];
@@ -120,21 +125,26 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(SelectArgs a
     pdl_trigger();
     const int tid = threadIdx.x;
     const int nblk = (a.C + kScrRows - 1) / kScrRows;
-    const int nq = a.B * a.H * a.Lq;
-    const int total = nq * nblk;  // checked on the host to fit in int
+    const int gh = kFold ? a.G : 1;           // heads folded per item (1: one query head)
+    const int nu = a.B * (a.H / gh) * a.Lq;   // query units: queries, or (b, group, query)
+    const int total = nu * nblk;  // checked on the host to fit in int
     const ScreenWs ws = screen_ws(a);
     const int G = groups_of(a.C);
-    // items are query-major (item = query * nblk + block), walked with a stride of
-    // gridDim.x
+    float2 *tmp = reinterpret_cast<float2 *>(smem + Cfg::kFoldOff);  // one head's (s, e) per row
+    float2 *lohi = tmp + kScrRows;                                    // the group's (lo, hi) per row
+    // items are unit-major (item = unit * nblk + block), walked with a stride of
+    // gridDim.x; each item is gh stages, one per head, in turn
     const int first = blockIdx.x, stride = gridDim.x;
-    // every thread issues its share of the copies of item `item` into stage `stage`
-    auto issue = [&](int item, int stage) {
+    auto item_of_seq = [&](int sq) { return first + (sq / gh) * stride; };
+    // every thread issues its share of the copies of stage sequence number sq into stage `stage`
+    auto issue = [&](int sq, int stage) {
+        const int item = item_of_seq(sq);
         if (item < total) {
-            const int qi = item / nblk, blk = item - (item / nblk) * nblk;
-            const int i = qi % a.Lq;
-            const int bh = qi / a.Lq;
-            const int h = bh % a.H;
-            const int b = bh / a.H;
+            const int qu = item / nblk, blk = item - (item / nblk) * nblk;
+            const int i = qu % a.Lq;
+            const int bu = qu / a.Lq;
+            const int h = (bu % (a.H / gh)) * gh + sq % gh;
+            const int b = bu / (a.H / gh);
             const int c0 = blk * kScrRows;
             const T *kh = static_cast<const T *>(a.Ksum.ptr) + b * a.Ksum.sb + h * a.Ksum.sh;
             const T *qrow = static_cast<const T *>(a.Qcal.ptr) + b * a.Qcal.sb + h * a.Qcal.sh + i * a.Qcal.st;
@@ -145,22 +155,58 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(SelectArgs a
         cp_async_commit();
     };
 
-    for (int k = 0; k < Cfg::kStages - 1; ++k) issue(first + k * stride, k);
+    for (int k = 0; k < Cfg::kStages - 1; ++k) issue(k, k);
     int stage = 0;
-    for (int item = first; item < total; item += stride) {
-        issue(item + (Cfg::kStages - 1) * stride, (stage + Cfg::kStages - 1) % Cfg::kStages);
+    for (int sq = 0; item_of_seq(sq) < total; ++sq) {
+        const int item = item_of_seq(sq), hh = sq % gh;
+        issue(sq + Cfg::kStages - 1, (stage + Cfg::kStages - 1) % Cfg::kStages);
         cp_async_wait<Cfg::kStages - 1>();
         __syncthreads();
         const uint8_t *st = smem + stage * Cfg::kStageBytes;
-        const int qi = item / nblk, blk = item - (item / nblk) * nblk;
+        const int qu = item / nblk, blk = item - (item / nblk) * nblk;
         const int c0 = blk * kScrRows;
         const int ne = eligible(*reinterpret_cast<const int *>(st + Cfg::kPosOff) + a.qpos_bias, a.C);
+        float2 *out = kFold ? tmp : ws.scr + (int64_t)qu * a.C;
+        const int base = kFold ? c0 : 0;
         if (c0 < ne) {
-            if (Cfg::kMma) screen_stage_mma<D>(st, Cfg::kQOff, Cfg::kBiasOff, a.scale, c0, ne, ws.scr + (int64_t)qi * a.C, gscr);
-            else screen_stage_f32<T, D, Cfg>(st, a.scale, c0, ne, ws.scr + (int64_t)qi * a.C, gscr);
+            if (Cfg::kMma) screen_stage_mma<D>(st, Cfg::kQOff, Cfg::kBiasOff, a.scale, c0, ne, out, base, gscr);
+            else screen_stage_f32<T, D, Cfg>(st, a.scale, c0, ne, out, base, gscr);
         }
         __syncthreads();
-        if (c0 < ne && tid < Cfg::kGroupsPerBlock) {
+        if (kFold && c0 < ne) {
+            // fold this head's intervals into the group's; after the last head write the
+            // group's centre and radius, and its 64-chunk maxima through the slots
+            const bool last = hh == gh - 1;
+            for (int r = tid; r < kScrRows; r += kScrThreads) {
+                const int c = c0 + r;
+                float s = -INFINITY, e = 0.f;
+                if (c < ne) {
+                    const float2 v = tmp[r];
+                    float lo = __fsub_rd(v.x, v.y), hi = __fadd_ru(v.x, v.y);
+                    if (hh > 0) {
+                        lo = fmaxf(lo, lohi[r].x);
+                        hi = fmaxf(hi, lohi[r].y);
+                    }
+                    lohi[r] = make_float2(lo, hi);
+                    if (last) {
+                        interval_mid(lo, hi, s, e);
+                        ws.scr[(int64_t)qu * a.C + c] = make_float2(s, e);
+                    }
+                }
+                if (last) {  // 32-row slot maxima (kScrRows = 128 rows, one warp-row each)
+                    const float ms = warp_max(s), me = warp_max(e);
+                    if ((tid & 31) == 0) gscr[r >> 5] = make_float2(ms, me);
+                }
+            }
+            __syncthreads();
+            if (last && tid < Cfg::kGroupsPerBlock) {
+                float2 m = gscr[2 * tid];
+                m.x = fmaxf(m.x, gscr[2 * tid + 1].x);
+                m.y = fmaxf(m.y, gscr[2 * tid + 1].y);
+                const int g = blk * Cfg::kGroupsPerBlock + tid;
+                if (g * kGroupRows < ne) ws.gmax[(int64_t)qu * G + g] = m;
+            }
+        } else if (c0 < ne && tid < Cfg::kGroupsPerBlock) {
             const int g0 = tid * Cfg::kSlotsPerGroup;
             float2 m = gscr[g0];
             for (int k = 1; k < Cfg::kSlotsPerGroup; ++k) {
@@ -168,7 +214,7 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(SelectArgs a
                 m.y = fmaxf(m.y, gscr[g0 + k].y);
             }
             const int g = blk * Cfg::kGroupsPerBlock + tid;
-            if (g * kGroupRows < ne) ws.gmax[(int64_t)qi * G + g] = m;
+            if (g * kGroupRows < ne) ws.gmax[(int64_t)qu * G + g] = m;
         }
         __syncthreads();
         stage = (stage + 1) % Cfg::kStages;
@@ -179,16 +225,17 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(SelectArgs a
 template <typename T, int D>
 hils_status launch_screen(const SelectArgs &a, cudaStream_t s) {
     using Cfg = ScrCfg<T, D>;
-    static KernelSetup setup;
+    static KernelSetup setup1, setupg;
+    const void *fn = a.G > 1 ? (const void *)select_screen_kernel<T, D, true> : (const void *)select_screen_kernel<T, D, false>;
     int per_sm = 1;
-    const hils_status st = kernel_setup(setup, (const void *)select_screen_kernel<T, D>, kScrThreads,
-                                        Cfg::kSmemBytes, &per_sm);
+    const hils_status st = kernel_setup(a.G > 1 ? setupg : setup1, fn, kScrThreads, Cfg::kSmemBytes, &per_sm);
     if (st != HILS_OK) return st;
-    const int64_t nq = (int64_t)a.B * a.H * a.Lq;
-    const int64_t items = nq * ((a.C + kScrRows - 1) / kScrRows);
+    const int64_t nu = (int64_t)a.B * (a.H / a.G) * a.Lq;
+    const int64_t items = nu * ((a.C + kScrRows - 1) / kScrRows);
     const int64_t slots = (int64_t)per_sm * device_sm_count();
     const int64_t grid = items < slots ? items : slots;
-    select_screen_kernel<T, D><<<(unsigned)grid, kScrThreads, Cfg::kSmemBytes, s>>>(a);
+    if (a.G > 1) select_screen_kernel<T, D, true><<<(unsigned)grid, kScrThreads, Cfg::kSmemBytes, s>>>(a);
+    else select_screen_kernel<T, D, false><<<(unsigned)grid, kScrThreads, Cfg::kSmemBytes, s>>>(a);
     return record_cuda_error(cudaGetLastError());
 }
 

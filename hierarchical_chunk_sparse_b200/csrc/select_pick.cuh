@@ -99,89 +99,37 @@ __device__ void rescreen_pool(const QueryCtx &q, const float *qs, Pool64 &pool, 
     }
 }
 
-// Grouped heads: each head's tight interval, folded into the group maximum's interval;
-// each head's own value is kept in sh[head][entry] for the output. The rows of up to
-// kHB heads are loaded together before their sums run.
-template <typename T, int D, int NT>
-__device__ void rescreen_pool(const GroupCtx &g, const float *qs, Pool64 &pool, int total, float *sh) {
-    constexpr int kN = Vec<T>::kN, kQuarter = D / 4, kU = kQuarter / kN;
-    constexpr int kHB = sizeof(T) == 2 ? 4 : 2;
-    const int tid = threadIdx.x, sub = tid & 3;
-    for (int base = 0; base < total; base += NT / 4) {
-        const int j = base + (tid >> 2);
-        const bool ok = j < total;
-        const int c = ok ? pool.idx[j] : 0;
-        float lo = -INFINITY, hi = -INFINITY;
-        for (int h0 = 0; h0 < g.G; h0 += kHB) {
-            uint4 kv[kHB][kU];
-            float bias[kHB];
-#pragma unroll
-            for (int hb = 0; hb < kHB; ++hb) {
-                const bool live = ok && h0 + hb < g.G;
-                const QueryCtx q = head_ctx(g, h0 + hb < g.G ? h0 + hb : h0, (int)sizeof(T));
-                const uint4 *kr = reinterpret_cast<const uint4 *>(static_cast<const T *>(q.khead) +
-                                                                  (int64_t)c * q.kst + sub * kQuarter);
-#pragma unroll
-                for (int u = 0; u < kU; ++u) kv[hb][u] = live ? __ldg(kr + u) : make_uint4(0, 0, 0, 0);
-                bias[hb] = live ? __ldg(q.bhead + c) : 0.f;
-            }
-#pragma unroll
-            for (int hb = 0; hb < kHB; ++hb) {
-                if (h0 + hb >= g.G) break;  // uniform
-                const QueryCtx q = head_ctx(g, h0 + hb, (int)sizeof(T));
-                const float *qh = qs + (h0 + hb) * D + sub * kQuarter;
-                float dot = 0.f, ad = 0.f;
-#pragma unroll
-                for (int u = 0; u < kU; ++u) {
-                    float kf[kN];
-                    widen(kv[hb][u], kf, T());
-#pragma unroll
-                    for (int i = 0; i < kN; ++i) {
-                        dot = fmaf(qh[u * kN + i], kf[i], dot);
-                        ad = fmaf(fabsf(qh[u * kN + i]), fabsf(kf[i]), ad);
-                    }
-                }
-                dot += __shfl_xor_sync(kFull, dot, 1);
-                ad += __shfl_xor_sync(kFull, ad, 1);
-                dot += __shfl_xor_sync(kFull, dot, 2);
-                ad += __shfl_xor_sync(kFull, ad, 2);
-                const float s = ok ? fmaf(dot, q.scale, bias[hb]) : 0.f;
-                const float e = fmaf(q.scale * ad, (float)(D + 2) * 0x1p-23f, fabsf(s) * 0x1p-22f);
-                fold_interval(s, e, lo, hi);
-                if (ok && sub == 0) sh[(h0 + hb) * kPoolCap + j] = s;
-            }
-        }
-        if (ok && sub == 0) interval_mid(lo, hi, pool.s[j], pool.e[j]);
-    }
-}
-
-// A group's kept list from the pool: chunk indices ascending for the group, and each
-// head's own tight screen value (sh, from rescreen_pool) of the kept chunks.
+// The float64 score of chunk c for one query head, the same fixed-order chain as
+// exact_score (each product of the float64 values, summed in x order, then times scale
+// plus b'_c), with the query's elements from shared memory (float32 copies that hold
+// the input values exactly).
 template <typename T, int D>
-__device__ void group_write_pool(const GroupCtx &q, const EntryList &list, const Pool64 &pool, const float *sh,
-                                 int total, const SelectArgs &a, int64_t qg, int b, int g, int i) {
-    const int lane = threadIdx.x & 31;
-    const int K = a.topk, n = list.n;
-    int rank = lane, me = -1, slot = 0;
-    if (lane < n) {
-        me = list.idx[lane];
-        rank = 0;
+__device__ __forceinline__ double exact_row(const QueryCtx &q, const float *qs, int c) {
+    constexpr int kN = Vec<T>::kN, kHalf = D / kN / 2;
+    const uint4 *kr = reinterpret_cast<const uint4 *>(static_cast<const T *>(q.khead) + (int64_t)c * q.kst);
+    const float bias = __ldg(q.bhead + c);
+    double acc = 0.0;
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j) rank += (j < n && list.idx[j] < me) ? 1 : 0;
+    for (int h = 0; h < 2; ++h) {
+        uint4 kv[kHalf];
 #pragma unroll
-        for (int j = 0; j < kPoolCap; ++j) slot = (j < total && pool.idx[j] == me) ? j : slot;
+        for (int u = 0; u < kHalf; ++u) kv[u] = __ldg(kr + h * kHalf + u);
+#pragma unroll
+        for (int u = 0; u < kHalf; ++u) {
+            float kf[kN];
+            widen(kv[u], kf, T());
+#pragma unroll
+            for (int i = 0; i < kN; ++i)
+                acc = __dadd_rn(acc, __dmul_rn((double)qs[(h * kHalf + u) * kN + i], (double)kf[i]));
+        }
     }
-    if (lane < K) a.idx[qg * K + rank] = lane < n ? me : -1;
-    for (int hh = 0; hh < q.G; ++hh) {
-        const int64_t qh = ((int64_t)b * a.H + g * a.G + hh) * a.Lq + i;
-        if (lane < K) a.score[qh * K + rank] = lane < n ? sh[hh * kPoolCap + slot] : -INFINITY;
-    }
-    if (lane == 0) a.nsel[qg] = n;
+    return __dadd_rn(__dmul_rn(acc, (double)q.scale), (double)bias);
 }
 
 struct PickSmem {
     float qs[kMaxGroup * 128];  // the query rows (float32) of the unit's heads
-    float pool_sh[kMaxGroup * kPoolCap];  // grouped heads: each head's value of each pool entry
+    double xh[kMaxGroup * kPoolCap];  // float64 score of each (head, pool entry)
+    uint8_t kept[kPoolCap];
     float2 gm[kMaxGroups];
     __align__(16) unsigned gkey[kMaxGroups];  // order-preserving keys of gm[].x
     uint16_t cand_g[kMaxGroups];
@@ -204,47 +152,11 @@ __host__ __device__ __forceinline__ size_t dec_ws_bytes(int64_t queries, int C) 
     return kSelectStatusBytes + scr;
 }
 
-// The screen rows one pick unit reads: one query's, or the G rows of a group's heads
-// (consecutive query heads, Lq queries apart in the workspace).
+// The screen row one pick unit reads (one query's, or the group centres and radii the
+// screen folded for a (b, group, query)), and its 64-chunk maxima.
 struct ScrRows {
     const float2 *scr, *gmx;
-    int64_t scr_hs, gmx_hs;  // head strides
-    int G;
 };
-
-// Screen value and radius of chunk c < ne for the unit: a group's is the interval of
-// the maximum over its heads.
-template <bool kGroup>
-__device__ __forceinline__ float2 scr_at(const ScrRows &r, int c) {
-    if constexpr (!kGroup) {
-        return __ldcg(&r.scr[c]);
-    } else {
-        float lo = -INFINITY, hi = -INFINITY;
-        for (int hh = 0; hh < r.G; ++hh) {
-            const float2 v = __ldcg(&r.scr[hh * r.scr_hs + c]);
-            fold_interval(v.x, v.y, lo, hi);
-        }
-        float2 o;
-        interval_mid(lo, hi, o.x, o.y);
-        return o;
-    }
-}
-
-// Largest screen value and largest radius of 64-chunk group g: for a group of heads,
-// the largest over its heads of each (the value is still attained by one chunk of the
-// group, whose group score is at least that value minus the largest radius).
-template <bool kGroup>
-__device__ __forceinline__ float2 gmax_at(const ScrRows &r, int g) {
-    float2 m = __ldcg(&r.gmx[g]);
-    if constexpr (kGroup) {
-        for (int hh = 1; hh < r.G; ++hh) {
-            const float2 v = __ldcg(&r.gmx[hh * r.gmx_hs + g]);
-            m.x = fmaxf(m.x, v.x);
-            m.y = fmaxf(m.y, v.y);
-        }
-    }
-    return m;
-}
 
 __device__ __forceinline__ ScreenWs screen_ws(const SelectArgs &a) {
     const int64_t nq = (int64_t)a.B * a.H * a.Lq;
@@ -265,14 +177,8 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
     int t, b = 0, grp = 0, i = 0;
     Ctx q;
     ScrRows rows;
-    rows.G = 1;
-    rows.scr_hs = (int64_t)a.Lq * a.C;
-    rows.gmx_hs = (int64_t)a.Lq * groups_of(a.C);
-    int64_t q0 = u;  // the unit's first query head's query index
     if constexpr (kGroup) {
         q = make_group_ctx<T, D>(a, u, t, b, grp, i);
-        q0 = ((int64_t)b * a.H + (int64_t)grp * a.G) * a.Lq + i;
-        rows.G = a.G;
         for (int hh = 0; hh < a.G; ++hh)
             for (int x = tid; x < D; x += NT)
                 ps.qs[hh * D + x] = (float)static_cast<const T *>(q.head.qrow)[hh * q.qsh + x];
@@ -280,8 +186,8 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
         q = make_ctx<T, D>(a, u, t);
         for (int x = tid; x < D; x += NT) ps.qs[x] = (float)static_cast<const T *>(q.qrow)[x];
     }
-    rows.scr = ws.scr + q0 * a.C;
-    rows.gmx = ws.gmax + q0 * groups_of(a.C);
+    rows.scr = ws.scr + u * a.C;
+    rows.gmx = ws.gmax + u * groups_of(a.C);
     auto write = [&](const EntryList &list) {
         if constexpr (kGroup) group_write<T, D>(q, ps.qs, list, a, u, b, grp, i);
         else warp_write(list, a.topk, u, a.idx, a.score, a.nsel);
@@ -319,7 +225,7 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
     // chunks); e_max = largest radius; every chunk with hi < T - e_max is certainly out
     float em = 0.f;
     for (int g = tid; g < ((G + 3) & ~3); g += NT) {
-        const float2 v = g < G ? gmax_at<kGroup>(rows, g) : make_float2(-INFINITY, 0.f);
+        const float2 v = g < G ? __ldcg(&rows.gmx[g]) : make_float2(-INFINITY, 0.f);
         ps.gm[g] = v;
         ps.gkey[g] = g < G ? ordered_key(v.x) : 0u;  // 0: below every value's key
         em = fmaxf(em, v.y);
@@ -356,7 +262,7 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
         for (int j = 0; j < kPer; ++j) {
             const int e = e0 + j * NT + tid;
             cc[j] = e < ncg * kGroupRows ? ps.cand_g[e / kGroupRows] * kGroupRows + e % kGroupRows : ne;
-            v[j] = cc[j] < ne ? scr_at<kGroup>(rows, cc[j]) : make_float2(-INFINITY, 0.f);
+            v[j] = cc[j] < ne ? __ldcg(&rows.scr[cc[j]]) : make_float2(-INFINITY, 0.f);
         }
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
@@ -373,11 +279,11 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
     }
     __syncthreads();  // every candidate is in the pool before any thread reads it
     const int total = ps.pool_n;
-    if (total <= kPoolCap) {
+    if constexpr (!kGroup) {
+      if (total <= kPoolCap) {
         // the candidates are screened again on CUDA cores (round-to-nearest fused
         // multiply-adds: the tight radius), so that few need the float64 score
-        if constexpr (kGroup) rescreen_pool<T, D, NT>(q, ps.qs, ps.pool, total, ps.pool_sh);
-        else rescreen_pool<T, D, NT>(q, ps.qs, ps.pool, total);
+        rescreen_pool<T, D, NT>(q, ps.qs, ps.pool, total);
         __syncthreads();
         if (w == 0) {
             Slots<2> sl;
@@ -396,9 +302,51 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
             const int n = warp_append<2>(sl, keep, ps.out, 0);
             if (lane == 0) ps.out.n = n;
             __syncwarp();
-            if constexpr (kGroup) group_write_pool<T, D>(q, ps.out, ps.pool, ps.pool_sh, total, a, u, b, grp, i);
-            else write(ps.out);
+            write(ps.out);
         }
+        return;
+      }
+    } else if (total <= kPoolCap) {
+        // Grouped heads: every chunk outside the pool is certainly out, and the pool
+        // holds more than K chunks (the K+1 that attain the largest group maxima). The
+        // float64 score of every (head, pool entry), one thread each, decides the kept
+        // set exactly: the K largest by (score, then lower chunk index); a group's score
+        // is the largest of its heads'.
+        const int nh = a.G;
+        for (int p = tid; p < total * nh; p += NT) {
+            const int j = p % total, hh = p / total;
+            ps.xh[hh * kPoolCap + j] = exact_row<T, D>(head_ctx(q, hh, (int)sizeof(T)), ps.qs + hh * D, ps.pool.idx[j]);
+        }
+        __syncthreads();
+        for (int j = tid; j < total; j += NT) {
+            double x = ps.xh[j];
+            for (int hh = 1; hh < nh; ++hh) x = fmax(x, ps.xh[hh * kPoolCap + j]);
+            ps.pool.x[j] = x;
+        }
+        __syncthreads();
+        for (int j = tid; j < total; j += NT) {
+            const double xj = ps.pool.x[j];
+            const int cj = ps.pool.idx[j];
+            int rank = 0;
+            for (int k = 0; k < total; ++k) {
+                const double xk = ps.pool.x[k];
+                rank += (xk > xj || (xk == xj && ps.pool.idx[k] < cj)) ? 1 : 0;
+            }
+            ps.kept[j] = rank < K ? 1 : 0;
+        }
+        __syncthreads();
+        // outputs in ascending chunk index: each kept entry's position is the number of
+        // kept entries with a lower index; scores are the heads' own (rounded) values
+        for (int j = tid; j < total; j += NT) {
+            if (!ps.kept[j]) continue;
+            const int cj = ps.pool.idx[j];
+            int pos = 0;
+            for (int k = 0; k < total; ++k) pos += (ps.kept[k] && ps.pool.idx[k] < cj) ? 1 : 0;
+            a.idx[u * K + pos] = cj;
+            for (int hh = 0; hh < a.G; ++hh)
+                a.score[(((int64_t)b * a.H + grp * a.G + hh) * a.Lq + i) * K + pos] = (float)ps.xh[hh * kPoolCap + j];
+        }
+        if (tid == 0) a.nsel[u] = K;
         return;
     }
     if (w != 0) return;
@@ -406,7 +354,7 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
     int n = 0;
     for (int c0 = 0; c0 < ne; c0 += 32) {
         const int c = c0 + lane;
-        const float2 v = c < ne ? scr_at<kGroup>(rows, c) : make_float2(-INFINITY, 0.f);
+        const float2 v = c < ne ? __ldcg(&rows.scr[c]) : make_float2(-INFINITY, 0.f);
         const bool cand = c < ne && __fadd_ru(v.x, v.y) >= cut;
         if (!__any_sync(kFull, cand)) continue;
         Slots<2> sl;
