@@ -292,7 +292,7 @@ def prefill_flops(w, part: str = "step") -> float:
 # measured for the current kernels, each with its command in profiles/: select_decode512k.md
 # (screen + pick of one select call), attend_decode_128k.md, attend_prefill_tc_prefill8k.md.
 # A kernel that changes after its capture reports null here until it is captured again.
-MEASURED_TRAFFIC = {"select": 69_300_992, "attend_decode": 25_235_968, "attend_prefill": 666_330_112}
+MEASURED_TRAFFIC = {"select": 69_358_080, "attend_decode": 25_235_968, "attend_prefill": 661_831_680}
 
 
 class PrefillBench:
@@ -485,17 +485,28 @@ def run_profile_case(args):
     print(json.dumps({"profile_case": case, "launches": args.warmup + args.steps}))
 
 
-def mean_item_union(idx: torch.Tensor, nsel: torch.Tensor, C: int) -> float:
-    """Mean number of distinct chunks kept by the queries of one 256-query work item."""
+def mean_item_union(idx: torch.Tensor, nsel: torch.Tensor, C: int, q: int = 256) -> float:
+    """Mean number of distinct chunks kept by the q consecutive queries of one work item of
+    the tensor-core prefill attend (256 queries of one head, or 256 / P queries of P
+    packed heads of a group, which share one kept list)."""
     B, H, N, K = idx.shape
-    nb = N // 256
+    nb = N // q
     if nb == 0:
         return 0.0
-    i = idx[:, :, : nb * 256].reshape(B, H, nb, 256 * K).long()
-    keep = (torch.arange(K, device=idx.device).view(1, 1, 1, K) < nsel[:, :, : nb * 256, None]).reshape(B, H, nb, 256 * K)
+    i = idx[:, :, : nb * q].reshape(B, H, nb, q * K).long()
+    keep = (torch.arange(K, device=idx.device).view(1, 1, 1, K) < nsel[:, :, : nb * q, None]).reshape(B, H, nb, q * K)
     bits = torch.zeros(B, H, nb, C + 1, dtype=torch.int32, device=idx.device)
     bits.scatter_(3, torch.where(keep & (i >= 0), i, torch.full_like(i, C)), 1)
     return float(bits[..., :C].sum(-1).float().mean())
+
+
+def packed_heads(G: int) -> int:
+    """Query heads the tensor-core prefill attend packs into one tile: the largest power of
+    two <= 8 that divides the group size."""
+    p = 1
+    while p < 8 and G % (2 * p) == 0:
+        p *= 2
+    return p
 
 
 def measure_prefill(wp, dev, stream, flush, args, world, peaks, peak_src, traffic):
@@ -522,7 +533,7 @@ def measure_prefill(wp, dev, stream, flush, args, world, peaks, peak_src, traffi
            "algorithmic_gflop_per_step": fl / 1e9, "steps": n,
            "kernel_ms": ks, "clocks": pclk.summary(),
            "step_frac_of_peak": tf / peaks["bf16_tflops"],
-           "mean_item_union_chunks": mean_item_union(pb.idx, pb.nsel, wp.C),
+           "mean_item_union_chunks": mean_item_union(pb.idx, pb.nsel, wp.C, 256 // packed_heads(wp.G)),
            "roofline": {"bound": "tensor", "kernel": "attend", "achieved": tf_att,
                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                         "frac": tf_att / peaks["bf16_tflops"], "traffic": traffic,
