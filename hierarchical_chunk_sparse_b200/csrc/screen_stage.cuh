@@ -4,6 +4,7 @@
 // tensor cores (bf16) or CUDA cores (float32), for the decode select's screen kernel.
 #pragma once
 #include "select_pick.cuh"
+#include "tc_common.cuh"
 
 namespace hils {
 namespace {
@@ -62,18 +63,20 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
                  : "r"(addr));
 }
 
-// Tensor-core screen of one stage (bf16): warp w takes rows 16w..16w+15. Per k-step one
-// ldmatrix.x4 of the 16x16 row tile A and three m16n8k16 MMAs: A times q (q in column 0
+// Tensor-core screen of one stage (bf16): warp w takes rows 16w..16w+15. The stage's rows
+// are ROWS x 128-byte column blocks (64 elements each) as TMA writes them with the
+// 128-byte swizzle: 16-byte unit u of row r sits in block u / 8 at r * 128 + ((u % 8) ^
+// (r % 8)) * 16. Per k-step one ldmatrix.x4 of the 16x16 row tile A and three m16n8k16
+// MMAs: A times q (q in column 0
 // of B), and A times its own rows 0-7 and 8-15 (Gram blocks whose diagonals are |k'|^2;
 // the B fragments of those are A's own registers). Radius: the tensor-core float32
 // accumulation order and rounding are not specified, so the bound allows d * 2^-16 of
 // scale |q| |k'| (about 2^7 times the round-to-nearest bound), plus 2^-22 |s| for the
 // final fused multiply-add; |k'|^2 itself carries a 2^-8 margin.
 // (s_c, e_c) of chunk c goes to out[c - base].
-template <int D>
+template <int D, int ROWS>
 __device__ void screen_stage_mma(const uint8_t *st, int q_off, int bias_off, float scale, int c0, int ne,
                                  float2 *out, int base, float2 *slots) {
-    constexpr int kRowBytes = D * 2;
     constexpr int kKSteps = D / 16;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
     const int rbase = warp * 16;
@@ -85,13 +88,13 @@ __device__ void screen_stage_mma(const uint8_t *st, int q_off, int bias_off, flo
     }
     qn2 = warp_sum(qn2);
     const int lrow = rbase + (lane & 7) + ((lane >> 3) & 1) * 8;
-    const uint32_t row_addr = (uint32_t)__cvta_generic_to_shared(st + lrow * kRowBytes);
+    const uint32_t row_addr = (uint32_t)__cvta_generic_to_shared(st + lrow * 128);
     float dacc[4] = {0.f, 0.f, 0.f, 0.f}, g1[4] = {0.f, 0.f, 0.f, 0.f}, g2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < kKSteps; ++ks) {
         uint32_t a[4];
         const int unit = ks * 2 + (lane >> 4);
-        ldmatrix_x4(a, row_addr + (uint32_t)((unit ^ (lrow & 7)) * 16));
+        ldmatrix_x4(a, row_addr + (uint32_t)((unit >> 3) * (ROWS * 128) + (((unit & 7) ^ (lrow & 7)) << 4)));
         const uint32_t b0 = g == 0 ? qw[ks * 8 + tq] : 0u;
         const uint32_t b1 = g == 0 ? qw[ks * 8 + 4 + tq] : 0u;
         mma_bf16_16816(dacc, a, b0, b1);
@@ -180,8 +183,9 @@ __device__ void screen_stage_f32(const uint8_t *st, float scale, int c0, int ne,
 }
 
 // Layout of one pipeline stage of ROWS summary rows screened by NT threads: the rows
-// (16-byte units of bf16 rows permuted by (unit ^ (row & 7))), their biases, the query
-// row and the query's position.
+// (bf16: 128-byte column blocks written by TMA, see screen_stage_mma; float32: plain
+// rows), their biases, the query row and the query's position. bf16 stages start on
+// 1024-byte boundaries (the swizzle's period).
 template <typename T, int D, int NT, int ROWS>
 struct StageCfg {
     static constexpr int kThreads = NT;
@@ -193,7 +197,7 @@ struct StageCfg {
     static constexpr int kBiasOff = ROWS * kRowBytes;
     static constexpr int kQOff = kBiasOff + ROWS * 4;
     static constexpr int kPosOff = kQOff + kRowBytes;
-    static constexpr int kStageBytes = kPosOff + 16;
+    static constexpr int kStageBytes = sizeof(T) == 2 ? (kPosOff + 16 + 1023) / 1024 * 1024 : kPosOff + 16;
     static constexpr int kGroupsPerBlock = ROWS / kGroupRows;
     static constexpr int kCopies = ROWS * kTPR / NT;  // 16-byte copies per thread
     static_assert(2 * kRPT == kTPR, "half-square transpose reduction");
@@ -207,21 +211,23 @@ struct StageCfg {
 };
 
 // Every thread issues its share of the cp.async copies of one stage: `rows` summary
-// rows from `kh` (row stride kst elements) starting at chunk c0, their biases, the query
-// row, and the position (from `pos` if not null, else the value `pos_value`).
+// rows from `kh` (row stride kst elements) starting at chunk c0 (float32 only: bf16 rows
+// come by TMA), their biases, the query row, and the position (from `pos` if not null,
+// else the value `pos_value`).
 template <typename T, typename Cfg>
 __device__ __forceinline__ void stage_issue(uint8_t *st, const T *kh, int64_t kst, int c0, int rows, const float *brow,
                                             const T *qrow, const int32_t *pos, int pos_value) {
     const int tid = threadIdx.x, col = tid % Cfg::kTPR;
     const int r0 = tid / Cfg::kTPR;
-    const uint8_t *src = reinterpret_cast<const uint8_t *>(kh + (int64_t)(c0 + r0) * kst) + col * 16;
-    const int dcol = Cfg::kMma ? (col ^ (r0 & 7)) : col;
-    uint8_t *dst = st + r0 * Cfg::kRowBytes + dcol * 16;
-    constexpr int kStep = Cfg::kThreads / Cfg::kTPR;
-    const int64_t src_step = (int64_t)kStep * kst * (int64_t)sizeof(T);
+    if constexpr (!Cfg::kMma) {
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(kh + (int64_t)(c0 + r0) * kst) + col * 16;
+        uint8_t *dst = st + r0 * Cfg::kRowBytes + col * 16;
+        constexpr int kStep = Cfg::kThreads / Cfg::kTPR;
+        const int64_t src_step = (int64_t)kStep * kst * (int64_t)sizeof(T);
 #pragma unroll
-    for (int k = 0; k < Cfg::kCopies; ++k)
-        if (r0 + k * kStep < rows) cp_async16(dst + k * kStep * Cfg::kRowBytes, src + k * src_step);
+        for (int k = 0; k < Cfg::kCopies; ++k)
+            if (r0 + k * kStep < rows) cp_async16(dst + k * kStep * Cfg::kRowBytes, src + k * src_step);
+    }
     for (int r = tid; r < rows; r += Cfg::kThreads) cp_async4(st + Cfg::kBiasOff + r * 4, brow + r);
     for (int u = tid; u < Cfg::kTPR; u += Cfg::kThreads)
         cp_async16(st + Cfg::kQOff + u * 16, reinterpret_cast<const uint8_t *>(qrow) + u * 16);

@@ -71,8 +71,11 @@ __global__ void __launch_bounds__(kWarpKernelThreads) select_warp_kernel(SelectA
 //
 // select_screen_kernel: a persistent grid of 256-thread CTAs (2 per SM) walks the
 // (query, 128-row block) items, query-major, with a stride of the grid size, through a
-// 3-stage cp.async ring; a stage holds the block's summary rows, their biases, the
-// query row and the query's position, so no load waits on another. bf16 rows are
+// 3-stage ring; a stage holds the block's summary rows (bf16: one TMA tile load per
+// 64-column block, completing on the stage's mbarrier; float32: cp.async), their
+// biases, the query row and the query's position (cp.async), so no load waits on
+// another. Every mbarrier wait is bounded: on expiry the CTA sets the select's status
+// word, stops, and lets its copies in flight land before it exits. bf16 rows are
 // screened on the tensor cores (mma.sync, 16 rows per warp; |k'|^2 from the Gram
 // diagonal), float32 rows on CUDA cores (kTPR threads per row, packed FMAs, a
 // transpose reduction). Written to the workspace: the screen value s_c and radius e_c
@@ -97,6 +100,7 @@ constexpr int kScrThreads = 256;
 constexpr int kPickThreads = 256;
 constexpr int kScrRows = 128;   // summary rows per item (one pipeline stage)
 constexpr int kDecStages = 3;   // pipeline stages (2 CTAs per SM for bf16 rows of d = 128)
+constexpr long long kScreenWaitLimit = 1ll << 26;  // polls of a stage's barrier before giving up
 
 template <typename T, int D>
 struct ScrCfg : StageCfg<T, D, kScrThreads, kScrRows> {
@@ -104,7 +108,7 @@ struct ScrCfg : StageCfg<T, D, kScrThreads, kScrRows> {
     static constexpr int kStages = Base::kStageBytes > 40000 ? 2 : kDecStages;
     static constexpr int kGscrOff = kStages * Base::kStageBytes;
     static constexpr int kFoldOff = kGscrOff + kScrRows * 8;  // grouped heads: one head's (s, e), the group's (lo, hi)
-    static constexpr int kSmemBytes = kFoldOff + 2 * kScrRows * 8;
+    static constexpr int kSmemBytes = kFoldOff + 2 * kScrRows * 8 + (Base::kMma ? 1024 : 0);  // + alignment slack
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 // One CTA per query (per (b, group, query) for grouped heads), dependent-launched after
@@ -118,12 +122,26 @@ __global__ void __launch_bounds__(kPickThreads) select_pick_kernel(SelectArgs a)
 }
 
 template <typename T, int D, bool kFold>
-__global__ void __launch_bounds__(kScrThreads) select_screen_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                    SelectArgs a) {
     using Cfg = ScrCfg<T, D>;
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    // bf16 stages: 1024-byte alignment by pointer arithmetic on the shared array
+    uint8_t *smem = Cfg::kMma ? smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u) : smem_raw;
+    __shared__ unsigned long long sbar[kDecStages];
+    __shared__ uint32_t sabort;
     float2 *gscr = reinterpret_cast<float2 *>(smem + Cfg::kGscrOff);
     pdl_trigger();
     const int tid = threadIdx.x;
+    if (tid == 0) {
+        sabort = 0u;
+        if (Cfg::kMma) {
+            for (int k = 0; k < Cfg::kStages; ++k) tc::mbar_init(tc::smem_u32(&sbar[k]), 1);
+            asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        }
+    }
+    __syncthreads();
+    int tma_issued[kDecStages] = {0, 0, 0};  // thread 0: row loads started per stage
     const int nblk = (a.C + kScrRows - 1) / kScrRows;
     const int gh = kFold ? a.G : 1;           // heads folded per item (1: one query head)
     const int nu = a.B * (a.H / gh) * a.Lq;   // query units: queries, or (b, group, query)
@@ -151,6 +169,14 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(SelectArgs a
             stage_issue<T, Cfg>(smem + stage * Cfg::kStageBytes, kh, a.Ksum.st, c0, min(kScrRows, a.C - c0),
                                 a.Bsum + ((int64_t)b * a.H + h) * a.C + c0, qrow,
                                 a.qpos ? a.qpos + (int64_t)b * a.Lq + i : nullptr, i);
+            if (Cfg::kMma && tid == 0) {  // the rows: (D / 64) boxes of 128 rows x 64 columns
+                const uint32_t bar = tc::smem_u32(&sbar[stage]);
+                const uint32_t dst = tc::smem_u32(smem + stage * Cfg::kStageBytes);
+                ++tma_issued[stage];
+                tc::mbar_expect_tx(bar, kScrRows * D * 2);
+#pragma unroll
+                for (int x = 0; x < D / 64; ++x) tc::tma_load_4d(dst + x * kScrRows * 128, &tmK, bar, x * 64, c0, h, b);
+            }
         }
         cp_async_commit();
     };
@@ -161,7 +187,17 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(SelectArgs a
         const int item = item_of_seq(sq), hh = sq % gh;
         issue(sq + Cfg::kStages - 1, (stage + Cfg::kStages - 1) % Cfg::kStages);
         cp_async_wait<Cfg::kStages - 1>();
+        if (Cfg::kMma) {  // the stage's rows: use sq / kStages of its barrier
+            const uint32_t bar = tc::smem_u32(&sbar[stage]), par = (uint32_t)(sq / Cfg::kStages) & 1u;
+            bool ok = false;
+            for (long long it = 0; it < kScreenWaitLimit && !ok; ++it) ok = tc::mbar_try_wait(bar, par);
+            if (!ok) {
+                sabort = 1u;
+                atomicOr(static_cast<uint32_t *>(a.ws), 1u);
+            }
+        }
         __syncthreads();
+        if (Cfg::kMma && sabort) break;  // uniform: read after the barrier
         const uint8_t *st = smem + stage * Cfg::kStageBytes;
         const int qu = item / nblk, blk = item - (item / nblk) * nblk;
         const int c0 = blk * kScrRows;
@@ -169,7 +205,7 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(SelectArgs a
         float2 *out = kFold ? tmp : ws.scr + (int64_t)qu * a.C;
         const int base = kFold ? c0 : 0;
         if (c0 < ne) {
-            if (Cfg::kMma) screen_stage_mma<D>(st, Cfg::kQOff, Cfg::kBiasOff, a.scale, c0, ne, out, base, gscr);
+            if (Cfg::kMma) screen_stage_mma<D, kScrRows>(st, Cfg::kQOff, Cfg::kBiasOff, a.scale, c0, ne, out, base, gscr);
             else screen_stage_f32<T, D, Cfg>(st, a.scale, c0, ne, out, base, gscr);
         }
         __syncthreads();
@@ -220,6 +256,16 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(SelectArgs a
         stage = (stage + 1) % Cfg::kStages;
     }
     cp_async_wait<0>();
+    if (Cfg::kMma && tid == 0) {
+        // after an abort: every row load started lands before the CTA releases its memory
+        // (each was issued after the previous use of its stage had completed)
+        for (int k = 0; k < Cfg::kStages; ++k) {
+            if (tma_issued[k] == 0) continue;
+            const uint32_t bar = tc::smem_u32(&sbar[k]), par = (uint32_t)(tma_issued[k] - 1) & 1u;
+            for (long long it = 0; it < kScreenWaitLimit; ++it)
+                if (tc::mbar_try_wait(bar, par)) break;
+        }
+    }
 }
 
 template <typename T, int D>
@@ -234,8 +280,11 @@ hils_status launch_screen(const SelectArgs &a, cudaStream_t s) {
     const int64_t items = nu * ((a.C + kScrRows - 1) / kScrRows);
     const int64_t slots = (int64_t)per_sm * device_sm_count();
     const int64_t grid = items < slots ? items : slots;
-    if (a.G > 1) select_screen_kernel<T, D, true><<<(unsigned)grid, kScrThreads, Cfg::kSmemBytes, s>>>(a);
-    else select_screen_kernel<T, D, false><<<(unsigned)grid, kScrThreads, Cfg::kSmemBytes, s>>>(a);
+    CUtensorMap mk{};  // bf16 rows come by TMA; float32 rows do not use the map
+    if (Cfg::kMma && !tc::make_map(&mk, View{a.Ksum.ptr, a.Ksum.sb, a.Ksum.sh, a.Ksum.st}, a.B, a.H, a.C, kScrRows, D))
+        return HILS_ERR_CUDA;
+    if (a.G > 1) select_screen_kernel<T, D, true><<<(unsigned)grid, kScrThreads, Cfg::kSmemBytes, s>>>(mk, a);
+    else select_screen_kernel<T, D, false><<<(unsigned)grid, kScrThreads, Cfg::kSmemBytes, s>>>(mk, a);
     return record_cuda_error(cudaGetLastError());
 }
 

@@ -132,11 +132,12 @@ inline EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [B, H, N, 128] bf16 view -> 4-D map with a (64 elements x rows) box, 128-byte swizzle.
-inline bool make_map(CUtensorMap *m, const View &v, int B, int H, int N, int box_rows) {
+// [B, H, N, d] bf16 view (d = 128 unless given) -> 4-D map with a (64 elements x rows)
+// box, 128-byte swizzle.
+inline bool make_map(CUtensorMap *m, const View &v, int B, int H, int N, int box_rows, int d = 128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[4] = {(cuuint64_t)128, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)v.st * 2, (cuuint64_t)v.sh * 2, (cuuint64_t)v.sb * 2};
     const cuuint32_t box[4] = {64u, (cuuint32_t)box_rows, 1u, 1u};
     const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};

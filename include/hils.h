@@ -157,9 +157,10 @@ int hils_summarize(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ,
  *   nsel  [B, Hk, Lq] int32 out: number of kept chunks, min(K, eligible)
  *   workspace, ws_bytes: scratch of hils_workspace_bytes(p, HILS_CALL_SELECT, Lq, C) bytes
  *         (at least 256), zeroed before first use. Its first 32-bit word is a status
- *         word: the tensor-core path (bf16, d = 128, many queries; bounded waits) sets it
- *         nonzero if a wait on its own asynchronous copies or matrix operations ever
- *         expires, and then writes no output for the affected 128-query tile. */
+ *         word: the paths with bounded waits (the tensor-core path for bf16, d = 128 and
+ *         many queries; the bf16 decode-shaped screen, whose rows arrive by TMA) set it
+ *         nonzero if a wait on their own asynchronous copies or matrix operations ever
+ *         expires, and then write no output for the affected queries. */
 int hils_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *qpos,
                 hils_ctensor Ksum, const float *Bsum, int C,
                 int32_t *idx, float *score, int32_t *nsel,
