@@ -63,8 +63,8 @@ def _load():
         lib.or_set_threads.argtypes = [i]
         lib.or_get_threads.restype = i
         lib.or_summarize.argtypes = [i, i, i, i, i, d_, T, i, T, p, p]
-        lib.or_score_all.argtypes = [i, i, i, i, d_, T, i, p, T, T, i, p]
-        lib.or_select.argtypes = [i, i, i, i, i, i, d_, T, i, p, T, T, i, p, p, p]
+        lib.or_score_all.argtypes = [i, i, i, i, i, d_, T, i, p, T, T, i, p]
+        lib.or_select.argtypes = [i, i, i, i, i, i, i, d_, T, i, p, T, T, i, p, p, p]
         lib.or_attend.argtypes = [i, i, i, i, i, i, i, d_, T, i, p, T, T, p, T, p, p, p]
         lib.or_brute_weights.argtypes = [i, i, i, i, i, d_, T, i, i, i, i, T, p, T,
                                          ctypes.c_longlong, i, p]
@@ -140,21 +140,23 @@ def _as_tensor(a) -> torch.Tensor:
     return a if isinstance(a, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(a))
 
 
-def score_all(Qcal, Ksum, Bsum, S: int, scale: float, qpos=None):
-    """Eq. 7 scores of every chunk for every query; -inf where not eligible."""
+def score_all(Qcal, Ksum, Bsum, S: int, scale: float, qpos=None, exclude_window: int = 0):
+    """Eq. 7 scores of every chunk for every query; -inf where not eligible
+    (exclude_window = W > 0: chunks wholly inside the query's window are not eligible)."""
     Qcal, Ksum, Bsum = _as_tensor(Qcal), _as_tensor(Ksum), _as_tensor(Bsum)
     B, H, Lq, d = Qcal.shape
     C = Ksum.shape[2]
     out = np.zeros((B, H, Lq, C), np.float64)
     qp = None if qpos is None else _i32(qpos)
-    _check(_load().or_score_all(B, H, d, S, float(scale), _desc(Qcal), Lq,
+    _check(_load().or_score_all(B, H, d, S, int(exclude_window), float(scale), _desc(Qcal), Lq,
                                 None if qp is None else _ptr(qp), _desc(Ksum), _desc(Bsum), C,
                                 _ptr(out)), "score_all")
     return out
 
 
-def select(Qcal, Ksum, Bsum, S: int, K: int, scale: float, qpos=None, group: int = 1):
-    """Top-K selection, shared by each group of `group` consecutive query heads.
+def select(Qcal, Ksum, Bsum, S: int, K: int, scale: float, qpos=None, group: int = 1, exclude_window: int = 0):
+    """Top-K selection, shared by each group of `group` consecutive query heads; with
+    exclude_window = W > 0, chunks wholly inside the query's window are not eligible.
     Returns (idx int32 [B,H/G,Lq,K], score float64 [B,H,Lq,K], nsel int32 [B,H/G,Lq])."""
     Qcal, Ksum, Bsum = _as_tensor(Qcal), _as_tensor(Ksum), _as_tensor(Bsum)
     B, H, Lq, d = Qcal.shape
@@ -164,7 +166,7 @@ def select(Qcal, Ksum, Bsum, S: int, K: int, scale: float, qpos=None, group: int
     score = np.zeros((B, H, Lq, K), np.float64)
     nsel = np.zeros((B, H // G, Lq), np.int32)
     qp = None if qpos is None else _i32(qpos)
-    _check(_load().or_select(B, H, G, d, S, K, float(scale), _desc(Qcal), Lq,
+    _check(_load().or_select(B, H, G, d, S, K, int(exclude_window), float(scale), _desc(Qcal), Lq,
                              None if qp is None else _ptr(qp), _desc(Ksum), _desc(Bsum), C,
                              _ptr(idx), _ptr(score), _ptr(nsel)), "select")
     return idx, score, nsel

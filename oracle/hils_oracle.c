@@ -29,6 +29,11 @@
  *   - top-K ties go to the lower chunk index; the kept list is reported in
  *     ascending chunk index.
  *   - a query with no selected chunk and an empty window gets o = 0, lse = -inf.
+ *   - the window-exclusion variant (excl_w = W, the `flags` bit of the library): a
+ *     chunk that lies wholly inside the query's window is not eligible, since the
+ *     window already attends its tokens exactly; the chunk holding the window's first
+ *     token, when the window starts inside a chunk, stays eligible (excluding it would
+ *     leave its earlier tokens unreachable), so its window tokens still count twice.
  *   - grouped-query attention ([summary] Methodology 3, GQA adaptation): H query heads
  *     share H / G key-value heads, query head h reading key-value head h / G. Each query
  *     head has its own landmark queries, summaries and chunk scores; a group's G heads
@@ -102,10 +107,18 @@ static double dot(const double *a, const double *b, int d) {
 }
 
 /* Number of chunks the query at position t may select: complete chunks strictly
- * before its own chunk, capped by the number of summarised chunks. */
-static int eligible_chunks(int t, int S, int C) {
+ * before its own chunk, capped by the number of summarised chunks. With the window
+ * exclusion (excl_w = W > 0) only chunks that start before the window
+ * [max(0, t-W+1), t], that is, that do not lie wholly inside it: c*S < max(0, t-W+1). */
+static int eligible_chunks(int t, int S, int C, int excl_w) {
     int e = t >= 0 ? t / S : 0;
-    return e < C ? e : C;
+    if (e > C) e = C;
+    if (excl_w > 0 && t >= 0) {
+        const int w0 = t - excl_w + 1 > 0 ? t - excl_w + 1 : 0;
+        const int nw = (w0 + S - 1) / S;
+        if (e > nw) e = nw;
+    }
+    return e;
 }
 
 /* --------------------------------------------------------------- Eq. 8 summaries */
@@ -173,10 +186,10 @@ static double chunk_score(const double *q, const or_tensor *Ksum, const or_tenso
     return acc * scale + bias;
 }
 
-int or_score_all(int B, int H, int d, int S, double scale,
+int or_score_all(int B, int H, int d, int S, int excl_w, double scale,
                  or_tensor Qcal, int Lq, const int *qpos,
                  or_tensor Ksum, or_tensor Bsum, int C, double *out) {
-    if (B < 0 || H < 0 || d <= 0 || S <= 0 || Lq < 0 || C < 0 || !out) return -1;
+    if (B < 0 || H < 0 || d <= 0 || S <= 0 || Lq < 0 || C < 0 || excl_w < 0 || !out) return -1;
     if (!valid_dtype(&Qcal) || (C > 0 && (!valid_dtype(&Ksum) || !valid_dtype(&Bsum)))) return -1;
     const long long units = (long long)B * H * Lq;
 #pragma omp parallel num_threads(or_get_threads())
@@ -189,7 +202,7 @@ int or_score_all(int B, int H, int d, int S, double scale,
             const int h = (int)((u / Lq) % H);
             const int b = (int)(u / ((long long)Lq * H));
             const int t = qpos ? qpos[(long long)b * Lq + i] : i;
-            const int ne = eligible_chunks(t, S, C);
+            const int ne = eligible_chunks(t, S, C, excl_w);
             load_vec(&Qcal, b, h, i, d, q);
             double *row = out + u * C;
             for (int c = 0; c < C; ++c)
@@ -219,11 +232,11 @@ static int by_index(const void *pa, const void *pb) {
     return (a->c > b->c) - (a->c < b->c);
 }
 
-int or_select(int B, int H, int G, int d, int S, int K, double scale,
+int or_select(int B, int H, int G, int d, int S, int K, int excl_w, double scale,
               or_tensor Qcal, int Lq, const int *qpos,
               or_tensor Ksum, or_tensor Bsum, int C,
               int *idx, double *score, int *nsel) {
-    if (B < 0 || H < 0 || G <= 0 || H % G != 0 || d <= 0 || S <= 0 || K < 0 || Lq < 0 || C < 0) return -1;
+    if (B < 0 || H < 0 || G <= 0 || H % G != 0 || d <= 0 || S <= 0 || K < 0 || Lq < 0 || C < 0 || excl_w < 0) return -1;
     if (!valid_dtype(&Qcal) || !idx || !score || !nsel) return -1;
     if (C > 0 && (!valid_dtype(&Ksum) || !valid_dtype(&Bsum))) return -1;
     const int Hk = H / G;
@@ -239,7 +252,7 @@ int or_select(int B, int H, int G, int d, int S, int K, double scale,
             const int g = (int)((u / Lq) % Hk);
             const int b = (int)(u / ((long long)Lq * Hk));
             const int t = qpos ? qpos[(long long)b * Lq + i] : i;
-            const int ne = eligible_chunks(t, S, C);
+            const int ne = eligible_chunks(t, S, C, excl_w);
             for (int hh = 0; hh < G; ++hh) load_vec(&Qcal, b, g * G + hh, i, d, q + (long long)hh * d);
             /* the group's selection score of chunk c: the largest of its heads' s^ */
             for (int c = 0; c < ne; ++c) {

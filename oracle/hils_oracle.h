@@ -54,8 +54,9 @@ int or_summarize(int B, int H, int G, int d, int S, double scale,
 /* Eq. 7 with the calibrated query (Methodology 2): the surrogate log-mass of every
  * chunk for every query. Qcal: [B,H,Lq,d]; Ksum: [B,H,C,d]; Bsum: [B,H,C] (x = 0).
  * qpos: [B, Lq] query positions t, or NULL for t = i. A chunk c is eligible for the
- * query at t when c < min(floor(t / S), C). out: [B,H,Lq,C]; ineligible = -inf. */
-int or_score_all(int B, int H, int d, int S, double scale,
+ * query at t when c < min(floor(t / S), C), and, when excl_w = W > 0 (the window
+ * exclusion), c * S < max(0, t - W + 1). out: [B,H,Lq,C]; ineligible = -inf. */
+int or_score_all(int B, int H, int d, int S, int excl_w, double scale,
                  or_tensor Qcal, int Lq, const int *qpos,
                  or_tensor Ksum, or_tensor Bsum, int C, double *out);
 
@@ -64,7 +65,7 @@ int or_score_all(int B, int H, int d, int S, double scale,
  * listed in ascending chunk index. idx: [B,H/G,Lq,K] int (-1 padding), nsel:
  * [B,H/G,Lq] = min(K, number of eligible chunks); score: [B,H,Lq,K] double, each
  * head's own score of the kept chunks (-inf padding). */
-int or_select(int B, int H, int G, int d, int S, int K, double scale,
+int or_select(int B, int H, int G, int d, int S, int K, int excl_w, double scale,
               or_tensor Qcal, int Lq, const int *qpos,
               or_tensor Ksum, or_tensor Bsum, int C,
               int *idx, double *score, int *nsel);
