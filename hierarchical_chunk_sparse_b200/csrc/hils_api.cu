@@ -60,7 +60,7 @@ int check_params(const hils_params *p, float *scale) {
     if (p->d != 64 && p->d != 128) return HILS_ERR_UNSUPPORTED;
     if (p->S != kChunk) return HILS_ERR_UNSUPPORTED;
     if (p->K > 32) return HILS_ERR_UNSUPPORTED;
-    if (p->flags != 0) return HILS_ERR_UNSUPPORTED;
+    if (p->flags & ~(uint32_t)HILS_FLAG_EXCLUDE_WINDOW_CHUNKS) return HILS_ERR_UNSUPPORTED;
     if (!isfinite(p->scale)) return HILS_ERR_INVALID_ARG;
     if (p->H_kv < 0 || (p->H_kv > 0 && p->H % p->H_kv != 0)) return HILS_ERR_INVALID_ARG;
     if (p->H_kv > 0 && p->H / p->H_kv > kMaxGroupHeads) return HILS_ERR_UNSUPPORTED;
@@ -149,6 +149,7 @@ int prepare_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_
     a->topk = p->K;
     a->scale = scale;
     a->G = groups(p);
+    a->excl_w = (p->flags & HILS_FLAG_EXCLUDE_WINDOW_CHUNKS) ? p->W : 0;
     if (nq > 0) select_plan(p->dtype, p->d, p->B, p->H, Lq, C, p->K, qpos != nullptr, device_sm_count(), a);
     return HILS_OK;
 }
@@ -203,7 +204,7 @@ const char *hils_status_string(int status) {
     switch (status) {
     case HILS_OK: return "ok";
     case HILS_ERR_INVALID_ARG: return "invalid argument";
-    case HILS_ERR_UNSUPPORTED: return "unsupported configuration (d in {64,128}, S = 64, K <= 32, flags = 0, H / H_kv <= 8)";
+    case HILS_ERR_UNSUPPORTED: return "unsupported configuration (d in {64,128}, S = 64, K <= 32, known flags, H / H_kv <= 8)";
     case HILS_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
     case HILS_ERR_WORKSPACE: return "workspace missing or too small";
     case HILS_ERR_CUDA: return "CUDA launch error";

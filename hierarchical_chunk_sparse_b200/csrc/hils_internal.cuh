@@ -47,6 +47,7 @@ struct SelectArgs {
     float scale;
     int path;              // SelectPath chosen by select_plan
     int G = 1;             // query heads per group: idx and nsel have H / G heads
+    int excl_w = 0;        // > 0: the window length; chunks wholly inside a query's window are not eligible
     // split search over chunk ranges (decode-like shapes)
     int ctas_per_query;    // summary blocks per query of the screen kernel
     int tiles_per_warp;    // 128-chunk tiles each warp scans

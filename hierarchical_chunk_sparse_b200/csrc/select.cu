@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(kWarpKernelThreads) select_group_kernel(Select
     if (qg >= (int64_t)a.B * (a.H / a.G) * a.Lq) return;
     int t, b, g, i;
     const GroupCtx q = make_group_ctx<T, D>(a, qg, t, b, g, i);
-    const int ne = eligible(t, a.C);
+    const int ne = eligible(t, a.C, a.excl_w);
     for (int hh = 0; hh < q.G; ++hh) load_query_f32<T, D>(head_ctx(q, hh, (int)sizeof(T)), qs_all[w] + hh * D);
     __syncwarp();
     warp_scan<T, D>(q, qs_all[w], 0, ne, a.topk, lists[w]);
@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kWarpKernelThreads) select_warp_kernel(SelectA
     if (qi >= nq) return;
     int t;
     const QueryCtx q = make_ctx<T, D>(a, qi, t);
-    const int ne = eligible(t, a.C);
+    const int ne = eligible(t, a.C, a.excl_w);
     load_query_f32<T, D>(q, qs_all[w]);
     __syncwarp();
     warp_scan<T, D>(q, qs_all[w], 0, ne, a.topk, lists[w]);
@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid
         const uint8_t *st = smem + stage * Cfg::kStageBytes;
         const int qu = item / nblk, blk = item - (item / nblk) * nblk;
         const int c0 = blk * kScrRows;
-        const int ne = eligible(*reinterpret_cast<const int *>(st + Cfg::kPosOff) + a.qpos_bias, a.C);
+        const int ne = eligible(*reinterpret_cast<const int *>(st + Cfg::kPosOff) + a.qpos_bias, a.C, a.excl_w);
         float2 *out = kFold ? tmp : ws.scr + (int64_t)qu * a.C;
         const int base = kFold ? c0 : 0;
         if (c0 < ne) {

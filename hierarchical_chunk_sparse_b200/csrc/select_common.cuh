@@ -322,9 +322,18 @@ __device__ __forceinline__ QueryCtx make_ctx(const SelectArgs &a, int64_t qi, in
     return q;
 }
 
-__device__ __forceinline__ int eligible(int t, int C) {
-    const int e = t >= 0 ? t / kChunk : 0;
-    return e < C ? e : C;
+// Chunks the query at position t may select: complete chunks before its own chunk,
+// capped by C; with the window exclusion (excl_w = W > 0) only those that start before
+// the window's first token max(0, t - W + 1), i.e. that do not lie wholly inside it.
+__device__ __forceinline__ int eligible(int t, int C, int excl_w) {
+    int e = t >= 0 ? t / kChunk : 0;
+    e = e < C ? e : C;
+    if (excl_w > 0 && t >= 0) {
+        const int w0 = t - excl_w + 1 > 0 ? t - excl_w + 1 : 0;
+        const int nw = (w0 + kChunk - 1) / kChunk;
+        e = e < nw ? e : nw;
+    }
+    return e;
 }
 
 template <typename T, int D>

@@ -192,7 +192,7 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
         if constexpr (kGroup) group_write<T, D>(q, ps.qs, list, a, u, b, grp, i);
         else warp_write(list, a.topk, u, a.idx, a.score, a.nsel);
     };
-    const int ne = eligible(t, a.C);
+    const int ne = eligible(t, a.C, a.excl_w);
     const int K = a.topk;
     if (ne <= K) {  // every eligible chunk is kept, in index order
         if constexpr (kGroup) {

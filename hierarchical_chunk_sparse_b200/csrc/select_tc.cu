@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
     const bool row_ok = i < a.Lq;
     int t = -1;
     if (row_ok) t = a.qpos ? a.qpos[(int64_t)b * a.Lq + i] + a.qpos_bias : i;
-    const int ne = row_ok ? eligible(t, a.C) : 0;
+    const int ne = row_ok ? eligible(t, a.C, a.excl_w) : 0;
     if (tid == 0) {
         misc->nc = 0;
         misc->knmax = 0u;
@@ -653,14 +653,14 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
                 const GroupCtx q = make_group_ctx<bf16, kHD>(a, qbase + row, tq, bb, gg, ii);
                 for (int hh = 0; hh < G; ++hh) load_query_f32<bf16, kHD>(head_ctx(q, hh, (int)sizeof(bf16)), qs + hh * kHD);
                 __syncwarp();
-                warp_scan<bf16, kHD>(q, qs, 0, eligible(tq, a.C), K, list);
+                warp_scan<bf16, kHD>(q, qs, 0, eligible(tq, a.C, a.excl_w), K, list);
                 group_write<bf16, kHD>(q, qs, list, a, qbase + row, bb, gg, ii);
             } else {
                 float *qs = reinterpret_cast<float *>(smem + kFbQ) + warp * kHD;
                 const QueryCtx q = make_ctx<bf16, kHD>(a, qbase + row, tq);
                 load_query_f32<bf16, kHD>(q, qs);
                 __syncwarp();
-                warp_scan<bf16, kHD>(q, qs, 0, eligible(tq, a.C), K, list);
+                warp_scan<bf16, kHD>(q, qs, 0, eligible(tq, a.C, a.excl_w), K, list);
                 warp_write(list, K, qbase + row, a.idx, a.score, a.nsel);
             }
             __syncwarp();

@@ -77,7 +77,7 @@ typedef enum { HILS_F32 = 0, HILS_BF16 = 1 } hils_dtype;
 typedef enum {
     HILS_OK = 0,
     HILS_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent shape */
-    HILS_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, S != 64, K > 32, flags != 0, H / H_kv > 8 */
+    HILS_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, S != 64, K > 32, unknown flags, H / H_kv > 8 */
     HILS_ERR_ALIGNMENT = 3,    /* pointer or stride not 16-byte aligned */
     HILS_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
     HILS_ERR_CUDA = 5          /* a kernel launch failed; see hils_last_cuda_error() */
@@ -94,6 +94,18 @@ typedef struct {
     int64_t sb, sh, st;
 } hils_tensor;
 
+/* Flags (hils_params.flags).
+ *   HILS_FLAG_EXCLUDE_WINDOW_CHUNKS: the window-exclusion variant. A chunk that lies
+ *     wholly inside the query's window [max(0, t-W+1), t] is not eligible for
+ *     selection (the window already attends its tokens exactly), so no token is
+ *     counted twice except in the chunk holding the window's first token when the
+ *     window starts inside a chunk (that chunk stays eligible, or its earlier tokens
+ *     would be reached by neither term). The pages' normaliser over the selected chunks
+ *     and the window (summary page, Methodology 2) does not say whether a token may be
+ *     counted in both; without the flag it may (the default). Only hils_select and
+ *     hils_decode read the flag; summaries and the attend calls are unchanged. */
+#define HILS_FLAG_EXCLUDE_WINDOW_CHUNKS 1u
+
 /* Problem description shared by every call.
  *   B      batch (sequences), H query heads,
  *   d      head dimension: 64 or 128,
@@ -102,7 +114,7 @@ typedef struct {
  *   W      sliding-window length in tokens: >= 0,
  *   dtype  element type of every Q/K/V/LQ/Ksum/O tensor,
  *   scale  softmax scale; 0 selects (float)(1/sqrt(d)),
- *   flags  reserved, must be 0,
+ *   flags  0, or HILS_FLAG_EXCLUDE_WINDOW_CHUNKS (below); other bits are rejected,
  *   H_kv   key-value heads: 0 (= H) or a divisor of H with H / H_kv <= 8; groups of
  *          G = H / H_kv query heads share a key-value head and their chunk selection
  *          (see above). */

@@ -58,7 +58,7 @@ def _summ(lib, p, K=None, N=256, LQ=None, Ksum=None, Bsum=ALIGNED):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(d=96), 2), (dict(S=32), 2), (dict(K=33), 2), (dict(flags=1), 2),
+    (dict(d=96), 2), (dict(S=32), 2), (dict(K=33), 2), (dict(flags=2), 2), (dict(flags=3), 2),
     (dict(B=-1), 1), (dict(W=-1), 1), (dict(K=-2), 1), (dict(scale=float("nan")), 1),
 ])
 def test_invalid_params_rejected(lib, kw, code):
@@ -181,3 +181,15 @@ def test_binding_rejects_mismatched_shapes():
         hils.hils_select(p2, Q.float(), Ksum, Bsum, idx, idx.float(), idx[..., 0])
     with pytest.raises(ValueError, match="CUDA"):
         hils.hils_select(p2, Q, Ksum, Bsum, idx, idx.float(), idx[..., 0])
+
+
+def test_window_exclusion_flag_accepted(lib):
+    """flags = HILS_FLAG_EXCLUDE_WINDOW_CHUNKS passes the parameter checks, other bits do
+    not (hils_workspace_bytes runs the checks and returns 0 on a rejection; it launches
+    nothing)."""
+    p = _p(B=1, H=2)
+    c = p.c()
+    c.flags = hils.HILS_FLAG_EXCLUDE_WINDOW_CHUNKS
+    assert lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_SELECT, 1, 8000) > 0
+    c.flags = 2
+    assert lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_SELECT, 1, 8000) == 0
