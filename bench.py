@@ -292,7 +292,7 @@ def prefill_flops(w, part: str = "step") -> float:
 # measured for the current kernels, each with its command in profiles/: select_decode512k.md
 # (screen + pick of one select call), attend_decode_128k.md, attend_prefill_tc_prefill8k.md.
 # A kernel that changes after its capture reports null here until it is captured again.
-MEASURED_TRAFFIC = {"select": 69_358_080, "attend_decode": 25_235_968, "attend_prefill": 661_831_680}
+MEASURED_TRAFFIC = {"select": 69_647_616, "attend_decode": 25_235_968, "attend_prefill": 661_831_680}
 
 
 class PrefillBench:
