@@ -66,6 +66,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib = ctypes.CDLL(path)
         T, P, vp, i, sz = _CTensor, ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         lib.hils_summarize.argtypes = [P, T, i, T, T, vp, vp]
+        lib.hils_summarize_append.argtypes = [P, T, vp, T, T, vp, i, vp]
         lib.hils_select.argtypes = [P, T, i, vp, T, vp, i, vp, vp, vp, vp, sz, vp]
         lib.hils_attend_prefill.argtypes = [P, T, T, T, i, vp, vp, vp, T, vp, vp, sz, vp]
         lib.hils_attend_decode.argtypes = [P, T, T, T, vp, vp, vp, vp, T, vp, vp, sz, vp]
@@ -77,7 +78,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hils_status_string.argtypes = [i]
         lib.hils_status_string.restype = ctypes.c_char_p
         lib.hils_last_cuda_error.restype = ctypes.c_char_p
-        for name in ("hils_summarize", "hils_select", "hils_attend_prefill", "hils_attend_decode", "hils_decode",
+        for name in ("hils_summarize", "hils_summarize_append", "hils_select", "hils_attend_prefill", "hils_attend_decode", "hils_decode",
                      "hils_attend_decode_noalloc", "hils_workspace_init"):
             getattr(lib, name).restype = i
         _lib = lib
@@ -181,6 +182,25 @@ def hils_summarize(p: Params, K, LQ, Ksum, Bsum, N: int | None = None, stream=No
     _expect("hils_summarize", "Bsum", Bsum, (B, H, C), torch.float32)
     _check("hils_summarize", load_library().hils_summarize(
         ctypes.byref(p.c()), _view(K), n, _view(LQ), _view(Ksum), _ptr(Bsum), _stream(stream)))
+
+
+def hils_summarize_append(p: Params, K, cache_len, LQ, Ksum, Bsum, stream=None) -> None:
+    """Decode-time summary of the chunk each sequence's newest token completed: for b
+    with cache_len[b] a positive multiple of 64, chunk cache_len[b] / 64 - 1 of every
+    head into Ksum [B,H,C,d] and Bsum [B,H,C]; everything else is left as it was.
+    K [B,Hk,T,d] is the KV cache's keys, LQ [B,H,C,d] the landmark queries."""
+    B, H, d = p.B, p.H, p.d
+    C = Ksum.shape[2]
+    if K.shape[0] != B or K.shape[1] != p.Hk or K.shape[3] != d or K.dtype != p.dtype or not K.is_cuda:
+        raise ValueError(f"hils_summarize_append: K has shape {tuple(K.shape)} / {K.dtype}")
+    if K.shape[2] < C * p.S:
+        raise ValueError("hils_summarize_append: the cache holds fewer than C chunks")
+    _expect("hils_summarize_append", "cache_len", cache_len, (B,), torch.int32)
+    _expect("hils_summarize_append", "LQ", LQ, (B, H, C, d), p.dtype)
+    _expect("hils_summarize_append", "Ksum", Ksum, (B, H, C, d), p.dtype)
+    _expect("hils_summarize_append", "Bsum", Bsum, (B, H, C), torch.float32)
+    _check("hils_summarize_append", load_library().hils_summarize_append(
+        ctypes.byref(p.c()), _view(K), _ptr(cache_len), _view(LQ), _view(Ksum), _ptr(Bsum), C, _stream(stream)))
 
 
 def hils_select(p: Params, Qcal, Ksum, Bsum, idx, score, nsel, qpos=None, workspace=None,

@@ -257,6 +257,31 @@ int hils_summarize(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ,
     return launch_summarize(p->dtype, p->d, a, stream);
 }
 
+int hils_summarize_append(const hils_params *p, hils_ctensor K, const int32_t *cache_len, hils_ctensor LQ,
+                          hils_tensor Ksum, float *Bsum, int C, cudaStream_t stream) {
+    float scale;
+    HILS_TRY(check_params(p, &scale));
+    if (C < 0) return HILS_ERR_INVALID_ARG;
+    if ((int64_t)p->B * p->H * C > 0xffffffffll) return HILS_ERR_INVALID_ARG;
+    HILS_TRY(check_view(K.ptr, K.sb, K.sh, K.st, (int64_t)C * kChunk, p));
+    HILS_TRY(check_view(LQ.ptr, LQ.sb, LQ.sh, LQ.st, C, p));
+    HILS_TRY(check_view(Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st, C, p));
+    HILS_TRY(check_array(Bsum, (int64_t)p->B * p->H * C));
+    HILS_TRY(check_array(cache_len, C > 0 ? p->B : 0));
+    SummarizeArgs a;
+    a.K = {K.ptr, K.sb, K.sh, K.st};
+    a.LQ = {LQ.ptr, LQ.sb, LQ.sh, LQ.st};
+    a.Ksum = {Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st};
+    a.Bsum = Bsum;
+    a.B = p->B;
+    a.H = p->H;
+    a.C = C;
+    a.scale = scale;
+    a.G = groups(p);
+    a.cache_len = cache_len;
+    return launch_summarize(p->dtype, p->d, a, stream);
+}
+
 int hils_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *qpos, hils_ctensor Ksum,
                 const float *Bsum, int C, int32_t *idx, float *score, int32_t *nsel, void *workspace,
                 size_t ws_bytes, cudaStream_t stream) {

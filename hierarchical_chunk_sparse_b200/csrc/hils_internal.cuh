@@ -33,6 +33,7 @@ struct SummarizeArgs {
     int B, H, C;
     float scale;
     int G = 1;             // query heads per key-value head: K has H / G heads
+    const int32_t *cache_len = nullptr;  // non-null: only the chunk each sequence's newest token completed
 };
 
 struct SelectArgs {

@@ -12,6 +12,10 @@
 // cp.async copies, three chunks in flight per CTA. Logits use two threads per key
 // row; the landmark softmax runs in one warp; the weighted key sum gives each
 // thread two adjacent columns over a quarter or half of the rows.
+//
+// Decode-time (incremental) form, with cache_len: one unit per (b, h); the unit is the
+// chunk that sequence b's newest token completed (cache_len[b] a positive multiple of
+// 64), or nothing. The same per-chunk arithmetic writes the same bits as the full pass.
 #include "hils_internal.cuh"
 
 namespace hils {
@@ -49,13 +53,25 @@ __global__ void __launch_bounds__(128) summarize_kernel(SummarizeArgs a) {
     float *red = prob + kChunk;
 
     const int tid = threadIdx.x;
-    const unsigned total = (unsigned)a.B * a.H * a.C;  // chunk count is checked to fit
+    // units: every (b, h, chunk), or with cache_len one per (b, h)
+    const unsigned total = a.cache_len ? (unsigned)a.B * a.H : (unsigned)a.B * a.H * a.C;  // checked to fit
     const unsigned stride = gridDim.x;
+    // the unit's (b, h) and chunk; chunk -1: nothing to summarise
+    auto unit_chunk = [&](unsigned u, int &bh, int &c) {
+        if (a.cache_len) {
+            bh = (int)u;
+            const int L = a.cache_len[bh / a.H];
+            c = (L >= kChunk && L % kChunk == 0 && L / kChunk <= a.C) ? L / kChunk - 1 : -1;
+        } else {
+            c = (int)(u % (unsigned)a.C);
+            bh = (int)(u / (unsigned)a.C);
+        }
+    };
 
     auto issue = [&](unsigned u, int stage) {
-        if (u < total) {
-            const int c = (int)(u % (unsigned)a.C);
-            const int bh = (int)(u / (unsigned)a.C);
+        int c = -1, bh = 0;
+        if (u < total) unit_chunk(u, bh, c);
+        if (c >= 0) {
             const int h = bh % a.H;
             const int b = bh / a.H;
             const T *k0 = static_cast<const T *>(a.K.ptr) + b * a.K.sb + (h / a.G) * a.K.sh +
@@ -81,6 +97,9 @@ __global__ void __launch_bounds__(128) summarize_kernel(SummarizeArgs a) {
         __syncthreads();
 
         const uint8_t *tile = smem + stage * Cfg::kStageBytes;
+        int ubh, uc;
+        unit_chunk(u, ubh, uc);
+        if (uc >= 0) {  // uniform over the CTA
         // landmark logits, two threads per key row
         {
             const int row = tid >> 1, half = tid & 1;
@@ -107,7 +126,7 @@ __global__ void __launch_bounds__(128) summarize_kernel(SummarizeArgs a) {
             prob[tid] = p0;
             prob[tid + 32] = p1;
             const float ent = warp_sum(p0 * (lz - (l0 - m)) + p1 * (lz - (l1 - m)));
-            if (tid == 0) a.Bsum[u] = ent;
+            if (tid == 0) a.Bsum[(int64_t)ubh * a.C + uc] = ent;
         }
         __syncthreads();
         // k'_c = sum_j p_j k_j: thread owns columns 2*cu, 2*cu+1 over rows rg, rg+G, ...
@@ -130,13 +149,12 @@ __global__ void __launch_bounds__(128) summarize_kernel(SummarizeArgs a) {
                     a0 += red[g * D + 2 * cu];
                     a1 += red[g * D + 2 * cu + 1];
                 }
-                const int c = (int)(u % (unsigned)a.C);
-                const int bh = (int)(u / (unsigned)a.C);
-                const int h = bh % a.H;
-                const int b = bh / a.H;
-                T *out = static_cast<T *>(a.Ksum.ptr) + b * a.Ksum.sb + h * a.Ksum.sh + c * a.Ksum.st;
+                const int h = ubh % a.H;
+                const int b = ubh / a.H;
+                T *out = static_cast<T *>(a.Ksum.ptr) + b * a.Ksum.sb + h * a.Ksum.sh + uc * a.Ksum.st;
                 store2(out + 2 * cu, a0, a1);
             }
+        }
         }
         __syncthreads();
         stage = (stage + 1) % Cfg::kStages;
@@ -147,8 +165,8 @@ __global__ void __launch_bounds__(128) summarize_kernel(SummarizeArgs a) {
 template <typename T, int D>
 hils_status launch(const SummarizeArgs &a, cudaStream_t s) {
     using Cfg = SumCfg<T, D>;
-    const int64_t total = (int64_t)a.B * a.H * a.C;
-    if (total == 0) return HILS_OK;
+    const int64_t total = a.cache_len ? (int64_t)a.B * a.H : (int64_t)a.B * a.H * a.C;
+    if (total == 0 || a.C == 0) return HILS_OK;
     static KernelSetup setup;
     int per_sm = 1;
     const hils_status st = kernel_setup(setup, (const void *)summarize_kernel<T, D>, Cfg::kThreads,

@@ -148,6 +148,21 @@ typedef enum {
 int hils_summarize(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ,
                    hils_tensor Ksum, float *Bsum, cudaStream_t stream);
 
+/* Decode-time summary of the chunk each sequence's newest token completed (the same
+ * Eq. 8 arithmetic, and the same bits, as hils_summarize): for every b whose
+ * cache_len[b] is a positive multiple of S with cache_len[b] / S <= C, chunk
+ * c = cache_len[b] / S - 1 of every head h is summarised into Ksum[b, h, c] and
+ * Bsum[b, h, c]; every other entry of Ksum and Bsum, and every other sequence, is left
+ * as it was. Run after appending a token and before the next decode step's selection:
+ * the chunk becomes eligible for the query at position cache_len[b].
+ *   K          [B, Hk, T, d] the KV cache's keys, T >= cache_len[b]
+ *   cache_len  [B] int32, device
+ *   LQ         [B, H, C, d] landmark queries
+ *   Ksum, Bsum [B, H, C, d] / [B, H, C] the summary table (capacity C chunks)
+ * Returns HILS_OK, or an error before any launch. */
+int hils_summarize_append(const hils_params *p, hils_ctensor K, const int32_t *cache_len, hils_ctensor LQ,
+                          hils_tensor Ksum, float *Bsum, int C, cudaStream_t stream);
+
 /* Chunk scores and top-K (summary page, Eq. 7 and Methodology 2; post, pseudocode).
  * For every query i at position t_i, every eligible chunk c < min(floor(t_i/S), C) gets
  *   s^_{i,c} = scale * (q~_i . k'_c) + b'_c,

@@ -656,3 +656,34 @@ def test_screen_radius_covers_the_float64_score(oracle, cuda_device, d):
     assert (err / tc).max() <= 1 / 16, f"observed error {float((err / tc).max()):.3f} of the bound"
     i_ref, s_ref, n_ref = oracle.select(Q, Ksum, Bsum, 64, w.K, w.scale, qpos=qpos)
     assert_same_selection(idx, nsel, i_ref, n_ref)
+
+
+@pytest.mark.parametrize("cfg,Hk,dtype,d", [(4, 0, torch.bfloat16, 128), (8, 2, torch.bfloat16, 128),
+                                             (4, 0, torch.float32, 64)])
+def test_summarize_append_decode_time(oracle, cuda_device, cfg, Hk, dtype, d):
+    """hils_summarize_append summarises exactly the chunk each sequence's newest token
+    completed (cache_len a positive multiple of 64), with the bits of the full pass, and
+    leaves every other entry of the table untouched."""
+    w = WORKLOADS[cfg].replace(B=5, H=4, Hk=Hk, d=d, dtype=dtype, N=64 * 40, needles=0)
+    inp = make_decode(w)
+    dv = to_dev(inp, cuda_device)
+    Ksum_full, Bsum_full = gpu_summarize(w, dv["K"], dv["LQ"])
+    lens = [64 * 17, 64 * 17 + 5, 64, 1, 64 * 40]
+    cache_len = torch.tensor(lens, dtype=torch.int32, device=cuda_device)
+    Ksum = torch.full_like(Ksum_full, 7.0)
+    Bsum = torch.full_like(Bsum_full, 99.0)
+    hils.hils_summarize_append(P(w), dv["K"], cache_len, dv["LQ"], Ksum, Bsum)
+    torch.cuda.synchronize()
+    done = {b: L // 64 - 1 for b, L in enumerate(lens) if L >= 64 and L % 64 == 0}
+    assert done == {0: 16, 2: 0, 4: 39}
+    for b in range(w.B):
+        for c in range(w.C):
+            if done.get(b) == c:
+                assert torch.equal(Ksum[b, :, c], Ksum_full[b, :, c]), (b, c)
+                assert torch.equal(Bsum[b, :, c], Bsum_full[b, :, c]), (b, c)
+            else:
+                assert (Ksum[b, :, c] == 7.0).all() and (Bsum[b, :, c] == 99.0).all(), (b, c)
+    # the appended chunk of sequence 0 against the oracle
+    ks_ref, bs_ref = oracle.summarize(inp["K"][:1, :, : 64 * 17], inp["LQ"][:1, :, :17], 64, w.scale)
+    assert_close(Ksum[:1, :, 16], ks_ref[:, :, 16], dtype, "Ksum")
+    assert np.abs(host(Bsum[:1, :, 16]).double().numpy() - bs_ref[:, :, 16]).max() <= BSUM_ATOL
