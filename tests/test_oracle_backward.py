@@ -1,0 +1,127 @@
+"""Pins of the backward oracle (``oracle/backward.py``): its forward against the pinned C
+oracle, and its autograd gradients against central finite differences (float64
+``torch.autograd.gradcheck``), for multi-head and grouped heads, with and without a
+window, so that a wrong term of the backward cannot pass."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import backward as ob
+
+S = 64
+
+
+def _rand(*shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(*shape, generator=g, dtype=torch.float64) * scale)
+
+
+def _selection(B, Hk, N, K, seed):
+    """A random valid selection: for query i, K distinct eligible chunks (c < i // 64)."""
+    g = np.random.default_rng(seed)
+    idx = np.full((B, Hk, N, K), -1, np.int32)
+    nsel = np.zeros((B, Hk, N), np.int32)
+    for b in range(B):
+        for h in range(Hk):
+            for i in range(N):
+                ne = i // S
+                n = min(K, ne)
+                if n:
+                    idx[b, h, i, :n] = np.sort(g.choice(ne, n, replace=False))
+                nsel[b, h, i] = n
+    return idx, nsel
+
+
+def _problem(B=1, H=2, G=1, N=64 * 4 + 9, d=8, K=2, seed=0):
+    Hk = H // G
+    C = N // S
+    Q = _rand(B, H, N, d, seed=seed + 1, scale=0.6)
+    Kc = _rand(B, Hk, N, d, seed=seed + 2, scale=0.6)
+    Vc = _rand(B, Hk, N, d, seed=seed + 3)
+    Qcal = _rand(B, H, N, d, seed=seed + 4, scale=0.6)
+    LQ = _rand(B, H, C, d, seed=seed + 5, scale=0.6)
+    idx, nsel = _selection(B, Hk, N, K, seed + 6)
+    return Q, Kc, Vc, Qcal, LQ, idx, nsel
+
+
+@pytest.mark.parametrize("G,W", [(1, 40), (2, 70), (1, 0)])
+def test_forward_matches_the_c_oracle(G, W):
+    Q, Kc, Vc, Qcal, LQ, idx, nsel = _problem(H=4, G=G, N=64 * 5 + 17, d=16, K=3, seed=10)
+    O, lse, score, Ksum, Bsum = ob.forward(Q, Kc, Vc, Qcal, LQ, idx, nsel, S, W, 0.3)
+    ks, bs = oracle.summarize(Kc, LQ, S, 0.3)
+    assert np.abs(Ksum.numpy() - ks).max() < 1e-12 and np.abs(Bsum.numpy() - bs).max() < 1e-12
+    sall = oracle.score_all(Qcal, torch.from_numpy(ks), torch.from_numpy(bs), S, 0.3)
+    Hk = Kc.shape[1]
+    for h in range(4):
+        for i in range(Q.shape[2]):
+            n = nsel[0, h // G, i]
+            cs = idx[0, h // G, i, :n]
+            if n:
+                assert np.abs(score[0, h, i, :n].numpy() - sall[0, h, i, cs]).max() < 1e-12
+            assert np.isneginf(score[0, h, i, n:].numpy()).all()
+    O_ref, lse_ref = oracle.attend(Q, Kc, Vc, idx, score.numpy(), nsel, S, W, 0.3)
+    assert np.abs(O.numpy() - O_ref).max() < 1e-12
+    fin = np.isfinite(lse_ref)
+    assert (np.isfinite(lse.numpy()) == fin).all()
+    assert np.abs(lse.numpy()[fin] - lse_ref[fin]).max() < 1e-12
+    assert Hk * G == 4
+
+
+@pytest.mark.parametrize("G,W", [(1, 30), (2, 70), (1, 0)])
+def test_gradients_match_finite_differences(G, W):
+    """float64 gradcheck of every input's gradient (central differences, eps 1e-6; the
+    fast mode checks the gradients along random directions of every input)."""
+    Q, Kc, Vc, Qcal, LQ, idx, nsel = _problem(H=2, G=G, N=64 * 3 + 5, d=4, K=2, seed=20 + G)
+    dO = _rand(*Q.shape, seed=99)
+
+    def f(q, k, v, qc, lq):
+        O, _, _, _, _ = ob.forward(q, k, v, qc, lq, idx, nsel, S, W, 0.4)
+        return (O * dO).sum()
+
+    ins = [x.clone().requires_grad_(True) for x in (Q, Kc, Vc, Qcal, LQ)]
+    assert torch.autograd.gradcheck(f, ins, eps=1e-6, atol=1e-7, rtol=1e-5, fast_mode=True)
+    # the grads() wrapper returns the same gradients
+    g = ob.grads(Q, Kc, Vc, Qcal, LQ, idx, nsel, dO, S, W, 0.4)
+    auto = torch.autograd.grad(f(*ins), ins)
+    for name, a in zip(("dQ", "dK", "dV", "dQcal", "dLQ"), auto):
+        assert torch.allclose(g[name], a, atol=1e-14, rtol=0), name
+
+
+def test_intermediate_gradients_by_the_chain_rule():
+    """dscore, dKsum, dBsum against their closed forms from the other gradients:
+    dQcal = scale sum_k dscore_k k'_{c_k}; dBsum_c = sum over the queries that kept c
+    of dscore; dKsum_c = scale sum of dscore q~."""
+    Q, Kc, Vc, Qcal, LQ, idx, nsel = _problem(H=2, G=1, N=64 * 4 + 3, d=8, K=3, seed=30)
+    dO = _rand(*Q.shape, seed=31)
+    g = ob.grads(Q, Kc, Vc, Qcal, LQ, idx, nsel, dO, S, 50, 0.35)
+    _, _, _, Ksum, Bsum = ob.forward(Q, Kc, Vc, Qcal, LQ, idx, nsel, S, 50, 0.35)
+    B, H, N, d = Q.shape
+    dq = torch.zeros_like(Qcal)
+    dks = torch.zeros_like(Ksum)
+    dbs = torch.zeros_like(Bsum)
+    for h in range(H):
+        for i in range(N):
+            for k in range(int(nsel[0, h, i])):
+                c = int(idx[0, h, i, k])
+                ds = g["dscore"][0, h, i, k]
+                dq[0, h, i] += 0.35 * ds * Ksum[0, h, c].detach()
+                dks[0, h, c] += 0.35 * ds * Qcal[0, h, i]
+                dbs[0, h, c] += ds
+    assert torch.allclose(g["dQcal"], dq, atol=1e-12)
+    assert torch.allclose(g["dKsum"], dks, atol=1e-12)
+    assert torch.allclose(g["dBsum"], dbs, atol=1e-12)
+
+
+def test_gradients_match_finite_differences_elementwise():
+    """The full (element by element) float64 gradcheck on a small case: two chunks, a
+    window crossing a chunk boundary, two query heads sharing a key-value head."""
+    Q, Kc, Vc, Qcal, LQ, idx, nsel = _problem(H=2, G=2, N=64 * 2 + 7, d=2, K=1, seed=40)
+    dO = _rand(*Q.shape, seed=41)
+
+    def f(q, k, v, qc, lq):
+        O, _, _, _, _ = ob.forward(q, k, v, qc, lq, idx, nsel, S, 20, 0.5)
+        return (O * dO).sum()
+
+    ins = [x.clone().requires_grad_(True) for x in (Q, Kc, Vc, Qcal, LQ)]
+    assert torch.autograd.gradcheck(f, ins, eps=1e-6, atol=1e-7, rtol=1e-5)
