@@ -544,6 +544,61 @@ def measure_prefill(wp, dev, stream, flush, args, world, peaks, peak_src, traffi
     return out
 
 
+def backward_flops(w) -> float:
+    """Algorithmic flops of the backward pass for the kept chunks and window of every
+    query (recomputed logits, dO.v, and the dq, dk, dv products: 10 d per query-token),
+    the score backward (4 d per kept chunk) and the summaries' backward (8 d per chunk
+    token): per batch."""
+    d, S, K, W, N, C = w.d, w.S, w.K, w.W, w.N, w.C
+    tok = sel = 0
+    for i in range(N):
+        e = min(i // S, C)
+        tok += S * min(K, e) + min(W, i + 1)
+        sel += min(K, e)
+    return float(w.B * w.H * (10 * d * tok + 4 * d * sel + 8 * d * S * C))
+
+
+def measure_prefill_backward(w, dev, stream, flush, args, world):
+    """The three backward calls of the 8K prefill for the forward's selection (L2
+    flushed before each timed pass; the accumulated gradients are zeroed inside it)."""
+    import hierarchical_chunk_sparse_b200 as hils
+
+    pb = PrefillBench(w, dev)
+    pb.step()
+    torch.cuda.synchronize()
+    B, H, N, d, Hk, K, C = w.B, w.H, w.N, w.d, w.Hkv, w.K, w.C
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = torch.Generator(device=dev).manual_seed(3)
+    dO = torch.randn(B, H, N, d, generator=g, **f32)
+    dQ, dK, dV = torch.empty(B, H, N, d, **f32), torch.zeros(B, Hk, N, d, **f32), torch.zeros(B, Hk, N, d, **f32)
+    dscore, dQcal = torch.empty(B, H, N, K, **f32), torch.empty(B, H, N, d, **f32)
+    dKsum, dBsum, dLQ = torch.zeros(B, H, C, d, **f32), torch.zeros(B, H, C, **f32), torch.empty(B, H, C, d, **f32)
+    i = pb.inp
+
+    def bwd():
+        for t in (dK, dV, dKsum, dBsum):
+            t.zero_()
+        hils.hils_attend_prefill_backward(pb.p, i["Q"], i["K"], i["V"], pb.idx, pb.score, pb.nsel, pb.O, pb.lse, dO,
+                                          dQ, dK, dV, dscore)
+        hils.hils_select_backward(pb.p, i["Qcal"], pb.Ksum, pb.idx, pb.nsel, dscore, dQcal, dKsum, dBsum)
+        hils.hils_summarize_backward(pb.p, i["K"], i["LQ"], dKsum, dBsum, dK, dLQ)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            bwd()
+    stream.synchronize()
+    n = 3
+    ms = statistics.mean(time_steps(bwd, n, flush, stream))
+    ms = max_over_ranks(ms, world, dev)
+    fl = backward_flops(w)
+    out = {"ms_per_step": ms, "unit": "TFLOP/s", "value": fl / (ms * 1e-3) / 1e12 * world, "workload": w.name,
+           "algorithmic_gflop_per_step": fl / 1e9, "steps": n,
+           "note": "first version: CUDA-core kernels, float32 atomic accumulation of dK, dV, dKsum, dBsum"}
+    del pb
+    torch.cuda.empty_cache()
+    return out
+
+
 def measure_decode(w, dev, stream, flush, args, world, peaks):
     """A secondary decode workload: hils_decode step time and its select and attend
     kernels (L2 flushed), tokens/s and algorithmic GB/s."""
@@ -664,6 +719,8 @@ def main():
         prefill_gqa = measure_prefill(WORKLOADS[7], dev, stream, flush, args, world, peaks, peak_src, None)
     # ---------------- grouped-query decode @512K (32 query heads, 8 key-value heads)
     decode_gqa = measure_decode(WORKLOADS[8], dev, stream, flush, args, world, peaks)
+    # ---------------- backward of the 8K prefill (fixed selection)
+    prefill_bwd = None if args.no_prefill else measure_prefill_backward(WORKLOADS[2], dev, stream, flush, args, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -693,6 +750,7 @@ def main():
             "prefill_local": prefill_local,
             "prefill_gqa": prefill_gqa,
             "decode_gqa": decode_gqa,
+            "prefill_backward": prefill_bwd,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

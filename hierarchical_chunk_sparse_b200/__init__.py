@@ -67,6 +67,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         T, P, vp, i, sz = _CTensor, ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         lib.hils_summarize.argtypes = [P, T, i, T, T, vp, vp]
         lib.hils_summarize_append.argtypes = [P, T, vp, T, T, vp, i, vp]
+        lib.hils_attend_prefill_backward.argtypes = [P, T, T, T, i, vp, vp, vp, T, vp, vp, vp, vp, vp, vp, vp]
+        lib.hils_select_backward.argtypes = [P, T, i, T, i, vp, vp, vp, vp, vp, vp, vp]
+        lib.hils_summarize_backward.argtypes = [P, T, i, T, vp, vp, vp, vp, vp]
         lib.hils_select.argtypes = [P, T, i, vp, T, vp, i, vp, vp, vp, vp, sz, vp]
         lib.hils_attend_prefill.argtypes = [P, T, T, T, i, vp, vp, vp, T, vp, vp, sz, vp]
         lib.hils_attend_decode.argtypes = [P, T, T, T, vp, vp, vp, vp, T, vp, vp, sz, vp]
@@ -78,7 +81,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hils_status_string.argtypes = [i]
         lib.hils_status_string.restype = ctypes.c_char_p
         lib.hils_last_cuda_error.restype = ctypes.c_char_p
-        for name in ("hils_summarize", "hils_summarize_append", "hils_select", "hils_attend_prefill", "hils_attend_decode", "hils_decode",
+        for name in ("hils_summarize", "hils_summarize_append", "hils_attend_prefill_backward",
+                     "hils_select_backward", "hils_summarize_backward", "hils_select", "hils_attend_prefill", "hils_attend_decode", "hils_decode",
                      "hils_attend_decode_noalloc", "hils_workspace_init"):
             getattr(lib, name).restype = i
         _lib = lib
@@ -313,6 +317,70 @@ def hils_attend_decode_noalloc(p: Params, Q, Kc, Vc, cache_len, idx, score, nsel
     _check("hils_attend_decode_noalloc", load_library().hils_attend_decode_noalloc(
         ctypes.byref(p.c()), _view(Q), _view(Kc), _view(Vc), _ptr(cache_len), _ptr(idx), _ptr(score),
         _ptr(nsel), _view(O), _ptr(lse), _stream(stream)))
+
+
+def _dense32(call: str, name: str, t, shape) -> None:
+    _expect(call, name, t, shape, torch.float32)
+    if not t.is_contiguous():
+        raise ValueError(f"{call}: {name} must be dense (contiguous)")
+
+
+def hils_attend_prefill_backward(p: Params, Q, K, V, idx, score, nsel, O, lse, dO, dQ, dK, dV, dscore,
+                                 stream=None) -> None:
+    """Eq. 10 backward for the kept chunks of hils_select: dQ [B,H,N,d] (written),
+    dK, dV [B,Hk,N,d] (accumulated: zero them first), dscore [B,H,N,K] (written); all
+    float32 and dense. O, lse are the forward's outputs, dO [B,H,N,d] float32."""
+    n = Q.shape[2]
+    B, H, d, k, Hk = p.B, p.H, p.d, p.K, p.Hk
+    for name, t, h in (("Q", Q, H), ("K", K, Hk), ("V", V, Hk), ("O", O, H)):
+        _expect("hils_attend_prefill_backward", name, t, (B, h, n, d), p.dtype)
+    if k > 0:
+        _expect("hils_attend_prefill_backward", "idx", idx, (B, Hk, n, k), torch.int32)
+        _expect("hils_attend_prefill_backward", "score", score, (B, H, n, k), torch.float32)
+        _expect("hils_attend_prefill_backward", "nsel", nsel, (B, Hk, n), torch.int32)
+        _dense32("hils_attend_prefill_backward", "dscore", dscore, (B, H, n, k))
+    _expect("hils_attend_prefill_backward", "lse", lse, (B, H, n), torch.float32)
+    for name, t, h in (("dO", dO, H), ("dQ", dQ, H), ("dK", dK, Hk), ("dV", dV, Hk)):
+        _dense32("hils_attend_prefill_backward", name, t, (B, h, n, d))
+    _check("hils_attend_prefill_backward", load_library().hils_attend_prefill_backward(
+        ctypes.byref(p.c()), _view(Q), _view(K), _view(V), n, _ptr(idx), _ptr(score), _ptr(nsel), _view(O),
+        _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dscore), _stream(stream)))
+
+
+def hils_select_backward(p: Params, Qcal, Ksum, idx, nsel, dscore, dQcal, dKsum, dBsum, stream=None) -> None:
+    """Eq. 7 backward: dQcal [B,H,Lq,d] (written), dKsum [B,H,C,d] and dBsum [B,H,C]
+    (accumulated), float32 and dense, from dscore [B,H,Lq,K]."""
+    lq, c = Qcal.shape[2], Ksum.shape[2]
+    B, H, d, k, Hk = p.B, p.H, p.d, p.K, p.Hk
+    _expect("hils_select_backward", "Qcal", Qcal, (B, H, lq, d), p.dtype)
+    _expect("hils_select_backward", "Ksum", Ksum, (B, H, c, d), p.dtype)
+    _expect("hils_select_backward", "idx", idx, (B, Hk, lq, k), torch.int32)
+    _expect("hils_select_backward", "nsel", nsel, (B, Hk, lq), torch.int32)
+    _dense32("hils_select_backward", "dscore", dscore, (B, H, lq, k))
+    _dense32("hils_select_backward", "dQcal", dQcal, (B, H, lq, d))
+    _dense32("hils_select_backward", "dKsum", dKsum, (B, H, c, d))
+    _dense32("hils_select_backward", "dBsum", dBsum, (B, H, c))
+    _check("hils_select_backward", load_library().hils_select_backward(
+        ctypes.byref(p.c()), _view(Qcal), lq, _view(Ksum), c, _ptr(idx), _ptr(nsel), _ptr(dscore), _ptr(dQcal),
+        _ptr(dKsum), _ptr(dBsum), _stream(stream)))
+
+
+def hils_summarize_backward(p: Params, K, LQ, dKsum, dBsum, dK, dLQ, N: int | None = None, stream=None) -> None:
+    """Eq. 8 backward over the complete chunks: dLQ [B,H,C,d] (written), dK [B,Hk,N,d]
+    (accumulated), float32 and dense, from dKsum [B,H,C,d] and dBsum [B,H,C]."""
+    n = K.shape[2] if N is None else N
+    B, H, d, Hk = p.B, p.H, p.d, p.Hk
+    C = n // p.S
+    if K.shape[0] != B or K.shape[1] != Hk or K.shape[3] != d or K.shape[2] < n or K.dtype != p.dtype:
+        raise ValueError(f"hils_summarize_backward: K has shape {tuple(K.shape)}")
+    _expect("hils_summarize_backward", "LQ", LQ, (B, H, C, d), p.dtype)
+    _dense32("hils_summarize_backward", "dKsum", dKsum, (B, H, C, d))
+    _dense32("hils_summarize_backward", "dBsum", dBsum, (B, H, C))
+    _dense32("hils_summarize_backward", "dK", dK, (B, Hk, n, d))
+    _dense32("hils_summarize_backward", "dLQ", dLQ, (B, H, C, d))
+    _check("hils_summarize_backward", load_library().hils_summarize_backward(
+        ctypes.byref(p.c()), _view(K), n, _view(LQ), _ptr(dKsum), _ptr(dBsum), _ptr(dK), _ptr(dLQ),
+        _stream(stream)))
 
 
 def alloc_workspace(p: Params, call: int, Lq: int, C: int, device="cuda") -> torch.Tensor | None:

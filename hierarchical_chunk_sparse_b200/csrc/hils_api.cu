@@ -282,6 +282,117 @@ int hils_summarize_append(const hils_params *p, hils_ctensor K, const int32_t *c
     return launch_summarize(p->dtype, p->d, a, stream);
 }
 
+int hils_attend_prefill_backward(const hils_params *p, hils_ctensor Q, hils_ctensor K, hils_ctensor V, int N,
+                                 const int32_t *idx, const float *score, const int32_t *nsel, hils_ctensor O,
+                                 const float *lse, const float *dO, float *dQ, float *dK, float *dV, float *dscore,
+                                 cudaStream_t stream) {
+    float scale;
+    HILS_TRY(check_params(p, &scale));
+    if (N < 0) return HILS_ERR_INVALID_ARG;
+    const int64_t nq = (int64_t)p->B * p->H * N;
+    if (nq > 0x7fffffffll) return HILS_ERR_INVALID_ARG;
+    const int64_t nkv = (int64_t)p->B * (p->H / groups(p)) * N * p->d;
+    HILS_TRY(check_view(Q.ptr, Q.sb, Q.sh, Q.st, N, p));
+    HILS_TRY(check_view(K.ptr, K.sb, K.sh, K.st, N, p));
+    HILS_TRY(check_view(V.ptr, V.sb, V.sh, V.st, N, p));
+    HILS_TRY(check_view(O.ptr, O.sb, O.sh, O.st, N, p));
+    HILS_TRY(check_array(idx, nq / groups(p) * p->K));
+    HILS_TRY(check_array(score, nq * p->K));
+    HILS_TRY(check_array(nsel, p->K > 0 ? nq / groups(p) : 0));
+    HILS_TRY(check_array(lse, nq));
+    HILS_TRY(check_array(dO, nq * p->d));
+    HILS_TRY(check_array(dQ, nq * p->d));
+    HILS_TRY(check_array(dK, nkv));
+    HILS_TRY(check_array(dV, nkv));
+    HILS_TRY(check_array(dscore, nq * p->K));
+    BwdAttendArgs a;
+    a.Q = {Q.ptr, Q.sb, Q.sh, Q.st};
+    a.K = {K.ptr, K.sb, K.sh, K.st};
+    a.V = {V.ptr, V.sb, V.sh, V.st};
+    a.O = {O.ptr, O.sb, O.sh, O.st};
+    a.lse = lse;
+    a.dO = dO;
+    a.score = score;
+    a.idx = idx;
+    a.nsel = nsel;
+    a.dQ = dQ;
+    a.dK = dK;
+    a.dV = dV;
+    a.dscore = dscore;
+    a.B = p->B;
+    a.H = p->H;
+    a.N = N;
+    a.topk = p->K;
+    a.W = p->W;
+    a.G = groups(p);
+    a.scale = scale;
+    return launch_attend_backward(p->dtype, p->d, a, stream);
+}
+
+int hils_select_backward(const hils_params *p, hils_ctensor Qcal, int Lq, hils_ctensor Ksum, int C,
+                         const int32_t *idx, const int32_t *nsel, const float *dscore, float *dQcal, float *dKsum,
+                         float *dBsum, cudaStream_t stream) {
+    float scale;
+    HILS_TRY(check_params(p, &scale));
+    if (Lq < 0 || C < 0) return HILS_ERR_INVALID_ARG;
+    const int64_t nq = (int64_t)p->B * p->H * Lq;
+    if (nq > 0x7fffffffll) return HILS_ERR_INVALID_ARG;
+    HILS_TRY(check_view(Qcal.ptr, Qcal.sb, Qcal.sh, Qcal.st, Lq, p));
+    HILS_TRY(check_view(Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st, C, p));
+    HILS_TRY(check_array(idx, nq / groups(p) * p->K));
+    HILS_TRY(check_array(nsel, p->K > 0 ? nq / groups(p) : 0));
+    HILS_TRY(check_array(dscore, nq * p->K));
+    HILS_TRY(check_array(dQcal, nq * p->d));
+    HILS_TRY(check_array(dKsum, (int64_t)p->B * p->H * C * p->d));
+    HILS_TRY(check_array(dBsum, (int64_t)p->B * p->H * C));
+    BwdSelectArgs a;
+    a.Qcal = {Qcal.ptr, Qcal.sb, Qcal.sh, Qcal.st};
+    a.Ksum = {Ksum.ptr, Ksum.sb, Ksum.sh, Ksum.st};
+    a.idx = idx;
+    a.nsel = nsel;
+    a.dscore = dscore;
+    a.dQcal = dQcal;
+    a.dKsum = dKsum;
+    a.dBsum = dBsum;
+    a.B = p->B;
+    a.H = p->H;
+    a.Lq = Lq;
+    a.C = C;
+    a.topk = p->K;
+    a.G = groups(p);
+    a.scale = scale;
+    return launch_select_backward(p->dtype, p->d, a, stream);
+}
+
+int hils_summarize_backward(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ, const float *dKsum,
+                            const float *dBsum, float *dK, float *dLQ, cudaStream_t stream) {
+    float scale;
+    HILS_TRY(check_params(p, &scale));
+    if (N < 0) return HILS_ERR_INVALID_ARG;
+    const int C = N / kChunk;
+    if ((int64_t)p->B * p->H * C > 0x7fffffffll) return HILS_ERR_INVALID_ARG;
+    HILS_TRY(check_view(K.ptr, K.sb, K.sh, K.st, (int64_t)C * kChunk, p));
+    HILS_TRY(check_view(LQ.ptr, LQ.sb, LQ.sh, LQ.st, C, p));
+    HILS_TRY(check_array(dKsum, (int64_t)p->B * p->H * C * p->d));
+    HILS_TRY(check_array(dBsum, (int64_t)p->B * p->H * C));
+    HILS_TRY(check_array(dK, (int64_t)p->B * (p->H / groups(p)) * N * p->d));
+    HILS_TRY(check_array(dLQ, (int64_t)p->B * p->H * C * p->d));
+    BwdSummarizeArgs a;
+    a.K = {K.ptr, K.sb, K.sh, K.st};
+    a.LQ = {LQ.ptr, LQ.sb, LQ.sh, LQ.st};
+    a.dKsum = dKsum;
+    a.dBsum = dBsum;
+    a.dK = dK;
+    a.dLQ = dLQ;
+    a.B = p->B;
+    a.H = p->H;
+    a.N = N;
+    a.C = C;
+    a.G = groups(p);
+    a.scale = scale;
+    return launch_summarize_backward(p->dtype, p->d, a, stream);
+}
+
 int hils_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_t *qpos, hils_ctensor Ksum,
                 const float *Bsum, int C, int32_t *idx, float *score, int32_t *nsel, void *workspace,
                 size_t ws_bytes, cudaStream_t stream) {

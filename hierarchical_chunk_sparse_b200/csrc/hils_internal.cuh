@@ -80,6 +80,34 @@ struct AttendArgs {
 };
 
 // Host launchers (one translation unit each). They return HILS_OK or HILS_ERR_CUDA.
+// Backward pass (fixed selection; float32 dense gradients, the shared ones accumulated).
+struct BwdAttendArgs {
+    View Q, K, V, O;
+    const float *lse, *dO, *score;
+    const int32_t *idx, *nsel;
+    float *dQ, *dK, *dV, *dscore;
+    int B, H, N, topk, W, G;
+    float scale;
+};
+struct BwdSelectArgs {
+    View Qcal, Ksum;
+    const int32_t *idx, *nsel;
+    const float *dscore;
+    float *dQcal, *dKsum, *dBsum;
+    int B, H, Lq, C, topk, G;
+    float scale;
+};
+struct BwdSummarizeArgs {
+    View K, LQ;
+    const float *dKsum, *dBsum;
+    float *dK, *dLQ;
+    int B, H, N, C, G;
+    float scale;
+};
+hils_status launch_attend_backward(hils_dtype dt, int d, const BwdAttendArgs &a, cudaStream_t s);
+hils_status launch_select_backward(hils_dtype dt, int d, const BwdSelectArgs &a, cudaStream_t s);
+hils_status launch_summarize_backward(hils_dtype dt, int d, const BwdSummarizeArgs &a, cudaStream_t s);
+
 hils_status launch_summarize(hils_dtype dt, int d, const SummarizeArgs &a, cudaStream_t s);
 hils_status launch_select(hils_dtype dt, int d, const SelectArgs &a, cudaStream_t s);
 hils_status launch_attend_decode(hils_dtype dt, int d, const AttendArgs &a, cudaStream_t s);

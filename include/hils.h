@@ -271,6 +271,37 @@ int hils_attend_decode_noalloc(const hils_params *p, hils_ctensor Q, hils_ctenso
                                const int32_t *idx, const float *score, const int32_t *nsel,
                                hils_tensor O, float *lse, cudaStream_t stream);
 
+/* Backward pass for a fixed selection (summary page, Methodology 1-2, Eq. 7, 8, 10;
+ * top-K is piecewise constant, so no gradient flows through the choice of chunks).
+ * Gradients are float32, dense and row-major, in the shapes of their tensors. Three
+ * calls, in this order, give every gradient of sum(O * dO):
+ *   hils_attend_prefill_backward -> dQ, dK and dV (token terms), dscore
+ *   hils_select_backward         -> dQcal, dKsum, dBsum
+ *   hils_summarize_backward      -> dLQ, and the summaries' share of dK
+ * Arrays marked "accumulated" are added to with atomic adds (in no fixed order): zero
+ * them before the first call. Queries are prefill positions t = i. */
+
+/* Eq. 10 backward. Inputs as hils_attend_prefill (idx, score, nsel from hils_select),
+ * with its outputs O [B,H,N,d] (dtype) and lse [B,H,N], and dO [B,H,N,d] float32.
+ *   dQ     [B, H, N, d]   out (written)
+ *   dK, dV [B, Hk, N, d]  accumulated
+ *   dscore [B, H, N, K]   out: the gradient of each kept chunk's score, 0 padding */
+int hils_attend_prefill_backward(const hils_params *p, hils_ctensor Q, hils_ctensor K, hils_ctensor V, int N,
+                                 const int32_t *idx, const float *score, const int32_t *nsel,
+                                 hils_ctensor O, const float *lse, const float *dO,
+                                 float *dQ, float *dK, float *dV, float *dscore, cudaStream_t stream);
+
+/* Eq. 7 backward: dQcal [B,H,Lq,d] (written) = scale sum_k dscore_k k'_{idx_k};
+ * dKsum [B,H,C,d] += scale dscore q~ and dBsum [B,H,C] += dscore (accumulated). */
+int hils_select_backward(const hils_params *p, hils_ctensor Qcal, int Lq, hils_ctensor Ksum, int C,
+                         const int32_t *idx, const int32_t *nsel, const float *dscore,
+                         float *dQcal, float *dKsum, float *dBsum, cudaStream_t stream);
+
+/* Eq. 8 backward for the C = floor(N / S) complete chunks: dLQ [B,H,C,d] (written),
+ * dK [B,Hk,N,d] (accumulated) from dKsum [B,H,C,d] and dBsum [B,H,C]. */
+int hils_summarize_backward(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ,
+                            const float *dKsum, const float *dBsum, float *dK, float *dLQ, cudaStream_t stream);
+
 /* Bytes of workspace a call needs for these sizes (Lq = queries per (b, h); C =
  * summarised chunks). Returns 0 for invalid parameters. */
 size_t hils_workspace_bytes(const hils_params *p, int call, int Lq, int C);

@@ -1,0 +1,76 @@
+"""GPU parity of the backward pass (fixed selection) against the float64 autograd oracle
+(``oracle/backward.py``, pinned by finite differences): the GPU's forward chain
+(summarise, select, attend) gives the selection, O and lse; the three backward calls
+then give dscore, dQ, dK, dV, dQcal, dKsum, dBsum and dLQ, each compared with the
+oracle's gradient of sum(O * dO) for the same selection. Bars, as relative L2 error of
+each gradient: float32 inputs 1e-5 (float32 arithmetic and atomic accumulation order;
+observed about 5e-7); bf16 inputs 1e-2, the forward's bar (the forward's O and summary
+table are stored in bf16, which moves D_i and the chunk scores by up to 2^-9 relative;
+observed about 2e-3)."""
+import numpy as np
+import pytest
+import torch
+
+import hierarchical_chunk_sparse_b200 as hils
+from hils_synth import WORKLOADS, make_prefill
+from hils_testutil import host
+from oracle import backward as ob
+from test_gpu_parity import P, gpu_prefill, gpu_select, gpu_summarize, to_dev
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "fp32_d64": (WORKLOADS[1].replace(H=2, N=64 * 5 + 17, K=3, W=70), 1e-5),
+    "fp32_d128_grouped": (WORKLOADS[1].replace(H=4, Hk=2, d=128, N=64 * 4 + 9, K=2, W=90), 1e-5),
+    "bf16_d128": (WORKLOADS[2].replace(H=2, N=64 * 6 + 9, K=4, W=100), 1e-2),
+    "bf16_d64_grouped": (WORKLOADS[7].replace(H=4, Hk=1, d=64, N=64 * 5 + 3, K=3, W=130), 1e-2),
+}
+
+
+def _rel(g, r):
+    g = host(g).double().numpy() if isinstance(g, torch.Tensor) else np.asarray(g, np.float64)
+    r = r.numpy() if isinstance(r, torch.Tensor) else np.asarray(r, np.float64)
+    den = np.linalg.norm(r)
+    return float(np.linalg.norm(g - r) / den) if den > 0 else float(np.abs(g).max())
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_backward_matches_oracle(cuda_device, case):
+    w, tol = CASES[case]
+    inp = make_prefill(w)
+    d = to_dev(inp, cuda_device)
+    Ksum, Bsum = gpu_summarize(w, d["K"], d["LQ"])
+    idx, score, nsel = gpu_select(w, d["Qcal"], Ksum, Bsum)
+    O, lse = gpu_prefill(w, d["Q"], d["K"], d["V"], idx, score, nsel)
+    g = torch.Generator().manual_seed(7)
+    dO = torch.randn(O.shape, generator=g).to(cuda_device)
+    p = P(w)
+    B, H, N, dd, Hk, K, C = w.B, w.H, w.N, w.d, w.Hkv, w.K, w.C
+    f32 = dict(dtype=torch.float32, device=cuda_device)
+    dQ, dK, dV = torch.empty(B, H, N, dd, **f32), torch.zeros(B, Hk, N, dd, **f32), torch.zeros(B, Hk, N, dd, **f32)
+    dscore = torch.empty(B, H, N, K, **f32)
+    hils.hils_attend_prefill_backward(p, d["Q"], d["K"], d["V"], idx, score, nsel, O, lse, dO, dQ, dK, dV, dscore)
+    dQcal = torch.empty(B, H, N, dd, **f32)
+    dKsum, dBsum = torch.zeros(B, H, C, dd, **f32), torch.zeros(B, H, C, **f32)
+    hils.hils_select_backward(p, d["Qcal"], Ksum, idx, nsel, dscore, dQcal, dKsum, dBsum)
+    dLQ = torch.empty(B, H, C, dd, **f32)
+    hils.hils_summarize_backward(p, d["K"], d["LQ"], dKsum, dBsum, dK, dLQ)
+    torch.cuda.synchronize()
+    ref = ob.grads(inp["Q"], inp["K"], inp["V"], inp["Qcal"], inp["LQ"], host(idx), host(nsel), host(dO), 64, w.W,
+                   w.scale)
+    errs = {
+        "dscore": _rel(dscore, ref["dscore"]),
+        "dQ": _rel(dQ, ref["dQ"]),
+        "dV": _rel(dV, ref["dV"]),
+        "dQcal": _rel(dQcal, ref["dQcal"]),
+        "dKsum": _rel(dKsum, ref["dKsum"]),
+        "dBsum": _rel(dBsum, ref["dBsum"]),
+        "dLQ": _rel(dLQ, ref["dLQ"]),
+        "dK": _rel(dK, ref["dK"]),
+    }
+    print(case, {k: f"{v:.2e}" for k, v in errs.items()})
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, f"relative L2 errors above {tol}: {bad} (all: {errs})"
+    # padding of dscore is exactly zero
+    kept = torch.arange(K, device=cuda_device).view(1, 1, 1, K) < nsel.repeat_interleave(w.G, dim=1).unsqueeze(-1)
+    assert (dscore[~kept] == 0).all()
