@@ -574,12 +574,13 @@ def measure_prefill_backward(w, dev, stream, flush, args, world):
     dscore, dQcal = torch.empty(B, H, N, K, **f32), torch.empty(B, H, N, d, **f32)
     dKsum, dBsum, dLQ = torch.zeros(B, H, C, d, **f32), torch.zeros(B, H, C, **f32), torch.empty(B, H, C, d, **f32)
     i = pb.inp
+    ws = hils.alloc_workspace(pb.p, hils.HILS_CALL_ATTEND_BACKWARD, N, 0, device=dev)
 
     def bwd():
         for t in (dK, dV, dKsum, dBsum):
             t.zero_()
         hils.hils_attend_prefill_backward(pb.p, i["Q"], i["K"], i["V"], pb.idx, pb.score, pb.nsel, pb.O, pb.lse, dO,
-                                          dQ, dK, dV, dscore)
+                                          dQ, dK, dV, dscore, workspace=ws)
         hils.hils_select_backward(pb.p, i["Qcal"], pb.Ksum, pb.idx, pb.nsel, dscore, dQcal, dKsum, dBsum)
         hils.hils_summarize_backward(pb.p, i["K"], i["LQ"], dKsum, dBsum, dK, dLQ)
 
@@ -593,7 +594,7 @@ def measure_prefill_backward(w, dev, stream, flush, args, world):
     fl = backward_flops(w)
     out = {"ms_per_step": ms, "unit": "TFLOP/s", "value": fl / (ms * 1e-3) / 1e12 * world, "workload": w.name,
            "algorithmic_gflop_per_step": fl / 1e9, "steps": n,
-           "note": "first version: CUDA-core kernels, float32 atomic accumulation of dK, dV, dKsum, dBsum"}
+           "note": "CUDA-core kernels: key-major attend backward (dK, dV accumulated per key block), float32 atomics for dQ, dKsum, dBsum"}
     del pb
     torch.cuda.empty_cache()
     return out

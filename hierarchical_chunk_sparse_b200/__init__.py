@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(_PKG, "libhils.so")
 
 HILS_F32, HILS_BF16 = 0, 1
 HILS_CALL_SELECT, HILS_CALL_ATTEND_PREFILL, HILS_CALL_ATTEND_DECODE, HILS_CALL_DECODE = 0, 1, 2, 3
+HILS_CALL_ATTEND_BACKWARD = 4
 # hils_params.flags: chunks wholly inside a query's window are not selected
 HILS_FLAG_EXCLUDE_WINDOW_CHUNKS = 1
 STATUS = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARG", 2: "HILS_ERR_UNSUPPORTED",
@@ -67,7 +68,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         T, P, vp, i, sz = _CTensor, ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         lib.hils_summarize.argtypes = [P, T, i, T, T, vp, vp]
         lib.hils_summarize_append.argtypes = [P, T, vp, T, T, vp, i, vp]
-        lib.hils_attend_prefill_backward.argtypes = [P, T, T, T, i, vp, vp, vp, T, vp, vp, vp, vp, vp, vp, vp]
+        lib.hils_attend_prefill_backward.argtypes = [P, T, T, T, i, vp, vp, vp, T, vp, vp, vp, vp, vp, vp, vp, sz,
+                                                     vp]
         lib.hils_select_backward.argtypes = [P, T, i, T, i, vp, vp, vp, vp, vp, vp, vp]
         lib.hils_summarize_backward.argtypes = [P, T, i, T, vp, vp, vp, vp, vp]
         lib.hils_select.argtypes = [P, T, i, vp, T, vp, i, vp, vp, vp, vp, sz, vp]
@@ -326,7 +328,7 @@ def _dense32(call: str, name: str, t, shape) -> None:
 
 
 def hils_attend_prefill_backward(p: Params, Q, K, V, idx, score, nsel, O, lse, dO, dQ, dK, dV, dscore,
-                                 stream=None) -> None:
+                                 workspace=None, stream=None) -> None:
     """Eq. 10 backward for the kept chunks of hils_select: dQ [B,H,N,d] (written),
     dK, dV [B,Hk,N,d] (accumulated: zero them first), dscore [B,H,N,K] (written); all
     float32 and dense. O, lse are the forward's outputs, dO [B,H,N,d] float32."""
@@ -342,9 +344,12 @@ def hils_attend_prefill_backward(p: Params, Q, K, V, idx, score, nsel, O, lse, d
     _expect("hils_attend_prefill_backward", "lse", lse, (B, H, n), torch.float32)
     for name, t, h in (("dO", dO, H), ("dQ", dQ, H), ("dK", dK, Hk), ("dV", dV, Hk)):
         _dense32("hils_attend_prefill_backward", name, t, (B, h, n, d))
+    if workspace is None:
+        workspace = alloc_workspace(p, HILS_CALL_ATTEND_BACKWARD, n, 0, device=Q.device)
+    wp, wn = _ws(workspace)
     _check("hils_attend_prefill_backward", load_library().hils_attend_prefill_backward(
         ctypes.byref(p.c()), _view(Q), _view(K), _view(V), n, _ptr(idx), _ptr(score), _ptr(nsel), _view(O),
-        _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dscore), _stream(stream)))
+        _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dscore), wp, wn, _stream(stream)))
 
 
 def hils_select_backward(p: Params, Qcal, Ksum, idx, nsel, dscore, dQcal, dKsum, dBsum, stream=None) -> None:

@@ -18,9 +18,14 @@
 //   dp_j = k_j . dk'_c - db'_c (log p_j + 1),  dl_j = p_j (dp_j - sum_i p_i dp_i),
 //   dq'_c = scale sum_j dl_j k_j,  dk_j += p_j dk'_c + scale dl_j q'_c.
 //
-// One 128-thread CTA per query (attend, score) or per chunk (summaries); the key and
-// value gradients, which many queries and chunks share, are accumulated with float32
-// atomic adds (the order of the additions is not fixed). Gradients are float32, dense.
+// Attend: key-major. A 128-thread CTA owns one 64-key block of one (b, h) and walks the
+// queries that attend it, accumulating the block's dk and dv in shared memory and adding
+// each query's dq share to dQ with float32 atomics: for a window block, the contiguous
+// range of queries whose window reaches it; for a chunk, the queries that kept it, from
+// an inverted index of the selection built first (count, scan, scatter). D_i = dO_i . o_i
+// is computed once per query beforehand. Score and summaries: one CTA per query or per
+// chunk. Shared gradients (dK, dV, dKsum, dBsum, dQ) are float32 atomic adds, in no fixed
+// order. Gradients are float32, dense.
 #include <math.h>
 
 #include "hils_internal.cuh"
@@ -30,11 +35,32 @@ namespace {
 
 constexpr int kThreads = 128;
 
-template <typename T, int D>
-struct BwdCfg {
-    // key and value rows of one unit as float32, then the per-row scalars
-    static constexpr int kSmemBytes = (2 * kChunk * D + 3 * D + 6 * kChunk + 8) * 4;
+// Workspace of the attend backward: D_i per query, then per (b, group) the chunk counts,
+// starts (C + 1), cursors and the inverted index (N * K entries).
+struct BwdWs {
+    float *D;
+    int *count, *start, *cursor, *entries;
+    size_t bytes;
 };
+inline size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
+inline BwdWs bwd_ws(void *ws, int B, int H, int Hk, int N, int K) {
+    const int C = N / kChunk;
+    uint8_t *p = static_cast<uint8_t *>(ws);
+    BwdWs w;
+    size_t off = 0;
+    w.D = reinterpret_cast<float *>(p + off);
+    off += a256((size_t)B * H * N * 4);
+    w.count = reinterpret_cast<int *>(p + off);
+    off += a256((size_t)B * Hk * C * 4);
+    w.start = reinterpret_cast<int *>(p + off);
+    off += a256((size_t)B * Hk * (C + 1) * 4);
+    w.cursor = reinterpret_cast<int *>(p + off);
+    off += a256((size_t)B * Hk * C * 4);
+    w.entries = reinterpret_cast<int *>(p + off);
+    off += a256((size_t)B * Hk * N * (K > 0 ? K : 1) * 4);
+    w.bytes = off;
+    return w;
+}
 
 template <typename T>
 __device__ __forceinline__ float elem(const T *p, int x) {
@@ -53,117 +79,274 @@ __device__ __forceinline__ float block_sum(float v, float *scratch) {
     return r;
 }
 
-// grid: B*H*N, one query each.
+// ---- key-major attend backward
+
+// D_i = dO_i . o_i, one warp per query.
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads) attend_backward_kernel(BwdAttendArgs a) {
-    extern __shared__ __align__(16) float fsm[];
-    float *kt = fsm, *vt = kt + kChunk * D;          // [64][D] each
-    float *qf = vt + kChunk * D, *dof = qf + D, *of = dof + D;
-    float *lg = of + D, *tj = lg + kChunk, *dl = tj + kChunk, *cv = dl + kChunk;
-    float *scratch = cv + kChunk;                     // 8 floats
-    const int tid = threadIdx.x;
-    const int64_t qi = blockIdx.x;
+__global__ void __launch_bounds__(kThreads) bwd_dot_kernel(BwdAttendArgs a, float *Dv) {
+    const int64_t qi = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (qi >= (int64_t)a.B * a.H * a.N) return;
     const int i = (int)(qi % a.N);
     const int h = (int)((qi / a.N) % a.H);
     const int b = (int)(qi / ((int64_t)a.N * a.H));
-    const int Hk = a.H / a.G, hk = h / a.G;
-    const int64_t qg = ((int64_t)b * Hk + hk) * a.N + i;
-    const T *qrow = static_cast<const T *>(a.Q.ptr) + b * a.Q.sb + h * a.Q.sh + (int64_t)i * a.Q.st;
     const T *orow = static_cast<const T *>(a.O.ptr) + b * a.O.sb + h * a.O.sh + (int64_t)i * a.O.st;
-    const float *dorow = a.dO + qi * D;
-    for (int x = tid; x < D; x += kThreads) {
-        qf[x] = elem(qrow, x);
-        dof[x] = dorow[x];
-        of[x] = elem(orow, x);
-    }
+    float acc = 0.f;
+    for (int x = lane; x < D; x += 32) acc = fmaf(a.dO[qi * D + x], elem(orow, x), acc);
+    acc = warp_sum(acc);
+    if (lane == 0) Dv[qi] = acc;
+}
+
+// Inverted index of the selection per (b, group): count[c], then (after the scan)
+// cursor[c] = start[c] + filled so far; entries hold i * 32 + k.
+__global__ void bwd_count_kernel(BwdAttendArgs a, int *count) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // (b, group, i, k)
+    const int Hk = a.H / a.G, K = a.topk;
+    if (e >= (int64_t)a.B * Hk * a.N * K) return;
+    const int64_t qg = e / K;
+    const int k = (int)(e % K);
+    if (k >= min(max(a.nsel[qg], 0), K)) return;
+    const int c = a.idx[e];
+    const int64_t bg = qg / a.N;
+    if (c >= 0 && c < a.N / kChunk) atomicAdd(&count[bg * (a.N / kChunk) + c], 1);
+}
+
+// exclusive scan of count over the C chunks of one (b, group): start[c], cursor[c]
+__global__ void __launch_bounds__(1024) bwd_scan_kernel(int C, const int *count, int *start, int *cursor) {
+    __shared__ int part[1024];
+    const int64_t bg = blockIdx.x;
+    const int *cnt = count + bg * C;
+    const int per = (C + 1023) / 1024, t = threadIdx.x;
+    int sum = 0;
+    for (int c = t * per; c < min(C, (t + 1) * per); ++c) sum += cnt[c];
+    part[t] = sum;
     __syncthreads();
-    float part = 0.f;
-    for (int x = tid; x < D; x += kThreads) part = fmaf(dof[x], of[x], part);
-    const float Di = block_sum(part, scratch);  // dO . o
-    const float lse = a.lse[qi];
-    const int K = a.topk;
-    const int ns = (K > 0 && isfinite(lse)) ? min(max(a.nsel[qg], 0), K) : 0;
-    float dq = 0.f;  // column tid of dq (tid < D)
-    const int w0 = max(0, i - a.W + 1);
-    const int nwin = (a.W > 0 && isfinite(lse)) ? (i - w0) / kChunk + 1 : 0;
+    for (int o = 1; o < 1024; o <<= 1) {  // inclusive scan of the per-thread sums
+        const int v = t >= o ? part[t - o] : 0;
+        __syncthreads();
+        part[t] += v;
+        __syncthreads();
+    }
+    int run = part[t] - sum;
+    for (int c = t * per; c < min(C, (t + 1) * per); ++c) {
+        start[bg * (C + 1) + c] = run;
+        cursor[bg * C + c] = run;
+        run += cnt[c];
+    }
+    if (t == 1023) start[bg * (C + 1) + C] = part[1023];
+}
+
+__global__ void bwd_scatter_kernel(BwdAttendArgs a, int *cursor, int *entries) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int Hk = a.H / a.G, K = a.topk, C = a.N / kChunk;
+    if (e >= (int64_t)a.B * Hk * a.N * K) return;
+    const int64_t qg = e / K;
+    const int k = (int)(e % K);
+    if (k >= min(max(a.nsel[qg], 0), K)) return;
+    const int c = a.idx[e];
+    if (c < 0 || c >= C) return;
+    const int64_t bg = qg / a.N;
+    const int i = (int)(qg % a.N);
+    const int pos = atomicAdd(&cursor[bg * C + c], 1);
+    entries[bg * (int64_t)a.N * K + pos] = i * 32 + k;
+}
+
+constexpr int kQT = 16;  // queries per step of the key-major kernel
+
+template <typename T, int D>
+struct KmCfg {
+    static constexpr int kLd = D + 1;  // padded row stride: column x of rows j in distinct banks
+    // K and V rows of the block, the dk and dv accumulators ([64][kLd] float32 each), a
+    // step's q and dO rows ([kQT][D]), their logits/dl and dO.v/cv ([kQT][64]), and the
+    // step's per-query scalars
+    static constexpr int kSmemBytes = (4 * kChunk * kLd + 2 * kQT * D + 2 * kQT * kChunk + 4 * kQT) * 4;
+};
+
+// One 64-key block of (b, h): window queries (kChunkMode = false) or the queries that
+// kept chunk c (true), kQT at a time. grid: (key blocks or chunks, B * H).
+template <typename T, int D, bool kChunkMode>
+__global__ void __launch_bounds__(kThreads) attend_bwd_keymajor_kernel(BwdAttendArgs a, const float *Dv,
+                                                                       const int *start, const int *entries) {
+    using Cfg = KmCfg<T, D>;
+    constexpr int kLd = Cfg::kLd;
+    extern __shared__ __align__(16) float fsm[];
+    float *kt = fsm, *vt = kt + kChunk * kLd, *dka = vt + kChunk * kLd, *dva = dka + kChunk * kLd;
+    float *qs = dva + kChunk * kLd, *dos = qs + kQT * D;   // [kQT][D]
+    float *lg = dos + kQT * D, *tj = lg + kQT * kChunk;    // [kQT][64]: logits -> dl, dO.v -> cv
+    float *q_lse = tj + kQT * kChunk, *q_D = q_lse + kQT, *q_w = q_D + kQT;
+    int *q_i = reinterpret_cast<int *>(q_w + kQT);
+    const int tid = threadIdx.x;
+    const int blk = blockIdx.x;
+    const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+    const int Hk = a.H / a.G, hk = h / a.G, K = a.topk, C = a.N / kChunk;
+    const int j0 = blk * kChunk;
+    const int rows = min(kChunk, a.N - j0);
     const T *kbase = static_cast<const T *>(a.K.ptr) + b * a.K.sb + hk * a.K.sh;
     const T *vbase = static_cast<const T *>(a.V.ptr) + b * a.V.sb + hk * a.V.sh;
-    float *dkbase = a.dK + ((int64_t)b * Hk + hk) * a.N * D;
-    float *dvbase = a.dV + ((int64_t)b * Hk + hk) * a.N * D;
-    for (int u = 0; u < ns + nwin; ++u) {
-        const bool chunk = u < ns;
-        int start, rows;
-        float mass = 0.f;
-        if (chunk) {
-            const int c = a.idx[qg * K + u];
-            start = c * kChunk;
-            rows = kChunk;
-            mass = a.score[qi * K + u];
-        } else {
-            start = w0 + (u - ns) * kChunk;
-            rows = min(kChunk, i - start + 1);
-        }
-        for (int e = tid; e < rows * D; e += kThreads) {
-            const int j = e / D, x = e - (e / D) * D;
-            kt[e] = elem(kbase + (int64_t)(start + j) * a.K.st, x);
-            vt[e] = elem(vbase + (int64_t)(start + j) * a.V.st, x);
+    int q_begin, q_end;
+    const int *list = nullptr;
+    if (kChunkMode) {
+        const int64_t bg = (int64_t)b * Hk + hk;
+        q_begin = start[bg * (C + 1) + blk];
+        q_end = start[bg * (C + 1) + blk + 1];
+        list = entries + bg * (int64_t)a.N * K;
+    } else {
+        q_begin = j0;
+        q_end = a.W > 0 ? min(a.N, j0 + rows - 1 + a.W) : j0;  // i with a window key in the block
+    }
+    if (q_begin >= q_end) return;
+    for (int e = tid; e < kChunk * D; e += kThreads) {
+        const int j = e / D, x = e - (e / D) * D;
+        kt[j * kLd + x] = j < rows ? elem(kbase + (int64_t)(j0 + j) * a.K.st, x) : 0.f;
+        vt[j * kLd + x] = j < rows ? elem(vbase + (int64_t)(j0 + j) * a.V.st, x) : 0.f;
+        dka[j * kLd + x] = 0.f;
+        dva[j * kLd + x] = 0.f;
+    }
+    const int64_t qhead = ((int64_t)b * a.H + h) * a.N;
+    for (int q0 = q_begin; q0 < q_end; q0 += kQT) {
+        const int nq = min(kQT, q_end - q0);
+        __syncthreads();  // the previous step's rows and scalars are no longer read
+        if (tid < kQT) {  // the step's queries: index, lse, D, and (chunks) slot k and score weight
+            int i = -1, k = 0;
+            float lse = -INFINITY, w = 0.f;
+            if (tid < nq) {
+                if (kChunkMode) {
+                    const int en = list[q0 + tid];
+                    i = en >> 5;
+                    k = en & 31;
+                } else {
+                    i = q0 + tid;
+                }
+                lse = a.lse[qhead + i];
+                if (kChunkMode && isfinite(lse)) w = expf(a.score[(qhead + i) * K + k] - lse);
+            }
+            q_i[tid] = isfinite(lse) ? (kChunkMode ? (i * 32 + k) : i) : -1;
+            q_lse[tid] = lse;
+            q_D[tid] = (i >= 0 && isfinite(lse)) ? Dv[qhead + i] : 0.f;
+            q_w[tid] = w;
         }
         __syncthreads();
-        {  // l_j = scale q . k_j and t_j = dO . v_j, two threads per row
-            const int row = tid >> 1, half = tid & 1;
-            float al = 0.f, at = 0.f;
-            if (row < rows) {
-                for (int x = half * (D / 2); x < (half + 1) * (D / 2); ++x) {
-                    al = fmaf(qf[x], kt[row * D + x], al);
-                    at = fmaf(dof[x], vt[row * D + x], at);
+        for (int e = tid; e < kQT * D; e += kThreads) {
+            const int r = e / D, x = e - (e / D) * D;
+            const int en = q_i[r];
+            const int i = en < 0 ? -1 : (kChunkMode ? en >> 5 : en);
+            float qv = 0.f, dv = 0.f;
+            if (i >= 0) {
+                qv = elem(static_cast<const T *>(a.Q.ptr) + b * a.Q.sb + h * a.Q.sh + (int64_t)i * a.Q.st, x);
+                dv = a.dO[(qhead + i) * D + x];
+            }
+            qs[e] = qv;
+            dos[e] = dv;
+        }
+        __syncthreads();
+        {  // logits l[r][j] = scale q_r . k_j and t[r][j] = dO_r . v_j: key j, queries r0..r0+7
+            const int j = tid & (kChunk - 1), r0 = (tid >> 6) * (kQT / 2);
+            float al[kQT / 2], at[kQT / 2];
+#pragma unroll
+            for (int r = 0; r < kQT / 2; ++r) al[r] = at[r] = 0.f;
+            for (int x = 0; x < D; ++x) {
+                const float kv = kt[j * kLd + x], vv = vt[j * kLd + x];
+#pragma unroll
+                for (int r = 0; r < kQT / 2; ++r) {
+                    al[r] = fmaf(qs[(r0 + r) * D + x], kv, al[r]);
+                    at[r] = fmaf(dos[(r0 + r) * D + x], vv, at[r]);
                 }
             }
-            al += __shfl_xor_sync(kFull, al, 1);
-            at += __shfl_xor_sync(kFull, at, 1);
-            if (half == 0 && row < kChunk) {
-                lg[row] = row < rows ? al * a.scale : -INFINITY;
-                tj[row] = row < rows ? at : 0.f;
+#pragma unroll
+            for (int r = 0; r < kQT / 2; ++r) {
+                const int rr = r0 + r, en = q_i[rr];
+                bool ok = en >= 0 && j < rows;
+                if (!kChunkMode && ok) ok = j0 + j <= en && j0 + j > en - a.W;  // in query en's window
+                lg[rr * kChunk + j] = ok ? al[r] * a.scale : -INFINITY;
+                tj[rr * kChunk + j] = ok ? at[r] : 0.f;
             }
         }
         __syncthreads();
-        if (tid < 32) {
-            const int lane = tid;
-            const float l0 = lg[lane], l1 = lg[lane + 32];
-            if (chunk) {
-                const float m = warp_max(fmaxf(l0, l1));
-                const float e0 = expf(l0 - m), e1 = expf(l1 - m);
-                const float inv = 1.f / warp_sum(e0 + e1);
-                const float p0 = e0 * inv, p1 = e1 * inv;
-                const float oc = warp_sum(p0 * tj[lane] + p1 * tj[lane + 32]);  // dO . o_c
-                const float w = expf(mass - lse);
-                dl[lane] = w * p0 * (tj[lane] - oc);
-                dl[lane + 32] = w * p1 * (tj[lane + 32] - oc);
-                cv[lane] = w * p0;
-                cv[lane + 32] = w * p1;
-                if (lane == 0) a.dscore[qi * K + u] = w * (oc - Di);
-            } else {
-                const float w0j = expf(l0 - lse), w1j = expf(l1 - lse);  // 0 past the rows
-                dl[lane] = w0j * (tj[lane] - Di);
-                dl[lane + 32] = w1j * (tj[lane + 32] - Di);
-                cv[lane] = w0j;
-                cv[lane + 32] = w1j;
+        {  // per query (a warp takes four): weights, dl (into lg) and cv (into tj), dscore
+            const int lane = tid & 31, w = tid >> 5;
+#pragma unroll
+            for (int r4 = 0; r4 < kQT / 4; ++r4) {
+                const int r = w * (kQT / 4) + r4;
+                const int en = q_i[r];
+                if (en < 0) {  // warp-uniform
+                    lg[r * kChunk + lane] = lg[r * kChunk + lane + 32] = 0.f;
+                    tj[r * kChunk + lane] = tj[r * kChunk + lane + 32] = 0.f;
+                    continue;
+                }
+                const float l0 = lg[r * kChunk + lane], l1 = lg[r * kChunk + lane + 32];
+                const float t0 = tj[r * kChunk + lane], t1 = tj[r * kChunk + lane + 32];
+                const float Di = q_D[r];
+                float d0, d1, c0, c1;
+                if (kChunkMode) {
+                    const float m = warp_max(fmaxf(l0, l1));
+                    const float e0 = expf(l0 - m), e1 = expf(l1 - m);
+                    const float inv = 1.f / warp_sum(e0 + e1);
+                    const float p0 = e0 * inv, p1 = e1 * inv;
+                    const float oc = warp_sum(p0 * t0 + p1 * t1);
+                    const float wc = q_w[r];
+                    d0 = wc * p0 * (t0 - oc);
+                    d1 = wc * p1 * (t1 - oc);
+                    c0 = wc * p0;
+                    c1 = wc * p1;
+                    if (lane == 0) a.dscore[(qhead + (en >> 5)) * K + (en & 31)] = wc * (oc - Di);
+                } else {
+                    const float lse = q_lse[r];
+                    c0 = expf(l0 - lse);  // 0 outside the window
+                    c1 = expf(l1 - lse);
+                    d0 = c0 * (t0 - Di);
+                    d1 = c1 * (t1 - Di);
+                }
+                lg[r * kChunk + lane] = d0;
+                lg[r * kChunk + lane + 32] = d1;
+                tj[r * kChunk + lane] = c0;
+                tj[r * kChunk + lane + 32] = c1;
             }
         }
         __syncthreads();
-        if (tid < D) {
-            float acc = 0.f;
-            for (int j = 0; j < rows; ++j) acc = fmaf(dl[j], kt[j * D + tid], acc);
-            dq = fmaf(a.scale, acc, dq);
+        {  // dk_j += scale sum_r dl[r][j] q_r and dv_j += sum_r cv[r][j] dO_r: key j, a column half
+            const int j = tid & (kChunk - 1), xh = (tid >> 6) * (D / 2);
+            float dlr[kQT], cvr[kQT];
+#pragma unroll
+            for (int r = 0; r < kQT; ++r) {
+                dlr[r] = a.scale * lg[r * kChunk + j];
+                cvr[r] = tj[r * kChunk + j];
+            }
+            for (int x = xh; x < xh + D / 2; ++x) {
+                float sk = dka[j * kLd + x], sv = dva[j * kLd + x];
+#pragma unroll
+                for (int r = 0; r < kQT; ++r) {
+                    sk = fmaf(dlr[r], qs[r * D + x], sk);
+                    sv = fmaf(cvr[r], dos[r * D + x], sv);
+                }
+                dka[j * kLd + x] = sk;
+                dva[j * kLd + x] = sv;
+            }
         }
-        for (int e = tid; e < rows * D; e += kThreads) {
-            const int j = e / D, x = e - (e / D) * D;
-            atomicAdd(dkbase + (int64_t)(start + j) * D + x, a.scale * dl[j] * qf[x]);
-            atomicAdd(dvbase + (int64_t)(start + j) * D + x, cv[j] * dof[x]);
+        if (tid < D) {  // this block's share of dq_r: column tid
+            float acc[kQT];
+#pragma unroll
+            for (int r = 0; r < kQT; ++r) acc[r] = 0.f;
+            for (int j = 0; j < rows; ++j) {
+                const float kv = kt[j * kLd + tid];
+#pragma unroll
+                for (int r = 0; r < kQT; ++r) acc[r] = fmaf(lg[r * kChunk + j], kv, acc[r]);
+            }
+            for (int r = 0; r < nq; ++r) {
+                const int en = q_i[r];
+                if (en < 0) continue;
+                const int i = kChunkMode ? en >> 5 : en;
+                atomicAdd(a.dQ + (qhead + i) * D + tid, a.scale * acc[r]);
+            }
         }
-        __syncthreads();  // the unit's rows are no longer read
     }
-    if (tid < D) a.dQ[qi * D + tid] = dq;
-    for (int k = ns + tid; k < K; k += kThreads) a.dscore[qi * K + k] = 0.f;
+    __syncthreads();
+    float *dkb = a.dK + ((int64_t)b * Hk + hk) * a.N * D + (int64_t)j0 * D;
+    float *dvb = a.dV + ((int64_t)b * Hk + hk) * a.N * D + (int64_t)j0 * D;
+    for (int e = tid; e < rows * D; e += kThreads) {
+        const int j = e / D, x = e - (e / D) * D;
+        atomicAdd(dkb + e, dka[j * kLd + x]);
+        atomicAdd(dvb + e, dva[j * kLd + x]);
+    }
 }
 
 // grid: B*H*Lq, one query each: Eq. 7 backward.
@@ -269,12 +452,36 @@ __global__ void __launch_bounds__(kThreads) summarize_backward_kernel(BwdSummari
 }
 
 template <typename T, int D>
-hils_status launch_attend_bwd(const BwdAttendArgs &a, cudaStream_t s) {
-    constexpr int smem = BwdCfg<T, D>::kSmemBytes;
-    static KernelSetup setup;
-    const hils_status st = kernel_setup(setup, (const void *)attend_backward_kernel<T, D>, kThreads, smem, nullptr);
+hils_status launch_attend_bwd(const BwdAttendArgs &a, void *ws, cudaStream_t s) {
+    const int64_t nq = (int64_t)a.B * a.H * a.N;
+    const int Hk = a.H / a.G, C = a.N / kChunk;
+    const BwdWs w = bwd_ws(ws, a.B, a.H, Hk, a.N, a.topk);
+    hils_status st = record_cuda_error(cudaMemsetAsync(a.dQ, 0, (size_t)nq * D * sizeof(float), s));
     if (st != HILS_OK) return st;
-    attend_backward_kernel<T, D><<<(unsigned)((int64_t)a.B * a.H * a.N), kThreads, smem, s>>>(a);
+    if (a.topk > 0) {  // dscore padding stays 0
+        st = record_cuda_error(cudaMemsetAsync(a.dscore, 0, (size_t)nq * a.topk * sizeof(float), s));
+        if (st != HILS_OK) return st;
+    }
+    bwd_dot_kernel<T, D><<<(unsigned)((nq + 3) / 4), kThreads, 0, s>>>(a, w.D);
+    constexpr int smem = KmCfg<T, D>::kSmemBytes;
+    static KernelSetup setup_w, setup_c;
+    st = kernel_setup(setup_w, (const void *)attend_bwd_keymajor_kernel<T, D, false>, kThreads, smem, nullptr);
+    if (st != HILS_OK) return st;
+    st = kernel_setup(setup_c, (const void *)attend_bwd_keymajor_kernel<T, D, true>, kThreads, smem, nullptr);
+    if (st != HILS_OK) return st;
+    if (a.topk > 0 && C > 0) {
+        const int64_t ne = (int64_t)a.B * Hk * a.N * a.topk;
+        st = record_cuda_error(cudaMemsetAsync(w.count, 0, (size_t)a.B * Hk * C * sizeof(int), s));
+        if (st != HILS_OK) return st;
+        bwd_count_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.count);
+        bwd_scan_kernel<<<(unsigned)(a.B * Hk), 1024, 0, s>>>(C, w.count, w.start, w.cursor);
+        bwd_scatter_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.cursor, w.entries);
+        attend_bwd_keymajor_kernel<T, D, true><<<dim3(C, a.B * a.H), kThreads, smem, s>>>(a, w.D, w.start,
+                                                                                            w.entries);
+    }
+    if (a.W > 0)
+        attend_bwd_keymajor_kernel<T, D, false><<<dim3((a.N + kChunk - 1) / kChunk, a.B * a.H), kThreads, smem, s>>>(
+            a, w.D, nullptr, nullptr);
     return record_cuda_error(cudaGetLastError());
 }
 
@@ -296,10 +503,15 @@ hils_status launch_summarize_bwd(const BwdSummarizeArgs &a, cudaStream_t s) {
 
 }  // namespace
 
-hils_status launch_attend_backward(hils_dtype dt, int d, const BwdAttendArgs &a, cudaStream_t s) {
+hils_status launch_attend_backward(hils_dtype dt, int d, const BwdAttendArgs &a, void *ws, cudaStream_t s) {
     if ((int64_t)a.B * a.H * a.N == 0) return HILS_OK;
-    if (dt == HILS_BF16) return d == 64 ? launch_attend_bwd<bf16, 64>(a, s) : launch_attend_bwd<bf16, 128>(a, s);
-    return d == 64 ? launch_attend_bwd<float, 64>(a, s) : launch_attend_bwd<float, 128>(a, s);
+    if (dt == HILS_BF16)
+        return d == 64 ? launch_attend_bwd<bf16, 64>(a, ws, s) : launch_attend_bwd<bf16, 128>(a, ws, s);
+    return d == 64 ? launch_attend_bwd<float, 64>(a, ws, s) : launch_attend_bwd<float, 128>(a, ws, s);
+}
+
+size_t attend_backward_ws_bytes(int B, int H, int Hk, int N, int K) {
+    return bwd_ws(nullptr, B, H, Hk, N, K).bytes;
 }
 
 hils_status launch_select_backward(hils_dtype dt, int d, const BwdSelectArgs &a, cudaStream_t s) {

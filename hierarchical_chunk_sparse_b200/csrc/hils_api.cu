@@ -221,6 +221,7 @@ size_t hils_workspace_bytes(const hils_params *p, int call, int Lq, int C) {
     case HILS_CALL_SELECT: return select_ws_for(p, Lq, C);
     case HILS_CALL_ATTEND_PREFILL: return kPrefillWsBytes;
     case HILS_CALL_ATTEND_DECODE: return attend_decode_ws_bytes(p->B * p->H, decode_units(p), p->d);
+    case HILS_CALL_ATTEND_BACKWARD: return attend_backward_ws_bytes(p->B, p->H, p->H / groups(p), Lq, p->K);
     case HILS_CALL_DECODE:
         return decode_select_part(select_ws_for(p, 1, C)) + attend_decode_ws_bytes(p->B * p->H, decode_units(p), p->d);
     default: return 0;
@@ -285,7 +286,7 @@ int hils_summarize_append(const hils_params *p, hils_ctensor K, const int32_t *c
 int hils_attend_prefill_backward(const hils_params *p, hils_ctensor Q, hils_ctensor K, hils_ctensor V, int N,
                                  const int32_t *idx, const float *score, const int32_t *nsel, hils_ctensor O,
                                  const float *lse, const float *dO, float *dQ, float *dK, float *dV, float *dscore,
-                                 cudaStream_t stream) {
+                                 void *workspace, size_t ws_bytes, cudaStream_t stream) {
     float scale;
     HILS_TRY(check_params(p, &scale));
     if (N < 0) return HILS_ERR_INVALID_ARG;
@@ -305,6 +306,9 @@ int hils_attend_prefill_backward(const hils_params *p, hils_ctensor Q, hils_cten
     HILS_TRY(check_array(dK, nkv));
     HILS_TRY(check_array(dV, nkv));
     HILS_TRY(check_array(dscore, nq * p->K));
+    if (nq == 0) return HILS_OK;
+    HILS_TRY(check_workspace(workspace, ws_bytes,
+                             attend_backward_ws_bytes(p->B, p->H, p->H / groups(p), N, p->K)));
     BwdAttendArgs a;
     a.Q = {Q.ptr, Q.sb, Q.sh, Q.st};
     a.K = {K.ptr, K.sb, K.sh, K.st};
@@ -326,7 +330,7 @@ int hils_attend_prefill_backward(const hils_params *p, hils_ctensor Q, hils_cten
     a.W = p->W;
     a.G = groups(p);
     a.scale = scale;
-    return launch_attend_backward(p->dtype, p->d, a, stream);
+    return launch_attend_backward(p->dtype, p->d, a, workspace, stream);
 }
 
 int hils_select_backward(const hils_params *p, hils_ctensor Qcal, int Lq, hils_ctensor Ksum, int C,

@@ -104,7 +104,8 @@ struct BwdSummarizeArgs {
     int B, H, N, C, G;
     float scale;
 };
-hils_status launch_attend_backward(hils_dtype dt, int d, const BwdAttendArgs &a, cudaStream_t s);
+hils_status launch_attend_backward(hils_dtype dt, int d, const BwdAttendArgs &a, void *ws, cudaStream_t s);
+size_t attend_backward_ws_bytes(int B, int H, int Hk, int N, int K);
 hils_status launch_select_backward(hils_dtype dt, int d, const BwdSelectArgs &a, cudaStream_t s);
 hils_status launch_summarize_backward(hils_dtype dt, int d, const BwdSummarizeArgs &a, cudaStream_t s);
 

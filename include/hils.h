@@ -131,7 +131,8 @@ typedef enum {
     HILS_CALL_SELECT = 0,
     HILS_CALL_ATTEND_PREFILL = 1,
     HILS_CALL_ATTEND_DECODE = 2,
-    HILS_CALL_DECODE = 3
+    HILS_CALL_DECODE = 3,
+    HILS_CALL_ATTEND_BACKWARD = 4
 } hils_call;
 
 /* Landmark chunk summaries (summary page, Methodology 1, Eq. 8).
@@ -285,11 +286,15 @@ int hils_attend_decode_noalloc(const hils_params *p, hils_ctensor Q, hils_ctenso
  * with its outputs O [B,H,N,d] (dtype) and lse [B,H,N], and dO [B,H,N,d] float32.
  *   dQ     [B, H, N, d]   out (written)
  *   dK, dV [B, Hk, N, d]  accumulated
- *   dscore [B, H, N, K]   out: the gradient of each kept chunk's score, 0 padding */
+ *   dscore [B, H, N, K]   out: the gradient of each kept chunk's score, 0 padding
+ *   workspace, ws_bytes: hils_workspace_bytes(p, HILS_CALL_ATTEND_BACKWARD, N, 0) bytes
+ *         (the inverted index of the selection and D_i = dO_i . o_i), no initialisation
+ *         needed. */
 int hils_attend_prefill_backward(const hils_params *p, hils_ctensor Q, hils_ctensor K, hils_ctensor V, int N,
                                  const int32_t *idx, const float *score, const int32_t *nsel,
                                  hils_ctensor O, const float *lse, const float *dO,
-                                 float *dQ, float *dK, float *dV, float *dscore, cudaStream_t stream);
+                                 float *dQ, float *dK, float *dV, float *dscore, void *workspace,
+                                 size_t ws_bytes, cudaStream_t stream);
 
 /* Eq. 7 backward: dQcal [B,H,Lq,d] (written) = scale sum_k dscore_k k'_{idx_k};
  * dKsum [B,H,C,d] += scale dscore q~ and dBsum [B,H,C] += dscore (accumulated). */
