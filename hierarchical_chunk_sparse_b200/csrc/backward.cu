@@ -349,6 +349,254 @@ __global__ void __launch_bounds__(kThreads) attend_bwd_keymajor_kernel(BwdAttend
     }
 }
 
+// ---- the same key-major walk on the tensor cores (bf16 inputs): per step of 16 queries
+// the products S = Q K^T and T = dO V^T (16 x 64), dK += dl^T Q, dV += cv^T dO (64 x d)
+// and dQ += dl K (16 x d) are mma.sync m16n8k16 bf16 tiles with float32 accumulation; dO,
+// dl and cv enter them rounded to bf16. Warp w owns keys 16w..16w+15 of the block (its
+// dK and dV rows stay in registers for the whole walk) and a quarter of dQ's columns.
+
+__device__ __forceinline__ void bw_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void bw_ldsm4(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+__device__ __forceinline__ void bw_ldsm4t(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+
+template <int D>
+struct MmaCfg {
+    static constexpr int kLds = D + 8;       // bf16 row stride of K, V, Q, dO (rows 16 B apart mod 128)
+    static constexpr int kLdp = kChunk + 8;  // bf16 row stride of dl and cv
+    static constexpr int kSmemBytes =
+        (2 * kChunk * kLds + 2 * kQT * kLds + 2 * kQT * kLdp) * 2 + 2 * kQT * kChunk * 4 + 4 * kQT * 4;
+};
+
+template <int D, bool kChunkMode>
+__global__ void __launch_bounds__(kThreads) attend_bwd_mma_kernel(BwdAttendArgs a, const float *Dv,
+                                                                  const int *start, const int *entries) {
+    using Cfg = MmaCfg<D>;
+    constexpr int kLds = Cfg::kLds, kLdp = Cfg::kLdp, kNT = D / 8;
+    extern __shared__ __align__(16) uint8_t bsm[];
+    bf16 *kb = reinterpret_cast<bf16 *>(bsm), *vb = kb + kChunk * kLds;
+    bf16 *qb = vb + kChunk * kLds, *dob = qb + kQT * kLds;
+    bf16 *dlb = dob + kQT * kLds, *cvb = dlb + kQT * kLdp;             // [kQT][kLdp]
+    float *lg = reinterpret_cast<float *>(cvb + kQT * kLdp), *tj = lg + kQT * kChunk;  // [kQT][64]
+    float *q_lse = tj + kQT * kChunk, *q_D = q_lse + kQT, *q_w = q_D + kQT;
+    int *q_i = reinterpret_cast<int *>(q_w + kQT);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
+    const int blk = blockIdx.x;
+    const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+    const int Hk = a.H / a.G, hk = h / a.G, K = a.topk, C = a.N / kChunk;
+    const int j0 = blk * kChunk;
+    const int rows = min(kChunk, a.N - j0);
+    const bf16 *kbase = static_cast<const bf16 *>(a.K.ptr) + b * a.K.sb + hk * a.K.sh;
+    const bf16 *vbase = static_cast<const bf16 *>(a.V.ptr) + b * a.V.sb + hk * a.V.sh;
+    int q_begin, q_end;
+    const int *list = nullptr;
+    if (kChunkMode) {
+        const int64_t bg = (int64_t)b * Hk + hk;
+        q_begin = start[bg * (C + 1) + blk];
+        q_end = start[bg * (C + 1) + blk + 1];
+        list = entries + bg * (int64_t)a.N * K;
+    } else {
+        q_begin = j0;
+        q_end = a.W > 0 ? min(a.N, j0 + rows - 1 + a.W) : j0;
+    }
+    if (q_begin >= q_end) return;
+    for (int e = tid; e < kChunk * D; e += kThreads) {
+        const int j = e / D, x = e - (e / D) * D;
+        const bf16 z = __float2bfloat16(0.f);
+        kb[j * kLds + x] = j < rows ? kbase[(int64_t)(j0 + j) * a.K.st + x] : z;
+        vb[j * kLds + x] = j < rows ? vbase[(int64_t)(j0 + j) * a.V.st + x] : z;
+    }
+    float dka[kNT][4], dva[kNT][4];  // this warp's 16 keys x D columns
+#pragma unroll
+    for (int n = 0; n < kNT; ++n)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) dka[n][r] = dva[n][r] = 0.f;
+    const int64_t qhead = ((int64_t)b * a.H + h) * a.N;
+    for (int q0 = q_begin; q0 < q_end; q0 += kQT) {
+        const int nq = min(kQT, q_end - q0);
+        __syncthreads();
+        if (tid < kQT) {
+            int i = -1, k = 0;
+            float lse = -INFINITY, w = 0.f;
+            if (tid < nq) {
+                if (kChunkMode) {
+                    const int en = list[q0 + tid];
+                    i = en >> 5;
+                    k = en & 31;
+                } else {
+                    i = q0 + tid;
+                }
+                lse = a.lse[qhead + i];
+                if (kChunkMode && isfinite(lse)) w = expf(a.score[(qhead + i) * K + k] - lse);
+            }
+            q_i[tid] = isfinite(lse) ? (kChunkMode ? (i * 32 + k) : i) : -1;
+            q_lse[tid] = lse;
+            q_D[tid] = (i >= 0 && isfinite(lse)) ? Dv[qhead + i] : 0.f;
+            q_w[tid] = w;
+        }
+        __syncthreads();
+        for (int e = tid; e < kQT * D; e += kThreads) {
+            const int r = e / D, x = e - (e / D) * D;
+            const int en = q_i[r];
+            const int i = en < 0 ? -1 : (kChunkMode ? en >> 5 : en);
+            bf16 qv = __float2bfloat16(0.f), dv = qv;
+            if (i >= 0) {
+                qv = static_cast<const bf16 *>(a.Q.ptr)[b * a.Q.sb + h * a.Q.sh + (int64_t)i * a.Q.st + x];
+                dv = __float2bfloat16(a.dO[(qhead + i) * D + x]);
+            }
+            qb[r * kLds + x] = qv;
+            dob[r * kLds + x] = dv;
+        }
+        __syncthreads();
+        {  // S = Q K^T and T = dO V^T for this warp's 16 keys (two n-tiles of 8)
+            float sa[2][4] = {}, ta[2][4] = {};
+            const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t qa[4], da[4], kf[4], vf[4];
+                const int arow = rr + (mi & 1) * 8, acol = ks * 16 + (mi >> 1) * 8;
+                bw_ldsm4(qa, qb + arow * kLds + acol);
+                bw_ldsm4(da, dob + arow * kLds + acol);
+                const int brow = warp * 16 + (mi >> 1) * 8 + rr, bcol = ks * 16 + (mi & 1) * 8;
+                bw_ldsm4(kf, kb + brow * kLds + bcol);
+                bw_ldsm4(vf, vb + brow * kLds + bcol);
+                bw_mma(sa[0], qa, kf[0], kf[1]);
+                bw_mma(sa[1], qa, kf[2], kf[3]);
+                bw_mma(ta[0], da, vf[0], vf[1]);
+                bw_mma(ta[1], da, vf[2], vf[3]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int hv = 0; hv < 2; ++hv)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const int r = g + hv * 8, j = warp * 16 + nt * 8 + 2 * t4 + c;
+                        const int en = q_i[r];
+                        bool ok = en >= 0 && j < rows;
+                        if (!kChunkMode && ok) ok = j0 + j <= en && j0 + j > en - a.W;
+                        lg[r * kChunk + j] = ok ? sa[nt][hv * 2 + c] * a.scale : -INFINITY;
+                        tj[r * kChunk + j] = ok ? ta[nt][hv * 2 + c] : 0.f;
+                    }
+        }
+        __syncthreads();
+        {  // per query (a warp takes four): weights, scale * dl and cv as bf16, dscore
+#pragma unroll
+            for (int r4 = 0; r4 < kQT / 4; ++r4) {
+                const int r = warp * (kQT / 4) + r4;
+                const int en = q_i[r];
+                float d0 = 0.f, d1 = 0.f, c0 = 0.f, c1 = 0.f;
+                if (en >= 0) {  // warp-uniform
+                    const float l0 = lg[r * kChunk + lane], l1 = lg[r * kChunk + lane + 32];
+                    const float t0 = tj[r * kChunk + lane], t1 = tj[r * kChunk + lane + 32];
+                    const float Di = q_D[r];
+                    if (kChunkMode) {
+                        const float m = warp_max(fmaxf(l0, l1));
+                        const float e0 = expf(l0 - m), e1 = expf(l1 - m);
+                        const float inv = 1.f / warp_sum(e0 + e1);
+                        const float p0 = e0 * inv, p1 = e1 * inv;
+                        const float oc = warp_sum(p0 * t0 + p1 * t1);
+                        const float wc = q_w[r];
+                        d0 = wc * p0 * (t0 - oc);
+                        d1 = wc * p1 * (t1 - oc);
+                        c0 = wc * p0;
+                        c1 = wc * p1;
+                        if (lane == 0) a.dscore[(qhead + (en >> 5)) * K + (en & 31)] = wc * (oc - Di);
+                    } else {
+                        const float lse = q_lse[r];
+                        c0 = expf(l0 - lse);
+                        c1 = expf(l1 - lse);
+                        d0 = c0 * (t0 - Di);
+                        d1 = c1 * (t1 - Di);
+                    }
+                }
+                dlb[r * kLdp + lane] = __float2bfloat16(a.scale * d0);
+                dlb[r * kLdp + lane + 32] = __float2bfloat16(a.scale * d1);
+                cvb[r * kLdp + lane] = __float2bfloat16(c0);
+                cvb[r * kLdp + lane + 32] = __float2bfloat16(c1);
+            }
+        }
+        __syncthreads();
+        {  // dK += (scale dl)^T Q and dV += cv^T dO for this warp's keys: A = dl^T from the
+           // [query][key] array (transposed load), B = Q / dO rows (transposed load)
+            const int mi = lane >> 3, rr = lane & 7;
+            uint32_t af[4], cf[4];
+            const int arow = rr + (mi >> 1) * 8, acol = warp * 16 + (mi & 1) * 8;
+            bw_ldsm4t(af, dlb + arow * kLdp + acol);
+            bw_ldsm4t(cf, cvb + arow * kLdp + acol);
+#pragma unroll
+            for (int n2 = 0; n2 < kNT / 2; ++n2) {
+                uint32_t qf4[4], df4[4];
+                const int brow = rr + (mi & 1) * 8, bcol = n2 * 16 + (mi >> 1) * 8;
+                bw_ldsm4t(qf4, qb + brow * kLds + bcol);
+                bw_ldsm4t(df4, dob + brow * kLds + bcol);
+                bw_mma(dka[2 * n2], af, qf4[0], qf4[1]);
+                bw_mma(dka[2 * n2 + 1], af, qf4[2], qf4[3]);
+                bw_mma(dva[2 * n2], cf, df4[0], df4[1]);
+                bw_mma(dva[2 * n2 + 1], cf, df4[2], df4[3]);
+            }
+        }
+        {  // dQ share: (scale dl) K for this warp's quarter of the columns
+            constexpr int kWn = kNT / 4;  // n-tiles per warp
+            float qa2[kWn][4] = {};
+            const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+            for (int ks = 0; ks < kChunk / 16; ++ks) {
+                uint32_t af[4];
+                bw_ldsm4(af, dlb + (rr + (mi & 1) * 8) * kLdp + ks * 16 + (mi >> 1) * 8);
+#pragma unroll
+                for (int n2 = 0; n2 < kWn; n2 += 2) {
+                    uint32_t kf4[4];
+                    const int ncol = warp * kWn * 8 + n2 * 8;
+                    bw_ldsm4t(kf4, kb + (ks * 16 + rr + (mi & 1) * 8) * kLds + ncol + (mi >> 1) * 8);
+                    bw_mma(qa2[n2], af, kf4[0], kf4[1]);
+                    if (n2 + 1 < kWn) bw_mma(qa2[n2 + 1], af, kf4[2], kf4[3]);
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < kWn; ++n)
+#pragma unroll
+                for (int hv = 0; hv < 2; ++hv) {
+                    const int r = g + hv * 8, en = q_i[r];
+                    if (en < 0) continue;
+                    const int i = kChunkMode ? en >> 5 : en;
+                    float *dst = a.dQ + (qhead + i) * D + warp * kWn * 8 + n * 8 + 2 * t4;
+                    atomicAdd(dst, qa2[n][hv * 2]);
+                    atomicAdd(dst + 1, qa2[n][hv * 2 + 1]);
+                }
+        }
+    }
+    // this warp's keys' dK and dV into the global arrays
+    float *dkb = a.dK + ((int64_t)b * Hk + hk) * a.N * D;
+    float *dvb = a.dV + ((int64_t)b * Hk + hk) * a.N * D;
+#pragma unroll
+    for (int n = 0; n < kNT; ++n)
+#pragma unroll
+        for (int hv = 0; hv < 2; ++hv) {
+            const int j = warp * 16 + g + hv * 8;
+            if (j >= rows) continue;
+            float *pk = dkb + (int64_t)(j0 + j) * D + n * 8 + 2 * t4;
+            float *pv = dvb + (int64_t)(j0 + j) * D + n * 8 + 2 * t4;
+            atomicAdd(pk, dka[n][hv * 2]);
+            atomicAdd(pk + 1, dka[n][hv * 2 + 1]);
+            atomicAdd(pv, dva[n][hv * 2]);
+            atomicAdd(pv + 1, dva[n][hv * 2 + 1]);
+        }
+}
+
 // grid: B*H*Lq, one query each: Eq. 7 backward.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) select_backward_kernel(BwdSelectArgs a) {
@@ -463,11 +711,17 @@ hils_status launch_attend_bwd(const BwdAttendArgs &a, void *ws, cudaStream_t s) 
         if (st != HILS_OK) return st;
     }
     bwd_dot_kernel<T, D><<<(unsigned)((nq + 3) / 4), kThreads, 0, s>>>(a, w.D);
-    constexpr int smem = KmCfg<T, D>::kSmemBytes;
+    // bf16: the tensor-core walk; float32: the CUDA-core walk (full float32 products)
+    constexpr bool kMma = sizeof(T) == 2;
+    constexpr int smem = kMma ? MmaCfg<D>::kSmemBytes : KmCfg<T, D>::kSmemBytes;
+    const void *fw = kMma ? (const void *)attend_bwd_mma_kernel<D, false>
+                          : (const void *)attend_bwd_keymajor_kernel<T, D, false>;
+    const void *fc = kMma ? (const void *)attend_bwd_mma_kernel<D, true>
+                          : (const void *)attend_bwd_keymajor_kernel<T, D, true>;
     static KernelSetup setup_w, setup_c;
-    st = kernel_setup(setup_w, (const void *)attend_bwd_keymajor_kernel<T, D, false>, kThreads, smem, nullptr);
+    st = kernel_setup(setup_w, fw, kThreads, smem, nullptr);
     if (st != HILS_OK) return st;
-    st = kernel_setup(setup_c, (const void *)attend_bwd_keymajor_kernel<T, D, true>, kThreads, smem, nullptr);
+    st = kernel_setup(setup_c, fc, kThreads, smem, nullptr);
     if (st != HILS_OK) return st;
     if (a.topk > 0 && C > 0) {
         const int64_t ne = (int64_t)a.B * Hk * a.N * a.topk;
@@ -476,12 +730,17 @@ hils_status launch_attend_bwd(const BwdAttendArgs &a, void *ws, cudaStream_t s) 
         bwd_count_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.count);
         bwd_scan_kernel<<<(unsigned)(a.B * Hk), 1024, 0, s>>>(C, w.count, w.start, w.cursor);
         bwd_scatter_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.cursor, w.entries);
-        attend_bwd_keymajor_kernel<T, D, true><<<dim3(C, a.B * a.H), kThreads, smem, s>>>(a, w.D, w.start,
-                                                                                            w.entries);
+        if constexpr (kMma)
+            attend_bwd_mma_kernel<D, true><<<dim3(C, a.B * a.H), kThreads, smem, s>>>(a, w.D, w.start, w.entries);
+        else
+            attend_bwd_keymajor_kernel<T, D, true><<<dim3(C, a.B * a.H), kThreads, smem, s>>>(a, w.D, w.start,
+                                                                                                w.entries);
     }
-    if (a.W > 0)
-        attend_bwd_keymajor_kernel<T, D, false><<<dim3((a.N + kChunk - 1) / kChunk, a.B * a.H), kThreads, smem, s>>>(
-            a, w.D, nullptr, nullptr);
+    if (a.W > 0) {
+        const dim3 grid((a.N + kChunk - 1) / kChunk, a.B * a.H);
+        if constexpr (kMma) attend_bwd_mma_kernel<D, false><<<grid, kThreads, smem, s>>>(a, w.D, nullptr, nullptr);
+        else attend_bwd_keymajor_kernel<T, D, false><<<grid, kThreads, smem, s>>>(a, w.D, nullptr, nullptr);
+    }
     return record_cuda_error(cudaGetLastError());
 }
 

@@ -5,8 +5,8 @@ then give dscore, dQ, dK, dV, dQcal, dKsum, dBsum and dLQ, each compared with th
 oracle's gradient of sum(O * dO) for the same selection. Bars, as relative L2 error of
 each gradient: float32 inputs 1e-5 (float32 arithmetic and atomic accumulation order;
 observed about 5e-7); bf16 inputs 1e-2, the forward's bar (the forward's O and summary
-table are stored in bf16, which moves D_i and the chunk scores by up to 2^-9 relative;
-observed about 2e-3)."""
+table are stored in bf16, which moves D_i and the chunk scores by up to 2^-9 relative,
+and the tensor-core products take dO, dl and cv rounded to bf16; observed about 3e-3)."""
 import numpy as np
 import pytest
 import torch
