@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import hierarchical_chunk_sparse_b200 as hils
 from hierarchical_chunk_sparse_b200 import build as hbuild
@@ -193,3 +194,82 @@ def test_window_exclusion_flag_accepted(lib):
     assert lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_SELECT, 1, 8000) > 0
     c.flags = 2
     assert lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_SELECT, 1, 8000) == 0
+
+
+class _OnDevice:
+    """Stands in for a CUDA tensor in the binding's argument checks (shape, dtype and
+    device are all they read before the C call)."""
+
+    is_cuda = True
+
+    def __init__(self, *shape, dtype=torch.bfloat16):
+        self.shape = torch.Size(shape)
+        self.dtype = dtype
+
+    def is_contiguous(self):
+        return True
+
+
+def test_grouped_query_shapes_checked_by_the_binding():
+    """With H_kv, the binding expects idx/nsel and K/V with the key-value heads and score
+    with the query heads; a tensor with the wrong head count is refused before any C
+    call."""
+    D = _OnDevice
+    p = hils.Params(B=1, H=8, d=128, K=4, W=64, dtype=torch.bfloat16, H_kv=2)
+    assert p.Hk == 2
+    Q, Ksum, Bsum = D(1, 8, 300, 128), D(1, 8, 4, 128), D(1, 8, 4, dtype=torch.float32)
+    idx_ok, nsel = D(1, 2, 300, 4, dtype=torch.int32), D(1, 2, 300, dtype=torch.int32)
+    score = D(1, 8, 300, 4, dtype=torch.float32)
+    with pytest.raises(ValueError, match="idx has shape"):
+        hils.hils_select(p, Q, Ksum, Bsum, D(1, 8, 300, 4, dtype=torch.int32), score, nsel)
+    with pytest.raises(ValueError, match="score has shape"):
+        hils.hils_select(p, Q, Ksum, Bsum, idx_ok, D(1, 2, 300, 4, dtype=torch.float32), nsel)
+    with pytest.raises(ValueError, match="nsel has shape"):
+        hils.hils_select(p, Q, Ksum, Bsum, idx_ok, score, D(1, 8, 300, dtype=torch.int32))
+    with pytest.raises(ValueError, match="K has shape"):
+        hils.hils_attend_prefill(p, Q, D(1, 8, 300, 128), D(1, 2, 300, 128), idx_ok, score, nsel, Q)
+    with pytest.raises(ValueError, match="hils_summarize: K has shape"):
+        hils.hils_summarize(p, D(1, 8, 300, 128), D(1, 8, 4, 128), Ksum, Bsum)
+    with pytest.raises(ValueError, match="Kc has shape"):
+        hils.hils_attend_decode(p, D(1, 8, 1, 128), D(1, 8, 5000, 128), D(1, 2, 5000, 128),
+                                D(1, dtype=torch.int32), D(1, 2, 1, 4, dtype=torch.int32),
+                                D(1, 8, 1, 4, dtype=torch.float32), D(1, 2, 1, dtype=torch.int32), D(1, 8, 1, 128))
+
+
+def test_backward_binding_checks():
+    """The backward calls want float32 dense gradients of the forward's shapes."""
+    D = _OnDevice
+    p = hils.Params(B=1, H=2, d=64, K=3, W=64, dtype=torch.bfloat16)
+    N = 200
+    Q = D(1, 2, N, 64)
+    idx, nsel = D(1, 2, N, 3, dtype=torch.int32), D(1, 2, N, dtype=torch.int32)
+    score, lse = D(1, 2, N, 3, dtype=torch.float32), D(1, 2, N, dtype=torch.float32)
+    g = D(1, 2, N, 64, dtype=torch.float32)
+    with pytest.raises(ValueError, match="dscore has shape"):
+        hils.hils_attend_prefill_backward(p, Q, Q, Q, idx, score, nsel, Q, lse, g, g, g, g,
+                                          D(1, 2, N, 4, dtype=torch.float32))
+    with pytest.raises(ValueError, match="dQ has dtype"):
+        hils.hils_attend_prefill_backward(p, Q, Q, Q, idx, score, nsel, Q, lse, g, D(1, 2, N, 64), g, g,
+                                          D(1, 2, N, 3, dtype=torch.float32))
+    with pytest.raises(ValueError, match="dKsum has shape"):
+        hils.hils_select_backward(p, Q, D(1, 2, 3, 64), idx, nsel, score, g, D(1, 2, 4, 64, dtype=torch.float32),
+                                  D(1, 2, 3, dtype=torch.float32))
+    with pytest.raises(ValueError, match="dLQ has shape"):
+        hils.hils_summarize_backward(p, Q, D(1, 2, 3, 64), D(1, 2, 3, 64, dtype=torch.float32),
+                                     D(1, 2, 3, dtype=torch.float32), g, D(1, 2, 4, 64, dtype=torch.float32))
+
+
+def test_backward_workspace_size(lib):
+    """HILS_CALL_ATTEND_BACKWARD: D_i per query, then per (b, group) chunk counts, starts,
+    cursors and the inverted index, each part rounded up to 256 bytes."""
+    p = hils.Params(B=2, H=4, d=128, K=16, W=512, dtype=torch.bfloat16, H_kv=2)
+    c = p.c()
+    N = 8192
+    C = N // 64
+
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    want = a256(2 * 4 * N * 4) + a256(2 * 2 * C * 4) + a256(2 * 2 * (C + 1) * 4) + a256(2 * 2 * C * 4) + \
+        a256(2 * 2 * N * 16 * 4)
+    assert lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_ATTEND_BACKWARD, N, 0) == want
