@@ -1,5 +1,5 @@
 /*
- * libhils: HiLS-Attention forward pass on NVIDIA B200 (sm_100a). C ABI.
+ * libhils: HiLS-Attention forward pass (and its backward) on NVIDIA B200 (sm_100a). C ABI.
  *
  * The method is Hierarchical Landmark Sparse attention, from "Hierarchical Sparse
  * Attention Done Right: Toward Infinite Context Modeling" (arXiv 2607.02980). The
@@ -14,6 +14,10 @@
  *   hils_attend_decode   window, for every position of a sequence, or for one new token
  *                        per sequence against a KV cache            (summary, Methodology 2, Eq. 10;
  *                                                                     post, pseudocode figure)
+ *   hils_decode          one decode step: hils_select then hils_attend_decode, chained
+ *   hils_summarize_append  decode-time summary of the chunk each newest token completed
+ *   hils_attend_prefill_backward, hils_select_backward, hils_summarize_backward
+ *                        gradients for a fixed selection            (Eq. 10, Eq. 7, Eq. 8)
  *
  * Conventions shared by every call
  * --------------------------------
