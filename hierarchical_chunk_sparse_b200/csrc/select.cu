@@ -92,9 +92,13 @@ __global__ void __launch_bounds__(kWarpKernelThreads) select_warp_kernel(SelectA
 // at least T - e_max and every chunk with hi < T - e_max is certainly out. Only the
 // groups whose max s + max e reaches that cut are read again; their candidates
 // (typically K + a few) are screened again on CUDA cores with the tight radius and go
-// through the exact interval top-K in one warp. With fewer than K+1 groups the exact
-// running-list scan runs over every chunk instead. Heavy ties (more than 64
-// candidates) fall back to folding the candidates in batches of 32, always exact.
+// through the exact interval top-K in one warp; for grouped heads (one CTA per (b,
+// group, query)) every candidate gets each head's float64 score instead, one thread per
+// (head, candidate), and a parallel rank of the group maxima keeps the top K. With fewer
+// than K+1 groups the exact running-list scan runs over every chunk instead. Heavy ties
+// (more than 64 candidates) fall back to folding the candidates in batches of 32, always
+// exact. The (K+1)-th group maximum is found by a parallel rank count over at most 256
+// values.
 
 constexpr int kScrThreads = 256;
 constexpr int kPickThreads = 256;

@@ -1,6 +1,7 @@
-// Exact top-K pick of one decode query from the screen values of the decode select
-// ("Hierarchical Sparse Attention Done Right" (picx.dev summary), Eq. 7 and
-// Methodology 2; rcap.io post, pseudocode figure), for the decode select's pick kernel.
+// Exact top-K pick of one decode query, or of one (b, group, query) for grouped heads
+// (summary page, Methodology 3), from the screen values of the decode select ("Hierarchical
+// Sparse Attention Done Right" (picx.dev summary), Eq. 7 and Methodology 2; rcap.io post,
+// pseudocode figure), for the decode select's pick kernel.
 //
 // Workspace of the decode select: a 256-byte status header, then the screen value and
 // radius (s_c, e_c) of every eligible chunk per query, then the largest s and e of every
