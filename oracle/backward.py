@@ -39,43 +39,48 @@ def summaries(K, LQ, S: int, scale: float):
     return Ksum, Bsum
 
 
-def forward(Q, K, V, Qcal, LQ, idx, nsel, S: int, W: int, scale: float):
-    """Eq. 8 -> Eq. 7 (kept chunks) -> Eq. 10. Returns O [B,H,N,d], lse [B,H,N] and the
-    kept chunks' scores [B,H,N,Kk] (padding -inf), with Ksum and Bsum."""
+def forward(Q, K, V, Qcal, LQ, idx, nsel, S: int, W: int, scale: float, rows=None):
+    """Eq. 8 -> Eq. 7 (kept chunks) -> Eq. 10. Returns O [B,H,R,d], lse [B,H,R] and the
+    kept chunks' scores [B,H,R,Kk] (padding -inf), with Ksum and Bsum, for the query rows
+    ``rows`` (a 1-D index array; all N rows when None). Query row i's output depends on
+    Q_i, Qcal_i and its own selection only, so a subset of rows gives those rows'
+    outputs exactly, and the gradients of a sum over rows add up over disjoint subsets."""
     B, H, N, d = Q.shape
     Hk = K.shape[1]
     G = H // Hk
     Ksum, Bsum = summaries(K, LQ, S, scale)
     C = LQ.shape[2]
-    idx = torch.as_tensor(np.asarray(idx), dtype=torch.int64).reshape(B, Hk, N, -1)
-    nsel = torch.as_tensor(np.asarray(nsel), dtype=torch.int64).reshape(B, Hk, N)
+    rows = torch.arange(N) if rows is None else torch.as_tensor(np.asarray(rows), dtype=torch.int64).reshape(-1)
+    R = rows.numel()
+    idx = torch.as_tensor(np.asarray(idx), dtype=torch.int64).reshape(B, Hk, N, -1)[:, :, rows]
+    nsel = torch.as_tensor(np.asarray(nsel), dtype=torch.int64).reshape(B, Hk, N)[:, :, rows]
+    Qr, Qcr = Q[:, :, rows], Qcal[:, :, rows]
     Kk = idx.shape[-1]
-    idx_h = idx.repeat_interleave(G, dim=1)  # [B,H,N,Kk]
+    idx_h = idx.repeat_interleave(G, dim=1)  # [B,H,R,Kk]
     nsel_h = nsel.repeat_interleave(G, dim=1)
     kept = (torch.arange(Kk).view(1, 1, 1, Kk) < nsel_h.unsqueeze(-1)) & (idx_h >= 0)
     cidx = idx_h.clamp(min=0, max=max(C - 1, 0))
     # Eq. 7: s^ = scale q~ . k'_c + b'_c of each kept chunk
-    ks = torch.gather(Ksum, 2, cidx.reshape(B, H, N * Kk, 1).expand(B, H, N * Kk, d)).reshape(B, H, N, Kk, d)
-    bs = torch.gather(Bsum, 2, cidx.reshape(B, H, N * Kk)).reshape(B, H, N, Kk)
-    score = scale * torch.einsum("bhnd,bhnkd->bhnk", Qcal, ks) + bs
+    ks = torch.gather(Ksum, 2, cidx.reshape(B, H, R * Kk, 1).expand(B, H, R * Kk, d)).reshape(B, H, R, Kk, d)
+    bs = torch.gather(Bsum, 2, cidx.reshape(B, H, R * Kk)).reshape(B, H, R, Kk)
+    score = scale * torch.einsum("bhnd,bhnkd->bhnk", Qcr, ks) + bs
     score = torch.where(kept, score, torch.full_like(score, -torch.inf))
     # token logits and the sliding window [max(0, i-W+1), i]
     Kh = K.repeat_interleave(G, dim=1)
     Vh = V.repeat_interleave(G, dim=1)
-    L = scale * torch.einsum("bhid,bhjd->bhij", Q, Kh)
-    i = torch.arange(N).view(N, 1)
+    L = scale * torch.einsum("bhid,bhjd->bhij", Qr, Kh)  # [B,H,R,N]
+    i = rows.view(R, 1)
     j = torch.arange(N).view(1, N)
     win = (j <= i) & (j > i - W)
     Lw = torch.where(win, L, torch.full_like(L, -torch.inf))
     # each kept chunk's own softmax output o_c over its S tokens
-    tok = cidx.unsqueeze(-1) * S + torch.arange(S).view(1, 1, 1, 1, S)  # [B,H,N,Kk,S]
-    Lc = torch.gather(L.unsqueeze(3).expand(B, H, N, Kk, N), 4, tok)
+    tok = cidx.unsqueeze(-1) * S + torch.arange(S).view(1, 1, 1, 1, S)  # [B,H,R,Kk,S]
+    Lc = torch.gather(L, 3, tok.reshape(B, H, R, Kk * S)).reshape(B, H, R, Kk, S)
     pc = torch.softmax(Lc, dim=-1)
-    Vc = torch.gather(Vh.unsqueeze(2).unsqueeze(2).expand(B, H, N, Kk, N, d), 4,
-                      tok.unsqueeze(-1).expand(B, H, N, Kk, S, d))
+    Vc = Vh[torch.arange(B).view(B, 1, 1, 1, 1), torch.arange(H).view(1, H, 1, 1, 1), tok]  # [B,H,R,Kk,S,d]
     oc = torch.einsum("bhnks,bhnksd->bhnkd", pc, Vc)
     # Eq. 10: one normaliser over the kept chunks' masses and the window's tokens
-    masses = torch.cat([score, Lw], dim=-1)  # [B,H,N,Kk+N]
+    masses = torch.cat([score, Lw], dim=-1)  # [B,H,R,Kk+N]
     lse = torch.logsumexp(masses, dim=-1)
     finite = torch.isfinite(lse)
     lse_safe = torch.where(finite, lse, torch.zeros_like(lse))
@@ -86,21 +91,37 @@ def forward(Q, K, V, Qcal, LQ, idx, nsel, S: int, W: int, scale: float):
     return O, lse, score, Ksum, Bsum
 
 
-def grads(Q, K, V, Qcal, LQ, idx, nsel, dO, S: int, W: int, scale: float):
+def grads(Q, K, V, Qcal, LQ, idx, nsel, dO, S: int, W: int, scale: float, batch=None):
     """Gradients of sum(O * dO) for the given selection: a dict with dQ, dK, dV, dQcal,
     dLQ (the inputs), and the intermediate dscore [B,H,N,Kk] (0 padding), dKsum, dBsum,
-    with the forward's O and lse."""
+    with the forward's O and lse. With ``batch`` set, the forward and backward run over
+    consecutive blocks of that many query rows and the gradients are summed over the
+    blocks (the loss is a sum over rows), which bounds the memory at long sequences."""
     leaves = [_t(x).clone().requires_grad_(True) for x in (Q, K, V, Qcal, LQ)]
     Qd, Kd, Vd, Qcd, LQd = leaves
-    O, lse, score, Ksum, Bsum = forward(Qd, Kd, Vd, Qcd, LQd, idx, nsel, S, W, scale)
-    score.retain_grad()
-    Ksum.retain_grad()
-    Bsum.retain_grad()
-    (O * _t(dO)).sum().backward()
-    out = {name: leaf.grad.detach() for name, leaf in zip(("dQ", "dK", "dV", "dQcal", "dLQ"), leaves)}
-    ds = score.grad.detach() if score.grad is not None else torch.zeros_like(score)
-    out["dscore"] = torch.where(torch.isfinite(score.detach()), ds, torch.zeros_like(ds))
-    out["dKsum"] = Ksum.grad.detach() if Ksum.grad is not None else torch.zeros_like(Ksum)
-    out["dBsum"] = Bsum.grad.detach() if Bsum.grad is not None else torch.zeros_like(Bsum)
-    out["O"], out["lse"] = O.detach(), lse.detach()
+    dO = _t(dO)
+    B, H, N, d = Q.shape
+    Kk = np.asarray(idx).shape[-1]
+    C = LQ.shape[2]
+    f64 = dict(dtype=torch.float64)
+    out = {"dscore": torch.zeros(B, H, N, Kk, **f64), "dKsum": torch.zeros(B, H, C, d, **f64),
+           "dBsum": torch.zeros(B, H, C, **f64), "O": torch.zeros(B, H, N, d, **f64),
+           "lse": torch.zeros(B, H, N, **f64)}
+    step = N if batch is None else int(batch)
+    for r0 in range(0, N, step):
+        rows = torch.arange(r0, min(N, r0 + step))
+        O, lse, score, Ksum, Bsum = forward(Qd, Kd, Vd, Qcd, LQd, idx, nsel, S, W, scale, rows=rows)
+        score.retain_grad()
+        Ksum.retain_grad()
+        Bsum.retain_grad()
+        (O * dO[:, :, rows]).sum().backward()
+        if score.grad is not None:
+            out["dscore"][:, :, rows] = torch.where(torch.isfinite(score.detach()), score.grad, torch.zeros_like(score))
+        if Ksum.grad is not None:
+            out["dKsum"] += Ksum.grad
+        if Bsum.grad is not None:
+            out["dBsum"] += Bsum.grad
+        out["O"][:, :, rows], out["lse"][:, :, rows] = O.detach(), lse.detach()
+    for name, leaf in zip(("dQ", "dK", "dV", "dQcal", "dLQ"), leaves):
+        out[name] = leaf.grad.detach() if leaf.grad is not None else torch.zeros_like(leaf.detach())
     return out

@@ -74,3 +74,63 @@ def test_backward_matches_oracle(cuda_device, case):
     # padding of dscore is exactly zero
     kept = torch.arange(K, device=cuda_device).view(1, 1, 1, K) < nsel.repeat_interleave(w.G, dim=1).unsqueeze(-1)
     assert (dscore[~kept] == 0).all()
+
+
+FULL = {
+    # the 8K prefill (B1 H32 d128 N8192, K16, W512): two sampled query heads
+    "prefill8k": (2, 2),
+    # the grouped 8K prefill (32 query heads, 8 key-value heads): one sampled group
+    "prefill8k_grouped": (7, 1),
+}
+
+
+@pytest.mark.parametrize("case", list(FULL))
+def test_backward_full_size(cuda_device, case):
+    """The 8K prefill backward at full size, in the launch configuration the benchmark
+    times (forward chain, then the three backward calls with an allocated workspace):
+    for sampled key-value heads, every gradient of that head's slice (dscore, dQ, dQcal
+    of its query heads; dK, dV; dKsum, dBsum, dLQ) against the float64 oracle, which
+    runs over blocks of 256 query rows and sums the blocks' gradients. Heads and groups
+    are independent, so a slice's gradients are its own problem's. Bar as above for
+    bf16 inputs."""
+    wid, nsample = FULL[case]
+    w = WORKLOADS[wid]
+    inp = make_prefill(w)
+    d = to_dev(inp, cuda_device)
+    Ksum, Bsum = gpu_summarize(w, d["K"], d["LQ"])
+    idx, score, nsel = gpu_select(w, d["Qcal"], Ksum, Bsum)
+    O, lse = gpu_prefill(w, d["Q"], d["K"], d["V"], idx, score, nsel)
+    g = torch.Generator().manual_seed(17)
+    dO = torch.randn(O.shape, generator=g).to(cuda_device)
+    p = P(w)
+    B, H, N, dd, Hk, K, C, G = w.B, w.H, w.N, w.d, w.Hkv, w.K, w.C, w.G
+    f32 = dict(dtype=torch.float32, device=cuda_device)
+    dQ, dK, dV = torch.empty(B, H, N, dd, **f32), torch.zeros(B, Hk, N, dd, **f32), torch.zeros(B, Hk, N, dd, **f32)
+    dscore, dQcal = torch.empty(B, H, N, K, **f32), torch.empty(B, H, N, dd, **f32)
+    dKsum, dBsum, dLQ = torch.zeros(B, H, C, dd, **f32), torch.zeros(B, H, C, **f32), torch.empty(B, H, C, dd, **f32)
+    ws = hils.alloc_workspace(p, hils.HILS_CALL_ATTEND_BACKWARD, N, 0, device=cuda_device)
+    hils.hils_attend_prefill_backward(p, d["Q"], d["K"], d["V"], idx, score, nsel, O, lse, dO, dQ, dK, dV, dscore,
+                                      workspace=ws)
+    hils.hils_select_backward(p, d["Qcal"], Ksum, idx, nsel, dscore, dQcal, dKsum, dBsum)
+    hils.hils_summarize_backward(p, d["K"], d["LQ"], dKsum, dBsum, dK, dLQ)
+    torch.cuda.synchronize()
+    kept = torch.arange(K, device=cuda_device).view(1, 1, 1, K) < nsel.repeat_interleave(G, dim=1).unsqueeze(-1)
+    assert (dscore[~kept] == 0).all()
+    dO_h = host(dO)
+    for hk in torch.randperm(Hk, generator=g)[:nsample].tolist():
+        qs, ks = slice(hk * G, (hk + 1) * G), slice(hk, hk + 1)
+        ref = ob.grads(inp["Q"][:, qs], inp["K"][:, ks], inp["V"][:, ks], inp["Qcal"][:, qs], inp["LQ"][:, qs],
+                       host(idx[:, ks]), host(nsel[:, ks]), dO_h[:, qs], 64, w.W, w.scale, batch=256)
+        errs = {
+            "dscore": _rel(dscore[:, qs], ref["dscore"]),
+            "dQ": _rel(dQ[:, qs], ref["dQ"]),
+            "dQcal": _rel(dQcal[:, qs], ref["dQcal"]),
+            "dK": _rel(dK[:, ks], ref["dK"]),
+            "dV": _rel(dV[:, ks], ref["dV"]),
+            "dKsum": _rel(dKsum[:, qs], ref["dKsum"]),
+            "dBsum": _rel(dBsum[:, qs], ref["dBsum"]),
+            "dLQ": _rel(dLQ[:, qs], ref["dLQ"]),
+        }
+        print(case, hk, {k: f"{v:.2e}" for k, v in errs.items()})
+        bad = {k: v for k, v in errs.items() if not v <= 1e-2}
+        assert not bad, f"kv head {hk}: relative L2 errors above 1e-2: {bad} (all: {errs})"

@@ -125,3 +125,40 @@ def test_gradients_match_finite_differences_elementwise():
 
     ins = [x.clone().requires_grad_(True) for x in (Q, Kc, Vc, Qcal, LQ)]
     assert torch.autograd.gradcheck(f, ins, eps=1e-6, atol=1e-7, rtol=1e-5)
+
+
+@pytest.mark.parametrize("G,W,batch", [(1, 60, 50), (2, 90, 64), (1, 0, 7)])
+def test_row_blocks_give_the_same_gradients(G, W, batch):
+    """The row-block form used at long sequences: forward over a subset of rows equals
+    those rows of the full forward, and gradients summed over row blocks (a block size
+    that does not divide N) equal the gradients of the whole problem."""
+    Q, Kc, Vc, Qcal, LQ, idx, nsel = _problem(H=2, G=G, N=64 * 4 + 21, d=8, K=3, seed=50 + G)
+    dO = _rand(*Q.shape, seed=51)
+    full = ob.grads(Q, Kc, Vc, Qcal, LQ, idx, nsel, dO, S, W, 0.45)
+    blk = ob.grads(Q, Kc, Vc, Qcal, LQ, idx, nsel, dO, S, W, 0.45, batch=batch)
+    for name in ("dQ", "dK", "dV", "dQcal", "dLQ", "dscore", "dKsum", "dBsum", "O"):
+        assert torch.allclose(blk[name], full[name], atol=1e-12, rtol=0), name
+    fin = torch.isfinite(full["lse"])
+    assert torch.equal(torch.isfinite(blk["lse"]), fin)
+    assert torch.allclose(blk["lse"][fin], full["lse"][fin], atol=1e-12, rtol=0)
+    rows = np.array([0, 5, 64, 65, 200, Q.shape[2] - 1])
+    O, lse, score, _, _ = ob.forward(Q, Kc, Vc, Qcal, LQ, idx, nsel, S, W, 0.45, rows=rows)
+    assert torch.allclose(O, full["O"][:, :, rows], atol=1e-12, rtol=0)
+
+
+def test_key_value_head_slices_are_independent_problems():
+    """Each key-value head with its G query heads is a problem of its own: the gradients
+    of a slice computed alone equal that slice of the whole problem's gradients (the
+    form the full-size GPU test compares on)."""
+    G = 2
+    Q, Kc, Vc, Qcal, LQ, idx, nsel = _problem(H=4, G=G, N=64 * 3 + 11, d=8, K=2, seed=60)
+    dO = _rand(*Q.shape, seed=61)
+    full = ob.grads(Q, Kc, Vc, Qcal, LQ, idx, nsel, dO, S, 80, 0.5)
+    hk = 1
+    qs, ks = slice(hk * G, (hk + 1) * G), slice(hk, hk + 1)
+    part = ob.grads(Q[:, qs], Kc[:, ks], Vc[:, ks], Qcal[:, qs], LQ[:, qs], idx[:, ks], nsel[:, ks], dO[:, qs], S, 80,
+                    0.5, batch=64)
+    for name in ("dQ", "dQcal", "dLQ", "dscore", "dKsum", "dBsum"):
+        assert torch.allclose(part[name], full[name][:, qs], atol=1e-12, rtol=0), name
+    for name in ("dK", "dV"):
+        assert torch.allclose(part[name], full[name][:, ks], atol=1e-12, rtol=0), name
