@@ -73,3 +73,26 @@ def test_single_rank_needs_no_process_group():
     assert bench.max_over_ranks(4.5, 1, torch.device("cpu")) == 4.5
     bench.barrier(1)
     assert bench.job_throughput(units_per_rank=1, world=1, ms_per_step=0.5) == pytest.approx(2000.0)
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` at N=1 runs on the host cores only: one JSON line with
+    the arm's metric, unit and workload, the oracle's throughput as `value`, a
+    `cpu_baseline` describing the run and an `e2e` with no host-device bytes, and at
+    least three warm-up steps whatever is asked."""
+    import subprocess
+
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["n_gpus"] == 1 and j["steps"] == 1 and j["warmup"] >= 3
+    assert j["unit"] == "tokens/s" and j["higher_is_better"] is True and j["value"] > 0
+    assert j["ms_per_step"] > 0 and j["dtype"] == "f64" and j["data"] == "synthetic"
+    assert j["config"]["workload"] == "decode_bf16_512k" and j["config"]["kv_len"] == 524288
+    cb = j["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == j["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert j["e2e"] == {"value": j["value"], "unit": j["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
