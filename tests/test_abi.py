@@ -273,3 +273,42 @@ def test_backward_workspace_size(lib):
     want = a256(2 * 4 * N * 4) + a256(2 * 2 * C * 4) + a256(2 * 2 * (C + 1) * 4) + a256(2 * 2 * C * 4) + \
         a256(2 * 2 * N * 16 * 4)
     assert lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_ATTEND_BACKWARD, N, 0) == want
+
+
+def test_decode_time_and_backward_entry_points_validate_first(lib):
+    """hils_summarize_append and the three backward calls reject bad arguments with the
+    documented codes before any launch: null arrays (1), negative sizes (1), misaligned
+    views (3), a workspace smaller than hils_workspace_bytes (4), unsupported params (2)."""
+    p = _p(B=1, H=2, d=128, K=4, W=64)
+    c = ctypes.byref(p.c())
+    v = T(ALIGNED, 4 * 8192 * 128, 8192 * 128, 128)   # [1, 2, 8192, 128] view
+    s = T(ALIGNED, 2 * 128 * 128, 128 * 128, 128)     # [1, 2, 128, 128] table
+    bad = T(ALIGNED + 8, 4 * 8192 * 128, 8192 * 128, 128)
+    A = ALIGNED
+    N, C = 8192, 128
+    # hils_summarize_append(p, K, cache_len, LQ, Ksum, Bsum, C, stream)
+    assert lib.hils_summarize_append(c, v, None, s, s, A, C, None) == 1
+    assert lib.hils_summarize_append(c, v, A, s, s, A, -1, None) == 1
+    assert lib.hils_summarize_append(c, bad, A, s, s, A, C, None) == 3
+    assert lib.hils_summarize_append(ctypes.byref(_p(d=96).c()), v, A, s, s, A, C, None) == 2
+    # hils_attend_prefill_backward(p, Q, K, V, N, idx, score, nsel, O, lse, dO, dQ, dK, dV, dscore, ws, n, stream)
+    need = lib.hils_workspace_bytes(c, hils.HILS_CALL_ATTEND_BACKWARD, N, 0)
+    assert need > 0
+    args = [v, v, v, N, A, A, A, v, A, A, A, A, A, A]
+    assert lib.hils_attend_prefill_backward(c, *args, A, need - 1, None) == 4
+    assert lib.hils_attend_prefill_backward(c, *args, None, need, None) == 4
+    assert lib.hils_attend_prefill_backward(c, *args[:9], None, *args[10:], A, need, None) == 1  # dO
+    assert lib.hils_attend_prefill_backward(c, *args[:3], -1, *args[4:], A, need, None) == 1
+    assert lib.hils_attend_prefill_backward(c, bad, *args[1:], A, need, None) == 3
+    assert lib.hils_attend_prefill_backward(c, *args[:8], A + 2, *args[9:], A, need, None) == 3  # lse
+    # hils_select_backward(p, Qcal, Lq, Ksum, C, idx, nsel, dscore, dQcal, dKsum, dBsum, stream)
+    assert lib.hils_select_backward(c, v, N, s, C, A, A, None, A, A, A, None) == 1
+    assert lib.hils_select_backward(c, v, -1, s, C, A, A, A, A, A, A, None) == 1
+    assert lib.hils_select_backward(c, bad, N, s, C, A, A, A, A, A, A, None) == 3
+    assert lib.hils_select_backward(ctypes.byref(_p(K=40).c()), v, N, s, C, A, A, A, A, A, A, None) == 2
+    # hils_summarize_backward(p, K, N, LQ, dKsum, dBsum, dK, dLQ, stream)
+    assert lib.hils_summarize_backward(c, v, N, s, A, A, None, A, None) == 1
+    assert lib.hils_summarize_backward(c, v, -64, s, A, A, A, A, None) == 1
+    assert lib.hils_summarize_backward(c, v, N, bad, A, A, A, A, None) == 3
+    g = _p(H=4, H_kv=3)
+    assert lib.hils_summarize_backward(ctypes.byref(g.c()), v, N, s, A, A, A, A, None) == 1
