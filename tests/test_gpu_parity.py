@@ -9,7 +9,6 @@ test), copied to the GPU; the oracle reads the very same stored bits. Bars:
 Attend stages are checked with the oracle fed the GPU's own selection, so a
 selection difference can never hide inside an output check.
 """
-import math
 
 import numpy as np
 import pytest
