@@ -590,10 +590,29 @@ def measure_prefill_backward(w, dev, stream, flush, args, world):
     n = 3
     ms = statistics.mean(time_steps(bwd, n, flush, stream))
     ms = max_over_ranks(ms, world, dev)
+
+    # each call timed alone (L2 flushed), with the zeroing of what it accumulates into
+    def attend_bwd():
+        dK.zero_()
+        dV.zero_()
+        hils.hils_attend_prefill_backward(pb.p, i["Q"], i["K"], i["V"], pb.idx, pb.score, pb.nsel, pb.O, pb.lse, dO,
+                                          dQ, dK, dV, dscore, workspace=ws)
+
+    def select_bwd():
+        dKsum.zero_()
+        dBsum.zero_()
+        hils.hils_select_backward(pb.p, i["Qcal"], pb.Ksum, pb.idx, pb.nsel, dscore, dQcal, dKsum, dBsum)
+
+    def summarize_bwd():
+        hils.hils_summarize_backward(pb.p, i["K"], i["LQ"], dKsum, dBsum, dK, dLQ)
+
+    split = {name: statistics.mean(time_steps(f, n, flush, stream))
+             for name, f in (("attend_backward", attend_bwd), ("select_backward", select_bwd),
+                             ("summarize_backward", summarize_bwd))}
     fl = backward_flops(w)
     out = {"ms_per_step": ms, "unit": "TFLOP/s", "value": fl / (ms * 1e-3) / 1e12 * world, "workload": w.name,
-           "algorithmic_gflop_per_step": fl / 1e9, "steps": n,
-           "note": "key-major attend backward on the tensor cores (mma.sync bf16, dK and dV accumulated per key block), float32 atomics for dQ, dKsum, dBsum"}
+           "algorithmic_gflop_per_step": fl / 1e9, "steps": n, "ms_per_call": split,
+           "note": "key-major attend backward on the tensor cores (mma.sync bf16, dK and dV accumulated per key block), float32 atomics for dQ, dKsum, dBsum; ms_per_call times each call alone"}
     del pb
     torch.cuda.empty_cache()
     return out
