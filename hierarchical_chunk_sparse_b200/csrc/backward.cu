@@ -626,6 +626,80 @@ __global__ void __launch_bounds__(kThreads) select_backward_kernel(BwdSelectArgs
     a.dQcal[qi * D + tid] = a.scale * acc;
 }
 
+// Eq. 7 backward with the chunk sums kept in shared memory: a CTA takes kSelBwdRows
+// consecutive queries of one (b, h), adds scale ds q~ into its own [C][D] table (and ds
+// into [C]) with shared-memory atomics, writes dQcal, and then adds each table row that
+// a kept chunk touched to dKsum and dBsum once. Adjacent queries keep mostly the same
+// chunks, so the global atomics drop from one per (query, kept chunk, x) to about one
+// per (CTA, touched chunk, x). Used when the table fits in shared memory.
+constexpr int kSelBwdRows = 128;
+constexpr int kSelBwdSmemMax = 200 * 1024;
+
+inline size_t select_bwd_table_bytes(int C, int D) {
+    return (size_t)C * D * 4 + (size_t)C * 4 + (size_t)((C + 31) / 32) * 4;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) select_backward_table_kernel(BwdSelectArgs a) {
+    extern __shared__ __align__(16) float tsm[];
+    constexpr int kPer = D / 32;  // elements of a row per lane
+    const int C = a.C;
+    float *tk = tsm;                                           // [C][D]
+    float *tb = tk + (int64_t)C * D;                           // [C]
+    unsigned *touched = reinterpret_cast<unsigned *>(tb + C);  // C bits
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nblk = (a.Lq + kSelBwdRows - 1) / kSelBwdRows;
+    const int64_t bh = blockIdx.x / nblk;
+    const int i0 = (int)(blockIdx.x % nblk) * kSelBwdRows;
+    const int h = (int)(bh % a.H), b = (int)(bh / a.H);
+    const int Hk = a.H / a.G;
+    const int K = a.topk;
+    for (int e = tid; e < C * D; e += kThreads) tk[e] = 0.f;
+    for (int e = tid; e < C; e += kThreads) tb[e] = 0.f;
+    for (int e = tid; e < (C + 31) / 32; e += kThreads) touched[e] = 0u;
+    __syncthreads();
+    const T *khead = static_cast<const T *>(a.Ksum.ptr) + b * a.Ksum.sb + h * a.Ksum.sh;
+    const int iend = min(a.Lq, i0 + kSelBwdRows);
+    for (int i = i0 + warp; i < iend; i += kThreads / 32) {  // a warp per query
+        const int64_t qi = bh * a.Lq + i;
+        const int64_t qg = ((int64_t)b * Hk + h / a.G) * a.Lq + i;
+        const int ns = K > 0 ? min(max(a.nsel[qg], 0), K) : 0;
+        const T *qrow = static_cast<const T *>(a.Qcal.ptr) + b * a.Qcal.sb + h * a.Qcal.sh + (int64_t)i * a.Qcal.st;
+        float qx[kPer], acc[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            qx[u] = a.scale * elem(qrow, lane + 32 * u);
+            acc[u] = 0.f;
+        }
+        for (int k = 0; k < ns; ++k) {
+            const int c = a.idx[qg * K + k];
+            if ((unsigned)c >= (unsigned)C) continue;
+            const float ds = a.dscore[qi * K + k];
+            const T *krow = khead + (int64_t)c * a.Ksum.st;
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                acc[u] = fmaf(ds, elem(krow, lane + 32 * u), acc[u]);
+                atomicAdd(&tk[c * D + lane + 32 * u], ds * qx[u]);
+            }
+            if (lane == 0) {
+                atomicAdd(&tb[c], ds);
+                atomicOr(&touched[c >> 5], 1u << (c & 31));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) a.dQcal[qi * D + lane + 32 * u] = a.scale * acc[u];
+    }
+    __syncthreads();
+    float *dks = a.dKsum + bh * C * D;
+    float *dbs = a.dBsum + bh * C;
+    for (int c = warp; c < C; c += kThreads / 32) {
+        if (!((touched[c >> 5] >> (c & 31)) & 1u)) continue;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) atomicAdd(dks + (int64_t)c * D + lane + 32 * u, tk[c * D + lane + 32 * u]);
+        if (lane == 0) atomicAdd(dbs + c, tb[c]);
+    }
+}
+
 // grid: B*H*C, one chunk each: Eq. 8 backward.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) summarize_backward_kernel(BwdSummarizeArgs a) {
@@ -746,6 +820,16 @@ hils_status launch_attend_bwd(const BwdAttendArgs &a, void *ws, cudaStream_t s) 
 
 template <typename T, int D>
 hils_status launch_select_bwd(const BwdSelectArgs &a, cudaStream_t s) {
+    const size_t table = select_bwd_table_bytes(a.C, D);
+    if (a.C > 0 && table <= (size_t)kSelBwdSmemMax) {
+        static KernelSetup setup;
+        const hils_status st =
+            kernel_setup(setup, (const void *)select_backward_table_kernel<T, D>, kThreads, kSelBwdSmemMax, nullptr);
+        if (st != HILS_OK) return st;
+        const int64_t grid = (int64_t)a.B * a.H * ((a.Lq + kSelBwdRows - 1) / kSelBwdRows);
+        select_backward_table_kernel<T, D><<<(unsigned)grid, kThreads, table, s>>>(a);
+        return record_cuda_error(cudaGetLastError());
+    }
     select_backward_kernel<T, D><<<(unsigned)((int64_t)a.B * a.H * a.Lq), kThreads, 0, s>>>(a);
     return record_cuda_error(cudaGetLastError());
 }
