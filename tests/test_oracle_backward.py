@@ -162,3 +162,18 @@ def test_key_value_head_slices_are_independent_problems():
         assert torch.allclose(part[name], full[name][:, qs], atol=1e-12, rtol=0), name
     for name in ("dK", "dV"):
         assert torch.allclose(part[name], full[name][:, ks], atol=1e-12, rtol=0), name
+
+
+@pytest.mark.parametrize("G,W", [(1, 50), (2, 90)])
+def test_value_gradients_sum_to_the_output_gradients(G, W):
+    """Eq. 10 gives every query one normaliser over its kept chunks and its window, so
+    the token weights of a query with a finite lse sum to 1 and dO_i reaches the values
+    with total weight 1: for each key-value head, sum_j dV_j = sum of dO_i over its
+    query heads' queries (all of them here: W > 0 puts each query's own token in its
+    window). Independent of autograd: a wrong weight or a dropped term breaks it."""
+    Q, Kc, Vc, Qcal, LQ, idx, nsel = _problem(H=4, G=G, N=64 * 4 + 29, d=8, K=3, seed=70 + G)
+    dO = _rand(*Q.shape, seed=71)
+    g = ob.grads(Q, Kc, Vc, Qcal, LQ, idx, nsel, dO, S, W, 0.4)
+    assert torch.isfinite(g["lse"]).all()
+    want = dO.reshape(1, 4 // G, G, *dO.shape[2:]).sum(dim=(2, 3))  # [B, Hk, d]
+    assert torch.allclose(g["dV"].sum(dim=2), want, atol=1e-11, rtol=0)
