@@ -177,3 +177,35 @@ def test_value_gradients_sum_to_the_output_gradients(G, W):
     assert torch.isfinite(g["lse"]).all()
     want = dO.reshape(1, 4 // G, G, *dO.shape[2:]).sum(dim=(2, 3))  # [B, Hk, d]
     assert torch.allclose(g["dV"].sum(dim=2), want, atol=1e-11, rtol=0)
+
+
+def test_score_gradient_closed_form():
+    """dscore against its closed form from Eq. 10, with every ingredient from the C
+    oracle rather than autograd: for query i and kept chunk c, with w_c = exp(s^_c -
+    lse_i), o_c the chunk's own softmax average of its values, and D_i = dO_i . o_i,
+    the gradient of sum(O * dO) with respect to s^_c is w_c (dO_i . o_c - D_i)."""
+    Q, Kc, Vc, Qcal, LQ, idx, nsel = _problem(H=2, G=1, N=64 * 4 + 13, d=8, K=3, seed=80)
+    dO = _rand(*Q.shape, seed=81)
+    W, sc = 45, 0.5
+    g = ob.grads(Q, Kc, Vc, Qcal, LQ, idx, nsel, dO, S, W, sc)
+    ks, bs = oracle.summarize(Kc, LQ, S, sc)
+    sall = oracle.score_all(Qcal, torch.from_numpy(ks), torch.from_numpy(bs), S, sc)
+    score = np.full(idx.shape, -np.inf)
+    for h in range(2):
+        for i in range(Q.shape[2]):
+            n = nsel[0, h, i]
+            score[0, h, i, :n] = sall[0, h, i, idx[0, h, i, :n]]
+    O, lse = oracle.attend(Q, Kc, Vc, idx, score, nsel, S, W, sc)
+    q, k, v, do = (x.numpy() for x in (Q, Kc, Vc, dO))
+    want = np.zeros(idx.shape)
+    for h in range(2):
+        for i in range(Q.shape[2]):
+            Di = do[0, h, i] @ O[0, h, i]
+            for slot in range(nsel[0, h, i]):
+                c = idx[0, h, i, slot]
+                lg = sc * (k[0, h, c * S:(c + 1) * S] @ q[0, h, i])
+                p = np.exp(lg - lg.max())
+                oc = (p / p.sum()) @ v[0, h, c * S:(c + 1) * S]
+                want[0, h, i, slot] = np.exp(score[0, h, i, slot] - lse[0, h, i]) * (do[0, h, i] @ oc - Di)
+    assert np.abs(g["dscore"].numpy() - want).max() < 1e-12
+    assert (nsel > 0).any() and (nsel < 3).any()
