@@ -209,3 +209,18 @@ def test_score_gradient_closed_form():
                 want[0, h, i, slot] = np.exp(score[0, h, i, slot] - lse[0, h, i]) * (do[0, h, i] @ oc - Di)
     assert np.abs(g["dscore"].numpy() - want).max() < 1e-12
     assert (nsel > 0).any() and (nsel < 3).any()
+
+
+def test_empty_queries_pass_no_gradient():
+    """With W = 0, the first 64 queries keep no chunk and have an empty window: o = 0 and
+    lse = -inf, a constant output, so their dQ, dQcal and dscore are exactly 0 and no
+    gradient is NaN anywhere."""
+    Q, Kc, Vc, Qcal, LQ, idx, nsel = _problem(H=2, G=1, N=64 * 3 + 7, d=8, K=2, seed=90)
+    dO = _rand(*Q.shape, seed=91)
+    g = ob.grads(Q, Kc, Vc, Qcal, LQ, idx, nsel, dO, S, 0, 0.5)
+    assert torch.isneginf(g["lse"][..., :64]).all() and torch.isfinite(g["lse"][..., 64:]).all()
+    for name in ("dQ", "dQcal", "dscore"):
+        assert (g[name][:, :, :64] == 0).all(), name
+    for name in ("dQ", "dK", "dV", "dQcal", "dLQ", "dscore", "dKsum", "dBsum"):
+        assert torch.isfinite(g[name]).all(), name
+    assert (g["O"][:, :, :64] == 0).all()
