@@ -25,9 +25,25 @@ def assert_close(gpu, ref, dtype, what=""):
     max_abs = float(diff.max()) if diff.size else 0.0
     denom = float(np.linalg.norm(r[fin]))
     rel = float(np.linalg.norm(g[fin] - r[fin]) / denom) if denom > 0 else max_abs
-    assert max_abs <= atol, f"{what}: max abs err {max_abs:.3e} > {atol}"
-    assert rel <= rtol, f"{what}: rel L2 err {rel:.3e} > {rtol}"
+    assert max_abs <= atol, f"{what}: max abs err {max_abs:.3e} > {atol} (worst row: {_worst_row(g, r)})"
+    assert rel <= rtol, f"{what}: rel L2 err {rel:.3e} > {rtol} (worst row: {_worst_row(g, r)})"
     return max_abs, rel
+
+
+def _worst_row(g, r):
+    """Index and relative L2 error of the worst row along the last axis (for failure
+    messages only)."""
+    if r.ndim < 2 or r.size == 0:
+        return None
+    gg, rr = g.reshape(-1, r.shape[-1]), r.reshape(-1, r.shape[-1])
+    ok = np.isfinite(rr).all(-1)
+    if not ok.any():
+        return None
+    num = np.linalg.norm(gg - np.where(np.isfinite(rr), rr, 0), axis=-1)
+    den = np.linalg.norm(np.where(np.isfinite(rr), rr, 0), axis=-1)
+    rel = np.where(ok, num / np.where(den > 0, den, 1.0), -1.0)
+    row = int(np.argmax(rel))
+    return tuple(int(x) for x in np.unravel_index(row, r.shape[:-1])), float(rel[row])
 
 
 def assert_same_selection(idx_gpu, nsel_gpu, idx_ref, nsel_ref, what=""):
