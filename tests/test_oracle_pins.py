@@ -374,3 +374,27 @@ def test_window_overlapping_a_selected_chunk_counts_twice(oracle):
     want[8:12] += np.exp(logits[8:12]) / zc * math.exp(s2) / zhat
     want[10:14] += np.exp(logits[10:14]) / zhat
     np.testing.assert_allclose(w, want, rtol=0, atol=1e-14)
+
+
+def test_decode_form_equals_the_prefill_row(oracle):
+    """The decode form (one query at an explicit position t, qpos) selects and attends
+    exactly as row t of the prefill form over the same sequence: same kept chunks, same
+    scores, same output and lse, and tokens after t (present in the keys and values)
+    take no part."""
+    g = np.random.default_rng(123)
+    B, H, d, S, N, K, W, sc = 1, 2, 16, 64, 64 * 5 + 11, 3, 70, 0.3
+    Q, Qcal, Kc, Vc = (torch.from_numpy(g.standard_normal((B, H, N, d))) for _ in range(4))
+    LQ = torch.from_numpy(g.standard_normal((B, H, N // S, d)))
+    ks, bs = oracle.summarize(Kc, LQ, S, sc)
+    idx, score, nsel = oracle.select(Qcal, ks, bs, S, K, sc)
+    O, lse = oracle.attend(Q, Kc, Vc, idx, score, nsel, S, W, sc)
+    for t in (0, 63, 64, 130, 200, N - 1):
+        qpos = np.full((B, 1), t, np.int32)
+        i1, s1, n1 = oracle.select(Qcal[:, :, t:t + 1], ks, bs, S, K, sc, qpos=qpos)
+        assert (n1 == nsel[:, :, t:t + 1]).all() and (i1 == idx[:, :, t:t + 1]).all(), t
+        assert np.array_equal(s1, score[:, :, t:t + 1]), t
+        Vj = Vc.clone()
+        Vj[:, :, t + 1:] += 1000.0  # tokens after the query must not matter
+        O1, l1 = oracle.attend(Q[:, :, t:t + 1], Kc, Vj, i1, s1, n1, S, W, sc, qpos=qpos)
+        assert np.abs(O1[:, :, 0] - O[:, :, t]).max() < 1e-12, t
+        assert np.abs(l1[:, :, 0] - lse[:, :, t]).max() < 1e-12, t
