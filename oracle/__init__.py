@@ -125,6 +125,7 @@ def _group(h_query: int, h_kv: int) -> int:
 def summarize(K: torch.Tensor, LQ: torch.Tensor, S: int, scale: float):
     """Eq. 8 summaries of every query head (LQ [B,H,C,d]) over the keys of its key-value
     head (K [B,H/G,N,d]). Returns (Ksum [B,H,C,d], Bsum [B,H,C]) in float64."""
+    K, LQ = _as_tensor(K), _as_tensor(LQ)
     B, Hk, N, d = K.shape
     H = LQ.shape[1]
     G = _group(H, Hk)
