@@ -1,7 +1,7 @@
 """The seeded input generators (no GPU): determinism and the planted structure."""
 import torch
 
-from hils_synth import WORKLOADS, make_prefill
+from hils_synth import WORKLOADS, make_decode, make_prefill
 
 
 def test_prefill_generator_is_deterministic():
@@ -52,3 +52,33 @@ def test_prefill_workload_stresses_near_ties():
             tot += 1
             band += bool(s[-w.K] - s[-w.K - 1] <= 1e-6)
     assert 0.008 < band / tot < 0.03, (band, tot)
+
+
+def test_decode_needles_are_planted_and_dominate_their_chunks():
+    """Decode workloads plant needle keys in distinct chunks wholly before the window,
+    each with logit scale q.k_p = 8 before bf16 rounding, so each needle's chunk has an
+    exact log-mass log Z_c near 8 (the max-dominant regime) and the largest of all the
+    query's eligible chunks. Q_cal is a copy of Q."""
+    import numpy as np
+
+    import oracle
+
+    w = WORKLOADS[5].replace(H=2, N=64 * 60, K=8, W=256)  # four needles per head
+    inp = make_decode(w)
+    q, k = inp["Q"].double(), inp["K"].double()
+    assert torch.equal(inp["Qcal"], inp["Q"])
+    t = w.N - 1
+    first_window_chunk = (t - w.W + 1) // 64
+    ce = t // 64
+    idx = np.broadcast_to(np.arange(ce, dtype=np.int32), (w.B, w.H, 1, ce)).copy()
+    nsel = np.full((w.B, w.H, 1), ce, np.int32)
+    logz = oracle.chunk_logmass(inp["Q"], inp["K"], idx, nsel, 64, w.scale)
+    for h in range(w.H):
+        pos = inp["needles"][0, h]
+        chunks = (pos // 64).tolist()
+        assert len(pos) == 4 and len(set(chunks)) == 4 and max(chunks) < first_window_chunk
+        logit = w.scale * (k[0, h, pos] @ q[0, h, 0])
+        assert (logit - 8).abs().max() < 0.1, logit
+        order = np.argsort(-logz[0, h, 0])
+        assert set(order[:4].tolist()) == set(chunks)
+        assert logz[0, h, 0, chunks].min() > 7.9 and np.delete(logz[0, h, 0], chunks).max() < 7.0
