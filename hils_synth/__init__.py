@@ -25,6 +25,10 @@ Workloads (one attention layer; chunk size S = 64 everywhere):
   8 decode bf16 512K, grouped-query: as 4 with 8 key-value heads (groups of 4); the
                          needle of each key-value head is planted against the query of
                          the group's first head.
+  9 decode bf16 512K, retrieval: as 4 with four needles per head, and the landmark query
+                         of each needle's chunk set to point at the needle key, with a
+                         landmark logit of 8: the summary of that chunk then concentrates
+                         on the needle, as a trained landmark would for a salient token.
 Every workload with Hk = 0 has as many key-value heads as query heads.
 bf16 tensors are drawn in float32 and rounded to nearest-even.
 
@@ -62,6 +66,7 @@ class Workload:
     needle_logit: float = 8.0
     qcal_block: int = 0  # > 0: Q_cal = block base vector + qcal_noise * iid noise
     qcal_noise: float = 0.0
+    needle_landmark: bool = False  # the needle chunk's landmark query points at the needle
     Hk: int = 0  # key-value heads (0: one per query head)
 
     @property
@@ -101,6 +106,8 @@ WORKLOADS = {
                 qkv_scaled=True, Hk=8),
     8: Workload(8, "decode_bf16_512k_gqa", "decode", 1, 32, 128, 64, 16, 512, 524288,
                 torch.bfloat16, needles=1, Hk=8),
+    9: Workload(9, "decode_bf16_512k_retrieval", "decode", 1, 32, 128, 64, 16, 512, 524288,
+                torch.bfloat16, needles=4, needle_landmark=True),
 }
 
 
@@ -177,6 +184,11 @@ def make_decode(w: Workload, device="cpu") -> dict:
             for p in pos[b, h].tolist():
                 # k_p <- k_p + (L/scale - q.k_p) q / |q|^2, so that scale * q.k_p = L
                 k[p] += (w.needle_logit / w.scale - torch.dot(q, k[p])) * q / torch.dot(q, q)
+                if w.needle_landmark:
+                    # landmark query L/scale * k_p / |k_p|^2: scale * q'_c . k_p = L
+                    lm = (w.needle_logit / w.scale) * k[p] / torch.dot(k[p], k[p])
+                    for hq in range(h * w.G, (h + 1) * w.G):
+                        lq[b, hq, p // w.S] = lm.to(w.dtype)
             kc[b, h] = k.to(w.dtype)
             vc[b, h] = _randn((N, d), g_v, device).to(w.dtype)
             del k

@@ -82,3 +82,29 @@ def test_decode_needles_are_planted_and_dominate_their_chunks():
         order = np.argsort(-logz[0, h, 0])
         assert set(order[:4].tolist()) == set(chunks)
         assert logz[0, h, 0, chunks].min() > 7.9 and np.delete(logz[0, h, 0], chunks).max() < 7.0
+
+
+def test_retrieval_workload_selects_every_needle():
+    """Workload 9 points each needle chunk's landmark query at the needle (landmark logit
+    8), so the chunk's summary concentrates on it (k' near k_p, b' near 0) and its
+    surrogate score is near the needle's logit: the oracle's selection keeps every
+    needle's chunk. Everything else follows workload 4's recipe."""
+    import oracle
+
+    w = WORKLOADS[9].replace(H=4, N=64 * 200)
+    inp = make_decode(w)
+    t = w.N - 1
+    ks, bs = oracle.summarize(inp["K"], inp["LQ"], 64, w.scale)
+    qpos = torch.full((w.B, 1), t, dtype=torch.int32)
+    idx, score, nsel = oracle.select(inp["Qcal"], ks, bs, 64, w.K, w.scale, qpos=qpos)
+    k, lq = inp["K"].double(), inp["LQ"].double()
+    for h in range(w.H):
+        pos = inp["needles"][0, h]
+        chunks = (pos // 64).tolist()
+        assert (w.scale * (lq[0, h, chunks] * k[0, h, pos]).sum(-1) - 8).abs().max() < 0.1
+        assert set(chunks) <= set(idx[0, h, 0, : nsel[0, h, 0]].tolist())
+        assert (bs[0, h, chunks] < 0.5).all()  # entropy far below log 64: the softmax sits on the needle
+    # the other workloads' draws are untouched by the flag
+    w4 = WORKLOADS[4].replace(H=2, N=64 * 40)
+    a, b = make_decode(w4), make_decode(w4.replace(needle_landmark=False))
+    assert torch.equal(a["LQ"], b["LQ"]) and torch.equal(a["K"], b["K"])
