@@ -9,19 +9,28 @@ Headline (one JSON line on rank 0):
   chunks + the window). Summaries are built once beforehand (hils_summarize), as a
   server keeps them with its KV cache.
 Beside it, in the same line:
-  "prefill": algorithmic TFLOP/s of summarise + select + prefill attend on the 8K
-  prefill workload (B=1, H=32, d=128, K=16, W=512);
   "roofline": the dominant decode kernel against the measured HBM copy bandwidth;
   "e2e": the same decode metric through the Python binding with pinned host
   buffers: the step's query (Q, Q_cal, positions) copied in and (O, lse) copied out
   inside the timed region; KV cache and summaries stay resident in HBM;
+  "cold_single_step": the same step with L2 flushed before it, timed alone;
+  "prefill", "prefill_local", "prefill_gqa": algorithmic TFLOP/s of summarise + select +
+  prefill attend on the 8K prefill workloads (B=1, H=32, d=128, K=16, W=512);
+  "decode_b8_128k", "decode_1m" (with the full summary rebuild at 1M, timed alone),
+  "decode_gqa", "decode_retrieval": the other decode workloads, each with its own
+  roofline;
+  "prefill_backward": the backward of the 8K prefill for its selection;
   "cpu_baseline": the float64 oracle on this host's cores, on a sample of heads.
 
-Timing: W warm-up steps, then exactly K timed steps, each preceded by a write of
-2x the L2 size (outside the step's events), timed with CUDA events on the launching
-stream; barrier + synchronize around the region; the max over ranks is reported.
-Multi-GPU (torchrun): every rank runs its own replica of the workload (weak
-scaling; the path has no exchange step) and value = all ranks' tokens / max time.
+Timing: decode steps run back to back over R independent copies of the workload's
+inputs (R copies of KV cache, summaries, queries and outputs, cycled in order) whose
+bytes per cycle are at least three times the L2 size, so every step reads its data
+cold, as each layer of a model reads its own cache. W warm-up steps, then exactly K
+timed steps between two CUDA events on the launching stream; barrier + synchronize
+around the region; the max over ranks is reported. Prefill and backward passes (and
+the cold single step) are timed one at a time with L2 flushed before each. Multi-GPU
+(torchrun): every rank runs its own replica of the workload (weak scaling; the path
+has no exchange step) and value = all ranks' tokens / max time.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hils|reference]
 """
@@ -212,30 +221,35 @@ def decode_bytes(w) -> dict:
     return {"select": table + small, "attend": kv + small, "step": table + kv + small}
 
 
-class DecodeBench:
-    def __init__(self, w, dev):
-        import hierarchical_chunk_sparse_b200 as hils
+# Decode steps are timed back to back over R independent copies of the workload's inputs
+# (R copies of the KV cache, summary table, queries and outputs, cycled in order), with R
+# chosen so that the R steps together touch at least three times the L2 size: every step
+# reads its data cold, as each layer of a model reads its own KV cache and summaries.
+DECODE_L2 = ("inputs larger than L2: steps cycle over R independent input copies whose bytes per "
+             "cycle are >= 3x L2; timed back to back")
 
-        self.hils, self.w, self.dev = hils, w, dev
-        inp = make_decode(w, device=dev)
-        self.inp = inp
-        self.p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype, H_kv=w.Hk)
+
+def decode_sets(w, l2_bytes: int) -> int:
+    step = decode_bytes(w)["step"]
+    return max(2, -(-3 * l2_bytes // step))
+
+
+class DecodeSet:
+    """One copy of a decode workload's inputs, summaries, outputs and workspaces."""
+
+    def __init__(self, hils, p, w, inp, Ksum, Bsum, dev):
+        self.hils, self.p, self.w = hils, p, w
+        self.inp, self.Ksum, self.Bsum = inp, Ksum, Bsum
         C = w.C
-        self.Ksum = torch.empty(w.B, w.H, C, w.d, dtype=w.dtype, device=dev)
-        self.Bsum = torch.empty(w.B, w.H, C, dtype=torch.float32, device=dev)
-        hils.hils_summarize(self.p, inp["K"], inp["LQ"], self.Ksum, self.Bsum)
         self.qpos = (inp["cache_len"] - 1).reshape(w.B, 1).contiguous()
         self.idx = torch.empty(w.B, w.Hkv, 1, w.K, dtype=torch.int32, device=dev)
         self.score = torch.empty(w.B, w.H, 1, w.K, dtype=torch.float32, device=dev)
         self.nsel = torch.empty(w.B, w.Hkv, 1, dtype=torch.int32, device=dev)
-        self.ws_sel = hils.alloc_workspace(self.p, hils.HILS_CALL_SELECT, 1, C, device=dev)
-        self.ws_dec = hils.alloc_workspace(self.p, hils.HILS_CALL_ATTEND_DECODE, 1, 0, device=dev)
-        self.ws_step = hils.alloc_workspace(self.p, hils.HILS_CALL_DECODE, 1, C, device=dev)
+        self.ws_sel = hils.alloc_workspace(p, hils.HILS_CALL_SELECT, 1, C, device=dev)
+        self.ws_dec = hils.alloc_workspace(p, hils.HILS_CALL_ATTEND_DECODE, 1, 0, device=dev)
+        self.ws_step = hils.alloc_workspace(p, hils.HILS_CALL_DECODE, 1, C, device=dev)
         self.O = torch.empty_like(inp["Q"])
         self.lse = torch.empty(w.B, w.H, dtype=torch.float32, device=dev)
-        torch.cuda.synchronize()
-        # one step = hils_decode: the screen and pick kernels of the select, then the attend
-        self.launches_per_step = 3
 
     def select(self):
         i = self.inp
@@ -253,6 +267,8 @@ class DecodeBench:
                               self.idx, self.score, self.nsel, self.O, self.lse, workspace=self.ws_step)
 
     def e2e_setup(self):
+        """Pinned host copies of the step's inputs (query, calibrated query, cache
+        lengths) and of its results (O, lse)."""
         i = self.inp
         self.h_in = {k: i[k].cpu().pin_memory() for k in ("Q", "Qcal", "cache_len")}
         self.h_O = torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory()
@@ -268,6 +284,69 @@ class DecodeBench:
         self.step()
         self.h_O.copy_(self.O, non_blocking=True)
         self.h_lse.copy_(self.lse, non_blocking=True)
+
+
+class DecodeBench:
+    """R copies of a decode workload (R >= 2, see decode_sets); summaries built once by
+    hils_summarize (untimed), as a server keeps them with its KV cache."""
+
+    def __init__(self, w, dev, sets: int | None = None):
+        import hierarchical_chunk_sparse_b200 as hils
+
+        self.hils, self.w, self.dev = hils, w, dev
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.R = sets if sets is not None else decode_sets(w, l2)
+        self.p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype, H_kv=w.Hk)
+        inp = make_decode(w, device=dev)
+        Ksum = torch.empty(w.B, w.H, w.C, w.d, dtype=w.dtype, device=dev)
+        Bsum = torch.empty(w.B, w.H, w.C, dtype=torch.float32, device=dev)
+        hils.hils_summarize(self.p, inp["K"], inp["LQ"], Ksum, Bsum)
+        self.needles = inp["needles"]
+        self.sets = []
+        for r in range(self.R):
+            if r == 0:
+                ir, kr, br = inp, Ksum, Bsum
+            else:
+                ir = {k: (v.clone() if isinstance(v, torch.Tensor) and v.is_cuda else v) for k, v in inp.items()}
+                kr, br = Ksum.clone(), Bsum.clone()
+            ir.pop("LQ", None)  # landmark queries are only needed for the summaries
+            self.sets.append(DecodeSet(hils, self.p, w, ir, kr, br, dev))
+        del inp
+        torch.cuda.synchronize()
+        # one step = hils_decode: the screen and pick kernels of the select, then the attend
+        self.launches_per_step = 3
+
+    def graphs(self, name, stream):
+        """CUDA graphs of `name` (step, select, attend or e2e_step): one over all R sets in
+        order, and one per set."""
+        fns = [getattr(s, name) for s in self.sets]
+        with torch.cuda.stream(stream):
+            for f in fns:  # warm (and, for e2e_step, not captured cold)
+                f()
+        stream.synchronize()
+
+        def run_all():
+            for f in fns:
+                f()
+
+        return graphed(run_all, stream), [graphed(f, stream) for f in fns]
+
+
+def time_rotating(graphs, steps: int, stream) -> float:
+    """Device milliseconds per step of `steps` steps run back to back: whole cycles over
+    the R sets, then the first steps % R sets."""
+    g_all, g_one = graphs
+    R = len(g_one)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s.record(stream)
+        for _ in range(steps // R):
+            g_all()
+        for r in range(steps % R):
+            g_one[r]()
+        e.record(stream)
+    stream.synchronize()
+    return s.elapsed_time(e) / steps
 
 
 # ----------------------------------------------------------------- prefill workload
@@ -288,10 +367,40 @@ def prefill_flops(w, part: str = "step") -> float:
 
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) that Nsight Compute
-# measured for the current kernels, each with its command in profiles/: select_decode512k.md
-# (screen + pick of one select call), attend_decode_128k.md, attend_prefill_tc_prefill8k.md.
-# A kernel that changes after its capture reports null here until it is captured again.
-MEASURED_TRAFFIC = {"select": 69_647_616, "attend_decode": 25_235_968, "attend_prefill": 661_831_680}
+# measured, each with its command in profiles/, keyed by the kernel it describes and the
+# digest of that kernel's source files at capture time. A kernel whose sources changed
+# after its capture reports null until it is captured again.
+CSRC = os.path.join(ROOT, "hierarchical_chunk_sparse_b200", "csrc")
+KERNEL_SOURCES = {
+    "decode_select": ["select.cu", "screen_stage.cuh", "select_pick.cuh", "select_common.cuh", "tc_common.cuh",
+                      "hils_internal.cuh"],
+    "decode_attend": ["attend.cu", "hils_internal.cuh"],
+    "attend_prefill": ["attend_prefill_tc.cu", "tc_common.cuh", "hils_internal.cuh"],
+    "summarize": ["summarize.cu", "hils_internal.cuh"],
+}
+# kernel -> (DRAM bytes per unit, source digest at capture). Units: decode_select and
+# decode_attend per algorithmic byte of the launch (the captured traffic / algorithmic
+# bytes), summarize per chunk, attend_prefill per launch of the 8K prefill workload.
+MEASURED_TRAFFIC = {}
+
+
+def source_digest(kernel: str) -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, scale: float = 1.0):
+    """DRAM bytes of one timed launch of `kernel`: the captured bytes per unit times the
+    launch's units (`scale`), or None if the kernel's sources changed since its capture."""
+    rec = MEASURED_TRAFFIC.get(kernel)
+    if rec is None or rec[1] != source_digest(kernel):
+        return None
+    return rec[0] * scale
 
 
 class PrefillBench:
@@ -342,28 +451,20 @@ class PrefillBench:
 # ----------------------------------------------------------------- CPU oracle baseline
 
 def oracle_decode_sample(w, dev, heads: int):
-    """Host copies of the first `heads` heads of a decode workload, with summaries."""
-    import hierarchical_chunk_sparse_b200 as hils
+    """Host copies of the first `heads` heads of a decode workload, with their Eq. 8
+    summaries from the oracle. The inputs are drawn by hils_synth (on the GPU when one is
+    present, through torch alone: the same values as the first heads of the full
+    workload), so nothing here touches the CUDA library."""
+    import oracle
 
     ws = w.replace(H=heads)
-    gen_dev = dev if dev is not None else "cpu"
-    inp = make_decode(ws, device=gen_dev)
+    inp = make_decode(ws, device=dev if dev is not None else "cpu")
+    host = {k: v.cpu() for k, v in inp.items() if isinstance(v, torch.Tensor)}
+    del inp
     if dev is not None:
-        p = hils.Params(B=ws.B, H=ws.H, d=ws.d, K=ws.K, W=ws.W, dtype=ws.dtype)
-        Ksum = torch.empty(ws.B, ws.H, ws.C, ws.d, dtype=ws.dtype, device=dev)
-        Bsum = torch.empty(ws.B, ws.H, ws.C, dtype=torch.float32, device=dev)
-        hils.hils_summarize(p, inp["K"], inp["LQ"], Ksum, Bsum)
-        torch.cuda.synchronize()
-        host = {k: v.cpu() for k, v in inp.items() if isinstance(v, torch.Tensor)}
-        host["Ksum"], host["Bsum"] = Ksum.cpu(), Bsum.cpu()
-        del inp
         torch.cuda.empty_cache()
-    else:
-        import oracle
-
-        host = dict(inp)
-        ks, bs = oracle.summarize(host["K"], host["LQ"], ws.S, ws.scale)
-        host["Ksum"], host["Bsum"] = torch.from_numpy(ks).to(ws.dtype), torch.from_numpy(bs).float()
+    ks, bs = oracle.summarize(host["K"], host["LQ"], ws.S, ws.scale)
+    host["Ksum"], host["Bsum"] = torch.from_numpy(ks).to(ws.dtype), torch.from_numpy(bs).float()
     host["qpos"] = (host["cache_len"] - 1).reshape(ws.B, 1)
     return ws, host
 
@@ -376,7 +477,29 @@ def oracle_decode_step(ws, host):
     oracle.attend(host["Q"], host["K"], host["V"], idx, score, nsel, ws.S, ws.W, ws.scale, qpos=host["qpos"])
 
 
-def cpu_baseline(w, dev, heads=4, min_s=5.0, max_s=20.0):
+def oracle_single_thread():
+    """One-thread oracle times (seconds): the tiny float32 prefill (summarise, select,
+    attend over all 512 queries) and one head of the 8K prefill."""
+    import oracle
+
+    out = {}
+    n0 = oracle.get_threads()
+    oracle.set_threads(1)
+    try:
+        for name, w in (("tiny_fp32_prefill_s", WORKLOADS[1]), ("prefill_8k_one_head_s", WORKLOADS[2].replace(H=1))):
+            inp = make_prefill(w)
+            t0 = time.perf_counter()
+            ks, bs = oracle.summarize(inp["K"], inp["LQ"], w.S, w.scale)
+            ksum, bsum = torch.from_numpy(ks).to(w.dtype), torch.from_numpy(bs).float()
+            idx, score, nsel = oracle.select(inp["Qcal"], ksum, bsum, w.S, w.K, w.scale)
+            oracle.attend(inp["Q"], inp["K"], inp["V"], idx, score, nsel, w.S, w.W, w.scale)
+            out[name] = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(n0)
+    return out
+
+
+def cpu_baseline(w, dev, heads=4, min_s=5.0, max_s=20.0, single_thread=True):
     import oracle
 
     oracle.build()
@@ -390,15 +513,26 @@ def cpu_baseline(w, dev, heads=4, min_s=5.0, max_s=20.0):
         if el >= min_s or (el >= max_s):
             break
     per_step = el / reps * (w.H / heads)  # seconds for all heads of one token
-    return {"value": w.B / per_step, "unit": "tokens/s", "cores": oracle.get_threads(), "kind": "oracle",
-            "sample": f"{heads} of {w.H} heads of one decode step (select over {w.C - 1} chunks + attend), "
-                      f"{reps} repetitions in {el:.1f} s, time scaled by {w.H}/{heads}"}
+    out = {"value": w.B / per_step, "unit": "tokens/s", "cores": oracle.get_threads(), "kind": "oracle",
+           "sample": f"{heads} of {w.H} heads of one decode step (select over {w.C - 1} chunks + attend), "
+                     f"{reps} repetitions in {el:.1f} s, time scaled by {w.H}/{heads}; summaries by the "
+                     f"oracle (untimed)"}
+    if single_thread:
+        out["single_thread"] = oracle_single_thread()
+    return out
+
+
+def decode_config(w, world: int) -> dict:
+    """The `config` of a decode line, the same for both arms."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.Hkv, "d": w.d, "kv_len": w.N, "chunk": w.S,
+            "top_k": w.K, "window": w.W, "parallelism": f"replicas{world}", "l2": DECODE_L2}
 
 
 # ----------------------------------------------------------------- main
 
 def run_reference(args, w):
-    """The oracle as the reference arm: same metric and workload, on host cores."""
+    """The oracle as the reference arm: same metric, workload and config, on host cores;
+    the CUDA library is never loaded."""
     world, rank, local = dist_ctx()
     if world > 1 and rank != 0:
         return
@@ -416,15 +550,15 @@ def run_reference(args, w):
         oracle_decode_step(ws, host)
         t.append((time.perf_counter() - t0) * (w.H / heads))
     ms = 1e3 * statistics.mean(t)
-    value = w.B / (ms / 1e3)
+    value = world * w.B / (ms / 1e3)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "kv_len": w.N, "chunk": w.S,
-                       "top_k": w.K, "window": w.W, "parallelism": "replicas"},
+            "config": decode_config(w, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.get_threads(),
                              "kind": "oracle",
-                             "sample": f"{heads} of {w.H} heads per step, time scaled by {w.H}/{heads}"},
+                             "sample": f"{heads} of {w.H} heads per step, time scaled by {w.H}/{heads}; "
+                                       f"summaries by the oracle (untimed)"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -436,6 +570,8 @@ def run_profile_case(args):
                    random summary table (68 MB) without a KV cache;
     decode-select-gqa: the same with 8 key-value heads (groups of 4 query heads);
     decode-attend: the decode attend with H=32, K=16, W=512 on a 128K-token cache (2.1 GB);
+    decode-step:   the whole hils_decode step on that cache (select over 2047 chunks, attend);
+    summarize:     hils_summarize over a 1M-token cache of 4 heads (16384 chunks each, 1.1 GB of keys);
     prefill:       the full 8K prefill workload (summarise, select, attend);
     prefill-select: the select of the 8K prefill, multi-head then grouped-query (32 query
                    heads, 8 key-value heads), `warmup + steps` launches each.
@@ -459,10 +595,19 @@ def run_profile_case(args):
         nsel = torch.empty(w.B, w.Hkv, 1, dtype=torch.int32, device=dev)
         ws = hils.alloc_workspace(p, hils.HILS_CALL_SELECT, 1, w.C, device=dev)
         fn = lambda: hils.hils_select(p, Q, Ksum, Bsum, idx, score, nsel, qpos=qpos, workspace=ws)  # noqa
-    elif case == "decode-attend":
-        db = DecodeBench(WORKLOADS[4].replace(N=131072, needles=0), dev)
-        db.select()
-        fn = db.attend
+    elif case in ("decode-attend", "decode-step"):
+        db = DecodeBench(WORKLOADS[4].replace(N=131072, needles=0), dev, sets=1)
+        db.sets[0].select()
+        fn = db.sets[0].attend if case == "decode-attend" else db.sets[0].step
+    elif case == "summarize":
+        w = WORKLOADS[5].replace(H=4, needles=0)
+        p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype)
+        g = torch.Generator(device=dev).manual_seed(11)
+        K = torch.randn(w.B, w.H, w.N, w.d, generator=g, device=dev).to(w.dtype)
+        LQ = torch.randn(w.B, w.H, w.C, w.d, generator=g, device=dev).to(w.dtype)
+        Ksum = torch.empty(w.B, w.H, w.C, w.d, dtype=w.dtype, device=dev)
+        Bsum = torch.empty(w.B, w.H, w.C, dtype=torch.float32, device=dev)
+        fn = lambda: hils.hils_summarize(p, K, LQ, Ksum, Bsum)  # noqa
     elif case == "prefill":
         fn = PrefillBench(WORKLOADS[2], dev).step
     elif case == "prefill-select":
@@ -618,46 +763,133 @@ def measure_prefill_backward(w, dev, stream, flush, args, world):
     return out
 
 
-def measure_decode(w, dev, stream, flush, args, world, peaks):
-    """A secondary decode workload: hils_decode step time and its select and attend
-    kernels (L2 flushed), tokens/s and algorithmic GB/s."""
+def measure_decode(w, dev, stream, flush, args, world, peaks, peak_src, steps: int, headline: bool = False,
+                   rebuild: bool = False):
+    """One decode workload: the hils_decode step back to back over rotating input copies
+    (value, clocks), its select and attend kernels timed alone the same way, the same
+    step with per-step L2 flushes and events (cold single step), the HBM roofline of the
+    dominant kernel, and needle retention for workloads with planted needles.
+    headline: also the end-to-end figure with host buffers. rebuild: also a full
+    hils_summarize pass over every chunk of the cache, timed alone."""
     db = DecodeBench(w, dev)
-    n = max(3, min(args.steps, 50))
-    step_g, sel_g, att_g = graphed(db.step, stream), graphed(db.select, stream), graphed(db.attend, stream)
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            step_g()
-    stream.synchronize()
-    with ClockSampler(dev) as clk:
-        ms = statistics.mean(time_steps(step_g, n, flush, stream))
-    ms = max_over_ranks(ms, world, dev)
-    t_sel = statistics.mean(time_steps(sel_g, n, flush, stream))
-    t_att = statistics.mean(time_steps(att_g, n, flush, stream))
+    g_step = db.graphs("step", stream)
+    g_sel = db.graphs("select", stream)
+    g_att = db.graphs("attend", stream)
+    for _ in range(max(1, args.warmup // db.R)):
+        time_rotating(g_step, db.R, stream)
+    barrier(world)
     torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        ms = time_rotating(g_step, steps, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(ms, world, dev)
+    t_sel = time_rotating(g_sel, steps, stream)
+    t_att = time_rotating(g_att, steps, stream)
+    n_cold = max(3, min(steps, 50))
+    ms_cold = statistics.mean(time_steps(g_step[1][0], n_cold, flush, stream))
     by = decode_bytes(w)
     hbm = peaks["hbm_gbs"]
+    sel_gbs = by["select"] / (t_sel * 1e-3) / 1e9
+    att_gbs = by["attend"] / (t_att * 1e-3) / 1e9
+    step_gbs = by["step"] / (ms * 1e-3) / 1e9
+    dominant = "select" if t_sel >= t_att else "attend"
+    dom_gbs, dom_bytes = {"select": (sel_gbs, by["select"]), "attend": (att_gbs, by["attend"])}[dominant]
+    traffic = measured_traffic("decode_" + dominant, scale=dom_bytes)
     out = {"value": job_throughput(w.B, world, ms), "unit": "tokens/s", "ms_per_step": ms, "workload": w.name,
-           "H": w.H, "H_kv": w.Hkv, "steps": n, "clocks": clk.summary(),
-           "kernel_us": {"select": 1e3 * t_sel, "attend": 1e3 * t_att},
+           "config": decode_config(w, world), "steps": steps, "input_copies": db.R, "clocks": clk.summary(),
+           "kernel_us": {"select": 1e3 * t_sel, "attend": 1e3 * t_att, "select_gbs": sel_gbs,
+                         "attend_gbs": att_gbs},
            "algorithmic_bytes": by,
-           "select_frac_of_hbm": by["select"] / (t_sel * 1e-3) / 1e9 / hbm,
-           "attend_gbs": by["attend"] / (t_att * 1e-3) / 1e9,
-           "step_frac_of_hbm": by["step"] / (ms * 1e-3) / 1e9 / hbm}
-    del db, step_g, sel_g, att_g
+           "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom_gbs, "peak": hbm, "unit": "GB/s",
+                        "frac": dom_gbs / hbm, "traffic": traffic, "algorithmic_bytes": dom_bytes,
+                        "peak_source": f"{peak_src} HBM copy"},
+           "step_roofline": {"bytes": by["step"], "achieved_gbs": step_gbs, "frac_measured": step_gbs / hbm,
+                             "frac_8tbs": step_gbs / 8000.0},
+           "cold_single_step": {"ms": ms_cold, "tokens_per_s": job_throughput(w.B, world, ms_cold),
+                                "protocol": Flusher.DESCRIPTION + "; CUDA events around each step"},
+           "gpu_launches": steps * db.launches_per_step}
+    if w.needles:
+        s0 = db.sets[0]
+        ih, nh = s0.idx.cpu().numpy(), s0.nsel.cpu().numpy()
+        kept = total = 0
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                ks = set(ih[b, h, 0, : nh[b, h, 0]].tolist())
+                for pos in db.needles[b, h].tolist():
+                    total += 1
+                    kept += (pos // w.S) in ks
+        out["needle_chunks_kept"] = {"kept": kept, "of": total}
+    if headline:
+        sizes = [s.e2e_setup() for s in db.sets]
+        h2d, d2h = sizes[0]
+        try:
+            g_e2e = db.graphs("e2e_step", stream)
+            mode = "CUDA graph of the binding calls: H2D copies, hils_decode, D2H copies"
+        except Exception as e:  # noqa: BLE001  (capture of the copies refused: time the calls themselves)
+            def run_all():
+                for s in db.sets:
+                    s.e2e_step()
+            g_e2e = (run_all, [s.e2e_step for s in db.sets])
+            mode = f"binding calls launched eagerly (graph capture failed: {type(e).__name__})"
+        time_rotating(g_e2e, db.R, stream)
+        ms_e2e = max_over_ranks(time_rotating(g_e2e, steps, stream), world, dev)
+        out["e2e"] = {"value": job_throughput(w.B, world, ms_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h, "mode": mode}
+    del db, g_step, g_sel, g_att
     torch.cuda.empty_cache()
+    if rebuild:
+        out["summary_rebuild"] = measure_rebuild(w, dev, stream, flush, peaks, peak_src)
     return out
+
+
+def measure_rebuild(w, dev, stream, flush, peaks, peak_src, reps: int = 5):
+    """hils_summarize over every chunk of every head of the cache (Eq. 8), timed alone with
+    L2 flushed before each pass: algorithmic bytes = the keys, the landmark queries and
+    the written summaries."""
+    import hierarchical_chunk_sparse_b200 as hils
+
+    p = hils.Params(B=w.B, H=w.H, d=w.d, K=w.K, W=w.W, dtype=w.dtype, H_kv=w.Hk)
+    g = torch.Generator(device=dev).manual_seed(11)
+    K = torch.randn(w.B, w.Hkv, w.N, w.d, generator=g, device=dev).to(w.dtype)
+    LQ = torch.randn(w.B, w.H, w.C, w.d, generator=g, device=dev).to(w.dtype)
+    Ksum = torch.empty(w.B, w.H, w.C, w.d, dtype=w.dtype, device=dev)
+    Bsum = torch.empty(w.B, w.H, w.C, dtype=torch.float32, device=dev)
+
+    def fn():
+        hils.hils_summarize(p, K, LQ, Ksum, Bsum)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            fn()
+    stream.synchronize()
+    ms = statistics.mean(time_steps(fn, reps, flush, stream))
+    es = 2 if w.dtype == torch.bfloat16 else 4
+    nbytes = w.B * w.H * w.C * (w.S * w.d * es + w.d * es + w.d * es + 4)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del K, LQ, Ksum, Bsum
+    torch.cuda.empty_cache()
+    return {"ms": ms, "chunks": w.B * w.H * w.C, "algorithmic_bytes": nbytes,
+            "roofline": {"bound": "hbm", "kernel": "summarize", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "frac_8tbs": gbs / 8000.0,
+                         "traffic": measured_traffic("summarize", scale=w.B * w.H * w.C),
+                         "peak_source": f"{peak_src} HBM copy"},
+            "protocol": Flusher.DESCRIPTION + f"; {reps} passes, CUDA events around each"}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None,
-                    choices=["decode-select", "decode-select-gqa", "decode-attend", "prefill", "prefill-select"],
+                    choices=["decode-select", "decode-select-gqa", "decode-attend", "decode-step", "prefill",
+                             "prefill-select", "summarize"],
                     help="run a small case for an ncu capture and exit")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="hils", choices=["hils", "reference"])
-    ap.add_argument("--no-prefill", action="store_true", help="skip the 8K prefill measurement")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill and backward measurements")
+    ap.add_argument("--no-extra-decode", action="store_true",
+                    help="skip the decode workloads other than the 512K headline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -685,61 +917,28 @@ def main():
     stream = torch.cuda.Stream(dev)
     flush = Flusher(dev)
 
-    # ---------------- headline: decode @512K
-    db = DecodeBench(w, dev)
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            db.step()
-    stream.synchronize()
-    # one decode step = hils_decode (select, then attend, as one chain), replayed as a CUDA graph
-    step_g = graphed(db.step, stream)
-    sel_g = graphed(db.select, stream)
-    att_g = graphed(db.attend, stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step_g()
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(dev) as clk:
-        per = time_steps(step_g, args.steps, flush, stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    ms = max_over_ranks(statistics.mean(per), world, dev)
-    value = job_throughput(w.B, world, ms)
-    # per-kernel times (same protocol)
-    t_sel = statistics.mean(time_steps(sel_g, args.steps, flush, stream))
-    t_att = statistics.mean(time_steps(att_g, args.steps, flush, stream))
-    by = decode_bytes(w)
-    hbm = peaks["hbm_gbs"]
-    sel_gbs = by["select"] / (t_sel * 1e-3) / 1e9
-    att_gbs = by["attend"] / (t_att * 1e-3) / 1e9
-    step_gbs = by["step"] / (ms * 1e-3) / 1e9
-    dominant = "select" if t_sel >= t_att else "attend"
-    dom = {"select": (sel_gbs, by["select"]), "attend": (att_gbs, by["attend"])}[dominant]
-    # end to end through the binding with host buffers
-    h2d, d2h = db.e2e_setup()
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            db.e2e_step()
-    per_e2e = time_steps(db.e2e_step, args.steps, flush, stream)
-    ms_e2e = max_over_ranks(statistics.mean(per_e2e), world, dev)
-    launches = args.steps * db.launches_per_step
-    del db
-    torch.cuda.empty_cache()
+    # ---------------- headline: decode @512K, one step = hils_decode (select then attend)
+    head = measure_decode(w, dev, stream, flush, args, world, peaks, peak_src, args.steps, headline=True)
 
-    # ---------------- prefill @8K (iid queries; and the query-locality variant)
-    prefill = None
-    prefill_local = None
-    prefill_gqa = None
+    # ---------------- prefill @8K (iid queries; query locality; grouped-query heads)
+    prefill = prefill_local = prefill_gqa = prefill_bwd = None
     if not args.no_prefill:
         prefill = measure_prefill(WORKLOADS[2], dev, stream, flush, args, world, peaks, peak_src,
-                                  MEASURED_TRAFFIC["attend_prefill"])
+                                  measured_traffic("attend_prefill"))
         prefill_local = measure_prefill(WORKLOADS[6], dev, stream, flush, args, world, peaks, peak_src, None)
         prefill_gqa = measure_prefill(WORKLOADS[7], dev, stream, flush, args, world, peaks, peak_src, None)
-    # ---------------- grouped-query decode @512K (32 query heads, 8 key-value heads)
-    decode_gqa = measure_decode(WORKLOADS[8], dev, stream, flush, args, world, peaks)
+    # ---------------- the other decode workloads: batch of 8 at 128K, 1M (with the summary
+    # rebuild), grouped-query 512K, retrieval 512K
+    extra = {}
+    if not args.no_extra_decode:
+        n_extra = max(3, min(args.steps, 50))
+        for key, cfg, rb in (("decode_b8_128k", 3, False), ("decode_1m", 5, True), ("decode_gqa", 8, False),
+                             ("decode_retrieval", 9, False)):
+            extra[key] = measure_decode(WORKLOADS[cfg], dev, stream, flush, args, world, peaks, peak_src, n_extra,
+                                        rebuild=rb)
     # ---------------- backward of the 8K prefill (fixed selection)
-    prefill_bwd = None if args.no_prefill else measure_prefill_backward(WORKLOADS[2], dev, stream, flush, args, world)
+    if not args.no_prefill:
+        prefill_bwd = measure_prefill_backward(WORKLOADS[2], dev, stream, flush, args, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -747,28 +946,23 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "kv_len": w.N, "chunk": w.S,
-                       "top_k": w.K, "window": w.W, "parallelism": f"replicas{world}",
-                       "l2": Flusher.DESCRIPTION},
-            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom[0], "peak": hbm,
-                         "unit": "GB/s", "frac": dom[0] / hbm,
-                         "traffic": MEASURED_TRAFFIC[dominant if dominant == "select" else "attend_decode"],
-                         "algorithmic_bytes": dom[1], "peak_source": f"{peak_src} HBM copy"},
-            "step_roofline": {"bytes": by["step"], "achieved_gbs": step_gbs, "frac_measured": step_gbs / hbm,
-                              "frac_8tbs": step_gbs / 8000.0},
-            "kernel_us": {"select": 1e3 * t_sel, "attend": 1e3 * t_att,
-                          "select_gbs": sel_gbs, "attend_gbs": att_gbs},
-            "e2e": {"value": job_throughput(w.B, world, ms_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches,
-            "clocks": clk.summary(),
+            "config": head["config"],
+            "roofline": head["roofline"],
+            "step_roofline": head["step_roofline"],
+            "kernel_us": head["kernel_us"],
+            "cold_single_step": head["cold_single_step"],
+            "input_copies": head["input_copies"],
+            "needle_chunks_kept": head.get("needle_chunks_kept"),
+            "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"],
+            "clocks": head["clocks"],
             "prefill": prefill,
             "prefill_local": prefill_local,
             "prefill_gqa": prefill_gqa,
-            "decode_gqa": decode_gqa,
+            **extra,
             "prefill_backward": prefill_bwd,
             "cpu_baseline": cpu,
         }

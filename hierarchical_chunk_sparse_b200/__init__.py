@@ -33,7 +33,8 @@ _DTYPES = {torch.float32: HILS_F32, torch.bfloat16: HILS_BF16}
 # Every function the C header declares (checked by the tests against the header).
 EXPORTS = ("hils_summarize", "hils_select", "hils_attend_prefill", "hils_attend_decode", "hils_decode",
            "hils_attend_decode_noalloc", "hils_workspace_bytes", "hils_workspace_init",
-           "hils_status_string", "hils_last_cuda_error")
+           "hils_status_string", "hils_last_cuda_error", "hils_summarize_append", "hils_attend_prefill_backward",
+           "hils_select_backward", "hils_summarize_backward", "hils_selftest_fast_math")
 
 
 class HilsError(RuntimeError):
@@ -83,9 +84,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hils_status_string.argtypes = [i]
         lib.hils_status_string.restype = ctypes.c_char_p
         lib.hils_last_cuda_error.restype = ctypes.c_char_p
+        lib.hils_selftest_fast_math.argtypes = [vp, vp, i, vp, vp, vp]
         for name in ("hils_summarize", "hils_summarize_append", "hils_attend_prefill_backward",
-                     "hils_select_backward", "hils_summarize_backward", "hils_select", "hils_attend_prefill", "hils_attend_decode", "hils_decode",
-                     "hils_attend_decode_noalloc", "hils_workspace_init"):
+                     "hils_select_backward", "hils_summarize_backward", "hils_select", "hils_attend_prefill",
+                     "hils_attend_decode", "hils_decode", "hils_attend_decode_noalloc", "hils_workspace_init",
+                     "hils_selftest_fast_math"):
             getattr(lib, name).restype = i
         _lib = lib
     return _lib
@@ -396,3 +399,14 @@ def alloc_workspace(p: Params, call: int, Lq: int, C: int, device="cuda") -> tor
     ws = torch.empty((n + 15) // 16 * 16, dtype=torch.uint8, device=device)
     hils_workspace_init(ws)
     return ws
+
+
+def hils_selftest_fast_math(x, z, exp2_out, recip_out, stream=None) -> None:
+    """The library's FMA-pipe 2^x and 1/z helpers on every element of x and z (float32
+    CUDA tensors of one size), written to exp2_out and recip_out."""
+    n = x.numel()
+    for name, t in (("x", x), ("z", z), ("exp2_out", exp2_out), ("recip_out", recip_out)):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.numel() != n:
+            raise ValueError(f"hils_selftest_fast_math: {name} must be a dense float32 CUDA tensor of {n} elements")
+    _check("hils_selftest_fast_math", load_library().hils_selftest_fast_math(
+        _ptr(x), _ptr(z), n, _ptr(exp2_out), _ptr(recip_out), _stream(stream)))

@@ -51,6 +51,10 @@ extern "C" int hils_attend_decode_noalloc(const hils_params *p, hils_ctensor Q, 
                                           const int32_t *cache_len, const int32_t *idx, const float *score,
                                           const int32_t *nsel, hils_tensor O, float *lse, cudaStream_t stream) {
     using namespace hils;
+    // every argument check runs before anything touches the shared scratch, so a call
+    // that is rejected leaves no work queued on the stream
+    const int chk = check_attend_decode_args(p, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse);
+    if (chk != HILS_OK) return chk;
     const size_t need = hils_workspace_bytes(p, HILS_CALL_ATTEND_DECODE, 1, 0);
     if (need > kScratchBytes) return HILS_ERR_WORKSPACE;  // beyond the built-in capacity
     void *scratch = nullptr;

@@ -665,27 +665,35 @@ __global__ void __launch_bounds__(kThreads) select_backward_table_kernel(BwdSele
         const int64_t qg = ((int64_t)b * Hk + h / a.G) * a.Lq + i;
         const int ns = K > 0 ? min(max(a.nsel[qg], 0), K) : 0;
         const T *qrow = static_cast<const T *>(a.Qcal.ptr) + b * a.Qcal.sb + h * a.Qcal.sh + (int64_t)i * a.Qcal.st;
+        // lane k holds kept chunk k's index and gradient (K <= 32), so the k' row loads
+        // below depend only on shuffles and several can be in flight
+        int myc = 0;
+        float myds = 0.f;
+        if (lane < ns) {
+            const int c = a.idx[qg * K + lane];
+            const bool ok = (unsigned)c < (unsigned)C;
+            myc = ok ? c : 0;
+            myds = ok ? a.dscore[qi * K + lane] : 0.f;
+            if (ok) atomicOr(&touched[c >> 5], 1u << (c & 31));
+        }
         float qx[kPer], acc[kPer];
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
             qx[u] = a.scale * elem(qrow, lane + 32 * u);
             acc[u] = 0.f;
         }
+#pragma unroll 4
         for (int k = 0; k < ns; ++k) {
-            const int c = a.idx[qg * K + k];
-            if ((unsigned)c >= (unsigned)C) continue;
-            const float ds = a.dscore[qi * K + k];
+            const int c = __shfl_sync(kFull, myc, k);
+            const float ds = __shfl_sync(kFull, myds, k);
             const T *krow = khead + (int64_t)c * a.Ksum.st;
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
                 acc[u] = fmaf(ds, elem(krow, lane + 32 * u), acc[u]);
                 atomicAdd(&tk[c * D + lane + 32 * u], ds * qx[u]);
             }
-            if (lane == 0) {
-                atomicAdd(&tb[c], ds);
-                atomicOr(&touched[c >> 5], 1u << (c & 31));
-            }
         }
+        if (lane < ns) atomicAdd(&tb[myc], myds);
 #pragma unroll
         for (int u = 0; u < kPer; ++u) a.dQcal[qi * D + lane + 32 * u] = a.scale * acc[u];
     }

@@ -190,6 +190,17 @@ int prepare_attend_decode(const hils_params *p, hils_ctensor Q, hils_ctensor Kc,
     return HILS_OK;
 }
 
+}  // namespace
+
+int check_attend_decode_args(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hils_ctensor Vc,
+                             const int32_t *cache_len, const int32_t *idx, const float *score, const int32_t *nsel,
+                             hils_tensor O, float *lse) {
+    AttendArgs a{};
+    return prepare_attend_decode(p, Q, Kc, Vc, cache_len, idx, score, nsel, O, lse, &a);
+}
+
+namespace {
+
 // The select part of a hils_decode workspace, rounded so the attend part starts aligned.
 size_t decode_select_part(size_t select_bytes) { return (select_bytes + 255) & ~(size_t)255; }
 

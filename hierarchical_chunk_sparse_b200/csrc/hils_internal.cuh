@@ -138,6 +138,10 @@ bool select_tc_supported(hils_dtype dt, int d, int B, int H, int Lq, int C, int 
 hils_status launch_select_tc(const SelectArgs &a, cudaStream_t s);
 
 int device_sm_count();
+// The argument checks of hils_attend_decode (parameters, views, arrays), without launching.
+int check_attend_decode_args(const hils_params *p, hils_ctensor Q, hils_ctensor Kc, hils_ctensor Vc,
+                             const int32_t *cache_len, const int32_t *idx, const float *score, const int32_t *nsel,
+                             hils_tensor O, float *lse);
 hils_status record_cuda_error(cudaError_t e);
 
 // Per-kernel launch set-up done once per device: the dynamic shared memory opt-in and

@@ -311,6 +311,17 @@ int hils_select_backward(const hils_params *p, hils_ctensor Qcal, int Lq, hils_c
 int hils_summarize_backward(const hils_params *p, hils_ctensor K, int N, hils_ctensor LQ,
                             const float *dKsum, const float *dBsum, float *dK, float *dLQ, cudaStream_t stream);
 
+/* Diagnostic (no counterpart on the pages): evaluates the two FMA-pipe helpers that the
+ * tensor-core prefill attend uses instead of MUFU instructions, element by element:
+ *   exp2_out[i]  = 2^x[i]  (a fitted degree-5 polynomial; relative error <= 2.4e-7 for
+ *                  x in [-125, 127]; x below -125 gives 2^-125)
+ *   recip_out[i] = 1/z[i]  (an integer seed and two Newton steps; relative error
+ *                  <= 7e-6 for normal positive z)
+ * x, z, exp2_out, recip_out: device arrays of n floats. Returns HILS_ERR_INVALID_ARG
+ * for n < 0 or a null pointer with n > 0. */
+int hils_selftest_fast_math(const float *x, const float *z, int n, float *exp2_out, float *recip_out,
+                            cudaStream_t stream);
+
 /* Bytes of workspace a call needs for these sizes (Lq = queries per (b, h); C =
  * summarised chunks). Returns 0 for invalid parameters. */
 size_t hils_workspace_bytes(const hils_params *p, int call, int Lq, int C);

@@ -64,3 +64,47 @@ def test_backward_flops_8k():
     want = H * (10 * d * tok + 4 * d * kept + 8 * d * S * 128)
     assert bench.backward_flops(w) == want
     assert round(want / 1e9, 1) == 489.5
+
+
+def test_decode_input_copies_cover_three_l2_sizes():
+    """Decode steps cycle over R input copies; R is the least count >= 2 whose bytes per
+    cycle reach three L2 sizes, so a copy is evicted before it is read again."""
+    l2 = 126 * 2**20
+    for cfg in (3, 4, 5, 8, 9):
+        w = WORKLOADS[cfg]
+        step = bench.decode_bytes(w)["step"]
+        R = bench.decode_sets(w, l2)
+        assert R >= 2 and R * step >= 3 * l2
+        assert R == 2 or (R - 1) * step < 3 * l2
+    assert bench.decode_sets(WORKLOADS[4], l2) == 5  # 93.3 MB per step
+
+
+def test_traffic_record_goes_null_when_the_kernel_changes(monkeypatch):
+    """A traffic capture counts only for the source it was taken on."""
+    dig = bench.source_digest("summarize")
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "summarize", (17000.0, dig))
+    assert bench.measured_traffic("summarize", scale=10) == 170000.0
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "summarize", (17000.0, "0" * 16))
+    assert bench.measured_traffic("summarize", scale=10) is None
+
+
+def test_reference_arm_runs_the_oracle_alone(tmp_path):
+    """The reference arm on a small decode workload: one JSON line with the config of
+    the library's arm, and the CUDA library never imported."""
+    import json
+    import subprocess
+
+    code = (
+        "import sys, json, types; sys.path.insert(0, %r); import bench; from hils_synth import WORKLOADS;"
+        "w = WORKLOADS[4].replace(H=4, N=64 * 300, needles=1);"
+        "bench.run_reference(types.SimpleNamespace(gpus=1, steps=2, warmup=1), w);"
+        "assert 'hierarchical_chunk_sparse_b200' not in sys.modules;"
+        "print(json.dumps(bench.decode_config(w, 1)))" % ROOT)
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, timeout=300)
+    assert out.returncode == 0, out.stderr
+    lines = [json.loads(x) for x in out.stdout.strip().splitlines()]
+    ref, cfg = lines[0], lines[1]
+    assert ref["impl"] == "reference" and ref["config"] == cfg
+    assert ref["value"] > 0 and ref["steps"] == 2 and ref["warmup"] == 1
+    assert ref["e2e"]["h2d_bytes_per_step"] == 0 and ref["cpu_baseline"]["kind"] == "oracle"

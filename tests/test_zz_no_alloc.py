@@ -13,7 +13,7 @@ from hils_testutil import assert_close
 pytestmark = pytest.mark.gpu
 
 
-def test_noalloc_decode_matches_workspace_decode(cuda_device):
+def test_noalloc_decode_matches_workspace_decode(oracle, cuda_device):
     w = WORKLOADS[4].replace(B=2, H=4, N=6000, needles=0)
     inp = make_decode(w)
     inp["cache_len"] = torch.tensor([6000, 4097], dtype=torch.int32)
@@ -36,6 +36,9 @@ def test_noalloc_decode_matches_workspace_decode(cuda_device):
     hils.hils_attend_decode(p, d["Q"], d["K"], d["V"], d["cache_len"], idx, score, nsel, O_ref, lse_ref,
                             workspace=ws)
     ref = O_ref.double().cpu().numpy()
+    # the float64 oracle fed the same selection
+    O_or, lse_or = oracle.attend(inp["Q"], inp["K"], inp["V"], idx.cpu(), score.cpu(), nsel.cpu(), 64, w.W,
+                                 w.scale, qpos=qpos.cpu())
     for call in range(2):  # the second call reuses the scratch left by the first
         O = torch.full_like(d["Q"], 7.0)
         lse = torch.full((w.B, w.H), 7.0, dtype=torch.float32, device=cuda_device)
@@ -43,6 +46,24 @@ def test_noalloc_decode_matches_workspace_decode(cuda_device):
         torch.cuda.synchronize()
         assert_close(O, ref, w.dtype, f"O call {call}")
         assert_close(lse, lse_ref.double().cpu().numpy(), torch.float32, f"lse call {call}")
+        assert_close(O, O_or, w.dtype, f"O call {call} vs oracle")
+        assert_close(lse, lse_or[:, :, 0], torch.float32, f"lse call {call} vs oracle")
+
+
+def test_noalloc_rejects_bad_arguments_before_any_work(cuda_device):
+    """A misaligned output view is rejected with the same status as hils_attend_decode,
+    before the call queues anything."""
+    p = hils.Params(B=1, H=2, d=128, K=4, W=64, dtype=torch.bfloat16)
+    Q = torch.zeros(1, 2, 1, 128, dtype=torch.bfloat16, device=cuda_device)
+    KV = torch.zeros(1, 2, 640, 128, dtype=torch.bfloat16, device=cuda_device)
+    cl = torch.full((1,), 640, dtype=torch.int32, device=cuda_device)
+    idx = torch.zeros(1, 2, 1, 4, dtype=torch.int32, device=cuda_device)
+    sc = torch.zeros(1, 2, 1, 4, device=cuda_device)
+    ns = torch.zeros(1, 2, 1, dtype=torch.int32, device=cuda_device)
+    O = torch.zeros(1, 2, 1, 136, dtype=torch.bfloat16, device=cuda_device)[..., 1:129]  # 2-byte offset
+    with pytest.raises(hils.HilsError) as err:
+        hils.hils_attend_decode_noalloc(p, Q, KV, KV, cl, idx, sc, ns, O)
+    assert err.value.status == 3
 
 
 def test_noalloc_rejects_problems_beyond_its_capacity(cuda_device):
