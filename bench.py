@@ -267,23 +267,41 @@ class DecodeSet:
                               self.idx, self.score, self.nsel, self.O, self.lse, workspace=self.ws_step)
 
     def e2e_setup(self):
-        """Pinned host copies of the step's inputs (query, calibrated query, cache
-        lengths) and of its results (O, lse)."""
+        """The step's inputs (query, calibrated query, cache lengths) and results (O, lse)
+        move through one pinned host buffer each way: the device tensors the library
+        reads and writes become views of one staging buffer per direction, so a step
+        costs one host-to-device and one device-to-host copy."""
         i = self.inp
-        self.h_in = {k: i[k].cpu().pin_memory() for k in ("Q", "Qcal", "cache_len")}
-        self.h_O = torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory()
-        self.h_lse = torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
-        d2h = self.h_O.numel() * self.h_O.element_size() + self.h_lse.numel() * self.h_lse.element_size()
-        return h2d, d2h
+        ins = [("Q", i["Q"]), ("Qcal", i["Qcal"]), ("cache_len", i["cache_len"])]
+        outs = [("O", self.O), ("lse", self.lse)]
+        self.d_in, views_in = _staging(ins, self.O.device)
+        self.d_out, views_out = _staging(outs, self.O.device)
+        for k, v in views_in.items():
+            v.copy_(i[k])
+            i[k] = v
+        self.O, self.lse = views_out["O"], views_out["lse"]
+        self.h_in = self.d_in.cpu().pin_memory()
+        self.h_out = torch.empty(self.d_out.shape, dtype=torch.uint8).pin_memory()
+        return self.h_in.numel(), self.h_out.numel()
 
     def e2e_step(self):
-        i = self.inp
-        for k, t in self.h_in.items():
-            i[k].copy_(t, non_blocking=True)
+        self.d_in.copy_(self.h_in, non_blocking=True)
         self.step()
-        self.h_O.copy_(self.O, non_blocking=True)
-        self.h_lse.copy_(self.lse, non_blocking=True)
+        self.h_out.copy_(self.d_out, non_blocking=True)
+
+
+def _staging(named, dev):
+    """One device byte buffer holding every tensor of `named` (16-byte aligned offsets),
+    and a view of the buffer for each tensor with its shape and dtype."""
+    off, spans = 0, []
+    for name, t in named:
+        off = (off + 15) // 16 * 16
+        n = t.numel() * t.element_size()
+        spans.append((name, t, off, n))
+        off += n
+    buf = torch.zeros(off, dtype=torch.uint8, device=dev)
+    views = {name: buf[o:o + n].view(t.dtype).view(t.shape) for name, t, o, n in spans}
+    return buf, views
 
 
 class DecodeBench:

@@ -603,6 +603,12 @@ def test_decode_workload_full_size(oracle, cuda_device, cfg):
                 kept = set(ih[b, h, 0, : nh[b, h, 0]].tolist())
                 assert set((inp["needles"][b, h] // 64).tolist()) <= kept, (b, h)
     O, lse = gpu_decode(w, inp["Q"], inp["K"], inp["V"], inp["cache_len"], idx, score, nsel)
+    # the whole step in one call (the launch configuration the benchmark times): the same
+    # selection, and the outputs of the separate calls within rounding
+    i2, s2, n2, O2, l2, _ = _decode_chain(w, inp, Ksum, Bsum)
+    assert torch.equal(idx, i2) and torch.equal(nsel, n2) and torch.equal(score, s2), f"cfg{cfg} hils_decode"
+    assert_close(O2, host(O).double().numpy(), w.dtype, "O hils_decode vs separate calls")
+    assert np.abs(host(l2).double().numpy() - host(lse).double().numpy()).max() <= 1e-4
     g = torch.Generator().manual_seed(cfg)
     for _ in range(3):
         b = int(torch.randint(0, w.B, (1,), generator=g))
@@ -620,7 +626,9 @@ def test_decode_workload_full_size(oracle, cuda_device, cfg):
                                        host(nsel[b:b + 1, h:h + 1]), 64, w.W, w.scale,
                                        qpos=host(qpos[b:b + 1]))
         assert_close(O[b:b + 1, h:h + 1], O_ref, w.dtype, f"O b{b} h{h}")
+        assert_close(O2[b:b + 1, h:h + 1], O_ref, w.dtype, f"O hils_decode b{b} h{h}")
         assert abs(float(lse[b, h]) - lse_ref[0, 0, 0]) <= 1e-4
+        assert abs(float(l2[b, h]) - lse_ref[0, 0, 0]) <= 1e-4
     del inp
     torch.cuda.empty_cache()
 
