@@ -26,6 +26,8 @@ HILS_CALL_SELECT, HILS_CALL_ATTEND_PREFILL, HILS_CALL_ATTEND_DECODE, HILS_CALL_D
 HILS_CALL_ATTEND_BACKWARD = 4
 # hils_params.flags: chunks wholly inside a query's window are not selected
 HILS_FLAG_EXCLUDE_WINDOW_CHUNKS = 1
+# hils_params.flags, diagnostic: the tensor-core kernels' waits on work in progress expire at once
+HILS_FLAG_DIAG_EXPIRE_WAITS = 0x80000000
 STATUS = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARG", 2: "HILS_ERR_UNSUPPORTED",
           3: "HILS_ERR_ALIGNMENT", 4: "HILS_ERR_WORKSPACE", 5: "HILS_ERR_CUDA"}
 _DTYPES = {torch.float32: HILS_F32, torch.bfloat16: HILS_BF16}

@@ -33,9 +33,10 @@
 // reuses the buffer), which also makes the softmax's waits for O on it exact.
 // TMEM: S_A0 [0,64), S_A1 [64,128), S_B0 [128,192), S_B1 [192,256), O_A [256,384),
 // O_B [384,512).
-// Every mbarrier wait is bounded: on expiry the CTA records an error in the status word,
-// every role stops issuing work, the CTA drains the copies and MMAs it started, frees
-// its TMEM and exits; outputs of unfinished items are not written.
+// Every mbarrier wait is bounded in time (the global timer): on expiry the CTA records an
+// error in the status word, every role stops issuing work, the CTA drains the copies and
+// MMAs it started (each drain wait bounded again), frees its TMEM and exits; outputs of
+// unfinished items are not written.
 #include "tc_common.cuh"
 #include "fast_math.cuh"
 
@@ -54,7 +55,6 @@ constexpr int kThreads = 384;
 constexpr int kStages = 4;       // K/V ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxBitmapWords = 256;  // union bitmap: up to 8192 chunks
-constexpr long long kWaitLimit = 1ll << 26;
 
 // shared memory map (offsets from the 1024-aligned base)
 constexpr int kQOff = 0;                                  // 2 tiles x 2 blocks x [128 rows x 128 B]
@@ -199,16 +199,30 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     tc_fence_after();
     const uint32_t tmem = misc[0];
 
-    // bounded wait; false once the CTA has aborted (the first expiry sets the flag)
+    // bounded wait on work in progress (a.wait_ns of the global timer; zero, a diagnostic:
+    // every such wait expires at once); false once the CTA has aborted (the first expiry
+    // sets the flag)
     auto wait = [&](uint32_t barrier, uint32_t parity) -> bool {
-        if (mbar_try_wait(barrier, parity)) return true;
-        for (long long it = 0; it < kWaitLimit; ++it) {
+        if (a.wait_ns > 0) {
             if (mbar_try_wait(barrier, parity)) return true;
-            if ((it & 255) == 255 && *abort_flag) return false;
+            const uint64_t t0 = global_ns();
+            for (int it = 0;; ++it) {
+                if (mbar_try_wait(barrier, parity)) return true;
+                if ((it & 15) == 15) {
+                    if (*abort_flag) return false;
+                    if ((long long)(global_ns() - t0) > a.wait_ns) break;
+                }
+            }
         }
         *abort_flag = 1u;
         atomicOr(args.status, 1u);
         return false;
+    };
+    // bounded wait for a phase of this CTA's own copies or MMAs while it stops
+    auto drain_wait = [&](uint32_t barrier, uint32_t parity) {
+        const uint64_t t0 = global_ns();
+        while (!mbar_try_wait(barrier, parity))
+            if ((long long)(global_ns() - t0) > kDrainLimitNs) break;
     };
     // warp-uniform form: every lane waits, the warp goes on only if all succeeded
     auto wait_warp = [&](uint32_t barrier, uint32_t parity) -> bool {
@@ -330,12 +344,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             __syncwarp();
             if (lane == 0) arrive(bar(kBarMapFree + par));
         }
-        // after an abort: the copies this warp started land before the CTA releases its memory
-        if (lane == 0 && *abort_flag) {
+        // every copy this warp started lands before the CTA releases its memory (after a
+        // normal finish every one was awaited by the MMA warps, so this returns at once)
+        if (lane == 0) {
             auto drain = [&](uint32_t b, int issued) {
                 if (issued == 0) return;
-                for (long long it = 0; it < kWaitLimit; ++it)
-                    if (mbar_try_wait(b, (uint32_t)(issued - 1) & 1u)) break;
+                drain_wait(b, (uint32_t)(issued - 1) & 1u);
             };
             drain(bar(kBarQfull), issuedQ);
             for (int s = 0; s < kStages; ++s) {  // uses of slot s among the first n ring entries
@@ -418,8 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         // every MMA this warp issued completes before TMEM and shared memory are released
         if (lane == 0) {
             mma_commit(bar(kBarDrain + xm));
-            for (long long it = 0; it < kWaitLimit; ++it)
-                if (mbar_try_wait(bar(kBarDrain + xm), 0)) break;
+            drain_wait(bar(kBarDrain + xm), 0);
         }
         __syncwarp();
     } else {

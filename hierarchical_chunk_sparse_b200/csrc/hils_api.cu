@@ -60,7 +60,8 @@ int check_params(const hils_params *p, float *scale) {
     if (p->d != 64 && p->d != 128) return HILS_ERR_UNSUPPORTED;
     if (p->S != kChunk) return HILS_ERR_UNSUPPORTED;
     if (p->K > 32) return HILS_ERR_UNSUPPORTED;
-    if (p->flags & ~(uint32_t)HILS_FLAG_EXCLUDE_WINDOW_CHUNKS) return HILS_ERR_UNSUPPORTED;
+    if (p->flags & ~(uint32_t)(HILS_FLAG_EXCLUDE_WINDOW_CHUNKS | HILS_FLAG_DIAG_EXPIRE_WAITS))
+        return HILS_ERR_UNSUPPORTED;
     if (!isfinite(p->scale)) return HILS_ERR_INVALID_ARG;
     if (p->H_kv < 0 || (p->H_kv > 0 && p->H % p->H_kv != 0)) return HILS_ERR_INVALID_ARG;
     if (p->H_kv > 0 && p->H / p->H_kv > kMaxGroupHeads) return HILS_ERR_UNSUPPORTED;
@@ -151,6 +152,8 @@ int prepare_select(const hils_params *p, hils_ctensor Qcal, int Lq, const int32_
     a->G = groups(p);
     a->excl_w = (p->flags & HILS_FLAG_EXCLUDE_WINDOW_CHUNKS) ? p->W : 0;
     if (nq > 0) select_plan(p->dtype, p->d, p->B, p->H, Lq, C, p->K, qpos != nullptr, device_sm_count(), a);
+    // the diagnostic expiry applies to the tensor-core select, which writes nothing after one
+    a->wait_ns = a->path == kSelectTc ? work_wait_ns(p->flags) : kWaitLimitNs;
     return HILS_OK;
 }
 
@@ -457,6 +460,7 @@ int hils_attend_prefill(const hils_params *p, hils_ctensor Q, hils_ctensor K, hi
     a.units = decode_units(p);
     a.ws = workspace;
     a.G = groups(p);
+    a.wait_ns = work_wait_ns(p->flags);
     if (attend_prefill_tc_supported(p->dtype, p->d, N))
         return launch_attend_prefill_tc(a, N, static_cast<uint32_t *>(workspace), stream);
     return launch_attend_prefill_general(p->dtype, p->d, a, stream);

@@ -14,6 +14,14 @@ constexpr unsigned kFull = 0xffffffffu;
 
 typedef __nv_bfloat16 bf16;
 
+// Time limits of the kernels' bounded waits (mbarrier phases of copies, tensor-core
+// operations and other warps' hand-offs): a wait that runs past its limit sets the
+// call's status word and the kernel stops, drains what it started and returns.
+constexpr long long kWaitLimitNs = 100ll * 1000 * 1000;   // waits on work in progress
+constexpr long long kDrainLimitNs = 100ll * 1000 * 1000;  // waits for a stopped CTA's own copies and MMAs
+// The work-wait limit of a call: zero under HILS_FLAG_DIAG_EXPIRE_WAITS (diagnostic).
+inline long long work_wait_ns(uint32_t flags) { return (flags & HILS_FLAG_DIAG_EXPIRE_WAITS) ? 0 : kWaitLimitNs; }
+
 // ------------------------------------------------------------------ launch args
 
 // Strided [B, H, T, d] view in elements.
@@ -53,6 +61,7 @@ struct SelectArgs {
     int ctas_per_query;    // summary blocks per query of the screen kernel
     int tiles_per_warp;    // 128-chunk tiles each warp scans
     void *ws;              // status word, then the screen values of the split search
+    long long wait_ns = kWaitLimitNs;  // limit of a bounded wait on work in progress (0: expire at once)
 };
 
 // Which select kernels run: one warp per query; screen + pick (few queries, long
@@ -77,6 +86,7 @@ struct AttendArgs {
     int window_early;      // decode: window tiles may start before the preceding grid ends
     void *ws;
     int G = 1;             // query heads per key-value head: K, V, idx and nsel have H / G heads
+    long long wait_ns = kWaitLimitNs;  // limit of a bounded wait on work in progress (0: expire at once)
 };
 
 // Host launchers (one translation unit each). They return HILS_OK or HILS_ERR_CUDA.
@@ -177,6 +187,13 @@ hils_status launch_dependent(const void *func, dim3 grid, dim3 block, size_t sme
 // Programmatic dependent launch: wait for the preceding grid's completion (and its
 // memory), and allow the next dependent-launched grid to be scheduled.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Nanoseconds of the GPU's global timer: the clock of every bounded wait.
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
 template <typename T>

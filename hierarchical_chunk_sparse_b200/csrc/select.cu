@@ -104,7 +104,6 @@ constexpr int kScrThreads = 256;
 constexpr int kPickThreads = 256;
 constexpr int kScrRows = 128;   // summary rows per item (one pipeline stage)
 constexpr int kDecStages = 3;   // pipeline stages (2 CTAs per SM for bf16 rows of d = 128)
-constexpr long long kScreenWaitLimit = 1ll << 26;  // polls of a stage's barrier before giving up
 
 template <typename T, int D>
 struct ScrCfg : StageCfg<T, D, kScrThreads, kScrRows> {
@@ -193,8 +192,12 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid
         cp_async_wait<Cfg::kStages - 1>();
         if (Cfg::kMma) {  // the stage's rows: use sq / kStages of its barrier
             const uint32_t bar = tc::smem_u32(&sbar[stage]), par = (uint32_t)(sq / Cfg::kStages) & 1u;
-            bool ok = false;
-            for (long long it = 0; it < kScreenWaitLimit && !ok; ++it) ok = tc::mbar_try_wait(bar, par);
+            bool ok = tc::mbar_try_wait(bar, par);
+            const uint64_t t0 = global_ns();
+            for (int it = 0; !ok; ++it) {
+                ok = tc::mbar_try_wait(bar, par);
+                if (!ok && (it & 15) == 15 && (long long)(global_ns() - t0) > a.wait_ns) break;
+            }
             if (!ok) {
                 sabort = 1u;
                 atomicOr(static_cast<uint32_t *>(a.ws), 1u);
@@ -266,8 +269,9 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid
         for (int k = 0; k < Cfg::kStages; ++k) {
             if (tma_issued[k] == 0) continue;
             const uint32_t bar = tc::smem_u32(&sbar[k]), par = (uint32_t)(tma_issued[k] - 1) & 1u;
-            for (long long it = 0; it < kScreenWaitLimit; ++it)
-                if (tc::mbar_try_wait(bar, par)) break;
+            const uint64_t t0 = global_ns();
+            while (!tc::mbar_try_wait(bar, par))
+                if ((long long)(global_ns() - t0) > kDrainLimitNs) break;
         }
     }
 }

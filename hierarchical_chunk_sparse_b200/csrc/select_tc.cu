@@ -57,7 +57,6 @@ constexpr int kMaxCols = 512;      // TMEM columns: eligible chunks per CTA time
 constexpr int kCap = 32;           // candidate slots per query (one spare slot absorbs overflow)
 constexpr int kBandCap = 8;        // float64 rescoring slots per query
 constexpr int kCollectPasses = 6;
-constexpr long long kSelWaitLimit = 1ll << 26;
 constexpr int kQBytes = 2 * kQM * 128;  // one head's query tile: 2 column blocks x 128 rows x 128 B
 
 // Reused region (after the MMAs have read the operands): per-thread candidate lists,
@@ -237,13 +236,26 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
     const int nrows = (nc + 63) & ~63;
 
     volatile uint32_t *abort_flag = &misc->abort;
+    // bounded wait on work in progress (a.wait_ns of the global timer; zero, a diagnostic:
+    // every such wait expires at once)
     auto wait = [&](uint32_t barrier, uint32_t parity) {
         if (*abort_flag) return false;
-        for (long long it = 0; it < kSelWaitLimit; ++it)
+        if (a.wait_ns > 0) {
             if (mbar_try_wait(barrier, parity)) return true;
+            const uint64_t t0 = global_ns();
+            for (int it = 0;; ++it) {
+                if (mbar_try_wait(barrier, parity)) return true;
+                if ((it & 15) == 15 && (long long)(global_ns() - t0) > a.wait_ns) break;
+            }
+        }
         *abort_flag = 1u;
         atomicOr(args.status, 1u);
         return false;
+    };
+    auto drain_wait = [&](uint32_t barrier, uint32_t parity) {  // this CTA's own copies and MMAs
+        const uint64_t t0 = global_ns();
+        while (!mbar_try_wait(barrier, parity))
+            if ((long long)(global_ns() - t0) > kDrainLimitNs) break;
     };
 
     // thread 0's record of what it started: loads per buffer, MMAs, the final commit
@@ -340,13 +352,11 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
         if (tid == 0) {  // let every started copy and MMA complete before leaving
             for (int bf = 0; bf < 2; ++bf) {
                 if (loads[bf] == 0) continue;  // each load was issued after the previous one of its buffer completed
-                for (long long it = 0; it < kSelWaitLimit; ++it)
-                    if (mbar_try_wait(bar_load[bf], (uint32_t)(loads[bf] - 1) & 1u)) break;
+                drain_wait(bar_load[bf], (uint32_t)(loads[bf] - 1) & 1u);
             }
             if (issued_mma) {
                 if (!committed) mma_commit(bar_done);
-                for (long long it = 0; it < kSelWaitLimit; ++it)
-                    if (mbar_try_wait(bar_done, 0)) break;
+                drain_wait(bar_done, 0);
             }
         }
         tc_fence_before();

@@ -109,6 +109,17 @@ typedef struct {
  *     counted in both; without the flag it may (the default). Only hils_select and
  *     hils_decode read the flag; summaries and the attend calls are unchanged. */
 #define HILS_FLAG_EXCLUDE_WINDOW_CHUNKS 1u
+/*   HILS_FLAG_DIAG_EXPIRE_WAITS: diagnostic, for tests of the failure path. The
+ *     tensor-core kernels of hils_select (bf16, d = 128, many queries) and of
+ *     hils_attend_prefill (bf16, d = 128) bound every wait on work in progress (copies,
+ *     tensor-core operations, other warps' hand-offs) by a time limit of the GPU's
+ *     global timer (0.1 s). With this flag every such wait expires at its first check,
+ *     whether or not its phase has completed. The kernel then sets the call's status word (the
+ *     first 4 bytes of its workspace, bit 0), stops issuing work, waits (bounded by the
+ *     normal limit) for the copies and operations it already started, releases its
+ *     tensor memory and returns without writing the outputs of unfinished work. Other
+ *     calls and other kernels ignore the flag. */
+#define HILS_FLAG_DIAG_EXPIRE_WAITS 0x80000000u
 
 /* Problem description shared by every call.
  *   B      batch (sequences), H query heads,
@@ -118,7 +129,8 @@ typedef struct {
  *   W      sliding-window length in tokens: >= 0,
  *   dtype  element type of every Q/K/V/LQ/Ksum/O tensor,
  *   scale  softmax scale; 0 selects (float)(1/sqrt(d)),
- *   flags  0, or HILS_FLAG_EXCLUDE_WINDOW_CHUNKS (below); other bits are rejected,
+ *   flags  0, or HILS_FLAG_EXCLUDE_WINDOW_CHUNKS and HILS_FLAG_DIAG_EXPIRE_WAITS (above);
+ *          other bits are rejected,
  *   H_kv   key-value heads: 0 (= H) or a divisor of H with H / H_kv <= 8; groups of
  *          G = H / H_kv query heads share a key-value head and their chunk selection
  *          (see above). */

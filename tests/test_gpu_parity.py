@@ -425,6 +425,46 @@ def test_prefill_query_locality_workload(oracle, cuda_device):
     assert np.mean(unions) < 40, np.mean(unions)
 
 
+def test_bounded_waits_expire_and_recover(oracle, cuda_device):
+    """The tensor-core select and prefill attend with every wait on work in progress made
+    to expire at its first check (HILS_FLAG_DIAG_EXPIRE_WAITS): each call returns with
+    bit 0 of its status word set and every output left as it was (the copies and
+    tensor-core operations started before the expiry are drained, tensor memory is
+    released); then the same calls with the normal time limit give the oracle's
+    results."""
+    w = WORKLOADS[2].replace(H=2, N=1536 + 37)  # 3146 queries: the tensor-core select
+    inp = make_prefill(w)
+    d = to_dev(inp, cuda_device)
+    Ksum, Bsum = gpu_summarize(w, d["K"], d["LQ"])
+    pd = P(w, flags=hils.HILS_FLAG_DIAG_EXPIRE_WAITS)
+    B, H, N, K = w.B, w.H, w.N, w.K
+    # select
+    ws = hils.alloc_workspace(pd, hils.HILS_CALL_SELECT, N, Ksum.shape[2], device=cuda_device)
+    idx = torch.full((B, H, N, K), 7777, dtype=torch.int32, device=cuda_device)
+    score = torch.full((B, H, N, K), 7777.0, device=cuda_device)
+    nsel = torch.full((B, H, N), 7777, dtype=torch.int32, device=cuda_device)
+    hils.hils_select(pd, d["Qcal"], Ksum, Bsum, idx, score, nsel, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(host(ws[:4]).view(torch.int32)[0]) & 1, "select: no wait expired"
+    i1, s1, n1 = gpu_select(w, d["Qcal"], Ksum, Bsum)
+    i_ref, _, n_ref = oracle.select(inp["Qcal"], host(Ksum), host(Bsum), 64, K, w.scale)
+    assert_same_selection(i1, n1, i_ref, n_ref, "select after the diagnostic call")
+    assert (host(nsel) == 7777).all() and (host(idx) == 7777).all() and (host(score) == 7777.0).all(), \
+        "the diagnostic select wrote outputs"
+    # prefill attend
+    wsa = hils.alloc_workspace(pd, hils.HILS_CALL_ATTEND_PREFILL, N, 0, device=cuda_device)
+    O = torch.full_like(d["Q"], 99.0)
+    lse = torch.full((B, H, N), 99.0, device=cuda_device)
+    hils.hils_attend_prefill(pd, d["Q"], d["K"], d["V"], i1, s1, n1, O, lse, workspace=wsa)
+    torch.cuda.synchronize()
+    assert int(host(wsa[:4]).view(torch.int32)[0]) & 1, "attend: no wait expired"
+    O1, l1 = gpu_prefill(w, d["Q"], d["K"], d["V"], i1, s1, n1)
+    O_ref, lse_ref = oracle.attend(inp["Q"], inp["K"], inp["V"], host(i1), host(s1), host(n1), 64, w.W, w.scale)
+    assert_close(O1, O_ref, w.dtype, "O after the diagnostic call")
+    assert_close(l1, lse_ref, torch.float32, "lse after the diagnostic call")
+    assert (host(lse) == 99.0).all() and (host(O).float() == 99.0).all(), "the diagnostic attend wrote outputs"
+
+
 def _decode_small(cuda_device, lens=(5000, 3001), K=16, W=512, H=3):
     w = WORKLOADS[4].replace(B=len(lens), H=H, N=max(lens), K=K, W=W, needles=0)
     inp = make_decode(w)
