@@ -1,7 +1,7 @@
 // One pipeline stage of the chunk screen (Eq. 7 of "Hierarchical Sparse Attention Done
 // Right" (picx.dev summary), with the rigorous radius of the exact selection): the
-// stage layout, the cooperative copies that fill it, and the screen of its rows on
-// tensor cores (bf16) or CUDA cores (float32), for the decode select's screen kernel.
+// stage layout, the cooperative copies that fill it, and the screen of its rows on CUDA
+// cores, for the decode select's screen kernel.
 #pragma once
 #include "select_pick.cuh"
 #include "tc_common.cuh"
@@ -49,93 +49,17 @@ __device__ __forceinline__ void transpose_reduce(float (&v)[N], int lane_in_grou
     v[0] += __shfl_xor_sync(kFull, v[0], 1);
 }
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};\n"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-
-// Tensor-core screen of one stage (bf16): warp w takes rows 16w..16w+15. The stage's rows
-// are ROWS x 128-byte column blocks (64 elements each) as TMA writes them with the
-// 128-byte swizzle: 16-byte unit u of row r sits in block u / 8 at r * 128 + ((u % 8) ^
-// (r % 8)) * 16. Per k-step one ldmatrix.x4 of the 16x16 row tile A and three m16n8k16
-// MMAs: A times q (q in column 0
-// of B), and A times its own rows 0-7 and 8-15 (Gram blocks whose diagonals are |k'|^2;
-// the B fragments of those are A's own registers). Radius: the tensor-core float32
-// accumulation order and rounding are not specified, so the bound allows d * 2^-16 of
-// scale |q| |k'| (about 2^7 times the round-to-nearest bound), plus 2^-22 |s| for the
-// final fused multiply-add; |k'|^2 itself carries a 2^-8 margin.
-// (s_c, e_c) of chunk c goes to out[c - base].
-template <int D, int ROWS>
-__device__ void screen_stage_mma(const uint8_t *st, int q_off, int bias_off, float scale, int c0, int ne,
-                                 float2 *out, int base, float2 *slots) {
-    constexpr int kKSteps = D / 16;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-    const int rbase = warp * 16;
-    const uint32_t *qw = reinterpret_cast<const uint32_t *>(st + q_off);
-    float qn2 = 0.f;
-    for (int pidx = lane; pidx < D / 2; pidx += 32) {
-        const uint32_t w = qw[pidx];
-        qn2 = fmaf(bf16lo(w), bf16lo(w), fmaf(bf16hi(w), bf16hi(w), qn2));
-    }
-    qn2 = warp_sum(qn2);
-    const int lrow = rbase + (lane & 7) + ((lane >> 3) & 1) * 8;
-    const uint32_t row_addr = (uint32_t)__cvta_generic_to_shared(st + lrow * 128);
-    float dacc[4] = {0.f, 0.f, 0.f, 0.f}, g1[4] = {0.f, 0.f, 0.f, 0.f}, g2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < kKSteps; ++ks) {
-        uint32_t a[4];
-        const int unit = ks * 2 + (lane >> 4);
-        ldmatrix_x4(a, row_addr + (uint32_t)((unit >> 3) * (ROWS * 128) + (((unit & 7) ^ (lrow & 7)) << 4)));
-        const uint32_t b0 = g == 0 ? qw[ks * 8 + tq] : 0u;
-        const uint32_t b1 = g == 0 ? qw[ks * 8 + 4 + tq] : 0u;
-        mma_bf16_16816(dacc, a, b0, b1);
-        mma_bf16_16816(g1, a, a[0], a[2]);
-        mma_bf16_16816(g2, a, a[1], a[3]);
-    }
-    // diagonal of the Gram blocks: row g in lane (g, g>>1), element (g & 1)
-    const float d1 = (g & 1) ? g1[1] : g1[0];
-    const float d2 = (g & 1) ? g2[3] : g2[2];
-    const int src = g * 4 + (g >> 1);
-    const float k1 = __shfl_sync(kFull, d1, src);
-    const float k2 = __shfl_sync(kFull, d2, src);
-    const float *bias = reinterpret_cast<const float *>(st + bias_off);
-    const float ecoef = scale * sqrt_approx(qn2) * ((float)D * 0x1p-16f) * (1.f + 0x1p-8f);
-    float ms = -INFINITY, me = 0.f;
-    if (tq == 0) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int row = rbase + g + 8 * h;
-            const int c = c0 + row;
-            const float dot = h ? dacc[2] : dacc[0];
-            const float sv = fmaf(dot, scale, bias[row]);
-            const float ev = fmaf(ecoef, sqrt_approx(h ? k2 : k1), fabsf(sv) * 0x1p-22f);
-            if (c < ne) {
-                out[c - base] = make_float2(sv, ev);
-                ms = fmaxf(ms, sv);
-                me = fmaxf(me, ev);
-            }
-        }
-    }
-    ms = warp_max(ms);
-    me = warp_max(me);
-    if (lane == 0) slots[warp] = make_float2(ms, me);
-}
-
-// Float32 screen of one stage on CUDA cores (all threads): kTPR threads share a row
-// (one 16-byte unit each), each accumulates its unit's partial dot and |k|^2 for kRPT
-// rows with packed float32 FMAs, and a transpose reduction across the kTPR lanes
-// leaves each lane the totals of one row.
+// Screen of one stage on CUDA cores (all threads), float32 arithmetic for either input
+// type: kTPR threads share a row (one 16-byte unit each), each accumulates its unit's
+// partial dot and |k|^2 for kRPT rows with packed float32 FMAs, and a transpose
+// reduction across the kTPR lanes leaves each lane the totals of one row. Radius: any
+// order of the float32 sums stays within (d+1) 2^-24 sum|q k| <= (d+1) 2^-24 |q~| |k'|
+// (Cauchy-Schwarz), doubled, plus 2^-22 |s| for the final fused multiply-add:
+//   e_c = scale |q~| |k'_c| (d+2) 2^-23 + |s_c| 2^-22.
+// bf16 rows sit as TMA wrote them with the 128-byte swizzle (16-byte unit u of row r in
+// column block u / 8 at r * 128 + ((u % 8) ^ (r % 8)) * 16), float32 rows plainly.
 template <typename T, int D, typename Cfg>
-__device__ void screen_stage_f32(const uint8_t *st, float scale, int c0, int ne, float2 *out, int base,
+__device__ void screen_stage_fma(const uint8_t *st, float scale, int c0, int ne, float2 *out, int base,
                                  float2 *gscr) {
     constexpr int kN = Vec<T>::kN;
     const int tid = threadIdx.x, col = tid % Cfg::kTPR, rg = tid / Cfg::kTPR;
@@ -153,7 +77,10 @@ __device__ void screen_stage_f32(const uint8_t *st, float scale, int c0, int ne,
     float dotv[Cfg::kRPT], ksqv[Cfg::kRPT];
 #pragma unroll
     for (int r = 0; r < Cfg::kRPT; ++r) {
-        const uint4 kv = *reinterpret_cast<const uint4 *>(st + (rg * Cfg::kRPT + r) * Cfg::kRowBytes + col * 16);
+        const int row = rg * Cfg::kRPT + r;
+        const uint8_t *unit = Cfg::kTma ? st + (col >> 3) * (Cfg::kRows * 128) + row * 128 + (((col & 7) ^ (row & 7)) << 4)
+                                        : st + row * Cfg::kRowBytes + col * 16;
+        const uint4 kv = *reinterpret_cast<const uint4 *>(unit);
         float2 d2 = make_float2(0.f, 0.f), k2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int p = 0; p < kN / 2; ++p) {
@@ -183,9 +110,9 @@ __device__ void screen_stage_f32(const uint8_t *st, float scale, int c0, int ne,
 }
 
 // Layout of one pipeline stage of ROWS summary rows screened by NT threads: the rows
-// (bf16: 128-byte column blocks written by TMA, see screen_stage_mma; float32: plain
-// rows), their biases, the query row and the query's position. bf16 stages start on
-// 1024-byte boundaries (the swizzle's period).
+// (bf16: 128-byte column blocks written by TMA with the 128-byte swizzle, see
+// screen_stage_fma; float32: plain rows), their biases, the query row and the query's
+// position. bf16 stages start on 1024-byte boundaries (the swizzle's period).
 template <typename T, int D, int NT, int ROWS>
 struct StageCfg {
     static constexpr int kThreads = NT;
@@ -201,11 +128,10 @@ struct StageCfg {
     static constexpr int kGroupsPerBlock = ROWS / kGroupRows;
     static constexpr int kCopies = ROWS * kTPR / NT;  // 16-byte copies per thread
     static_assert(2 * kRPT == kTPR, "half-square transpose reduction");
-    // bf16 tables are screened on tensor cores (16 rows per warp, swizzled shared rows);
-    // float32 tables on CUDA cores (kRPT rows per thread group).
-    static constexpr bool kMma = sizeof(T) == 2;
-    static_assert(!kMma || ROWS == 16 * (NT / 32), "tensor-core screen: 16 rows per warp");
-    static constexpr int kSlotRows = kMma ? 16 : kRPT;
+    // bf16 rows come by TMA (swizzled), float32 rows by cp.async; both are screened on
+    // CUDA cores, kRPT rows per group of kTPR threads
+    static constexpr bool kTma = sizeof(T) == 2;
+    static constexpr int kSlotRows = kRPT;
     static constexpr int kSlots = ROWS / kSlotRows;
     static constexpr int kSlotsPerGroup = kGroupRows / kSlotRows;
 };
@@ -219,7 +145,7 @@ __device__ __forceinline__ void stage_issue(uint8_t *st, const T *kh, int64_t ks
                                             const T *qrow, const int32_t *pos, int pos_value) {
     const int tid = threadIdx.x, col = tid % Cfg::kTPR;
     const int r0 = tid / Cfg::kTPR;
-    if constexpr (!Cfg::kMma) {
+    if constexpr (!Cfg::kTma) {
         const uint8_t *src = reinterpret_cast<const uint8_t *>(kh + (int64_t)(c0 + r0) * kst) + col * 16;
         uint8_t *dst = st + r0 * Cfg::kRowBytes + col * 16;
         constexpr int kStep = Cfg::kThreads / Cfg::kTPR;

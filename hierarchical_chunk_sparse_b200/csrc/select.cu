@@ -75,24 +75,23 @@ __global__ void __launch_bounds__(kWarpKernelThreads) select_warp_kernel(SelectA
 // 64-column block, completing on the stage's mbarrier; float32: cp.async), their
 // biases, the query row and the query's position (cp.async), so no load waits on
 // another. Every mbarrier wait is bounded: on expiry the CTA sets the select's status
-// word, stops, and lets its copies in flight land before it exits. bf16 rows are
-// screened on the tensor cores (mma.sync, 16 rows per warp; |k'|^2 from the Gram
-// diagonal), float32 rows on CUDA cores (kTPR threads per row, packed FMAs, a
-// transpose reduction). Written to the workspace: the screen value s_c and radius e_c
-// of every eligible chunk and the largest s and e of every 64-chunk group. For grouped
+// word, stops, and lets its copies in flight land before it exits. Rows of either type
+// are screened on CUDA cores (kTPR threads per row, packed float32 FMAs, a transpose
+// reduction; |k'|^2 from the same loads). Written to the workspace: the screen value s_c
+// and radius e_c of every eligible chunk and the largest s and e of every 64-chunk
+// group. For grouped
 // heads an item is a (b, group, query) and its block of the G heads' tables, screened
 // head after head by the same CTA; each head's interval s_c +- e_c is folded into the
 // group's [max lo, max hi] in shared memory, and the group's centre and radius are
 // written once, so the pick reads one row per group as for one head.
-//   CUDA cores:    e_c = scale |q~| |k'_c| (d+2) 2^-23 + |s_c| 2^-22 (Cauchy-Schwarz form
-//                  of the fused-multiply-add bound, doubled);
-//   tensor cores:  e_c = scale |q~| |k'_c| d 2^-16 (1 + 2^-8) + |s_c| 2^-22.
+//   e_c = scale |q~| |k'_c| (d+2) 2^-23 + |s_c| 2^-22 (Cauchy-Schwarz form of the
+//   fused-multiply-add bound, doubled).
 // select_pick_kernel (one 256-thread CTA per query, dependent launch): T = the (K+1)-th
 // largest group maximum is attained by K+1 distinct chunks, so the K-th largest lo is
 // at least T - e_max and every chunk with hi < T - e_max is certainly out. Only the
 // groups whose max s + max e reaches that cut are read again; their candidates
-// (typically K + a few) are screened again on CUDA cores with the tight radius and go
-// through the exact interval top-K in one warp; for grouped heads (one CTA per (b,
+// (typically K + a few) go through the exact interval top-K in one warp with their
+// screen values and radii; for grouped heads (one CTA per (b,
 // group, query)) every candidate gets each head's float64 score instead, one thread per
 // (head, candidate), and a parallel rank of the group maxima keeps the top K. With fewer
 // than K+1 groups the exact running-list scan runs over every chunk instead. Heavy ties
@@ -111,7 +110,7 @@ struct ScrCfg : StageCfg<T, D, kScrThreads, kScrRows> {
     static constexpr int kStages = Base::kStageBytes > 40000 ? 2 : kDecStages;
     static constexpr int kGscrOff = kStages * Base::kStageBytes;
     static constexpr int kFoldOff = kGscrOff + kScrRows * 8;  // grouped heads: one head's (s, e), the group's (lo, hi)
-    static constexpr int kSmemBytes = kFoldOff + 2 * kScrRows * 8 + (Base::kMma ? 1024 : 0);  // + alignment slack
+    static constexpr int kSmemBytes = kFoldOff + 2 * kScrRows * 8 + (Base::kTma ? 1024 : 0);  // + alignment slack
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 // One CTA per query (per (b, group, query) for grouped heads), dependent-launched after
@@ -130,7 +129,7 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid
     using Cfg = ScrCfg<T, D>;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // bf16 stages: 1024-byte alignment by pointer arithmetic on the shared array
-    uint8_t *smem = Cfg::kMma ? smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u) : smem_raw;
+    uint8_t *smem = Cfg::kTma ? smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u) : smem_raw;
     __shared__ unsigned long long sbar[kDecStages];
     __shared__ uint32_t sabort;
     float2 *gscr = reinterpret_cast<float2 *>(smem + Cfg::kGscrOff);
@@ -138,7 +137,7 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid
     const int tid = threadIdx.x;
     if (tid == 0) {
         sabort = 0u;
-        if (Cfg::kMma) {
+        if (Cfg::kTma) {
             for (int k = 0; k < Cfg::kStages; ++k) tc::mbar_init(tc::smem_u32(&sbar[k]), 1);
             asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
         }
@@ -172,7 +171,7 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid
             stage_issue<T, Cfg>(smem + stage * Cfg::kStageBytes, kh, a.Ksum.st, c0, min(kScrRows, a.C - c0),
                                 a.Bsum + ((int64_t)b * a.H + h) * a.C + c0, qrow,
                                 a.qpos ? a.qpos + (int64_t)b * a.Lq + i : nullptr, i);
-            if (Cfg::kMma && tid == 0) {  // the rows: (D / 64) boxes of 128 rows x 64 columns
+            if (Cfg::kTma && tid == 0) {  // the rows: (D / 64) boxes of 128 rows x 64 columns
                 const uint32_t bar = tc::smem_u32(&sbar[stage]);
                 const uint32_t dst = tc::smem_u32(smem + stage * Cfg::kStageBytes);
                 ++tma_issued[stage];
@@ -190,7 +189,7 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid
         const int item = item_of_seq(sq), hh = sq % gh;
         issue(sq + Cfg::kStages - 1, (stage + Cfg::kStages - 1) % Cfg::kStages);
         cp_async_wait<Cfg::kStages - 1>();
-        if (Cfg::kMma) {  // the stage's rows: use sq / kStages of its barrier
+        if (Cfg::kTma) {  // the stage's rows: use sq / kStages of its barrier
             const uint32_t bar = tc::smem_u32(&sbar[stage]), par = (uint32_t)(sq / Cfg::kStages) & 1u;
             bool ok = tc::mbar_try_wait(bar, par);
             const uint64_t t0 = global_ns();
@@ -204,7 +203,7 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid
             }
         }
         __syncthreads();
-        if (Cfg::kMma && sabort) break;  // uniform: read after the barrier
+        if (Cfg::kTma && sabort) break;  // uniform: read after the barrier
         const uint8_t *st = smem + stage * Cfg::kStageBytes;
         const int qu = item / nblk, blk = item - (item / nblk) * nblk;
         const int c0 = blk * kScrRows;
@@ -212,8 +211,7 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid
         float2 *out = kFold ? tmp : ws.scr + (int64_t)qu * a.C;
         const int base = kFold ? c0 : 0;
         if (c0 < ne) {
-            if (Cfg::kMma) screen_stage_mma<D, kScrRows>(st, Cfg::kQOff, Cfg::kBiasOff, a.scale, c0, ne, out, base, gscr);
-            else screen_stage_f32<T, D, Cfg>(st, a.scale, c0, ne, out, base, gscr);
+            screen_stage_fma<T, D, Cfg>(st, a.scale, c0, ne, out, base, gscr);
         }
         __syncthreads();
         if (kFold && c0 < ne) {
@@ -263,7 +261,7 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid
         stage = (stage + 1) % Cfg::kStages;
     }
     cp_async_wait<0>();
-    if (Cfg::kMma && tid == 0) {
+    if (Cfg::kTma && tid == 0) {
         // after an abort: every row load started lands before the CTA releases its memory
         // (each was issued after the previous use of its stage had completed)
         for (int k = 0; k < Cfg::kStages; ++k) {
@@ -289,7 +287,7 @@ hils_status launch_screen(const SelectArgs &a, cudaStream_t s) {
     const int64_t slots = (int64_t)per_sm * device_sm_count();
     const int64_t grid = items < slots ? items : slots;
     CUtensorMap mk{};  // bf16 rows come by TMA; float32 rows do not use the map
-    if (Cfg::kMma && !tc::make_map(&mk, View{a.Ksum.ptr, a.Ksum.sb, a.Ksum.sh, a.Ksum.st}, a.B, a.H, a.C, kScrRows, D))
+    if (Cfg::kTma && !tc::make_map(&mk, View{a.Ksum.ptr, a.Ksum.sb, a.Ksum.sh, a.Ksum.st}, a.B, a.H, a.C, kScrRows, D))
         return HILS_ERR_CUDA;
     if (a.G > 1) select_screen_kernel<T, D, true><<<(unsigned)grid, kScrThreads, Cfg::kSmemBytes, s>>>(mk, a);
     else select_screen_kernel<T, D, false><<<(unsigned)grid, kScrThreads, Cfg::kSmemBytes, s>>>(mk, a);

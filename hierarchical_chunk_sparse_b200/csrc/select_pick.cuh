@@ -50,56 +50,6 @@ __device__ void block_kth_plus_one(const unsigned *key, int n, int K, float *out
     }
 }
 
-// The float32 screen value and tight radius of chunk c for one query head, four
-// threads per chunk (a quarter of the row each, then two shuffle steps; every lane of
-// the warp takes part, lanes with ok = false contribute zero). Any order of the float32
-// sums stays within the radius scale sum|q k| (d+2) 2^-23 + |s| 2^-22.
-template <typename T, int D>
-__device__ __forceinline__ void rescreen_one(const QueryCtx &q, const float *qs, int c, bool ok, float &s,
-                                             float &e) {
-    constexpr int kN = Vec<T>::kN, kQuarter = D / 4;
-    const int sub = threadIdx.x & 3;
-    const float bias = ok ? __ldg(q.bhead + c) : 0.f;
-    float dot = 0.f, ad = 0.f;
-    if (ok) {
-        const uint4 *kr = reinterpret_cast<const uint4 *>(static_cast<const T *>(q.khead) + (int64_t)c * q.kst +
-                                                          sub * kQuarter);
-#pragma unroll
-        for (int u = 0; u < kQuarter / kN; ++u) {
-            float kf[kN];
-            widen(__ldg(kr + u), kf, T());
-#pragma unroll
-            for (int i = 0; i < kN; ++i) {
-                const float qv = qs[sub * kQuarter + u * kN + i];
-                dot = fmaf(qv, kf[i], dot);
-                ad = fmaf(fabsf(qv), fabsf(kf[i]), ad);
-            }
-        }
-    }
-    dot += __shfl_xor_sync(kFull, dot, 1);
-    ad += __shfl_xor_sync(kFull, ad, 1);
-    dot += __shfl_xor_sync(kFull, dot, 2);
-    ad += __shfl_xor_sync(kFull, ad, 2);
-    s = ok ? fmaf(dot, q.scale, bias) : 0.f;
-    e = fmaf(q.scale * ad, (float)(D + 2) * 0x1p-23f, fabsf(s) * 0x1p-22f);
-}
-
-// Every pool entry screened again on CUDA cores with the tight radius.
-template <typename T, int D, int NT>
-__device__ void rescreen_pool(const QueryCtx &q, const float *qs, Pool64 &pool, int total) {
-    const int tid = threadIdx.x;
-    for (int base = 0; base < total; base += NT / 4) {  // the same trip count in every lane
-        const int j = base + (tid >> 2);
-        const bool ok = j < total;
-        float s, e;
-        rescreen_one<T, D>(q, qs, ok ? pool.idx[j] : 0, ok, s, e);
-        if (ok && (tid & 3) == 0) {
-            pool.s[j] = s;
-            pool.e[j] = e;
-        }
-    }
-}
-
 // The float64 score of chunk c for one query head, the same fixed-order chain as
 // exact_score (each product of the float64 values, summed in x order, then times scale
 // plus b'_c), with the query's elements from shared memory (float32 copies that hold
@@ -282,10 +232,8 @@ __device__ void pick_unit(const SelectArgs &a, const ScreenWs &ws, int64_t u, Pi
     const int total = ps.pool_n;
     if constexpr (!kGroup) {
       if (total <= kPoolCap) {
-        // the candidates are screened again on CUDA cores (round-to-nearest fused
-        // multiply-adds: the tight radius), so that few need the float64 score
-        rescreen_pool<T, D, NT>(q, ps.qs, ps.pool, total);
-        __syncthreads();
+        // the candidates' screen values carry the fused-multiply-add radius already, so
+        // few need the float64 score
         if (w == 0) {
             Slots<2> sl;
 #pragma unroll

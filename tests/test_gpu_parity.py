@@ -677,10 +677,11 @@ def test_decode_workload_full_size(oracle, cuda_device, cfg):
 def test_screen_radius_covers_the_float64_score(oracle, cuda_device, d):
     """The decode-shaped select writes every eligible chunk's float32 screen value s_c and
     radius e_c to its workspace (B*H*Lq*C float pairs after the 256-byte status header,
-    which must stay zero). The kept set is only
-    exact if |s_c - x_c| <= e_c, with x_c the oracle's float64 score: check it for every
-    chunk, and check that the observed error stays far (1/16) inside the tensor-core
-    part of the bound, scale |q| |k'| d 2^-16, so the bound is not merely lucky."""
+    which must stay zero). The kept set is only exact if |s_c - x_c| <= e_c, with x_c the
+    oracle's float64 score: check it for every chunk; check that the radius is the
+    fused-multiply-add bound scale |q| |k'| (d+2) 2^-23 + |s| 2^-22 (within its own float32
+    rounding), and that the observed error stays well inside it (1/4), so the bound is
+    not merely lucky."""
     w = WORKLOADS[4].replace(B=2, H=4, d=d, K=16)
     C = 5000
     g = torch.Generator().manual_seed(31)
@@ -705,8 +706,9 @@ def test_screen_radius_covers_the_float64_score(oracle, cuda_device, d):
     assert (err <= scr[..., 1]).all(), f"radius violated: {float((err - scr[..., 1]).max()):.3e}"
     qn = np.linalg.norm(Q.double().numpy(), axis=-1)            # [B,H,1]
     kn = np.linalg.norm(Ksum.double().numpy(), axis=-1)         # [B,H,C]
-    tc = w.scale * qn * kn * d * 2.0 ** -16 + np.abs(x) * 2.0 ** -22
-    assert (err / tc).max() <= 1 / 16, f"observed error {float((err / tc).max()):.3f} of the bound"
+    fma = w.scale * qn * kn * (d + 2) * 2.0 ** -23 + np.abs(x) * 2.0 ** -22
+    assert np.allclose(scr[..., 1], fma, rtol=1e-5, atol=0), "radius is not the fused-multiply-add bound"
+    assert (err / scr[..., 1]).max() <= 1 / 4, f"observed error {float((err / scr[..., 1]).max()):.3f} of the bound"
     i_ref, s_ref, n_ref = oracle.select(Q, Ksum, Bsum, 64, w.K, w.scale, qpos=qpos)
     assert_same_selection(idx, nsel, i_ref, n_ref)
 
