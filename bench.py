@@ -392,14 +392,19 @@ CSRC = os.path.join(ROOT, "hierarchical_chunk_sparse_b200", "csrc")
 KERNEL_SOURCES = {
     "decode_select": ["select.cu", "screen_stage.cuh", "select_pick.cuh", "select_common.cuh", "tc_common.cuh",
                       "hils_internal.cuh"],
-    "decode_attend": ["attend.cu", "hils_internal.cuh"],
-    "attend_prefill": ["attend_prefill_tc.cu", "tc_common.cuh", "hils_internal.cuh"],
-    "summarize": ["summarize.cu", "hils_internal.cuh"],
+    "decode_attend": ["attend.cu", "attend_common.cuh", "hils_internal.cuh"],
+    "attend_prefill": ["attend_prefill_tc.cu", "tc_common.cuh", "fast_math.cuh", "hils_internal.cuh"],
+    "summarize": ["summarize.cu", "tc_common.cuh", "hils_internal.cuh"],
 }
 # kernel -> (DRAM bytes per unit, source digest at capture). Units: decode_select and
 # decode_attend per algorithmic byte of the launch (the captured traffic / algorithmic
 # bytes), summarize per chunk, attend_prefill per launch of the 8K prefill workload.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    'decode_select': (1.0156747581565824, '8d557f9cb7a44ff0'),
+    'decode_attend': (1.001956609018697, '4b092b3b75bf0e3a'),
+    'summarize': (16922.4921875, '453a85260e417f60'),
+    'attend_prefill': (659396864, '53ec368d0a713d57'),
+}
 
 
 def source_digest(kernel: str) -> str:
