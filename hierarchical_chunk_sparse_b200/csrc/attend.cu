@@ -162,6 +162,7 @@ __global__ void __launch_bounds__(kThreads) attend_decode_kernel(AttendArgs a) {
     // the caller guarantees that the preceding grid is this library's select, which
     // itself started after all earlier work on the stream (hils_decode).
     if (chunk_unit || !a.window_early) pdl_wait();
+    pdl_trigger();  // a dependent-launched successor may be scheduled; it waits for this grid
     // the unit's small inputs, loaded together before anything depends on them
     const int clen = a.cache_len[b];
     const int ns = chunk_unit ? a.nsel[qg] : 0;
@@ -277,6 +278,7 @@ __global__ void __launch_bounds__(kThreads) attend_decode_group_kernel(AttendArg
     const int64_t qi0 = (int64_t)b * a.H + h0;  // the group's first query head
     const bool chunk_unit = u < a.topk;
     if (chunk_unit || !a.window_early) pdl_wait();  // as in the per-head kernel
+    pdl_trigger();
     const int clen = a.cache_len[b];
     const int ns = chunk_unit ? a.nsel[qg] : 0;
     const int cidx = chunk_unit ? a.idx[qg * a.topk + u] : -1;

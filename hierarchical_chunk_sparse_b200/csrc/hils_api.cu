@@ -492,9 +492,9 @@ int hils_decode(const hils_params *p, hils_ctensor Qcal, hils_ctensor Ksum, cons
     HILS_TRY(check_workspace(workspace, ws_bytes, sel_bytes + attend_decode_ws_bytes((int)nq, aa.units, p->d)));
     sa.ws = workspace;
     aa.ws = static_cast<uint8_t *>(workspace) + sel_bytes;
-    // the select's first kernel is an ordinary launch, so every earlier write on the
-    // stream is complete before it starts; the attend follows the select's last kernel,
-    // so its window tiles need not wait for the select
+    // the select's first kernel waits for every earlier write on the stream before it
+    // reads anything, and each later kernel of the chain is scheduled only after the one
+    // before it passed that point: the attend's window tiles need not wait for the select
     aa.window_early = 1;
     HILS_TRY(launch_select(p->dtype, p->d, sa, stream));
     return launch_attend_decode(p->dtype, p->d, aa, stream);

@@ -133,6 +133,10 @@ __global__ void __launch_bounds__(kScrThreads) select_screen_kernel(const __grid
     __shared__ unsigned long long sbar[kDecStages];
     __shared__ uint32_t sabort;
     float2 *gscr = reinterpret_cast<float2 *>(smem + Cfg::kGscrOff);
+    // dependent launch: this grid may be scheduled while the preceding kernel drains, so
+    // it waits for that kernel (and its memory) before touching anything; then it lets the
+    // pick be scheduled
+    pdl_wait();
     pdl_trigger();
     const int tid = threadIdx.x;
     if (tid == 0) {
@@ -289,9 +293,19 @@ hils_status launch_screen(const SelectArgs &a, cudaStream_t s) {
     CUtensorMap mk{};  // bf16 rows come by TMA; float32 rows do not use the map
     if (Cfg::kTma && !tc::make_map(&mk, View{a.Ksum.ptr, a.Ksum.sb, a.Ksum.sh, a.Ksum.st}, a.B, a.H, a.C, kScrRows, D))
         return HILS_ERR_CUDA;
-    if (a.G > 1) select_screen_kernel<T, D, true><<<(unsigned)grid, kScrThreads, Cfg::kSmemBytes, s>>>(mk, a);
-    else select_screen_kernel<T, D, false><<<(unsigned)grid, kScrThreads, Cfg::kSmemBytes, s>>>(mk, a);
-    return record_cuda_error(cudaGetLastError());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kScrThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    SelectArgs args = a;
+    void *argv[] = {&mk, &args};
+    return record_cuda_error(cudaLaunchKernelExC(&cfg, fn, argv));
 }
 
 template <typename T, int D>
