@@ -400,8 +400,8 @@ KERNEL_SOURCES = {
 # decode_attend per algorithmic byte of the launch (the captured traffic / algorithmic
 # bytes), summarize per chunk, attend_prefill per launch of the 8K prefill workload.
 MEASURED_TRAFFIC = {
-    'decode_select': (1.0156747581565824, '8d557f9cb7a44ff0'),
-    'decode_attend': (1.001956609018697, '4b092b3b75bf0e3a'),
+    'decode_select': (1.0172632638346453, '89390ce2ed3f933e'),
+    'decode_attend': (1.002088743653726, 'bf37b6a22e9eedbe'),
     'summarize': (16922.4921875, '453a85260e417f60'),
     'attend_prefill': (659396864, '53ec368d0a713d57'),
 }
@@ -597,7 +597,8 @@ def run_profile_case(args):
     summarize:     hils_summarize over a 1M-token cache of 4 heads (16384 chunks each, 1.1 GB of keys);
     prefill:       the full 8K prefill workload (summarise, select, attend);
     prefill-select: the select of the 8K prefill, multi-head then grouped-query (32 query
-                   heads, 8 key-value heads), `warmup + steps` launches each.
+                   heads, 8 key-value heads), `warmup + steps` launches each;
+    prefill-backward: the attend backward of the 8K prefill for the forward's selection.
     Runs `warmup + steps` plain launches of the case and exits."""
     import hierarchical_chunk_sparse_b200 as hils
 
@@ -633,6 +634,19 @@ def run_profile_case(args):
         fn = lambda: hils.hils_summarize(p, K, LQ, Ksum, Bsum)  # noqa
     elif case == "prefill":
         fn = PrefillBench(WORKLOADS[2], dev).step
+    elif case == "prefill-backward":
+        pb = PrefillBench(WORKLOADS[2], dev)
+        pb.step()
+        w = WORKLOADS[2]
+        f32 = dict(dtype=torch.float32, device=dev)
+        g = torch.Generator(device=dev).manual_seed(3)
+        dO = torch.randn(w.B, w.H, w.N, w.d, generator=g, **f32)
+        dQ, dscore = torch.empty(w.B, w.H, w.N, w.d, **f32), torch.empty(w.B, w.H, w.N, w.K, **f32)
+        dK, dV = torch.zeros(w.B, w.Hkv, w.N, w.d, **f32), torch.zeros(w.B, w.Hkv, w.N, w.d, **f32)
+        ws = hils.alloc_workspace(pb.p, hils.HILS_CALL_ATTEND_BACKWARD, w.N, 0, device=dev)
+        i = pb.inp
+        fn = lambda: hils.hils_attend_prefill_backward(pb.p, i["Q"], i["K"], i["V"], pb.idx, pb.score,  # noqa
+                                                       pb.nsel, pb.O, pb.lse, dO, dQ, dK, dV, dscore, workspace=ws)
     elif case == "prefill-select":
         benches = [PrefillBench(WORKLOADS[n], dev) for n in (2, 7)]
         for pb in benches:
@@ -904,7 +918,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None,
                     choices=["decode-select", "decode-select-gqa", "decode-attend", "decode-step", "prefill",
-                             "prefill-select", "summarize"],
+                             "prefill-select", "prefill-backward", "summarize"],
                     help="run a small case for an ncu capture and exit")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
