@@ -794,7 +794,7 @@ def measure_prefill_backward(w, dev, stream, flush, args, world):
     fl = backward_flops(w)
     out = {"ms_per_step": ms, "unit": "TFLOP/s", "value": fl / (ms * 1e-3) / 1e12 * world, "workload": w.name,
            "algorithmic_gflop_per_step": fl / 1e9, "steps": n, "ms_per_call": split,
-           "note": "key-major attend backward on the tensor cores (mma.sync bf16, dK and dV accumulated per key block), float32 atomics for dQ, dKsum and dBsum summed per CTA in shared memory first; ms_per_call times each call alone"}
+           "note": "key-major attend backward on tcgen05 (bf16, d = 128: 128 queries per step of a 64-key block, dK and dV accumulated in TMEM per work item, Q and dO rows by TMA row gathers), float32 atomics for dQ (vector) and dK, dV; dKsum and dBsum summed per CTA in shared memory first; ms_per_call times each call alone"}
     del pb
     torch.cuda.empty_cache()
     return out

@@ -25,7 +25,10 @@
 // an inverted index of the selection built first (count, scan, scatter). D_i = dO_i . o_i
 // is computed once per query beforehand. Score and summaries: one CTA per query or per
 // chunk. Shared gradients (dK, dV, dKsum, dBsum, dQ) are float32 atomic adds, in no fixed
-// order. Gradients are float32, dense.
+// order. Gradients are float32, dense. bf16 with d = 128 takes the tensor-core form of the
+// same walk (backward_tc.cu: 128 queries per step on tcgen05, chunk lists cut into runs
+// of at most 1024 queries); bf16 with d = 64 the mma.sync form below; float32 the
+// CUDA-core form.
 #include <math.h>
 
 #include "hils_internal.cuh"
@@ -35,19 +38,30 @@ namespace {
 
 constexpr int kThreads = 128;
 
-// Workspace of the attend backward: D_i per query, then per (b, group) the chunk counts,
-// starts (C + 1), cursors and the inverted index (N * K entries).
+// Workspace of the attend backward: a status word (256 bytes), D_i per query, then per
+// (b, group) the chunk counts, starts (C + 1), cursors and the inverted index (N * K
+// entries). The tensor-core walk (bf16, d = 128) adds: one record per (query head,
+// index entry), the chunk items per (b, group) and their count, and contiguous bf16
+// copies of dO and Q ([B*H*N][d] rows, the row gathers' source).
 struct BwdWs {
+    uint32_t *status;
     float *D;
     int *count, *start, *cursor, *entries;
+    int4 *recs, *items;
+    int *nitems;
+    bf16 *dOb, *Qc;
+    int max_items;
     size_t bytes;
 };
 inline size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
-inline BwdWs bwd_ws(void *ws, int B, int H, int Hk, int N, int K) {
+inline bool bwd_tc_layout(hils_dtype dt, int d) { return dt == HILS_BF16 && d == 128; }
+inline BwdWs bwd_ws(void *ws, bool tc, int B, int H, int Hk, int N, int K, int d) {
     const int C = N / kChunk;
     uint8_t *p = static_cast<uint8_t *>(ws);
-    BwdWs w;
+    BwdWs w = {};
     size_t off = 0;
+    w.status = reinterpret_cast<uint32_t *>(p + off);
+    off += 256;
     w.D = reinterpret_cast<float *>(p + off);
     off += a256((size_t)B * H * N * 4);
     w.count = reinterpret_cast<int *>(p + off);
@@ -58,6 +72,20 @@ inline BwdWs bwd_ws(void *ws, int B, int H, int Hk, int N, int K) {
     off += a256((size_t)B * Hk * C * 4);
     w.entries = reinterpret_cast<int *>(p + off);
     off += a256((size_t)B * Hk * N * (K > 0 ? K : 1) * 4);
+    if (tc) {
+        // chunk items: sum over chunks of ceil(count / kBwdItemQueries) <= C + N K / kBwdItemQueries
+        w.max_items = C + (int)(((int64_t)N * K + kBwdItemQueries - 1) / kBwdItemQueries);
+        w.recs = reinterpret_cast<int4 *>(p + off);
+        off += a256((size_t)B * H * N * K * 16);
+        w.items = reinterpret_cast<int4 *>(p + off);
+        off += a256((size_t)B * Hk * w.max_items * 16);
+        w.nitems = reinterpret_cast<int *>(p + off);
+        off += a256((size_t)B * Hk * 4);
+        w.dOb = reinterpret_cast<bf16 *>(p + off);
+        off += a256((size_t)B * H * N * d * 2);
+        w.Qc = reinterpret_cast<bf16 *>(p + off);
+        off += a256((size_t)B * H * N * d * 2);
+    }
     w.bytes = off;
     return w;
 }
@@ -97,6 +125,34 @@ __global__ void __launch_bounds__(kThreads) bwd_dot_kernel(BwdAttendArgs a, floa
     if (lane == 0) Dv[qi] = acc;
 }
 
+// The tensor-core walk's preparation (bf16, d = 128), one warp per query row: D_i, and
+// the row of dO rounded to bf16 and the row of Q, both into contiguous [B*H*N][128]
+// arrays (lane l holds elements 4l..4l+3).
+__global__ void __launch_bounds__(kThreads) bwd_prep_kernel(BwdAttendArgs a, float *Dv, bf16 *dOb, bf16 *Qc) {
+    const int64_t qi = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (qi >= (int64_t)a.B * a.H * a.N) return;
+    const int i = (int)(qi % a.N);
+    const int h = (int)((qi / a.N) % a.H);
+    const int b = (int)(qi / ((int64_t)a.N * a.H));
+    const bf16 *orow = static_cast<const bf16 *>(a.O.ptr) + b * a.O.sb + h * a.O.sh + (int64_t)i * a.O.st;
+    const bf16 *qrow = static_cast<const bf16 *>(a.Q.ptr) + b * a.Q.sb + h * a.Q.sh + (int64_t)i * a.Q.st;
+    const float *g = a.dO + qi * 128 + 4 * lane;
+    const float g0 = g[0], g1 = g[1], g2 = g[2], g3 = g[3];
+    const uint2 ov = *reinterpret_cast<const uint2 *>(orow + 4 * lane);
+    const uint2 qv = *reinterpret_cast<const uint2 *>(qrow + 4 * lane);
+    float acc = g0 * bf16lo(ov.x);
+    acc = fmaf(g1, bf16hi(ov.x), acc);
+    acc = fmaf(g2, bf16lo(ov.y), acc);
+    acc = fmaf(g3, bf16hi(ov.y), acc);
+    acc = warp_sum(acc);
+    if (lane == 0) Dv[qi] = acc;
+    const __nv_bfloat162 d01 = __floats2bfloat162_rn(g0, g1), d23 = __floats2bfloat162_rn(g2, g3);
+    *reinterpret_cast<uint2 *>(dOb + qi * 128 + 4 * lane) =
+        make_uint2(*reinterpret_cast<const uint32_t *>(&d01), *reinterpret_cast<const uint32_t *>(&d23));
+    *reinterpret_cast<uint2 *>(Qc + qi * 128 + 4 * lane) = qv;
+}
+
 // Inverted index of the selection per (b, group): count[c], then (after the scan)
 // cursor[c] = start[c] + filled so far; entries hold i * 32 + k.
 __global__ void bwd_count_kernel(BwdAttendArgs a, int *count) {
@@ -111,32 +167,56 @@ __global__ void bwd_count_kernel(BwdAttendArgs a, int *count) {
     if (c >= 0 && c < a.N / kChunk) atomicAdd(&count[bg * (a.N / kChunk) + c], 1);
 }
 
-// exclusive scan of count over the C chunks of one (b, group): start[c], cursor[c]
-__global__ void __launch_bounds__(1024) bwd_scan_kernel(int C, const int *count, int *start, int *cursor) {
+// exclusive scan of count over the C chunks of one (b, group): start[c], cursor[c]; with
+// `items`, also the group's chunk items: chunk c's entries cut into runs of at most
+// kBwdItemQueries, {c, first entry, end entry, 0}, in chunk order, and their number.
+__global__ void __launch_bounds__(1024) bwd_scan_kernel(int C, const int *count, int *start, int *cursor,
+                                                        int4 *items, int *nitems, int max_items) {
     __shared__ int part[1024];
     const int64_t bg = blockIdx.x;
     const int *cnt = count + bg * C;
     const int per = (C + 1023) / 1024, t = threadIdx.x;
+    const int c_lo = min(C, t * per), c_hi = min(C, (t + 1) * per);
+    // inclusive scan of one value per thread, in place in part[]
+    auto block_scan = [&](int v) {
+        part[t] = v;
+        __syncthreads();
+        for (int o = 1; o < 1024; o <<= 1) {
+            const int u = t >= o ? part[t - o] : 0;
+            __syncthreads();
+            part[t] += u;
+            __syncthreads();
+        }
+    };
     int sum = 0;
-    for (int c = t * per; c < min(C, (t + 1) * per); ++c) sum += cnt[c];
-    part[t] = sum;
-    __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {  // inclusive scan of the per-thread sums
-        const int v = t >= o ? part[t - o] : 0;
-        __syncthreads();
-        part[t] += v;
-        __syncthreads();
-    }
+    for (int c = c_lo; c < c_hi; ++c) sum += cnt[c];
+    block_scan(sum);
     int run = part[t] - sum;
-    for (int c = t * per; c < min(C, (t + 1) * per); ++c) {
+    for (int c = c_lo; c < c_hi; ++c) {
         start[bg * (C + 1) + c] = run;
         cursor[bg * C + c] = run;
         run += cnt[c];
     }
     if (t == 1023) start[bg * (C + 1) + C] = part[1023];
+    if (!items) return;
+    int segs = 0;
+    for (int c = c_lo; c < c_hi; ++c) segs += (cnt[c] + kBwdItemQueries - 1) / kBwdItemQueries;
+    run = part[t] - sum;  // this thread's first entry
+    __syncthreads();
+    block_scan(segs);
+    int o = part[t] - segs;
+    int4 *it = items + bg * max_items;
+    for (int c = c_lo; c < c_hi; ++c) {
+        const int n = cnt[c];
+        for (int e = 0; e < n; e += kBwdItemQueries) it[o++] = make_int4(c, run + e, run + min(n, e + kBwdItemQueries), 0);
+        run += n;
+    }
+    if (t == 1023) nitems[bg] = part[1023];
 }
 
-__global__ void bwd_scatter_kernel(BwdAttendArgs a, int *cursor, int *entries) {
+// Fills the inverted index; with `recs`, also each query head's record of the entry:
+// {i * 32 + k (or -1 when the row's lse is not finite), w = exp(s^_{i,c} - lse_i), D_i, i}.
+__global__ void bwd_scatter_kernel(BwdAttendArgs a, int *cursor, int *entries, const float *Dv, int4 *recs) {
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int Hk = a.H / a.G, K = a.topk, C = a.N / kChunk;
     if (e >= (int64_t)a.B * Hk * a.N * K) return;
@@ -149,6 +229,16 @@ __global__ void bwd_scatter_kernel(BwdAttendArgs a, int *cursor, int *entries) {
     const int i = (int)(qg % a.N);
     const int pos = atomicAdd(&cursor[bg * C + c], 1);
     entries[bg * (int64_t)a.N * K + pos] = i * 32 + k;
+    if (!recs) return;
+    const int b = (int)(bg / Hk), g = (int)(bg % Hk);
+    for (int hh = 0; hh < a.G; ++hh) {
+        const int64_t bh = (int64_t)b * a.H + g * a.G + hh;
+        const int64_t qh = bh * a.N + i;
+        const float lse = a.lse[qh];
+        const bool fin = isfinite(lse);
+        const float w = fin ? expf(a.score[qh * K + k] - lse) : 0.f;
+        recs[bh * a.N * K + pos] = make_int4(fin ? i * 32 + k : -1, __float_as_int(w), __float_as_int(Dv[qh]), i);
+    }
 }
 
 constexpr int kQT = 16;  // queries per step of the key-major kernel
@@ -785,45 +875,78 @@ template <typename T, int D>
 hils_status launch_attend_bwd(const BwdAttendArgs &a, void *ws, cudaStream_t s) {
     const int64_t nq = (int64_t)a.B * a.H * a.N;
     const int Hk = a.H / a.G, C = a.N / kChunk;
-    const BwdWs w = bwd_ws(ws, a.B, a.H, Hk, a.N, a.topk);
-    hils_status st = record_cuda_error(cudaMemsetAsync(a.dQ, 0, (size_t)nq * D * sizeof(float), s));
+    constexpr bool kTc = sizeof(T) == 2 && D == 128;
+    const BwdWs w = bwd_ws(ws, kTc, a.B, a.H, Hk, a.N, a.topk, D);
+    hils_status st = record_cuda_error(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), s));
+    if (st != HILS_OK) return st;
+    st = record_cuda_error(cudaMemsetAsync(a.dQ, 0, (size_t)nq * D * sizeof(float), s));
     if (st != HILS_OK) return st;
     if (a.topk > 0) {  // dscore padding stays 0
         st = record_cuda_error(cudaMemsetAsync(a.dscore, 0, (size_t)nq * a.topk * sizeof(float), s));
         if (st != HILS_OK) return st;
     }
-    bwd_dot_kernel<T, D><<<(unsigned)((nq + 3) / 4), kThreads, 0, s>>>(a, w.D);
-    // bf16: the tensor-core walk; float32: the CUDA-core walk (full float32 products)
-    constexpr bool kMma = sizeof(T) == 2;
-    constexpr int smem = kMma ? MmaCfg<D>::kSmemBytes : KmCfg<T, D>::kSmemBytes;
-    const void *fw = kMma ? (const void *)attend_bwd_mma_kernel<D, false>
-                          : (const void *)attend_bwd_keymajor_kernel<T, D, false>;
-    const void *fc = kMma ? (const void *)attend_bwd_mma_kernel<D, true>
-                          : (const void *)attend_bwd_keymajor_kernel<T, D, true>;
-    static KernelSetup setup_w, setup_c;
-    st = kernel_setup(setup_w, fw, kThreads, smem, nullptr);
-    if (st != HILS_OK) return st;
-    st = kernel_setup(setup_c, fc, kThreads, smem, nullptr);
-    if (st != HILS_OK) return st;
-    if (a.topk > 0 && C > 0) {
-        const int64_t ne = (int64_t)a.B * Hk * a.N * a.topk;
-        st = record_cuda_error(cudaMemsetAsync(w.count, 0, (size_t)a.B * Hk * C * sizeof(int), s));
+    if constexpr (kTc) {
+        // tensor-core walk: D_i and the contiguous bf16 rows, the inverted index with its
+        // per-head records and chunk items, then one launch over all work items
+        bwd_prep_kernel<<<(unsigned)((nq + 3) / 4), kThreads, 0, s>>>(a, w.D, w.dOb, w.Qc);
+        const bool chunks = a.topk > 0 && C > 0;
+        if (chunks) {
+            const int64_t ne = (int64_t)a.B * Hk * a.N * a.topk;
+            st = record_cuda_error(cudaMemsetAsync(w.count, 0, (size_t)a.B * Hk * C * sizeof(int), s));
+            if (st != HILS_OK) return st;
+            bwd_count_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.count);
+            bwd_scan_kernel<<<(unsigned)(a.B * Hk), 1024, 0, s>>>(C, w.count, w.start, w.cursor, w.items, w.nitems,
+                                                                 w.max_items);
+            bwd_scatter_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.cursor, w.entries, w.D, w.recs);
+        }
+        BwdTcArgs t;
+        t.a = a;
+        t.Dv = w.D;
+        t.recs = w.recs;
+        t.items = w.items;
+        t.nitems = w.nitems;
+        t.max_items = chunks ? w.max_items : 0;
+        t.nsegw = a.W > 0 ? (kChunk - 1 + a.W + kBwdItemQueries - 1) / kBwdItemQueries : 0;
+        t.nwin = a.W > 0 ? ((a.N + kChunk - 1) / kChunk) * t.nsegw : 0;
+        t.vec_ok = ((uintptr_t)a.dQ & 15u) == 0;
+        t.status = w.status;
+        st = record_cuda_error(cudaGetLastError());
         if (st != HILS_OK) return st;
-        bwd_count_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.count);
-        bwd_scan_kernel<<<(unsigned)(a.B * Hk), 1024, 0, s>>>(C, w.count, w.start, w.cursor);
-        bwd_scatter_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.cursor, w.entries);
-        if constexpr (kMma)
-            attend_bwd_mma_kernel<D, true><<<dim3(C, a.B * a.H), kThreads, smem, s>>>(a, w.D, w.start, w.entries);
-        else
-            attend_bwd_keymajor_kernel<T, D, true><<<dim3(C, a.B * a.H), kThreads, smem, s>>>(a, w.D, w.start,
-                                                                                                w.entries);
+        return launch_attend_bwd_tc(t, w.Qc, w.dOb, s);
+    } else {
+        bwd_dot_kernel<T, D><<<(unsigned)((nq + 3) / 4), kThreads, 0, s>>>(a, w.D);
+        // bf16, d = 64: the mma.sync walk; float32: the CUDA-core walk (full float32 products)
+        constexpr bool kMma = sizeof(T) == 2;
+        constexpr int smem = kMma ? MmaCfg<D>::kSmemBytes : KmCfg<T, D>::kSmemBytes;
+        const void *fw = kMma ? (const void *)attend_bwd_mma_kernel<D, false>
+                              : (const void *)attend_bwd_keymajor_kernel<T, D, false>;
+        const void *fc = kMma ? (const void *)attend_bwd_mma_kernel<D, true>
+                              : (const void *)attend_bwd_keymajor_kernel<T, D, true>;
+        static KernelSetup setup_w, setup_c;
+        st = kernel_setup(setup_w, fw, kThreads, smem, nullptr);
+        if (st != HILS_OK) return st;
+        st = kernel_setup(setup_c, fc, kThreads, smem, nullptr);
+        if (st != HILS_OK) return st;
+        if (a.topk > 0 && C > 0) {
+            const int64_t ne = (int64_t)a.B * Hk * a.N * a.topk;
+            st = record_cuda_error(cudaMemsetAsync(w.count, 0, (size_t)a.B * Hk * C * sizeof(int), s));
+            if (st != HILS_OK) return st;
+            bwd_count_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.count);
+            bwd_scan_kernel<<<(unsigned)(a.B * Hk), 1024, 0, s>>>(C, w.count, w.start, w.cursor, nullptr, nullptr, 0);
+            bwd_scatter_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.cursor, w.entries, nullptr, nullptr);
+            if constexpr (kMma)
+                attend_bwd_mma_kernel<D, true><<<dim3(C, a.B * a.H), kThreads, smem, s>>>(a, w.D, w.start, w.entries);
+            else
+                attend_bwd_keymajor_kernel<T, D, true><<<dim3(C, a.B * a.H), kThreads, smem, s>>>(a, w.D, w.start,
+                                                                                                    w.entries);
+        }
+        if (a.W > 0) {
+            const dim3 grid((a.N + kChunk - 1) / kChunk, a.B * a.H);
+            if constexpr (kMma) attend_bwd_mma_kernel<D, false><<<grid, kThreads, smem, s>>>(a, w.D, nullptr, nullptr);
+            else attend_bwd_keymajor_kernel<T, D, false><<<grid, kThreads, smem, s>>>(a, w.D, nullptr, nullptr);
+        }
+        return record_cuda_error(cudaGetLastError());
     }
-    if (a.W > 0) {
-        const dim3 grid((a.N + kChunk - 1) / kChunk, a.B * a.H);
-        if constexpr (kMma) attend_bwd_mma_kernel<D, false><<<grid, kThreads, smem, s>>>(a, w.D, nullptr, nullptr);
-        else attend_bwd_keymajor_kernel<T, D, false><<<grid, kThreads, smem, s>>>(a, w.D, nullptr, nullptr);
-    }
-    return record_cuda_error(cudaGetLastError());
 }
 
 template <typename T, int D>
@@ -861,8 +984,8 @@ hils_status launch_attend_backward(hils_dtype dt, int d, const BwdAttendArgs &a,
     return d == 64 ? launch_attend_bwd<float, 64>(a, ws, s) : launch_attend_bwd<float, 128>(a, ws, s);
 }
 
-size_t attend_backward_ws_bytes(int B, int H, int Hk, int N, int K) {
-    return bwd_ws(nullptr, B, H, Hk, N, K).bytes;
+size_t attend_backward_ws_bytes(hils_dtype dt, int d, int B, int H, int Hk, int N, int K) {
+    return bwd_ws(nullptr, bwd_tc_layout(dt, d), B, H, Hk, N, K, d).bytes;
 }
 
 hils_status launch_select_backward(hils_dtype dt, int d, const BwdSelectArgs &a, cudaStream_t s) {

@@ -1,0 +1,483 @@
+// Attend backward on the 5th-generation tensor cores (bf16, d = 128): the key-major walk
+// of the hierarchical softmax's gradient ("Hierarchical Sparse Attention Done Right"
+// (picx.dev summary), Methodology 2, Eq. 10, differentiated by hand; the formulas are
+// listed at the top of backward.cu).
+//
+// A CTA takes one work item: a 64-key block of one (b, h), either a kept chunk with a run
+// of at most 1024 of the queries that kept it (entries of the group's inverted index), or
+// a block of window keys with a run of at most 1024 of the consecutive queries whose
+// window reaches it. It walks the run 128 queries per step. With Q and dO the step's 128
+// query rows and K, V the block's 64 keys:
+//   S = Q K^T, T = dO V^T            tcgen05, M = 128 queries, N = 64 keys, K = 128 dims
+//   per query row (thread = row = TMEM lane): the softmax-backward weights of the row,
+//     dl = scale * weights and cv, both rounded to bf16 into shared memory, and for a
+//     kept chunk the score gradient dscore
+//   dK^T += Q^T dl, dV^T += dO^T cv  tcgen05, M = 128 dims, N = 64 keys, K = 128 queries
+//                                    (Q, dO and dl, cv read as MN-major operands)
+//   dQ = dl K                        tcgen05, M = 128 queries, N = 128 dims, K = 64 keys
+// Each step's dQ rows are added to the float32 dQ with vector atomic adds; dK^T and dV^T
+// stay in TMEM for the whole item and are added to dK and dV once at its end.
+// Warp roles (192 threads), all hand-offs through mbarriers:
+//   warps 0-3  softmax rows and the dQ, dK, dV epilogues (TMEM lane quadrant = warp);
+//   warp 4     loads: the block's K and V (TMA tiles), each step's Q and dO rows (TMA row
+//              gathers, four rows per copy, from the contiguous bf16 copies) and the rows'
+//              scalars, into a ring of two stages;
+//   warp 5     allocates TMEM and issues tcgen05.mma (one lane).
+// S and T are double-buffered in TMEM, so that the products of step s+1 run while the
+// softmax of step s does. TMEM columns: S, T of buffer 0 [0, 128), of buffer 1
+// [128, 256), dK^T [256, 320), dV^T [320, 384), dQ [384, 512).
+// Every mbarrier wait is bounded in time (the global timer): on expiry the CTA sets bit 0
+// of the call's status word, every role stops, the copies and MMAs already started are
+// awaited (bounded again), TMEM is freed and the CTA exits without its remaining
+// gradient adds.
+#include "tc_common.cuh"
+
+namespace hils {
+namespace {
+
+using namespace tc;
+
+constexpr int kQ = 128;      // queries per step (TMEM lanes)
+constexpr int kKeys = 64;    // keys per block
+constexpr int kDim = 128;    // head dimension
+constexpr int kThr = 192;
+constexpr int kLoadWarp = 4, kMmaWarp = 5;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// shared memory map (offsets from the 1024-aligned base); every operand region holds
+// 128-byte rows with the 128-byte swizzle (16-byte unit u of row r at r * 128 +
+// ((u ^ (r % 8)) * 16)), 64-column halves of a 128-column row in separate regions
+constexpr int kKOff = 0;                 // K block: 2 halves x [64 keys x 128 B]
+constexpr int kVOff = 16384;             // V block, same
+constexpr int kQOff = 32768;             // 2 stages x 2 halves x [128 rows x 128 B]
+constexpr int kDOOff = kQOff + 65536;    // dO rows, same
+constexpr int kDLOff = kDOOff + 65536;   // dl [128 queries x 64 keys] bf16
+constexpr int kCVOff = kDLOff + 16384;   // cv, same
+constexpr int kScOff = kCVOff + 16384;   // 2 stages x [128] row scalars (int4)
+constexpr int kBarOff = kScOff + 4096;   // mbarriers
+constexpr int kMiscOff = kBarOff + 256;  // TMEM base, abort flag
+constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
+
+enum {
+    kBarFull = 0,     // + stage: Q, dO rows and scalars of a step landed (32 arrivals + bytes)
+    kBarEmpty = 2,    // + stage: every MMA that read the stage completed
+    kBarKV = 4,       // K and V of the block landed
+    kBarStFull = 5,   // + buffer: S, T written
+    kBarStFree = 7,   // + buffer: the softmax warps read S, T (4 arrivals)
+    kBarDlFull = 9,   // dl, cv of the step written (4 arrivals)
+    kBarDqFull = 10,  // dQ of the step (and every earlier MMA) completed
+    kBarDqFree = 11,  // the softmax warps read dQ (4 arrivals)
+    kBarDone = 12,    // every MMA of the item completed: dK^T, dV^T final
+    kBarDrain = 13,   // the MMA warp's own drain
+    kNumBars = 14
+};
+
+// Four rows (y0..y3) of 64 bf16 at column x of a 2-D tensor map into 512 consecutive
+// bytes of shared memory (128-byte swizzle, rows in order).
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y0,
+                                            int y1, int y2, int y3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4, %5, %6, %7}], [%2];\n" ::"r"(dst),
+        "l"(map), "r"(bar), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+        : "memory");
+}
+
+__global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                 const __grid_constant__ CUtensorMap tmV,
+                                                                 const __grid_constant__ CUtensorMap tmQ,
+                                                                 const __grid_constant__ CUtensorMap tmDO,
+                                                                 BwdTcArgs t) {
+    const BwdAttendArgs &a = t.a;
+    const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+    const int Hk = a.H / a.G, hk = h / a.G;
+    // ---- the work item (uniform over the CTA)
+    bool chunk;
+    int blk, qb, qe;
+    if ((int)blockIdx.x < t.nwin) {
+        blk = blockIdx.x / t.nsegw;
+        const int seg = blockIdx.x - blk * t.nsegw;
+        const int jb = blk * kKeys, nk = min(kKeys, a.N - jb);
+        const int qend = min(a.N, jb + nk - 1 + a.W);  // queries whose window reaches the block
+        qb = jb + seg * kBwdItemQueries;
+        qe = min(qend, qb + kBwdItemQueries);
+        chunk = false;
+    } else {
+        const int ci = blockIdx.x - t.nwin;
+        const int64_t bg = (int64_t)b * Hk + hk;
+        if (ci >= t.nitems[bg]) return;
+        const int4 it = t.items[bg * t.max_items + ci];
+        blk = it.x;
+        qb = it.y;
+        qe = it.z;
+        chunk = true;
+    }
+    if (qb >= qe) return;
+    const int ns = (qe - qb + kQ - 1) / kQ;
+    const int j0 = blk * kKeys, rows = min(kKeys, a.N - j0);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t sbase = smem_u32(smem);
+    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + kMiscOff);
+    volatile uint32_t *abort_flag = misc + 1;
+    int4 *scal = reinterpret_cast<int4 *>(smem + kScOff);
+    auto bar = [&](int i) { return sbase + kBarOff + 8u * i; };
+
+    if (tid == 0) {
+        for (int i = 0; i < kNumBars; ++i) {
+            uint32_t cnt = 1;
+            if (i == kBarFull || i == kBarFull + 1) cnt = 32;
+            if (i == kBarStFree || i == kBarStFree + 1 || i == kBarDlFull || i == kBarDqFree) cnt = 4;
+            mbar_init(bar(i), cnt);
+        }
+        misc[1] = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == kMmaWarp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(sbase + kMiscOff),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+
+    // bounded wait on work in progress (a.wait_ns of the global timer; zero, a diagnostic:
+    // every such wait expires at once); false once the CTA has aborted
+    auto wait = [&](uint32_t barrier, uint32_t parity) -> bool {
+        if (a.wait_ns > 0) {
+            if (mbar_try_wait(barrier, parity)) return true;
+            const uint64_t t0 = global_ns();
+            for (int it = 0;; ++it) {
+                if (mbar_try_wait(barrier, parity)) return true;
+                if ((it & 15) == 15) {
+                    if (*abort_flag) return false;
+                    if ((long long)(global_ns() - t0) > a.wait_ns) break;
+                }
+            }
+        }
+        *abort_flag = 1u;
+        atomicOr(t.status, 1u);
+        return false;
+    };
+    auto drain_wait = [&](uint32_t barrier, uint32_t parity) {
+        const uint64_t t0 = global_ns();
+        while (!mbar_try_wait(barrier, parity))
+            if ((long long)(global_ns() - t0) > kDrainLimitNs) break;
+    };
+    auto wait_warp = [&](uint32_t barrier, uint32_t parity) -> bool {
+        const bool ok = wait(barrier, parity);
+        return __all_sync(kFull, ok);
+    };
+    auto arrive = [&](uint32_t barrier) {
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(barrier) : "memory");
+    };
+
+    if (warp == kLoadWarp) {
+        // ---------------------------------------------------------------- loads
+        if (lane == 0) {
+            mbar_expect_tx(bar(kBarKV), 4 * kKeys * 128);
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                tma_load_4d(sbase + kKOff + x * 8192, &tmK, bar(kBarKV), x * 64, j0, hk, b);
+                tma_load_4d(sbase + kVOff + x * 8192, &tmV, bar(kBarKV), x * 64, j0, hk, b);
+            }
+        }
+        const int64_t row0 = (int64_t)bh * a.N;  // row of query 0 of (b, h) in the contiguous copies
+        const int4 *rec = t.recs + row0 * a.topk;
+        int issued[2] = {0, 0};
+        for (int s = 0; s < ns; ++s) {
+            const int st = s & 1, u = s >> 1;
+            if (u > 0 && !wait_warp(bar(kBarEmpty + st), (u - 1) & 1)) break;
+            const int q0 = qb + s * kQ;
+            int gy[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {  // rows 4 lane .. 4 lane + 3 of the step
+                const int r = 4 * lane + k, q = q0 + r;
+                int4 sc = make_int4(-1, 0, 0, 0);
+                if (q < qe) {
+                    if (chunk) {
+                        sc = __ldg(rec + q);
+                    } else {
+                        const float l = __ldg(a.lse + row0 + q);
+                        sc = make_int4(isfinite(l) ? q : -1, __float_as_int(l), __float_as_int(__ldg(t.Dv + row0 + q)),
+                                       q);
+                    }
+                }
+                scal[st * kQ + r] = sc;
+                gy[k] = (int)(row0 + (sc.x >= 0 ? sc.w : 0));  // an unused row reads query 0
+            }
+            const uint32_t dq = sbase + kQOff + st * 32768 + lane * 512;
+            const uint32_t dd = sbase + kDOOff + st * 32768 + lane * 512;
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                tma_gather4(dq + x * 16384, &tmQ, bar(kBarFull + st), x * 64, gy[0], gy[1], gy[2], gy[3]);
+                tma_gather4(dd + x * 16384, &tmDO, bar(kBarFull + st), x * 64, gy[0], gy[1], gy[2], gy[3]);
+            }
+            if (lane == 0) mbar_expect_tx(bar(kBarFull + st), 4 * kQ * 128);
+            else arrive(bar(kBarFull + st));
+            ++issued[st];
+        }
+        // every copy started lands before the CTA releases its memory
+        if (lane == 0) {
+            drain_wait(bar(kBarKV), 0);
+            for (int st = 0; st < 2; ++st)
+                if (issued[st] > 0) drain_wait(bar(kBarFull + st), (uint32_t)(issued[st] - 1) & 1u);
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ---------------------------------------------------------------- MMA issue
+        const uint32_t idS = idesc_bf16(kQ, kKeys, false);            // K-major A and B
+        const uint32_t idKV = idesc_bf16_ab(kDim, kKeys, true, true);  // MN-major A and B
+        const uint32_t idQ = idesc_bf16(kQ, kDim, true);              // K-major A, MN-major B
+        auto issue_st = [&](int s) {  // S, T of step s into buffer s % 2
+            const int st = s & 1;
+            const uint32_t dS = tmem + st * 128, dT = dS + 64;
+#pragma unroll
+            for (int ks = 0; ks < kDim / 16; ++ks) {
+                const uint32_t qo = st * 32768 + (ks >> 2) * 16384 + (ks & 3) * 32;
+                const uint32_t ko = (ks >> 2) * 8192 + (ks & 3) * 32;
+                mma_ss(dS, smem_desc(sbase + kQOff + qo, 16, 1024), smem_desc(sbase + kKOff + ko, 16, 1024), idS,
+                       ks > 0);
+                mma_ss(dT, smem_desc(sbase + kDOOff + qo, 16, 1024), smem_desc(sbase + kVOff + ko, 16, 1024), idS,
+                       ks > 0);
+            }
+            mma_commit(bar(kBarStFull + st));
+        };
+        bool ok = wait_warp(bar(kBarKV), 0) && wait_warp(bar(kBarFull), 0);
+        if (ok) {
+            tc_fence_after();
+            if (lane == 0) issue_st(0);
+            __syncwarp();
+        }
+        for (int s = 0; s < ns && ok; ++s) {
+            const int st = s & 1;
+            if (s + 1 < ns) {  // S, T of the next step, into the other buffer
+                const int s1 = s + 1, st1 = s1 & 1;
+                if (!(ok = wait_warp(bar(kBarFull + st1), (s1 >> 1) & 1))) break;
+                if (s1 >= 2 && !(ok = wait_warp(bar(kBarStFree + st1), ((s1 >> 1) - 1) & 1))) break;
+                tc_fence_after();
+                if (lane == 0) issue_st(s1);
+                __syncwarp();
+            }
+            if (!(ok = wait_warp(bar(kBarDlFull), s & 1))) break;
+            tc_fence_after();
+            if (lane == 0) {  // dK^T += Q^T dl, dV^T += dO^T cv: 16 queries per MMA
+#pragma unroll
+                for (int ks = 0; ks < kQ / 16; ++ks) {
+                    const uint32_t ro = st * 32768 + ks * 2048;
+                    mma_ss(tmem + 256, smem_desc(sbase + kQOff + ro, 16384, 1024),
+                           smem_desc(sbase + kDLOff + ks * 2048, 8192, 1024), idKV, (s > 0 || ks > 0) ? 1u : 0u);
+                    mma_ss(tmem + 320, smem_desc(sbase + kDOOff + ro, 16384, 1024),
+                           smem_desc(sbase + kCVOff + ks * 2048, 8192, 1024), idKV, (s > 0 || ks > 0) ? 1u : 0u);
+                }
+            }
+            __syncwarp();
+            if (s > 0 && !(ok = wait_warp(bar(kBarDqFree), (s - 1) & 1))) break;
+            tc_fence_after();
+            if (lane == 0) {  // dQ = dl K: 16 keys per MMA
+#pragma unroll
+                for (int ks = 0; ks < kKeys / 16; ++ks)
+                    mma_ss(tmem + 384, smem_desc(sbase + kDLOff + ks * 32, 16, 1024),
+                           smem_desc(sbase + kKOff + ks * 2048, 8192, 1024), idQ, ks > 0 ? 1u : 0u);
+                mma_commit(bar(kBarDqFull));
+                mma_commit(bar(kBarEmpty + st));
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            if (ok) mma_commit(bar(kBarDone));
+            // every MMA issued completes before TMEM and shared memory are released
+            mma_commit(bar(kBarDrain));
+            drain_wait(bar(kBarDrain), 0);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- softmax rows
+        const int r = warp * 32 + lane;  // query row of the step = TMEM lane
+        const uint32_t lb = (uint32_t)(warp * 32) << 16;
+        const float sl2 = a.scale * kLog2e;
+        const int K = a.topk;
+        int prev = -1;  // query of this row in the previous step (its dQ row), or -1
+        // this row's dQ of the last completed step into the global dQ
+        auto dq_out = [&](int qrow) {
+            float *dst = a.dQ + ((int64_t)bh * a.N + (qrow < 0 ? 0 : qrow)) * kDim;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lb + 384 + c * 32, v);
+                tmem_wait_ld();
+                if (qrow >= 0) {
+                    if (t.vec_ok) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            atomicAdd(reinterpret_cast<float4 *>(dst + c * 32 + 4 * u),
+                                      make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
+                                                  __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3])));
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) atomicAdd(dst + c * 32 + u, __uint_as_float(v[u]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive(bar(kBarDqFree));
+        };
+        bool ok = true;
+        for (int s = 0; s < ns; ++s) {
+            const int st = s & 1;
+            if (!(ok = wait_warp(bar(kBarStFull + st), (s >> 1) & 1))) break;
+            tc_fence_after();
+            uint32_t s0[32], s1[32], t0[32], t1[32];
+            tmem_ld32(tmem + lb + st * 128, s0);
+            tmem_ld32(tmem + lb + st * 128 + 32, s1);
+            tmem_ld32(tmem + lb + st * 128 + 64, t0);
+            tmem_ld32(tmem + lb + st * 128 + 96, t1);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive(bar(kBarStFree + st));
+            const int4 sc = scal[st * kQ + r];
+            const int en = sc.x, qi = sc.w;
+            const float wl = __int_as_float(sc.y), Dd = __int_as_float(sc.z);
+            auto S = [&](int j) { return __uint_as_float(j < 32 ? s0[j] : s1[j - 32]); };
+            auto T = [&](int j) { return __uint_as_float(j < 32 ? t0[j] : t1[j - 32]); };
+            uint32_t dlp[32], cvp[32];  // bf16 pairs of keys 2p, 2p + 1
+            if (en < 0) {
+#pragma unroll
+                for (int p = 0; p < 32; ++p) dlp[p] = cvp[p] = 0u;
+            } else if (chunk) {
+                // p_j = softmax over the chunk of scale S_j; o_c . dO = sum_j p_j T_j;
+                // dl_j = w p_j (T_j - o_c . dO), cv_j = w p_j; dscore = w (o_c . dO - D_i)
+                float m = S(0);
+#pragma unroll
+                for (int j = 1; j < kKeys; ++j) m = fmaxf(m, S(j));
+                float e[kKeys], z = 0.f, oc = 0.f;
+#pragma unroll
+                for (int j = 0; j < kKeys; ++j) {
+                    e[j] = ex2((S(j) - m) * sl2);
+                    z += e[j];
+                    oc = fmaf(e[j], T(j), oc);
+                }
+                const float inv = 1.f / z;
+                oc *= inv;
+                const float wc = wl * inv;
+#pragma unroll
+                for (int p = 0; p < 32; ++p) {
+                    const float c0 = wc * e[2 * p], c1 = wc * e[2 * p + 1];
+                    cvp[p] = pack_bf16(c0, c1);
+                    dlp[p] = pack_bf16(a.scale * c0 * (T(2 * p) - oc), a.scale * c1 * (T(2 * p + 1) - oc));
+                }
+                a.dscore[((int64_t)bh * a.N + qi) * K + (en & 31)] = wl * (oc - Dd);
+            } else {
+                // window key j0 + j of query qi: c_j = exp(scale S_j - lse), dl_j = c_j (T_j - D_i)
+                const float l2 = wl * kLog2e;
+#pragma unroll
+                for (int p = 0; p < 32; ++p) {
+                    float c[2];
+#pragma unroll
+                    for (int hv = 0; hv < 2; ++hv) {
+                        const int j = 2 * p + hv, key = j0 + j;
+                        const bool in = j < rows && key <= qi && key > qi - a.W;
+                        c[hv] = in ? ex2(fmaf(S(j), sl2, -l2)) : 0.f;
+                    }
+                    cvp[p] = pack_bf16(c[0], c[1]);
+                    dlp[p] = pack_bf16(a.scale * c[0] * (T(2 * p) - Dd), a.scale * c[1] * (T(2 * p + 1) - Dd));
+                }
+            }
+            // dl, cv of the previous step were read by its MMAs once its dQ completed
+            if (s > 0) {
+                if (!(ok = wait_warp(bar(kBarDqFull), (s - 1) & 1))) break;
+                tc_fence_after();
+            }
+            uint8_t *dlrow = smem + kDLOff + r * 128, *cvrow = smem + kCVOff + r * 128;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int o = (u ^ (r & 7)) << 4;
+                *reinterpret_cast<uint4 *>(dlrow + o) = make_uint4(dlp[4 * u], dlp[4 * u + 1], dlp[4 * u + 2], dlp[4 * u + 3]);
+                *reinterpret_cast<uint4 *>(cvrow + o) = make_uint4(cvp[4 * u], cvp[4 * u + 1], cvp[4 * u + 2], cvp[4 * u + 3]);
+            }
+            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            __syncwarp();
+            if (lane == 0) arrive(bar(kBarDlFull));
+            if (s > 0) dq_out(prev);
+            prev = en >= 0 ? qi : -1;
+        }
+        if (ok && wait_warp(bar(kBarDqFull), (ns - 1) & 1)) {
+            tc_fence_after();
+            dq_out(prev);
+        } else {
+            ok = false;
+        }
+        // dK^T and dV^T: row r of TMEM is dimension x = r; key j in column j
+        if (ok && wait_warp(bar(kBarDone), 0)) {
+            tc_fence_after();
+            const int64_t kvrow = ((int64_t)b * Hk + hk) * a.N + j0;
+            float *dk = a.dK + kvrow * kDim + r;
+            float *dv = a.dV + kvrow * kDim + r;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t vk[32], vv[32];
+                tmem_ld32(tmem + lb + 256 + c * 32, vk);
+                tmem_ld32(tmem + lb + 320 + c * 32, vv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const int j = c * 32 + u;
+                    if (j < rows) {
+                        atomicAdd(dk + (int64_t)j * kDim, __uint_as_float(vk[u]));
+                        atomicAdd(dv + (int64_t)j * kDim, __uint_as_float(vv[u]));
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+// [rows, 128] contiguous bf16 -> 2-D map for four-row gathers: a (64 elements x 1 row)
+// box, 128-byte swizzle.
+bool make_row_map(CUtensorMap *m, const void *ptr, int64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kDim * 2};
+    const cuuint32_t box[2] = {64u, 1u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+hils_status launch_attend_bwd_tc(const BwdTcArgs &t, const void *Qc, const void *dOb, cudaStream_t s) {
+    const BwdAttendArgs &a = t.a;
+    const int Hk = a.H / a.G;
+    const int64_t nrows = (int64_t)a.B * a.H * a.N;
+    const int gx = t.nwin + t.max_items;
+    if (gx == 0 || nrows == 0) return HILS_OK;
+    CUtensorMap mk, mv, mq, mdo;
+    if (!make_map(&mk, a.K, a.B, Hk, a.N, kKeys) || !make_map(&mv, a.V, a.B, Hk, a.N, kKeys) ||
+        !make_row_map(&mq, Qc, nrows) || !make_row_map(&mdo, dOb, nrows))
+        return HILS_ERR_CUDA;
+    static KernelSetup setup;
+    int per_sm = 0;
+    const hils_status st = kernel_setup(setup, (const void *)attend_bwd_tc_kernel, kThr, kSmemBytes, &per_sm);
+    if (st != HILS_OK) return st;
+    if (per_sm < 1) return HILS_ERR_CUDA;
+    attend_bwd_tc_kernel<<<dim3(gx, a.B * a.H), kThr, kSmemBytes, s>>>(mk, mv, mq, mdo, t);
+    return record_cuda_error(cudaGetLastError());
+}
+
+}  // namespace hils

@@ -235,7 +235,7 @@ size_t hils_workspace_bytes(const hils_params *p, int call, int Lq, int C) {
     case HILS_CALL_SELECT: return select_ws_for(p, Lq, C);
     case HILS_CALL_ATTEND_PREFILL: return kPrefillWsBytes;
     case HILS_CALL_ATTEND_DECODE: return attend_decode_ws_bytes(p->B * p->H, decode_units(p), p->d);
-    case HILS_CALL_ATTEND_BACKWARD: return attend_backward_ws_bytes(p->B, p->H, p->H / groups(p), Lq, p->K);
+    case HILS_CALL_ATTEND_BACKWARD: return attend_backward_ws_bytes(p->dtype, p->d, p->B, p->H, p->H / groups(p), Lq, p->K);
     case HILS_CALL_DECODE:
         return decode_select_part(select_ws_for(p, 1, C)) + attend_decode_ws_bytes(p->B * p->H, decode_units(p), p->d);
     default: return 0;
@@ -322,7 +322,7 @@ int hils_attend_prefill_backward(const hils_params *p, hils_ctensor Q, hils_cten
     HILS_TRY(check_array(dscore, nq * p->K));
     if (nq == 0) return HILS_OK;
     HILS_TRY(check_workspace(workspace, ws_bytes,
-                             attend_backward_ws_bytes(p->B, p->H, p->H / groups(p), N, p->K)));
+                             attend_backward_ws_bytes(p->dtype, p->d, p->B, p->H, p->H / groups(p), N, p->K)));
     BwdAttendArgs a;
     a.Q = {Q.ptr, Q.sb, Q.sh, Q.st};
     a.K = {K.ptr, K.sb, K.sh, K.st};
@@ -344,6 +344,7 @@ int hils_attend_prefill_backward(const hils_params *p, hils_ctensor Q, hils_cten
     a.W = p->W;
     a.G = groups(p);
     a.scale = scale;
+    a.wait_ns = work_wait_ns(p->flags);
     return launch_attend_backward(p->dtype, p->d, a, workspace, stream);
 }
 

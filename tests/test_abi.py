@@ -260,19 +260,27 @@ def test_backward_binding_checks():
 
 
 def test_backward_workspace_size(lib):
-    """HILS_CALL_ATTEND_BACKWARD: D_i per query, then per (b, group) chunk counts, starts,
-    cursors and the inverted index, each part rounded up to 256 bytes."""
-    p = hils.Params(B=2, H=4, d=128, K=16, W=512, dtype=torch.bfloat16, H_kv=2)
-    c = p.c()
+    """HILS_CALL_ATTEND_BACKWARD: a 256-byte status word, D_i per query, then per (b,
+    group) chunk counts, starts, cursors and the inverted index; for bf16 with d = 128 (the
+    tensor-core walk) also one 16-byte record per (query head, index entry), the chunk
+    items (at most C + ceil(N K / 1024) per group, 16 bytes each) and their counts, and
+    bf16 copies of dO and Q; each part rounded up to 256 bytes."""
     N = 8192
     C = N // 64
 
     def a256(x):
         return (x + 255) // 256 * 256
 
-    want = a256(2 * 4 * N * 4) + a256(2 * 2 * C * 4) + a256(2 * 2 * (C + 1) * 4) + a256(2 * 2 * C * 4) + \
+    base = 256 + a256(2 * 4 * N * 4) + a256(2 * 2 * C * 4) + a256(2 * 2 * (C + 1) * 4) + a256(2 * 2 * C * 4) + \
         a256(2 * 2 * N * 16 * 4)
-    assert lib.hils_workspace_bytes(ctypes.byref(c), hils.HILS_CALL_ATTEND_BACKWARD, N, 0) == want
+    p = hils.Params(B=2, H=4, d=64, K=16, W=512, dtype=torch.bfloat16, H_kv=2)
+    assert lib.hils_workspace_bytes(ctypes.byref(p.c()), hils.HILS_CALL_ATTEND_BACKWARD, N, 0) == base
+    p = hils.Params(B=2, H=4, d=128, K=16, W=512, dtype=torch.float32, H_kv=2)
+    assert lib.hils_workspace_bytes(ctypes.byref(p.c()), hils.HILS_CALL_ATTEND_BACKWARD, N, 0) == base
+    p = hils.Params(B=2, H=4, d=128, K=16, W=512, dtype=torch.bfloat16, H_kv=2)
+    items = C + (N * 16 + 1023) // 1024
+    tc = a256(2 * 4 * N * 16 * 16) + a256(2 * 2 * items * 16) + a256(2 * 2 * 4) + 2 * a256(2 * 4 * N * 128 * 2)
+    assert lib.hils_workspace_bytes(ctypes.byref(p.c()), hils.HILS_CALL_ATTEND_BACKWARD, N, 0) == base + tc
 
 
 def test_decode_time_and_backward_entry_points_validate_first(lib):

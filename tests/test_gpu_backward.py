@@ -8,8 +8,10 @@ observed about 5e-7); bf16 inputs 1e-2, the forward's bar (the forward's O and s
 table are stored in bf16, which moves D_i and the chunk scores by up to 2^-9 relative,
 and the tensor-core products take dO, dl and cv rounded to bf16; observed about 3e-3).
 Element-wise, every gradient's largest error is within twice that bar times the
-gradient's largest magnitude. The cases cover K = 0 (no kept chunk), W = 0 (no window)
-and a table of 400 chunks (the score backward's per-query kernel)."""
+gradient's largest magnitude. The cases cover K = 0 (no kept chunk), W = 0 (no window),
+a table of 400 chunks (the score backward's per-query kernel; chunk 0's list of
+thousands of queries is cut into runs of 1024), grouped heads and a window longer than
+a run. The last test makes every bounded wait of the tensor-core walk expire."""
 import numpy as np
 import pytest
 import torch
@@ -36,6 +38,11 @@ CASES = {
     # 400 chunks: the score backward's [C][d] table no longer fits in shared memory, so
     # the per-query kernel with global atomics runs
     "bf16_d128_C400": (WORKLOADS[2].replace(H=1, N=64 * 400, K=16, W=512), 1e-2),
+    # the tensor-core walk (bf16, d = 128) with query heads sharing a kept list
+    "bf16_d128_grouped": (WORKLOADS[7].replace(H=4, Hk=2, d=128, N=64 * 5 + 3, K=3, W=130), 1e-2),
+    # a window longer than one work item's 1024 queries: each window block's queries are
+    # cut into two runs, whose dK and dV shares add up
+    "bf16_d128_W1500": (WORKLOADS[2].replace(H=1, N=64 * 40 + 5, K=4, W=1500), 1e-2),
 }
 
 
@@ -175,3 +182,43 @@ def test_backward_full_size(cuda_device, case):
         assert not bad, f"kv head {hk}: relative L2 errors above 1e-2: {bad} (all: {errs})"
         bad = {k: v for k, v in maxe.items() if not v <= 2e-2}
         assert not bad, f"kv head {hk}: max-abs errors above 2e-2 of the largest gradient: {bad} (all: {maxe})"
+
+
+def test_backward_waits_expire_and_recover(cuda_device):
+    """The tensor-core attend backward (bf16, d = 128) with every wait on work in progress
+    made to expire at its first check (HILS_FLAG_DIAG_EXPIRE_WAITS): the call returns
+    with bit 0 of its status word set, dK and dV (accumulated) left as they were, dQ and
+    dscore as the call's own clearing left them (zero); then the same call with the normal
+    time limit gives the oracle's gradients."""
+    w = WORKLOADS[2].replace(H=2, N=64 * 6 + 9, K=4, W=100)
+    inp = make_prefill(w)
+    d = to_dev(inp, cuda_device)
+    Ksum, Bsum = gpu_summarize(w, d["K"], d["LQ"])
+    idx, score, nsel = gpu_select(w, d["Qcal"], Ksum, Bsum)
+    O, lse = gpu_prefill(w, d["Q"], d["K"], d["V"], idx, score, nsel)
+    g = torch.Generator().manual_seed(7)
+    dO = torch.randn(O.shape, generator=g).to(cuda_device)
+    B, H, N, dd, Hk, K = w.B, w.H, w.N, w.d, w.Hkv, w.K
+    f32 = dict(dtype=torch.float32, device=cuda_device)
+    dQ, dscore = torch.full((B, H, N, dd), 5.0, **f32), torch.full((B, H, N, K), 5.0, **f32)
+    dK, dV = torch.full((B, Hk, N, dd), 3.0, **f32), torch.full((B, Hk, N, dd), 3.0, **f32)
+    pd = P(w, flags=hils.HILS_FLAG_DIAG_EXPIRE_WAITS)
+    ws = hils.alloc_workspace(pd, hils.HILS_CALL_ATTEND_BACKWARD, N, 0, device=cuda_device)
+    hils.hils_attend_prefill_backward(pd, d["Q"], d["K"], d["V"], idx, score, nsel, O, lse, dO, dQ, dK, dV, dscore,
+                                      workspace=ws)
+    torch.cuda.synchronize()
+    assert int(host(ws[:4]).view(torch.int32)[0]) & 1, "no wait expired"
+    assert (host(dK) == 3.0).all() and (host(dV) == 3.0).all(), "the diagnostic call added to dK or dV"
+    assert (host(dQ) == 0.0).all() and (host(dscore) == 0.0).all(), "the diagnostic call wrote dQ or dscore"
+    p = P(w)
+    dK.zero_()
+    dV.zero_()
+    hils.hils_attend_prefill_backward(p, d["Q"], d["K"], d["V"], idx, score, nsel, O, lse, dO, dQ, dK, dV, dscore,
+                                      workspace=ws)
+    torch.cuda.synchronize()
+    assert int(host(ws[:4]).view(torch.int32)[0]) == 0, "the status word was not cleared by the normal call"
+    full = ob.grads(inp["Q"], inp["K"], inp["V"], inp["Qcal"], inp["LQ"], host(idx), host(nsel), host(dO), 64, w.W,
+                    w.scale, batch=256)
+    # the attend call's own gradients (dK also takes the summaries' share, added later)
+    for name, got in (("dQ", dQ), ("dV", dV), ("dscore", dscore)):
+        assert _rel(got, full[name]) <= 1e-2, f"{name} after the diagnostic call"
