@@ -598,7 +598,8 @@ def run_profile_case(args):
     prefill:       the full 8K prefill workload (summarise, select, attend);
     prefill-select: the select of the 8K prefill, multi-head then grouped-query (32 query
                    heads, 8 key-value heads), `warmup + steps` launches each;
-    prefill-backward: the attend backward of the 8K prefill for the forward's selection.
+    prefill-backward: the attend backward of the 8K prefill for the forward's selection, then
+                   its score backward (hils_select_backward), `warmup + steps` launches each.
     Runs `warmup + steps` plain launches of the case and exits."""
     import hierarchical_chunk_sparse_b200 as hils
 
@@ -645,8 +646,13 @@ def run_profile_case(args):
         dK, dV = torch.zeros(w.B, w.Hkv, w.N, w.d, **f32), torch.zeros(w.B, w.Hkv, w.N, w.d, **f32)
         ws = hils.alloc_workspace(pb.p, hils.HILS_CALL_ATTEND_BACKWARD, w.N, 0, device=dev)
         i = pb.inp
-        fn = lambda: hils.hils_attend_prefill_backward(pb.p, i["Q"], i["K"], i["V"], pb.idx, pb.score,  # noqa
-                                                       pb.nsel, pb.O, pb.lse, dO, dQ, dK, dV, dscore, workspace=ws)
+        dQcal = torch.empty(w.B, w.H, w.N, w.d, **f32)
+        dKsum, dBsum = torch.zeros(w.B, w.H, w.C, w.d, **f32), torch.zeros(w.B, w.H, w.C, **f32)
+        for _ in range(args.warmup + args.steps):
+            hils.hils_attend_prefill_backward(pb.p, i["Q"], i["K"], i["V"], pb.idx, pb.score, pb.nsel, pb.O, pb.lse,
+                                              dO, dQ, dK, dV, dscore, workspace=ws)
+        fn = lambda: hils.hils_select_backward(pb.p, i["Qcal"], pb.Ksum, pb.idx, pb.nsel, dscore, dQcal,  # noqa
+                                               dKsum, dBsum)
     elif case == "prefill-select":
         benches = [PrefillBench(WORKLOADS[n], dev) for n in (2, 7)]
         for pb in benches:

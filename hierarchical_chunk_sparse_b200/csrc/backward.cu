@@ -214,8 +214,23 @@ __global__ void __launch_bounds__(1024) bwd_scan_kernel(int C, const int *count,
     if (t == 1023) nitems[bg] = part[1023];
 }
 
-// Fills the inverted index; with `recs`, also each query head's record of the entry:
+// The record of index entry `pos` (query i, slot k) for each query head of group g:
 // {i * 32 + k (or -1 when the row's lse is not finite), w = exp(s^_{i,c} - lse_i), D_i, i}.
+__device__ __forceinline__ void write_records(const BwdAttendArgs &a, const float *Dv, int4 *recs, int b, int g,
+                                              int i, int k, int pos) {
+    const int K = a.topk;
+    for (int hh = 0; hh < a.G; ++hh) {
+        const int64_t bh = (int64_t)b * a.H + g * a.G + hh;
+        const int64_t qh = bh * a.N + i;
+        const float lse = a.lse[qh];
+        const bool fin = isfinite(lse);
+        const float w = fin ? expf(a.score[qh * K + k] - lse) : 0.f;
+        recs[bh * a.N * K + pos] = make_int4(fin ? i * 32 + k : -1, __float_as_int(w), __float_as_int(Dv[qh]), i);
+    }
+}
+
+// Fills the inverted index (`entries`: i * 32 + k, or null) and/or each query head's
+// records of its entries (`recs`, or null); one thread per (b, group, i, k).
 __global__ void bwd_scatter_kernel(BwdAttendArgs a, int *cursor, int *entries, const float *Dv, int4 *recs) {
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int Hk = a.H / a.G, K = a.topk, C = a.N / kChunk;
@@ -228,17 +243,93 @@ __global__ void bwd_scatter_kernel(BwdAttendArgs a, int *cursor, int *entries, c
     const int64_t bg = qg / a.N;
     const int i = (int)(qg % a.N);
     const int pos = atomicAdd(&cursor[bg * C + c], 1);
-    entries[bg * (int64_t)a.N * K + pos] = i * 32 + k;
-    if (!recs) return;
-    const int b = (int)(bg / Hk), g = (int)(bg % Hk);
-    for (int hh = 0; hh < a.G; ++hh) {
-        const int64_t bh = (int64_t)b * a.H + g * a.G + hh;
-        const int64_t qh = bh * a.N + i;
-        const float lse = a.lse[qh];
-        const bool fin = isfinite(lse);
-        const float w = fin ? expf(a.score[qh * K + k] - lse) : 0.f;
-        recs[bh * a.N * K + pos] = make_int4(fin ? i * 32 + k : -1, __float_as_int(w), __float_as_int(Dv[qh]), i);
+    if (entries) entries[bg * (int64_t)a.N * K + pos] = i * 32 + k;
+    if (recs) write_records(a, Dv, recs, (int)(bg / Hk), (int)(bg % Hk), i, k, pos);
+}
+
+// The same two passes with the counts of a run of kIdxQueries queries first summed in
+// shared memory (one counter per chunk): the global counters and cursors then take one
+// atomic add per (CTA, chunk touched) instead of one per entry. Dynamic shared memory:
+// C ints (count), 2 C ints (scatter). grid: (ceil(N / kIdxQueries), B * Hk).
+constexpr int kIdxQueries = 256;
+constexpr int kIdxThreads = 256;
+constexpr int kIdxSmemMax = 96 * 1024;
+
+__device__ __forceinline__ void run_histogram(const BwdAttendArgs &a, int64_t bg, int i0, int i1, int *hist) {
+    const int K = a.topk, C = a.N / kChunk;
+    for (int c = threadIdx.x; c < C; c += kIdxThreads) hist[c] = 0;
+    __syncthreads();
+    for (int64_t e = (bg * a.N + i0) * K + threadIdx.x; e < (bg * a.N + i1) * K; e += kIdxThreads) {
+        const int64_t qg = e / K;
+        const int k = (int)(e - qg * K);
+        if (k >= min(max(a.nsel[qg], 0), K)) continue;
+        const int c = a.idx[e];
+        if (c >= 0 && c < C) atomicAdd(&hist[c], 1);
     }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(kIdxThreads) bwd_count_runs_kernel(BwdAttendArgs a, int *count) {
+    extern __shared__ int hist[];
+    const int C = a.N / kChunk;
+    const int64_t bg = blockIdx.y;
+    const int i0 = blockIdx.x * kIdxQueries, i1 = min(a.N, i0 + kIdxQueries);
+    run_histogram(a, bg, i0, i1, hist);
+    for (int c = threadIdx.x; c < C; c += kIdxThreads)
+        if (hist[c]) atomicAdd(&count[bg * C + c], hist[c]);
+}
+
+__global__ void __launch_bounds__(kIdxThreads) bwd_scatter_runs_kernel(BwdAttendArgs a, int *cursor, int *entries,
+                                                                       const float *Dv, int4 *recs) {
+    extern __shared__ int hist[];  // [C] counts, then [C] this run's first positions
+    const int C = a.N / kChunk, K = a.topk, Hk = a.H / a.G;
+    int *base = hist + C;
+    const int64_t bg = blockIdx.y;
+    const int i0 = blockIdx.x * kIdxQueries, i1 = min(a.N, i0 + kIdxQueries);
+    run_histogram(a, bg, i0, i1, hist);
+    for (int c = threadIdx.x; c < C; c += kIdxThreads) {
+        base[c] = hist[c] ? atomicAdd(&cursor[bg * C + c], hist[c]) : 0;
+        hist[c] = 0;
+    }
+    __syncthreads();
+    for (int64_t e = (bg * a.N + i0) * K + threadIdx.x; e < (bg * a.N + i1) * K; e += kIdxThreads) {
+        const int64_t qg = e / K;
+        const int k = (int)(e - qg * K);
+        if (k >= min(max(a.nsel[qg], 0), K)) continue;
+        const int c = a.idx[e];
+        if (c < 0 || c >= C) continue;
+        const int i = (int)(qg - bg * a.N);
+        const int pos = base[c] + atomicAdd(&hist[c], 1);
+        if (entries) entries[bg * (int64_t)a.N * K + pos] = i * 32 + k;
+        if (recs) write_records(a, Dv, recs, (int)(bg / Hk), (int)(bg % Hk), i, k, pos);
+    }
+}
+
+// Builds the group's inverted index (counts, starts and cursors; chunk items when `items`
+// is given) and fills `entries` and/or `recs`.
+hils_status build_index(const BwdAttendArgs &a, const BwdWs &w, int *entries, int4 *recs, int4 *items, int *nitems,
+                        int max_items, cudaStream_t s) {
+    const int Hk = a.H / a.G, C = a.N / kChunk;
+    hils_status st = record_cuda_error(cudaMemsetAsync(w.count, 0, (size_t)a.B * Hk * C * sizeof(int), s));
+    if (st != HILS_OK) return st;
+    const size_t smem = (size_t)2 * C * sizeof(int);
+    if (smem <= (size_t)kIdxSmemMax) {
+        static KernelSetup setup_c, setup_s;
+        st = kernel_setup(setup_c, (const void *)bwd_count_runs_kernel, kIdxThreads, kIdxSmemMax / 2, nullptr);
+        if (st != HILS_OK) return st;
+        st = kernel_setup(setup_s, (const void *)bwd_scatter_runs_kernel, kIdxThreads, kIdxSmemMax, nullptr);
+        if (st != HILS_OK) return st;
+        const dim3 grid((a.N + kIdxQueries - 1) / kIdxQueries, a.B * Hk);
+        bwd_count_runs_kernel<<<grid, kIdxThreads, smem / 2, s>>>(a, w.count);
+        bwd_scan_kernel<<<(unsigned)(a.B * Hk), 1024, 0, s>>>(C, w.count, w.start, w.cursor, items, nitems, max_items);
+        bwd_scatter_runs_kernel<<<grid, kIdxThreads, smem, s>>>(a, w.cursor, entries, w.D, recs);
+    } else {
+        const int64_t ne = (int64_t)a.B * Hk * a.N * a.topk;
+        bwd_count_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.count);
+        bwd_scan_kernel<<<(unsigned)(a.B * Hk), 1024, 0, s>>>(C, w.count, w.start, w.cursor, items, nitems, max_items);
+        bwd_scatter_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.cursor, entries, w.D, recs);
+    }
+    return record_cuda_error(cudaGetLastError());
 }
 
 constexpr int kQT = 16;  // queries per step of the key-major kernel
@@ -717,26 +808,36 @@ __global__ void __launch_bounds__(kThreads) select_backward_kernel(BwdSelectArgs
 }
 
 // Eq. 7 backward with the chunk sums kept in shared memory: a CTA takes kSelBwdRows
-// consecutive queries of one (b, h), adds scale ds q~ into its own [C][D] table (and ds
-// into [C]) with shared-memory atomics, writes dQcal, and then adds each table row that
-// a kept chunk touched to dKsum and dBsum once. Adjacent queries keep mostly the same
-// chunks, so the global atomics drop from one per (query, kept chunk, x) to about one
-// per (CTA, touched chunk, x). Used when the table fits in shared memory.
-constexpr int kSelBwdRows = 128;
+// consecutive queries of one (b, h), a warp one query at a time, adds scale ds q~ into
+// its own [C][D] table (and ds into [C]) with shared-memory atomics, writes dQcal, and
+// then adds each table row that a kept chunk touched to dKsum and dBsum once (vector
+// atomics when dKsum is 16-byte aligned). Adjacent queries keep mostly the same chunks,
+// so the global atomics drop from one per (query, kept chunk, x) to about one per (CTA,
+// touched chunk, x). When it fits, the head's k' table is first copied into shared
+// memory, so that a query's kept rows are read there, not from L2; each warp loads the
+// next query's kept list before working on the current one. Used when the tables fit.
+constexpr int kSelBwdRows = 256;
+constexpr int kSelBwdThreads = 256;
 constexpr int kSelBwdSmemMax = 200 * 1024;
 
-inline size_t select_bwd_table_bytes(int C, int D) {
-    return (size_t)C * D * 4 + (size_t)C * 4 + (size_t)((C + 31) / 32) * 4;
+__host__ __device__ inline size_t select_bwd_table_bytes(int C, int D) {
+    return ((size_t)C * D * 4 + (size_t)C * 4 + (size_t)((C + 31) / 32) * 4 + 15) & ~(size_t)15;
+}
+template <typename T>
+inline size_t select_bwd_smem_bytes(int C, int D, bool stage) {
+    return select_bwd_table_bytes(C, D) + (stage ? (size_t)C * D * sizeof(T) : 0);
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads) select_backward_table_kernel(BwdSelectArgs a) {
+__global__ void __launch_bounds__(kSelBwdThreads) select_backward_table_kernel(BwdSelectArgs a, int stage, int vec) {
     extern __shared__ __align__(16) float tsm[];
     constexpr int kPer = D / 32;  // elements of a row per lane
+    constexpr int kWarps = kSelBwdThreads / 32;
     const int C = a.C;
     float *tk = tsm;                                           // [C][D]
     float *tb = tk + (int64_t)C * D;                           // [C]
     unsigned *touched = reinterpret_cast<unsigned *>(tb + C);  // C bits
+    T *ks = reinterpret_cast<T *>(reinterpret_cast<uint8_t *>(tsm) + select_bwd_table_bytes(C, D));  // [C][D]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nblk = (a.Lq + kSelBwdRows - 1) / kSelBwdRows;
     const int64_t bh = blockIdx.x / nblk;
@@ -744,28 +845,49 @@ __global__ void __launch_bounds__(kThreads) select_backward_table_kernel(BwdSele
     const int h = (int)(bh % a.H), b = (int)(bh / a.H);
     const int Hk = a.H / a.G;
     const int K = a.topk;
-    for (int e = tid; e < C * D; e += kThreads) tk[e] = 0.f;
-    for (int e = tid; e < C; e += kThreads) tb[e] = 0.f;
-    for (int e = tid; e < (C + 31) / 32; e += kThreads) touched[e] = 0u;
-    __syncthreads();
     const T *khead = static_cast<const T *>(a.Ksum.ptr) + b * a.Ksum.sb + h * a.Ksum.sh;
+    for (int e = tid; e < C * D; e += kSelBwdThreads) tk[e] = 0.f;
+    for (int e = tid; e < C; e += kSelBwdThreads) tb[e] = 0.f;
+    for (int e = tid; e < (C + 31) / 32; e += kSelBwdThreads) touched[e] = 0u;
+    if (stage) {  // the head's k' rows, 16 bytes per copy
+        constexpr int kU = D * (int)sizeof(T) / 16;  // 16-byte units per row
+        for (int e = tid; e < C * kU; e += kSelBwdThreads) {
+            const int c = e / kU, u = e - c * kU;
+            reinterpret_cast<uint4 *>(ks + (int64_t)c * D)[u] =
+                reinterpret_cast<const uint4 *>(khead + (int64_t)c * a.Ksum.st)[u];
+        }
+    }
+    __syncthreads();
+    const T *kbase = stage ? ks : khead;
+    const int64_t kst = stage ? D : a.Ksum.st;
     const int iend = min(a.Lq, i0 + kSelBwdRows);
-    for (int i = i0 + warp; i < iend; i += kThreads / 32) {  // a warp per query
+    // lane k holds kept chunk k's index and gradient (K <= 32)
+    auto load_list = [&](int i, int &c, float &ds, int &ns) {
+        ns = 0;
+        c = 0;
+        ds = 0.f;
+        if (i >= iend) return;
         const int64_t qi = bh * a.Lq + i;
         const int64_t qg = ((int64_t)b * Hk + h / a.G) * a.Lq + i;
-        const int ns = K > 0 ? min(max(a.nsel[qg], 0), K) : 0;
-        const T *qrow = static_cast<const T *>(a.Qcal.ptr) + b * a.Qcal.sb + h * a.Qcal.sh + (int64_t)i * a.Qcal.st;
-        // lane k holds kept chunk k's index and gradient (K <= 32), so the k' row loads
-        // below depend only on shuffles and several can be in flight
-        int myc = 0;
-        float myds = 0.f;
-        if (lane < ns) {
-            const int c = a.idx[qg * K + lane];
-            const bool ok = (unsigned)c < (unsigned)C;
-            myc = ok ? c : 0;
-            myds = ok ? a.dscore[qi * K + lane] : 0.f;
-            if (ok) atomicOr(&touched[c >> 5], 1u << (c & 31));
+        ns = K > 0 ? min(max(a.nsel[qg], 0), K) : 0;
+        if (lane < K) {
+            const int cc = a.idx[qg * K + lane];
+            const float d = a.dscore[qi * K + lane];
+            const bool ok = lane < ns && (unsigned)cc < (unsigned)C;
+            c = ok ? cc : 0;
+            ds = ok ? d : 0.f;
         }
+    };
+    int myc, ns;
+    float myds;
+    load_list(i0 + warp, myc, myds, ns);
+    for (int i = i0 + warp; i < iend; i += kWarps) {
+        int nc, nn;
+        float nd;
+        load_list(i + kWarps, nc, nd, nn);  // the next query's list, in flight meanwhile
+        const int64_t qi = bh * a.Lq + i;
+        const T *qrow = static_cast<const T *>(a.Qcal.ptr) + b * a.Qcal.sb + h * a.Qcal.sh + (int64_t)i * a.Qcal.st;
+        if (lane < ns && myds != 0.f) atomicOr(&touched[myc >> 5], 1u << (myc & 31));
         float qx[kPer], acc[kPer];
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
@@ -776,7 +898,7 @@ __global__ void __launch_bounds__(kThreads) select_backward_table_kernel(BwdSele
         for (int k = 0; k < ns; ++k) {
             const int c = __shfl_sync(kFull, myc, k);
             const float ds = __shfl_sync(kFull, myds, k);
-            const T *krow = khead + (int64_t)c * a.Ksum.st;
+            const T *krow = kbase + (int64_t)c * kst;
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
                 acc[u] = fmaf(ds, elem(krow, lane + 32 * u), acc[u]);
@@ -786,14 +908,25 @@ __global__ void __launch_bounds__(kThreads) select_backward_table_kernel(BwdSele
         if (lane < ns) atomicAdd(&tb[myc], myds);
 #pragma unroll
         for (int u = 0; u < kPer; ++u) a.dQcal[qi * D + lane + 32 * u] = a.scale * acc[u];
+        myc = nc;
+        myds = nd;
+        ns = nn;
     }
     __syncthreads();
     float *dks = a.dKsum + bh * C * D;
     float *dbs = a.dBsum + bh * C;
-    for (int c = warp; c < C; c += kThreads / 32) {
+    for (int c = warp; c < C; c += kWarps) {
         if (!((touched[c >> 5] >> (c & 31)) & 1u)) continue;
+        if (vec && D == 128) {  // lane l: elements 4 l .. 4 l + 3
+            const float4 v = *reinterpret_cast<const float4 *>(&tk[c * D + 4 * lane]);
+            atomicAdd(reinterpret_cast<float4 *>(dks + (int64_t)c * D + 4 * lane), v);
+        } else if (vec) {  // D = 64: lane l: elements 2 l, 2 l + 1
+            const float2 v = *reinterpret_cast<const float2 *>(&tk[c * D + 2 * lane]);
+            atomicAdd(reinterpret_cast<float2 *>(dks + (int64_t)c * D + 2 * lane), v);
+        } else {
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) atomicAdd(dks + (int64_t)c * D + lane + 32 * u, tk[c * D + lane + 32 * u]);
+            for (int u = 0; u < kPer; ++u) atomicAdd(dks + (int64_t)c * D + lane + 32 * u, tk[c * D + lane + 32 * u]);
+        }
         if (lane == 0) atomicAdd(dbs + c, tb[c]);
     }
 }
@@ -891,13 +1024,8 @@ hils_status launch_attend_bwd(const BwdAttendArgs &a, void *ws, cudaStream_t s) 
         bwd_prep_kernel<<<(unsigned)((nq + 3) / 4), kThreads, 0, s>>>(a, w.D, w.dOb, w.Qc);
         const bool chunks = a.topk > 0 && C > 0;
         if (chunks) {
-            const int64_t ne = (int64_t)a.B * Hk * a.N * a.topk;
-            st = record_cuda_error(cudaMemsetAsync(w.count, 0, (size_t)a.B * Hk * C * sizeof(int), s));
+            st = build_index(a, w, nullptr, w.recs, w.items, w.nitems, w.max_items, s);
             if (st != HILS_OK) return st;
-            bwd_count_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.count);
-            bwd_scan_kernel<<<(unsigned)(a.B * Hk), 1024, 0, s>>>(C, w.count, w.start, w.cursor, w.items, w.nitems,
-                                                                 w.max_items);
-            bwd_scatter_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.cursor, w.entries, w.D, w.recs);
         }
         BwdTcArgs t;
         t.a = a;
@@ -928,12 +1056,8 @@ hils_status launch_attend_bwd(const BwdAttendArgs &a, void *ws, cudaStream_t s) 
         st = kernel_setup(setup_c, fc, kThreads, smem, nullptr);
         if (st != HILS_OK) return st;
         if (a.topk > 0 && C > 0) {
-            const int64_t ne = (int64_t)a.B * Hk * a.N * a.topk;
-            st = record_cuda_error(cudaMemsetAsync(w.count, 0, (size_t)a.B * Hk * C * sizeof(int), s));
+            st = build_index(a, w, w.entries, nullptr, nullptr, nullptr, 0, s);
             if (st != HILS_OK) return st;
-            bwd_count_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.count);
-            bwd_scan_kernel<<<(unsigned)(a.B * Hk), 1024, 0, s>>>(C, w.count, w.start, w.cursor, nullptr, nullptr, 0);
-            bwd_scatter_kernel<<<(unsigned)((ne + 255) / 256), 256, 0, s>>>(a, w.cursor, w.entries, nullptr, nullptr);
             if constexpr (kMma)
                 attend_bwd_mma_kernel<D, true><<<dim3(C, a.B * a.H), kThreads, smem, s>>>(a, w.D, w.start, w.entries);
             else
@@ -953,12 +1077,17 @@ template <typename T, int D>
 hils_status launch_select_bwd(const BwdSelectArgs &a, cudaStream_t s) {
     const size_t table = select_bwd_table_bytes(a.C, D);
     if (a.C > 0 && table <= (size_t)kSelBwdSmemMax) {
+        const bool stage = select_bwd_smem_bytes<T>(a.C, D, true) <= (size_t)kSelBwdSmemMax &&
+                           ((uintptr_t)a.Ksum.ptr & 15u) == 0;
+        const size_t smem = select_bwd_smem_bytes<T>(a.C, D, stage);
+        // dKsum rows start 16 (D = 128) or 8 (D = 64) bytes apart from an aligned base
+        const int vec = ((uintptr_t)a.dKsum & (D == 128 ? 15u : 7u)) == 0;
         static KernelSetup setup;
-        const hils_status st =
-            kernel_setup(setup, (const void *)select_backward_table_kernel<T, D>, kThreads, kSelBwdSmemMax, nullptr);
+        const hils_status st = kernel_setup(setup, (const void *)select_backward_table_kernel<T, D>, kSelBwdThreads,
+                                            kSelBwdSmemMax, nullptr);
         if (st != HILS_OK) return st;
         const int64_t grid = (int64_t)a.B * a.H * ((a.Lq + kSelBwdRows - 1) / kSelBwdRows);
-        select_backward_table_kernel<T, D><<<(unsigned)grid, kThreads, table, s>>>(a);
+        select_backward_table_kernel<T, D><<<(unsigned)grid, kSelBwdThreads, smem, s>>>(a, stage ? 1 : 0, vec);
         return record_cuda_error(cudaGetLastError());
     }
     select_backward_kernel<T, D><<<(unsigned)((int64_t)a.B * a.H * a.Lq), kThreads, 0, s>>>(a);

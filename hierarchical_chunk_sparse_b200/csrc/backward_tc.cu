@@ -17,12 +17,16 @@
 //   dQ = dl K                        tcgen05, M = 128 queries, N = 128 dims, K = 64 keys
 // Each step's dQ rows are added to the float32 dQ with vector atomic adds; dK^T and dV^T
 // stay in TMEM for the whole item and are added to dK and dV once at its end.
-// Warp roles (192 threads), all hand-offs through mbarriers:
-//   warps 0-3  softmax rows and the dQ, dK, dV epilogues (TMEM lane quadrant = warp);
-//   warp 4     loads: the block's K and V (TMA tiles), each step's Q and dO rows (TMA row
-//              gathers, four rows per copy, from the contiguous bf16 copies) and the rows'
-//              scalars, into a ring of two stages;
-//   warp 5     allocates TMEM and issues tcgen05.mma (one lane).
+// Warp roles (352 threads), all hand-offs through mbarriers:
+//   warps 0-7  softmax rows and the dQ, dK, dV epilogues: warp w takes the rows of TMEM
+//              lane quadrant w % 4 and half w / 4 of the keys (and of dQ's columns); the
+//              two halves of a row exchange its max and sums through shared memory;
+//   warps 8-9  loads, into a ring of two stages: the block's K and V (TMA tiles), each
+//              step's rows of Q (warp 8) and of dO (warp 9), TMA row gathers (four rows
+//              per copy) from the contiguous bf16 copies, and the rows' scalars (warp 8),
+//              loaded a step ahead;
+//   warp 10    allocates TMEM and issues tcgen05.mma (one lane), each product as soon as
+//              its inputs are ready.
 // S and T are double-buffered in TMEM, so that the products of step s+1 run while the
 // softmax of step s does. TMEM columns: S, T of buffer 0 [0, 128), of buffer 1
 // [128, 256), dK^T [256, 320), dV^T [320, 384), dQ [384, 512).
@@ -40,8 +44,8 @@ using namespace tc;
 constexpr int kQ = 128;      // queries per step (TMEM lanes)
 constexpr int kKeys = 64;    // keys per block
 constexpr int kDim = 128;    // head dimension
-constexpr int kThr = 192;
-constexpr int kLoadWarp = 4, kMmaWarp = 5;
+constexpr int kThr = 352;
+constexpr int kLoadWarp = 8, kMmaWarp = 10;  // load warps 8 (Q, scalars) and 9 (dO)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -55,22 +59,25 @@ constexpr int kDOOff = kQOff + 65536;    // dO rows, same
 constexpr int kDLOff = kDOOff + 65536;   // dl [128 queries x 64 keys] bf16
 constexpr int kCVOff = kDLOff + 16384;   // cv, same
 constexpr int kScOff = kCVOff + 16384;   // 2 stages x [128] row scalars (int4)
-constexpr int kBarOff = kScOff + 4096;   // mbarriers
+constexpr int kXOff = kScOff + 4096;    // softmax half-row exchange: [2][128] max, [2][128] (sum, o.dO)
+constexpr int kBarOff = kXOff + 3072;    // mbarriers
 constexpr int kMiscOff = kBarOff + 256;  // TMEM base, abort flag
 constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
 
 enum {
-    kBarFull = 0,     // + stage: Q, dO rows and scalars of a step landed (32 arrivals + bytes)
+    kBarFull = 0,     // + stage: Q, dO rows (bytes) and scalars (32 arrivals of warp 8) of a step landed
     kBarEmpty = 2,    // + stage: every MMA that read the stage completed
     kBarKV = 4,       // K and V of the block landed
     kBarStFull = 5,   // + buffer: S, T written
-    kBarStFree = 7,   // + buffer: the softmax warps read S, T (4 arrivals)
-    kBarDlFull = 9,   // dl, cv of the step written (4 arrivals)
+    kBarStFree = 7,   // + buffer: the softmax warps read S, T (8 arrivals)
+    kBarDlFull = 9,   // dl, cv of the step written (8 arrivals)
     kBarDqFull = 10,  // dQ of the step (and every earlier MMA) completed
-    kBarDqFree = 11,  // the softmax warps read dQ (4 arrivals)
+    kBarDqFree = 11,  // the softmax warps read dQ (8 arrivals)
     kBarDone = 12,    // every MMA of the item completed: dK^T, dV^T final
     kBarDrain = 13,   // the MMA warp's own drain
-    kNumBars = 14
+    kBarPair = 14,    // + 2 quadrant + round: the two warps of a row quadrant exchanged half-row
+                      //   maxima (round 0) or sums (round 1) (64 arrivals)
+    kNumBars = 22
 };
 
 // Four rows (y0..y3) of 64 bf16 at column x of a 2-D tensor map into 512 consecutive
@@ -82,6 +89,17 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map
         "%4, %5, %6, %7}], [%2];\n" ::"r"(dst),
         "l"(map), "r"(bar), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
         : "memory");
+}
+
+// Non-blocking test of an mbarrier phase.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
 }
 
 __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -130,7 +148,8 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
         for (int i = 0; i < kNumBars; ++i) {
             uint32_t cnt = 1;
             if (i == kBarFull || i == kBarFull + 1) cnt = 32;
-            if (i == kBarStFree || i == kBarStFree + 1 || i == kBarDlFull || i == kBarDqFree) cnt = 4;
+            if (i == kBarStFree || i == kBarStFree + 1 || i == kBarDlFull || i == kBarDqFree) cnt = 8;
+            if (i >= kBarPair) cnt = 64;
             mbar_init(bar(i), cnt);
         }
         misc[1] = 0u;
@@ -177,9 +196,10 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(barrier) : "memory");
     };
 
-    if (warp == kLoadWarp) {
+    if (warp == kLoadWarp || warp == kLoadWarp + 1) {
         // ---------------------------------------------------------------- loads
-        if (lane == 0) {
+        const int lw = warp - kLoadWarp;  // 0: Q rows and the scalars, 1: dO rows
+        if (lw == 0 && lane == 0) {
             mbar_expect_tx(bar(kBarKV), 4 * kKeys * 128);
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
@@ -189,42 +209,53 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
         }
         const int64_t row0 = (int64_t)bh * a.N;  // row of query 0 of (b, h) in the contiguous copies
         const int4 *rec = t.recs + row0 * a.topk;
+        const CUtensorMap *tm = lw == 0 ? &tmQ : &tmDO;
+        const uint32_t dst0 = sbase + (lw == 0 ? kQOff : kDOOff) + lane * 512;  // rows 4 lane .. 4 lane + 3
+        // the scalars of rows 4 lane + m of a step, as loaded (records, or lse and D_i of window
+        // queries): all four loads at once, for the next step before its stage is free
+        int4 raw[4];
+        auto load_scalars = [&](int s) {
+            const int q0 = qb + s * kQ;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int q = min(q0 + 4 * lane + m, qe - 1);
+                if (chunk) {
+                    raw[m] = __ldg(rec + q);
+                } else {
+                    raw[m] = make_int4(q, __float_as_int(__ldg(a.lse + row0 + q)), __float_as_int(__ldg(t.Dv + row0 + q)),
+                                       q);
+                }
+            }
+        };
+        load_scalars(0);
         int issued[2] = {0, 0};
         for (int s = 0; s < ns; ++s) {
             const int st = s & 1, u = s >> 1;
             if (u > 0 && !wait_warp(bar(kBarEmpty + st), (u - 1) & 1)) break;
             const int q0 = qb + s * kQ;
-            int gy[4];
+            int gy[4];  // rows in the contiguous copies (query 0's row for an unused one, read but ignored)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {  // rows 4 lane .. 4 lane + 3 of the step
-                const int r = 4 * lane + k, q = q0 + r;
-                int4 sc = make_int4(-1, 0, 0, 0);
-                if (q < qe) {
-                    if (chunk) {
-                        sc = __ldg(rec + q);
-                    } else {
-                        const float l = __ldg(a.lse + row0 + q);
-                        sc = make_int4(isfinite(l) ? q : -1, __float_as_int(l), __float_as_int(__ldg(t.Dv + row0 + q)),
-                                       q);
-                    }
-                }
-                scal[st * kQ + r] = sc;
-                gy[k] = (int)(row0 + (sc.x >= 0 ? sc.w : 0));  // an unused row reads query 0
+            for (int m = 0; m < 4; ++m) {
+                const int r = 4 * lane + m;
+                int4 sc = raw[m];
+                if (!chunk && !isfinite(__int_as_float(sc.y))) sc.x = -1;
+                if (q0 + r >= qe) sc = make_int4(-1, 0, 0, 0);
+                if (lw == 0) scal[st * kQ + r] = sc;
+                gy[m] = (int)(row0 + (sc.x >= 0 ? sc.w : 0));
             }
-            const uint32_t dq = sbase + kQOff + st * 32768 + lane * 512;
-            const uint32_t dd = sbase + kDOOff + st * 32768 + lane * 512;
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                tma_gather4(dq + x * 16384, &tmQ, bar(kBarFull + st), x * 64, gy[0], gy[1], gy[2], gy[3]);
-                tma_gather4(dd + x * 16384, &tmDO, bar(kBarFull + st), x * 64, gy[0], gy[1], gy[2], gy[3]);
+            const uint32_t dst = dst0 + st * 32768;
+            tma_gather4(dst, tm, bar(kBarFull + st), 0, gy[0], gy[1], gy[2], gy[3]);
+            tma_gather4(dst + 16384, tm, bar(kBarFull + st), 64, gy[0], gy[1], gy[2], gy[3]);
+            if (lw == 0) {  // the scalars, and the bytes of both warps' row copies
+                if (lane == 0) mbar_expect_tx(bar(kBarFull + st), 4 * kQ * 128);
+                else arrive(bar(kBarFull + st));
             }
-            if (lane == 0) mbar_expect_tx(bar(kBarFull + st), 4 * kQ * 128);
-            else arrive(bar(kBarFull + st));
             ++issued[st];
+            if (s + 1 < ns) load_scalars(s + 1);
         }
         // every copy started lands before the CTA releases its memory
         if (lane == 0) {
-            drain_wait(bar(kBarKV), 0);
+            if (lw == 0) drain_wait(bar(kBarKV), 0);
             for (int st = 0; st < 2; ++st)
                 if (issued[st] > 0) drain_wait(bar(kBarFull + st), (uint32_t)(issued[st] - 1) & 1u);
         }
@@ -248,46 +279,74 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
             }
             mma_commit(bar(kBarStFull + st));
         };
-        bool ok = wait_warp(bar(kBarKV), 0) && wait_warp(bar(kBarFull), 0);
-        if (ok) {
-            tc_fence_after();
-            if (lane == 0) issue_st(0);
-            __syncwarp();
-        }
-        for (int s = 0; s < ns && ok; ++s) {
+        auto issue_kv = [&](int s) {  // dK^T += Q^T dl, dV^T += dO^T cv: 16 queries per MMA
             const int st = s & 1;
-            if (s + 1 < ns) {  // S, T of the next step, into the other buffer
-                const int s1 = s + 1, st1 = s1 & 1;
-                if (!(ok = wait_warp(bar(kBarFull + st1), (s1 >> 1) & 1))) break;
-                if (s1 >= 2 && !(ok = wait_warp(bar(kBarStFree + st1), ((s1 >> 1) - 1) & 1))) break;
+#pragma unroll
+            for (int ks = 0; ks < kQ / 16; ++ks) {
+                const uint32_t ro = st * 32768 + ks * 2048;
+                mma_ss(tmem + 256, smem_desc(sbase + kQOff + ro, 16384, 1024),
+                       smem_desc(sbase + kDLOff + ks * 2048, 8192, 1024), idKV, (s > 0 || ks > 0) ? 1u : 0u);
+                mma_ss(tmem + 320, smem_desc(sbase + kDOOff + ro, 16384, 1024),
+                       smem_desc(sbase + kCVOff + ks * 2048, 8192, 1024), idKV, (s > 0 || ks > 0) ? 1u : 0u);
+            }
+            mma_commit(bar(kBarEmpty + st));  // the last reads of the stage's Q and dO rows
+        };
+        auto issue_dq = [&]() {  // dQ = dl K: 16 keys per MMA
+#pragma unroll
+            for (int ks = 0; ks < kKeys / 16; ++ks)
+                mma_ss(tmem + 384, smem_desc(sbase + kDLOff + ks * 32, 16, 1024),
+                       smem_desc(sbase + kKOff + ks * 2048, 8192, 1024), idQ, ks > 0 ? 1u : 0u);
+            mma_commit(bar(kBarDqFull));
+        };
+        // Issue each product as soon as its inputs are ready, earliest step first within a
+        // kind, S/T ahead of the rest: S, T of step n need its rows (full) and their TMEM
+        // buffer read (the softmax of step n - 2); dK, dV of step k need dl, cv of k; dQ of
+        // step k needs dK, dV of k issued and dQ of k - 1 read. Every test is a
+        // non-blocking look at a phase whose predecessor this warp has already seen.
+        bool ok = wait_warp(bar(kBarKV), 0);
+        int nS = 0, nK = 0, nQ = 0;
+        uint64_t idle_since = 0;
+        int idle = 0;
+        while (ok && nQ < ns) {
+            bool ready = false;
+            int kind = -1;
+            if (lane == 0) {
+                if (nS < ns && mbar_test(bar(kBarFull + (nS & 1)), (nS >> 1) & 1) &&
+                    (nS < 2 || mbar_test(bar(kBarStFree + (nS & 1)), ((nS >> 1) - 1) & 1)))
+                    kind = 0;
+                else if (nK < nS && mbar_test(bar(kBarDlFull), nK & 1))
+                    kind = 1;
+                else if (nQ < nK && (nQ == 0 || mbar_test(bar(kBarDqFree), (nQ - 1) & 1)))
+                    kind = 2;
+            }
+            kind = __shfl_sync(kFull, kind, 0);
+            ready = kind >= 0;
+            if (ready) {
                 tc_fence_after();
-                if (lane == 0) issue_st(s1);
-                __syncwarp();
-            }
-            if (!(ok = wait_warp(bar(kBarDlFull), s & 1))) break;
-            tc_fence_after();
-            if (lane == 0) {  // dK^T += Q^T dl, dV^T += dO^T cv: 16 queries per MMA
-#pragma unroll
-                for (int ks = 0; ks < kQ / 16; ++ks) {
-                    const uint32_t ro = st * 32768 + ks * 2048;
-                    mma_ss(tmem + 256, smem_desc(sbase + kQOff + ro, 16384, 1024),
-                           smem_desc(sbase + kDLOff + ks * 2048, 8192, 1024), idKV, (s > 0 || ks > 0) ? 1u : 0u);
-                    mma_ss(tmem + 320, smem_desc(sbase + kDOOff + ro, 16384, 1024),
-                           smem_desc(sbase + kCVOff + ks * 2048, 8192, 1024), idKV, (s > 0 || ks > 0) ? 1u : 0u);
+                if (lane == 0) {
+                    if (kind == 0) issue_st(nS);
+                    else if (kind == 1) issue_kv(nK);
+                    else issue_dq();
                 }
+                __syncwarp();
+                if (kind == 0) ++nS;
+                else if (kind == 1) ++nK;
+                else ++nQ;
+                idle = 0;
+                continue;
             }
-            __syncwarp();
-            if (s > 0 && !(ok = wait_warp(bar(kBarDqFree), (s - 1) & 1))) break;
-            tc_fence_after();
-            if (lane == 0) {  // dQ = dl K: 16 keys per MMA
-#pragma unroll
-                for (int ks = 0; ks < kKeys / 16; ++ks)
-                    mma_ss(tmem + 384, smem_desc(sbase + kDLOff + ks * 32, 16, 1024),
-                           smem_desc(sbase + kKOff + ks * 2048, 8192, 1024), idQ, ks > 0 ? 1u : 0u);
-                mma_commit(bar(kBarDqFull));
-                mma_commit(bar(kBarEmpty + st));
+            // nothing ready: bounded like every other wait
+            __nanosleep(32);
+            if (idle == 0) idle_since = global_ns();
+            if ((++idle & 15) == 0 || a.wait_ns <= 0) {
+                bool stop = *abort_flag != 0u;
+                if (!stop && (a.wait_ns <= 0 || (long long)(global_ns() - idle_since) > a.wait_ns)) {
+                    *abort_flag = 1u;
+                    atomicOr(t.status, 1u);
+                    stop = true;
+                }
+                ok = !__any_sync(kFull, stop);
             }
-            __syncwarp();
         }
         if (lane == 0) {
             if (ok) mma_commit(bar(kBarDone));
@@ -298,18 +357,30 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- softmax rows
-        const int r = warp * 32 + lane;  // query row of the step = TMEM lane
-        const uint32_t lb = (uint32_t)(warp * 32) << 16;
+        // warp w: rows r = 32 (w % 4) + lane (its TMEM lane quadrant), half g = w / 4 of the
+        // keys (columns 32 g .. 32 g + 31 of S and T) and of dQ's columns (64 g .. 64 g + 63);
+        // the two halves of a row meet through shared memory (row max, then sum and o_c . dO)
+        const int g = warp >> 2, quad = warp & 3;
+        const int r = quad * 32 + lane;  // query row of the step = TMEM lane
+        const uint32_t lb = (uint32_t)(quad * 32) << 16;
         const float sl2 = a.scale * kLog2e;
         const int K = a.topk;
+        float *xm = reinterpret_cast<float *>(smem + kXOff);        // [2][128] half-row maxima
+        float2 *xz = reinterpret_cast<float2 *>(smem + kXOff + 1024);  // [2][128] half-row sum, o_c . dO
+        // the two warps of a row quadrant (quad and quad + 4) meet on mbarrier kBarPair + 2
+        // quad + round (64 arrivals, one phase per step), a bounded wait like every other
+        auto pair_sync = [&](int round, int s) -> bool {
+            arrive(bar(kBarPair + 2 * quad + round));
+            return wait_warp(bar(kBarPair + 2 * quad + round), s & 1);
+        };
         int prev = -1;  // query of this row in the previous step (its dQ row), or -1
-        // this row's dQ of the last completed step into the global dQ
+        // this row's half of the dQ of the last completed step into the global dQ
         auto dq_out = [&](int qrow) {
-            float *dst = a.dQ + ((int64_t)bh * a.N + (qrow < 0 ? 0 : qrow)) * kDim;
+            float *dst = a.dQ + ((int64_t)bh * a.N + (qrow < 0 ? 0 : qrow)) * kDim + g * 64;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t v[32];
-                tmem_ld32(tmem + lb + 384 + c * 32, v);
+                tmem_ld32(tmem + lb + 384 + g * 64 + c * 32, v);
                 tmem_wait_ld();
                 if (qrow >= 0) {
                     if (t.vec_ok) {
@@ -333,11 +404,9 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
             const int st = s & 1;
             if (!(ok = wait_warp(bar(kBarStFull + st), (s >> 1) & 1))) break;
             tc_fence_after();
-            uint32_t s0[32], s1[32], t0[32], t1[32];
-            tmem_ld32(tmem + lb + st * 128, s0);
-            tmem_ld32(tmem + lb + st * 128 + 32, s1);
-            tmem_ld32(tmem + lb + st * 128 + 64, t0);
-            tmem_ld32(tmem + lb + st * 128 + 96, t1);
+            uint32_t sv[32], tv[32];
+            tmem_ld32(tmem + lb + st * 128 + g * 32, sv);
+            tmem_ld32(tmem + lb + st * 128 + 64 + g * 32, tv);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -345,46 +414,49 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
             const int4 sc = scal[st * kQ + r];
             const int en = sc.x, qi = sc.w;
             const float wl = __int_as_float(sc.y), Dd = __int_as_float(sc.z);
-            auto S = [&](int j) { return __uint_as_float(j < 32 ? s0[j] : s1[j - 32]); };
-            auto T = [&](int j) { return __uint_as_float(j < 32 ? t0[j] : t1[j - 32]); };
-            uint32_t dlp[32], cvp[32];  // bf16 pairs of keys 2p, 2p + 1
-            if (en < 0) {
-#pragma unroll
-                for (int p = 0; p < 32; ++p) dlp[p] = cvp[p] = 0u;
-            } else if (chunk) {
+            auto S = [&](int j) { return __uint_as_float(sv[j]); };
+            auto T = [&](int j) { return __uint_as_float(tv[j]); };
+            uint32_t dlp[16], cvp[16];  // bf16 pairs of keys 32 g + 2 p, + 1
+            if (chunk) {
                 // p_j = softmax over the chunk of scale S_j; o_c . dO = sum_j p_j T_j;
                 // dl_j = w p_j (T_j - o_c . dO), cv_j = w p_j; dscore = w (o_c . dO - D_i)
-                float m = S(0);
+                float mx[4] = {S(0), S(1), S(2), S(3)};
 #pragma unroll
-                for (int j = 1; j < kKeys; ++j) m = fmaxf(m, S(j));
-                float e[kKeys], z = 0.f, oc = 0.f;
+                for (int j = 4; j < 32; ++j) mx[j & 3] = fmaxf(mx[j & 3], S(j));
+                xm[g * kQ + r] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                if (!(ok = pair_sync(0, s))) break;
+                const float ms = fmaxf(xm[r], xm[kQ + r]) * sl2;
+                float e[32], zp[4] = {0.f, 0.f, 0.f, 0.f}, op[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int j = 0; j < kKeys; ++j) {
-                    e[j] = ex2((S(j) - m) * sl2);
-                    z += e[j];
-                    oc = fmaf(e[j], T(j), oc);
+                for (int j = 0; j < 32; ++j) {
+                    e[j] = ex2(fmaf(S(j), sl2, -ms));
+                    zp[j & 3] += e[j];
+                    op[j & 3] = fmaf(e[j], T(j), op[j & 3]);
                 }
-                const float inv = 1.f / z;
-                oc *= inv;
-                const float wc = wl * inv;
+                xz[g * kQ + r] = make_float2((zp[0] + zp[1]) + (zp[2] + zp[3]), (op[0] + op[1]) + (op[2] + op[3]));
+                if (!(ok = pair_sync(1, s))) break;
+                const float2 z0 = xz[r], z1 = xz[kQ + r];
+                const float inv = 1.f / (z0.x + z1.x);
+                const float oc = (z0.y + z1.y) * inv;
+                const float wc = en >= 0 ? wl * inv : 0.f;
 #pragma unroll
-                for (int p = 0; p < 32; ++p) {
+                for (int p = 0; p < 16; ++p) {
                     const float c0 = wc * e[2 * p], c1 = wc * e[2 * p + 1];
                     cvp[p] = pack_bf16(c0, c1);
                     dlp[p] = pack_bf16(a.scale * c0 * (T(2 * p) - oc), a.scale * c1 * (T(2 * p + 1) - oc));
                 }
-                a.dscore[((int64_t)bh * a.N + qi) * K + (en & 31)] = wl * (oc - Dd);
+                if (g == 0 && en >= 0) a.dscore[((int64_t)bh * a.N + qi) * K + (en & 31)] = wl * (oc - Dd);
             } else {
                 // window key j0 + j of query qi: c_j = exp(scale S_j - lse), dl_j = c_j (T_j - D_i)
                 const float l2 = wl * kLog2e;
 #pragma unroll
-                for (int p = 0; p < 32; ++p) {
+                for (int p = 0; p < 16; ++p) {
                     float c[2];
 #pragma unroll
                     for (int hv = 0; hv < 2; ++hv) {
-                        const int j = 2 * p + hv, key = j0 + j;
-                        const bool in = j < rows && key <= qi && key > qi - a.W;
-                        c[hv] = in ? ex2(fmaf(S(j), sl2, -l2)) : 0.f;
+                        const int j = 32 * g + 2 * p + hv, key = j0 + j;
+                        const bool in = en >= 0 && j < rows && key <= qi && key > qi - a.W;
+                        c[hv] = in ? ex2(fmaf(S(2 * p + hv), sl2, -l2)) : 0.f;
                     }
                     cvp[p] = pack_bf16(c[0], c[1]);
                     dlp[p] = pack_bf16(a.scale * c[0] * (T(2 * p) - Dd), a.scale * c[1] * (T(2 * p + 1) - Dd));
@@ -397,8 +469,8 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
             }
             uint8_t *dlrow = smem + kDLOff + r * 128, *cvrow = smem + kCVOff + r * 128;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int o = (u ^ (r & 7)) << 4;
+            for (int u = 0; u < 4; ++u) {  // 16-byte units 4 g + u of the row (keys 32 g + 8 u ..)
+                const int o = ((4 * g + u) ^ (r & 7)) << 4;
                 *reinterpret_cast<uint4 *>(dlrow + o) = make_uint4(dlp[4 * u], dlp[4 * u + 1], dlp[4 * u + 2], dlp[4 * u + 3]);
                 *reinterpret_cast<uint4 *>(cvrow + o) = make_uint4(cvp[4 * u], cvp[4 * u + 1], cvp[4 * u + 2], cvp[4 * u + 3]);
             }
@@ -414,25 +486,22 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
         } else {
             ok = false;
         }
-        // dK^T and dV^T: row r of TMEM is dimension x = r; key j in column j
+        // dK^T and dV^T: row r of TMEM is dimension x = r; key j in column j (this warp's half)
         if (ok && wait_warp(bar(kBarDone), 0)) {
             tc_fence_after();
             const int64_t kvrow = ((int64_t)b * Hk + hk) * a.N + j0;
             float *dk = a.dK + kvrow * kDim + r;
             float *dv = a.dV + kvrow * kDim + r;
+            uint32_t vk[32], vv[32];
+            tmem_ld32(tmem + lb + 256 + g * 32, vk);
+            tmem_ld32(tmem + lb + 320 + g * 32, vv);
+            tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t vk[32], vv[32];
-                tmem_ld32(tmem + lb + 256 + c * 32, vk);
-                tmem_ld32(tmem + lb + 320 + c * 32, vv);
-                tmem_wait_ld();
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const int j = c * 32 + u;
-                    if (j < rows) {
-                        atomicAdd(dk + (int64_t)j * kDim, __uint_as_float(vk[u]));
-                        atomicAdd(dv + (int64_t)j * kDim, __uint_as_float(vv[u]));
-                    }
+            for (int u = 0; u < 32; ++u) {
+                const int j = g * 32 + u;
+                if (j < rows) {
+                    atomicAdd(dk + (int64_t)j * kDim, __uint_as_float(vk[u]));
+                    atomicAdd(dv + (int64_t)j * kDim, __uint_as_float(vv[u]));
                 }
             }
         }
