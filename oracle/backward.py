@@ -60,9 +60,14 @@ def forward(Q, K, V, Qcal, LQ, idx, nsel, S: int, W: int, scale: float, rows=Non
     nsel_h = nsel.repeat_interleave(G, dim=1)
     kept = (torch.arange(Kk).view(1, 1, 1, Kk) < nsel_h.unsqueeze(-1)) & (idx_h >= 0)
     cidx = idx_h.clamp(min=0, max=max(C - 1, 0))
+    # slots that are not kept still gather (their values are masked below): with no
+    # complete chunk (C = 0) nothing can be kept, and one zero row keeps those gathers in
+    # range
+    Kg = torch.cat([Ksum, Ksum.new_zeros(B, H, 1, d)], dim=2) if C == 0 else Ksum
+    Bg = torch.cat([Bsum, Bsum.new_zeros(B, H, 1)], dim=2) if C == 0 else Bsum
     # Eq. 7: s^ = scale q~ . k'_c + b'_c of each kept chunk
-    ks = torch.gather(Ksum, 2, cidx.reshape(B, H, R * Kk, 1).expand(B, H, R * Kk, d)).reshape(B, H, R, Kk, d)
-    bs = torch.gather(Bsum, 2, cidx.reshape(B, H, R * Kk)).reshape(B, H, R, Kk)
+    ks = torch.gather(Kg, 2, cidx.reshape(B, H, R * Kk, 1).expand(B, H, R * Kk, d)).reshape(B, H, R, Kk, d)
+    bs = torch.gather(Bg, 2, cidx.reshape(B, H, R * Kk)).reshape(B, H, R, Kk)
     score = scale * torch.einsum("bhnd,bhnkd->bhnk", Qcr, ks) + bs
     score = torch.where(kept, score, torch.full_like(score, -torch.inf))
     # token logits and the sliding window [max(0, i-W+1), i]
@@ -74,7 +79,8 @@ def forward(Q, K, V, Qcal, LQ, idx, nsel, S: int, W: int, scale: float, rows=Non
     win = (j <= i) & (j > i - W)
     Lw = torch.where(win, L, torch.full_like(L, -torch.inf))
     # each kept chunk's own softmax output o_c over its S tokens
-    tok = cidx.unsqueeze(-1) * S + torch.arange(S).view(1, 1, 1, 1, S)  # [B,H,R,Kk,S]
+    # [B,H,R,Kk,S]; a kept chunk's tokens are all < C S <= N, the clamp only touches masked slots
+    tok = (cidx.unsqueeze(-1) * S + torch.arange(S).view(1, 1, 1, 1, S)).clamp(max=N - 1)
     Lc = torch.gather(L, 3, tok.reshape(B, H, R, Kk * S)).reshape(B, H, R, Kk, S)
     pc = torch.softmax(Lc, dim=-1)
     Vc = Vh[torch.arange(B).view(B, 1, 1, 1, 1), torch.arange(H).view(1, H, 1, 1, 1), tok]  # [B,H,R,Kk,S,d]
