@@ -778,77 +778,71 @@ __global__ void __launch_bounds__(kThreads) attend_bwd_mma_kernel(BwdAttendArgs 
         }
 }
 
-// grid: B*H*Lq, one query each: Eq. 7 backward.
-template <typename T, int D>
-__global__ void __launch_bounds__(kThreads) select_backward_kernel(BwdSelectArgs a) {
-    const int tid = threadIdx.x;
-    const int64_t qi = blockIdx.x;
-    const int i = (int)(qi % a.Lq);
-    const int h = (int)((qi / a.Lq) % a.H);
-    const int b = (int)(qi / ((int64_t)a.Lq * a.H));
-    const int Hk = a.H / a.G;
-    const int64_t qg = ((int64_t)b * Hk + h / a.G) * a.Lq + i;
-    const int K = a.topk;
-    const int ns = K > 0 ? min(max(a.nsel[qg], 0), K) : 0;
-    const T *qrow = static_cast<const T *>(a.Qcal.ptr) + b * a.Qcal.sb + h * a.Qcal.sh + (int64_t)i * a.Qcal.st;
-    const T *khead = static_cast<const T *>(a.Ksum.ptr) + b * a.Ksum.sb + h * a.Ksum.sh;
-    float *dks = a.dKsum + ((int64_t)b * a.H + h) * a.C * D;
-    float *dbs = a.dBsum + ((int64_t)b * a.H + h) * a.C;
-    if (tid >= D) return;
-    const float qx = elem(qrow, tid);
-    float acc = 0.f;
-    for (int k = 0; k < ns; ++k) {
-        const int c = a.idx[qg * K + k];
-        const float ds = a.dscore[qi * K + k];
-        acc = fmaf(ds, elem(khead + (int64_t)c * a.Ksum.st, tid), acc);
-        atomicAdd(dks + (int64_t)c * D + tid, a.scale * ds * qx);
-        if (tid == 0) atomicAdd(dbs + c, ds);
-    }
-    a.dQcal[qi * D + tid] = a.scale * acc;
-}
-
-// Eq. 7 backward with the chunk sums kept in shared memory: a CTA takes kSelBwdRows
-// consecutive queries of one (b, h), a warp one query at a time, adds scale ds q~ into
-// its own [C][D] table (and ds into [C]) with shared-memory atomics, writes dQcal, and
-// then adds each table row that a kept chunk touched to dKsum and dBsum once (vector
-// atomics when dKsum is 16-byte aligned). Adjacent queries keep mostly the same chunks,
-// so the global atomics drop from one per (query, kept chunk, x) to about one per (CTA,
-// touched chunk, x). When it fits, the head's k' table is first copied into shared
-// memory, so that a query's kept rows are read there, not from L2; each warp loads the
-// next query's kept list before working on the current one. Used when the tables fit.
+// Eq. 7 backward, a CTA per kSelBwdRows consecutive queries of one (b, h):
+//   1. dQcal = scale sum_k ds_k k'_{c_k}, a warp per query, the k' rows read from a copy
+//      of the head's table in shared memory (or from global memory when it does not
+//      fit); the kept entries are counted per chunk meanwhile;
+//   2. the entries are sorted by chunk in shared memory (counting sort: a scan of the
+//      counts, then each entry's slot from a cursor), as (query, ds) pairs;
+//   3. warp w sums the entries of chunks c = w (mod 8) in registers, scale ds q~ over the
+//      chunk's queries (eight q~ rows in flight) and ds for b', and adds the sums to dKsum
+//      and dBsum once per (CTA, chunk) (vector atomics when dKsum is aligned).
+// Used when the k' copy, the counts and the entries fit in shared memory.
 constexpr int kSelBwdRows = 256;
 constexpr int kSelBwdThreads = 256;
+constexpr int kSelBwdWarps = kSelBwdThreads / 32;
 constexpr int kSelBwdSmemMax = 200 * 1024;
 
-__host__ __device__ inline size_t select_bwd_table_bytes(int C, int D) {
-    return ((size_t)C * D * 4 + (size_t)C * 4 + (size_t)((C + 31) / 32) * 4 + 15) & ~(size_t)15;
+// shared memory of the table kernel: counts / cursors [C], starts [C + 1], entries
+// [kSelBwdRows * K] (query, ds), then (stage) the k' table [C][D]
+__host__ __device__ inline size_t select_bwd_sort_bytes(int C, int K) {
+    return ((size_t)(2 * C + 1) * 4 + 15) / 16 * 16 + (size_t)kSelBwdRows * (K > 0 ? K : 1) * 8;
 }
 template <typename T>
-inline size_t select_bwd_smem_bytes(int C, int D, bool stage) {
-    return select_bwd_table_bytes(C, D) + (stage ? (size_t)C * D * sizeof(T) : 0);
+inline size_t select_bwd_smem_bytes(int C, int D, int K, bool stage) {
+    return select_bwd_sort_bytes(C, K) + (stage ? (size_t)C * D * sizeof(T) : 0);
+}
+
+// E consecutive elements of a T row starting at element x, as floats (one vector load)
+template <int E>
+__device__ __forceinline__ void load_run(const bf16 *p, int x, float (&v)[E]) {
+    if constexpr (E == 4) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p + x);
+        v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+    } else {
+        const uint32_t u = *reinterpret_cast<const uint32_t *>(p + x);
+        v[0] = bf16lo(u); v[1] = bf16hi(u);
+    }
+}
+template <int E>
+__device__ __forceinline__ void load_run(const float *p, int x, float (&v)[E]) {
+    if constexpr (E == 4) {
+        const float4 u = *reinterpret_cast<const float4 *>(p + x);
+        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+    } else {
+        const float2 u = *reinterpret_cast<const float2 *>(p + x);
+        v[0] = u.x; v[1] = u.y;
+    }
 }
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kSelBwdThreads) select_backward_table_kernel(BwdSelectArgs a, int stage, int vec) {
-    extern __shared__ __align__(16) float tsm[];
-    constexpr int kPer = D / 32;  // elements of a row per lane
-    constexpr int kWarps = kSelBwdThreads / 32;
-    const int C = a.C;
-    float *tk = tsm;                                           // [C][D]
-    float *tb = tk + (int64_t)C * D;                           // [C]
-    unsigned *touched = reinterpret_cast<unsigned *>(tb + C);  // C bits
-    T *ks = reinterpret_cast<T *>(reinterpret_cast<uint8_t *>(tsm) + select_bwd_table_bytes(C, D));  // [C][D]
+    extern __shared__ __align__(16) uint8_t ssm[];
+    constexpr int kE = D / 32;  // consecutive elements of a row per lane: 4 (D = 128) or 2
+    const int C = a.C, K = a.topk;
+    int *cnt = reinterpret_cast<int *>(ssm);  // [C] counts, then cursors
+    int *off = cnt + C;                       // [C + 1] starts
+    int2 *ent = reinterpret_cast<int2 *>(ssm + ((size_t)(2 * C + 1) * 4 + 15) / 16 * 16);  // (query, ds)
+    T *ks = reinterpret_cast<T *>(ssm + select_bwd_sort_bytes(C, K));                        // [C][D]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nblk = (a.Lq + kSelBwdRows - 1) / kSelBwdRows;
     const int64_t bh = blockIdx.x / nblk;
     const int i0 = (int)(blockIdx.x % nblk) * kSelBwdRows;
     const int h = (int)(bh % a.H), b = (int)(bh / a.H);
     const int Hk = a.H / a.G;
-    const int K = a.topk;
     const T *khead = static_cast<const T *>(a.Ksum.ptr) + b * a.Ksum.sb + h * a.Ksum.sh;
-    for (int e = tid; e < C * D; e += kSelBwdThreads) tk[e] = 0.f;
-    for (int e = tid; e < C; e += kSelBwdThreads) tb[e] = 0.f;
-    for (int e = tid; e < (C + 31) / 32; e += kSelBwdThreads) touched[e] = 0u;
+    const T *qhead = static_cast<const T *>(a.Qcal.ptr) + b * a.Qcal.sb + h * a.Qcal.sh;
+    for (int e = tid; e < C; e += kSelBwdThreads) cnt[e] = 0;
     if (stage) {  // the head's k' rows, 16 bytes per copy
         constexpr int kU = D * (int)sizeof(T) / 16;  // 16-byte units per row
         for (int e = tid; e < C * kU; e += kSelBwdThreads) {
@@ -861,73 +855,110 @@ __global__ void __launch_bounds__(kSelBwdThreads) select_backward_table_kernel(B
     const T *kbase = stage ? ks : khead;
     const int64_t kst = stage ? D : a.Ksum.st;
     const int iend = min(a.Lq, i0 + kSelBwdRows);
-    // lane k holds kept chunk k's index and gradient (K <= 32)
-    auto load_list = [&](int i, int &c, float &ds, int &ns) {
-        ns = 0;
-        c = 0;
+    // lane k < K: kept chunk k's index and gradient (c = -1 when not kept)
+    auto load_list = [&](int i, int &c, float &ds) {
+        c = -1;
         ds = 0.f;
-        if (i >= iend) return;
-        const int64_t qi = bh * a.Lq + i;
+        if (i >= iend || lane >= K) return;
         const int64_t qg = ((int64_t)b * Hk + h / a.G) * a.Lq + i;
-        ns = K > 0 ? min(max(a.nsel[qg], 0), K) : 0;
-        if (lane < K) {
-            const int cc = a.idx[qg * K + lane];
-            const float d = a.dscore[qi * K + lane];
-            const bool ok = lane < ns && (unsigned)cc < (unsigned)C;
-            c = ok ? cc : 0;
-            ds = ok ? d : 0.f;
+        const int ns = min(max(__ldg(&a.nsel[qg]), 0), K);
+        const int cc = __ldg(&a.idx[qg * K + lane]);
+        const float d = __ldg(&a.dscore[(bh * a.Lq + i) * K + lane]);
+        if (lane < ns && (unsigned)cc < (unsigned)C) {
+            c = cc;
+            ds = d;
         }
     };
-    int myc, ns;
-    float myds;
-    load_list(i0 + warp, myc, myds, ns);
-    for (int i = i0 + warp; i < iend; i += kWarps) {
-        int nc, nn;
-        float nd;
-        load_list(i + kWarps, nc, nd, nn);  // the next query's list, in flight meanwhile
-        const int64_t qi = bh * a.Lq + i;
-        const T *qrow = static_cast<const T *>(a.Qcal.ptr) + b * a.Qcal.sb + h * a.Qcal.sh + (int64_t)i * a.Qcal.st;
-        if (lane < ns && myds != 0.f) atomicOr(&touched[myc >> 5], 1u << (myc & 31));
-        float qx[kPer], acc[kPer];
+    // ---- 1. dQcal, a warp per query; counts per chunk
+    {
+        int myc, nc;
+        float myds, nd;
+        load_list(i0 + warp, myc, myds);
+        for (int i = i0 + warp; i < iend; i += kSelBwdWarps) {
+            load_list(i + kSelBwdWarps, nc, nd);  // the next query's list, in flight meanwhile
+            if (myc >= 0) atomicAdd(&cnt[myc], 1);
+            float acc[kE] = {};
+            unsigned m = __ballot_sync(kFull, myc >= 0);
+            while (m) {
+                const int k = __ffs(m) - 1;
+                m &= m - 1;
+                const int c = __shfl_sync(kFull, myc, k);
+                const float ds = __shfl_sync(kFull, myds, k);
+                float kv[kE];
+                load_run<kE>(kbase + (int64_t)c * kst, kE * lane, kv);
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-            qx[u] = a.scale * elem(qrow, lane + 32 * u);
-            acc[u] = 0.f;
-        }
-#pragma unroll 4
-        for (int k = 0; k < ns; ++k) {
-            const int c = __shfl_sync(kFull, myc, k);
-            const float ds = __shfl_sync(kFull, myds, k);
-            const T *krow = kbase + (int64_t)c * kst;
-#pragma unroll
-            for (int u = 0; u < kPer; ++u) {
-                acc[u] = fmaf(ds, elem(krow, lane + 32 * u), acc[u]);
-                atomicAdd(&tk[c * D + lane + 32 * u], ds * qx[u]);
+                for (int u = 0; u < kE; ++u) acc[u] = fmaf(ds, kv[u], acc[u]);
             }
-        }
-        if (lane < ns) atomicAdd(&tb[myc], myds);
+            float *dq = a.dQcal + (bh * a.Lq + i) * D + kE * lane;
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) a.dQcal[qi * D + lane + 32 * u] = a.scale * acc[u];
-        myc = nc;
-        myds = nd;
-        ns = nn;
+            for (int u = 0; u < kE; ++u) dq[u] = a.scale * acc[u];
+            myc = nc;
+            myds = nd;
+        }
     }
     __syncthreads();
+    // ---- 2. starts (exclusive scan of the counts, warp 0), cursors, then each entry's slot
+    if (warp == 0) {
+        int run = 0;
+        for (int c0 = 0; c0 < C; c0 += 32) {
+            const int c = c0 + lane;
+            const int v = c < C ? cnt[c] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += u;
+            }
+            if (c < C) {
+                off[c] = run + incl - v;
+                cnt[c] = run + incl - v;
+            }
+            run += __shfl_sync(kFull, incl, 31);
+        }
+        if (lane == 0) off[C] = run;
+    }
+    __syncthreads();
+    for (int i = i0 + warp; i < iend; i += kSelBwdWarps) {
+        int c;
+        float ds;
+        load_list(i, c, ds);
+        if (c >= 0) ent[atomicAdd(&cnt[c], 1)] = make_int2(i, __float_as_int(ds));
+    }
+    __syncthreads();
+    // ---- 3. chunk sums of this warp's chunks, in registers
     float *dks = a.dKsum + bh * C * D;
     float *dbs = a.dBsum + bh * C;
-    for (int c = warp; c < C; c += kWarps) {
-        if (!((touched[c >> 5] >> (c & 31)) & 1u)) continue;
-        if (vec && D == 128) {  // lane l: elements 4 l .. 4 l + 3
-            const float4 v = *reinterpret_cast<const float4 *>(&tk[c * D + 4 * lane]);
-            atomicAdd(reinterpret_cast<float4 *>(dks + (int64_t)c * D + 4 * lane), v);
-        } else if (vec) {  // D = 64: lane l: elements 2 l, 2 l + 1
-            const float2 v = *reinterpret_cast<const float2 *>(&tk[c * D + 2 * lane]);
-            atomicAdd(reinterpret_cast<float2 *>(dks + (int64_t)c * D + 2 * lane), v);
+    for (int c = warp; c < C; c += kSelBwdWarps) {
+        const int e0 = off[c], e1 = off[c + 1];
+        if (e0 == e1) continue;
+        float acc[kE] = {};
+        float db = 0.f;
+        for (int e = e0; e < e1; e += 8) {
+            float q[8][kE], dsv[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {  // eight rows in flight
+                const int2 en = ent[min(e + k, e1 - 1)];
+                dsv[k] = e + k < e1 ? __int_as_float(en.y) : 0.f;
+                load_run<kE>(qhead + (int64_t)en.x * a.Qcal.st, kE * lane, q[k]);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                db += dsv[k];
+#pragma unroll
+                for (int u = 0; u < kE; ++u) acc[u] = fmaf(dsv[k], q[k][u], acc[u]);
+            }
+        }
+        float *dst = dks + (int64_t)c * D + kE * lane;
+#pragma unroll
+        for (int u = 0; u < kE; ++u) acc[u] *= a.scale;
+        if (vec) {
+            if constexpr (kE == 4) atomicAdd(reinterpret_cast<float4 *>(dst), make_float4(acc[0], acc[1], acc[2], acc[3]));
+            else atomicAdd(reinterpret_cast<float2 *>(dst), make_float2(acc[0], acc[1]));
         } else {
 #pragma unroll
-            for (int u = 0; u < kPer; ++u) atomicAdd(dks + (int64_t)c * D + lane + 32 * u, tk[c * D + lane + 32 * u]);
+            for (int u = 0; u < kE; ++u) atomicAdd(dst + u, acc[u]);
         }
-        if (lane == 0) atomicAdd(dbs + c, tb[c]);
+        if (lane == 0) atomicAdd(dbs + c, db);
     }
 }
 
@@ -1075,11 +1106,11 @@ hils_status launch_attend_bwd(const BwdAttendArgs &a, void *ws, cudaStream_t s) 
 
 template <typename T, int D>
 hils_status launch_select_bwd(const BwdSelectArgs &a, cudaStream_t s) {
-    const size_t table = select_bwd_table_bytes(a.C, D);
-    if (a.C > 0 && table <= (size_t)kSelBwdSmemMax) {
-        const bool stage = select_bwd_smem_bytes<T>(a.C, D, true) <= (size_t)kSelBwdSmemMax &&
-                           ((uintptr_t)a.Ksum.ptr & 15u) == 0;
-        const size_t smem = select_bwd_smem_bytes<T>(a.C, D, stage);
+    // the per-chunk counts and starts and the CTA's entries must fit in shared memory:
+    // C up to about 21,000 chunks (1.3M tokens) at K = 16
+    if (a.C > 0 && select_bwd_smem_bytes<T>(a.C, D, a.topk, false) <= (size_t)kSelBwdSmemMax) {
+        const bool stage = select_bwd_smem_bytes<T>(a.C, D, a.topk, true) <= (size_t)kSelBwdSmemMax;
+        const size_t smem = select_bwd_smem_bytes<T>(a.C, D, a.topk, stage);
         // dKsum rows start 16 (D = 128) or 8 (D = 64) bytes apart from an aligned base
         const int vec = ((uintptr_t)a.dKsum & (D == 128 ? 15u : 7u)) == 0;
         static KernelSetup setup;
@@ -1090,8 +1121,9 @@ hils_status launch_select_bwd(const BwdSelectArgs &a, cudaStream_t s) {
         select_backward_table_kernel<T, D><<<(unsigned)grid, kSelBwdThreads, smem, s>>>(a, stage ? 1 : 0, vec);
         return record_cuda_error(cudaGetLastError());
     }
-    select_backward_kernel<T, D><<<(unsigned)((int64_t)a.B * a.H * a.Lq), kThreads, 0, s>>>(a);
-    return record_cuda_error(cudaGetLastError());
+    if (a.C > 0) return HILS_ERR_UNSUPPORTED;
+    // no summarised chunk: nothing was kept, dQcal is zero
+    return record_cuda_error(cudaMemsetAsync(a.dQcal, 0, (size_t)a.B * a.H * a.Lq * D * sizeof(float), s));
 }
 
 template <typename T, int D>

@@ -81,7 +81,8 @@ typedef enum { HILS_F32 = 0, HILS_BF16 = 1 } hils_dtype;
 typedef enum {
     HILS_OK = 0,
     HILS_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent shape */
-    HILS_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, S != 64, K > 32, unknown flags, H / H_kv > 8 */
+    HILS_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, S != 64, K > 32, unknown flags, H / H_kv > 8,
+                                  hils_select_backward over too many chunks */
     HILS_ERR_ALIGNMENT = 3,    /* pointer or stride not 16-byte aligned */
     HILS_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
     HILS_ERR_CUDA = 5          /* a kernel launch failed; see hils_last_cuda_error() */
@@ -313,7 +314,9 @@ int hils_attend_prefill_backward(const hils_params *p, hils_ctensor Q, hils_cten
                                  size_t ws_bytes, cudaStream_t stream);
 
 /* Eq. 7 backward: dQcal [B,H,Lq,d] (written) = scale sum_k dscore_k k'_{idx_k};
- * dKsum [B,H,C,d] += scale dscore q~ and dBsum [B,H,C] += dscore (accumulated). */
+ * dKsum [B,H,C,d] += scale dscore q~ and dBsum [B,H,C] += dscore (accumulated).
+ * Returns HILS_ERR_UNSUPPORTED when C is too large for one CTA's sort of its kept entries
+ * in shared memory (8 C bytes plus 2 K KB within 200 KB: C up to about 21,000 at K = 16). */
 int hils_select_backward(const hils_params *p, hils_ctensor Qcal, int Lq, hils_ctensor Ksum, int C,
                          const int32_t *idx, const int32_t *nsel, const float *dscore,
                          float *dQcal, float *dKsum, float *dBsum, cudaStream_t stream);

@@ -9,9 +9,9 @@ table are stored in bf16, which moves D_i and the chunk scores by up to 2^-9 rel
 and the tensor-core products take dO, dl and cv rounded to bf16; observed about 3e-3).
 Element-wise, every gradient's largest error is within twice that bar times the
 gradient's largest magnitude. The cases cover K = 0 (no kept chunk), W = 0 (no window),
-a table of 400 chunks (the score backward's per-query kernel; chunk 0's list of
-thousands of queries is cut into runs of 1024), grouped heads and a window longer than
-a run. The last test makes every bounded wait of the tensor-core walk expire."""
+a table of 400 chunks (chunk 0's list of thousands of queries is cut into runs of 1024),
+grouped heads and a window longer than a run. The last test makes every bounded wait
+of the tensor-core walk expire."""
 import numpy as np
 import pytest
 import torch
@@ -35,11 +35,14 @@ CASES = {
     # no window (W = 0): the kept chunks alone
     "bf16_d128_W0": (WORKLOADS[2].replace(H=2, N=64 * 6 + 9, K=4, W=0), 1e-2),
     "fp32_d128_W0_grouped": (WORKLOADS[1].replace(H=4, Hk=2, d=128, N=64 * 4 + 9, K=2, W=0), 1e-5),
-    # 400 chunks: the score backward's [C][d] table no longer fits in shared memory, so
-    # the per-query kernel with global atomics runs
+    # 400 chunks: chunk 0's list of thousands of queries is cut into several runs of the
+    # tensor-core walk, and the score backward sorts and sums a large table (its k' copy
+    # still fits in shared memory)
     "bf16_d128_C400": (WORKLOADS[2].replace(H=1, N=64 * 400, K=16, W=512), 1e-2),
     # the tensor-core walk (bf16, d = 128) with query heads sharing a kept list
     "bf16_d128_grouped": (WORKLOADS[7].replace(H=4, Hk=2, d=128, N=64 * 5 + 3, K=3, W=130), 1e-2),
+    # fewer tokens than one chunk (C = 0): no summary, nothing kept; dQcal is zero
+    "bf16_d128_N40": (WORKLOADS[2].replace(H=2, N=40, K=4, W=16), 1e-2),
     # a window longer than one work item's 1024 queries: each window block's queries are
     # cut into two runs, whose dK and dV shares add up
     "bf16_d128_W1500": (WORKLOADS[2].replace(H=1, N=64 * 40 + 5, K=4, W=1500), 1e-2),
