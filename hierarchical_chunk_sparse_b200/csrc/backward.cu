@@ -31,7 +31,7 @@
 // CUDA-core form.
 #include <math.h>
 
-#include "hils_internal.cuh"
+#include "backward_common.cuh"
 
 namespace hils {
 namespace {

@@ -34,6 +34,7 @@
 // of the call's status word, every role stops, the copies and MMAs already started are
 // awaited (bounded again), TMEM is freed and the CTA exits without its remaining
 // gradient adds.
+#include "backward_common.cuh"
 #include "tc_common.cuh"
 
 namespace hils {

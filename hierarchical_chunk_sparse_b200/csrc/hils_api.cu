@@ -4,6 +4,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include "backward_common.cuh"
 #include "hils_internal.cuh"
 
 namespace hils {

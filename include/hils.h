@@ -111,10 +111,10 @@ typedef struct {
  *     hils_decode read the flag; summaries and the attend calls are unchanged. */
 #define HILS_FLAG_EXCLUDE_WINDOW_CHUNKS 1u
 /*   HILS_FLAG_DIAG_EXPIRE_WAITS: diagnostic, for tests of the failure path. The
- *     tensor-core kernels of hils_select (bf16, d = 128, many queries) and of
- *     hils_attend_prefill (bf16, d = 128) bound every wait on work in progress (copies,
- *     tensor-core operations, other warps' hand-offs) by a time limit of the GPU's
- *     global timer (0.1 s). With this flag every such wait expires at its first check,
+ *     tensor-core kernels of hils_select (bf16, d = 128, many queries), of
+ *     hils_attend_prefill and of hils_attend_prefill_backward (bf16, d = 128) bound every
+ *     wait on work in progress (copies, tensor-core operations, other warps' hand-offs)
+ *     by a time limit of the GPU's global timer (0.1 s). With this flag every such wait expires at its first check,
  *     whether or not its phase has completed. The kernel then sets the call's status word (the
  *     first 4 bytes of its workspace, bit 0), stops issuing work, waits (bounded by the
  *     normal limit) for the copies and operations it already started, releases its
@@ -305,8 +305,12 @@ int hils_attend_decode_noalloc(const hils_params *p, hils_ctensor Q, hils_ctenso
  *   dK, dV [B, Hk, N, d]  accumulated
  *   dscore [B, H, N, K]   out: the gradient of each kept chunk's score, 0 padding
  *   workspace, ws_bytes: hils_workspace_bytes(p, HILS_CALL_ATTEND_BACKWARD, N, 0) bytes
- *         (the inverted index of the selection and D_i = dO_i . o_i), no initialisation
- *         needed. */
+ *         (the inverted index of the selection, D_i = dO_i . o_i, and for bf16 with
+ *         d = 128 per-entry records and bf16 copies of dO and Q), no initialisation
+ *         needed. Its first 32-bit word is a status word that each call clears: the bf16,
+ *         d = 128 path (tensor cores, bounded waits) sets it nonzero if a wait on its own
+ *         asynchronous copies or matrix operations ever expires, and then adds nothing
+ *         more for the affected work item. */
 int hils_attend_prefill_backward(const hils_params *p, hils_ctensor Q, hils_ctensor K, hils_ctensor V, int N,
                                  const int32_t *idx, const float *score, const int32_t *nsel,
                                  hils_ctensor O, const float *lse, const float *dO,
