@@ -22,9 +22,10 @@
 //              lane quadrant w % 4 and half w / 4 of the keys (and of dQ's columns); the
 //              two halves of a row exchange its max and sums through shared memory;
 //   warps 8-9  loads, into a ring of two stages: the block's K and V (TMA tiles), each
-//              step's rows of Q (warp 8) and of dO (warp 9), TMA row gathers (four rows
-//              per copy) from the contiguous bf16 copies, and the rows' scalars (warp 8),
-//              loaded a step ahead;
+//              step's rows of Q (warp 8) and of dO (warp 9) from the contiguous bf16
+//              copies (a chunk's scattered queries: TMA row gathers, four rows per copy;
+//              a window block's consecutive queries: one 128-row TMA tile per 64-column
+//              half), and the rows' scalars (warp 8), loaded a step ahead;
 //   warp 10    allocates TMEM and issues tcgen05.mma (one lane), each product as soon as
 //              its inputs are ready.
 // S and T are double-buffered in TMEM, so that the products of step s+1 run while the
@@ -92,6 +93,15 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// A (64 elements x 128 rows) tile at column x, row y of a 2-D tensor map (128-byte swizzle).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n" ::"r"(
+            dst),
+        "l"(map), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
 // Non-blocking test of an mbarrier phase.
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
     uint32_t ok;
@@ -107,6 +117,8 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
                                                                  const __grid_constant__ CUtensorMap tmV,
                                                                  const __grid_constant__ CUtensorMap tmQ,
                                                                  const __grid_constant__ CUtensorMap tmDO,
+                                                                 const __grid_constant__ CUtensorMap tmQt,
+                                                                 const __grid_constant__ CUtensorMap tmDOt,
                                                                  BwdTcArgs t) {
     const BwdAttendArgs &a = t.a;
     const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
@@ -210,7 +222,8 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
         }
         const int64_t row0 = (int64_t)bh * a.N;  // row of query 0 of (b, h) in the contiguous copies
         const int4 *rec = t.recs + row0 * a.topk;
-        const CUtensorMap *tm = lw == 0 ? &tmQ : &tmDO;
+        const CUtensorMap *tm = lw == 0 ? &tmQ : &tmDO;     // four-row gathers (chunk items)
+        const CUtensorMap *tmt = lw == 0 ? &tmQt : &tmDOt;  // 128-row tiles (window items: consecutive queries)
         const uint32_t dst0 = sbase + (lw == 0 ? kQOff : kDOOff) + lane * 512;  // rows 4 lane .. 4 lane + 3
         // the scalars of rows 4 lane + m of a step, as loaded (records, or lse and D_i of window
         // queries): all four loads at once, for the next step before its stage is free
@@ -244,9 +257,16 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
                 if (lw == 0) scal[st * kQ + r] = sc;
                 gy[m] = (int)(row0 + (sc.x >= 0 ? sc.w : 0));
             }
-            const uint32_t dst = dst0 + st * 32768;
-            tma_gather4(dst, tm, bar(kBarFull + st), 0, gy[0], gy[1], gy[2], gy[3]);
-            tma_gather4(dst + 16384, tm, bar(kBarFull + st), 64, gy[0], gy[1], gy[2], gy[3]);
+            if (chunk) {
+                const uint32_t dst = dst0 + st * 32768;
+                tma_gather4(dst, tm, bar(kBarFull + st), 0, gy[0], gy[1], gy[2], gy[3]);
+                tma_gather4(dst + 16384, tm, bar(kBarFull + st), 64, gy[0], gy[1], gy[2], gy[3]);
+            } else if (lane == 0) {  // rows q0 .. q0 + 127: one tile per 64-column half (rows past
+                                     // the run are read and ignored; past the array, zero-filled)
+                const uint32_t dst = sbase + (lw == 0 ? kQOff : kDOOff) + st * 32768;
+                tma_load_2d(dst, tmt, bar(kBarFull + st), 0, (int)(row0 + q0));
+                tma_load_2d(dst + 16384, tmt, bar(kBarFull + st), 64, (int)(row0 + q0));
+            }
             if (lw == 0) {  // the scalars, and the bytes of both warps' row copies
                 if (lane == 0) mbar_expect_tx(bar(kBarFull + st), 4 * kQ * 128);
                 else arrive(bar(kBarFull + st));
@@ -515,14 +535,14 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
     }
 }
 
-// [rows, 128] contiguous bf16 -> 2-D map for four-row gathers: a (64 elements x 1 row)
-// box, 128-byte swizzle.
-bool make_row_map(CUtensorMap *m, const void *ptr, int64_t rows) {
+// [rows, 128] contiguous bf16 -> 2-D map with a (64 elements x box_rows) box, 128-byte
+// swizzle: one row for four-row gathers, 128 for tiles of consecutive rows.
+bool make_row_map(CUtensorMap *m, const void *ptr, int64_t rows, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)kDim * 2};
-    const cuuint32_t box[2] = {64u, 1u};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1u, 1u};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -537,16 +557,17 @@ hils_status launch_attend_bwd_tc(const BwdTcArgs &t, const void *Qc, const void 
     const int64_t nrows = (int64_t)a.B * a.H * a.N;
     const int gx = t.nwin + t.max_items;
     if (gx == 0 || nrows == 0) return HILS_OK;
-    CUtensorMap mk, mv, mq, mdo;
+    CUtensorMap mk, mv, mq, mdo, mqt, mdot;
     if (!make_map(&mk, a.K, a.B, Hk, a.N, kKeys) || !make_map(&mv, a.V, a.B, Hk, a.N, kKeys) ||
-        !make_row_map(&mq, Qc, nrows) || !make_row_map(&mdo, dOb, nrows))
+        !make_row_map(&mq, Qc, nrows, 1) || !make_row_map(&mdo, dOb, nrows, 1) || !make_row_map(&mqt, Qc, nrows, kQ) ||
+        !make_row_map(&mdot, dOb, nrows, kQ))
         return HILS_ERR_CUDA;
     static KernelSetup setup;
     int per_sm = 0;
     const hils_status st = kernel_setup(setup, (const void *)attend_bwd_tc_kernel, kThr, kSmemBytes, &per_sm);
     if (st != HILS_OK) return st;
     if (per_sm < 1) return HILS_ERR_CUDA;
-    attend_bwd_tc_kernel<<<dim3(gx, a.B * a.H), kThr, kSmemBytes, s>>>(mk, mv, mq, mdo, t);
+    attend_bwd_tc_kernel<<<dim3(gx, a.B * a.H), kThr, kSmemBytes, s>>>(mk, mv, mq, mdo, mqt, mdot, t);
     return record_cuda_error(cudaGetLastError());
 }
 
