@@ -927,7 +927,7 @@ def main():
                              "prefill-select", "prefill-backward", "summarize"],
                     help="run a small case for an ncu capture and exit")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="hils", choices=["hils", "reference"])
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill and backward measurements")
