@@ -9,9 +9,9 @@
 // window reaches it. It walks the run 128 queries per step. With Q and dO the step's 128
 // query rows and K, V the block's 64 keys:
 //   S = Q K^T, T = dO V^T            tcgen05, M = 128 queries, N = 64 keys, K = 128 dims
-//   per query row (thread = row = TMEM lane): the softmax-backward weights of the row,
-//     dl = scale * weights and cv, both rounded to bf16 into shared memory, and for a
-//     kept chunk the score gradient dscore
+//   per query row (its TMEM lane, two threads with half of the keys each): the
+//     softmax-backward weights of the row, dl = scale * weights and cv, both rounded to
+//     bf16 into shared memory, and for a kept chunk the score gradient dscore
 //   dK^T += Q^T dl, dV^T += dO^T cv  tcgen05, M = 128 dims, N = 64 keys, K = 128 queries
 //                                    (Q, dO and dl, cv read as MN-major operands)
 //   dQ = dl K                        tcgen05, M = 128 queries, N = 128 dims, K = 64 keys
