@@ -400,10 +400,10 @@ KERNEL_SOURCES = {
 # decode_attend per algorithmic byte of the launch (the captured traffic / algorithmic
 # bytes), summarize per chunk, attend_prefill per launch of the 8K prefill workload.
 MEASURED_TRAFFIC = {
-    'decode_select': (1.0172632638346453, '89390ce2ed3f933e'),
-    'decode_attend': (1.002088743653726, 'bf37b6a22e9eedbe'),
-    'summarize': (16922.4921875, '453a85260e417f60'),
-    'attend_prefill': (659396864, '53ec368d0a713d57'),
+    'decode_select': (1.0161366640629694, '6aa4e612a5e31e4c'),
+    'decode_attend': (1.0020989078564204, 'cb90a6455b1fa122'),
+    'summarize': (16926.2578125, '853b63865c7de306'),
+    'attend_prefill': (661702656, '04b39bda6acf4099'),
 }
 
 
