@@ -3,11 +3,12 @@
 // (picx.dev summary), Methodology 2, Eq. 10, differentiated by hand; the formulas are
 // listed at the top of backward.cu).
 //
-// A CTA takes one work item: a 64-key block of one (b, h), either a kept chunk with a run
-// of at most 1024 of the queries that kept it (entries of the group's inverted index), or
-// a block of window keys with a run of at most 1024 of the consecutive queries whose
-// window reaches it. It walks the run 128 queries per step. With Q and dO the step's 128
-// query rows and K, V the block's 64 keys:
+// A work item is a 64-key block of one (b, h), either a kept chunk with a run of at most
+// 1024 of the queries that kept it (entries of the group's inverted index), or a block of
+// window keys with a run of at most 1024 of the consecutive queries whose window reaches
+// it, walked 128 queries per step. One persistent CTA per SM takes the items in turn (its
+// stride over the item list), its pipelines running on across items. With Q and dO the
+// step's 128 query rows and K, V the block's 64 keys:
 //   S = Q K^T, T = dO V^T            tcgen05, M = 128 queries, N = 64 keys, K = 128 dims
 //   per query row (its TMEM lane, two threads with half of the keys each): the
 //     softmax-backward weights of the row, dl = scale * weights and cv, both rounded to
@@ -35,6 +36,8 @@
 // of the call's status word, every role stops, the copies and MMAs already started are
 // awaited (bounded again), TMEM is freed and the CTA exits without its remaining
 // gradient adds.
+#include <algorithm>
+
 #include "backward_common.cuh"
 #include "tc_common.cuh"
 
@@ -69,17 +72,18 @@ constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
 enum {
     kBarFull = 0,     // + stage: Q, dO rows (bytes) and scalars (32 arrivals of warp 8) of a step landed
     kBarEmpty = 2,    // + stage: every MMA that read the stage completed
-    kBarKV = 4,       // K and V of the block landed
+    kBarKV = 4,       // K and V of the item's block landed
     kBarStFull = 5,   // + buffer: S, T written
     kBarStFree = 7,   // + buffer: the softmax warps read S, T (8 arrivals)
     kBarDlFull = 9,   // dl, cv of the step written (8 arrivals)
     kBarDqFull = 10,  // dQ of the step (and every earlier MMA) completed
     kBarDqFree = 11,  // the softmax warps read dQ (8 arrivals)
-    kBarDone = 12,    // every MMA of the item completed: dK^T, dV^T final
+    kBarDone = 12,    // every MMA of the item completed: dK^T, dV^T final, K and V free
     kBarDrain = 13,   // the MMA warp's own drain
     kBarPair = 14,    // + 2 quadrant + round: the two warps of a row quadrant exchanged half-row
                       //   maxima (round 0) or sums (round 1) (64 arrivals)
-    kNumBars = 22
+    kBarDkvFree = 22, // the softmax warps read the item's dK^T, dV^T (8 arrivals)
+    kNumBars = 23
 };
 
 // Four rows (y0..y3) of 64 bf16 at column x of a 2-D tensor map into 512 consecutive
@@ -113,40 +117,77 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// One work item of the walk (uniform over the CTA): item j of the flattened grid of
+// (item slot x, (b, h)) pairs; slots beyond a group's chunk-item count, and empty runs,
+// are not valid.
+struct BwdItem {
+    bool valid, chunk;
+    int b, h, hk, bh, j0, rows, qb, qe, ns;
+};
+
+__device__ __forceinline__ BwdItem decode_item(const BwdTcArgs &t, int j, int gx) {
+    const BwdAttendArgs &a = t.a;
+    BwdItem it;
+    const int x = j % gx;
+    it.bh = j / gx;
+    it.b = it.bh / a.H;
+    it.h = it.bh % a.H;
+    const int Hk = a.H / a.G;
+    it.hk = it.h / a.G;
+    int blk;
+    it.valid = true;
+    if (x < t.nwin) {
+        blk = x / t.nsegw;
+        const int seg = x - blk * t.nsegw;
+        const int jb = blk * kKeys, nk = min(kKeys, a.N - jb);
+        const int qend = min(a.N, jb + nk - 1 + a.W);  // queries whose window reaches the block
+        it.qb = jb + seg * kBwdItemQueries;
+        it.qe = min(qend, it.qb + kBwdItemQueries);
+        it.chunk = false;
+    } else {
+        const int ci = x - t.nwin;
+        const int64_t bg = (int64_t)it.b * Hk + it.hk;
+        it.chunk = true;
+        if (ci >= t.nitems[bg]) {
+            it.valid = false;
+            blk = 0;
+            it.qb = it.qe = 0;
+        } else {
+            const int4 e = t.items[bg * t.max_items + ci];
+            blk = e.x;
+            it.qb = e.y;
+            it.qe = e.z;
+        }
+    }
+    it.valid = it.valid && it.qb < it.qe;
+    it.ns = it.valid ? (it.qe - it.qb + kQ - 1) / kQ : 0;
+    it.j0 = blk * kKeys;
+    it.rows = min(kKeys, a.N - it.j0);
+    return it;
+}
+
+// Persistent: CTA c walks items c, c + grid, c + 2 grid, ... (valid ones only). The load
+// ring, the S/T buffers and the dl / dQ hand-offs continue across items (phases counted by
+// the CTA's global step index), so the next item's rows and scalars are fetched while the
+// current item finishes; an item's K and V wait for the previous item's last MMA, and its
+// first dK, dV product for the softmax warps' read of the previous item's sums.
 __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                  const __grid_constant__ CUtensorMap tmV,
                                                                  const __grid_constant__ CUtensorMap tmQ,
                                                                  const __grid_constant__ CUtensorMap tmDO,
                                                                  const __grid_constant__ CUtensorMap tmQt,
                                                                  const __grid_constant__ CUtensorMap tmDOt,
-                                                                 BwdTcArgs t) {
+                                                                 BwdTcArgs t, int gx, int total) {
     const BwdAttendArgs &a = t.a;
-    const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
-    const int Hk = a.H / a.G, hk = h / a.G;
-    // ---- the work item (uniform over the CTA)
-    bool chunk;
-    int blk, qb, qe;
-    if ((int)blockIdx.x < t.nwin) {
-        blk = blockIdx.x / t.nsegw;
-        const int seg = blockIdx.x - blk * t.nsegw;
-        const int jb = blk * kKeys, nk = min(kKeys, a.N - jb);
-        const int qend = min(a.N, jb + nk - 1 + a.W);  // queries whose window reaches the block
-        qb = jb + seg * kBwdItemQueries;
-        qe = min(qend, qb + kBwdItemQueries);
-        chunk = false;
-    } else {
-        const int ci = blockIdx.x - t.nwin;
-        const int64_t bg = (int64_t)b * Hk + hk;
-        if (ci >= t.nitems[bg]) return;
-        const int4 it = t.items[bg * t.max_items + ci];
-        blk = it.x;
-        qb = it.y;
-        qe = it.z;
-        chunk = true;
-    }
-    if (qb >= qe) return;
-    const int ns = (qe - qb + kQ - 1) / kQ;
-    const int j0 = blk * kKeys, rows = min(kKeys, a.N - j0);
+    const int Hk = a.H / a.G;
+    // the next valid item at or after j, by this CTA's stride (j >= total: none)
+    auto next_valid = [&](int j) {
+        for (; j < total; j += (int)gridDim.x)
+            if (decode_item(t, j, gx).valid) return j;
+        return total;
+    };
+    const int jfirst = next_valid((int)blockIdx.x);
+    if (jfirst >= total) return;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -161,8 +202,8 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
         for (int i = 0; i < kNumBars; ++i) {
             uint32_t cnt = 1;
             if (i == kBarFull || i == kBarFull + 1) cnt = 32;
-            if (i == kBarStFree || i == kBarStFree + 1 || i == kBarDlFull || i == kBarDqFree) cnt = 8;
-            if (i >= kBarPair) cnt = 64;
+            if (i == kBarStFree || i == kBarStFree + 1 || i == kBarDlFull || i == kBarDqFree || i == kBarDkvFree) cnt = 8;
+            if (i >= kBarPair && i < kBarPair + 8) cnt = 64;
             mbar_init(bar(i), cnt);
         }
         misc[1] = 0u;
@@ -211,72 +252,87 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
 
     if (warp == kLoadWarp || warp == kLoadWarp + 1) {
         // ---------------------------------------------------------------- loads
-        const int lw = warp - kLoadWarp;  // 0: Q rows and the scalars, 1: dO rows
-        if (lw == 0 && lane == 0) {
-            mbar_expect_tx(bar(kBarKV), 4 * kKeys * 128);
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                tma_load_4d(sbase + kKOff + x * 8192, &tmK, bar(kBarKV), x * 64, j0, hk, b);
-                tma_load_4d(sbase + kVOff + x * 8192, &tmV, bar(kBarKV), x * 64, j0, hk, b);
-            }
-        }
-        const int64_t row0 = (int64_t)bh * a.N;  // row of query 0 of (b, h) in the contiguous copies
-        const int4 *rec = t.recs + row0 * a.topk;
+        const int lw = warp - kLoadWarp;  // 0: Q rows, K and V, and the scalars; 1: dO rows
         const CUtensorMap *tm = lw == 0 ? &tmQ : &tmDO;     // four-row gathers (chunk items)
         const CUtensorMap *tmt = lw == 0 ? &tmQt : &tmDOt;  // 128-row tiles (window items: consecutive queries)
         const uint32_t dst0 = sbase + (lw == 0 ? kQOff : kDOOff) + lane * 512;  // rows 4 lane .. 4 lane + 3
         // the scalars of rows 4 lane + m of a step, as loaded (records, or lse and D_i of window
         // queries): all four loads at once, for the next step before its stage is free
         int4 raw[4];
-        auto load_scalars = [&](int s) {
-            const int q0 = qb + s * kQ;
+        auto load_scalars = [&](const BwdItem &it, int s) {
+            const int64_t row0 = (int64_t)it.bh * a.N;
+            const int q0 = it.qb + s * kQ;
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                const int q = min(q0 + 4 * lane + m, qe - 1);
-                if (chunk) {
-                    raw[m] = __ldg(rec + q);
+                const int q = min(q0 + 4 * lane + m, it.qe - 1);
+                if (it.chunk) {
+                    raw[m] = __ldg(t.recs + row0 * a.topk + q);
                 } else {
                     raw[m] = make_int4(q, __float_as_int(__ldg(a.lse + row0 + q)), __float_as_int(__ldg(t.Dv + row0 + q)),
                                        q);
                 }
             }
         };
-        load_scalars(0);
+        int g = 0, nit = 0;  // steps and items issued
         int issued[2] = {0, 0};
-        for (int s = 0; s < ns; ++s) {
-            const int st = s & 1, u = s >> 1;
-            if (u > 0 && !wait_warp(bar(kBarEmpty + st), (u - 1) & 1)) break;
-            const int q0 = qb + s * kQ;
-            int gy[4];  // rows in the contiguous copies (query 0's row for an unused one, read but ignored)
+        bool ok = true;
+        BwdItem cur = decode_item(t, jfirst, gx);
+        load_scalars(cur, 0);
+        for (int j = jfirst; j < total && ok;) {
+            const int jn = next_valid(j + (int)gridDim.x);
+            const BwdItem nxt = jn < total ? decode_item(t, jn, gx) : cur;
+            const int64_t row0 = (int64_t)cur.bh * a.N;
+            for (int s = 0; s < cur.ns; ++s, ++g) {
+                const int st = g & 1, u = g >> 1;
+                if (u > 0 && !(ok = wait_warp(bar(kBarEmpty + st), (u - 1) & 1))) break;
+                const int q0 = cur.qb + s * kQ;
+                int gy[4];  // rows in the contiguous copies (query 0's row for an unused one, read but ignored)
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int r = 4 * lane + m;
-                int4 sc = raw[m];
-                if (!chunk && !isfinite(__int_as_float(sc.y))) sc.x = -1;
-                if (q0 + r >= qe) sc = make_int4(-1, 0, 0, 0);
-                if (lw == 0) scal[st * kQ + r] = sc;
-                gy[m] = (int)(row0 + (sc.x >= 0 ? sc.w : 0));
+                for (int m = 0; m < 4; ++m) {
+                    const int r = 4 * lane + m;
+                    int4 sc = raw[m];
+                    if (!cur.chunk && !isfinite(__int_as_float(sc.y))) sc.x = -1;
+                    if (q0 + r >= cur.qe) sc = make_int4(-1, 0, 0, 0);
+                    if (lw == 0) scal[st * kQ + r] = sc;
+                    gy[m] = (int)(row0 + (sc.x >= 0 ? sc.w : 0));
+                }
+                if (cur.chunk) {
+                    const uint32_t dst = dst0 + st * 32768;
+                    tma_gather4(dst, tm, bar(kBarFull + st), 0, gy[0], gy[1], gy[2], gy[3]);
+                    tma_gather4(dst + 16384, tm, bar(kBarFull + st), 64, gy[0], gy[1], gy[2], gy[3]);
+                } else if (lane == 0) {  // rows q0 .. q0 + 127: one tile per 64-column half (rows past
+                                         // the run are read and ignored; past the array, zero-filled)
+                    const uint32_t dst = sbase + (lw == 0 ? kQOff : kDOOff) + st * 32768;
+                    tma_load_2d(dst, tmt, bar(kBarFull + st), 0, (int)(row0 + q0));
+                    tma_load_2d(dst + 16384, tmt, bar(kBarFull + st), 64, (int)(row0 + q0));
+                }
+                if (lw == 0) {  // the scalars, and the bytes of both warps' row copies
+                    if (lane == 0) mbar_expect_tx(bar(kBarFull + st), 4 * kQ * 128);
+                    else arrive(bar(kBarFull + st));
+                }
+                ++issued[st];
+                if (s == 0 && lw == 0) {  // the item's K and V, once the previous item's MMAs are done
+                    if (nit > 0 && !(ok = wait_warp(bar(kBarDone), (nit - 1) & 1))) break;
+                    if (lane == 0) {
+                        mbar_expect_tx(bar(kBarKV), 4 * kKeys * 128);
+#pragma unroll
+                        for (int x = 0; x < 2; ++x) {
+                            tma_load_4d(sbase + kKOff + x * 8192, &tmK, bar(kBarKV), x * 64, cur.j0, cur.hk, cur.b);
+                            tma_load_4d(sbase + kVOff + x * 8192, &tmV, bar(kBarKV), x * 64, cur.j0, cur.hk, cur.b);
+                        }
+                    }
+                }
+                if (s + 1 < cur.ns) load_scalars(cur, s + 1);
+                else if (jn < total) load_scalars(nxt, 0);
             }
-            if (chunk) {
-                const uint32_t dst = dst0 + st * 32768;
-                tma_gather4(dst, tm, bar(kBarFull + st), 0, gy[0], gy[1], gy[2], gy[3]);
-                tma_gather4(dst + 16384, tm, bar(kBarFull + st), 64, gy[0], gy[1], gy[2], gy[3]);
-            } else if (lane == 0) {  // rows q0 .. q0 + 127: one tile per 64-column half (rows past
-                                     // the run are read and ignored; past the array, zero-filled)
-                const uint32_t dst = sbase + (lw == 0 ? kQOff : kDOOff) + st * 32768;
-                tma_load_2d(dst, tmt, bar(kBarFull + st), 0, (int)(row0 + q0));
-                tma_load_2d(dst + 16384, tmt, bar(kBarFull + st), 64, (int)(row0 + q0));
-            }
-            if (lw == 0) {  // the scalars, and the bytes of both warps' row copies
-                if (lane == 0) mbar_expect_tx(bar(kBarFull + st), 4 * kQ * 128);
-                else arrive(bar(kBarFull + st));
-            }
-            ++issued[st];
-            if (s + 1 < ns) load_scalars(s + 1);
+            if (!ok) break;
+            ++nit;
+            j = jn;
+            cur = nxt;
         }
         // every copy started lands before the CTA releases its memory
         if (lane == 0) {
-            if (lw == 0) drain_wait(bar(kBarKV), 0);
+            if (lw == 0 && nit > 0) drain_wait(bar(kBarKV), (uint32_t)(nit - 1) & 1u);
             for (int st = 0; st < 2; ++st)
                 if (issued[st] > 0) drain_wait(bar(kBarFull + st), (uint32_t)(issued[st] - 1) & 1u);
         }
@@ -286,8 +342,8 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
         const uint32_t idS = idesc_bf16(kQ, kKeys, false);            // K-major A and B
         const uint32_t idKV = idesc_bf16_ab(kDim, kKeys, true, true);  // MN-major A and B
         const uint32_t idQ = idesc_bf16(kQ, kDim, true);              // K-major A, MN-major B
-        auto issue_st = [&](int s) {  // S, T of step s into buffer s % 2
-            const int st = s & 1;
+        auto issue_st = [&](int g) {  // S, T of global step g into buffer g % 2
+            const int st = g & 1;
             const uint32_t dS = tmem + st * 128, dT = dS + 64;
 #pragma unroll
             for (int ks = 0; ks < kDim / 16; ++ks) {
@@ -300,15 +356,16 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
             }
             mma_commit(bar(kBarStFull + st));
         };
-        auto issue_kv = [&](int s) {  // dK^T += Q^T dl, dV^T += dO^T cv: 16 queries per MMA
-            const int st = s & 1;
+        auto issue_kv = [&](int g, bool first) {  // dK^T (+)= Q^T dl, dV^T (+)= dO^T cv: 16 queries per MMA
+            const int st = g & 1;
 #pragma unroll
             for (int ks = 0; ks < kQ / 16; ++ks) {
                 const uint32_t ro = st * 32768 + ks * 2048;
+                const uint32_t acc = (!first || ks > 0) ? 1u : 0u;
                 mma_ss(tmem + 256, smem_desc(sbase + kQOff + ro, 16384, 1024),
-                       smem_desc(sbase + kDLOff + ks * 2048, 8192, 1024), idKV, (s > 0 || ks > 0) ? 1u : 0u);
+                       smem_desc(sbase + kDLOff + ks * 2048, 8192, 1024), idKV, acc);
                 mma_ss(tmem + 320, smem_desc(sbase + kDOOff + ro, 16384, 1024),
-                       smem_desc(sbase + kCVOff + ks * 2048, 8192, 1024), idKV, (s > 0 || ks > 0) ? 1u : 0u);
+                       smem_desc(sbase + kCVOff + ks * 2048, 8192, 1024), idKV, acc);
             }
             mma_commit(bar(kBarEmpty + st));  // the last reads of the stage's Q and dO rows
         };
@@ -319,58 +376,69 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
                        smem_desc(sbase + kKOff + ks * 2048, 8192, 1024), idQ, ks > 0 ? 1u : 0u);
             mma_commit(bar(kBarDqFull));
         };
-        // Issue each product as soon as its inputs are ready, earliest step first within a
-        // kind, S/T ahead of the rest: S, T of step n need its rows (full) and their TMEM
-        // buffer read (the softmax of step n - 2); dK, dV of step k need dl, cv of k; dQ of
-        // step k needs dK, dV of k issued and dQ of k - 1 read. Every test is a
-        // non-blocking look at a phase whose predecessor this warp has already seen.
-        bool ok = wait_warp(bar(kBarKV), 0);
-        int nS = 0, nK = 0, nQ = 0;
-        uint64_t idle_since = 0;
-        int idle = 0;
-        while (ok && nQ < ns) {
-            bool ready = false;
-            int kind = -1;
-            if (lane == 0) {
-                if (nS < ns && mbar_test(bar(kBarFull + (nS & 1)), (nS >> 1) & 1) &&
-                    (nS < 2 || mbar_test(bar(kBarStFree + (nS & 1)), ((nS >> 1) - 1) & 1)))
-                    kind = 0;
-                else if (nK < nS && mbar_test(bar(kBarDlFull), nK & 1))
-                    kind = 1;
-                else if (nQ < nK && (nQ == 0 || mbar_test(bar(kBarDqFree), (nQ - 1) & 1)))
-                    kind = 2;
-            }
-            kind = __shfl_sync(kFull, kind, 0);
-            ready = kind >= 0;
-            if (ready) {
-                tc_fence_after();
+        // Per item, each product is issued as soon as its inputs are ready, earliest step
+        // first within a kind, S/T ahead of the rest: S, T of step n need its rows (full),
+        // their TMEM buffer read (the softmax of step n - 2) and the item's K and V; dK, dV
+        // of step n need dl, cv of n (and, for the item's first, the softmax warps' read of
+        // the previous item's sums); dQ of step n needs dK, dV of n issued and dQ of n - 1
+        // read. Every test is a non-blocking look at a phase whose predecessor this warp
+        // has already seen.
+        bool ok = true;
+        int g0 = 0, nit = 0;
+        for (int j = jfirst; j < total && ok; j = next_valid(j + (int)gridDim.x)) {
+            const BwdItem it = decode_item(t, j, gx);
+            if (!(ok = wait_warp(bar(kBarKV), nit & 1))) break;
+            int nS = 0, nK = 0, nQ = 0;
+            uint64_t idle_since = 0;
+            int idle = 0;
+            while (ok && nQ < it.ns) {
+                int kind = -1;
                 if (lane == 0) {
-                    if (kind == 0) issue_st(nS);
-                    else if (kind == 1) issue_kv(nK);
-                    else issue_dq();
+                    const int gS = g0 + nS, gK = g0 + nK, gQ = g0 + nQ;
+                    if (nS < it.ns && mbar_test(bar(kBarFull + (gS & 1)), (gS >> 1) & 1) &&
+                        (gS < 2 || mbar_test(bar(kBarStFree + (gS & 1)), ((gS >> 1) - 1) & 1)))
+                        kind = 0;
+                    else if (nK < nS && mbar_test(bar(kBarDlFull), gK & 1) &&
+                             (nK > 0 || nit == 0 || mbar_test(bar(kBarDkvFree), (nit - 1) & 1)))
+                        kind = 1;
+                    else if (nQ < nK && (gQ == 0 || mbar_test(bar(kBarDqFree), (gQ - 1) & 1)))
+                        kind = 2;
                 }
-                __syncwarp();
-                if (kind == 0) ++nS;
-                else if (kind == 1) ++nK;
-                else ++nQ;
-                idle = 0;
-                continue;
-            }
-            // nothing ready: bounded like every other wait
-            __nanosleep(32);
-            if (idle == 0) idle_since = global_ns();
-            if ((++idle & 15) == 0 || a.wait_ns <= 0) {
-                bool stop = *abort_flag != 0u;
-                if (!stop && (a.wait_ns <= 0 || (long long)(global_ns() - idle_since) > a.wait_ns)) {
-                    *abort_flag = 1u;
-                    atomicOr(t.status, 1u);
-                    stop = true;
+                kind = __shfl_sync(kFull, kind, 0);
+                if (kind >= 0) {
+                    tc_fence_after();
+                    if (lane == 0) {
+                        if (kind == 0) issue_st(g0 + nS);
+                        else if (kind == 1) issue_kv(g0 + nK, nK == 0);
+                        else issue_dq();
+                    }
+                    __syncwarp();
+                    if (kind == 0) ++nS;
+                    else if (kind == 1) ++nK;
+                    else ++nQ;
+                    idle = 0;
+                    continue;
                 }
-                ok = !__any_sync(kFull, stop);
+                // nothing ready: bounded like every other wait
+                __nanosleep(32);
+                if (idle == 0) idle_since = global_ns();
+                if ((++idle & 15) == 0 || a.wait_ns <= 0) {
+                    bool stop = *abort_flag != 0u;
+                    if (!stop && (a.wait_ns <= 0 || (long long)(global_ns() - idle_since) > a.wait_ns)) {
+                        *abort_flag = 1u;
+                        atomicOr(t.status, 1u);
+                        stop = true;
+                    }
+                    ok = !__any_sync(kFull, stop);
+                }
             }
+            if (!ok) break;
+            if (lane == 0) mma_commit(bar(kBarDone));  // every MMA of the item (dK^T, dV^T final)
+            __syncwarp();
+            g0 += it.ns;
+            ++nit;
         }
         if (lane == 0) {
-            if (ok) mma_commit(bar(kBarDone));
             // every MMA issued completes before TMEM and shared memory are released
             mma_commit(bar(kBarDrain));
             drain_wait(bar(kBarDrain), 0);
@@ -389,15 +457,15 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
         float *xm = reinterpret_cast<float *>(smem + kXOff);        // [2][128] half-row maxima
         float2 *xz = reinterpret_cast<float2 *>(smem + kXOff + 1024);  // [2][128] half-row sum, o_c . dO
         // the two warps of a row quadrant (quad and quad + 4) meet on mbarrier kBarPair + 2
-        // quad + round (64 arrivals, one phase per step), a bounded wait like every other
-        auto pair_sync = [&](int round, int s) -> bool {
+        // quad + round (64 arrivals, one phase per chunk step), a bounded wait like every other
+        auto pair_sync = [&](int round, int pc) -> bool {
             arrive(bar(kBarPair + 2 * quad + round));
-            return wait_warp(bar(kBarPair + 2 * quad + round), s & 1);
+            return wait_warp(bar(kBarPair + 2 * quad + round), pc & 1);
         };
-        int prev = -1;  // query of this row in the previous step (its dQ row), or -1
+        int64_t prev = -1;  // dQ row (b, h, query) of this row in the previous step, or -1
         // this row's half of the dQ of the last completed step into the global dQ
-        auto dq_out = [&](int qrow) {
-            float *dst = a.dQ + ((int64_t)bh * a.N + (qrow < 0 ? 0 : qrow)) * kDim + g * 64;
+        auto dq_out = [&](int64_t qrow) {
+            float *dst = a.dQ + (qrow < 0 ? 0 : qrow) * kDim + g * 64;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t v[32];
@@ -421,111 +489,122 @@ __global__ void __launch_bounds__(kThr, 1) attend_bwd_tc_kernel(const __grid_con
             if (lane == 0) arrive(bar(kBarDqFree));
         };
         bool ok = true;
-        for (int s = 0; s < ns; ++s) {
-            const int st = s & 1;
-            if (!(ok = wait_warp(bar(kBarStFull + st), (s >> 1) & 1))) break;
-            tc_fence_after();
-            uint32_t sv[32], tv[32];
-            tmem_ld32(tmem + lb + st * 128 + g * 32, sv);
-            tmem_ld32(tmem + lb + st * 128 + 64 + g * 32, tv);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) arrive(bar(kBarStFree + st));
-            const int4 sc = scal[st * kQ + r];
-            const int en = sc.x, qi = sc.w;
-            const float wl = __int_as_float(sc.y), Dd = __int_as_float(sc.z);
-            auto S = [&](int j) { return __uint_as_float(sv[j]); };
-            auto T = [&](int j) { return __uint_as_float(tv[j]); };
-            uint32_t dlp[16], cvp[16];  // bf16 pairs of keys 32 g + 2 p, + 1
-            if (chunk) {
-                // p_j = softmax over the chunk of scale S_j; o_c . dO = sum_j p_j T_j;
-                // dl_j = w p_j (T_j - o_c . dO), cv_j = w p_j; dscore = w (o_c . dO - D_i)
-                float mx[4] = {S(0), S(1), S(2), S(3)};
-#pragma unroll
-                for (int j = 4; j < 32; ++j) mx[j & 3] = fmaxf(mx[j & 3], S(j));
-                xm[g * kQ + r] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-                if (!(ok = pair_sync(0, s))) break;
-                const float ms = fmaxf(xm[r], xm[kQ + r]) * sl2;
-                float e[32], zp[4] = {0.f, 0.f, 0.f, 0.f}, op[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    e[j] = ex2(fmaf(S(j), sl2, -ms));
-                    zp[j & 3] += e[j];
-                    op[j & 3] = fmaf(e[j], T(j), op[j & 3]);
-                }
-                xz[g * kQ + r] = make_float2((zp[0] + zp[1]) + (zp[2] + zp[3]), (op[0] + op[1]) + (op[2] + op[3]));
-                if (!(ok = pair_sync(1, s))) break;
-                const float2 z0 = xz[r], z1 = xz[kQ + r];
-                const float inv = 1.f / (z0.x + z1.x);
-                const float oc = (z0.y + z1.y) * inv;
-                const float wc = en >= 0 ? wl * inv : 0.f;
-#pragma unroll
-                for (int p = 0; p < 16; ++p) {
-                    const float c0 = wc * e[2 * p], c1 = wc * e[2 * p + 1];
-                    cvp[p] = pack_bf16(c0, c1);
-                    dlp[p] = pack_bf16(a.scale * c0 * (T(2 * p) - oc), a.scale * c1 * (T(2 * p + 1) - oc));
-                }
-                if (g == 0 && en >= 0) a.dscore[((int64_t)bh * a.N + qi) * K + (en & 31)] = wl * (oc - Dd);
-            } else {
-                // window key j0 + j of query qi: c_j = exp(scale S_j - lse), dl_j = c_j (T_j - D_i)
-                const float l2 = wl * kLog2e;
-#pragma unroll
-                for (int p = 0; p < 16; ++p) {
-                    float c[2];
-#pragma unroll
-                    for (int hv = 0; hv < 2; ++hv) {
-                        const int j = 32 * g + 2 * p + hv, key = j0 + j;
-                        const bool in = en >= 0 && j < rows && key <= qi && key > qi - a.W;
-                        c[hv] = in ? ex2(fmaf(S(2 * p + hv), sl2, -l2)) : 0.f;
-                    }
-                    cvp[p] = pack_bf16(c[0], c[1]);
-                    dlp[p] = pack_bf16(a.scale * c[0] * (T(2 * p) - Dd), a.scale * c[1] * (T(2 * p + 1) - Dd));
-                }
-            }
-            // dl, cv of the previous step were read by its MMAs once its dQ completed
-            if (s > 0) {
-                if (!(ok = wait_warp(bar(kBarDqFull), (s - 1) & 1))) break;
+        int gs = 0, pc = 0, nit = 0;  // global step, chunk steps, items
+        for (int j = jfirst; j < total && ok; j = next_valid(j + (int)gridDim.x)) {
+            const BwdItem it = decode_item(t, j, gx);
+            const int j0 = it.j0, rows = it.rows;
+            for (int s = 0; s < it.ns; ++s, ++gs) {
+                const int st = gs & 1;
+                if (!(ok = wait_warp(bar(kBarStFull + st), (gs >> 1) & 1))) break;
                 tc_fence_after();
-            }
-            uint8_t *dlrow = smem + kDLOff + r * 128, *cvrow = smem + kCVOff + r * 128;
+                uint32_t sv[32], tv[32];
+                tmem_ld32(tmem + lb + st * 128 + g * 32, sv);
+                tmem_ld32(tmem + lb + st * 128 + 64 + g * 32, tv);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) arrive(bar(kBarStFree + st));
+                // the step's scalars: their producer's arrival on the stage (complete by now)
+                if (!(ok = wait_warp(bar(kBarFull + st), (gs >> 1) & 1))) break;
+                const int4 sc = scal[st * kQ + r];
+                const int en = sc.x, qi = sc.w;
+                const float wl = __int_as_float(sc.y), Dd = __int_as_float(sc.z);
+                auto S = [&](int jj) { return __uint_as_float(sv[jj]); };
+                auto T = [&](int jj) { return __uint_as_float(tv[jj]); };
+                uint32_t dlp[16], cvp[16];  // bf16 pairs of keys 32 g + 2 p, + 1
+                if (it.chunk) {
+                    // p_j = softmax over the chunk of scale S_j; o_c . dO = sum_j p_j T_j;
+                    // dl_j = w p_j (T_j - o_c . dO), cv_j = w p_j; dscore = w (o_c . dO - D_i)
+                    float mx[4] = {S(0), S(1), S(2), S(3)};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {  // 16-byte units 4 g + u of the row (keys 32 g + 8 u ..)
-                const int o = ((4 * g + u) ^ (r & 7)) << 4;
-                *reinterpret_cast<uint4 *>(dlrow + o) = make_uint4(dlp[4 * u], dlp[4 * u + 1], dlp[4 * u + 2], dlp[4 * u + 3]);
-                *reinterpret_cast<uint4 *>(cvrow + o) = make_uint4(cvp[4 * u], cvp[4 * u + 1], cvp[4 * u + 2], cvp[4 * u + 3]);
-            }
-            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-            __syncwarp();
-            if (lane == 0) arrive(bar(kBarDlFull));
-            if (s > 0) dq_out(prev);
-            prev = en >= 0 ? qi : -1;
-        }
-        if (ok && wait_warp(bar(kBarDqFull), (ns - 1) & 1)) {
-            tc_fence_after();
-            dq_out(prev);
-        } else {
-            ok = false;
-        }
-        // dK^T and dV^T: row r of TMEM is dimension x = r; key j in column j (this warp's half)
-        if (ok && wait_warp(bar(kBarDone), 0)) {
-            tc_fence_after();
-            const int64_t kvrow = ((int64_t)b * Hk + hk) * a.N + j0;
-            float *dk = a.dK + kvrow * kDim + r;
-            float *dv = a.dV + kvrow * kDim + r;
-            uint32_t vk[32], vv[32];
-            tmem_ld32(tmem + lb + 256 + g * 32, vk);
-            tmem_ld32(tmem + lb + 320 + g * 32, vv);
-            tmem_wait_ld();
+                    for (int jj = 4; jj < 32; ++jj) mx[jj & 3] = fmaxf(mx[jj & 3], S(jj));
+                    xm[g * kQ + r] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                    if (!(ok = pair_sync(0, pc))) break;
+                    const float ms = fmaxf(xm[r], xm[kQ + r]) * sl2;
+                    float e[32], zp[4] = {0.f, 0.f, 0.f, 0.f}, op[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int u = 0; u < 32; ++u) {
-                const int j = g * 32 + u;
-                if (j < rows) {
-                    atomicAdd(dk + (int64_t)j * kDim, __uint_as_float(vk[u]));
-                    atomicAdd(dv + (int64_t)j * kDim, __uint_as_float(vv[u]));
+                    for (int jj = 0; jj < 32; ++jj) {
+                        e[jj] = ex2(fmaf(S(jj), sl2, -ms));
+                        zp[jj & 3] += e[jj];
+                        op[jj & 3] = fmaf(e[jj], T(jj), op[jj & 3]);
+                    }
+                    xz[g * kQ + r] = make_float2((zp[0] + zp[1]) + (zp[2] + zp[3]), (op[0] + op[1]) + (op[2] + op[3]));
+                    if (!(ok = pair_sync(1, pc))) break;
+                    ++pc;
+                    const float2 z0 = xz[r], z1 = xz[kQ + r];
+                    const float inv = 1.f / (z0.x + z1.x);
+                    const float oc = (z0.y + z1.y) * inv;
+                    const float wc = en >= 0 ? wl * inv : 0.f;
+#pragma unroll
+                    for (int p = 0; p < 16; ++p) {
+                        const float c0 = wc * e[2 * p], c1 = wc * e[2 * p + 1];
+                        cvp[p] = pack_bf16(c0, c1);
+                        dlp[p] = pack_bf16(a.scale * c0 * (T(2 * p) - oc), a.scale * c1 * (T(2 * p + 1) - oc));
+                    }
+                    if (g == 0 && en >= 0) a.dscore[((int64_t)it.bh * a.N + qi) * K + (en & 31)] = wl * (oc - Dd);
+                } else {
+                    // window key j0 + j of query qi: c_j = exp(scale S_j - lse), dl_j = c_j (T_j - D_i)
+                    const float l2 = wl * kLog2e;
+#pragma unroll
+                    for (int p = 0; p < 16; ++p) {
+                        float c[2];
+#pragma unroll
+                        for (int hv = 0; hv < 2; ++hv) {
+                            const int jj = 32 * g + 2 * p + hv, key = j0 + jj;
+                            const bool in = en >= 0 && jj < rows && key <= qi && key > qi - a.W;
+                            c[hv] = in ? ex2(fmaf(S(2 * p + hv), sl2, -l2)) : 0.f;
+                        }
+                        cvp[p] = pack_bf16(c[0], c[1]);
+                        dlp[p] = pack_bf16(a.scale * c[0] * (T(2 * p) - Dd), a.scale * c[1] * (T(2 * p + 1) - Dd));
+                    }
+                }
+                // dl, cv of the previous step were read by its MMAs once its dQ completed
+                if (gs > 0) {
+                    if (!(ok = wait_warp(bar(kBarDqFull), (gs - 1) & 1))) break;
+                    tc_fence_after();
+                }
+                uint8_t *dlrow = smem + kDLOff + r * 128, *cvrow = smem + kCVOff + r * 128;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {  // 16-byte units 4 g + u of the row (keys 32 g + 8 u ..)
+                    const int o = ((4 * g + u) ^ (r & 7)) << 4;
+                    *reinterpret_cast<uint4 *>(dlrow + o) = make_uint4(dlp[4 * u], dlp[4 * u + 1], dlp[4 * u + 2], dlp[4 * u + 3]);
+                    *reinterpret_cast<uint4 *>(cvrow + o) = make_uint4(cvp[4 * u], cvp[4 * u + 1], cvp[4 * u + 2], cvp[4 * u + 3]);
+                }
+                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                __syncwarp();
+                if (lane == 0) arrive(bar(kBarDlFull));
+                if (gs > 0) dq_out(prev);
+                prev = en >= 0 ? (int64_t)it.bh * a.N + qi : -1;
+            }
+            if (!ok) break;
+            // the item's dK^T and dV^T: row r of TMEM is dimension x = r; key j in column j
+            // (this warp's half); then the next item's first dK, dV product may overwrite them
+            if (!(ok = wait_warp(bar(kBarDone), nit & 1))) break;
+            tc_fence_after();
+            {
+                const int64_t kvrow = ((int64_t)it.b * Hk + it.hk) * a.N + j0;
+                float *dk = a.dK + kvrow * kDim + r;
+                float *dv = a.dV + kvrow * kDim + r;
+                uint32_t vk[32], vv[32];
+                tmem_ld32(tmem + lb + 256 + g * 32, vk);
+                tmem_ld32(tmem + lb + 320 + g * 32, vv);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) arrive(bar(kBarDkvFree));
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const int jj = g * 32 + u;
+                    if (jj < rows) {
+                        atomicAdd(dk + (int64_t)jj * kDim, __uint_as_float(vk[u]));
+                        atomicAdd(dv + (int64_t)jj * kDim, __uint_as_float(vv[u]));
+                    }
                 }
             }
+            ++nit;
         }
+        // the last step's dQ (complete: the last item's MMAs were awaited above)
+        if (ok && gs > 0) dq_out(prev);
     }
     tc_fence_before();
     __syncthreads();
@@ -567,7 +646,10 @@ hils_status launch_attend_bwd_tc(const BwdTcArgs &t, const void *Qc, const void 
     const hils_status st = kernel_setup(setup, (const void *)attend_bwd_tc_kernel, kThr, kSmemBytes, &per_sm);
     if (st != HILS_OK) return st;
     if (per_sm < 1) return HILS_ERR_CUDA;
-    attend_bwd_tc_kernel<<<dim3(gx, a.B * a.H), kThr, kSmemBytes, s>>>(mk, mv, mq, mdo, mqt, mdot, t);
+    const int64_t total = (int64_t)gx * a.B * a.H;
+    if (total > 0x7fffffffll) return HILS_ERR_UNSUPPORTED;
+    const int grid = (int)std::min<int64_t>(total, (int64_t)per_sm * device_sm_count());
+    attend_bwd_tc_kernel<<<grid, kThr, kSmemBytes, s>>>(mk, mv, mq, mdo, mqt, mdot, t, gx, (int)total);
     return record_cuda_error(cudaGetLastError());
 }
 

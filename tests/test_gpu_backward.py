@@ -84,13 +84,16 @@ def test_backward_matches_oracle(cuda_device, case):
     f32 = dict(dtype=torch.float32, device=cuda_device)
     dQ, dK, dV = torch.empty(B, H, N, dd, **f32), torch.zeros(B, Hk, N, dd, **f32), torch.zeros(B, Hk, N, dd, **f32)
     dscore = torch.empty(B, H, N, K, **f32)
-    hils.hils_attend_prefill_backward(p, d["Q"], d["K"], d["V"], idx, score, nsel, O, lse, dO, dQ, dK, dV, dscore)
+    ws = hils.alloc_workspace(p, hils.HILS_CALL_ATTEND_BACKWARD, N, 0, device=cuda_device)
+    hils.hils_attend_prefill_backward(p, d["Q"], d["K"], d["V"], idx, score, nsel, O, lse, dO, dQ, dK, dV, dscore,
+                                      workspace=ws)
     dQcal = torch.empty(B, H, N, dd, **f32)
     dKsum, dBsum = torch.zeros(B, H, C, dd, **f32), torch.zeros(B, H, C, **f32)
     hils.hils_select_backward(p, d["Qcal"], Ksum, idx, nsel, dscore, dQcal, dKsum, dBsum)
     dLQ = torch.empty(B, H, C, dd, **f32)
     hils.hils_summarize_backward(p, d["K"], d["LQ"], dKsum, dBsum, dK, dLQ)
     torch.cuda.synchronize()
+    assert int(host(ws[:4]).view(torch.int32)[0]) == 0, "a bounded wait of the attend backward expired"
     ref = ob.grads(inp["Q"], inp["K"], inp["V"], inp["Qcal"], inp["LQ"], host(idx), host(nsel), host(dO), 64, w.W,
                    w.scale, batch=256)
     errs = {
@@ -153,6 +156,7 @@ def test_backward_full_size(cuda_device, case):
     hils.hils_select_backward(p, d["Qcal"], Ksum, idx, nsel, dscore, dQcal, dKsum, dBsum)
     hils.hils_summarize_backward(p, d["K"], d["LQ"], dKsum, dBsum, dK, dLQ)
     torch.cuda.synchronize()
+    assert int(host(ws[:4]).view(torch.int32)[0]) == 0, "a bounded wait of the attend backward expired"
     kept = torch.arange(K, device=cuda_device).view(1, 1, 1, K) < nsel.repeat_interleave(G, dim=1).unsqueeze(-1)
     assert (dscore[~kept] == 0).all()
     dO_h = host(dO)
