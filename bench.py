@@ -30,7 +30,9 @@ timed steps between two CUDA events on the launching stream; barrier + synchroni
 around the region; the max over ranks is reported. Prefill and backward passes (and
 the cold single step) are timed one at a time with L2 flushed before each. Multi-GPU
 (torchrun): every rank runs its own replica of the workload (weak scaling; the path
-has no exchange step) and value = all ranks' tokens / max time.
+has no exchange step) and value = all ranks' tokens / max time. Per-step timings also
+report their median and 90th percentile (p50_ms, p90_ms); fractions are given against
+the measured peaks (HBM copy, bf16 burst) and against 8 TB/s or the sustained bf16 peak.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hils|reference]
 """
@@ -164,6 +166,12 @@ def time_steps(fn, steps, flush, stream):
             e.record(stream)
     stream.synchronize()
     return [s.elapsed_time(e) for s, e in ev]
+
+
+def spread(ms_list):
+    """Median and 90th percentile of per-step milliseconds."""
+    v = sorted(ms_list)
+    return {"p50_ms": statistics.median(v), "p90_ms": v[min(len(v) - 1, int(round(0.9 * (len(v) - 1))))]}
 
 
 def graphed(fn, stream):
@@ -706,8 +714,8 @@ def measure_prefill(wp, dev, stream, flush, args, world, peaks, peak_src, traffi
     stream.synchronize()
     n = max(3, min(args.steps, 20))
     with ClockSampler(dev) as pclk:
-        pt = statistics.mean(time_steps(graphed(pb.step, stream), n, flush, stream))
-    pt = max_over_ranks(pt, world, dev)
+        pts = time_steps(graphed(pb.step, stream), n, flush, stream)
+    pt = max_over_ranks(statistics.mean(pts), world, dev)
     ks = {k: statistics.mean(time_steps(graphed(getattr(pb, k), stream), n, flush, stream))
           for k in ("summarize", "select", "attend")}
     torch.cuda.synchronize()
@@ -716,14 +724,16 @@ def measure_prefill(wp, dev, stream, flush, args, world, peaks, peak_src, traffi
     tf = fl / (pt * 1e-3) / 1e12
     fl_att = prefill_flops(wp, "attend")
     tf_att = fl_att / (ks["attend"] * 1e-3) / 1e12
-    out = {"value": tf * world, "unit": "TFLOP/s", "ms_per_step": pt, "workload": wp.name,
+    out = {"value": tf * world, "unit": "TFLOP/s", "ms_per_step": pt, **spread(pts), "workload": wp.name,
            "algorithmic_gflop_per_step": fl / 1e9, "steps": n,
            "kernel_ms": ks, "clocks": pclk.summary(),
            "step_frac_of_peak": tf / peaks["bf16_tflops"],
+           "step_frac_of_sustained_peak": tf / peaks["bf16_tflops_sustained"],
            "mean_item_union_chunks": mean_item_union(pb.idx, pb.nsel, wp.C, 256 // packed_heads(wp.G)),
            "roofline": {"bound": "tensor", "kernel": "attend", "achieved": tf_att,
                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                         "frac": tf_att / peaks["bf16_tflops"], "traffic": traffic,
+                        "frac_sustained": tf_att / peaks["bf16_tflops_sustained"],
                         "algorithmic_gflop": fl_att / 1e9,
                         "peak_source": f"{peak_src} bf16 dense (burst)"}}
     del pb
@@ -745,7 +755,7 @@ def backward_flops(w) -> float:
     return float(w.B * w.H * (10 * d * tok + 4 * d * sel + 8 * d * S * C))
 
 
-def measure_prefill_backward(w, dev, stream, flush, args, world):
+def measure_prefill_backward(w, dev, stream, flush, args, world, peaks):
     """The three backward calls of the 8K prefill for the forward's selection (L2
     flushed before each timed pass; the accumulated gradients are zeroed inside it)."""
     import hierarchical_chunk_sparse_b200 as hils
@@ -776,8 +786,8 @@ def measure_prefill_backward(w, dev, stream, flush, args, world):
             bwd()
     stream.synchronize()
     n = 3
-    ms = statistics.mean(time_steps(bwd, n, flush, stream))
-    ms = max_over_ranks(ms, world, dev)
+    bts = time_steps(bwd, n, flush, stream)
+    ms = max_over_ranks(statistics.mean(bts), world, dev)
 
     # each call timed alone (L2 flushed), with the zeroing of what it accumulates into
     def attend_bwd():
@@ -798,8 +808,10 @@ def measure_prefill_backward(w, dev, stream, flush, args, world):
              for name, f in (("attend_backward", attend_bwd), ("select_backward", select_bwd),
                              ("summarize_backward", summarize_bwd))}
     fl = backward_flops(w)
-    out = {"ms_per_step": ms, "unit": "TFLOP/s", "value": fl / (ms * 1e-3) / 1e12 * world, "workload": w.name,
+    tf = fl / (ms * 1e-3) / 1e12
+    out = {"ms_per_step": ms, **spread(bts), "unit": "TFLOP/s", "value": tf * world, "workload": w.name,
            "algorithmic_gflop_per_step": fl / 1e9, "steps": n, "ms_per_call": split,
+           "frac_of_peak": tf / peaks["bf16_tflops"], "frac_of_sustained_peak": tf / peaks["bf16_tflops_sustained"],
            "note": "key-major attend backward on tcgen05 (bf16, d = 128: 128 queries per step of a 64-key block, dK and dV accumulated in TMEM per work item, Q and dO rows by TMA row gathers), float32 atomics for dQ (vector) and dK, dV; dKsum and dBsum summed per CTA in shared memory first; ms_per_call times each call alone"}
     del pb
     torch.cuda.empty_cache()
@@ -830,7 +842,8 @@ def measure_decode(w, dev, stream, flush, args, world, peaks, peak_src, steps: i
     t_sel = time_rotating(g_sel, steps, stream)
     t_att = time_rotating(g_att, steps, stream)
     n_cold = max(3, min(steps, 50))
-    ms_cold = statistics.mean(time_steps(g_step[1][0], n_cold, flush, stream))
+    cold = time_steps(g_step[1][0], n_cold, flush, stream)
+    ms_cold = statistics.mean(cold)
     by = decode_bytes(w)
     hbm = peaks["hbm_gbs"]
     sel_gbs = by["select"] / (t_sel * 1e-3) / 1e9
@@ -846,10 +859,10 @@ def measure_decode(w, dev, stream, flush, args, world, peaks, peak_src, steps: i
            "algorithmic_bytes": by,
            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom_gbs, "peak": hbm, "unit": "GB/s",
                         "frac": dom_gbs / hbm, "traffic": traffic, "algorithmic_bytes": dom_bytes,
-                        "peak_source": f"{peak_src} HBM copy"},
+                        "frac_8tbs": dom_gbs / 8000.0, "peak_source": f"{peak_src} HBM copy"},
            "step_roofline": {"bytes": by["step"], "achieved_gbs": step_gbs, "frac_measured": step_gbs / hbm,
                              "frac_8tbs": step_gbs / 8000.0},
-           "cold_single_step": {"ms": ms_cold, "tokens_per_s": job_throughput(w.B, world, ms_cold),
+           "cold_single_step": {"ms": ms_cold, **spread(cold), "tokens_per_s": job_throughput(w.B, world, ms_cold),
                                 "protocol": Flusher.DESCRIPTION + "; CUDA events around each step"},
            "gpu_launches": steps * db.launches_per_step}
     if w.needles:
@@ -981,7 +994,7 @@ def main():
                                         rebuild=rb)
     # ---------------- backward of the 8K prefill (fixed selection)
     if not args.no_prefill:
-        prefill_bwd = measure_prefill_backward(WORKLOADS[2], dev, stream, flush, args, world)
+        prefill_bwd = measure_prefill_backward(WORKLOADS[2], dev, stream, flush, args, world, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
