@@ -20,7 +20,8 @@ Beside it, in the same line:
   "decode_gqa", "decode_retrieval": the other decode workloads, each with its own
   roofline;
   "prefill_backward": the backward of the 8K prefill for its selection;
-  "cpu_baseline": the float64 oracle on this host's cores, on a sample of heads.
+  "cpu_baseline": the float64 oracle on this host's cores, on a sample of heads (also
+  inside the B8 128K and 1M decode entries, on smaller samples).
 
 Timing: decode steps run back to back over R independent copies of the workload's
 inputs (R copies of KV cache, summaries, queries and outputs, cycled in order) whose
@@ -999,6 +1000,11 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, dev)
+        # the oracle beside the other decode configurations too (a smaller sample each)
+        for key, cfg in (("decode_b8_128k", 3), ("decode_1m", 5)):
+            if key in extra:
+                extra[key]["cpu_baseline"] = cpu_baseline(WORKLOADS[cfg], dev, heads=2, min_s=3.0, max_s=8.0,
+                                                          single_thread=False)
 
     if rank == 0:
         line = {
