@@ -229,3 +229,46 @@ def test_backward_waits_expire_and_recover(cuda_device):
     # the attend call's own gradients (dK also takes the summaries' share, added later)
     for name, got in (("dQ", dQ), ("dV", dV), ("dscore", dscore)):
         assert _rel(got, full[name]) <= 1e-2, f"{name} after the diagnostic call"
+
+
+def test_backward_unaligned_gradients(cuda_device):
+    """Gradient arrays need only 4-byte alignment: with dQ, dK, dV, dKsum and dBsum
+    starting 4 bytes past a 16-byte boundary the kernels take their scalar-atomic forms
+    (the vector adds need 16-byte rows); the gradients match the oracle as before."""
+    w = WORKLOADS[2].replace(H=2, N=64 * 6 + 9, K=4, W=100)
+    inp = make_prefill(w)
+    d = to_dev(inp, cuda_device)
+    Ksum, Bsum = gpu_summarize(w, d["K"], d["LQ"])
+    idx, score, nsel = gpu_select(w, d["Qcal"], Ksum, Bsum)
+    O, lse = gpu_prefill(w, d["Q"], d["K"], d["V"], idx, score, nsel)
+    g = torch.Generator().manual_seed(7)
+    dO = torch.randn(O.shape, generator=g).to(cuda_device)
+    p = P(w)
+    B, H, N, dd, Hk, K, C = w.B, w.H, w.N, w.d, w.Hkv, w.K, w.C
+
+    def offset(*shape):  # a dense float32 tensor whose data starts 4 bytes past 16-byte alignment
+        n = 1
+        for s in shape:
+            n *= s
+        base = torch.zeros(n + 4, dtype=torch.float32, device=cuda_device)
+        t = base[1:n + 1].view(*shape)
+        assert t.data_ptr() % 16 == 4
+        return t
+
+    dQ, dK, dV = offset(B, H, N, dd), offset(B, Hk, N, dd), offset(B, Hk, N, dd)
+    dscore = torch.empty(B, H, N, K, dtype=torch.float32, device=cuda_device)
+    ws = hils.alloc_workspace(p, hils.HILS_CALL_ATTEND_BACKWARD, N, 0, device=cuda_device)
+    hils.hils_attend_prefill_backward(p, d["Q"], d["K"], d["V"], idx, score, nsel, O, lse, dO, dQ, dK, dV, dscore,
+                                      workspace=ws)
+    dQcal = offset(B, H, N, dd)
+    dKsum, dBsum = offset(B, H, C, dd), offset(B, H, C)
+    hils.hils_select_backward(p, d["Qcal"], Ksum, idx, nsel, dscore, dQcal, dKsum, dBsum)
+    dLQ = offset(B, H, C, dd)
+    hils.hils_summarize_backward(p, d["K"], d["LQ"], dKsum, dBsum, dK, dLQ)
+    torch.cuda.synchronize()
+    assert int(host(ws[:4]).view(torch.int32)[0]) == 0
+    ref = ob.grads(inp["Q"], inp["K"], inp["V"], inp["Qcal"], inp["LQ"], host(idx), host(nsel), host(dO), 64, w.W,
+                   w.scale, batch=256)
+    for name, got in (("dQ", dQ), ("dK", dK), ("dV", dV), ("dscore", dscore), ("dQcal", dQcal), ("dKsum", dKsum),
+                      ("dBsum", dBsum), ("dLQ", dLQ)):
+        assert _rel(got, ref[name]) <= 1e-2, f"{name}: {_rel(got, ref[name])}"
