@@ -23,12 +23,13 @@
 // each query's dq share to dQ with float32 atomics: for a window block, the contiguous
 // range of queries whose window reaches it; for a chunk, the queries that kept it, from
 // an inverted index of the selection built first (count, scan, scatter). D_i = dO_i . o_i
-// is computed once per query beforehand. Score and summaries: one CTA per query or per
-// chunk. Shared gradients (dK, dV, dKsum, dBsum, dQ) are float32 atomic adds, in no fixed
-// order. Gradients are float32, dense. bf16 with d = 128 takes the tensor-core form of the
-// same walk (backward_tc.cu: 128 queries per step on tcgen05, chunk lists cut into runs
-// of at most 1024 queries); bf16 with d = 64 the mma.sync form below; float32 the
-// CUDA-core form.
+// is computed once per query beforehand. Score backward: a CTA per 256 queries of one
+// head (dQcal, then its kept entries sorted by chunk and summed per chunk). Summaries: a
+// CTA per chunk. Shared gradients (dK, dV, dKsum, dBsum, dQ) are float32 atomic adds, in
+// no fixed order. Gradients are float32, dense. bf16 with d = 128 takes the tensor-core
+// form of the walk (backward_tc.cu: 128 queries per step on tcgen05, chunk lists cut into
+// runs of at most 1024 queries, one persistent CTA per SM); bf16 with d = 64 the mma.sync
+// form below; float32 the CUDA-core form.
 #include <math.h>
 
 #include "backward_common.cuh"
