@@ -30,23 +30,29 @@ struct Pool64 {
 // (K+1)-th largest of n <= kMaxGroups values (duplicates counted) from their
 // order-preserving integer keys key[0..n), padded with zeros to a multiple of 4: value i
 // has the unique rank #{j: k_j > k_i} + #{j < i: k_j = k_i}, and the one of rank K is
-// the answer (n > K; all NT threads call; the result in *out). The keys are read four
-// at a time by every thread at once (a broadcast), with no dependence between steps.
+// the answer (n > K; all NT threads call; the result in *out). Two threads share a key,
+// each counting over half of the keys (read four at a time by every thread at once, a
+// broadcast), and add their counts with one shuffle.
 template <int NT>
 __device__ void block_kth_plus_one(const unsigned *key, int n, int K, float *out) {
     const uint4 *k4 = reinterpret_cast<const uint4 *>(key);
-    const int n4 = (n + 3) >> 2;
-    for (int i = threadIdx.x; i < n; i += NT) {
-        const unsigned ki = key[i];
+    const int n4 = (n + 3) >> 2, h4 = (n4 + 1) >> 1;
+    const int half = threadIdx.x & 1;
+    const int j4lo = half ? h4 : 0, j4hi = half ? n4 : h4;
+    for (int i0 = 0; i0 < n; i0 += NT / 2) {  // uniform over the CTA: the shuffle needs every lane
+        const int i = i0 + (threadIdx.x >> 1);
+        const unsigned ki = i < n ? key[i] : 0u;
         int gt = 0, eq = 0;
-#pragma unroll 8
-        for (int j4 = 0; j4 < n4; ++j4) {
+#pragma unroll 4
+        for (int j4 = j4lo; j4 < j4hi; ++j4) {
             const uint4 k = k4[j4];
             const int j = 4 * j4;
             gt += (k.x > ki) + (k.y > ki) + (k.z > ki) + (k.w > ki);
             eq += (k.x == ki && j < i) + (k.y == ki && j + 1 < i) + (k.z == ki && j + 2 < i) + (k.w == ki && j + 3 < i);
         }
-        if (gt + eq == K) *out = key_to_float(ki);
+        gt += __shfl_xor_sync(kFull, gt, 1);
+        eq += __shfl_xor_sync(kFull, eq, 1);
+        if (i < n && half == 0 && gt + eq == K) *out = key_to_float(ki);
     }
 }
 
