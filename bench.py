@@ -409,7 +409,7 @@ KERNEL_SOURCES = {
 # decode_attend per algorithmic byte of the launch (the captured traffic / algorithmic
 # bytes), summarize per chunk, attend_prefill per launch of the 8K prefill workload.
 MEASURED_TRAFFIC = {
-    'decode_select': (1.0161366640629694, '6aa4e612a5e31e4c'),
+    'decode_select': (1.0160202487532295, 'bee0ccd8a98086ff'),
     'decode_attend': (1.0020989078564204, 'cb90a6455b1fa122'),
     'summarize': (16926.2578125, '853b63865c7de306'),
     'attend_prefill': (661702656, '04b39bda6acf4099'),
