@@ -159,6 +159,38 @@ def test_select_split_paths_bit_exact(oracle, cuda_device, C, K, tpos):
     scores_close(score, s_ref, n_ref)
 
 
+@pytest.mark.parametrize("Hk", [0, 2])
+def test_select_split_repeated_calls_on_one_workspace(oracle, cuda_device, Hk):
+    """The decode select (screen, then the dependent-launched pick) called back to back
+    on one workspace, cycling over three tables with nothing synchronising the calls:
+    every call keeps the oracle's chunks bit-exactly (no call reads another's screen
+    values), and the status word stays zero."""
+    w = WORKLOADS[4].replace(B=1, H=8, K=16, Hk=Hk)
+    C, G = 8191, w.H // w.Hkv
+    qpos = torch.tensor([[64 * C + 3]], dtype=torch.int32)
+    sets = []
+    for seed in (11, 12, 13):
+        Q, Ksum, Bsum = _decode_like(w, C, seed=seed)
+        i_ref, _, n_ref = oracle.select(Q, Ksum, Bsum, 64, w.K, w.scale, qpos=qpos, group=G)
+        sets.append((Q.to(cuda_device), Ksum.to(cuda_device), Bsum.to(cuda_device), i_ref, n_ref))
+    p = P(w)
+    qpos_d = qpos.to(cuda_device)
+    ws = hils.alloc_workspace(p, hils.HILS_CALL_SELECT, 1, C, device=cuda_device)
+    outs = []
+    for r in range(24):
+        Q, Ksum, Bsum, _, _ = sets[r % 3]
+        idx = torch.full((1, w.Hkv, 1, w.K), 7777, dtype=torch.int32, device=cuda_device)
+        score = torch.full((1, w.H, 1, w.K), 7777.0, device=cuda_device)
+        nsel = torch.full((1, w.Hkv, 1), 7777, dtype=torch.int32, device=cuda_device)
+        hils.hils_select(p, Q, Ksum, Bsum, idx, score, nsel, qpos=qpos_d, workspace=ws)
+        outs.append((idx, nsel))
+    torch.cuda.synchronize()
+    for r, (idx, nsel) in enumerate(outs):
+        _, _, _, i_ref, n_ref = sets[r % 3]
+        assert_same_selection(idx, nsel, i_ref, n_ref, f"call {r}")
+    assert int(host(ws[:4]).view(torch.int32)[0]) == 0, "a bounded wait expired"
+
+
 def test_select_planted_exact_ties(oracle, cuda_device):
     """Twenty duplicated summaries give bit-identical scores above all others; only 16
     fit, and the lower chunk indices win. A second planted group ties lower down."""
