@@ -37,11 +37,14 @@
 // Grouped heads (summary page, Methodology 3, GQA adaptation): a CTA takes 128 queries
 // of one (b, group) and puts S_h = Q~_h K'_h^T of each of the group's G heads into its
 // own TMEM columns (the heads' operands pass through two shared-memory buffers). A
-// chunk's group value is the maximum over the heads of s_h,c; each pass folds the
-// heads' intervals s_h,c +- e_h,c into [max lo, max hi] and works on its centre and
-// radius, so the steps above apply unchanged with e_max the row's largest radius. The
-// band's float64 score is the largest of the heads' float64 scores, and each head's
-// output score of a kept chunk is its own screen value, read back from its columns.
+// chunk's group value is the maximum over the heads of s_h,c. Once the MMAs are done,
+// one pass folds the heads' intervals s_h,c +- e_h,c into [max lo, max hi] per chunk
+// and keeps the centre in shared memory (in the operand buffers, which the MMAs no
+// longer read); every later pass reads the centres, and every chunk takes the row's
+// largest folded radius e_max as its radius (an upper bound on its own), so the steps
+// above apply unchanged. The band's float64 score is the largest of the heads' float64
+// scores, and each head's output score of a kept chunk is its own screen value, read
+// back from its columns.
 #include "select_common.cuh"
 #include "tc_common.cuh"
 
@@ -69,14 +72,14 @@ constexpr int kWork = kBandJ + kBandCap * kQM;             // uint16 [128 * kBan
 constexpr int kFbQ = kWork + kQM * kBandCap * 2;           // float  [4][128]
 constexpr int kFbList = kFbQ + 4 * kHD * 4;                // EntryList [4]
 constexpr int kReuseBytes = kFbList + 4 * kListBytes;
-// grouped heads also keep each candidate's radius, and the fallback needs the query
-// rows of all the group's heads
-constexpr int kListE = kReuseBytes;                        // float  [kCap + 1][128]
-constexpr int kFbQG = kListE + (kCap + 1) * kQM * 4;       // float  [4][kMaxGroup][128]
-constexpr int kReuseBytesG = kFbQG + 4 * kMaxGroup * kHD * 4;
-static_assert(kBandX % 8 == 0 && kFbList % 8 == 0, "alignment");
+// grouped heads: the fallback needs the query rows of all the group's heads, and the
+// folded centre of every (chunk, row) follows
+constexpr int kFbQG = kReuseBytes;                         // float  [4][kMaxGroup][128]
+constexpr int kFold = kFbQG + 4 * kMaxGroup * kHD * 4;     // float  [ncpad][128]
+static_assert(kBandX % 8 == 0 && kFbList % 8 == 0 && kFold % 16 == 0, "alignment");
 static_assert(kReuseBytes <= kQBytes + 2 * 64 * 128, "reused region fits the smallest operand area");
-static_assert(kReuseBytesG <= 2 * (kQBytes + 2 * 64 * 128), "grouped reused region fits two operand buffers");
+// two operand buffers of kQBytes + 2 * ncpad * 128 bytes each hold kFold + ncpad * 128 * 4
+static_assert(kFold <= 2 * kQBytes, "grouped reused region and folded centres fit two operand buffers");
 
 struct Misc {
     unsigned long long bar[5];  // operands loaded (2 buffers), MMAs read a buffer (2), all MMAs done
@@ -371,7 +374,6 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
     // ---- per-row selection (thread = query row = TMEM lane)
     float *ls = reinterpret_cast<float *>(smem + kListS);
     uint16_t *lc = reinterpret_cast<uint16_t *>(smem + kListC);
-    float *le = reinterpret_cast<float *>(smem + kListE);
     double *bx = reinterpret_cast<double *>(smem + kBandX);
     uint8_t *bj_s = smem + kBandJ;
     uint16_t *work = reinterpret_cast<uint16_t *>(smem + kWork);
@@ -380,61 +382,70 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
     const float knmax = __uint_as_float(misc->knmax);
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     const int nbat = (ne_w + 31) >> 5;  // warp-uniform: tcgen05.ld is warp-collective
-    // f(c, s, e) over this row's eligible chunks, ascending; e is the radius for grouped
-    // heads (unused for one head, whose radius follows from |k'_c|)
-    auto for_each = [&](auto &&f) {
+    // grouped heads: fold the heads' intervals of every eligible chunk once; the centre
+    // goes to shared memory, the largest radius of the row to emx
+    float *fold = reinterpret_cast<float *>(smem + kFold);  // [chunk][row]
+    float emx = 0.f;
+    if constexpr (kGroup) {
         for (int bi = 0; bi < nbat; ++bi) {
-            if constexpr (!kGroup) {
+            float lo[32], hi[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) lo[j] = hi[j] = -INFINITY;
+            for (int hh = 0; hh < G; ++hh) {
+                uint32_t r[32];
+                tmem_ld32(trow + hh * args.hcols + bi * 32, r);
+                tmem_wait_ld();
+                const float eqh = sc * qn_s[hh * kQM + tid] * ((float)kHD * 0x1p-16f) * (1.f + 0x1p-8f);
+                const float *bh = bias_s + hh * ncpad + bi * 32;
+                const float *kh = kn_s + hh * ncpad + bi * 32;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    if (bi * 32 + j < ne) {
+                        const float sh = fmaf(__uint_as_float(r[j]), sc, bh[j]);
+                        fold_interval(sh, fmaf(eqh, kh[j], fabsf(sh) * 0x1p-22f), lo[j], hi[j]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int c = bi * 32 + j;
+                if (c < ne) {
+                    float s, e;
+                    interval_mid(lo[j], hi[j], s, e);
+                    fold[c * kQM + tid] = s;
+                    emx = fmaxf(emx, e);
+                }
+            }
+        }
+    }
+    // f(c, s) over this row's eligible chunks, ascending
+    auto for_each = [&](auto &&f) {
+        if constexpr (!kGroup) {
+            for (int bi = 0; bi < nbat; ++bi) {
                 uint32_t r[32];
                 tmem_ld32(trow + bi * 32, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int c = bi * 32 + j;
-                    if (c < ne) f(c, fmaf(__uint_as_float(r[j]), sc, bias_s[c]), 0.f);
-                }
-            } else {
-                float lo[32], hi[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) lo[j] = hi[j] = -INFINITY;
-                for (int hh = 0; hh < G; ++hh) {
-                    uint32_t r[32];
-                    tmem_ld32(trow + hh * args.hcols + bi * 32, r);
-                    tmem_wait_ld();
-                    const float eqh = sc * qn_s[hh * kQM + tid] * ((float)kHD * 0x1p-16f) * (1.f + 0x1p-8f);
-                    const float *bh = bias_s + hh * ncpad + bi * 32;
-                    const float *kh = kn_s + hh * ncpad + bi * 32;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        if (bi * 32 + j < ne) {
-                            const float sh = fmaf(__uint_as_float(r[j]), sc, bh[j]);
-                            fold_interval(sh, fmaf(eqh, kh[j], fabsf(sh) * 0x1p-22f), lo[j], hi[j]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int c = bi * 32 + j;
-                    if (c < ne) {
-                        float s, e;
-                        interval_mid(lo[j], hi[j], s, e);
-                        f(c, s, e);
-                    }
+                    if (c < ne) f(c, fmaf(__uint_as_float(r[j]), sc, bias_s[c]));
                 }
             }
+        } else {
+#pragma unroll 8
+            for (int c = 0; c < ne; ++c) f(c, fold[c * kQM + tid]);
         }
     };
 
     // pass A: range and moments of the row (shifted by b'_0, which lies near every s)
     const float sref = nc > 0 ? bias_s[0] : 0.f;
-    float mn = INFINITY, mx = -INFINITY, sum = 0.f, sq = 0.f, emx = 0.f;
-    for_each([&](int, float s, float e) {
+    float mn = INFINITY, mx = -INFINITY, sum = 0.f, sq = 0.f;
+    for_each([&](int, float s) {
         mn = fminf(mn, s);
         mx = fmaxf(mx, s);
         const float dv = s - sref;
         sum += dv;
         sq = fmaf(dv, dv, sq);
-        if (kGroup) emx = fmaxf(emx, e);
     });
     const float emax = kGroup ? emx : fmaf(eq, knmax, fmaxf(fabsf(mn), fabsf(mx)) * 0x1p-22f);
 
@@ -455,13 +466,12 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
     for (int pass = 0; pass < kCollectPasses && __any_sync(kFull, pending); ++pass) {
         const float tcut = g == -INFINITY ? -INFINITY : __fsub_rd(__fsub_rd(g, emax), emax);
         int mm = 0;
-        for_each([&](int c, float s, float e) {
+        for_each([&](int c, float s) {
             const bool take = pending && s >= tcut;
             const int slot = min(mm, kCap);  // entries past the capacity land in the spare slot
             if (take) {
                 ls[slot * kQM + tid] = s;
                 lc[slot * kQM + tid] = (uint16_t)c;
-                if (kGroup) le[slot * kQM + tid] = e;
             }
             mm += take ? 1 : 0;
         });
@@ -522,7 +532,7 @@ __global__ void __launch_bounds__(kTcThreads) select_tc_kernel(const __grid_cons
             const float hi_cut = __fadd_ru(sK1, emax);
             for (int j = 0; j < m; ++j) {
                 const float s = ls[j * kQM + tid];
-                const float e = kGroup ? le[j * kQM + tid] : fmaf(eq, kn_s[lc[j * kQM + tid]], fabsf(s) * 0x1p-22f);
+                const float e = kGroup ? emax : fmaf(eq, kn_s[lc[j * kQM + tid]], fabsf(s) * 0x1p-22f);
                 if (__fsub_rd(s, e) > hi_cut) keep |= 1u << j;
                 else if (__fadd_ru(s, e) >= lo_cut) bandm |= 1u << j;
             }
