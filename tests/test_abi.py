@@ -320,3 +320,68 @@ def test_decode_time_and_backward_entry_points_validate_first(lib):
     assert lib.hils_summarize_backward(c, v, N, bad, A, A, A, A, None) == 3
     g = _p(H=4, H_kv=3)
     assert lib.hils_summarize_backward(ctypes.byref(g.c()), v, N, s, A, A, A, A, None) == 1
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "hils.h"
+
+/* every entry point the header declares, taken by address: the program links only if
+   the library defines each one with C linkage */
+typedef void (*any_fn)(void);
+static const any_fn entry_points[] = {
+%(entries)s
+};
+
+int main(void) {
+    hils_params p;
+    size_t n;
+    int i;
+    memset(&p, 0, sizeof p);
+    p.B = 1; p.H = 32; p.d = 128; p.S = 64; p.K = 16; p.W = 512; p.dtype = HILS_BF16;
+    for (i = 0; i < (int)(sizeof entry_points / sizeof entry_points[0]); ++i)
+        if (!entry_points[i]) return 10;
+    for (i = HILS_OK; i <= HILS_ERR_CUDA; ++i)
+        if (!hils_status_string(i) || !hils_status_string(i)[0]) return 11;
+    n = hils_workspace_bytes(&p, HILS_CALL_DECODE, 1, 8191);
+    printf("decode_ws %%zu\n", n);
+    /* host checks run before anything is launched: no device is touched */
+    printf("null_params %%d\n", hils_summarize(NULL, (hils_ctensor){0}, 64, (hils_ctensor){0},
+                                              (hils_tensor){0}, NULL, 0));
+    p.d = 80;
+    printf("bad_d %%d\n", hils_summarize(&p, (hils_ctensor){0}, 64, (hils_ctensor){0},
+                                        (hils_tensor){0}, NULL, 0));
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links_from_a_c_program(lib, tmp_path):
+    """A C99 program (gcc, no C++) includes hils.h, takes the address of every declared
+    entry point, links against libhils.so and runs on the host: the status strings, the
+    decode chain's workspace size (equal to the value the binding sees) and two calls
+    that the host checks reject before any launch."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    cuda_inc = "/usr/local/cuda/include"
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER % {"entries": ",\n".join(f"    (any_fn)&{n}" for n in _declared())})
+    exe = tmp_path / "caller"
+    pkg = os.path.dirname(hils.LIB_PATH)
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+           "-I", os.path.join(ROOT, "include"), "-isystem", cuda_inc, str(src), "-o", str(exe),
+           "-L", pkg, "-l:libhils.so", f"-Wl,-rpath,{pkg}"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    got = dict(line.split() for line in r.stdout.strip().splitlines())
+    p = _p(B=1, H=32, K=16, W=512)
+    assert int(got["decode_ws"]) == lib.hils_workspace_bytes(ctypes.byref(p.c()), hils.HILS_CALL_DECODE, 1, 8191) > 0
+    assert int(got["null_params"]) == 1  # HILS_ERR_INVALID_ARG
+    assert int(got["bad_d"]) == 2  # HILS_ERR_UNSUPPORTED
